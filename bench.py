@@ -1,0 +1,342 @@
+"""Benchmark of the edge-aware attention layer (forward + backward) on B200.
+
+Workload (one step): one forward and one backward of the layer over one
+batch of the SBM-shaped training preset (B=32 graphs, n=192 padded nodes,
+n_real ~ U[44,187], dx=256, de=64, dy=64, H=8, dh=32, bf16 storage, fp32
+accumulation), synthetic seeded inputs (edge_aware_graph_b200/inputs.py).
+Metric: edge pairs (B*n^2, padded) per second, and the fraction of the HBM
+roofline of the dominant kernel.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own batch of the same shape
+(weak scaling) and the step adds the data-parallel all-reduce of the weight
+gradients over NCCL; rank 0 prints one JSON line.  `--impl reference` times
+the fp64 CPU oracle (the reference arm) on a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+
+WORKLOAD = "sbm"
+METRIC = "edge-pairs/sec (B·n²) fwd and fwd+bwd on 1 B200; % of HBM roofline"
+UNIT = "edge-pairs/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        if self._thr:
+            self._stop.set()
+            self._thr.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ bytes
+
+
+def compulsory_bytes(p, training=True):
+    """Algorithmic bytes of the layer (no recomputation, each tensor once)."""
+    s = 2 if p.dtype == "bf16" else 4
+    pairs, nodes = p.B * p.n * p.n, p.B * p.n
+    fwd = pairs * p.de * s * 2 + nodes * p.dx * s * 2
+    bwd = pairs * p.de * s * 3 + nodes * p.dx * s * 3
+    return fwd + (bwd if training else 0)
+
+
+def pair_kernel_bytes(p, which):
+    """Algorithmic bytes of one launch of the pair kernels: the E-sized
+    streams only (forward: E read, E' write; backward: E and dE' read, dE
+    write).  Node-sized terms (Q, K, V, O, LSE, ...) are left out."""
+    s = 2 if p.dtype == "bf16" else 4
+    per_pair = p.de * s * (2 if which == "fwd" else 3)
+    return p.B * p.n * p.n * per_pair
+
+
+# ------------------------------------------------------------------ our arm
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from edge_aware_graph_b200 import eaga
+    from edge_aware_graph_b200 import inputs as I
+    from edge_aware_graph_b200.buffers import LayerBuffers
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    p = I.preset(WORKLOAD)
+    d = I.draw_inputs(p, with_grads=True)
+    W = I.draw_weights(p)
+    buf = LayerBuffers(p.B, p.n, p.dx, p.de, p.dy, p.H, p.dh, dtype=p.dtype, backward=True)
+    buf.load_inputs(d, W)
+    stream = torch.cuda.current_stream()
+    flat_dw = buf.dW_flat
+
+    def step():
+        buf.forward(stream)
+        buf.backward(stream)
+        if world > 1:
+            dist.all_reduce(flat_dw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, events per step around the pair kernels
+    K = args.steps
+    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for k in range(K):
+        eaga.set_profile_events(0, *ev_f[k])
+        eaga.set_profile_events(1, *ev_b[k])
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    eaga.set_profile_events(0)
+    eaga.set_profile_events(1)
+    ms_total = t0.elapsed_time(t1)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
+    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_b)
+    if world > 1:
+        t = torch.tensor([ms_total], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, buf, d, stream, step)
+    if world > 1:
+        t = torch.tensor([e2e["ms"]], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms"] = float(t.item())
+
+    launches = (eaga.kernel_launches(buf.dims, False) + eaga.kernel_launches(buf.dims, True)) * K
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    pairs_step = p.B * p.n * p.n
+    ms_step = ms_total / K
+    value = world * pairs_step * K / (ms_total / 1e3)
+    peak, peak_kind = measured_peaks()
+    kb = pair_kernel_bytes(p, "bwd")
+    achieved = kb / (bwd_ms / 1e3) / 1e9
+    kf = pair_kernel_bytes(p, "fwd")
+    step_bytes = compulsory_bytes(p)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded SBM-shaped graphs; edge_aware_graph_b200/inputs.py)",
+        "config": {"workload": "sbm-shaped training step (fwd+bwd): B=32, n=192 padded, n_real~U[44,187], "
+                               "dx=256 de=64 dy=64 H=8 dh=32, bf16 storage / fp32 accumulation",
+                   "global_batch": p.B * world, "seq_len": p.n, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (E, dE' 144 MiB each; E', dE written each step)"},
+        "roofline": {"bound": "hbm", "kernel": "backward pair kernels", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes": kb, "ms_per_launch": bwd_ms},
+        "roofline_fwd": {"bound": "hbm", "kernel": "forward pair kernels", "achieved": kf / (fwd_ms / 1e3) / 1e9,
+                         "peak": peak, "unit": "GB/s", "frac": kf / (fwd_ms / 1e3) / 1e9 / peak,
+                         "algorithmic_bytes": kf, "ms_per_launch": fwd_ms},
+        "step_roofline": {"compulsory_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                          "frac_of_measured": step_bytes / (ms_step / 1e3) / 1e9 / peak,
+                          "frac_of_8tbs": step_bytes / (ms_step / 1e3) / 1e9 / 8000.0},
+        "clocks": clk,
+        "e2e": {"value": world * pairs_step / (e2e["ms"] / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"]},
+        "gpu_launches": launches,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(p, d, W, args.cpu_graphs)
+    return out
+
+
+def run_e2e(args, buf, d, stream, step):
+    """Steps whose timed region includes the pinned-host -> device copy of the
+    step's inputs and the device -> host read of its results."""
+    import torch
+
+    from edge_aware_graph_b200.buffers import host_to_storage_tensor
+    names_in = ["X", "E", "y", "dXout", "dEout"]
+    host_in = {k: host_to_storage_tensor(d[k], buf.dtype).pin_memory() for k in names_in}
+    host_M = torch.from_numpy(np.ascontiguousarray(d["M"])).pin_memory()
+    outs = [buf.Xout, buf.Eout, buf.dX, buf.dE, buf.dy, buf.dW_flat]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    dev_in = {"X": buf.X, "E": buf.E, "y": buf.y, "dXout": buf.dXout, "dEout": buf.dEout}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + host_M.numel()
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    def e2e_step():
+        for k in names_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        buf.M.copy_(host_M, non_blocking=True)
+        step()
+        for h, t in zip(host_out, outs):
+            h.copy_(t, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    n = args.e2e_steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(n):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    return {"ms": t0.elapsed_time(t1) / n, "h2d": h2d, "d2h": d2h, "steps": n}
+
+
+# ------------------------------------------------------------------ oracle arm
+
+
+def cpu_baseline(p, d, W, graphs):
+    """The fp64 oracle, as it stands, on a bounded sample: the first `graphs`
+    graphs of the batch, forward + backward, all usable host cores."""
+    import oracle
+    oracle.build()
+    sl = {k: d[k][:graphs] for k in ("X", "E", "y", "M", "dXout", "dEout")}
+    dims = dict(H=p.H, dh=p.dh)
+    t = time.perf_counter()
+    oracle.forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W)
+    oracle.backward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, sl["dXout"], sl["dEout"])
+    dt = time.perf_counter() - t
+    pairs = graphs * p.n * p.n
+    return {"value": pairs / dt, "unit": UNIT, "cores": oracle.threads_used(), "kind": "oracle",
+            "sample": f"{graphs} of {p.B} graphs of the workload (n={p.n}), forward + backward, fp64",
+            "seconds": dt}
+
+
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return None
+    from edge_aware_graph_b200 import inputs as I
+    p = I.preset(WORKLOAD)
+    d = I.draw_inputs(p, with_grads=True)
+    W = I.draw_weights(p)
+    for _ in range(args.warmup):
+        cpu_baseline(p, d, W, 1)
+    res = [cpu_baseline(p, d, W, args.ref_graphs) for _ in range(args.steps)]
+    secs = sum(r["seconds"] for r in res)
+    pairs = args.steps * args.ref_graphs * p.n * p.n
+    value = pairs / secs
+    cb = dict(res[0])
+    cb["value"] = value
+    cb.pop("seconds", None)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded SBM-shaped graphs)",
+            "config": {"workload": "sbm-shaped training step (fwd+bwd), bounded sample of "
+                                   f"{args.ref_graphs} graph(s) per step", "global_batch": args.ref_graphs,
+                       "seq_len": p.n, "parallelism": "cpu"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-graphs", type=int, default=16)
+    ap.add_argument("--ref-graphs", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

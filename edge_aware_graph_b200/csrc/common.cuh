@@ -1,0 +1,88 @@
+// Internal helpers shared by the CUDA translation units of libeaga.so.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include "../../include/eaga.h"
+
+namespace eaga {
+
+__device__ __forceinline__ float ldf(const float *p) { return *p; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void stf(float *p, float v) { *p = v; }
+__device__ __forceinline__ void stf(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float warp_max(float v) {
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Byte layout of the forward's saved state and of the workspaces.
+struct Layout {
+    size_t lse, q, k, v, o, saved_total;        // offsets inside `saved`
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline Layout saved_layout(const eaga_dims &d) {
+    const size_t es = d.dtype == EAGA_BF16 ? 2 : 4;
+    const size_t rows = size_t(d.B) * d.n, hd = size_t(d.H) * d.dh;
+    Layout L;
+    size_t off = 0;
+    L.lse = off; off = align256(off + size_t(d.B) * d.H * d.n * 4);
+    L.q = off; off = align256(off + rows * hd * es);
+    L.k = off; off = align256(off + rows * hd * es);
+    L.v = off; off = align256(off + rows * hd * es);
+    L.o = off; off = align256(off + rows * hd * es);
+    L.saved_total = off;
+    return L;
+}
+
+// Workspace: [status word (256 B)][g fp32 B*2H][forward: saved-equivalent if
+// no saved buffer given][backward: dO, dQ, dK, dV fp32 rows*hd; D fp32 B*H*n;
+// per-row parts fp32 rows*(de*2H + H*de + 2H); dg fp32 B*2H]
+struct WsLayout {
+    size_t status, g, fwd_saved, total_fwd;
+    size_t dO, dQ, dK, dV, D, parts, dg, total_bwd;
+    size_t part_stride;  // floats per row part
+};
+
+inline WsLayout ws_layout(const eaga_dims &d) {
+    WsLayout W;
+    const size_t rows = size_t(d.B) * d.n, hd = size_t(d.H) * d.dh, F = 2 * size_t(d.H);
+    size_t off = 0;
+    W.status = off; off = 256;
+    W.g = off; off = align256(off + size_t(d.B) * F * 4);
+    const size_t common = off;
+    W.fwd_saved = off; off = align256(off + saved_layout(d).saved_total);
+    W.total_fwd = off;
+    off = common;
+    W.dO = off; off = align256(off + rows * hd * 4);
+    W.dQ = off; off = align256(off + rows * hd * 4);
+    W.dK = off; off = align256(off + rows * hd * 4);
+    W.dV = off; off = align256(off + rows * hd * 4);
+    W.D = off; off = align256(off + size_t(d.B) * d.H * d.n * 4);
+    W.part_stride = size_t(d.de) * F + size_t(d.H) * d.de + F;
+    W.parts = off; off = align256(off + rows * W.part_stride * 4);
+    W.dg = off; off = align256(off + size_t(d.B) * F * 4);
+    W.total_bwd = off;
+    return W;
+}
+
+// Optional profiling events around the pair kernels (eaga_set_profile_events).
+extern void *g_prof_events[2][2];
+inline void prof_mark(int point, int which, cudaStream_t st) {
+    void *ev = g_prof_events[point][which];
+    if (ev) cudaEventRecord(static_cast<cudaEvent_t>(ev), st);
+}
+
+// Device status word values (first int of the workspace).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
+
+}  // namespace eaga

@@ -1,0 +1,198 @@
+// C ABI of libeaga.so (declared in include/eaga.h): argument validation,
+// saved-state and workspace layout, and the launch sequence on the caller's
+// stream.  No device memory is allocated here.
+#include <stdint.h>
+#include <string.h>
+#include "common.cuh"
+#include "generic.h"
+#include "fast.h"
+
+using namespace eaga;
+
+namespace eaga {
+void *g_prof_events[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+}
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+eaga_status check_dims(const eaga_dims *d) {
+    if (!d) return EAGA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->n < 1 || d->dx < 1 || d->de < 1 || d->dy < 1 || d->H < 1 || d->dh < 1)
+        return EAGA_ERR_INVALID_ARG;
+    if (d->dtype != EAGA_FP32 && d->dtype != EAGA_BF16) return EAGA_ERR_INVALID_ARG;
+    if (d->n > 1024 || d->H * d->dh > 256 || d->dh % 8 || d->de % 8 || d->de > 128 || d->dx % 8 ||
+        d->dx > 1024 || d->dy % 8 || d->dy > 1024 || 2 * d->H > 32 || d->H * d->n > 8192)
+        return EAGA_ERR_UNSUPPORTED;
+    if ((size_t)d->B * d->n > (size_t)1 << 26) return EAGA_ERR_UNSUPPORTED;
+    return EAGA_OK;
+}
+
+eaga_status check_ptrs(std::initializer_list<const void *> ps) {
+    for (const void *p : ps) {
+        if (!p) return EAGA_ERR_INVALID_ARG;
+        if (!aligned16(p)) return EAGA_ERR_MISALIGNED;
+    }
+    return EAGA_OK;
+}
+
+eaga_status check_weights(const eaga_weights *w) {
+    if (!w) return EAGA_ERR_INVALID_ARG;
+    return check_ptrs({w->Wq, w->bq, w->Wk, w->bk, w->Wv, w->bv, w->Wfe, w->Wfy, w->bf, w->We, w->Wo, w->bo});
+}
+
+void weight_array(const eaga_weights *w, const void *out[12]) {
+    const void *src[12] = {w->Wq, w->bq, w->Wk, w->bk, w->Wv, w->bv, w->Wfe, w->Wfy, w->bf, w->We, w->Wo, w->bo};
+    memcpy(out, src, sizeof(src));
+}
+
+eaga_status launch_status(cudaError_t e) { return e == cudaSuccess ? EAGA_OK : EAGA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t eaga_workspace_size(const eaga_dims *d, int for_backward) {
+    if (check_dims(d) != EAGA_OK) return 0;
+    const WsLayout W = ws_layout(*d);
+    size_t bytes = for_backward ? W.total_bwd : W.total_fwd;
+    const size_t extra = fast::workspace_extra(*d, for_backward);
+    return bytes + extra;
+}
+
+size_t eaga_saved_size(const eaga_dims *d) {
+    if (check_dims(d) != EAGA_OK) return 0;
+    return saved_layout(*d).saved_total;
+}
+
+eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
+                         const eaga_weights *w, void *Xout, void *Eout, void *saved, void *workspace,
+                         size_t ws_bytes, void *stream) {
+    eaga_status s = check_dims(d);
+    if (s != EAGA_OK) return s;
+    if ((s = check_weights(w)) != EAGA_OK) return s;
+    if ((s = check_ptrs({X, E, y, M, Xout, Eout, workspace})) != EAGA_OK) return s;
+    if (saved && !aligned16(saved)) return EAGA_ERR_MISALIGNED;
+    if (ws_bytes < eaga_workspace_size(d, 0)) return EAGA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsLayout W = ws_layout(*d);
+    const Layout L = saved_layout(*d);
+    char *ws = static_cast<char *>(workspace);
+    char *sv = saved ? static_cast<char *>(saved) : ws + W.fwd_saved;
+    FwdArgs a;
+    a.X = X; a.E = E; a.y = y; a.M = M;
+    weight_array(w, a.w);
+    a.Xout = Xout; a.Eout = Eout;
+    a.LSE = reinterpret_cast<float *>(sv + L.lse);
+    a.Q = sv + L.q; a.K = sv + L.k; a.V = sv + L.v; a.O = sv + L.o;
+    a.g = reinterpret_cast<float *>(ws + W.g);
+    a.status = reinterpret_cast<int *>(ws + W.status);
+    if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (fast::supports(*d)) {
+        return launch_status(fast::forward(*d, a, ws + W.total_fwd, st));
+    }
+    return launch_status(generic::forward(*d, a, st));
+}
+
+eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
+                          const eaga_weights *w, const void *saved, const void *dXout, const void *dEout,
+                          void *dX, void *dE, void *dy, const eaga_weight_grads *dW, void *workspace,
+                          size_t ws_bytes, void *stream) {
+    eaga_status s = check_dims(d);
+    if (s != EAGA_OK) return s;
+    if ((s = check_weights(w)) != EAGA_OK) return s;
+    if ((s = check_ptrs({X, E, y, M, saved, dXout, dEout, dX, dE, dy, workspace})) != EAGA_OK) return s;
+    if (!dW) return EAGA_ERR_INVALID_ARG;
+    if ((s = check_ptrs({dW->Wq, dW->bq, dW->Wk, dW->bk, dW->Wv, dW->bv, dW->Wfe, dW->Wfy, dW->bf, dW->We, dW->Wo,
+                         dW->bo})) != EAGA_OK)
+        return s;
+    if (ws_bytes < eaga_workspace_size(d, 1)) return EAGA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsLayout W = ws_layout(*d);
+    const Layout L = saved_layout(*d);
+    char *ws = static_cast<char *>(workspace);
+    const char *sv = static_cast<const char *>(saved);
+    BwdArgs a;
+    a.X = X; a.E = E; a.y = y; a.M = M;
+    weight_array(w, a.w);
+    a.Q = sv + L.q; a.K = sv + L.k; a.V = sv + L.v; a.O = sv + L.o;
+    a.LSE = reinterpret_cast<const float *>(sv + L.lse);
+    a.dXout = dXout; a.dEout = dEout;
+    a.dX = dX; a.dE = dE; a.dy = dy;
+    void *gsrc[12] = {dW->Wq, dW->bq, dW->Wk, dW->bk, dW->Wv, dW->bv, dW->Wfe, dW->Wfy, dW->bf, dW->We, dW->Wo, dW->bo};
+    for (int t = 0; t < 12; ++t) a.dW[t] = static_cast<float *>(gsrc[t]);
+    a.g = reinterpret_cast<float *>(ws + W.g);
+    a.dO = reinterpret_cast<float *>(ws + W.dO);
+    a.dQ = reinterpret_cast<float *>(ws + W.dQ);
+    a.dK = reinterpret_cast<float *>(ws + W.dK);
+    a.dV = reinterpret_cast<float *>(ws + W.dV);
+    a.D = reinterpret_cast<float *>(ws + W.D);
+    a.parts = reinterpret_cast<float *>(ws + W.parts);
+    a.dg = reinterpret_cast<float *>(ws + W.dg);
+    a.part_stride = W.part_stride;
+    a.status = reinterpret_cast<int *>(ws + W.status);
+    if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (fast::supports(*d)) {
+        return launch_status(fast::backward(*d, a, ws + W.total_bwd, st));
+    }
+    return launch_status(generic::backward(*d, a, st));
+}
+
+eaga_status eaga_debug_attention_map(const eaga_dims *d, const void *E, const uint8_t *M, const eaga_weights *w,
+                                     const void *y, const void *saved, float *A, void *stream) {
+    eaga_status s = check_dims(d);
+    if (s != EAGA_OK) return s;
+    if ((s = check_weights(w)) != EAGA_OK) return s;
+    if ((s = check_ptrs({E, M, y, saved, A})) != EAGA_OK) return s;
+    // g [B,2H] lives just past the A map the caller provides room for.
+    const Layout L = saved_layout(*d);
+    const char *sv = static_cast<const char *>(saved);
+    MapArgs a;
+    a.E = E; a.y = y; a.Wfe = w->Wfe; a.Wfy = w->Wfy; a.bf = w->bf; a.M = M;
+    a.Q = sv + L.q; a.K = sv + L.k;
+    a.LSE = reinterpret_cast<const float *>(sv + L.lse);
+    a.A = A;
+    a.g = A + (size_t)d->B * d->H * d->n * d->n;
+    return launch_status(generic::attention_map(*d, a, static_cast<cudaStream_t>(stream)));
+}
+
+eaga_status eaga_get_device_status(void *workspace, void *stream) {
+    if (!workspace) return EAGA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int h = 0;
+    if (cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return EAGA_ERR_CUDA;
+    return h == DEV_OK ? EAGA_OK : EAGA_ERR_TIMEOUT;
+}
+
+eaga_status eaga_set_profile_events(int point, void *before, void *after) {
+    if (point < 0 || point > 1) return EAGA_ERR_INVALID_ARG;
+    if ((before == nullptr) != (after == nullptr)) return EAGA_ERR_INVALID_ARG;
+    g_prof_events[point][0] = before;
+    g_prof_events[point][1] = after;
+    return EAGA_OK;
+}
+
+int eaga_kernel_launches(const eaga_dims *d, int for_backward) {
+    if (check_dims(d) != EAGA_OK) return -1;
+    if (fast::supports(*d)) return fast::kernel_launches(*d, for_backward);
+    return generic::kernel_launches(*d, for_backward);
+}
+
+const char *eaga_strerror(eaga_status s) {
+    switch (s) {
+    case EAGA_OK: return "ok";
+    case EAGA_ERR_INVALID_ARG: return "invalid argument";
+    case EAGA_ERR_UNSUPPORTED: return "unsupported dims";
+    case EAGA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case EAGA_ERR_WORKSPACE: return "workspace too small";
+    case EAGA_ERR_CUDA: return "CUDA error";
+    case EAGA_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+"""Thin ctypes binding of libeaga.so (include/eaga.h).
+
+Argument marshalling only: every function takes torch tensors that already
+live on the GPU (or plain ints), passes their data pointers and the current
+CUDA stream to the C entry point of the same name, and raises on a non-OK
+status.  All arithmetic runs in the library's CUDA kernels; there is no
+fallback of any kind.  The library must have been built in-tree
+(edge_aware_graph_b200/build.py); loading fails loudly otherwise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libeaga.so")
+
+WEIGHT_NAMES = ("Wq", "bq", "Wk", "bk", "Wv", "bv", "Wfe", "Wfy", "bf", "We", "Wo", "bo")
+EAGA_FP32, EAGA_BF16 = 0, 1
+STATUS = {0: "EAGA_OK", 1: "EAGA_ERR_INVALID_ARG", 2: "EAGA_ERR_UNSUPPORTED", 3: "EAGA_ERR_MISALIGNED",
+          4: "EAGA_ERR_WORKSPACE", 5: "EAGA_ERR_CUDA", 6: "EAGA_ERR_TIMEOUT"}
+EXPORTED = ("eaga_workspace_size", "eaga_saved_size", "eaga_forward", "eaga_backward",
+            "eaga_debug_attention_map", "eaga_get_device_status", "eaga_strerror",
+            "eaga_set_profile_events", "eaga_kernel_launches")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int) for k in ("B", "n", "dx", "de", "dy", "H", "dh", "dtype")]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in WEIGHT_NAMES]
+
+
+class EagaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load libeaga.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libeaga.so not built ({LIB_PATH}); run edge_aware_graph_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        L.eaga_workspace_size.argtypes = [ctypes.POINTER(Dims), i32]
+        L.eaga_workspace_size.restype = sz
+        L.eaga_saved_size.argtypes = [ctypes.POINTER(Dims)]
+        L.eaga_saved_size.restype = sz
+        L.eaga_forward.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.POINTER(Weights),
+                                   vp, vp, vp, vp, sz, vp]
+        L.eaga_forward.restype = i32
+        L.eaga_backward.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.POINTER(Weights), vp,
+                                    vp, vp, vp, vp, vp, ctypes.POINTER(Weights), vp, sz, vp]
+        L.eaga_backward.restype = i32
+        L.eaga_debug_attention_map.argtypes = [ctypes.POINTER(Dims), vp, vp, ctypes.POINTER(Weights), vp, vp,
+                                               vp, vp]
+        L.eaga_debug_attention_map.restype = i32
+        L.eaga_get_device_status.argtypes = [vp, vp]
+        L.eaga_get_device_status.restype = i32
+        L.eaga_set_profile_events.argtypes = [i32, vp, vp]
+        L.eaga_set_profile_events.restype = i32
+        L.eaga_kernel_launches.argtypes = [ctypes.POINTER(Dims), i32]
+        L.eaga_kernel_launches.restype = i32
+        L.eaga_strerror.argtypes = [i32]
+        L.eaga_strerror.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def dims(B, n, dx, de, dy, H, dh, dtype) -> Dims:
+    if isinstance(dtype, str):
+        dtype = EAGA_BF16 if dtype == "bf16" else EAGA_FP32
+    return Dims(B, n, dx, de, dy, H, dh, dtype)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _weights(W: dict) -> Weights:
+    return Weights(*(W[k].data_ptr() for k in WEIGHT_NAMES))
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise EagaError(rc, where)
+
+
+def workspace_size(d: Dims, for_backward: bool) -> int:
+    return int(lib().eaga_workspace_size(ctypes.byref(d), int(bool(for_backward))))
+
+
+def saved_size(d: Dims) -> int:
+    return int(lib().eaga_saved_size(ctypes.byref(d)))
+
+
+def forward(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, workspace, stream=None):
+    rc = lib().eaga_forward(ctypes.byref(d), _p(X), _p(E), _p(y), _p(M), ctypes.byref(_weights(W)),
+                            _p(Xout), _p(Eout), _p(saved), _p(workspace), workspace.numel() * workspace.element_size(),
+                            _stream(stream))
+    _check(rc, "eaga_forward")
+
+
+def backward(d: Dims, X, E, y, M, W: dict, saved, dXout, dEout, dX, dE, dy, dW: dict, workspace, stream=None):
+    rc = lib().eaga_backward(ctypes.byref(d), _p(X), _p(E), _p(y), _p(M), ctypes.byref(_weights(W)), _p(saved),
+                             _p(dXout), _p(dEout), _p(dX), _p(dE), _p(dy), ctypes.byref(_weights(dW)),
+                             _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "eaga_backward")
+
+
+def debug_attention_map(d: Dims, E, M, W: dict, y, saved, A, stream=None):
+    rc = lib().eaga_debug_attention_map(ctypes.byref(d), _p(E), _p(M), ctypes.byref(_weights(W)), _p(y), _p(saved),
+                                        _p(A), _stream(stream))
+    _check(rc, "eaga_debug_attention_map")
+
+
+def get_device_status(workspace, stream=None) -> int:
+    return int(lib().eaga_get_device_status(_p(workspace), _stream(stream)))
+
+
+def set_profile_events(point: int, before=None, after=None):
+    """point 0: forward pair kernels, 1: backward pair kernels; torch.cuda.Event or None."""
+    b = ctypes.c_void_p(before.cuda_event) if before is not None else None
+    a = ctypes.c_void_p(after.cuda_event) if after is not None else None
+    _check(lib().eaga_set_profile_events(int(point), b, a), "eaga_set_profile_events")
+
+
+def kernel_launches(d: Dims, for_backward: bool) -> int:
+    return int(lib().eaga_kernel_launches(ctypes.byref(d), int(bool(for_backward))))
+
+
+def strerror(code: int) -> str:
+    return lib().eaga_strerror(int(code)).decode()

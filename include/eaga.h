@@ -1,0 +1,155 @@
+/*
+ * eaga.h — C ABI of the edge-aware graph attention layer (libeaga.so).
+ *
+ * The layer is the FlexAttentionGT edge-aware attention layer of "Efficient
+ * Edge-aware Attention Network for Graph Generation": per-head scaled
+ * dot-product attention over the nodes of dense padded graphs, whose scores
+ * are modulated head-wise by a FiLM of the edge features E_ij and the graph's
+ * global features y (AI-summary page, method paragraph; blog summary, "Design
+ * Strategy of the Edge-aware Attention Layer"), restricted to real nodes by
+ * the node mask, returning both the node aggregation and the normalised
+ * attention coefficients in one pass, followed by a residual edge update from
+ * those coefficients and a residual node update (AI-summary page, method
+ * paragraph).  Per graph b, node i, j, head h:
+ *
+ *   Q,K,V   = X W{q,k,v} + b{q,k,v}                 head h = cols h*dh..h*dh+dh-1
+ *   g_b     = y_b Wfy + bf                           [2H]
+ *   f_bij   = E_bij Wfe + g_b;  gamma = f[h], beta = f[H+h]
+ *   s'_ij   = (q_i . k_j / sqrt(dh)) (1 + gamma) + beta
+ *   a_ij    = softmax over valid j of s'_ij          (valid: M_bi and M_bj; else 0)
+ *   O_ih    = sum_j a_ij v_jh
+ *   E'_bij  = E_bij + sum_h a^h_ij We[h,:]
+ *   X'_bi   = X_bi + M_bi (O_bi Wo + bo)
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers to contiguous row-major arrays,
+ *     owned by the caller; the library never allocates device memory.
+ *   - Storage dtype (dims.dtype) applies to X, E, y, weights, outputs X', E',
+ *     the gradients dX, dE, dy, dX', dE' and the saved Q,K,V,O.  Arithmetic
+ *     accumulates in fp32 in both modes.  Weight gradients are always fp32.
+ *   - M is uint8 [B,n] with values 0/1 (any pattern, not only a prefix).
+ *   - Weights are [in, out] (Y = X W): Wq,Wk,Wv [dx, H*dh]; bq,bk,bv [H*dh];
+ *     Wfe [de, 2H]; Wfy [dy, 2H]; bf [2H] (first H columns gamma, next H
+ *     beta); We [H, de] (no bias); Wo [H*dh, dx]; bo [dx].
+ *   - Shapes: X, X', dX, dX' [B,n,dx]; E, E', dE, dE' [B,n,n,de]; y, dy [B,dy].
+ *   - Every pointer must be 16-byte aligned; outputs must not alias inputs.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  The return value reports host-side validation and
+ *     launch errors only; device-side conditions (a bounded wait that ran out)
+ *     are recorded in the workspace status word and read by
+ *     eaga_get_device_status.
+ *   - No global state besides cached kernel attributes and the optional
+ *     profiling events; calls on distinct streams with distinct workspaces
+ *     are thread-safe.
+ */
+#ifndef EAGA_H
+#define EAGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EAGA_API __attribute__((visibility("default")))
+#else
+#define EAGA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EAGA_OK = 0,
+    EAGA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive dim, bad dtype */
+    EAGA_ERR_UNSUPPORTED = 2,   /* dims outside the supported limits below */
+    EAGA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+    EAGA_ERR_WORKSPACE = 4,     /* workspace smaller than eaga_workspace_size() */
+    EAGA_ERR_CUDA = 5,          /* a CUDA launch or runtime call failed */
+    EAGA_ERR_TIMEOUT = 6        /* device-side bounded wait ran out (status word) */
+} eaga_status;
+
+typedef enum { EAGA_FP32 = 0, EAGA_BF16 = 1 } eaga_dtype;
+
+/* Problem dims.  Limits: 1 <= n <= 1024; H*dh <= 256 and dh % 8 == 0;
+ * de % 8 == 0, de <= 128; dx % 8 == 0, dx <= 1024; dy % 8 == 0, dy <= 1024;
+ * 2*H <= 32; H*n <= 8192.  Anything else returns EAGA_ERR_UNSUPPORTED. */
+typedef struct {
+    int B, n, dx, de, dy, H, dh;
+    int dtype;                  /* eaga_dtype */
+} eaga_dims;
+
+typedef struct {
+    const void *Wq, *bq, *Wk, *bk, *Wv, *bv, *Wfe, *Wfy, *bf, *We, *Wo, *bo;
+} eaga_weights;
+
+/* fp32 weight gradients, same shapes as the weights; overwritten, not accumulated. */
+typedef struct {
+    void *Wq, *bq, *Wk, *bk, *Wv, *bv, *Wfe, *Wfy, *bf, *We, *Wo, *bo;
+} eaga_weight_grads;
+
+/* Bytes of workspace eaga_forward (for_backward = 0) or eaga_backward
+ * (for_backward = 1) needs.  Grows as O(B*n*H*dh) + O(B*n*de*H); it has no
+ * B*H*n*n term.  Returns 0 for invalid or unsupported dims. */
+EAGA_API size_t eaga_workspace_size(const eaga_dims *dims, int for_backward);
+
+/* Bytes of the forward's saved state that eaga_backward consumes:
+ * LSE [B,H,n] fp32, then Q, K, V, O [B,n,H*dh] in the storage dtype, each
+ * region 256-byte aligned.  Returns 0 for invalid or unsupported dims. */
+EAGA_API size_t eaga_saved_size(const eaga_dims *dims);
+
+/* Forward of the layer (the formulas above).  Writes Xout and Eout.  `saved`
+ * (nullable; eaga_saved_size bytes) receives the state eaga_backward needs;
+ * with saved == NULL that state lives in the workspace and is discarded.
+ * `workspace` must hold eaga_workspace_size(dims, 0) bytes. */
+EAGA_API eaga_status eaga_forward(const eaga_dims *dims,
+                         const void *X, const void *E, const void *y, const uint8_t *M,
+                         const eaga_weights *w,
+                         void *Xout, void *Eout, void *saved,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/* Backward of the layer.  Given the forward's inputs, its `saved` state and
+ * the upstream gradients dXout, dEout, writes dX, dE, dy and every weight
+ * gradient (fp32).  `workspace` must hold eaga_workspace_size(dims, 1) bytes.
+ * Gradients of masked nodes / invalid pairs are the residual ones
+ * (dX_i = dX'_i, dE_ij = dE'_ij). */
+EAGA_API eaga_status eaga_backward(const eaga_dims *dims,
+                          const void *X, const void *E, const void *y, const uint8_t *M,
+                          const eaga_weights *w, const void *saved,
+                          const void *dXout, const void *dEout,
+                          void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
+                          void *workspace, size_t ws_bytes, void *stream);
+
+/* Test aid: writes the normalised coefficients A [B,H,n,n] (fp32) that the
+ * forward used, recomputed from E, y and the forward's `saved` state.  `A`
+ * must hold B*H*n*n + 2*B*H floats (the tail is scratch).  Writes O(B*H*n*n)
+ * memory; meant for small graphs only. */
+EAGA_API eaga_status eaga_debug_attention_map(const eaga_dims *dims, const void *E, const uint8_t *M,
+                                     const eaga_weights *w, const void *y, const void *saved,
+                                     float *A, void *stream);
+
+/* Synchronises `stream`, then reads and clears the device status word kept at
+ * the start of `workspace`: EAGA_OK, or EAGA_ERR_TIMEOUT if a bounded
+ * device-side wait ran out during a call that used this workspace. */
+EAGA_API eaga_status eaga_get_device_status(void *workspace, void *stream);
+
+/* Profiling aid.  After eaga_set_profile_events(point, before, after) with
+ * two cudaEvent_t handles, every later eaga_forward (point 0: the pair
+ * kernels of the forward) or eaga_backward (point 1: the pair kernels of the
+ * backward) records `before` on its stream just before launching those
+ * kernels and `after` just after them.  NULL events clear the point.  This
+ * is a process-wide setting: not for concurrent calls. */
+typedef enum { EAGA_PROF_FWD_PAIR = 0, EAGA_PROF_BWD_PAIR = 1 } eaga_prof_point;
+EAGA_API eaga_status eaga_set_profile_events(int point, void *before, void *after);
+
+/* Number of kernel launches (this library's kernels) that one eaga_forward
+ * (for_backward = 0) or eaga_backward (for_backward = 1) call issues for
+ * these dims; -1 for invalid or unsupported dims. */
+EAGA_API int eaga_kernel_launches(const eaga_dims *dims, int for_backward);
+
+/* Static, human-readable name of a status code. */
+EAGA_API const char *eaga_strerror(eaga_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EAGA_H */

@@ -1,0 +1,50 @@
+"""Shared helpers of the GPU parity tests: seeded cases, oracle calls, errors."""
+import numpy as np
+
+from edge_aware_graph_b200 import inputs as I
+
+TOL = {"fp32": 1e-4, "bf16": 2e-2}
+
+
+def rel_err(gpu, ref) -> float:
+    """max |gpu - ref| / max |ref| over one tensor (the parity measure)."""
+    g = gpu.detach().float().cpu().numpy().astype(np.float64) if hasattr(gpu, "detach") else np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = np.abs(ref).max()
+    if scale == 0:
+        return float(np.abs(g).max())
+    return float(np.abs(g - ref).max() / scale)
+
+
+def custom_case(B, n, dx, de, dy, H, dh, dtype, seed, mask="random", with_grads=True):
+    """Dense-family case of arbitrary dims with a chosen mask pattern.
+
+    mask: "prefix" (random real counts), "random" (non-prefix, includes one
+    fully masked graph and one single-node graph when B >= 3), "full".
+    """
+    p = I.Preset("custom", seed, dtype, B=B, n=n, dx=dx, de=de, dy=dy, H=H, dh=dh, family="dense",
+                 training=with_grads, n_real=(n,))
+    d = I.draw_inputs(p, with_grads=with_grads)
+    rng = np.random.default_rng(seed + 99)
+    if mask == "random":
+        M = (rng.random((B, n)) < 0.7).astype(np.uint8)
+        M[:, 0] = 1
+        if B >= 3:
+            M[1] = 0
+            M[2] = 0
+            M[2, n // 2] = 1
+    elif mask == "prefix":
+        nr = rng.integers(1, n + 1, size=B)
+        M = (np.arange(n)[None] < nr[:, None]).astype(np.uint8)
+    else:
+        M = np.ones((B, n), np.uint8)
+    d["M"] = M
+    return p, d, I.draw_weights(p)
+
+
+def oracle_forward(oracle, p, d, W, want_attention=False):
+    return oracle.forward(dict(H=p.H, dh=p.dh), d["X"], d["E"], d["y"], d["M"], W, want_attention=want_attention)
+
+
+def oracle_backward(oracle, p, d, W):
+    return oracle.backward(dict(H=p.H, dh=p.dh), d["X"], d["E"], d["y"], d["M"], W, d["dXout"], d["dEout"])

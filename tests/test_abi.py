@@ -1,0 +1,94 @@
+"""CPU checks of the C ABI: the library loads, exports every declared entry
+point, and its host-side validation returns the documented codes without
+touching a GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from edge_aware_graph_b200 import build as B
+from edge_aware_graph_b200 import eaga
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return eaga.lib()
+
+
+def declared_symbols():
+    out = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            out += re.findall(r"EAGA_API\s+[\w\s\*]+?\b(eaga_\w+)\s*\(", txt)
+    return sorted(set(out))
+
+
+def test_exports_every_declared_symbol(L):
+    syms = declared_symbols()
+    assert len(syms) >= 7
+    for s in syms:
+        assert hasattr(L, s), s
+    assert set(eaga.EXPORTED) <= set(syms)
+
+
+def good_dims():
+    return eaga.dims(32, 192, 256, 64, 64, 8, 32, "bf16")
+
+
+def test_sizes(L):
+    d = good_dims()
+    ws_f, ws_b, sv = eaga.workspace_size(d, False), eaga.workspace_size(d, True), eaga.saved_size(d)
+    assert ws_f > 0 and ws_b > 0 and sv > 0
+    # saved: LSE [B,H,n] fp32 + Q,K,V,O [B,n,256] bf16
+    assert sv >= 32 * 8 * 192 * 4 + 4 * 32 * 192 * 256 * 2
+    # no B*H*n^2 term: doubling n at fixed B*n... workspace scales linearly in B*n
+    d2 = eaga.dims(16, 384, 256, 64, 64, 8, 32, "bf16")
+    assert eaga.workspace_size(d2, True) < 1.2 * ws_b
+    big = eaga.dims(4, 1024, 256, 64, 64, 8, 32, "bf16")
+    assert eaga.workspace_size(big, True) < 4 * 8 * 1024 * 1024 * 4 / 2   # well below one fp32 attention map
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("n", 0, 1), ("B", -1, 1), ("dtype", 7, 1),
+    ("n", 1025, 2), ("de", 12, 2), ("dh", 12, 2), ("H", 17, 2), ("dx", 1032, 2),
+])
+def test_bad_dims(L, field, value, code):
+    d = good_dims()
+    setattr(d, field, value)
+    assert eaga.workspace_size(d, True) == 0
+    fake = ctypes.c_void_p(0x100000)
+    w = eaga.Weights(*([0x100000] * 12))
+    rc = L.eaga_forward(ctypes.byref(d), fake, fake, fake, fake, ctypes.byref(w), fake, fake, None, fake, 1 << 40,
+                        None)
+    assert rc == code
+
+
+def test_null_and_misaligned_and_workspace(L):
+    d = good_dims()
+    ok = ctypes.c_void_p(0x100000)
+    w = eaga.Weights(*([0x100000] * 12))
+    big = eaga.workspace_size(d, False)
+    f = L.eaga_forward
+    assert f(None, ok, ok, ok, ok, ctypes.byref(w), ok, ok, None, ok, big, None) == 1
+    assert f(ctypes.byref(d), None, ok, ok, ok, ctypes.byref(w), ok, ok, None, ok, big, None) == 1
+    assert f(ctypes.byref(d), ctypes.c_void_p(0x100008), ok, ok, ok, ctypes.byref(w), ok, ok, None, ok, big,
+             None) == 3
+    w_bad = eaga.Weights(*([0x100000] * 11 + [0x100004]))
+    assert f(ctypes.byref(d), ok, ok, ok, ok, ctypes.byref(w_bad), ok, ok, None, ok, big, None) == 3
+    assert f(ctypes.byref(d), ok, ok, ok, ok, ctypes.byref(w), ok, ok, None, ok, big - 1, None) == 4
+    g = L.eaga_backward
+    bigb = eaga.workspace_size(d, True)
+    assert g(ctypes.byref(d), ok, ok, ok, ok, ctypes.byref(w), ok, ok, ok, ok, ok, ok, None, ok, bigb, None) == 1
+    assert g(ctypes.byref(d), ok, ok, ok, ok, ctypes.byref(w), ok, ok, ok, ok, ok, ok, ctypes.byref(w), ok,
+             bigb - 1, None) == 4
+
+
+def test_strerror(L):
+    for code in range(7):
+        assert eaga.strerror(code)
+    assert eaga.strerror(99) == "unknown status"

@@ -1,0 +1,206 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Error measure: max|gpu - oracle| / max|oracle| per output tensor; bound 1e-4
+in fp32 storage mode and 2e-2 in bf16 storage mode (fp32 accumulation in
+both).  Cases: the tiny preset (fp32 and bf16), ragged shapes with
+non-prefix masks (an empty graph, a single-node graph), the generic and the
+specialised dims, and the full-size planar, tree, SBM and large presets.
+"""
+import numpy as np
+import pytest
+import torch
+
+from edge_aware_graph_b200 import inputs as I
+from edge_aware_graph_b200.buffers import LayerBuffers
+
+from harness import TOL, custom_case, oracle_backward, oracle_forward, rel_err
+
+pytestmark = pytest.mark.gpu
+
+GRAD_KEYS = ("dX", "dE", "dy") + tuple("d" + k for k in I.WEIGHT_NAMES)
+
+
+def make(p, d, W, backward):
+    buf = LayerBuffers(p.B, p.n, p.dx, p.de, p.dy, p.H, p.dh, dtype=p.dtype, backward=backward)
+    buf.load_inputs(d, W)
+    return buf
+
+
+def gpu_grads(buf):
+    out = {"dX": buf.dX, "dE": buf.dE, "dy": buf.dy}
+    for k in I.WEIGHT_NAMES:
+        out["d" + k] = buf.dW[k]
+    return out
+
+
+def check_forward(buf, ref, tol, rows=None):
+    errs = {"Xout": rel_err(buf.Xout, ref["Xout"]), "Eout": rel_err(buf.Eout, ref["Eout"])}
+    sv = buf.saved_parts()
+    errs["O"] = rel_err(sv["O"], ref["O"])
+    valid = np.isfinite(ref["LSE"])
+    lse = sv["LSE"].cpu().numpy()
+    errs["LSE"] = float(np.abs(lse[valid] - ref["LSE"][valid]).max() / np.abs(ref["LSE"][valid]).max()) if valid.any() else 0.0
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f"forward errors above {tol}: {bad} (all: {errs})"
+    return errs
+
+
+def check_backward(buf, ref, tol):
+    g = gpu_grads(buf)
+    errs = {k: rel_err(g[k], ref[k]) for k in GRAD_KEYS}
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f"backward errors above {tol}: {bad} (all: {errs})"
+    return errs
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_tiny_forward_backward(oracle_lib, dtype):
+    p = I.preset("tiny", dtype=dtype)
+    d = I.draw_inputs(p, with_grads=True)
+    W = I.draw_weights(p)
+    buf = make(p, d, W, backward=True)
+    buf.forward()
+    buf.backward()
+    torch.cuda.synchronize()
+    ref = oracle_forward(oracle_lib, p, d, W, want_attention=True)
+    check_forward(buf, ref, TOL[dtype])
+    A = buf.attention_map()
+    assert rel_err(A, ref["A"]) <= TOL[dtype]
+    check_backward(buf, oracle_backward(oracle_lib, p, d, W), TOL[dtype])
+
+
+CASES = [
+    # B, n, dx, de, dy, H, dh, dtype, mask
+    (3, 37, 24, 24, 16, 3, 16, "fp32", "random"),
+    (4, 64, 256, 64, 64, 8, 32, "bf16", "random"),
+    (3, 100, 256, 64, 64, 8, 32, "bf16", "prefix"),
+    (2, 130, 256, 64, 64, 8, 32, "bf16", "random"),
+    (2, 200, 64, 32, 8, 4, 16, "bf16", "prefix"),
+    (5, 1, 16, 8, 8, 2, 8, "fp32", "full"),
+    (2, 257, 256, 64, 64, 8, 32, "bf16", "random"),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "x".join(map(str, c[:7])) + f"-{c[7]}-{c[8]}")
+def test_ragged_shapes(oracle_lib, case):
+    B, n, dx, de, dy, H, dh, dtype, mask = case
+    p, d, W = custom_case(B, n, dx, de, dy, H, dh, dtype, seed=10 + n, mask=mask)
+    buf = make(p, d, W, backward=True)
+    buf.forward()
+    buf.backward()
+    torch.cuda.synchronize()
+    check_forward(buf, oracle_forward(oracle_lib, p, d, W), TOL[dtype])
+    check_backward(buf, oracle_backward(oracle_lib, p, d, W), TOL[dtype])
+
+
+def test_masked_garbage_is_ignored():
+    """Large finite values in masked node rows and invalid pairs leave every
+    valid output bitwise unchanged; masked outputs equal their inputs."""
+    p, d, W = custom_case(4, 96, 256, 64, 64, 8, 32, "bf16", seed=3, mask="random")
+    buf = make(p, d, W, backward=True)
+    buf.forward(); buf.backward()
+    base = {k: getattr(buf, k).clone() for k in ("Xout", "Eout", "dX", "dE", "dy")}
+    base_dw = {k: v.clone() for k, v in buf.dW.items()}
+    rows = d["M"].astype(bool)
+    valid = rows[:, :, None] & rows[:, None, :]
+    rng = np.random.default_rng(1)
+    d2 = dict(d)
+    d2["X"] = d["X"].copy(); d2["X"][~rows] = I.to_storage(rng.standard_normal(d2["X"][~rows].shape) * 1e3, "bf16")
+    d2["E"] = d["E"].copy(); d2["E"][~valid] = I.to_storage(rng.standard_normal(d2["E"][~valid].shape) * 1e3, "bf16")
+    buf.load_inputs(d2, W)
+    buf.forward(); buf.backward()
+    torch.cuda.synchronize()
+    vt = torch.from_numpy(valid).cuda()
+    rt = torch.from_numpy(rows).cuda()
+    assert torch.equal(buf.Xout[rt], base["Xout"][rt])
+    assert torch.equal(buf.Eout[vt], base["Eout"][vt])
+    assert torch.equal(buf.dX[rt], base["dX"][rt])
+    assert torch.equal(buf.dE[vt], base["dE"][vt])
+    assert torch.equal(buf.dy, base["dy"])
+    for k in base_dw:
+        assert torch.equal(buf.dW[k], base_dw[k]), k
+    assert torch.equal(buf.Xout[~rt], buf.X[~rt])
+    assert torch.equal(buf.Eout[~vt], buf.E[~vt])
+    assert torch.equal(buf.dE[~vt], buf.dEout[~vt])
+
+
+def test_permutation_equivariance_gpu():
+    p, d, W = custom_case(2, 80, 256, 64, 64, 8, 32, "bf16", seed=8, mask="random", with_grads=False)
+    buf = make(p, d, W, backward=False)
+    buf.forward()
+    X0, E0 = buf.Xout.float().cpu().numpy(), buf.Eout.float().cpu().numpy()
+    perm = np.random.default_rng(2).permutation(p.n)
+    d2 = dict(d)
+    d2["X"], d2["E"], d2["M"] = d["X"][:, perm], d["E"][:, perm][:, :, perm], d["M"][:, perm]
+    buf.load_inputs(d2, W)
+    buf.forward()
+    torch.cuda.synchronize()
+    assert rel_err(buf.Xout, X0[:, perm]) <= TOL["bf16"]
+    assert rel_err(buf.Eout, E0[:, perm][:, :, perm]) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("name", ["planar", "tree"])
+def test_forward_presets(oracle_lib, name):
+    p = I.preset(name)
+    d = I.draw_inputs(p, with_grads=False)
+    W = I.draw_weights(p)
+    buf = make(p, d, W, backward=False)
+    buf.forward()
+    torch.cuda.synchronize()
+    check_forward(buf, oracle_forward(oracle_lib, p, d, W), TOL[p.dtype])
+
+
+def test_sbm_training_step(oracle_lib):
+    p = I.preset("sbm")
+    d = I.draw_inputs(p)
+    W = I.draw_weights(p)
+    buf = make(p, d, W, backward=True)
+    buf.forward()
+    buf.backward()
+    torch.cuda.synchronize()
+    check_forward(buf, oracle_forward(oracle_lib, p, d, W), TOL[p.dtype])
+    check_backward(buf, oracle_backward(oracle_lib, p, d, W), TOL[p.dtype])
+
+
+@pytest.mark.slow
+def test_large_training_step(oracle_lib):
+    """Full-size large preset on the GPU; the oracle runs one graph at a time
+    (graphs are independent; weight gradients are sums over graphs)."""
+    p = I.preset("large")
+    d = I.draw_inputs(p)
+    W = I.draw_weights(p)
+    buf = make(p, d, W, backward=True)
+    buf.forward()
+    buf.backward()
+    torch.cuda.synchronize()
+    tol = TOL[p.dtype]
+    gw = {k: np.zeros(W[k].shape) for k in I.WEIGHT_NAMES}
+    errs = {}
+    sv = buf.saved_parts()
+    for b in range(p.B):
+        sl = {k: d[k][b:b + 1] for k in ("X", "E", "y", "M", "dXout", "dEout")}
+        pb = I.preset("large", B=1)
+        rf = oracle_forward(oracle_lib, pb, sl, W)
+        errs[f"Xout{b}"] = rel_err(buf.Xout[b:b + 1], rf["Xout"])
+        errs[f"Eout{b}"] = rel_err(buf.Eout[b:b + 1], rf["Eout"])
+        errs[f"O{b}"] = rel_err(sv["O"][b:b + 1], rf["O"])
+        del rf
+        rb = oracle_backward(oracle_lib, pb, sl, W)
+        errs[f"dX{b}"] = rel_err(buf.dX[b:b + 1], rb["dX"])
+        errs[f"dE{b}"] = rel_err(buf.dE[b:b + 1], rb["dE"])
+        errs[f"dy{b}"] = rel_err(buf.dy[b:b + 1], rb["dy"])
+        for k in I.WEIGHT_NAMES:
+            gw[k] += rb["d" + k]
+        del rb
+    for k in I.WEIGHT_NAMES:
+        errs["d" + k] = rel_err(buf.dW[k], gw[k])
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f"errors above {tol}: {bad}"
+
+
+def test_device_status_ok():
+    from edge_aware_graph_b200 import eaga
+    p, d, W = custom_case(2, 16, 16, 8, 8, 2, 8, "fp32", seed=1, mask="full", with_grads=False)
+    buf = make(p, d, W, backward=False)
+    buf.forward()
+    assert eaga.get_device_status(buf.ws_fwd) == 0
