@@ -162,6 +162,9 @@ def run_ours(args):
     ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for a, b in ev_f + ev_b:          # torch creates the CUDA event on first record
+        a.record(stream)
+        b.record(stream)
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
