@@ -3,7 +3,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
-#include "../../include/eaga.h"
+#include "eaga.h"
 
 namespace eaga {
 

@@ -56,9 +56,8 @@ extern "C" {
 size_t eaga_workspace_size(const eaga_dims *d, int for_backward) {
     if (check_dims(d) != EAGA_OK) return 0;
     const WsLayout W = ws_layout(*d);
-    size_t bytes = for_backward ? W.total_bwd : W.total_fwd;
-    const size_t extra = fast::workspace_extra(*d, for_backward);
-    return bytes + extra;
+    if (fast::supports(*d)) return fast::workspace_size(*d, for_backward, W.total_fwd, W.fwd_saved);
+    return for_backward ? W.total_bwd : W.total_fwd;
 }
 
 size_t eaga_saved_size(const eaga_dims *d) {
@@ -134,7 +133,7 @@ eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, cons
     a.status = reinterpret_cast<int *>(ws + W.status);
     if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
     if (fast::supports(*d)) {
-        return launch_status(fast::backward(*d, a, ws + W.total_bwd, st));
+        return launch_status(fast::backward(*d, a, ws, W.fwd_saved, st));
     }
     return launch_status(generic::backward(*d, a, st));
 }

@@ -5,9 +5,11 @@
 namespace eaga {
 namespace fast {
 bool supports(const eaga_dims &d);
-size_t workspace_extra(const eaga_dims &d, int for_backward);
+// common_fwd: end of the common forward workspace; common_head: end of the
+// status word and g (start of the backward's own regions).
+size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, size_t common_head);
 int kernel_launches(const eaga_dims &d, int for_backward);
-cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_extra, cudaStream_t st);
-cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws_extra, cudaStream_t st);
+cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st);
+cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head, cudaStream_t st);
 }  // namespace fast
 }  // namespace eaga

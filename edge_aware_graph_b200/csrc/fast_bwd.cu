@@ -1,0 +1,752 @@
+// Backward pair kernels for de = 64, H = 8, dh = 32, bf16 storage (sm_100a).
+//
+// Chain rule of the layer (same formulas as the forward's, differentiated):
+//   u_ij^h = We[h,:] . dE'_ij          dA^h_ij = dO_ih . v_jh + u_ij^h
+//   D_ih   = sum_j a_ij dA_ij          dS'_ij  = a_ij (dA_ij - D_ih)
+//   dgamma = dS' s,  dbeta = dS',  ds = dS' (1 + gamma)
+//   dq_i = sum_j ds_ij k_j / sqrt(dh),  dk_j = sum_i ds_ij q_i / sqrt(dh),  dv_j = sum_i a_ij dO_i
+//   dE = dE' + [dgamma|dbeta] Wfe^T,  dWfe = sum E^T [dgamma|dbeta],  dWe = sum a^T dE',  dg = sum [dgamma|dbeta]
+// D needs a whole row of pairs before any dS' exists, so the work is split in
+//   k_bwd_rows: clusters along j (like the forward): a, u, dA, cluster-wide D,
+//               dS', dq (cluster-reduced), dE (tensor cores, written in place,
+//               TMA store), dWfe / dWe / dg partials reduced over the cluster;
+//   k_bwd_cols: clusters along i on the transposed tile: a and ds again from
+//               E, dE' and the D of the row kernel; dk, dv reduced over the
+//               cluster.
+// Both tiles are loaded once with TMA and stay in shared memory; the FiLM and
+// u = dE' We^T products run on tcgen05 with the same pair <-> TMEM lane map as
+// the forward.  16 warps: warp W reads TMEM quadrant W%4, heads 2(W/4)+{0,1}.
+// NR selects 32NR cluster rows per CTA (NR = 1: two CTAs share an SM).
+#include <math.h>
+#include "fast.h"
+#include "fast_common.cuh"
+
+namespace eaga {
+namespace fast {
+
+using namespace sm100;
+using namespace dev;
+
+struct BwdRowParams {
+    const __nv_bfloat16 *Q, *dO;
+    const float *LSE, *g;
+    const uint8_t *img, *M;
+    float *D;                // [B,H,n] out
+    __nv_bfloat16 *dQ;       // [B,n,256] out (scaled)
+    float *rparts;           // [graph * row block][RPART] out
+    int *status;
+    int n;
+};
+
+struct BwdColParams {
+    const __nv_bfloat16 *K, *V;
+    const float *LSE, *D, *g;
+    const uint8_t *img, *M;
+    __nv_bfloat16 *dK, *dV;  // [B,n,256] out (dK scaled)
+    int *status;
+    int n;
+};
+
+// ---------------------------------------------------------------- row kernel
+
+template <int NR>
+struct RowSmem {
+    static constexpr uint32_t E = 0, DEP = NR * 32768, K = NR * 65536, V = K + NR * 16384;
+    static constexpr uint32_t DF = V, AT = V + NR * 8192;          // reuse of the V chunk after dP
+    static constexpr uint32_t IMG = V + NR * 16384;                // Wfe^T sw, We sw, Wfe ns (2 KB each)
+    static constexpr uint32_t WD = IMG + 6144;                     // per-quadrant D partials [4][8][8]
+    static constexpr uint32_t CD = WD + 1024;                      // CTA D [64] (read by peers)
+    static constexpr uint32_t FD = CD + 256;                       // final D [64]
+    static constexpr uint32_t WDG = FD + 256;                      // per-warp dg [16][4]
+    static constexpr uint32_t G = WDG + 256;
+    static constexpr uint32_t LSE = G + 64;                        // [8 i][8 h]
+    static constexpr uint32_t MI = LSE + 256, MJ = MI + 16;
+    static constexpr uint32_t BAR = MJ + 64;                       // 6 mbarriers
+    static constexpr uint32_t TM = BAR + 48;
+    static constexpr uint32_t WP = TM + 16;                        // CTA weight-grad partial (read by peers)
+    static constexpr uint32_t BYTES = WP + RPART * 4 + 1024;
+    static constexpr uint32_t QPART = K;                           // 32 KB dq quadrant partials (K, V dead)
+};
+
+template <int NR>
+__global__ void __launch_bounds__(NTHR, NR == 1 ? 2 : 1)
+k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmDEp,
+           const __grid_constant__ CUtensorMap tmDE, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, BwdRowParams p) {
+    using S = RowSmem<NR>;
+    constexpr int TCN = tile_cols(NR), NE = 2 * NR;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
+    const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = W >> 2, t = tid & 31, c4 = t & 3, g8 = t >> 2;
+    const uint32_t rank = cluster_rank(), nclu = gridDim.x;
+    const int n = p.n;
+    const int j0 = blockIdx.x * TCN, i0 = blockIdx.y * TB, b = blockIdx.z;
+    const uint32_t bar_e = sbase + S::BAR, bar_dep = bar_e + 8, bar_kv = bar_e + 16, bar_film = bar_e + 24,
+                   bar_u = bar_e + 32, bar_de = bar_e + 40;
+    float *g = reinterpret_cast<float *>(sp + S::G);
+    float *lse = reinterpret_cast<float *>(sp + S::LSE);
+    uint8_t *mi = sp + S::MI, *mj = sp + S::MJ;
+    constexpr uint32_t TM_FILM = 0, TM_U = 64, TM_DE = 128, TM_COLS = 256;
+
+    if (tid == 0) {
+        mbar_init(bar_e, 1); mbar_init(bar_dep, 1); mbar_init(bar_kv, 1);
+        mbar_init(bar_film, 1); mbar_init(bar_u, 1); mbar_init(bar_de, 1);
+        fence_mbar_init();
+        mbar_expect_tx(bar_e, NR * 32768);
+        tma_load_5d(sbase + S::E, &tmE, bar_e, 0, i0 / 2, j0, 0, b);
+        mbar_expect_tx(bar_dep, NR * 32768);
+        tma_load_5d(sbase + S::DEP, &tmDEp, bar_dep, 0, i0 / 2, j0, 0, b);
+        mbar_expect_tx(bar_kv, NR * 32768);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            tma_load_3d(sbase + S::K + k * NR * 4096, &tmK, bar_kv, 64 * k, j0, b);
+            tma_load_3d(sbase + S::V + k * NR * 4096, &tmV, bar_kv, 64 * k, j0, b);
+        }
+    }
+    if (W == 0) {
+        tmem_alloc(sbase + S::TM, TM_COLS);
+        tmem_relinquish();
+    }
+    if (tid < 384) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.img);
+        const uint32_t img_off = (tid >> 7) == 0 ? IMG_WFE_T_SW : (tid >> 7) == 1 ? IMG_WE_SW : IMG_WFE_NS;
+        reinterpret_cast<uint4 *>(sp + S::IMG)[tid] = src[(img_off >> 4) + (tid & 127)];
+    }
+    if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
+    if (tid >= 32 && tid < 32 + TB) mi[tid - 32] = (i0 + tid - 32 < n) ? p.M[(size_t)b * n + i0 + tid - 32] : 0;
+    if (tid >= 64 && tid < 64 + TCN) mj[tid - 64] = (j0 + tid - 64 < n) ? p.M[(size_t)b * n + j0 + tid - 64] : 0;
+    if (tid >= 128 && tid < 192) {
+        const int x = tid - 128, il = x >> 3, h = x & 7;
+        lse[x] = (i0 + il < n) ? p.LSE[((size_t)b * NH + h) * n + i0 + il] : 0.f;
+    }
+    uint32_t qf[2][2][2], of[2][2][2];
+    load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
+    load_frags2(p.dO, b, n, i0, hq, g8, c4, of);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+
+    if (tid == 0) {
+        if (!mbar_wait(bar_e, 0)) flag_timeout(p.status);
+        tc_fence_after();
+        issue_pair_products<NR>(sbase + S::E, sbase + S::IMG, tmem + TM_FILM);
+        mma_commit(bar_film);
+        if (!mbar_wait(bar_dep, 0)) flag_timeout(p.status);
+        tc_fence_after();
+        issue_pair_products<NR>(sbase + S::DEP, sbase + S::IMG + 2048, tmem + TM_U);
+        mma_commit(bar_u);
+    }
+    __syncwarp();
+    if (!mbar_wait(bar_kv, 0)) flag_timeout(p.status);
+    float sv[2][4], da[2][4], av[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    warp_scores2<NR>(sbase + S::K, q, t, hq, qf, sv);
+    warp_scores2<NR>(sbase + S::V, q, t, hq, of, da);
+
+    if (!mbar_wait(bar_film, 0)) flag_timeout(p.status);
+    if (!mbar_wait(bar_u, 0)) flag_timeout(p.status);
+    tc_fence_after();
+    const float rs = rsqrtf((float)DH);
+    float gm[2][4];
+#pragma unroll
+    for (int e = 0; e < NE; ++e) {
+        const int jl = 32 * (e >> 1) + 8 * q + g8, il = 2 * c4 + (e & 1);
+        const bool valid = mi[il] && mj[jl];
+        float f0, f1, b0, b1, u0, u1;
+        tmem_ld2(tl + TM_FILM + 16 * e + 2 * hq, f0, f1);
+        tmem_ld2(tl + TM_FILM + 16 * e + NH + 2 * hq, b0, b1);
+        tmem_ld2(tl + TM_U + 16 * e + 2 * hq, u0, u1);
+        tmem_ld_wait();
+        const float fg[2] = {f0, f1}, fb[2] = {b0, b1}, fu[2] = {u0, u1};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int h = 2 * hq + hh;
+            const float s = sv[hh][e] * rs;
+            const float gam = fg[hh] + g[h], bet = fb[hh] + g[NH + h];
+            av[hh][e] = valid ? exp2f((s * (1.f + gam) + bet - lse[il * 8 + h]) * LOG2E) : 0.f;
+            sv[hh][e] = s;
+            gm[hh][e] = gam;
+            da[hh][e] += fu[hh];
+        }
+    }
+    // D_ih = sum_j a dA: warp, CTA, cluster
+    float *wd = reinterpret_cast<float *>(sp + S::WD);
+    float *cd = reinterpret_cast<float *>(sp + S::CD);
+    float *fd = reinterpret_cast<float *>(sp + S::FD);
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float x = av[hh][s] * da[hh][s];
+            if (NR == 2) x += av[hh][2 + s] * da[hh][2 + s];
+            x += __shfl_xor_sync(0xffffffffu, x, 4);
+            x += __shfl_xor_sync(0xffffffffu, x, 8);
+            x += __shfl_xor_sync(0xffffffffu, x, 16);
+            if (g8 == 0) wd[(q * 8 + 2 * c4 + s) * 8 + 2 * hq + hh] = x;
+        }
+    __syncthreads();
+    if (tid < 64) cd[tid] = wd[tid] + wd[64 + tid] + wd[128 + tid] + wd[192 + tid];
+    cluster_sync();
+    cluster_combine64<1>(sp, sbase, S::CD, S::FD, tid, nclu);
+    __syncthreads();
+    if (tid < 64) {
+        const int il = tid >> 3, h = tid & 7;
+        if (rank == 0 && i0 + il < n) p.D[((size_t)b * NH + h) * n + i0 + il] = fd[tid];
+    }
+
+    // dS', df = [dgamma | dbeta], ds = dS'(1+gamma); df and a tiles for the tensor cores
+    float dgp[4] = {0.f, 0.f, 0.f, 0.f};   // dgamma h0, h1, dbeta h0, h1
+    const uint32_t L = 32 * q + t;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        if (e >= NE) {
+            da[0][e] = da[1][e] = 0.f;
+            continue;
+        }
+        const int il = 2 * c4 + (e & 1);
+        float dgam[2], dbet[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const float dsp = av[hh][e] * (da[hh][e] - fd[il * 8 + 2 * hq + hh]);
+            dgam[hh] = dsp * sv[hh][e];
+            dbet[hh] = dsp;
+            da[hh][e] = dsp * (1.f + gm[hh][e]);     // ds (unscaled)
+            dgp[hh] += dgam[hh];
+            dgp[2 + hh] += dbet[hh];
+        }
+        *reinterpret_cast<uint32_t *>(sp + S::DF + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(dgam[0], dgam[1]);
+        *reinterpret_cast<uint32_t *>(sp + S::DF + e * 4096 + ns16(L, NH + 2 * hq)) = pack_bf16(dbet[0], dbet[1]);
+        *reinterpret_cast<uint32_t *>(sp + S::AT + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(av[0][e], av[1][e]);
+        if (hq == 0) *reinterpret_cast<uint4 *>(sp + S::AT + e * 4096 + ns16(L, 8)) = make_uint4(0, 0, 0, 0);
+    }
+    float *wdg = reinterpret_cast<float *>(sp + S::WDG);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float x = dgp[k];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (t == 0) wdg[W * 4 + k] = x;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    const uint32_t idesc_de = idesc_bf16_f32(128, DE);
+    if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ee = 0; ee < 2; ++ee)
+            mma_bf16_ss(tmem + TM_DE + 64 * ee, smem_desc(sbase + S::DF + ee * 4096, 128, 256, LAYOUT_NONE),
+                        smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_de, 0);
+        mma_commit(bar_de);
+    }
+    __syncwarp();
+
+    // dq partial = K^T ds^T (warp MMAs)
+    float qacc[2][2][4];
+    warp_contract2<NR>(sbase + S::K, q, t, hq, da, qacc);
+
+    // dWfe [64 c][16 k] and dWe^T [64 c][8 h] partials: warp W owns c in
+    // [16ct, 16ct+16) (ct = W%4) over k-range kr = W/4 of the CTA's pairs; the
+    // four k-ranges are added in a fixed order.
+    {
+        const int ct = W & 3, kr = W >> 2;
+        float wf[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float we4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int kk = 4 * NR * kr; kk < 4 * NR * (kr + 1); ++kk) {
+            const int e = kk >> 3, L0 = 16 * (kk & 7);
+            const uint32_t row0 = tile_off<NR>(e) / 128 + L0;
+            const uint32_t arow = row0 + (t & 7) + ((t >> 4) & 1) * 8;
+            const uint32_t ach = 2 * ct + ((t >> 3) & 1);
+            uint32_t aE[4], aD[4], bF[4], bA0, bA1;
+            ldsm_x4_t(sbase + S::E + sw128(arow, ach), aE);
+            ldsm_x4_t(sbase + S::DEP + sw128(arow, ach), aD);
+            const uint32_t Lr = L0 + (t & 7) + ((t >> 3) & 1) * 8;
+            ldsm_x4_t(sbase + S::DF + e * 4096 + ns16(Lr, 8 * (t >> 4)), bF);
+            ldsm_x2_t(sbase + S::AT + e * 4096 + ns16(Lr, 0), bA0, bA1);
+            mma16816(wf[0], aE, bF[0], bF[1]);
+            mma16816(wf[1], aE, bF[2], bF[3]);
+            mma16816(we4, aD, bA0, bA1);
+        }
+        float *rp = reinterpret_cast<float *>(sp + S::WP);
+        for (int phase = 0; phase < 4; ++phase) {
+            if (kr == phase) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 16 * ct + g8 + 8 * (e >> 1), k = nt * 8 + 2 * c4 + (e & 1);
+                        rp[c * NF + k] = (phase ? rp[c * NF + k] : 0.f) + wf[nt][e];
+                    }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 16 * ct + g8 + 8 * (e >> 1), h = 2 * c4 + (e & 1);
+                    float *dst = rp + DE * NF + h * DE + c;
+                    *dst = (phase ? *dst : 0.f) + we4[e];
+                }
+            }
+            __syncthreads();
+        }
+        if (tid < NF) {
+            const int which = tid >> 3, h = tid & 7, hq2 = h >> 1, hh = h & 1;
+            float x = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x += wdg[(4 * hq2 + k) * 4 + which * 2 + hh];
+            rp[DE * NF + NH * DE + tid] = x;
+        }
+    }
+    // sum the CTA partials over the cluster: one partial per (graph, row block)
+    cluster_sync();
+    {
+        float *rp = p.rparts + (size_t)(blockIdx.z * gridDim.y + blockIdx.y) * RPART;
+        const int per = (RPART + nclu - 1) / nclu;
+        for (int x = rank * per + tid; x < min((int)(rank + 1) * per, RPART); x += NTHR) {
+            float acc = 0.f;
+            for (uint32_t k0 = 0; k0 < nclu; k0 += 4) {
+                float v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) v[u] = (k0 + u < nclu) ? ld_peer_f32(map_peer(sbase + S::WP + x * 4, k0 + u)) : 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc += v[u];
+            }
+            rp[x] = acc;
+        }
+    }
+
+    // dE = dE' + df Wfe^T, written in place over the dE' tile, NR rounds of two MMAs
+    for (int round = 0; round < NR; ++round) {
+        if (!mbar_wait(bar_de, round)) flag_timeout(p.status);
+        tc_fence_after();
+#pragma unroll
+        for (int ee = 0; ee < 2; ++ee) {
+            const int e = 2 * round + ee;
+            float dv[16];
+            tmem_ld16(tl + TM_DE + 64 * ee + 16 * hq, dv);
+            tmem_ld_wait();
+            add_residual16(sp + S::DEP + tile_off<NR>(e) + L * 128, L, hq, dv);
+        }
+        if (round + 1 < NR) {
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ee = 0; ee < 2; ++ee)
+                    mma_bf16_ss(tmem + TM_DE + 64 * ee,
+                                smem_desc(sbase + S::DF + (2 * (round + 1) + ee) * 4096, 128, 256, LAYOUT_NONE),
+                                smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_de, 0);
+                mma_commit(bar_de);
+            }
+            __syncwarp();
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        tma_store_5d(&tmDE, sbase + S::DEP, 0, i0 / 2, j0, 0, b);
+        tma_store_commit();
+    }
+    // dq: reduce over the quadrant warps and the cluster
+    store_quadrant_part(sp, S::QPART, qacc, q, hq, t);
+    {
+        const uint32_t parts[1] = {S::QPART};
+        __nv_bfloat16 *const outs[1] = {p.dQ};
+        const float sc[1] = {rs};
+        cluster_reduce_rows<1>(sbase, parts, tid, rank, nclu, outs, b, n, i0, sc);
+    }
+    if (tid == 0) tma_store_wait_read0();
+    tc_fence_before();
+    cluster_wait();
+    if (W == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+// ---------------------------------------------------------------- column kernel
+
+template <int NR>
+struct ColSmem {
+    static constexpr uint32_t E = 0, DEP = NR * 32768, Q = NR * 65536, DO = Q + NR * 16384;
+    static constexpr uint32_t IMG = DO + NR * 16384;               // Wfe^T sw, We sw
+    static constexpr uint32_t G = IMG + 4096;
+    static constexpr uint32_t MI = G + 64, MJ = MI + 64;
+    static constexpr uint32_t BAR = MJ + 16;                       // 5 mbarriers
+    static constexpr uint32_t TM = BAR + 40;
+    static constexpr uint32_t BYTES = TM + 24 + 1024;
+    static constexpr uint32_t KPART = E, VPART = DEP;              // 32 KB quadrant partials each (tiles dead)
+};
+
+template <int NR>
+__global__ void __launch_bounds__(NTHR, NR == 1 ? 2 : 1)
+k_bwd_cols(const __grid_constant__ CUtensorMap tmEt, const __grid_constant__ CUtensorMap tmDEpt,
+           const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO, BwdColParams p) {
+    using S = ColSmem<NR>;
+    constexpr int TCN = tile_cols(NR), NE = 2 * NR;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
+    const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = W >> 2, t = tid & 31, c4 = t & 3, g8 = t >> 2;
+    const uint32_t rank = cluster_rank(), nclu = gridDim.x;
+    const int n = p.n;
+    const int i0 = blockIdx.x * TCN, j0 = blockIdx.y * TB, b = blockIdx.z;   // 32NR rows i, 8 columns j
+    const uint32_t bar_e = sbase + S::BAR, bar_dep = bar_e + 8, bar_q = bar_e + 16, bar_film = bar_e + 24,
+                   bar_u = bar_e + 32;
+    float *g = reinterpret_cast<float *>(sp + S::G);
+    uint8_t *mi = sp + S::MI, *mj = sp + S::MJ;
+    constexpr uint32_t TM_FILM = 0, TM_U = 64, TM_COLS = 128;
+
+    if (tid == 0) {
+        mbar_init(bar_e, 1); mbar_init(bar_dep, 1); mbar_init(bar_q, 1);
+        mbar_init(bar_film, 1); mbar_init(bar_u, 1);
+        fence_mbar_init();
+        mbar_expect_tx(bar_e, NR * 32768);
+        tma_load_5d(sbase + S::E, &tmEt, bar_e, 0, j0 / 2, i0, 0, b);
+        mbar_expect_tx(bar_dep, NR * 32768);
+        tma_load_5d(sbase + S::DEP, &tmDEpt, bar_dep, 0, j0 / 2, i0, 0, b);
+        mbar_expect_tx(bar_q, NR * 32768);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            tma_load_3d(sbase + S::Q + k * NR * 4096, &tmQ, bar_q, 64 * k, i0, b);
+            tma_load_3d(sbase + S::DO + k * NR * 4096, &tmDO, bar_q, 64 * k, i0, b);
+        }
+    }
+    if (W == 0) {
+        tmem_alloc(sbase + S::TM, TM_COLS);
+        tmem_relinquish();
+    }
+    if (tid < 256) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.img);
+        const uint32_t img_off = (tid >> 7) == 0 ? IMG_WFE_T_SW : IMG_WE_SW;
+        reinterpret_cast<uint4 *>(sp + S::IMG)[tid] = src[(img_off >> 4) + (tid & 127)];
+    }
+    if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
+    if (tid >= 64 && tid < 64 + TCN) mi[tid - 64] = (i0 + tid - 64 < n) ? p.M[(size_t)b * n + i0 + tid - 64] : 0;
+    if (tid >= 32 && tid < 32 + TB) mj[tid - 32] = (j0 + tid - 32 < n) ? p.M[(size_t)b * n + j0 + tid - 32] : 0;
+    // per-thread rows i = i0 + 32r + 8q + g8: LSE and D for the warp's 2 heads
+    float lse[2][2], dd[2][2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int i = i0 + 32 * r + 8 * q + g8;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const size_t o = ((size_t)b * NH + 2 * hq + hh) * n + i;
+            const bool ok = (r < NR) && i < n;
+            lse[r][hh] = ok ? p.LSE[o] : 0.f;
+            dd[r][hh] = ok ? p.D[o] : 0.f;
+        }
+    }
+    uint32_t kf[2][2][2], vf[2][2][2];
+    load_frags2(p.K, b, n, j0, hq, g8, c4, kf);
+    load_frags2(p.V, b, n, j0, hq, g8, c4, vf);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+
+    if (tid == 0) {
+        if (!mbar_wait(bar_e, 0)) flag_timeout(p.status);
+        tc_fence_after();
+        issue_pair_products<NR>(sbase + S::E, sbase + S::IMG, tmem + TM_FILM);
+        mma_commit(bar_film);
+        if (!mbar_wait(bar_dep, 0)) flag_timeout(p.status);
+        tc_fence_after();
+        issue_pair_products<NR>(sbase + S::DEP, sbase + S::IMG + 2048, tmem + TM_U);
+        mma_commit(bar_u);
+    }
+    __syncwarp();
+    if (!mbar_wait(bar_q, 0)) flag_timeout(p.status);
+    // S = Q K^T and dP = dO V^T on the transposed tile: rows i (M), columns j (N)
+    float sv[2][4], da[2][4];
+    warp_scores2<NR>(sbase + S::Q, q, t, hq, kf, sv);
+    warp_scores2<NR>(sbase + S::DO, q, t, hq, vf, da);
+
+    if (!mbar_wait(bar_film, 0)) flag_timeout(p.status);
+    if (!mbar_wait(bar_u, 0)) flag_timeout(p.status);
+    tc_fence_after();
+    const float rs = rsqrtf((float)DH);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        if (e >= NE) {
+            sv[0][e] = sv[1][e] = da[0][e] = da[1][e] = 0.f;
+            continue;
+        }
+        const int r = e >> 1, il = 32 * r + 8 * q + g8, jl = 2 * c4 + (e & 1);
+        const bool valid = mi[il] && mj[jl];
+        float f0, f1, b0, b1, u0, u1;
+        tmem_ld2(tl + TM_FILM + 16 * e + 2 * hq, f0, f1);
+        tmem_ld2(tl + TM_FILM + 16 * e + NH + 2 * hq, b0, b1);
+        tmem_ld2(tl + TM_U + 16 * e + 2 * hq, u0, u1);
+        tmem_ld_wait();
+        const float fg[2] = {f0, f1}, fb[2] = {b0, b1}, fu[2] = {u0, u1};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int h = 2 * hq + hh;
+            const float s = sv[hh][e] * rs;
+            const float gam = fg[hh] + g[h], bet = fb[hh] + g[NH + h];
+            const float a = valid ? exp2f((s * (1.f + gam) + bet - lse[r][hh]) * LOG2E) : 0.f;
+            const float dsp = a * (da[hh][e] + fu[hh] - dd[r][hh]);
+            sv[hh][e] = a;                       // a
+            da[hh][e] = dsp * (1.f + gam);       // ds
+        }
+    }
+    tc_fence_before();
+    __syncthreads();   // tiles are dead: their space holds the partials below
+    float kacc[2][2][4], vacc[2][2][4];
+    warp_contract2<NR>(sbase + S::Q, q, t, hq, da, kacc);    // dk^T = Q^T ds
+    warp_contract2<NR>(sbase + S::DO, q, t, hq, sv, vacc);   // dv^T = dO^T a
+    store_quadrant_part(sp, S::KPART, kacc, q, hq, t);
+    store_quadrant_part(sp, S::VPART, vacc, q, hq, t);
+    {
+        const uint32_t parts[2] = {S::KPART, S::VPART};
+        __nv_bfloat16 *const outs[2] = {p.dK, p.dV};
+        const float sc[2] = {rs, 1.f};
+        cluster_reduce_rows<2>(sbase, parts, tid, rank, nclu, outs, b, n, j0, sc);
+    }
+    tc_fence_before();
+    cluster_wait();
+    if (W == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+// ---------------------------------------------------------------- reductions
+// All sums run in a fixed order (deterministic): first over segments of rows
+// (or CTAs) in parallel blocks, then over the segments.
+
+// Column sums of segment z of a row-major matrix: out[z][col].  Sources by
+// column: [0,256) dQ, [256,512) dK, [512,768) dV, [768,768+dx) M-masked dX'.
+__global__ void k_bias_partial(const __nv_bfloat16 *dQ, const __nv_bfloat16 *dK, const __nv_bfloat16 *dV,
+                               const __nv_bfloat16 *dXo, const uint8_t *M, int rows, int dx, int seg_rows,
+                               float *out) {
+    const int col = blockIdx.x * blockDim.x + threadIdx.x;
+    const int ncol = 3 * HD + dx;
+    if (col >= ncol) return;
+    const int r0 = blockIdx.y * seg_rows, r1 = min(rows, r0 + seg_rows);
+    const __nv_bfloat16 *src;
+    int ld, c;
+    if (col < 3 * HD) {
+        src = col < HD ? dQ : col < 2 * HD ? dK : dV;
+        ld = HD;
+        c = col % HD;
+    } else {
+        src = dXo;
+        ld = dx;
+        c = col - 3 * HD;
+    }
+    float acc = 0.f;
+    const bool masked = col >= 3 * HD;
+    for (int r = r0; r < r1; ++r) {
+        const float v = __bfloat162float(src[(size_t)r * ld + c]);
+        acc += (!masked || M[r]) ? v : 0.f;
+    }
+    out[(size_t)blockIdx.y * ncol + col] = acc;
+}
+
+// Row-kernel partials: out[z][e] = sum over CTAs of segment z of rparts[cta][e], e < dWfe+dWe.
+__global__ void k_rparts_partial(const float *rparts, int ctas, int seg, float *out) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    constexpr int NE = DE * NF + NH * DE;
+    if (e >= NE) return;
+    const int c0 = blockIdx.y * seg, c1 = min(ctas, c0 + seg);
+    float acc = 0.f;
+    for (int c = c0; c < c1; ++c) acc += rparts[(size_t)c * RPART + e];
+    out[(size_t)blockIdx.y * NE + e] = acc;
+}
+
+struct DWPtrs {
+    float *p[12];
+};
+
+// Final sums: weight gradients of the four node projections (split-K
+// partials), bias gradients, dWfe / dWe, and the global FiLM term's dg_b,
+// dWfy, dbf, dy.
+__global__ void k_bwd_finish(const float *wparts, int wsplits, const float *bparts, int bsplits,
+                             const float *r2, int rsplits, const float *rparts, int ctas_per_graph, int B, int dx,
+                             int dy, const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy, DWPtrs dW,
+                             __nv_bfloat16 *dyo, float *dg) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int msz = dx * HD;
+    const int ncol = 3 * HD + dx;
+    constexpr int NE = DE * NF + NH * DE;
+    if (e < 4 * msz) {
+        const int q = e / msz, o = e % msz;
+        const float *src = wparts + (size_t)q * wsplits * msz + o;
+        float acc = 0.f;
+        for (int z = 0; z < wsplits; ++z) acc += src[(size_t)z * msz];
+        dW.p[q == 0 ? 0 : q == 1 ? 2 : q == 2 ? 4 : 10][o] = acc;
+        return;
+    }
+    int x = e - 4 * msz;
+    if (x < ncol) {
+        float acc = 0.f;
+        for (int z = 0; z < bsplits; ++z) acc += bparts[(size_t)z * ncol + x];
+        if (x < 3 * HD) dW.p[1 + 2 * (x / HD)][x % HD] = acc;
+        else dW.p[11][x - 3 * HD] = acc;
+        return;
+    }
+    x -= ncol;
+    if (x < NE) {
+        float acc = 0.f;
+        for (int z = 0; z < rsplits; ++z) acc += r2[(size_t)z * NE + x];
+        if (x < DE * NF) dW.p[6][x] = acc; else dW.p[9][x - DE * NF] = acc;
+        return;
+    }
+    x -= NE;
+    if (x < B * NF) {
+        const int b = x / NF, k = x % NF;
+        float acc = 0.f;
+        for (int c = 0; c < ctas_per_graph; ++c) acc += rparts[((size_t)b * ctas_per_graph + c) * RPART + NE + k];
+        dg[x] = acc;
+    }
+}
+
+// dbf, dWfy, dy from dg (after k_bwd_finish).
+__global__ void k_film_grads(const float *dg, int B, int dy, const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy,
+                             float *dbf, float *dWfy, __nv_bfloat16 *dyo) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e < NF) {
+        float acc = 0.f;
+        for (int b = 0; b < B; ++b) acc += dg[b * NF + e];
+        dbf[e] = acc;
+    } else if (e < NF + dy * NF) {
+        const int x = e - NF, c = x / NF, k = x % NF;
+        float acc = 0.f;
+        for (int b = 0; b < B; ++b) acc = fmaf(__bfloat162float(y[(size_t)b * dy + c]), dg[b * NF + k], acc);
+        dWfy[x] = acc;
+    } else if (e < NF + dy * NF + B * dy) {
+        const int x = e - NF - dy * NF, b = x / dy, c = x % dy;
+        float acc = 0.f;
+        for (int k = 0; k < NF; ++k) acc = fmaf(dg[b * NF + k], __bfloat162float(Wfy[c * NF + k]), acc);
+        dyo[x] = __float2bfloat16_rn(acc);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+template <int NR>
+static cudaError_t launch_bwd_nr(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
+                                 cudaStream_t st) {
+    constexpr int TCN = tile_cols(NR);
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e;
+        if ((e = cudaFuncSetAttribute(k_bwd_rows<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      RowSmem<NR>::BYTES)) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(k_bwd_rows<NR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+            cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(k_bwd_cols<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      ColSmem<NR>::BYTES)) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(k_bwd_cols<NR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+            cudaSuccess)
+            return e;
+        attr_done = true;
+    }
+    __nv_bfloat16 *dO = reinterpret_cast<__nv_bfloat16 *>(ws + W.dO);
+    __nv_bfloat16 *dQ = reinterpret_cast<__nv_bfloat16 *>(ws + W.dQ);
+    __nv_bfloat16 *dK = reinterpret_cast<__nv_bfloat16 *>(ws + W.dK);
+    __nv_bfloat16 *dV = reinterpret_cast<__nv_bfloat16 *>(ws + W.dV);
+    float *D = reinterpret_cast<float *>(ws + W.D);
+    const int nc = (d.n + TCN - 1) / TCN;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = nc;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(NTHR);
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    {
+        CUtensorMap mE, mDEp, mDE, mK, mV;
+        if (!encode_pair_map(&mE, a.E, d.B, d.n, false, TCN) ||
+            !encode_pair_map(&mDEp, a.dEout, d.B, d.n, false, TCN) ||
+            !encode_pair_map(&mDE, a.dE, d.B, d.n, false, TCN) || !encode_node_map(&mK, a.K, d.B, d.n, TCN) ||
+            !encode_node_map(&mV, a.V, d.B, d.n, TCN))
+            return cudaErrorInvalidValue;
+        BwdRowParams p;
+        p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
+        p.dO = dO;
+        p.LSE = a.LSE;
+        p.g = g;
+        p.img = reinterpret_cast<const uint8_t *>(ws + W.img);
+        p.M = a.M;
+        p.D = D;
+        p.dQ = dQ;
+        p.rparts = reinterpret_cast<float *>(ws + W.rparts);
+        p.status = a.status;
+        p.n = d.n;
+        cfg.gridDim = dim3(nc, (d.n + TB - 1) / TB, d.B);
+        cfg.dynamicSmemBytes = RowSmem<NR>::BYTES;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, k_bwd_rows<NR>, mE, mDEp, mDE, mK, mV, p);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        CUtensorMap mEt, mDEpt, mQ, mDO;
+        if (!encode_pair_map(&mEt, a.E, d.B, d.n, true, TCN) ||
+            !encode_pair_map(&mDEpt, a.dEout, d.B, d.n, true, TCN) || !encode_node_map(&mQ, a.Q, d.B, d.n, TCN) ||
+            !encode_node_map(&mDO, dO, d.B, d.n, TCN))
+            return cudaErrorInvalidValue;
+        BwdColParams p;
+        p.K = static_cast<const __nv_bfloat16 *>(a.K);
+        p.V = static_cast<const __nv_bfloat16 *>(a.V);
+        p.LSE = a.LSE;
+        p.D = D;
+        p.g = g;
+        p.img = reinterpret_cast<const uint8_t *>(ws + W.img);
+        p.M = a.M;
+        p.dK = dK;
+        p.dV = dV;
+        p.status = a.status;
+        p.n = d.n;
+        cfg.gridDim = dim3(nc, (d.n + TB - 1) / TB, d.B);
+        cfg.dynamicSmemBytes = ColSmem<NR>::BYTES;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, k_bwd_cols<NR>, mEt, mDEpt, mQ, mDO, p);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
+                             cudaStream_t st) {
+    return pick_nr(d.n) == 1 ? launch_bwd_nr<1>(d, a, W, ws, g, st) : launch_bwd_nr<2>(d, a, W, ws, g, st);
+}
+
+cudaError_t launch_bwd_finish(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
+                              cudaStream_t st) {
+    const __nv_bfloat16 *dQ = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dQ);
+    const __nv_bfloat16 *dK = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dK);
+    const __nv_bfloat16 *dV = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dV);
+    const int rows = d.B * d.n, ncol = 3 * HD + d.dx;
+    float *bparts = reinterpret_cast<float *>(ws + W.bparts);
+    const int seg_rows = (rows + W.bsplits - 1) / W.bsplits;
+    k_bias_partial<<<dim3((ncol + 255) / 256, W.bsplits), 256, 0, st>>>(
+        dQ, dK, dV, static_cast<const __nv_bfloat16 *>(a.dXout), a.M, rows, d.dx, seg_rows, bparts);
+    float *r2 = reinterpret_cast<float *>(ws + W.r2);
+    const int ctas = W.n_rparts, seg = (ctas + W.rsplits - 1) / W.rsplits;
+    constexpr int NE = DE * NF + NH * DE;
+    const float *rparts = reinterpret_cast<const float *>(ws + W.rparts);
+    k_rparts_partial<<<dim3((NE + 255) / 256, W.rsplits), 256, 0, st>>>(rparts, ctas, seg, r2);
+    DWPtrs dWdev;
+    for (int q = 0; q < 12; ++q) dWdev.p[q] = a.dW[q];
+    const int total = 4 * d.dx * HD + ncol + NE + d.B * NF;
+    const int cpg = (d.n + TB - 1) / TB;
+    k_bwd_finish<<<(total + 255) / 256, 256, 0, st>>>(reinterpret_cast<const float *>(ws + W.wparts), W.wsplits,
+                                                      bparts, W.bsplits, r2, W.rsplits, rparts, cpg, d.B, d.dx,
+                                                      d.dy, static_cast<const __nv_bfloat16 *>(a.y),
+                                                      static_cast<const __nv_bfloat16 *>(a.w[7]), dWdev,
+                                                      static_cast<__nv_bfloat16 *>(a.dy), dg);
+    const int tf = NF + d.dy * NF + d.B * d.dy;
+    k_film_grads<<<(tf + 255) / 256, 256, 0, st>>>(dg, d.B, d.dy, static_cast<const __nv_bfloat16 *>(a.y),
+                                                   static_cast<const __nv_bfloat16 *>(a.w[7]), a.dW[8], a.dW[7],
+                                                   static_cast<__nv_bfloat16 *>(a.dy));
+    return cudaGetLastError();
+}
+
+}  // namespace fast
+}  // namespace eaga

@@ -1,11 +1,14 @@
-// Node-side GEMMs of the layer on the tensor cores (bf16 in, fp32 accumulate):
-//   QKV:      [Q|K|V] = X [Wq|Wk|Wv] + b, rows of masked nodes written as zero
-//   out-proj: X' = X + M (O Wo + bo)
+// Node-side matrix products of the layer on the tensor cores (bf16 operands,
+// fp32 accumulation), one kernel template for all of them:
+//   QKV      [Q|K|V] = X [Wq|Wk|Wv] + b; rows of masked nodes written as zero
+//   out-proj X' = X + M (O Wo + bo)
+//   dO       dO = M (dX' Wo^T)
+//   dX       dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T
+//   dW       X^T dQ, X^T dK, X^T dV, O^T dX' as split-K fp32 partials
 // 64x64 output tile per CTA, 4 warps of 32x32, K in steps of 32 through a
 // two-stage cp.async pipeline, 16-byte swizzled shared-memory rows.
-#include "common.cuh"
 #include "fast.h"
-#include "sm100.cuh"
+#include "fast_common.cuh"
 
 namespace eaga {
 namespace fast {
@@ -13,16 +16,18 @@ namespace fast {
 using namespace sm100;
 
 constexpr int GBM = 64, GBN = 64, GBK = 32, GTHR = 128;
+enum GemmMode { GM_QKV = 0, GM_OUT = 1, GM_DO = 2, GM_DX = 3, GM_WGRAD = 4 };
 
 struct GemmParams {
-    const __nv_bfloat16 *A;          // [M, K]
-    const __nv_bfloat16 *B[3];       // [K, Nb] each; output column tile n0 uses B[n0 / Nb]
-    const __nv_bfloat16 *bias[3];    // [Nb]
-    __nv_bfloat16 *C[3];             // [M, Nb]
-    const __nv_bfloat16 *R;          // residual [M, Nb] (out-proj) or null
-    const uint8_t *mask;             // [M]
-    int M, K, Nb;
-    int mode;                        // 0: QKV, 1: out-proj with residual
+    const __nv_bfloat16 *A[3];       // per K-segment; [M,K] (or [K,M] when A is transposed)
+    const __nv_bfloat16 *B[3];       // per output matrix (QKV, wgrad) or per K-segment (dX)
+    const __nv_bfloat16 *bias[3];
+    __nv_bfloat16 *C[3];             // bf16 outputs [M, Nb]
+    float *P[3];                     // fp32 split-K partials [splits][M, Nb]
+    const __nv_bfloat16 *R;          // residual [M, Nb]
+    const uint8_t *mask;             // [M] (rows)
+    int M, K, Nb, lda, ldb, nseg, kchunk;
+    int mode;
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool pred) {
@@ -33,19 +38,22 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// A tile [64 rows][32 k] (64 B rows): chunk c of row r at r*64 + ((c ^ ((r>>1)&3)) << 4)
-__device__ __forceinline__ uint32_t a_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
-// B tile [32 k][64 n] (128 B rows): chunk c of row k at k*128 + ((c ^ (k&7)) << 4)
-__device__ __forceinline__ uint32_t b_off(int k, int c) { return k * 128 + ((c ^ (k & 7)) << 4); }
+// [rows][32] bf16 tile (64 B rows): chunk c of row r
+__device__ __forceinline__ uint32_t off64(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
+// [rows][64] bf16 tile (128 B rows): chunk c of row r
+__device__ __forceinline__ uint32_t off128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
+// AT: A is stored [K, M] (row stride lda) and read transposed.  BT: B is stored [N, K].
+template <bool AT, bool BT>
 __global__ void __launch_bounds__(GTHR) k_node_gemm(GemmParams p) {
     __shared__ __align__(128) uint8_t sA[2][GBM * GBK * 2];
     __shared__ __align__(128) uint8_t sB[2][GBK * GBN * 2];
     const int tid = threadIdx.x, w = tid >> 5, t = tid & 31;
     const int n0g = blockIdx.x * GBN, m0 = blockIdx.y * GBM;
     const int which = n0g / p.Nb, n0 = n0g % p.Nb;
-    const __nv_bfloat16 *Bm = p.B[which];
     const int wm = (w >> 1) * 32, wn = (w & 1) * 32;
+    const int kbeg = p.mode == GM_WGRAD ? blockIdx.z * p.kchunk : 0;
+    const int kend = p.mode == GM_WGRAD ? min(p.K, kbeg + p.kchunk) : p.K;
     float acc[2][4][4];
 #pragma unroll
     for (int a = 0; a < 2; ++a)
@@ -54,46 +62,75 @@ __global__ void __launch_bounds__(GTHR) k_node_gemm(GemmParams p) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.f;
 
-    auto load = [&](int stage, int k0) {
+    const int nseg = p.nseg;
+    const int nk_seg = (kend - kbeg + GBK - 1) / GBK;
+    const int nk = nk_seg * nseg;
+    auto load = [&](int stage, int it) {
+        const int seg = it / nk_seg, k0 = kbeg + (it % nk_seg) * GBK;
+        const __nv_bfloat16 *A = p.A[nseg > 1 ? seg : 0];
+        const __nv_bfloat16 *Bm = p.B[nseg > 1 ? seg : which];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            const int idx = tid + q * GTHR;      // 256 chunks of A: row idx/4, chunk idx%4
-            const int r = idx >> 2, c = idx & 3;
-            const int gm = m0 + r;
-            cp_async16(smem_u32(sA[stage]) + a_off(r, c), p.A + (size_t)min(gm, p.M - 1) * p.K + k0 + c * 8, gm < p.M);
-            const int kr = idx >> 3, cb = idx & 7;   // 256 chunks of B: row idx/8, chunk idx%8
-            cp_async16(smem_u32(sB[stage]) + b_off(kr, cb), Bm + (size_t)(k0 + kr) * p.Nb + n0 + cb * 8, true);
+            const int idx = tid + q * GTHR;
+            if (!AT) {   // [64 m][32 k]
+                const int r = idx >> 2, c = idx & 3, gm = m0 + r, gk = k0 + c * 8;
+                const bool ok = gm < p.M && gk < kend;
+                cp_async16(smem_u32(sA[stage]) + off64(r, c), A + (ok ? (size_t)gm * p.lda + gk : 0), ok);
+            } else {     // [32 k][64 m]
+                const int r = idx >> 3, c = idx & 7, gk = k0 + r, gm = m0 + c * 8;
+                const bool ok = gk < kend && gm < p.M;
+                cp_async16(smem_u32(sA[stage]) + off128(r, c), A + (ok ? (size_t)gk * p.lda + gm : 0), ok);
+            }
+            if (!BT) {   // [32 k][64 n]
+                const int r = idx >> 3, c = idx & 7, gk = k0 + r;
+                const bool ok = gk < kend;
+                cp_async16(smem_u32(sB[stage]) + off128(r, c), Bm + (ok ? (size_t)gk * p.ldb + n0 + c * 8 : 0), ok);
+            } else {     // [64 n][32 k]
+                const int r = idx >> 2, c = idx & 3, gk = k0 + c * 8;
+                const bool ok = gk < kend;
+                cp_async16(smem_u32(sB[stage]) + off64(r, c), Bm + (ok ? (size_t)(n0 + r) * p.ldb + gk : 0), ok);
+            }
         }
         cp_async_commit();
     };
 
-    const int nk = p.K / GBK;
-    load(0, 0);
-    for (int kt = 0; kt < nk; ++kt) {
-        if (kt + 1 < nk) {
-            load((kt + 1) & 1, (kt + 1) * GBK);
+    if (nk > 0) load(0, 0);
+    for (int it = 0; it < nk; ++it) {
+        if (it + 1 < nk) {
+            load((it + 1) & 1, it + 1);
             cp_async_wait1();
         } else {
             cp_async_wait0();
         }
         __syncthreads();
-        const uint32_t a_s = smem_u32(sA[kt & 1]), b_s = smem_u32(sB[kt & 1]);
+        const uint32_t a_s = smem_u32(sA[it & 1]), b_s = smem_u32(sB[it & 1]);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
             uint32_t af[2][4], bfr[2][4];
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
-                // matrices: (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
-                const int r = wm + mt * 16 + (t & 7) + ((t >> 3) & 1) * 8;
-                const int c = ks * 2 + (t >> 4);
-                ldsm_x4(a_s + a_off(r, c), af[mt]);
+                if (!AT) {
+                    // (m 0-7, k 0-7), (m 8-15, k 0-7), (m 0-7, k 8-15), (m 8-15, k 8-15)
+                    const int r = wm + mt * 16 + (t & 7) + ((t >> 3) & 1) * 8;
+                    ldsm_x4(a_s + off64(r, ks * 2 + (t >> 4)), af[mt]);
+                } else {
+                    // stored [k][m]: matrices as above via .trans of [k rows][m cols]
+                    const int kr = ks * 16 + (t & 7) + ((t >> 4) & 1) * 8;
+                    const int c = (wm + mt * 16) / 8 + ((t >> 3) & 1);
+                    ldsm_x4_t(a_s + off128(kr, c), af[mt]);
+                }
             }
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
-                // matrices: (k 0-7, n 0-7), (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15)
-                const int kr = ks * 16 + (t & 7) + ((t >> 3) & 1) * 8;
-                const int c = (wn + np * 16) / 8 + (t >> 4);
-                ldsm_x4_t(b_s + b_off(kr, c), bfr[np]);
+                if (!BT) {
+                    // (k 0-7, n 0-7), (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15)
+                    const int kr = ks * 16 + (t & 7) + ((t >> 3) & 1) * 8;
+                    ldsm_x4_t(b_s + off128(kr, (wn + np * 16) / 8 + (t >> 4)), bfr[np]);
+                } else {
+                    // stored [n][k]: non-trans rows n
+                    const int r = wn + np * 16 + (t & 7) + ((t >> 4) & 1) * 8;
+                    ldsm_x4(b_s + off64(r, ks * 2 + ((t >> 3) & 1)), bfr[np]);
+                }
             }
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
@@ -104,8 +141,6 @@ __global__ void __launch_bounds__(GTHR) k_node_gemm(GemmParams p) {
         __syncthreads();
     }
     // epilogue
-    const __nv_bfloat16 *bias = p.bias[which];
-    __nv_bfloat16 *C = p.C[which];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -115,60 +150,112 @@ __global__ void __launch_bounds__(GTHR) k_node_gemm(GemmParams p) {
                 const int row = m0 + wm + mt * 16 + (t >> 2) + hh * 8;
                 const int col = n0 + wn + nt * 8 + (t & 3) * 2;
                 if (row >= p.M) continue;
-                const float2 bb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(bias + col));
-                const bool mk = p.mask[row] != 0;
-                float v0 = acc[mt][nt][hh * 2] + bb.x, v1 = acc[mt][nt][hh * 2 + 1] + bb.y;
-                __nv_bfloat162 out;
-                if (p.mode == 0) {
-                    out = mk ? __floats2bfloat162_rn(v0, v1) : __floats2bfloat162_rn(0.f, 0.f);
-                } else {
-                    const __nv_bfloat162 rr = *reinterpret_cast<const __nv_bfloat162 *>(p.R + (size_t)row * p.Nb + col);
-                    if (mk) {
-                        const float2 x = __bfloat1622float2(rr);
-                        out = __floats2bfloat162_rn(x.x + v0, x.y + v1);
-                    } else {
-                        out = rr;
-                    }
+                float v0 = acc[mt][nt][hh * 2], v1 = acc[mt][nt][hh * 2 + 1];
+                const size_t o = (size_t)row * p.Nb + col;
+                if (p.mode == GM_WGRAD) {
+                    float *P = p.P[which] + (size_t)blockIdx.z * p.M * p.Nb;
+                    *reinterpret_cast<float2 *>(P + o) = make_float2(v0, v1);
+                    continue;
                 }
-                *reinterpret_cast<__nv_bfloat162 *>(C + (size_t)row * p.Nb + col) = out;
+                const bool mk = p.mask[row] != 0;
+                __nv_bfloat162 out;
+                if (p.mode == GM_QKV || p.mode == GM_OUT) {
+                    const float2 bb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p.bias[which] + col));
+                    v0 += bb.x;
+                    v1 += bb.y;
+                }
+                if (p.mode == GM_QKV || p.mode == GM_DO) {
+                    out = mk ? __floats2bfloat162_rn(v0, v1) : __floats2bfloat162_rn(0.f, 0.f);
+                } else if (p.mode == GM_OUT) {
+                    const __nv_bfloat162 rr = *reinterpret_cast<const __nv_bfloat162 *>(p.R + o);
+                    const float2 x = __bfloat1622float2(rr);
+                    out = mk ? __floats2bfloat162_rn(x.x + v0, x.y + v1) : rr;
+                } else {   // GM_DX
+                    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p.R + o));
+                    out = __floats2bfloat162_rn(x.x + v0, x.y + v1);
+                }
+                *reinterpret_cast<__nv_bfloat162 *>(p.C[which] + o) = out;
             }
 }
 
+static inline const __nv_bfloat16 *bf(const void *p) { return static_cast<const __nv_bfloat16 *>(p); }
+
 cudaError_t launch_qkv(const eaga_dims &d, const FwdArgs &a, cudaStream_t st) {
-    GemmParams p;
-    p.A = static_cast<const __nv_bfloat16 *>(a.X);
+    GemmParams p = {};
+    p.A[0] = bf(a.X);
     for (int q = 0; q < 3; ++q) {
-        p.B[q] = static_cast<const __nv_bfloat16 *>(a.w[2 * q]);
-        p.bias[q] = static_cast<const __nv_bfloat16 *>(a.w[2 * q + 1]);
+        p.B[q] = bf(a.w[2 * q]);
+        p.bias[q] = bf(a.w[2 * q + 1]);
     }
     p.C[0] = static_cast<__nv_bfloat16 *>(a.Q);
     p.C[1] = static_cast<__nv_bfloat16 *>(a.K);
     p.C[2] = static_cast<__nv_bfloat16 *>(a.V);
-    p.R = nullptr;
     p.mask = a.M;
-    p.M = d.B * d.n;
-    p.K = d.dx;
-    p.Nb = d.H * d.dh;
-    p.mode = 0;
-    dim3 grid(3 * p.Nb / GBN, (p.M + GBM - 1) / GBM);
-    k_node_gemm<<<grid, GTHR, 0, st>>>(p);
+    p.M = d.B * d.n; p.K = d.dx; p.Nb = HD; p.lda = d.dx; p.ldb = HD; p.nseg = 1; p.mode = GM_QKV;
+    k_node_gemm<false, false><<<dim3(3 * HD / GBN, (p.M + GBM - 1) / GBM), GTHR, 0, st>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_out_proj(const eaga_dims &d, const FwdArgs &a, cudaStream_t st) {
-    GemmParams p;
-    p.A = static_cast<const __nv_bfloat16 *>(a.O);
-    p.B[0] = p.B[1] = p.B[2] = static_cast<const __nv_bfloat16 *>(a.w[10]);
-    p.bias[0] = p.bias[1] = p.bias[2] = static_cast<const __nv_bfloat16 *>(a.w[11]);
-    p.C[0] = p.C[1] = p.C[2] = static_cast<__nv_bfloat16 *>(a.Xout);
-    p.R = static_cast<const __nv_bfloat16 *>(a.X);
+    GemmParams p = {};
+    p.A[0] = bf(a.O);
+    p.B[0] = bf(a.w[10]);
+    p.bias[0] = bf(a.w[11]);
+    p.C[0] = static_cast<__nv_bfloat16 *>(a.Xout);
+    p.R = bf(a.X);
     p.mask = a.M;
-    p.M = d.B * d.n;
-    p.K = d.H * d.dh;
-    p.Nb = d.dx;
-    p.mode = 1;
-    dim3 grid(p.Nb / GBN, (p.M + GBM - 1) / GBM);
-    k_node_gemm<<<grid, GTHR, 0, st>>>(p);
+    p.M = d.B * d.n; p.K = HD; p.Nb = d.dx; p.lda = HD; p.ldb = d.dx; p.nseg = 1; p.mode = GM_OUT;
+    k_node_gemm<false, false><<<dim3(d.dx / GBN, (p.M + GBM - 1) / GBM), GTHR, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+// dO = M (dX' Wo^T): A = dX' [rows, dx], B = Wo stored [N=256, K=dx].
+cudaError_t launch_dO(const eaga_dims &d, const BwdArgs &a, __nv_bfloat16 *dO, cudaStream_t st) {
+    GemmParams p = {};
+    p.A[0] = bf(a.dXout);
+    p.B[0] = bf(a.w[10]);
+    p.C[0] = dO;
+    p.mask = a.M;
+    p.M = d.B * d.n; p.K = d.dx; p.Nb = HD; p.lda = d.dx; p.ldb = d.dx; p.nseg = 1; p.mode = GM_DO;
+    k_node_gemm<false, true><<<dim3(HD / GBN, (p.M + GBM - 1) / GBM), GTHR, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+// dX = dX' + sum_q dN_q Wq^T over the three projections: B_q stored [N=dx, K=256].
+cudaError_t launch_dX(const eaga_dims &d, const BwdArgs &a, const __nv_bfloat16 *dN[3], cudaStream_t st) {
+    GemmParams p = {};
+    for (int q = 0; q < 3; ++q) {
+        p.A[q] = dN[q];
+        p.B[q] = bf(a.w[2 * q]);
+    }
+    p.C[0] = static_cast<__nv_bfloat16 *>(a.dX);
+    p.R = bf(a.dXout);
+    p.mask = a.M;
+    p.M = d.B * d.n; p.K = HD; p.Nb = d.dx; p.lda = HD; p.ldb = HD; p.nseg = 3; p.mode = GM_DX;
+    k_node_gemm<false, true><<<dim3(d.dx / GBN, (p.M + GBM - 1) / GBM), GTHR, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+// Split-K weight-gradient partials: P_q[z] = (rows of chunk z of A)^T B_q.
+//   X^T [dQ|dK|dV] -> 3 matrices [dx, 256];  O^T dX' -> [256, dx]
+cudaError_t launch_wgrad(const eaga_dims &d, const BwdArgs &a, const __nv_bfloat16 *dN[3], float *parts,
+                         int splits, cudaStream_t st) {
+    const int rows = d.B * d.n, kchunk = ((rows + splits - 1) / splits + GBK - 1) / GBK * GBK;
+    const size_t msz = (size_t)splits * d.dx * HD;
+    GemmParams p = {};
+    p.A[0] = bf(a.X);
+    for (int q = 0; q < 3; ++q) {
+        p.B[q] = dN[q];
+        p.P[q] = parts + q * msz;
+    }
+    p.M = d.dx; p.K = rows; p.Nb = HD; p.lda = d.dx; p.ldb = HD; p.nseg = 1; p.kchunk = kchunk; p.mode = GM_WGRAD;
+    k_node_gemm<true, false><<<dim3(3 * HD / GBN, (d.dx + GBM - 1) / GBM, splits), GTHR, 0, st>>>(p);
+    GemmParams o = {};
+    o.A[0] = bf(a.O);
+    o.B[0] = bf(a.dXout);
+    o.P[0] = parts + 3 * msz;
+    o.M = HD; o.K = rows; o.Nb = d.dx; o.lda = HD; o.ldb = d.dx; o.nseg = 1; o.kchunk = kchunk; o.mode = GM_WGRAD;
+    k_node_gemm<true, false><<<dim3(d.dx / GBN, HD / GBM, splits), GTHR, 0, st>>>(o);
     return cudaGetLastError();
 }
 

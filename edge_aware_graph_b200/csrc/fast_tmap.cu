@@ -1,0 +1,116 @@
+// TMA tensor maps of the specialised path and the per-call prologue kernel
+// (global FiLM term g_b and the tensor-core operand images of the small weights).
+#include "fast.h"
+#include "fast_common.cuh"
+
+namespace eaga {
+namespace fast {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// A [B, n, n, 64] bf16 pair tensor viewed as 5-D with a box of 8 x box_rows pairs.
+// Row tile (transposed = false): dims (c, ic, j, s, b) with i = 2ic + s, so the
+// box lands in shared memory as [s][j box_rows][ic 4][c 64].  Column tile
+// (transposed = true): dims (c, jc, i, s, b) with j = 2jc + s, landing as
+// [s][i box_rows][jc 4][c 64].  Requires n even (i = 2ic + s stays inside the graph).
+bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transposed, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t rowb = DE * 2;                       // one pair: 128 bytes
+    const cuuint64_t dims[5] = {DE, (cuuint64_t)(n / 2), (cuuint64_t)n, 2, (cuuint64_t)B};
+    cuuint64_t strides[4];
+    if (!transposed) {
+        strides[0] = 2 * (cuuint64_t)n * rowb;             // ic -> two rows i
+        strides[1] = rowb;                                  // j
+        strides[2] = (cuuint64_t)n * rowb;                  // s -> one row i
+    } else {
+        strides[0] = 2 * rowb;                              // jc -> two columns j
+        strides[1] = (cuuint64_t)n * rowb;                  // i
+        strides[2] = rowb;                                  // s -> one column j
+    }
+    strides[3] = (cuuint64_t)n * n * rowb;                  // b
+    const cuuint32_t box[5] = {64, 4, (cuuint32_t)box_rows, 2, 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A [B, n, 256] bf16 node tensor; box of 64 features x box_rows nodes, 128B-swizzled.
+bool encode_node_map(CUtensorMap *m, const void *base, int B, int n, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {HD, (cuuint64_t)n, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {HD * 2, (cuuint64_t)n * HD * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// g_b = y_b Wfy + bf (fp32) for every graph, and (block 0) the four operand images.
+__global__ void k_prologue(const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy, const __nv_bfloat16 *bf,
+                           const __nv_bfloat16 *Wfe, const __nv_bfloat16 *We, float *g, uint8_t *img, int B,
+                           int dy) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t < B * NF) {
+        const int b = t / NF, k = t % NF;
+        float acc = __bfloat162float(bf[k]);
+        for (int c = 0; c < dy; ++c)
+            acc = fmaf(__bfloat162float(y[(size_t)b * dy + c]), __bfloat162float(Wfy[c * NF + k]), acc);
+        g[t] = acc;
+    }
+    if (blockIdx.x != 0) return;
+    const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+    for (int e = threadIdx.x; e < NF * DE; e += blockDim.x) {
+        // IMG_WFE_T_SW: row k (16), element c (64)
+        {
+            const int k = e / DE, c = e % DE;
+            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WFE_T_SW + sw128(k, c >> 3) + (c & 7) * 2) = Wfe[c * NF + k];
+        }
+        // IMG_WE_SW: row h (16, zero for h >= 8), element c
+        {
+            const int h = e / DE, c = e % DE;
+            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WE_SW + sw128(h, c >> 3) + (c & 7) * 2) =
+                h < NH ? We[h * DE + c] : zero;
+        }
+        // IMG_WE_T_NS: row c (64), element h (16, zero for h >= 8)
+        {
+            const int c = e / NF, h = e % NF;
+            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WE_T_NS + ns16(c, h)) = h < NH ? We[h * DE + c] : zero;
+        }
+        // IMG_WFE_NS: row c (64), element k (16)
+        {
+            const int c = e / NF, k = e % NF;
+            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WFE_NS + ns16(c, k)) = Wfe[c * NF + k];
+        }
+    }
+}
+
+cudaError_t launch_prologue(const eaga_dims &d, const void *const w[12], const void *y, float *g, uint8_t *img,
+                            cudaStream_t st) {
+    const int threads = 256, blocks = (d.B * NF + threads - 1) / threads;
+    k_prologue<<<blocks, threads, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(y), static_cast<const __nv_bfloat16 *>(w[7]),
+        static_cast<const __nv_bfloat16 *>(w[8]), static_cast<const __nv_bfloat16 *>(w[6]),
+        static_cast<const __nv_bfloat16 *>(w[9]), g, img, d.B, d.dy);
+    return cudaGetLastError();
+}
+
+}  // namespace fast
+}  // namespace eaga

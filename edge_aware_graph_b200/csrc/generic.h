@@ -3,7 +3,7 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
-#include "../../include/eaga.h"
+#include "eaga.h"
 
 namespace eaga {
 

@@ -147,6 +147,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
     for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
 }
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, float &v0, float &v1) {
+    uint32_t r0, r1;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(taddr));
+    v0 = __uint_as_float(r0);
+    v1 = __uint_as_float(r1);
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ cluster
@@ -159,6 +165,25 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Asynchronous store into a (possibly remote) CTA's shared memory; the bytes
+// are counted on that CTA's mbarrier `cbar` (both shared::cluster addresses).
+__device__ __forceinline__ void st_async_v2(uint32_t caddr, float a, float b, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(caddr),
+                 "f"(a), "f"(b), "r"(cbar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_v4(uint32_t caddr, float4 v, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     caddr),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cbar)
+                 : "memory");
+}
+// Split cluster barrier: arrive now (after the last read of a peer's shared
+// memory), wait later (before this CTA's shared memory may disappear).
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 __device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
