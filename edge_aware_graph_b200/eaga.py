@@ -21,7 +21,7 @@ STATUS = {0: "EAGA_OK", 1: "EAGA_ERR_INVALID_ARG", 2: "EAGA_ERR_UNSUPPORTED", 3:
           4: "EAGA_ERR_WORKSPACE", 5: "EAGA_ERR_CUDA", 6: "EAGA_ERR_TIMEOUT"}
 EXPORTED = ("eaga_workspace_size", "eaga_saved_size", "eaga_forward", "eaga_backward",
             "eaga_debug_attention_map", "eaga_get_device_status", "eaga_strerror",
-            "eaga_set_profile_events", "eaga_kernel_launches")
+            "eaga_set_profile_events", "eaga_kernel_launches", "eaga_forward_noalloc")
 
 
 class Dims(ctypes.Structure):
@@ -59,6 +59,9 @@ def lib():
         L.eaga_backward.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.POINTER(Weights), vp,
                                     vp, vp, vp, vp, vp, ctypes.POINTER(Weights), vp, sz, vp]
         L.eaga_backward.restype = i32
+        L.eaga_forward_noalloc.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.POINTER(Weights),
+                                           vp, vp, vp, vp]
+        L.eaga_forward_noalloc.restype = i32
         L.eaga_debug_attention_map.argtypes = [ctypes.POINTER(Dims), vp, vp, ctypes.POINTER(Weights), vp, vp,
                                                vp, vp]
         L.eaga_debug_attention_map.restype = i32
@@ -113,6 +116,13 @@ def forward(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, workspace, stream=N
                             _p(Xout), _p(Eout), _p(saved), _p(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream))
     _check(rc, "eaga_forward")
+
+
+def forward_noalloc(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, stream=None):
+    """eaga_forward without a workspace argument (the library's own fixed scratch is used)."""
+    rc = lib().eaga_forward_noalloc(ctypes.byref(d), _p(X), _p(E), _p(y), _p(M), ctypes.byref(_weights(W)),
+                                    _p(Xout), _p(Eout), _p(saved), _stream(stream))
+    _check(rc, "eaga_forward_noalloc")
 
 
 def backward(d: Dims, X, E, y, M, W: dict, saved, dXout, dEout, dX, dE, dy, dW: dict, workspace, stream=None):

@@ -119,6 +119,33 @@ EAGA_API eaga_status eaga_backward(const eaga_dims *dims,
                           void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
                           void *workspace, size_t ws_bytes, void *stream);
 
+/* Forward without a caller-provided workspace.  The paper has no counterpart
+ * of this call; it exists for callers that cannot allocate device memory
+ * for scratch: plain C clients that link this library but no device
+ * allocator, or code under a framework whose memory pool only hands out the
+ * tensors it owns.  It computes exactly what eaga_forward computes, with the
+ * same arguments minus the workspace; `saved` is required (it is an output
+ * as large as the node tensors).
+ *
+ * The forward's small scratch (status word, global FiLM term g [B,2H] fp32,
+ * the tensor-core images of Wfe and We) lives in a 64 KiB array in the
+ * library's device memory, held by every GPU that loads the library until
+ * the process exits.  Limit: 256 + roundup256(8*H*B) + 8192 bytes must fit
+ * in 64 KiB (B <= 892 graphs at H = 8); larger B returns
+ * EAGA_ERR_UNSUPPORTED without launching.  No device memory is allocated or
+ * freed by this call.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call on a device shares the array and leaves its contents
+ * behind: calls that overlap on the GPU (other streams, other host threads)
+ * race on it and must be serialised by the caller.  The status word is
+ * cleared at the start of each call. */
+EAGA_API eaga_status eaga_forward_noalloc(const eaga_dims *dims,
+                                          const void *X, const void *E, const void *y, const uint8_t *M,
+                                          const eaga_weights *w, void *Xout, void *Eout, void *saved,
+                                          void *stream);
+
 /* Test aid: writes the normalised coefficients A [B,H,n,n] (fp32) that the
  * forward used, recomputed from E, y and the forward's `saved` state.  `A`
  * must hold B*H*n*n + 2*B*H floats (the tail is scratch).  Writes O(B*H*n*n)
