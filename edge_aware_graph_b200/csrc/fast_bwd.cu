@@ -61,11 +61,14 @@ struct RowSmem {
     static constexpr uint32_t G = WDG + 256;
     static constexpr uint32_t LSE = G + 64;                        // [8 i][8 h]
     static constexpr uint32_t MI = LSE + 256, MJ = MI + 16;
-    static constexpr uint32_t BAR = MJ + 64;                       // 6 mbarriers
-    static constexpr uint32_t TM = BAR + 48;
-    static constexpr uint32_t WP = TM + 16;                        // CTA weight-grad partial (read by peers)
-    static constexpr uint32_t BYTES = WP + RPART * 4 + 1024;
-    static constexpr uint32_t QPART = K;                           // 32 KB dq quadrant partials (K, V dead)
+    static constexpr uint32_t BAR = MJ + 64;                       // 9 mbarriers
+    static constexpr uint32_t TM = BAR + 72;
+    static constexpr uint32_t RD = TM + 24;                        // received D partials [16][64] f32
+    static constexpr uint32_t BYTES = RD + 4096 + 1024;
+    // in the E tile once it is dead: the CTA weight-grad partial, the pushed
+    // weight-grad slices and the pushed dq slices of the cluster
+    static constexpr uint32_t WP = E, RWP = E + 6400, RQ = E + 13056;
+    static constexpr uint32_t QPART = K;                           // 16 KB two-slot dq sums (K, V dead)
 };
 
 template <int NR>
@@ -83,7 +86,8 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
     const int n = p.n;
     const int j0 = blockIdx.x * TCN, i0 = blockIdx.y * TB, b = blockIdx.z;
     const uint32_t bar_e = sbase + S::BAR, bar_dep = bar_e + 8, bar_kv = bar_e + 16, bar_film = bar_e + 24,
-                   bar_u = bar_e + 32, bar_de = bar_e + 40;
+                   bar_u = bar_e + 32, bar_de = bar_e + 40, bar_d = bar_e + 48, bar_wp = bar_e + 56,
+                   bar_q = bar_e + 64;
     float *g = reinterpret_cast<float *>(sp + S::G);
     float *lse = reinterpret_cast<float *>(sp + S::LSE);
     uint8_t *mi = sp + S::MI, *mj = sp + S::MJ;
@@ -92,7 +96,11 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
     if (tid == 0) {
         mbar_init(bar_e, 1); mbar_init(bar_dep, 1); mbar_init(bar_kv, 1);
         mbar_init(bar_film, 1); mbar_init(bar_u, 1); mbar_init(bar_de, 1);
+        mbar_init(bar_d, 1); mbar_init(bar_wp, 1); mbar_init(bar_q, 1);
         fence_mbar_init();
+        mbar_expect_tx(bar_d, nclu * 64 * 4);
+        mbar_expect_tx(bar_wp, nclu * flat_slice(RPART, nclu, rank) * 16);
+        mbar_expect_tx(bar_q, nclu * rows_slice(1, nclu, rank) * 16);
         mbar_expect_tx(bar_e, NR * 32768);
         tma_load_5d(sbase + S::E, &tmE, bar_e, 0, i0 / 2, j0, 0, b);
         mbar_expect_tx(bar_dep, NR * 32768);
@@ -129,6 +137,7 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
     const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+    cluster_arrive();   // receive barriers of this CTA are armed
 
     if (tid == 0) {
         if (!mbar_wait(bar_e, 0)) flag_timeout(p.status);
@@ -189,8 +198,11 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
         }
     __syncthreads();
     if (tid < 64) cd[tid] = wd[tid] + wd[64 + tid] + wd[128 + tid] + wd[192 + tid];
-    cluster_sync();
-    cluster_combine64<1>(sp, sbase, S::CD, S::FD, tid, nclu);
+    __syncthreads();
+    cluster_wait();     // every peer's receive barriers are armed
+    push_rowvals_f32(sp, sbase, S::CD, S::RD, bar_d, tid, rank, nclu);
+    if (!mbar_wait(bar_d, 0)) flag_timeout(p.status);
+    combine_rowvals_f32(sp, S::RD, S::FD, tid, nclu);
     __syncthreads();
     if (tid < 64) {
         const int il = tid >> 3, h = tid & 7;
@@ -271,6 +283,8 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
             mma16816(wf[1], aE, bF[2], bF[3]);
             mma16816(we4, aD, bA0, bA1);
         }
+        __syncthreads();   // the E tile is dead from here on
+        cluster_arrive();  // peers may now push into this CTA's E tile space
         float *rp = reinterpret_cast<float *>(sp + S::WP);
         for (int phase = 0; phase < 4; ++phase) {
             if (kr == phase) {
@@ -299,22 +313,9 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
         }
     }
     // sum the CTA partials over the cluster: one partial per (graph, row block)
-    cluster_sync();
-    {
-        float *rp = p.rparts + (size_t)(blockIdx.z * gridDim.y + blockIdx.y) * RPART;
-        const int per = (RPART + nclu - 1) / nclu;
-        for (int x = rank * per + tid; x < min((int)(rank + 1) * per, RPART); x += NTHR) {
-            float acc = 0.f;
-            for (uint32_t k0 = 0; k0 < nclu; k0 += 4) {
-                float v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) v[u] = (k0 + u < nclu) ? ld_peer_f32(map_peer(sbase + S::WP + x * 4, k0 + u)) : 0.f;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) acc += v[u];
-            }
-            rp[x] = acc;
-        }
-    }
+    __syncthreads();
+    cluster_wait();
+    push_flat(sp, sbase, S::WP, RPART, S::RWP, bar_wp, tid, rank, nclu);
 
     // dE = dE' + df Wfe^T, written in place over the dE' tile, NR rounds of two MMAs
     for (int round = 0; round < NR; ++round) {
@@ -350,17 +351,34 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
         tma_store_5d(&tmDE, sbase + S::DEP, 0, i0 / 2, j0, 0, b);
         tma_store_commit();
     }
+    // weight-grad partial of the cluster: this CTA's slice of the sum over peers
+    if (!mbar_wait(bar_wp, 0)) flag_timeout(p.status);
+    {
+        float *rp = p.rparts + (size_t)(blockIdx.z * gridDim.y + blockIdx.y) * RPART;
+        const uint32_t per4 = (RPART / 4 + nclu - 1) / nclu, slice = flat_slice(RPART, nclu, rank);
+        const float4 *rv = reinterpret_cast<const float4 *>(sp + S::RWP);
+        for (uint32_t k0 = tid; k0 < slice; k0 += NTHR) {
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (uint32_t pp = 0; pp < nclu; ++pp) {
+                const float4 v = rv[pp * per4 + k0];
+                a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+            }
+            reinterpret_cast<float4 *>(rp)[rank * per4 + k0] = a;
+        }
+    }
     // dq: reduce over the quadrant warps and the cluster
-    store_quadrant_part(sp, S::QPART, qacc, q, hq, t);
+    store_quadrant_part_2ph(sp, S::QPART, qacc, q, hq, t);
     {
         const uint32_t parts[1] = {S::QPART};
+        push_rows_partials<1, 2>(sp, sbase, parts, S::RQ, bar_q, tid, rank, nclu);
+        if (!mbar_wait(bar_q, 0)) flag_timeout(p.status);
         __nv_bfloat16 *const outs[1] = {p.dQ};
         const float sc[1] = {rs};
-        cluster_reduce_rows<1>(sbase, parts, tid, rank, nclu, outs, b, n, i0, sc);
+        finish_rows_partials<1>(sp, S::RQ, tid, rank, nclu, outs, b, n, i0, sc);
     }
     if (tid == 0) tma_store_wait_read0();
     tc_fence_before();
-    cluster_wait();
+    __syncthreads();
     if (W == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
@@ -372,10 +390,12 @@ struct ColSmem {
     static constexpr uint32_t IMG = DO + NR * 16384;               // Wfe^T sw, We sw
     static constexpr uint32_t G = IMG + 4096;
     static constexpr uint32_t MI = G + 64, MJ = MI + 64;
-    static constexpr uint32_t BAR = MJ + 16;                       // 5 mbarriers
-    static constexpr uint32_t TM = BAR + 40;
-    static constexpr uint32_t BYTES = TM + 24 + 1024;
-    static constexpr uint32_t KPART = E, VPART = DEP;              // 32 KB quadrant partials each (tiles dead)
+    static constexpr uint32_t BAR = MJ + 16;                       // 6 mbarriers
+    static constexpr uint32_t TM = BAR + 48;
+    static constexpr uint32_t BYTES = TM + 16 + 1024;
+    // after the tiles are dead: two-slot quadrant sums of dk, dv in the E
+    // tile, the pushed cluster partials received in the dE' tile
+    static constexpr uint32_t KPART = E, VPART = E + 16384, RECV = DEP;
 };
 
 template <int NR>
@@ -392,15 +412,16 @@ k_bwd_cols(const __grid_constant__ CUtensorMap tmEt, const __grid_constant__ CUt
     const int n = p.n;
     const int i0 = blockIdx.x * TCN, j0 = blockIdx.y * TB, b = blockIdx.z;   // 32NR rows i, 8 columns j
     const uint32_t bar_e = sbase + S::BAR, bar_dep = bar_e + 8, bar_q = bar_e + 16, bar_film = bar_e + 24,
-                   bar_u = bar_e + 32;
+                   bar_u = bar_e + 32, bar_r = bar_e + 40;
     float *g = reinterpret_cast<float *>(sp + S::G);
     uint8_t *mi = sp + S::MI, *mj = sp + S::MJ;
     constexpr uint32_t TM_FILM = 0, TM_U = 64, TM_COLS = 128;
 
     if (tid == 0) {
         mbar_init(bar_e, 1); mbar_init(bar_dep, 1); mbar_init(bar_q, 1);
-        mbar_init(bar_film, 1); mbar_init(bar_u, 1);
+        mbar_init(bar_film, 1); mbar_init(bar_u, 1); mbar_init(bar_r, 1);
         fence_mbar_init();
+        mbar_expect_tx(bar_r, nclu * rows_slice(2, nclu, rank) * 16);
         mbar_expect_tx(bar_e, NR * 32768);
         tma_load_5d(sbase + S::E, &tmEt, bar_e, 0, j0 / 2, i0, 0, b);
         mbar_expect_tx(bar_dep, NR * 32768);
@@ -495,19 +516,23 @@ k_bwd_cols(const __grid_constant__ CUtensorMap tmEt, const __grid_constant__ CUt
     }
     tc_fence_before();
     __syncthreads();   // tiles are dead: their space holds the partials below
+    cluster_arrive();  // peers may now push into this CTA's dE' tile space
     float kacc[2][2][4], vacc[2][2][4];
     warp_contract2<NR>(sbase + S::Q, q, t, hq, da, kacc);    // dk^T = Q^T ds
     warp_contract2<NR>(sbase + S::DO, q, t, hq, sv, vacc);   // dv^T = dO^T a
-    store_quadrant_part(sp, S::KPART, kacc, q, hq, t);
-    store_quadrant_part(sp, S::VPART, vacc, q, hq, t);
+    store_quadrant_part_2ph(sp, S::KPART, kacc, q, hq, t);
+    store_quadrant_part_2ph(sp, S::VPART, vacc, q, hq, t);
+    cluster_wait();
     {
         const uint32_t parts[2] = {S::KPART, S::VPART};
+        push_rows_partials<2, 2>(sp, sbase, parts, S::RECV, bar_r, tid, rank, nclu);
+        if (!mbar_wait(bar_r, 0)) flag_timeout(p.status);
         __nv_bfloat16 *const outs[2] = {p.dK, p.dV};
         const float sc[2] = {rs, 1.f};
-        cluster_reduce_rows<2>(sbase, parts, tid, rank, nclu, outs, b, n, j0, sc);
+        finish_rows_partials<2>(sp, S::RECV, tid, rank, nclu, outs, b, n, j0, sc);
     }
     tc_fence_before();
-    cluster_wait();
+    __syncthreads();
     if (W == 0) tmem_dealloc(tmem, TM_COLS);
 }
 

@@ -14,6 +14,18 @@ constexpr int TB = 8;            // pair tile: 8 "own" rows x 32*NR "cluster" ro
 // NR = 2: 64 cluster rows per CTA (n <= 1024).
 __host__ __device__ constexpr int tile_cols(int NR) { return 32 * NR; }
 inline int pick_nr(int n) { return n <= 512 ? 1 : 2; }
+// Streaming multiprocessors of the current device (cached per process).
+inline int sm_count() {
+    static int cached = 0;
+    if (!cached) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+            cached = v;
+        else
+            cached = 148;
+    }
+    return cached;
+}
 
 // Operand images prepared once per call by the prologue kernel (bf16, in the
 // exact shared-memory layout the tensor-core descriptors expect).
@@ -351,10 +363,10 @@ __device__ __forceinline__ void combine_rowvals(uint8_t *sp, uint32_t s_recv, ui
     }
 }
 
-// Sum the 4 quadrant partials of NB [4][8][256] buffers and push float4
-// group gg (over the NB buffers) to its owner rank gg / per, slot
+// Sum the NSLOT slot partials of NB [NSLOT][8][256] fp32 buffers and push
+// float4 group gg (over the NB buffers) to its owner rank gg / per, slot
 // rank * per + (gg - owner * per) of the owner's receive buffer.
-template <int NB>
+template <int NB, int NSLOT = 4>
 __device__ __forceinline__ void push_rows_partials(uint8_t *sp, uint32_t sbase, const uint32_t (&s_part)[NB],
                                                    uint32_t s_recv, uint32_t bar, int tid, uint32_t rank,
                                                    uint32_t nclu) {
@@ -365,13 +377,79 @@ __device__ __forceinline__ void push_rows_partials(uint8_t *sp, uint32_t sbase, 
         const float4 *pt = reinterpret_cast<const float4 *>(sp + s_part[k]);
         float4 v = pt[g];
 #pragma unroll
-        for (int qq = 1; qq < 4; ++qq) {
+        for (int qq = 1; qq < NSLOT; ++qq) {
             const float4 w = pt[qq * G + g];
             v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
         }
         const uint32_t owner = gg / per, slot = rank * per + (gg - owner * per);
         st_async_v4(map_peer(sbase + s_recv + slot * 16, owner), v, map_peer(bar, owner));
     }
+}
+
+// The warps' [8 i][256 d] contributions summed over the 4 quadrants in two
+// fixed-order phases into a [2][8][256] fp32 buffer (16 KB): quadrants 0,1
+// write slots 0,1, then quadrants 2,3 add into them.  All threads call it.
+__device__ __forceinline__ void store_quadrant_part_2ph(uint8_t *sp, uint32_t s_part, const float (&acc)[2][2][4],
+                                                        int q, int hq, int t) {
+    const int c4 = t & 3, g8 = t >> 2;
+    float *dst = reinterpret_cast<float *>(sp + s_part) + (q & 1) * TB * HD;
+    for (int phase = 0; phase < 2; ++phase) {
+        if ((q >> 1) == phase) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int d = (2 * hq + hh) * DH + mt * 16 + g8 + 8 * (e >> 1), il = 2 * c4 + (e & 1);
+                        float *x = dst + il * HD + d;
+                        *x = (phase ? *x : 0.f) + acc[hh][mt][e];
+                    }
+        }
+        __syncthreads();
+    }
+}
+
+// Push 64 per-(row, head) floats src[x] to slot `rank` of every CTA's
+// receive buffer s_recv ([16][64] f32).
+__device__ __forceinline__ void push_rowvals_f32(uint8_t *sp, uint32_t sbase, uint32_t s_src, uint32_t s_recv,
+                                                 uint32_t bar, int tid, uint32_t rank, uint32_t nclu) {
+    const int x = tid >> 3, p0 = tid & 7;
+    const float v = reinterpret_cast<const float *>(sp + s_src)[x];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const uint32_t pp = p0 + 8 * u;
+        if (pp < nclu) st_async_f32(map_peer(sbase + s_recv + (rank * 64 + x) * 4, pp), v, map_peer(bar, pp));
+    }
+}
+
+// Sum of the nclu received copies of 64 floats ([16][64] f32), fixed order.
+__device__ __forceinline__ void combine_rowvals_f32(uint8_t *sp, uint32_t s_recv, uint32_t s_out, int tid,
+                                                    uint32_t nclu) {
+    const int x = tid >> 3, pp = tid & 7;
+    const float *rv = reinterpret_cast<const float *>(sp + s_recv);
+    float l = ((uint32_t)pp < nclu ? rv[pp * 64 + x] : 0.f) + ((uint32_t)(pp + 8) < nclu ? rv[(pp + 8) * 64 + x] : 0.f);
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (pp == 0) reinterpret_cast<float *>(sp + s_out)[x] = l;
+}
+
+// Push a flat fp32 array of `count` floats (count % 4 == 0) to its owners:
+// float4 group g goes to rank g / per4 (per4 = ceil(count/4 / nclu)), slot
+// rank * per4 + (g - owner * per4) of the owner's receive buffer.
+__device__ __forceinline__ void push_flat(uint8_t *sp, uint32_t sbase, uint32_t s_src, int count, uint32_t s_recv,
+                                          uint32_t bar, int tid, uint32_t rank, uint32_t nclu) {
+    const int g4 = count / 4;
+    const uint32_t per = (g4 + nclu - 1) / nclu;
+    const float4 *src = reinterpret_cast<const float4 *>(sp + s_src);
+    for (int g = tid; g < g4; g += NTHR) {
+        const uint32_t owner = g / per, slot = rank * per + (g - owner * per);
+        st_async_v4(map_peer(sbase + s_recv + slot * 16, owner), src[g], map_peer(bar, owner));
+    }
+}
+__host__ __device__ inline uint32_t flat_slice(int count, uint32_t nclu, uint32_t r) {
+    const int g4 = count / 4, per = (g4 + (int)nclu - 1) / (int)nclu, lo = (int)r * per, hi = min(g4, lo + per);
+    return hi > lo ? (uint32_t)(hi - lo) : 0u;
 }
 
 // Owner side: after its receive mbarrier completed, sum the nclu pushed

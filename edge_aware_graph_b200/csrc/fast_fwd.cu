@@ -67,6 +67,7 @@ struct FwdParams {
     float *LSE;
     int *status;
     int n;
+    uint32_t prefetch_ahead;   // CTAs between this one and the one whose tiles it prefetches (0: none)
 };
 
 template <int NR>
@@ -106,6 +107,16 @@ k_fwd_pairs(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUt
         for (int k = 0; k < 4; ++k) {
             tma_load_3d(sbase + S::K + k * NR * 4096, &tmK, bar_kv, 64 * k, j0, b);
             tma_load_3d(sbase + S::V + k * NR * 4096, &tmV, bar_kv, 64 * k, j0, b);
+        }        // L2 prefetch of the tiles of the CTA that runs about one wave later
+        const uint32_t cid = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x + p.prefetch_ahead;
+        if (p.prefetch_ahead && cid < gridDim.x * gridDim.y * gridDim.z) {
+            const int px = cid % gridDim.x, py = (cid / gridDim.x) % gridDim.y, pz = cid / (gridDim.x * gridDim.y);
+            tma_prefetch_5d(&tmE, 0, py * TB / 2, px * TCN, 0, pz);
+            if (py == 0)
+                for (int k = 0; k < 4; ++k) {
+                    tma_prefetch_3d(&tmK, 64 * k, px * TCN, pz);
+                    tma_prefetch_3d(&tmV, 64 * k, px * TCN, pz);
+                }
         }
     }
     if (W == 0) {
@@ -338,6 +349,7 @@ static cudaError_t launch_fwd_nr(const eaga_dims &d, const FwdArgs &a, const uin
     p.LSE = a.LSE;
     p.status = a.status;
     p.n = d.n;
+    p.prefetch_ahead = (uint32_t)(sm_count() * (NR == 1 ? 2 : 1));
     const int nc = (d.n + TCN - 1) / TCN;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nc, (d.n + TB - 1) / TB, d.B);
