@@ -5,9 +5,10 @@
 // clients that link this library but no device allocator, or code running
 // under a framework whose memory pool must not be bypassed and that only
 // hands out the tensors it owns (inputs, outputs, the saved state).  For them
-// the forward's small scratch (the status word, the per-graph global FiLM
-// term and the tensor-core operand images of the FiLM and edge weights) lives
-// in a fixed device array inside this library instead of a caller buffer.
+// the forward's scratch (the status word, the per-graph global FiLM term, the
+// tensor-core operand images of the FiLM and edge weights and the transposed
+// node weights) lives in a fixed device array inside this library instead of
+// a caller buffer.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds NOALLOC_SCRATCH_BYTES of it until the process exits.  All
@@ -23,9 +24,8 @@ using namespace eaga;
 
 namespace {
 
-constexpr size_t NOALLOC_SCRATCH_BYTES = 64 * 1024;   // status word + g [B,2H] fp32 + 8 KB of operand images
+constexpr size_t NOALLOC_SCRATCH_BYTES = 4u << 20;   // status word + g [B,2H] fp32 + weight images
 constexpr size_t NOALLOC_STATUS = 0, NOALLOC_G = 256;
-constexpr size_t IMAGE_BYTES = 8192;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
@@ -70,8 +70,9 @@ eaga_status eaga_forward_noalloc(const eaga_dims *d, const void *X, const void *
         if (!aligned16(p)) return EAGA_ERR_MISALIGNED;
     }
     const size_t g_bytes = align256(size_t(d->B) * 2 * d->H * sizeof(float));
-    const size_t needed = NOALLOC_G + g_bytes + IMAGE_BYTES;
-    if (needed > NOALLOC_SCRATCH_BYTES) return EAGA_ERR_UNSUPPORTED;   // too many graphs for the fixed array
+    const size_t images = fast::supports(*d) ? fast::forward_scratch_bytes(*d) : 0;
+    const size_t needed = NOALLOC_G + g_bytes + images;
+    if (needed > NOALLOC_SCRATCH_BYTES) return EAGA_ERR_UNSUPPORTED;   // too large for the fixed array
 
     void *base = nullptr;
     eaga_status s = scratch_address(&base);

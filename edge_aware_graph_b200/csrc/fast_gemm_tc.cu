@@ -1,0 +1,205 @@
+// Node-side GEMMs on tcgen05: C[M, N] = sum_seg A_seg[M, K] Bt_seg[N, K]^T,
+// both operands K-major (row-major with K contiguous), 128B-swizzled tiles
+// loaded by TMA through a 4-stage mbarrier pipeline, the 128 x BN fp32
+// accumulator in TMEM, and the layer's epilogues fused:
+//   QKV      [Q|K|V] = X [Wq|Wk|Wv] + b, masked rows zero   (Bt = the three W^T stacked)
+//   out-proj X' = X + M (O Wo + bo)                         (Bt = Wo^T)
+//   dO       dO = M (dX' Wo^T)                              (Bt = Wo)
+//   dX       dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T          (three segments, Bt = W)
+// One thread issues TMA and MMAs; the four warps run the epilogue from TMEM.
+#include "fast.h"
+#include "fast_common.cuh"
+
+namespace eaga {
+namespace fast {
+
+using namespace sm100;
+
+constexpr int TBM = 128, TBK = 64, TSTAGES = 4, TTHR = 128;
+enum TcMode { TC_QKV = 0, TC_OUT = 1, TC_DO = 2, TC_DX = 3 };
+
+struct TcParams {
+    const __nv_bfloat16 *bias[3];
+    __nv_bfloat16 *C[3];
+    const __nv_bfloat16 *R;      // residual [M, Nb]
+    const uint8_t *mask;         // [M]
+    int *status;
+    int M, K, Nb, nseg, mode;
+};
+
+template <int BN>
+struct TcSmem {
+    static constexpr uint32_t A_BYTES = TBM * TBK * 2, B_BYTES = BN * TBK * 2;
+    static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+    static constexpr uint32_t BAR = TSTAGES * STAGE;        // full[S], empty[S], done
+    static constexpr uint32_t TM = BAR + (2 * TSTAGES + 1) * 8;
+    static constexpr uint32_t BYTES = TM + 16 + 1024;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(TTHR, 1)
+k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtensorMap a1,
+          const __grid_constant__ CUtensorMap a2, const __grid_constant__ CUtensorMap b0,
+          const __grid_constant__ CUtensorMap b1, const __grid_constant__ CUtensorMap b2, TcParams p) {
+    using S = TcSmem<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
+    const int tid = threadIdx.x, w = tid >> 5, t = tid & 31;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * TBM;
+    const uint32_t bar0 = sbase + S::BAR;
+    auto full = [&](int s) { return bar0 + 8 * s; };
+    auto empty = [&](int s) { return bar0 + 8 * (TSTAGES + s); };
+    const uint32_t done = bar0 + 16 * TSTAGES;
+    const int kt_seg = p.K / TBK, nk = kt_seg * p.nseg;
+
+    if (tid == 0) {
+        for (int s = 0; s < TSTAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    if (w == 0) {
+        tmem_alloc(sbase + S::TM, BN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+
+    if (tid == 0) {
+        auto issue_load = [&](int kt) {
+            const int s = kt % TSTAGES, seg = kt / kt_seg, k0 = (kt % kt_seg) * TBK;
+            const CUtensorMap *am = seg == 0 ? &a0 : seg == 1 ? &a1 : &a2;
+            const CUtensorMap *bm = seg == 0 ? &b0 : seg == 1 ? &b1 : &b2;
+            const uint32_t st = sbase + s * S::STAGE;
+            mbar_expect_tx(full(s), S::STAGE);
+            tma_load_2d(st, am, full(s), k0, m0);
+            tma_load_2d(st + S::A_BYTES, bm, full(s), k0, n0);
+        };
+        for (int kt = 0; kt < TSTAGES && kt < nk; ++kt) issue_load(kt);
+        const uint32_t idesc = idesc_bf16_f32(TBM, BN);
+        for (int kt = 0; kt < nk; ++kt) {
+            const int s = kt % TSTAGES;
+            const uint32_t ph = (kt / TSTAGES) & 1;
+            if (!mbar_wait(full(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
+            tc_fence_after();
+            const uint32_t st = sbase + s * S::STAGE;
+#pragma unroll
+            for (int kk = 0; kk < TBK / 16; ++kk)
+                mma_bf16_ss(tmem, smem_desc(st + kk * 32, 16, 1024, LAYOUT_SW128),
+                            smem_desc(st + S::A_BYTES + kk * 32, 16, 1024, LAYOUT_SW128), idesc,
+                            (kt > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(empty(s));
+            if (kt + TSTAGES < nk) {
+                if (!mbar_wait(empty(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
+                issue_load(kt + TSTAGES);
+            }
+        }
+        mma_commit(done);
+    }
+    __syncwarp();
+    if (!mbar_wait(done, 0)) atomicExch(p.status, DEV_TIMEOUT);
+    tc_fence_after();
+
+    // epilogue: warp w holds rows m0 + 32w + t, 16 columns per TMEM load
+    const int row = m0 + 32 * w + t;
+    const bool in = row < p.M;
+    const bool mk = in && p.mask[in ? row : 0] != 0;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + c0, v);
+        tmem_ld_wait();
+        if (!in) continue;
+        const int ng = n0 + c0, which = ng / p.Nb, col = ng % p.Nb;
+        const size_t o = (size_t)row * p.Nb + col;
+        uint4 outv[2];
+        __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(outv);
+        if (p.mode == TC_QKV || p.mode == TC_OUT) {
+            const uint4 *bb = reinterpret_cast<const uint4 *>(p.bias[which] + col);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 bv = bb[h];
+                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&bv);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float2 f = __bfloat1622float2(b2[u]);
+                    v[8 * h + 2 * u] += f.x;
+                    v[8 * h + 2 * u + 1] += f.y;
+                }
+            }
+        }
+        if (p.mode == TC_QKV || p.mode == TC_DO) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                o2[u] = mk ? __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]) : __floats2bfloat162_rn(0.f, 0.f);
+        } else {
+            const uint4 *rr = reinterpret_cast<const uint4 *>(p.R + o);
+            const uint4 r0 = rr[0], r1 = rr[1];
+            const __nv_bfloat162 *x2[2] = {reinterpret_cast<const __nv_bfloat162 *>(&r0),
+                                           reinterpret_cast<const __nv_bfloat162 *>(&r1)};
+            const bool add = p.mode == TC_DX || mk;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const __nv_bfloat162 xr = x2[u >> 2][u & 3];
+                const float2 x = __bfloat1622float2(xr);
+                o2[u] = add ? __floats2bfloat162_rn(x.x + v[2 * u], x.y + v[2 * u + 1]) : xr;
+            }
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(p.C[which] + o);
+        dst[0] = outv[0];
+        dst[1] = outv[1];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tmem, BN);
+}
+
+// ------------------------------------------------------------------ host side
+
+bool encode_2d(CUtensorMap *m, const void *base, int rows, int cols, int box_rows);
+
+template <int BN>
+static cudaError_t tc_launch(const CUtensorMap (&am)[3], const CUtensorMap (&bm)[3], const TcParams &p, int N,
+                             cudaStream_t st) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             TcSmem<BN>::BYTES);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    dim3 grid(N / BN, (p.M + TBM - 1) / TBM);
+    k_tc_gemm<BN><<<grid, TTHR, TcSmem<BN>::BYTES, st>>>(am[0], am[1], am[2], bm[0], bm[1], bm[2], p);
+    return cudaGetLastError();
+}
+
+// Out = epilogue(sum_seg A[seg] Bt[seg]^T): A[seg] [M, K], Bt[seg] [N, K] row-major bf16.
+cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A[3], const void *const Bt[3],
+                    const void *const bias[3], void *const C[3], int Nb, const void *R, const uint8_t *mask,
+                    int *status, cudaStream_t st) {
+    CUtensorMap am[3], bm[3];
+    const int BN = N >= 512 ? 128 : 64;
+    for (int s = 0; s < 3; ++s) {
+        const int ss = s < nseg ? s : 0;
+        if (!encode_2d(&am[s], A[ss], M, K, TBM) || !encode_2d(&bm[s], Bt[ss], N, K, BN))
+            return cudaErrorInvalidValue;
+    }
+    TcParams p = {};
+    for (int s = 0; s < 3; ++s) {
+        p.bias[s] = static_cast<const __nv_bfloat16 *>(bias ? bias[s] : nullptr);
+        p.C[s] = static_cast<__nv_bfloat16 *>(C[s]);
+    }
+    p.R = static_cast<const __nv_bfloat16 *>(R);
+    p.mask = mask;
+    p.status = status;
+    p.M = M; p.K = K; p.Nb = Nb; p.nseg = nseg; p.mode = mode;
+    return BN == 128 ? tc_launch<128>(am, bm, p, N, st) : tc_launch<64>(am, bm, p, N, st);
+}
+
+}  // namespace fast
+}  // namespace eaga
