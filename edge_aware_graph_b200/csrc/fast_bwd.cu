@@ -9,11 +9,11 @@
 // D needs a whole row of pairs before any dS' exists, so the work is split in
 //   k_bwd_rows: clusters along j (like the forward): a, u, dA, cluster-wide D,
 //               dS', dq (cluster-reduced), dE (tensor cores, written in place,
-//               TMA store), dWfe / dWe / dg partials reduced over the cluster;
-//   k_bwd_cols: clusters along i on the transposed tile: a and ds again from
-//               E, dE' and the D of the row kernel; dk, dv reduced over the
-//               cluster.
-// Both tiles are loaded once with TMA and stay in shared memory; the FiLM and
+//               TMA store), dWfe / dWe / dg partials reduced over the cluster,
+//               and a, ds of every pair stored in bf16 (32 bytes per pair);
+//   k_bwd_kv:   dk, dv as sums over rows i of those a, ds times Q, dO (warp
+//               MMAs fed by a TMA pipeline), so E and dE' are read only once.
+// The row kernel loads both pair tiles once with TMA and keeps them in shared memory; the FiLM and
 // u = dE' We^T products run on tcgen05 with the same pair <-> TMEM lane map as
 // the forward.  16 warps: warp W reads TMEM quadrant W%4, heads 2(W/4)+{0,1}.
 // NR selects 32NR cluster rows per CTA (NR = 1: two CTAs share an SM).
@@ -34,14 +34,12 @@ struct BwdRowParams {
     float *D;                // [B,H,n] out
     __nv_bfloat16 *dQ;       // [B,n,256] out (scaled)
     float *rparts;           // [graph * row block][RPART] out
+    __nv_bfloat16 *Pa, *Pds; // [B,H,n,npad] out: a and ds (unscaled) of every pair
     int *status;
-    int n;
+    int n, npad;
 };
 
-struct BwdColParams {
-    const __nv_bfloat16 *K, *V;
-    const float *LSE, *D, *g;
-    const uint8_t *img, *M;
+struct BwdKvParams {
     __nv_bfloat16 *dK, *dV;  // [B,n,256] out (dK scaled)
     int *status;
     int n;
@@ -234,6 +232,23 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
         *reinterpret_cast<uint32_t *>(sp + S::AT + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(av[0][e], av[1][e]);
         if (hq == 0) *reinterpret_cast<uint4 *>(sp + S::AT + e * 4096 + ns16(L, 8)) = make_uint4(0, 0, 0, 0);
     }
+    // a and ds of the tile's pairs for the dk / dv pass: [b][h][i][j] bf16.
+    // Lanes t and t^4 hold neighbouring columns j; they swap one head so that
+    // each stores two columns of one head in a 4-byte word.
+    {
+        const bool odd = g8 & 1;
+#pragma unroll
+        for (int e = 0; e < NE; ++e) {
+            const float xa = __shfl_xor_sync(0xffffffffu, odd ? av[0][e] : av[1][e], 4);
+            const float xd = __shfl_xor_sync(0xffffffffu, odd ? da[0][e] : da[1][e], 4);
+            const int i = i0 + 2 * c4 + (e & 1), j = j0 + 32 * (e >> 1) + 8 * q + (g8 & ~1);
+            if (i < n && j < n) {
+                const size_t o = (((size_t)b * NH + 2 * hq + (odd ? 1 : 0)) * n + i) * p.npad + j;
+                *reinterpret_cast<uint32_t *>(p.Pa + o) = odd ? pack_bf16(xa, av[1][e]) : pack_bf16(av[0][e], xa);
+                *reinterpret_cast<uint32_t *>(p.Pds + o) = odd ? pack_bf16(xd, da[1][e]) : pack_bf16(da[0][e], xd);
+            }
+        }
+    }
     float *wdg = reinterpret_cast<float *>(sp + S::WDG);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -382,158 +397,108 @@ k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUte
     if (W == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
-// ---------------------------------------------------------------- column kernel
-
-template <int NR>
-struct ColSmem {
-    static constexpr uint32_t E = 0, DEP = NR * 32768, Q = NR * 65536, DO = Q + NR * 16384;
-    static constexpr uint32_t IMG = DO + NR * 16384;               // Wfe^T sw, We sw
-    static constexpr uint32_t G = IMG + 4096;
-    static constexpr uint32_t MI = G + 64, MJ = MI + 64;
-    static constexpr uint32_t BAR = MJ + 16;                       // 6 mbarriers
-    static constexpr uint32_t TM = BAR + 48;
-    static constexpr uint32_t BYTES = TM + 16 + 1024;
-    // after the tiles are dead: two-slot quadrant sums of dk, dv in the E
-    // tile, the pushed cluster partials received in the dE' tile
-    static constexpr uint32_t KPART = E, VPART = E + 16384, RECV = DEP;
+// ---------------------------------------------------------------- dk, dv pass
+// dk_j = sum_i ds_ij q_i / sqrt(dh) and dv_j = sum_i a_ij dO_i from the a and
+// ds the row kernel stored.  CTA = (32 columns j, graph), warp = head; each
+// pipeline stage brings 16 rows i of a, ds (all heads), Q and dO with TMA and
+// every warp adds their products on warp MMAs (M = j, N = d, K = i).
+constexpr int KV_J = 32, KV_I = 16, KV_STAGES = 3, KV_THR = 256;
+struct KvSmem {
+    static constexpr uint32_t PDS = 0, PA = 8192, QT = 16384, DOT = 24576, STAGE = 32768;
+    static constexpr uint32_t BAR = KV_STAGES * STAGE;            // full[S], empty[S]
+    static constexpr uint32_t BYTES = BAR + 2 * KV_STAGES * 8 + 1024;
 };
 
-template <int NR>
-__global__ void __launch_bounds__(NTHR, NR == 1 ? 2 : 1)
-k_bwd_cols(const __grid_constant__ CUtensorMap tmEt, const __grid_constant__ CUtensorMap tmDEpt,
-           const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO, BwdColParams p) {
-    using S = ColSmem<NR>;
-    constexpr int TCN = tile_cols(NR), NE = 2 * NR;
+__global__ void __launch_bounds__(KV_THR, 2)
+k_bwd_kv(const __grid_constant__ CUtensorMap tmPds, const __grid_constant__ CUtensorMap tmPa,
+         const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO, BwdKvParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
-    const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = W >> 2, t = tid & 31, c4 = t & 3, g8 = t >> 2;
-    const uint32_t rank = cluster_rank(), nclu = gridDim.x;
-    const int n = p.n;
-    const int i0 = blockIdx.x * TCN, j0 = blockIdx.y * TB, b = blockIdx.z;   // 32NR rows i, 8 columns j
-    const uint32_t bar_e = sbase + S::BAR, bar_dep = bar_e + 8, bar_q = bar_e + 16, bar_film = bar_e + 24,
-                   bar_u = bar_e + 32, bar_r = bar_e + 40;
-    float *g = reinterpret_cast<float *>(sp + S::G);
-    uint8_t *mi = sp + S::MI, *mj = sp + S::MJ;
-    constexpr uint32_t TM_FILM = 0, TM_U = 64, TM_COLS = 128;
-
+    const int tid = threadIdx.x, h = tid >> 5, t = tid & 31, g8 = t >> 2, c4 = t & 3;
+    const int n = p.n, j0 = blockIdx.x * KV_J, b = blockIdx.y;
+    const int nsteps = (n + KV_I - 1) / KV_I;
+    const uint32_t bar0 = sbase + KvSmem::BAR;
+    auto full = [&](int s) { return bar0 + 8 * s; };
+    auto empty = [&](int s) { return bar0 + 8 * (KV_STAGES + s); };
+    auto issue = [&](int k) {
+        const int s = k % KV_STAGES, i0 = k * KV_I;
+        const uint32_t st = sbase + s * KvSmem::STAGE;
+        mbar_expect_tx(full(s), KvSmem::STAGE);
+        tma_load_4d(st + KvSmem::PDS, &tmPds, full(s), j0, i0, 0, b);
+        tma_load_4d(st + KvSmem::PA, &tmPa, full(s), j0, i0, 0, b);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            tma_load_3d(st + KvSmem::QT + c * 2048, &tmQ, full(s), 64 * c, i0, b);
+            tma_load_3d(st + KvSmem::DOT + c * 2048, &tmDO, full(s), 64 * c, i0, b);
+        }
+    };
     if (tid == 0) {
-        mbar_init(bar_e, 1); mbar_init(bar_dep, 1); mbar_init(bar_q, 1);
-        mbar_init(bar_film, 1); mbar_init(bar_u, 1); mbar_init(bar_r, 1);
+        for (int s = 0; s < KV_STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), KV_THR / 32);
+        }
         fence_mbar_init();
-        mbar_expect_tx(bar_r, nclu * rows_slice(2, nclu, rank) * 16);
-        mbar_expect_tx(bar_e, NR * 32768);
-        tma_load_5d(sbase + S::E, &tmEt, bar_e, 0, j0 / 2, i0, 0, b);
-        mbar_expect_tx(bar_dep, NR * 32768);
-        tma_load_5d(sbase + S::DEP, &tmDEpt, bar_dep, 0, j0 / 2, i0, 0, b);
-        mbar_expect_tx(bar_q, NR * 32768);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            tma_load_3d(sbase + S::Q + k * NR * 4096, &tmQ, bar_q, 64 * k, i0, b);
-            tma_load_3d(sbase + S::DO + k * NR * 4096, &tmDO, bar_q, 64 * k, i0, b);
-        }
+        for (int k = 0; k < KV_STAGES && k < nsteps; ++k) issue(k);
     }
-    if (W == 0) {
-        tmem_alloc(sbase + S::TM, TM_COLS);
-        tmem_relinquish();
-    }
-    if (tid < 256) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.img);
-        const uint32_t img_off = (tid >> 7) == 0 ? IMG_WFE_T_SW : IMG_WE_SW;
-        reinterpret_cast<uint4 *>(sp + S::IMG)[tid] = src[(img_off >> 4) + (tid & 127)];
-    }
-    if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
-    if (tid >= 64 && tid < 64 + TCN) mi[tid - 64] = (i0 + tid - 64 < n) ? p.M[(size_t)b * n + i0 + tid - 64] : 0;
-    if (tid >= 32 && tid < 32 + TB) mj[tid - 32] = (j0 + tid - 32 < n) ? p.M[(size_t)b * n + j0 + tid - 32] : 0;
-    // per-thread rows i = i0 + 32r + 8q + g8: LSE and D for the warp's 2 heads
-    float lse[2][2], dd[2][2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int i = i0 + 32 * r + 8 * q + g8;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const size_t o = ((size_t)b * NH + 2 * hq + hh) * n + i;
-            const bool ok = (r < NR) && i < n;
-            lse[r][hh] = ok ? p.LSE[o] : 0.f;
-            dd[r][hh] = ok ? p.D[o] : 0.f;
-        }
-    }
-    uint32_t kf[2][2][2], vf[2][2][2];
-    load_frags2(p.K, b, n, j0, hq, g8, c4, kf);
-    load_frags2(p.V, b, n, j0, hq, g8, c4, vf);
-    fence_proxy_async_smem();
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
-    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
 
-    if (tid == 0) {
-        if (!mbar_wait(bar_e, 0)) flag_timeout(p.status);
-        tc_fence_after();
-        issue_pair_products<NR>(sbase + S::E, sbase + S::IMG, tmem + TM_FILM);
-        mma_commit(bar_film);
-        if (!mbar_wait(bar_dep, 0)) flag_timeout(p.status);
-        tc_fence_after();
-        issue_pair_products<NR>(sbase + S::DEP, sbase + S::IMG + 2048, tmem + TM_U);
-        mma_commit(bar_u);
+    float kacc[2][4][4], vacc[2][4][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) kacc[mt][nt][x] = vacc[mt][nt][x] = 0.f;
+    // ldmatrix lanes: A = P^T (stored [i][j]) and B = Q, dO (stored [i][d]), both transposed loads
+    const int arow = (t & 7) + ((t >> 4) & 1) * 8, ach = (t >> 3) & 1;
+    const int brow = (t & 7) + ((t >> 3) & 1) * 8, bch = t >> 4;
+    for (int k = 0; k < nsteps; ++k) {
+        const int s = k % KV_STAGES;
+        const uint32_t ph = (k / KV_STAGES) & 1;
+        if (!mbar_wait(full(s), ph)) flag_timeout(p.status);
+        const uint32_t st = sbase + s * KvSmem::STAGE;
+        uint32_t bq[2][4], bo[2][4];
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+            const uint32_t off = (h >> 1) * 2048 + sw128(brow, (h & 1) * 4 + 2 * np + bch);
+            ldsm_x4_t(st + KvSmem::QT + off, bq[np]);
+            ldsm_x4_t(st + KvSmem::DOT + off, bo[np]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            const uint32_t off = h * 1024 + sw64(arow, 2 * mt + ach);
+            uint32_t ad[4], aa[4];
+            ldsm_x4_t(st + KvSmem::PDS + off, ad);
+            ldsm_x4_t(st + KvSmem::PA + off, aa);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                mma16816(kacc[mt][nt], ad, bq[nt >> 1][2 * (nt & 1)], bq[nt >> 1][2 * (nt & 1) + 1]);
+                mma16816(vacc[mt][nt], aa, bo[nt >> 1][2 * (nt & 1)], bo[nt >> 1][2 * (nt & 1) + 1]);
+            }
+        }
+        __syncwarp();
+        if (t == 0) mbar_arrive(empty(s));
+        if (tid == 0 && k + KV_STAGES < nsteps) {
+            if (!mbar_wait(empty(s), ph)) flag_timeout(p.status);
+            issue(k + KV_STAGES);
+        }
+        __syncwarp();
     }
-    __syncwarp();
-    if (!mbar_wait(bar_q, 0)) flag_timeout(p.status);
-    // S = Q K^T and dP = dO V^T on the transposed tile: rows i (M), columns j (N)
-    float sv[2][4], da[2][4];
-    warp_scores2<NR>(sbase + S::Q, q, t, hq, kf, sv);
-    warp_scores2<NR>(sbase + S::DO, q, t, hq, vf, da);
-
-    if (!mbar_wait(bar_film, 0)) flag_timeout(p.status);
-    if (!mbar_wait(bar_u, 0)) flag_timeout(p.status);
-    tc_fence_after();
     const float rs = rsqrtf((float)DH);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        if (e >= NE) {
-            sv[0][e] = sv[1][e] = da[0][e] = da[1][e] = 0.f;
-            continue;
-        }
-        const int r = e >> 1, il = 32 * r + 8 * q + g8, jl = 2 * c4 + (e & 1);
-        const bool valid = mi[il] && mj[jl];
-        float f0, f1, b0, b1, u0, u1;
-        tmem_ld2(tl + TM_FILM + 16 * e + 2 * hq, f0, f1);
-        tmem_ld2(tl + TM_FILM + 16 * e + NH + 2 * hq, b0, b1);
-        tmem_ld2(tl + TM_U + 16 * e + 2 * hq, u0, u1);
-        tmem_ld_wait();
-        const float fg[2] = {f0, f1}, fb[2] = {b0, b1}, fu[2] = {u0, u1};
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int h = 2 * hq + hh;
-            const float s = sv[hh][e] * rs;
-            const float gam = fg[hh] + g[h], bet = fb[hh] + g[NH + h];
-            const float a = valid ? exp2f((s * (1.f + gam) + bet - lse[r][hh]) * LOG2E) : 0.f;
-            const float dsp = a * (da[hh][e] + fu[hh] - dd[r][hh]);
-            sv[hh][e] = a;                       // a
-            da[hh][e] = dsp * (1.f + gam);       // ds
+        for (int hf = 0; hf < 2; ++hf) {
+            const int j = j0 + 16 * mt + 8 * hf + g8;
+            if (j >= n) continue;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const size_t o = ((size_t)b * n + j) * HD + h * DH + nt * 8 + 2 * c4;
+                *reinterpret_cast<uint32_t *>(p.dK + o) =
+                    pack_bf16(kacc[mt][nt][2 * hf] * rs, kacc[mt][nt][2 * hf + 1] * rs);
+                *reinterpret_cast<uint32_t *>(p.dV + o) = pack_bf16(vacc[mt][nt][2 * hf], vacc[mt][nt][2 * hf + 1]);
+            }
         }
-    }
-    tc_fence_before();
-    __syncthreads();   // tiles are dead: their space holds the partials below
-    cluster_arrive();  // peers may now push into this CTA's dE' tile space
-    float kacc[2][2][4], vacc[2][2][4];
-    warp_contract2<NR>(sbase + S::Q, q, t, hq, da, kacc);    // dk^T = Q^T ds
-    warp_contract2<NR>(sbase + S::DO, q, t, hq, sv, vacc);   // dv^T = dO^T a
-    store_quadrant_part_2ph(sp, S::KPART, kacc, q, hq, t);
-    store_quadrant_part_2ph(sp, S::VPART, vacc, q, hq, t);
-    cluster_wait();
-    {
-        const uint32_t parts[2] = {S::KPART, S::VPART};
-        push_rows_partials<2, 2>(sp, sbase, parts, S::RECV, bar_r, tid, rank, nclu);
-        if (!mbar_wait(bar_r, 0)) flag_timeout(p.status);
-        __nv_bfloat16 *const outs[2] = {p.dK, p.dV};
-        const float sc[2] = {rs, 1.f};
-        finish_rows_partials<2>(sp, S::RECV, tid, rank, nclu, outs, b, n, j0, sc);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (W == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
 // ---------------------------------------------------------------- reductions
@@ -663,10 +628,7 @@ static cudaError_t launch_bwd_nr(const eaga_dims &d, const BwdArgs &a, const Fas
         if ((e = cudaFuncSetAttribute(k_bwd_rows<NR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
             cudaSuccess)
             return e;
-        if ((e = cudaFuncSetAttribute(k_bwd_cols<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      ColSmem<NR>::BYTES)) != cudaSuccess)
-            return e;
-        if ((e = cudaFuncSetAttribute(k_bwd_cols<NR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+        if ((e = cudaFuncSetAttribute(k_bwd_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, KvSmem::BYTES)) !=
             cudaSuccess)
             return e;
         attr_done = true;
@@ -704,34 +666,28 @@ static cudaError_t launch_bwd_nr(const eaga_dims &d, const BwdArgs &a, const Fas
         p.D = D;
         p.dQ = dQ;
         p.rparts = reinterpret_cast<float *>(ws + W.rparts);
+        p.Pa = reinterpret_cast<__nv_bfloat16 *>(ws + W.Pa);
+        p.Pds = reinterpret_cast<__nv_bfloat16 *>(ws + W.Pds);
         p.status = a.status;
         p.n = d.n;
+        p.npad = W.npad;
         cfg.gridDim = dim3(nc, (d.n + TB - 1) / TB, d.B);
         cfg.dynamicSmemBytes = RowSmem<NR>::BYTES;
         cudaError_t e = cudaLaunchKernelEx(&cfg, k_bwd_rows<NR>, mE, mDEp, mDE, mK, mV, p);
         if (e != cudaSuccess) return e;
     }
     {
-        CUtensorMap mEt, mDEpt, mQ, mDO;
-        if (!encode_pair_map(&mEt, a.E, d.B, d.n, true, TCN) ||
-            !encode_pair_map(&mDEpt, a.dEout, d.B, d.n, true, TCN) || !encode_node_map(&mQ, a.Q, d.B, d.n, TCN) ||
-            !encode_node_map(&mDO, dO, d.B, d.n, TCN))
+        CUtensorMap mPds, mPa, mQ, mDO;
+        if (!encode_p_map(&mPds, ws + W.Pds, d.B, d.n, W.npad) || !encode_p_map(&mPa, ws + W.Pa, d.B, d.n, W.npad) ||
+            !encode_node_map(&mQ, a.Q, d.B, d.n, KV_I) || !encode_node_map(&mDO, dO, d.B, d.n, KV_I))
             return cudaErrorInvalidValue;
-        BwdColParams p;
-        p.K = static_cast<const __nv_bfloat16 *>(a.K);
-        p.V = static_cast<const __nv_bfloat16 *>(a.V);
-        p.LSE = a.LSE;
-        p.D = D;
-        p.g = g;
-        p.img = reinterpret_cast<const uint8_t *>(ws + W.img);
-        p.M = a.M;
+        BwdKvParams p;
         p.dK = dK;
         p.dV = dV;
         p.status = a.status;
         p.n = d.n;
-        cfg.gridDim = dim3(nc, (d.n + TB - 1) / TB, d.B);
-        cfg.dynamicSmemBytes = ColSmem<NR>::BYTES;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, k_bwd_cols<NR>, mEt, mDEpt, mQ, mDO, p);
+        k_bwd_kv<<<dim3((d.n + KV_J - 1) / KV_J, d.B), KV_THR, KvSmem::BYTES, st>>>(mPds, mPa, mQ, mDO, p);
+        cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

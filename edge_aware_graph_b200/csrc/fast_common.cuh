@@ -40,14 +40,18 @@ __host__ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t ch) {
     return row * 128u + ((ch ^ (row & 7u)) << 4);
 }
 // byte offset of element (row, k) in a no-swizzle K-major [rows][16] bf16 tile
+// byte offset of 16-byte chunk `ch` of row `row` in a 64B-swizzled region of 64-byte rows
+__host__ __device__ __forceinline__ uint32_t sw64(uint32_t row, uint32_t ch) {
+    return row * 64u + ((ch ^ ((row >> 1) & 3u)) << 4);
+}
 __host__ __device__ __forceinline__ uint32_t ns16(uint32_t row, uint32_t k) {
     return (row >> 3) * 256u + (k >> 3) * 128u + (row & 7u) * 16u + (k & 7u) * 2u;
 }
 
 // Workspace of the fast path (after the common status word and g).
 struct FastWs {
-    size_t img, dO, dQ, dK, dV, D, rparts, wparts, bparts, r2, dg, total;
-    int n_rparts, wsplits, bsplits, rsplits;
+    size_t img, dO, dQ, dK, dV, D, Pa, Pds, rparts, wparts, bparts, r2, dg, total;
+    int n_rparts, wsplits, bsplits, rsplits, npad;
 };
 
 inline int row_blocks(const eaga_dims &d) { return ((d.n + TB - 1) / TB) * d.B; }
@@ -68,6 +72,10 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
     W.dK = off; off = align256(off + rows * HD * 2);
     W.dV = off; off = align256(off + rows * HD * 2);
     W.D = off; off = align256(off + size_t(d.B) * NH * d.n * 4);
+    // a and ds of every pair, [B][H][n][npad] bf16, for the dk / dv pass
+    W.npad = (d.n + 7) / 8 * 8;
+    W.Pa = off; off = align256(off + size_t(d.B) * NH * d.n * W.npad * 2);
+    W.Pds = off; off = align256(off + size_t(d.B) * NH * d.n * W.npad * 2);
     W.n_rparts = row_blocks(d);
     W.rparts = off; off = align256(off + size_t(W.n_rparts) * RPART * 4);
     W.wsplits = wgrad_splits(d);
@@ -84,6 +92,7 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
 
 bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transposed, int box_rows);
 bool encode_node_map(CUtensorMap *m, const void *base, int B, int n, int box_rows);
+bool encode_p_map(CUtensorMap *m, const void *base, int B, int n, int npad);
 
 
 // ------------------------------------------------------------------ device pieces

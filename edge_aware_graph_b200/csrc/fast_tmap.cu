@@ -76,6 +76,20 @@ bool encode_2d(CUtensorMap *m, const void *base, int rows, int cols, int box_row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The per-pair a or ds of the backward, [B][H][n][npad] bf16 (npad = n rounded
+// up to 8); box of 32 columns j x 16 rows i x 8 heads, 64B-swizzled.
+bool encode_p_map(CUtensorMap *m, const void *base, int B, int n, int npad) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)n, (cuuint64_t)n, NH, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)npad * 2, (cuuint64_t)n * npad * 2, (cuuint64_t)NH * n * npad * 2};
+    const cuuint32_t box[4] = {32, 16, NH, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Transposed weight images for the K-major tcgen05 GEMMs of the forward:
 // WqkvT [3*256][dx] (row n = column n%256 of W{q,k,v}[n/256]) and WoT [dx][256].
 __global__ void k_weight_images(const __nv_bfloat16 *Wq, const __nv_bfloat16 *Wk, const __nv_bfloat16 *Wv,

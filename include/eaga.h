@@ -88,8 +88,12 @@ typedef struct {
 } eaga_weight_grads;
 
 /* Bytes of workspace eaga_forward (for_backward = 0) or eaga_backward
- * (for_backward = 1) needs.  Grows as O(B*n*H*dh) + O(B*n*de*H); it has no
- * B*H*n*n term.  Returns 0 for invalid or unsupported dims. */
+ * (for_backward = 1) needs.  The forward's grows as O(B*n*H*dh) + O(B*H)
+ * plus the transposed node weights.  On the specialised bf16 path (de = 64,
+ * H = 8, dh = 32) the backward's also holds the attention weights a and the
+ * score gradients ds of every pair in bf16, 2*B*H*n*roundup8(n) elements:
+ * 32 bytes per pair, a quarter of E, so that E and dE' are read once.
+ * Returns 0 for invalid or unsupported dims. */
 EAGA_API size_t eaga_workspace_size(const eaga_dims *dims, int for_backward);
 
 /* Bytes of the forward's saved state that eaga_backward consumes:
