@@ -505,33 +505,46 @@ k_bwd_kv(const __grid_constant__ CUtensorMap tmPds, const __grid_constant__ CUte
 // All sums run in a fixed order (deterministic): first over segments of rows
 // (or CTAs) in parallel blocks, then over the segments.
 
-// Column sums of segment z of a row-major matrix: out[z][col].  Sources by
-// column: [0,256) dQ, [256,512) dK, [512,768) dV, [768,768+dx) M-masked dX'.
-__global__ void k_bias_partial(const __nv_bfloat16 *dQ, const __nv_bfloat16 *dK, const __nv_bfloat16 *dV,
-                               const __nv_bfloat16 *dXo, const uint8_t *M, int rows, int dx, int seg_rows,
-                               float *out) {
-    const int col = blockIdx.x * blockDim.x + threadIdx.x;
-    const int ncol = 3 * HD + dx;
-    if (col >= ncol) return;
+// Column sums of segment z of the rows: out[z][col].  Sources by column:
+// [0,256) dQ, [256,512) dK, [512,768) dV, [768,768+dx) M-masked dX'.  Block
+// (256-column strip, row segment): lane = 8 columns (one 16-byte load per
+// row), warp = every 8th row of the segment, warps added in a fixed order.
+__global__ void __launch_bounds__(256) k_bias_partial(const __nv_bfloat16 *dQ, const __nv_bfloat16 *dK,
+                                                      const __nv_bfloat16 *dV, const __nv_bfloat16 *dXo,
+                                                      const uint8_t *M, int rows, int dx, int seg_rows, float *out) {
+    __shared__ float red[8][256];
+    const int w = threadIdx.x >> 5, t = threadIdx.x & 31;
+    const int strip = blockIdx.x, ncol = 3 * HD + dx;
+    const bool masked = strip >= 3;
+    const __nv_bfloat16 *src = strip == 0 ? dQ : strip == 1 ? dK : strip == 2 ? dV : dXo;
+    const int ld = masked ? dx : HD, c0 = (masked ? (strip - 3) * 256 : 0) + 8 * t;
+    const bool active = c0 < ld;
     const int r0 = blockIdx.y * seg_rows, r1 = min(rows, r0 + seg_rows);
-    const __nv_bfloat16 *src;
-    int ld, c;
-    if (col < 3 * HD) {
-        src = col < HD ? dQ : col < 2 * HD ? dK : dV;
-        ld = HD;
-        c = col % HD;
-    } else {
-        src = dXo;
-        ld = dx;
-        c = col - 3 * HD;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (active) {
+#pragma unroll 4
+        for (int r = r0 + w; r < r1; r += 8) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * ld + c0);
+            const bool keep = !masked || M[r];
+            const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __bfloat1622float2(v2[u]);
+                acc[2 * u] += keep ? f.x : 0.f;
+                acc[2 * u + 1] += keep ? f.y : 0.f;
+            }
+        }
     }
-    float acc = 0.f;
-    const bool masked = col >= 3 * HD;
-    for (int r = r0; r < r1; ++r) {
-        const float v = __bfloat162float(src[(size_t)r * ld + c]);
-        acc += (!masked || M[r]) ? v : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) red[w][8 * t + u] = acc[u];
+    __syncthreads();
+    const int col = threadIdx.x, gcol = strip * 256 + col;
+    if (gcol < ncol && (!masked || (strip - 3) * 256 + col < dx)) {
+        float x = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x += red[k][col];
+        out[(size_t)blockIdx.y * ncol + gcol] = x;
     }
-    out[(size_t)blockIdx.y * ncol + col] = acc;
 }
 
 // Row-kernel partials: out[z][e] = sum over CTAs of segment z of rparts[cta][e], e < dWfe+dWe.
@@ -706,7 +719,7 @@ cudaError_t launch_bwd_finish(const eaga_dims &d, const BwdArgs &a, const FastWs
     const int rows = d.B * d.n, ncol = 3 * HD + d.dx;
     float *bparts = reinterpret_cast<float *>(ws + W.bparts);
     const int seg_rows = (rows + W.bsplits - 1) / W.bsplits;
-    k_bias_partial<<<dim3((ncol + 255) / 256, W.bsplits), 256, 0, st>>>(
+    k_bias_partial<<<dim3(3 + (d.dx + 255) / 256, W.bsplits), 256, 0, st>>>(
         dQ, dK, dV, static_cast<const __nv_bfloat16 *>(a.dXout), a.M, rows, d.dx, seg_rows, bparts);
     float *r2 = reinterpret_cast<float *>(ws + W.r2);
     const int ctas = W.n_rparts, seg = (ctas + W.rsplits - 1) / W.rsplits;

@@ -174,10 +174,10 @@ __device__ __forceinline__ void warp_scores2(uint32_t chunk, int q, int t, int h
     }
 }
 
-// acc[hh][mt] = Z^T[d, chunk rows] P[chunk rows, 8 cols] for heads 2hq+hh: Z
+// acc[hh][mt] (+)= Z^T[d, chunk rows] P[chunk rows, 8 cols] for heads 2hq+hh: Z
 // from the warp's rows of a [32NR][256] swizzled chunk, P the warp's m16n8
 // fragment (entries 2,3 are ignored when NR = 1).
-template <int NR>
+template <int NR, bool ACC = false>
 __device__ __forceinline__ void warp_contract2(uint32_t chunk, int q, int t, int hq, const float (&pv)[2][4],
                                                float (&acc)[2][2][4]) {
     const int vrow = frag_row<NR>(q, t, (t >> 4) & 1);
@@ -188,7 +188,7 @@ __device__ __forceinline__ void warp_contract2(uint32_t chunk, int q, int t, int
         const uint32_t b1 = NR == 2 ? movmatrix_t(pack_bf16(pv[hh][2], pv[hh][3])) : 0u;
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
-            acc[hh][mt][0] = acc[hh][mt][1] = acc[hh][mt][2] = acc[hh][mt][3] = 0.f;
+            if (!ACC) acc[hh][mt][0] = acc[hh][mt][1] = acc[hh][mt][2] = acc[hh][mt][3] = 0.f;
             const int d0 = (2 * hq + hh) * DH + mt * 16;
             uint32_t a[4];
             ldsm_x4_t(chunk + (d0 >> 6) * (NR * 4096) + sw128(vrow, (d0 & 63) / 8 + vch), a);

@@ -1,27 +1,30 @@
 // Forward pair kernel for de = 64, H = 8, dh = 32, bf16 storage (sm_100a).
 //
-// One CTA owns the tile of 8 query rows i x 32NR key columns j of one graph
-// (NR = 1 for n <= 512, so two CTAs share an SM; NR = 2 above); the CTAs
-// that share the 8 rows form a thread-block cluster.  Each CTA loads its E
-// tile once with TMA and keeps it in shared memory for both passes of the
-// layer ("large graphs need two passes", AI-summary page, method paragraph):
+// One CTA owns 8 query rows i of one graph and streams the columns j of those
+// rows through shared memory in chunks of 32 (256 pairs: a 32 KB E tile, the
+// 16 KB K and V chunks), twice, as the layer's two passes ("large graphs need
+// two passes", AI-summary page, method paragraph):
 //   pass 1: FiLM coefficients f = E Wfe on the tensor cores (tcgen05, fp32 in
 //           TMEM), scores S = Q K^T with warp MMAs, s' = S(1+gamma)+beta,
-//           masked row max / sum over the CTA's columns;
-//   cluster exchange of the (max, sum) pairs through distributed shared
-//           memory gives every CTA the final softmax statistics;
-//   pass 2: normalised a, O partial = a V (warp MMAs), edge update
-//           dE = a We on the tensor cores, E' = E + dE written in place and
-//           stored with TMA; O partials summed over the warps and the cluster.
-// So E is read from HBM once and E' written once; the [B,H,n,n] map never
-// leaves the chip.
+//           running masked row max / sum per thread (online softmax);
+//   pass 2: the same f and s' again, normalised a, O += a V (warp MMAs), edge
+//           update dE = a We on the tensor cores, E' = E + dE written in place
+//           and stored with TMA.
+// Pass 2 walks the chunks in reverse, so the E tiles it reads again are the
+// ones pass 1 brought into L2 last: E leaves HBM once, E' is written once and
+// the [B,H,n,n] map never leaves the chip.  No CTA waits for another one.
+//
+// Pipeline: three stages of {E, K, V}; stage loads are issued two iterations
+// ahead (one thread, TMA, mbarrier transaction counts) and pass-1 E tiles are
+// prefetched into L2 further ahead; the E' stores drain while the next
+// iterations run.
 //
 // Pair <-> lane mapping.  The E tile is loaded as [s][j][ic][c] (i = 2ic+s)
-// so that the 128 rows of FiLM MMA e = (r,s) are the pairs
-// (j = 32r + 8q + t/4, i = 2(t%4) + s) of lane t in the warps of quadrant q:
-// the same pair those lanes hold in accumulator register e of their m16n8
-// score tile S^T[j,i].  TMEM lane 32q+t therefore feeds lane t directly.
-// 16 warps: warp W reads quadrant q = W%4 and handles heads 2(W/4), 2(W/4)+1.
+// so that the 128 rows of FiLM MMA s are the pairs (j = 8q + t/4,
+// i = 2(t%4) + s) of lane t in the warps of quadrant q: the same pair those
+// lanes hold in accumulator register s of their m16n8 score tile S^T[j,i].
+// TMEM lane 32q+t therefore feeds lane t directly.  16 warps: warp W reads
+// quadrant q = W%4 and handles heads 2(W/4), 2(W/4)+1.
 #include <math.h>
 #include "fast.h"
 #include "fast_common.cuh"
@@ -32,31 +35,28 @@ namespace fast {
 using namespace sm100;
 using namespace dev;
 
+constexpr int FS_STAGES = 3;        // pipeline stages of {E, K, V}
+constexpr int FS_PF = 4;            // extra pass-1 chunks prefetched into L2
+
 // shared memory map (bytes from a 1024-aligned base)
-template <int NR>
-struct FwdSmem {
-    static constexpr uint32_t E = 0;                          // E tile [s 2][j 32NR][ic 4][c 64], swizzled rows
-    static constexpr uint32_t K = NR * 32768;                 // K chunk: 4 boxes [j 32NR][d 64], swizzled
-    static constexpr uint32_t V = K + NR * 16384;             // V chunk, same layout
-    static constexpr uint32_t WFE = V + NR * 16384;           // Wfe^T [16][64] swizzled (FiLM B)
+struct FsSmem {
+    static constexpr uint32_t STAGE = 65536;                  // E [32 KB] | K [16 KB] | V [16 KB]
+    static constexpr uint32_t SE = 0, SK = 32768, SV = 49152;
+    static constexpr uint32_t WFE = FS_STAGES * STAGE;        // Wfe^T [16][64] swizzled (FiLM B)
     static constexpr uint32_t WE = WFE + 2048;                // We^T [64][16] no swizzle (edge-update B)
-    static constexpr uint32_t A = WE + 2048;                  // 2NR tiles [128][16] no swizzle (edge-update A)
-    static constexpr uint32_t WST = A + 2 * NR * 4096;        // per-quadrant stats [4][8 i][8 h][2] f32
-    static constexpr uint32_t CST = WST + 4 * 8 * 8 * 2 * 4;  // CTA stats [8][8][2] (read by peers)
-    static constexpr uint32_t FIN = CST + 8 * 8 * 2 * 4;      // final m, 1/l [8][8][2] (m, l before inversion)
-    static constexpr uint32_t G = FIN + 8 * 8 * 2 * 4;        // g_b [16]
-    static constexpr uint32_t MI = G + 64;                    // mask of the 8 rows
-    static constexpr uint32_t MJ = MI + 16;                   // mask of the 32NR columns
-    static constexpr uint32_t BAR = MJ + 64;                  // 6 mbarriers
-    static constexpr uint32_t TM = BAR + 48;                  // TMEM base address
-    static constexpr uint32_t RST = TM + 16;                  // received softmax stats [16][64][2] f32
-    static constexpr uint32_t RO = RST + RECV_ROWVALS_BYTES;  // received O partial slices
-    static constexpr uint32_t BYTES = RO + recv_rows_bytes(1) + 1024;   // + alignment slack
-    static constexpr uint32_t OPART = K;                      // 32 KB quadrant partials of O (K, V chunks are dead)
+    static constexpr uint32_t A = WE + 2048;                  // 2 tiles [128][16] no swizzle (edge-update A)
+    static constexpr uint32_t WST = A + 8192;                 // per-quadrant stats [4][8 i][8 h][2] f32
+    static constexpr uint32_t FIN = WST + 2048;               // final m, 1/l [8][8][2]
+    static constexpr uint32_t G = FIN + 512;                  // g_b [16]
+    static constexpr uint32_t MJ = G + 64;                    // mask of the graph's nodes [n <= 1024]
+    static constexpr uint32_t BAR = MJ + 1024;                // full[3], film, edge
+    static constexpr uint32_t TM = BAR + 8 * (FS_STAGES + 2); // TMEM base address
+    static constexpr uint32_t BYTES = TM + 16 + 1024;         // + alignment slack
+    static constexpr uint32_t OPART = 0;                      // [4][8][256] f32 O partials (stages dead)
 };
 
-constexpr uint32_t TM_COLS = 256;            // FiLM: cols 0..32NR-1; edge update: cols 64..191
-constexpr uint32_t TM_FILM = 0, TM_EDGE = 64;
+constexpr uint32_t FS_TM_COLS = 256;          // FiLM: cols 0..31; edge update: cols 64..191
+constexpr uint32_t FS_TM_FILM = 0, FS_TM_EDGE = 64;
 
 struct FwdParams {
     const __nv_bfloat16 *Q;
@@ -67,278 +67,300 @@ struct FwdParams {
     float *LSE;
     int *status;
     int n;
-    uint32_t prefetch_ahead;   // CTAs between this one and the one whose tiles it prefetches (0: none)
+    uint32_t prefetch_ahead;   // CTAs between this one and the one whose first tiles it prefetches
 };
 
-template <int NR>
-__global__ void __launch_bounds__(NTHR, NR == 1 ? 2 : 1)
-k_fwd_pairs(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmEo,
-            const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, FwdParams p) {
-    using S = FwdSmem<NR>;
-    constexpr int TCN = tile_cols(NR), NE = 2 * NR;
+__global__ void __launch_bounds__(NTHR, 1)
+k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmEo,
+             const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, FwdParams p) {
+    using S = FsSmem;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
     const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = W >> 2, t = tid & 31, c4 = t & 3, g8 = t >> 2;
-    const uint32_t rank = cluster_rank();
-    const uint32_t nclu = gridDim.x;
-    const int n = p.n;
-    const int j0 = blockIdx.x * TCN, i0 = blockIdx.y * TB, b = blockIdx.z;
-    const uint32_t bar_e = sbase + S::BAR, bar_kv = bar_e + 8, bar_film = bar_e + 16, bar_edge = bar_e + 24,
-                   bar_st = bar_e + 32, bar_o = bar_e + 40;
+    const int n = p.n, nch = (n + 31) / 32, nit = 2 * nch;
+    const int b = blockIdx.y, i0 = blockIdx.x * TB;
+    const uint32_t bar_full = sbase + S::BAR, bar_film = bar_full + 8 * FS_STAGES, bar_edge = bar_film + 8;
     float *g = reinterpret_cast<float *>(sp + S::G);
-    uint8_t *mi = sp + S::MI, *mj = sp + S::MJ;
+    uint8_t *mj = sp + S::MJ;
 
-    // ---------------- setup: barriers, TMA, TMEM, operands
-    if (tid == 0) {
-        mbar_init(bar_e, 1);
-        mbar_init(bar_kv, 1);
-        mbar_init(bar_film, 1);
-        mbar_init(bar_edge, 1);
-        mbar_init(bar_st, 1);
-        mbar_init(bar_o, 1);
-        fence_mbar_init();
-        mbar_expect_tx(bar_st, nclu * 64 * 8);
-        mbar_expect_tx(bar_o, nclu * rows_slice(1, nclu, rank) * 16);
-        mbar_expect_tx(bar_e, NR * 32768);
-        tma_load_5d(sbase + S::E, &tmE, bar_e, 0, i0 / 2, j0, 0, b);
-        mbar_expect_tx(bar_kv, NR * 32768);
+    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0
+    auto chunk_of = [&](int it) { return it < nch ? it : nit - 1 - it; };
+    auto issue_load = [&](int it) {
+        const int s = it % FS_STAGES, j0 = 32 * chunk_of(it);
+        const bool pass2 = it >= nch;
+        const uint32_t st = sbase + s * S::STAGE, bar = bar_full + 8 * s;
+        mbar_expect_tx(bar, pass2 ? 65536 : 49152);
+        tma_load_5d(st + S::SE, &tmE, bar, 0, i0 / 2, j0, 0, b);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            tma_load_3d(sbase + S::K + k * NR * 4096, &tmK, bar_kv, 64 * k, j0, b);
-            tma_load_3d(sbase + S::V + k * NR * 4096, &tmV, bar_kv, 64 * k, j0, b);
-        }        // L2 prefetch of the tiles of the CTA that runs about one wave later
-        const uint32_t cid = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x + p.prefetch_ahead;
-        if (p.prefetch_ahead && cid < gridDim.x * gridDim.y * gridDim.z) {
-            const int px = cid % gridDim.x, py = (cid / gridDim.x) % gridDim.y, pz = cid / (gridDim.x * gridDim.y);
-            tma_prefetch_5d(&tmE, 0, py * TB / 2, px * TCN, 0, pz);
-            if (py == 0)
-                for (int k = 0; k < 4; ++k) {
-                    tma_prefetch_3d(&tmK, 64 * k, px * TCN, pz);
-                    tma_prefetch_3d(&tmV, 64 * k, px * TCN, pz);
-                }
+            tma_load_3d(st + S::SK + k * 4096, &tmK, bar, 64 * k, j0, b);
+            if (pass2) tma_load_3d(st + S::SV + k * 4096, &tmV, bar, 64 * k, j0, b);
         }
+    };
+
+    // ---------------- setup: barriers, first loads, TMEM, operands
+    if (tid == 0) {
+        for (int s = 0; s < FS_STAGES; ++s) mbar_init(bar_full + 8 * s, 1);
+        mbar_init(bar_film, 1);
+        mbar_init(bar_edge, 1);
+        fence_mbar_init();
+        issue_load(0);
+        issue_load(1);
+        for (int c = 2; c < nch && c < 2 + FS_PF; ++c) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * c, 0, b);
     }
     if (W == 0) {
-        tmem_alloc(sbase + S::TM, TM_COLS);
+        tmem_alloc(sbase + S::TM, FS_TM_COLS);
         tmem_relinquish();
     }
     // operand images: Wfe^T (FiLM B, swizzled) and We^T (edge-update B, no swizzle), 2 KB each
     if (tid < 256) reinterpret_cast<uint4 *>(sp + S::WFE)[tid] = reinterpret_cast<const uint4 *>(p.img)[tid];
     // edge-update A tiles: zero (the K half h >= 8 stays zero)
-    for (int e = tid; e < NE * 4096 / 16; e += NTHR) reinterpret_cast<uint4 *>(sp + S::A)[e] = make_uint4(0, 0, 0, 0);
+    for (int e = tid; e < 8192 / 16; e += NTHR) reinterpret_cast<uint4 *>(sp + S::A)[e] = make_uint4(0, 0, 0, 0);
     if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
-    if (tid >= 32 && tid < 32 + TB) mi[tid - 32] = (i0 + tid - 32 < n) ? p.M[(size_t)b * n + i0 + tid - 32] : 0;
-    if (tid >= 64 && tid < 64 + TCN) mj[tid - 64] = (j0 + tid - 64 < n) ? p.M[(size_t)b * n + j0 + tid - 64] : 0;
+    for (int j = tid; j < 32 * nch; j += NTHR) mj[j] = j < n ? p.M[(size_t)b * n + j] : 0;
     uint32_t qf[2][2][2];
     load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
+    // the thread's two rows i = i0 + 2c4 + s (s = 0, 1)
+    const bool mrow[2] = {i0 + 2 * c4 < n && p.M[(size_t)b * n + i0 + 2 * c4] != 0,
+                          i0 + 2 * c4 + 1 < n && p.M[(size_t)b * n + i0 + 2 * c4 + 1] != 0};
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
     const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
-    cluster_arrive();   // receive barriers of this CTA are armed
-
-    // ---------------- pass 1a: FiLM on the tensor cores (one thread issues)
-    if (tid == 0) {
-        if (!mbar_wait(bar_e, 0)) flag_timeout(p.status);
-        tc_fence_after();
-        issue_pair_products<NR>(sbase + S::E, sbase + S::WFE, tmem + TM_FILM);
-        mma_commit(bar_film);
-    }
-    __syncwarp();
-
-    // ---------------- pass 1b: scores S^T = K Q^T on warp MMAs (2 heads per warp)
-    if (!mbar_wait(bar_kv, 0)) flag_timeout(p.status);
-    float sacc[2][4];
-    warp_scores2<NR>(sbase + S::K, q, t, hq, qf, sacc);
-
-    // ---------------- combine with FiLM: s' = s(1+gamma)+beta, masked
-    if (!mbar_wait(bar_film, 0)) flag_timeout(p.status);
-    tc_fence_after();
     const float rs = rsqrtf((float)DH);
-    bool valid[4] = {false, false, false, false};
-#pragma unroll
-    for (int e = 0; e < NE; ++e) {
-        const int jl = 32 * (e >> 1) + 8 * q + g8, il = 2 * c4 + (e & 1);
-        valid[e] = mi[il] && mj[jl];
-        float gm[2], bt[2];
-        tmem_ld2(tl + TM_FILM + 16 * e + 2 * hq, gm[0], gm[1]);
-        tmem_ld2(tl + TM_FILM + 16 * e + NH + 2 * hq, bt[0], bt[1]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int h = 2 * hq + hh;
-            const float gam = gm[hh] + g[h], bet = bt[hh] + g[NH + h];
-            const float sv = sacc[hh][e] * rs * (1.f + gam) + bet;
-            sacc[hh][e] = valid[e] ? sv : -INFINITY;
-        }
-    }
+    const uint32_t L = 32 * q + t;
+    const uint32_t idesc_e = idesc_bf16_f32(128, DE);
 
-    // ---------------- row statistics: warp, CTA, cluster
-    float *wst = reinterpret_cast<float *>(sp + S::WST);
-    float *cst = reinterpret_cast<float *>(sp + S::CST);
-    float *fin = reinterpret_cast<float *>(sp + S::FIN);
+    float rm[2][2], rl[2][2];               // running max / sum [s][hh]
+    float fm[2][2], fl[2][2];               // final max, 1/sum [s][hh]
+    float oacc[2][2][4];
 #pragma unroll
     for (int s = 0; s < 2; ++s)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            float m = NR == 2 ? fmaxf(sacc[hh][s], sacc[hh][2 + s]) : sacc[hh][s];
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-            float l = 0.f;
-            if (m != -INFINITY) {
-                l = exp2f((sacc[hh][s] - m) * LOG2E);
-                if (NR == 2) l += exp2f((sacc[hh][2 + s] - m) * LOG2E);
+            rm[s][hh] = -INFINITY;
+            rl[s][hh] = 0.f;
+            fm[s][hh] = -INFINITY;
+            fl[s][hh] = 0.f;
+        }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) oacc[hh][mt][x] = 0.f;
+
+    for (int it = 0; it < nit; ++it) {
+        const int s = it % FS_STAGES, j0 = 32 * chunk_of(it);
+        const bool pass2 = it >= nch;
+        const uint32_t st = sbase + s * S::STAGE;
+        const uint32_t full_ph = (it / FS_STAGES) & 1;
+
+        if (it == nch) {
+            // ---------------- end of pass 1: statistics over lanes, then quadrants
+            float *wst = reinterpret_cast<float *>(sp + S::WST);
+            float *fin = reinterpret_cast<float *>(sp + S::FIN);
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float m = rm[s2][hh], l = rl[s2][hh];
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) {
+                        const float mo = __shfl_xor_sync(0xffffffffu, m, o), lo = __shfl_xor_sync(0xffffffffu, l, o);
+                        const float mn = fmaxf(m, mo);
+                        l = (mn == -INFINITY) ? 0.f
+                                              : l * exp2f((m - mn) * LOG2E) + lo * exp2f((mo - mn) * LOG2E);
+                        m = mn;
+                    }
+                    if (g8 == 0) {
+                        const int il = 2 * c4 + s2, h = 2 * hq + hh;
+                        wst[((q * 8 + il) * 8 + h) * 2 + 0] = m;
+                        wst[((q * 8 + il) * 8 + h) * 2 + 1] = l;
+                    }
+                }
+            __syncthreads();
+            if (tid < 64) {
+                float m = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) m = fmaxf(m, wst[(k * 64 + tid) * 2]);
+                float l = 0.f;
+                if (m != -INFINITY)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float mk = wst[(k * 64 + tid) * 2];
+                        if (mk != -INFINITY) l += wst[(k * 64 + tid) * 2 + 1] * exp2f((mk - m) * LOG2E);
+                    }
+                fin[tid * 2] = m;
+                fin[tid * 2 + 1] = (l > 0.f) ? 1.f / l : 0.f;
+                const int il = tid >> 3, h = tid & 7;
+                if (i0 + il < n)
+                    p.LSE[((size_t)b * NH + h) * n + i0 + il] = (m == -INFINITY) ? -INFINITY : m + logf(l);
             }
-            l += __shfl_xor_sync(0xffffffffu, l, 4);
-            l += __shfl_xor_sync(0xffffffffu, l, 8);
-            l += __shfl_xor_sync(0xffffffffu, l, 16);
-            if (g8 == 0) {
-                const int il = 2 * c4 + s, h = 2 * hq + hh;
-                wst[((q * 8 + il) * 8 + h) * 2 + 0] = m;
-                wst[((q * 8 + il) * 8 + h) * 2 + 1] = l;
+            __syncthreads();
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int il = 2 * c4 + s2, h = 2 * hq + hh;
+                    fm[s2][hh] = fin[(il * 8 + h) * 2];
+                    fl[s2][hh] = fin[(il * 8 + h) * 2 + 1];
+                }
+            // L2 prefetch of the first tiles of the CTA that runs about one wave later
+            if (tid == 0 && p.prefetch_ahead) {
+                const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
+                if (cid < gridDim.x * gridDim.y) {
+                    const int prb = cid % gridDim.x, pb = cid / gridDim.x;
+                    for (int cc = 0; cc < nch && cc < 2; ++cc)
+                        tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
+                }
             }
         }
-    __syncthreads();
-    if (tid < 64) {
-        float m = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) m = fmaxf(m, wst[(k * 64 + tid) * 2]);
-        float l = 0.f;
-        if (m != -INFINITY)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float mk = wst[(k * 64 + tid) * 2];
-                if (mk != -INFINITY) l += wst[(k * 64 + tid) * 2 + 1] * exp2f((mk - m) * LOG2E);
-            }
-        cst[tid * 2] = m;
-        cst[tid * 2 + 1] = l;
-    }
-    __syncthreads();
-    cluster_wait();     // every peer's receive barriers are armed
-    push_rowvals(sp, sbase, S::CST, S::RST, bar_st, tid, rank, nclu);
-    if (!mbar_wait(bar_st, 0)) flag_timeout(p.status);
-    combine_rowvals<0>(sp, S::RST, S::FIN, tid, nclu);
-    __syncthreads();
-    if (tid < 64) {
-        const float m = fin[tid * 2], l = fin[tid * 2 + 1];
-        fin[tid * 2 + 1] = (l > 0.f) ? 1.f / l : 0.f;
-        const int il = tid >> 3, h = tid & 7;
-        if (rank == 0 && i0 + il < n)
-            p.LSE[((size_t)b * NH + h) * n + i0 + il] = (m == -INFINITY) ? -INFINITY : m + logf(l);
-    }
-    __syncthreads();
 
-    // ---------------- pass 2: normalised coefficients
-    const uint32_t L = 32 * q + t;
+        // ---------------- FiLM on the tensor cores (one thread issues)
+        if (tid == 0) {
+            if (!mbar_wait(bar_full + 8 * s, full_ph)) flag_timeout(p.status);
+            tc_fence_after();
+            issue_pair_products<1>(st + S::SE, sbase + S::WFE, tmem + FS_TM_FILM);
+            mma_commit(bar_film);
+            if (!pass2 && it + 2 + FS_PF < nch) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (it + 2 + FS_PF), 0, b);
+        }
+        __syncwarp();
+
+        // ---------------- scores S^T = K Q^T on warp MMAs (2 heads per warp)
+        if (!mbar_wait(bar_full + 8 * s, full_ph)) flag_timeout(p.status);
+        float sacc[2][4];
+        warp_scores2<1>(st + S::SK, q, t, hq, qf, sacc);
+
+        // ---------------- combine with FiLM: s' = s(1+gamma)+beta, masked
+        if (!mbar_wait(bar_film, it & 1)) flag_timeout(p.status);
+        tc_fence_after();
+        const bool mcol = mj[j0 + 8 * q + g8] != 0;
+        bool valid[2];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        if (e >= NE) {
-            sacc[0][e] = sacc[1][e] = 0.f;
+        for (int e = 0; e < 2; ++e) {
+            valid[e] = mcol && mrow[e];
+            float gm[2], bt[2];
+            tmem_ld2(tl + FS_TM_FILM + 16 * e + 2 * hq, gm[0], gm[1]);
+            tmem_ld2(tl + FS_TM_FILM + 16 * e + NH + 2 * hq, bt[0], bt[1]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int h = 2 * hq + hh;
+                const float gam = gm[hh] + g[h], bet = bt[hh] + g[NH + h];
+                const float sv = sacc[hh][e] * rs * (1.f + gam) + bet;
+                sacc[hh][e] = valid[e] ? sv : -INFINITY;
+            }
+        }
+
+        if (!pass2) {
+            // running statistics (online softmax): one value per (row, head) and chunk
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const float x = sacc[hh][e];
+                    const float mn = fmaxf(rm[e][hh], x);
+                    if (mn != -INFINITY) {
+                        rl[e][hh] = rl[e][hh] * exp2f((rm[e][hh] - mn) * LOG2E) + exp2f((x - mn) * LOG2E);
+                        rm[e][hh] = mn;
+                    }
+                }
+            tc_fence_before();
+            __syncthreads();   // stage s and the FiLM columns are free again
+            if (tid == 0 && it + 2 < nit) issue_load(it + 2);
             continue;
         }
-        const int il = 2 * c4 + (e & 1);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int h = 2 * hq + hh;
-            const float m = fin[(il * 8 + h) * 2], linv = fin[(il * 8 + h) * 2 + 1];
-            sacc[hh][e] = valid[e] ? exp2f((sacc[hh][e] - m) * LOG2E) * linv : 0.f;
-        }
-        // edge-update A operand: row 32q+t of tile e, heads 2hq, 2hq+1
-        *reinterpret_cast<uint32_t *>(sp + S::A + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(sacc[0][e], sacc[1][e]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    const uint32_t idesc_e = idesc_bf16_f32(128, DE);
-    if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-            mma_bf16_ss(tmem + TM_EDGE + 64 * e, smem_desc(sbase + S::A + e * 4096, 128, 256, LAYOUT_NONE),
-                        smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
-        mma_commit(bar_edge);
-    }
-    __syncwarp();
 
-    // ---------------- O partial = a V on warp MMAs (overlaps the edge MMAs)
-    float oacc[2][2][4];
-    warp_contract2<NR>(sbase + S::V, q, t, hq, sacc, oacc);
-
-    // ---------------- E' = E + a We, NR rounds of two MMA tiles
-    if (!mbar_wait(bar_e, 0)) flag_timeout(p.status);
-    for (int round = 0; round < NR; ++round) {
-        if (!mbar_wait(bar_edge, round)) flag_timeout(p.status);
-        tc_fence_after();
+        // ---------------- pass 2: normalised coefficients, edge-update A operand
 #pragma unroll
-        for (int ee = 0; ee < 2; ++ee) {
-            const int e = 2 * round + ee;
-            float dv[16];
-            tmem_ld16(tl + TM_EDGE + 64 * ee + 16 * hq, dv);
-            tmem_ld_wait();
-            add_residual16(sp + S::E + tile_off<NR>(e) + L * 128, L, hq, dv);
+        for (int e = 0; e < 2; ++e) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                sacc[hh][e] = valid[e] ? exp2f((sacc[hh][e] - fm[e][hh]) * LOG2E) * fl[e][hh] : 0.f;
+            *reinterpret_cast<uint32_t *>(sp + S::A + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(sacc[0][e], sacc[1][e]);
         }
-        if (round + 1 < NR) {
-            tc_fence_before();
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
+        sacc[0][2] = sacc[0][3] = sacc[1][2] = sacc[1][3] = 0.f;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
 #pragma unroll
-                for (int ee = 0; ee < 2; ++ee)
-                    mma_bf16_ss(tmem + TM_EDGE + 64 * ee,
-                                smem_desc(sbase + S::A + (2 * (round + 1) + ee) * 4096, 128, 256, LAYOUT_NONE),
-                                smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
-                mma_commit(bar_edge);
+            for (int e = 0; e < 2; ++e)
+                mma_bf16_ss(tmem + FS_TM_EDGE + 64 * e, smem_desc(sbase + S::A + e * 4096, 128, 256, LAYOUT_NONE),
+                            smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
+            mma_commit(bar_edge);
+            // stage (it+2) % 3 held iteration it-1, whose E' store may still be reading it
+            if (it + 2 < nit) {
+                tma_store_wait_read0();
+                issue_load(it + 2);
             }
-            __syncwarp();
+        }
+        __syncwarp();
+
+        // ---------------- O += a V on warp MMAs (overlaps the edge MMAs)
+        warp_contract2<1, true>(st + S::SV, q, t, hq, sacc, oacc);
+
+        // ---------------- E' = E + a We, in place, then TMA store
+        if (!mbar_wait(bar_edge, (it - nch) & 1)) flag_timeout(p.status);
+        tc_fence_after();
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float dv[16];
+            tmem_ld16(tl + FS_TM_EDGE + 64 * e + 16 * hq, dv);
+            tmem_ld_wait();
+            add_residual16(sp + (st - sbase) + S::SE + tile_off<1>(e) + L * 128, L, hq, dv);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_5d(&tmEo, st + S::SE, 0, i0 / 2, j0, 0, b);
+            tma_store_commit();
         }
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-        tma_store_5d(&tmEo, sbase + S::E, 0, i0 / 2, j0, 0, b);
-        tma_store_commit();
-    }
 
-    // ---------------- O: sum over the quadrant warps and the cluster
+    // ---------------- O: sum over the quadrant warps
+    if (tid == 0) tma_store_wait_read0();
+    __syncthreads();   // every stage is free
     store_quadrant_part(sp, S::OPART, oacc, q, hq, t);
     __syncthreads();
     {
-        const uint32_t parts[1] = {S::OPART};
-        push_rows_partials<1>(sp, sbase, parts, S::RO, bar_o, tid, rank, nclu);
-        if (!mbar_wait(bar_o, 0)) flag_timeout(p.status);
-        __nv_bfloat16 *const outs[1] = {p.O};
-        const float sc[1] = {1.f};
-        finish_rows_partials<1>(sp, S::RO, tid, rank, nclu, outs, b, n, i0, sc);
+        const float *part = reinterpret_cast<const float *>(sp + S::OPART);
+        for (int x = tid; x < TB * HD / 2; x += NTHR) {
+            const int il = (2 * x) / HD, d = (2 * x) % HD;
+            if (i0 + il >= n) continue;
+            float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                o0 += part[k * TB * HD + il * HD + d];
+                o1 += part[k * TB * HD + il * HD + d + 1];
+            }
+            *reinterpret_cast<uint32_t *>(p.O + ((size_t)b * n + i0 + il) * HD + d) = pack_bf16(o0, o1);
+        }
     }
-    if (tid == 0) tma_store_wait_read0();
     tc_fence_before();
     __syncthreads();
-    if (W == 0) tmem_dealloc(tmem, TM_COLS);
+    if (W == 0) tmem_dealloc(tmem, FS_TM_COLS);
 }
 
 // ------------------------------------------------------------------ host side
 
-template <int NR>
-static cudaError_t launch_fwd_nr(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
-                                 cudaStream_t st) {
-    constexpr int TCN = tile_cols(NR);
+cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
+                             cudaStream_t st) {
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_fwd_pairs<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             FwdSmem<NR>::BYTES);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(k_fwd_pairs<NR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        cudaError_t e = cudaFuncSetAttribute(k_fwd_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, FsSmem::BYTES);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
     CUtensorMap mE, mEo, mK, mV;
-    if (!encode_pair_map(&mE, a.E, d.B, d.n, false, TCN) || !encode_pair_map(&mEo, a.Eout, d.B, d.n, false, TCN) ||
-        !encode_node_map(&mK, a.K, d.B, d.n, TCN) || !encode_node_map(&mV, a.V, d.B, d.n, TCN))
+    if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32) || !encode_pair_map(&mEo, a.Eout, d.B, d.n, false, 32) ||
+        !encode_node_map(&mK, a.K, d.B, d.n, 32) || !encode_node_map(&mV, a.V, d.B, d.n, 32))
         return cudaErrorInvalidValue;
     FwdParams p;
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
@@ -349,26 +371,9 @@ static cudaError_t launch_fwd_nr(const eaga_dims &d, const FwdArgs &a, const uin
     p.LSE = a.LSE;
     p.status = a.status;
     p.n = d.n;
-    p.prefetch_ahead = (uint32_t)(sm_count() * (NR == 1 ? 2 : 1));
-    const int nc = (d.n + TCN - 1) / TCN;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(nc, (d.n + TB - 1) / TB, d.B);
-    cfg.blockDim = dim3(NTHR);
-    cfg.dynamicSmemBytes = FwdSmem<NR>::BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = nc;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_fwd_pairs<NR>, mE, mEo, mK, mV, p);
-}
-
-cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
-                             cudaStream_t st) {
-    return pick_nr(d.n) == 1 ? launch_fwd_nr<1>(d, a, img, g, st) : launch_fwd_nr<2>(d, a, img, g, st);
+    p.prefetch_ahead = (uint32_t)sm_count();
+    k_fwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), NTHR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
+    return cudaGetLastError();
 }
 
 }  // namespace fast

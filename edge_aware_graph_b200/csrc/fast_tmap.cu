@@ -119,49 +119,82 @@ cudaError_t launch_weight_images(const eaga_dims &d, const void *const w[12], ui
     return cudaGetLastError();
 }
 
-// g_b = y_b Wfy + bf (fp32) for every graph, and (block 0) the four operand images.
-__global__ void k_prologue(const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy, const __nv_bfloat16 *bf,
-                           const __nv_bfloat16 *Wfe, const __nv_bfloat16 *We, float *g, uint8_t *img, int B,
-                           int dy) {
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t < B * NF) {
-        const int b = t / NF, k = t % NF;
-        float acc = __bfloat162float(bf[k]);
-        for (int c = 0; c < dy; ++c)
-            acc = fmaf(__bfloat162float(y[(size_t)b * dy + c]), __bfloat162float(Wfy[c * NF + k]), acc);
-        g[t] = acc;
+// g_b = y_b Wfy + bf (fp32) for every graph: one warp per graph, lanes split
+// the dy terms and add their 16 sums with shuffles in a fixed order.  The last
+// block writes the four operand images from Wfe and We staged in shared memory.
+__global__ void __launch_bounds__(256) k_prologue(const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy,
+                                                  const __nv_bfloat16 *bf, const __nv_bfloat16 *Wfe,
+                                                  const __nv_bfloat16 *We, float *g, uint8_t *img, int B, int dy) {
+    const int w = threadIdx.x >> 5, t = threadIdx.x & 31;
+    if (blockIdx.x + 1 < gridDim.x) {
+        const int b = blockIdx.x * 8 + w;
+        if (b >= B) return;
+        float acc[NF];
+#pragma unroll
+        for (int k = 0; k < NF; ++k) acc[k] = 0.f;
+        for (int c = t; c < dy; c += 32) {
+            const float yc = __bfloat162float(y[(size_t)b * dy + c]);
+            const uint4 *wr = reinterpret_cast<const uint4 *>(Wfy + (size_t)c * NF);
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                const uint4 v = wr[hlf];
+                const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float2 f = __bfloat1622float2(v2[u]);
+                    acc[8 * hlf + 2 * u] = fmaf(yc, f.x, acc[8 * hlf + 2 * u]);
+                    acc[8 * hlf + 2 * u + 1] = fmaf(yc, f.y, acc[8 * hlf + 2 * u + 1]);
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < NF; ++k)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
+        if (t < NF) {
+            float v = acc[0];
+#pragma unroll
+            for (int k = 1; k < NF; ++k) v = t == k ? acc[k] : v;
+            g[(size_t)b * NF + t] = v + __bfloat162float(bf[t]);
+        }
+        return;
     }
-    if (blockIdx.x != 0) return;
+    __shared__ __nv_bfloat16 sWfe[DE * NF], sWe[NH * DE];
+    for (int e = threadIdx.x; e < DE * NF / 8; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sWfe)[e] = reinterpret_cast<const uint4 *>(Wfe)[e];
+    for (int e = threadIdx.x; e < NH * DE / 8; e += blockDim.x)
+        reinterpret_cast<uint4 *>(sWe)[e] = reinterpret_cast<const uint4 *>(We)[e];
+    __syncthreads();
     const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
     for (int e = threadIdx.x; e < NF * DE; e += blockDim.x) {
         // IMG_WFE_T_SW: row k (16), element c (64)
         {
             const int k = e / DE, c = e % DE;
-            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WFE_T_SW + sw128(k, c >> 3) + (c & 7) * 2) = Wfe[c * NF + k];
+            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WFE_T_SW + sw128(k, c >> 3) + (c & 7) * 2) = sWfe[c * NF + k];
         }
         // IMG_WE_SW: row h (16, zero for h >= 8), element c
         {
             const int h = e / DE, c = e % DE;
             *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WE_SW + sw128(h, c >> 3) + (c & 7) * 2) =
-                h < NH ? We[h * DE + c] : zero;
+                h < NH ? sWe[h * DE + c] : zero;
         }
         // IMG_WE_T_NS: row c (64), element h (16, zero for h >= 8)
         {
             const int c = e / NF, h = e % NF;
-            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WE_T_NS + ns16(c, h)) = h < NH ? We[h * DE + c] : zero;
+            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WE_T_NS + ns16(c, h)) = h < NH ? sWe[h * DE + c] : zero;
         }
         // IMG_WFE_NS: row c (64), element k (16)
         {
             const int c = e / NF, k = e % NF;
-            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WFE_NS + ns16(c, k)) = Wfe[c * NF + k];
+            *reinterpret_cast<__nv_bfloat16 *>(img + IMG_WFE_NS + ns16(c, k)) = sWfe[c * NF + k];
         }
     }
 }
 
 cudaError_t launch_prologue(const eaga_dims &d, const void *const w[12], const void *y, float *g, uint8_t *img,
                             cudaStream_t st) {
-    const int threads = 256, blocks = (d.B * NF + threads - 1) / threads;
-    k_prologue<<<blocks, threads, 0, st>>>(
+    const int blocks = (d.B + 7) / 8 + 1;
+    k_prologue<<<blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16 *>(y), static_cast<const __nv_bfloat16 *>(w[7]),
         static_cast<const __nv_bfloat16 *>(w[8]), static_cast<const __nv_bfloat16 *>(w[6]),
         static_cast<const __nv_bfloat16 *>(w[9]), g, img, d.B, d.dy);
