@@ -1,9 +1,9 @@
 // Forward pair kernel for de = 64, H = 8, dh = 32, bf16 storage (sm_100a).
 //
 // One CTA owns 8 query rows i of one graph and streams the columns j of those
-// rows through shared memory in chunks of 32 (256 pairs: a 32 KB E tile, the
-// 16 KB K and V chunks), twice, as the layer's two passes ("large graphs need
-// two passes", AI-summary page, method paragraph):
+// rows through shared memory in chunks of 32 (256 pairs: two 16 KB E tiles,
+// the 16 KB K and V chunks), twice, as the layer's two passes ("large graphs
+// need two passes", AI-summary page, method paragraph):
 //   pass 1: FiLM coefficients f = E Wfe on the tensor cores (tcgen05, fp32 in
 //           TMEM), scores S = Q K^T with warp MMAs, s' = S(1+gamma)+beta,
 //           running masked row max / sum per thread (online softmax);
@@ -14,16 +14,18 @@
 // ones pass 1 brought into L2 last: E leaves HBM once, E' is written once and
 // the [B,H,n,n] map never leaves the chip.  No CTA waits for another one.
 //
-// Pipeline: three stages of {E, K, V}; stage loads are issued two iterations
-// ahead (one thread, TMA, mbarrier transaction counts) and pass-1 E tiles are
-// prefetched into L2 further ahead; the E' stores drain while the next
-// iterations run.
+// Warp roles.  Warps 0..15 compute.  Warp 17 (one thread) keeps a ring of
+// twelve 16 KB shared-memory slots filled with TMA loads (3 slots per pass-1
+// chunk, 4 per pass-2 chunk, so up to four chunks ahead) and stores E' once
+// the compute warps have written it.  Warp 16 (one thread) issues the FiLM
+// MMAs one chunk ahead into a double-buffered TMEM range and the edge-update
+// MMAs once the compute warps have written a.  They meet only on mbarriers.
 //
-// Pair <-> lane mapping.  The E tile is loaded as [s][j][ic][c] (i = 2ic+s)
-// so that the 128 rows of FiLM MMA s are the pairs (j = 8q + t/4,
+// Pair <-> lane mapping.  E tile s (i = 2ic + s) is loaded as [j][ic][c] so
+// that its 128 rows, the M rows of FiLM MMA s, are the pairs (j = 8q + t/4,
 // i = 2(t%4) + s) of lane t in the warps of quadrant q: the same pair those
 // lanes hold in accumulator register s of their m16n8 score tile S^T[j,i].
-// TMEM lane 32q+t therefore feeds lane t directly.  16 warps: warp W reads
+// TMEM lane 32q+t therefore feeds lane t directly.  Compute warp W reads
 // quadrant q = W%4 and handles heads 2(W/4), 2(W/4)+1.
 #include <math.h>
 #include "fast.h"
@@ -35,28 +37,35 @@ namespace fast {
 using namespace sm100;
 using namespace dev;
 
-constexpr int FS_STAGES = 3;        // pipeline stages of {E, K, V}
-constexpr int FS_PF = 4;            // extra pass-1 chunks prefetched into L2
+constexpr int FS_SLOTS = 12;              // 16 KB slots of the load ring
+constexpr uint32_t FS_SLOT = 16384;
+constexpr int FS_NFULL = 4;               // load barriers (at most four chunks in flight)
+constexpr int FS_PF = 4;                  // pass-1 chunks prefetched into L2 beyond the loads
+constexpr int FS_THR = NTHR + 64;         // 16 compute warps, the MMA warp, the TMA warp
 
 // shared memory map (bytes from a 1024-aligned base)
 struct FsSmem {
-    static constexpr uint32_t STAGE = 65536;                  // E [32 KB] | K [16 KB] | V [16 KB]
-    static constexpr uint32_t SE = 0, SK = 32768, SV = 49152;
-    static constexpr uint32_t WFE = FS_STAGES * STAGE;        // Wfe^T [16][64] swizzled (FiLM B)
+    static constexpr uint32_t WFE = FS_SLOTS * FS_SLOT;       // Wfe^T [16][64] swizzled (FiLM B)
     static constexpr uint32_t WE = WFE + 2048;                // We^T [64][16] no swizzle (edge-update B)
     static constexpr uint32_t A = WE + 2048;                  // 2 tiles [128][16] no swizzle (edge-update A)
     static constexpr uint32_t WST = A + 8192;                 // per-quadrant stats [4][8 i][8 h][2] f32
     static constexpr uint32_t FIN = WST + 2048;               // final m, 1/l [8][8][2]
     static constexpr uint32_t G = FIN + 512;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // mask of the graph's nodes [n <= 1024]
-    static constexpr uint32_t BAR = MJ + 1024;                // full[3], film, edge
-    static constexpr uint32_t TM = BAR + 8 * (FS_STAGES + 2); // TMEM base address
+    static constexpr uint32_t BAR = MJ + 1024;                // mbarriers, see below
+    static constexpr uint32_t TM = BAR + 8 * 12;              // TMEM base address
     static constexpr uint32_t BYTES = TM + 16 + 1024;         // + alignment slack
-    static constexpr uint32_t OPART = 0;                      // [4][8][256] f32 O partials (stages dead)
+    static constexpr uint32_t OPART = 0;                      // [4][8][256] f32 O partials (ring drained)
 };
+// mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full, edge_full, stage_done[2]
+constexpr int FB_FULL = 0, FB_FILM_FULL = 4, FB_FILM_EMPTY = 6, FB_A_FULL = 8, FB_EDGE_FULL = 9,
+              FB_STAGE_DONE = 10;
 
-constexpr uint32_t FS_TM_COLS = 256;          // FiLM: cols 0..31; edge update: cols 64..191
-constexpr uint32_t FS_TM_FILM = 0, FS_TM_EDGE = 64;
+// TMEM columns: FiLM 0..63 (two buffers), edge update 64..191, pass-1 scores
+// from 192 on (16 per chunk, kept when nch <= 20 so pass 2 needs no K)
+constexpr uint32_t FS_TM_COLS = 512;
+constexpr uint32_t FS_TM_FILM = 0, FS_TM_EDGE = 64, FS_TM_S = 192;
+constexpr int FS_KEEP_S_MAX_CHUNKS = (512 - 192) / 16;
 
 struct FwdParams {
     const __nv_bfloat16 *Q;
@@ -70,44 +79,43 @@ struct FwdParams {
     uint32_t prefetch_ahead;   // CTAs between this one and the one whose first tiles it prefetches
 };
 
-__global__ void __launch_bounds__(NTHR, 1)
+__global__ void __launch_bounds__(FS_THR, 1)
 k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmEo,
              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, FwdParams p) {
     using S = FsSmem;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
-    const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = W >> 2, t = tid & 31, c4 = t & 3, g8 = t >> 2;
+    const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = (W >> 2) & 3, t = tid & 31, c4 = t & 3, g8 = t >> 2;
     const int n = p.n, nch = (n + 31) / 32, nit = 2 * nch;
     const int b = blockIdx.y, i0 = blockIdx.x * TB;
-    const uint32_t bar_full = sbase + S::BAR, bar_film = bar_full + 8 * FS_STAGES, bar_edge = bar_film + 8;
+    const uint32_t bars = sbase + S::BAR;
+    auto bar = [&](int k) { return bars + 8 * k; };
     float *g = reinterpret_cast<float *>(sp + S::G);
     uint8_t *mj = sp + S::MJ;
 
-    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0
+    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0.  Its
+    // slots, from slot_base(it) on: pass 1 E(s=0), E(s=1), K; pass 2 E(s=0),
+    // E(s=1), V when the pass-1 scores stay in TMEM, else E, E, K, V.
+    const bool keep_s = nch <= FS_KEEP_S_MAX_CHUNKS;
+    const int ns2 = keep_s ? 3 : 4, vslot = ns2 - 1;
     auto chunk_of = [&](int it) { return it < nch ? it : nit - 1 - it; };
-    auto issue_load = [&](int it) {
-        const int s = it % FS_STAGES, j0 = 32 * chunk_of(it);
-        const bool pass2 = it >= nch;
-        const uint32_t st = sbase + s * S::STAGE, bar = bar_full + 8 * s;
-        mbar_expect_tx(bar, pass2 ? 65536 : 49152);
-        tma_load_5d(st + S::SE, &tmE, bar, 0, i0 / 2, j0, 0, b);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            tma_load_3d(st + S::SK + k * 4096, &tmK, bar, 64 * k, j0, b);
-            if (pass2) tma_load_3d(st + S::SV + k * 4096, &tmV, bar, 64 * k, j0, b);
-        }
-    };
+    auto nslots = [&](int it) { return it < nch ? 3 : ns2; };
+    auto slot_base = [&](int it) { return (3 * min(it, nch) + ns2 * max(it - nch, 0)) % FS_SLOTS; };
+    auto slot_addr = [&](int it, int k) { return sbase + (uint32_t)((slot_base(it) + k) % FS_SLOTS) * FS_SLOT; };
 
-    // ---------------- setup: barriers, first loads, TMEM, operands
+    // ---------------- setup: barriers, TMEM, operands
     if (tid == 0) {
-        for (int s = 0; s < FS_STAGES; ++s) mbar_init(bar_full + 8 * s, 1);
-        mbar_init(bar_film, 1);
-        mbar_init(bar_edge, 1);
+        for (int k = 0; k < FB_FILM_FULL; ++k) mbar_init(bar(FB_FULL + k), 1);
+        mbar_init(bar(FB_FILM_FULL), 1);
+        mbar_init(bar(FB_FILM_FULL + 1), 1);
+        mbar_init(bar(FB_FILM_EMPTY), NWARP);
+        mbar_init(bar(FB_FILM_EMPTY + 1), NWARP);
+        mbar_init(bar(FB_A_FULL), NWARP);
+        mbar_init(bar(FB_EDGE_FULL), 1);
+        mbar_init(bar(FB_STAGE_DONE), NWARP);
+        mbar_init(bar(FB_STAGE_DONE + 1), NWARP);
         fence_mbar_init();
-        issue_load(0);
-        issue_load(1);
-        for (int c = 2; c < nch && c < 2 + FS_PF; ++c) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * c, 0, b);
     }
     if (W == 0) {
         tmem_alloc(sbase + S::TM, FS_TM_COLS);
@@ -116,220 +124,293 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     // operand images: Wfe^T (FiLM B, swizzled) and We^T (edge-update B, no swizzle), 2 KB each
     if (tid < 256) reinterpret_cast<uint4 *>(sp + S::WFE)[tid] = reinterpret_cast<const uint4 *>(p.img)[tid];
     // edge-update A tiles: zero (the K half h >= 8 stays zero)
-    for (int e = tid; e < 8192 / 16; e += NTHR) reinterpret_cast<uint4 *>(sp + S::A)[e] = make_uint4(0, 0, 0, 0);
+    for (int e = tid; e < 8192 / 16; e += FS_THR) reinterpret_cast<uint4 *>(sp + S::A)[e] = make_uint4(0, 0, 0, 0);
     if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
-    for (int j = tid; j < 32 * nch; j += NTHR) mj[j] = j < n ? p.M[(size_t)b * n + j] : 0;
-    uint32_t qf[2][2][2];
-    load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
-    // the thread's two rows i = i0 + 2c4 + s (s = 0, 1)
-    const bool mrow[2] = {i0 + 2 * c4 < n && p.M[(size_t)b * n + i0 + 2 * c4] != 0,
-                          i0 + 2 * c4 + 1 < n && p.M[(size_t)b * n + i0 + 2 * c4 + 1] != 0};
+    for (int j = tid; j < 32 * nch; j += FS_THR) mj[j] = j < n ? p.M[(size_t)b * n + j] : 0;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
-    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
-    const float rs = rsqrtf((float)DH);
-    const uint32_t L = 32 * q + t;
-    const uint32_t idesc_e = idesc_bf16_f32(128, DE);
 
-    float rm[2][2], rl[2][2];               // running max / sum [s][hh]
-    float fm[2][2], fl[2][2];               // final max, 1/sum [s][hh]
-    float oacc[2][2][4];
+    if (W == NWARP) {
+        // ================= MMA issuer: FiLM one chunk ahead, edge update on demand
+        if (t == 0) {
+            const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_e = idesc_bf16_f32(128, DE);
+            auto issue_film = [&](int it) {
+                const uint32_t fb = bar(FB_FULL + it % FS_NFULL);
+                if (!mbar_wait(fb, (it / FS_NFULL) & 1)) flag_timeout(p.status);
+                if (it >= 2 && !mbar_wait(bar(FB_FILM_EMPTY + (it & 1)), ((it - 2) >> 1) & 1)) flag_timeout(p.status);
+                tc_fence_after();
 #pragma unroll
-    for (int s = 0; s < 2; ++s)
+                for (int s = 0; s < 2; ++s) {
+                    const uint32_t a0 = slot_addr(it, s);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            rm[s][hh] = -INFINITY;
-            rl[s][hh] = 0.f;
-            fm[s][hh] = -INFINITY;
-            fl[s][hh] = 0.f;
-        }
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int x = 0; x < 4; ++x) oacc[hh][mt][x] = 0.f;
-
-    for (int it = 0; it < nit; ++it) {
-        const int s = it % FS_STAGES, j0 = 32 * chunk_of(it);
-        const bool pass2 = it >= nch;
-        const uint32_t st = sbase + s * S::STAGE;
-        const uint32_t full_ph = (it / FS_STAGES) & 1;
-
-        if (it == nch) {
-            // ---------------- end of pass 1: statistics over lanes, then quadrants
-            float *wst = reinterpret_cast<float *>(sp + S::WST);
-            float *fin = reinterpret_cast<float *>(sp + S::FIN);
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float m = rm[s2][hh], l = rl[s2][hh];
-#pragma unroll
-                    for (int o = 4; o < 32; o <<= 1) {
-                        const float mo = __shfl_xor_sync(0xffffffffu, m, o), lo = __shfl_xor_sync(0xffffffffu, l, o);
-                        const float mn = fmaxf(m, mo);
-                        l = (mn == -INFINITY) ? 0.f
-                                              : l * exp2f((m - mn) * LOG2E) + lo * exp2f((mo - mn) * LOG2E);
-                        m = mn;
-                    }
-                    if (g8 == 0) {
-                        const int il = 2 * c4 + s2, h = 2 * hq + hh;
-                        wst[((q * 8 + il) * 8 + h) * 2 + 0] = m;
-                        wst[((q * 8 + il) * 8 + h) * 2 + 1] = l;
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tmem + FS_TM_FILM + 32 * (it & 1) + 16 * s,
+                                    smem_desc(a0 + kk * 32, 16, 1024, LAYOUT_SW128),
+                                    smem_desc(sbase + S::WFE + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f, kk > 0);
                 }
-            __syncthreads();
-            if (tid < 64) {
-                float m = -INFINITY;
+                mma_commit(bar(FB_FILM_FULL + (it & 1)));
+            };
+            issue_film(0);
+            for (int it = 0; it < nit; ++it) {
+                if (it >= nch) {
+                    if (!mbar_wait(bar(FB_A_FULL), (it - nch) & 1)) flag_timeout(p.status);
+                    tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < 4; ++k) m = fmaxf(m, wst[(k * 64 + tid) * 2]);
-                float l = 0.f;
-                if (m != -INFINITY)
+                    for (int e = 0; e < 2; ++e)
+                        mma_bf16_ss(tmem + FS_TM_EDGE + 64 * e,
+                                    smem_desc(sbase + S::A + e * 4096, 128, 256, LAYOUT_NONE),
+                                    smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
+                    mma_commit(bar(FB_EDGE_FULL));
+                }
+                if (it + 1 < nit) issue_film(it + 1);
+            }
+        }
+        __syncwarp();
+        named_bar_sync(2, FS_THR);
+    } else if (W == NWARP + 1) {
+        // ================= TMA: loads into the slot ring, E' stores
+        if (t == 0) {
+            int next_load = 0, free_slots = FS_SLOTS;
+            auto issue_loads = [&]() {
+                while (next_load < nit && nslots(next_load) <= free_slots) {
+                    const int it = next_load, j0 = 32 * chunk_of(it);
+                    const bool pass2 = it >= nch;
+                    const uint32_t fb = bar(FB_FULL + it % FS_NFULL);
+                    mbar_expect_tx(fb, nslots(it) * FS_SLOT);
+                    tma_load_5d(slot_addr(it, 0), &tmE, fb, 0, i0 / 2, j0, 0, b);
+                    tma_load_5d(slot_addr(it, 1), &tmE, fb, 0, i0 / 2, j0, 1, b);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const float mk = wst[(k * 64 + tid) * 2];
-                        if (mk != -INFINITY) l += wst[(k * 64 + tid) * 2 + 1] * exp2f((mk - m) * LOG2E);
+                        if (!pass2 || !keep_s) tma_load_3d(slot_addr(it, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
+                        if (pass2) tma_load_3d(slot_addr(it, vslot) + k * 4096, &tmV, fb, 64 * k, j0, b);
                     }
-                fin[tid * 2] = m;
-                fin[tid * 2 + 1] = (l > 0.f) ? 1.f / l : 0.f;
-                const int il = tid >> 3, h = tid & 7;
-                if (i0 + il < n)
-                    p.LSE[((size_t)b * NH + h) * n + i0 + il] = (m == -INFINITY) ? -INFINITY : m + logf(l);
-            }
-            __syncthreads();
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int il = 2 * c4 + s2, h = 2 * hq + hh;
-                    fm[s2][hh] = fin[(il * 8 + h) * 2];
-                    fl[s2][hh] = fin[(il * 8 + h) * 2 + 1];
+                    if (!pass2 && it + FS_PF < nch) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (it + FS_PF), 0, b);
+                    free_slots -= nslots(it);
+                    ++next_load;
                 }
-            // L2 prefetch of the first tiles of the CTA that runs about one wave later
-            if (tid == 0 && p.prefetch_ahead) {
-                const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
-                if (cid < gridDim.x * gridDim.y) {
-                    const int prb = cid % gridDim.x, pb = cid / gridDim.x;
-                    for (int cc = 0; cc < nch && cc < 2; ++cc)
-                        tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
+            };
+            for (int c = 0; c < nch && c < FS_PF; ++c) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * c, 0, b);
+            issue_loads();
+            for (int it = 0; it < nit; ++it) {
+                const bool pass2 = it >= nch;
+                if (it == nch && p.prefetch_ahead) {
+                    // L2 prefetch of the first tiles of the CTA that runs about one wave later
+                    const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
+                    if (cid < gridDim.x * gridDim.y) {
+                        const int prb = cid % gridDim.x, pb = cid / gridDim.x;
+                        for (int cc = 0; cc < nch && cc < 2; ++cc)
+                            tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
+                    }
                 }
+                if (!mbar_wait(bar(FB_STAGE_DONE + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
+                if (pass2) {
+                    const int j0 = 32 * chunk_of(it);
+                    tma_store_5d(&tmEo, slot_addr(it, 0), 0, i0 / 2, j0, 0, b);
+                    tma_store_5d(&tmEo, slot_addr(it, 1), 0, i0 / 2, j0, 1, b);
+                    tma_store_commit();
+                    // the previous pass-2 chunk's slots are free once its store has read them
+                    if (it > nch) {
+                        tma_store_wait_read1();
+                        free_slots += ns2;
+                    }
+                } else {
+                    free_slots += 3;
+                }
+                issue_loads();
             }
-        }
-
-        // ---------------- FiLM on the tensor cores (one thread issues)
-        if (tid == 0) {
-            if (!mbar_wait(bar_full + 8 * s, full_ph)) flag_timeout(p.status);
-            tc_fence_after();
-            issue_pair_products<1>(st + S::SE, sbase + S::WFE, tmem + FS_TM_FILM);
-            mma_commit(bar_film);
-            if (!pass2 && it + 2 + FS_PF < nch) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (it + 2 + FS_PF), 0, b);
+            tma_store_wait_read0();
         }
         __syncwarp();
-
-        // ---------------- scores S^T = K Q^T on warp MMAs (2 heads per warp)
-        if (!mbar_wait(bar_full + 8 * s, full_ph)) flag_timeout(p.status);
-        float sacc[2][4];
-        warp_scores2<1>(st + S::SK, q, t, hq, qf, sacc);
-
-        // ---------------- combine with FiLM: s' = s(1+gamma)+beta, masked
-        if (!mbar_wait(bar_film, it & 1)) flag_timeout(p.status);
-        tc_fence_after();
-        const bool mcol = mj[j0 + 8 * q + g8] != 0;
-        bool valid[2];
+        named_bar_sync(2, FS_THR);   // the ring is drained: the compute warps may reuse it
+    } else {
+        // ================= compute warps
+        const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+        const float rs = rsqrtf((float)DH);
+        const uint32_t L = 32 * q + t;
+        uint32_t qf[2][2][2];
+        load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
+        // the thread's two rows i = i0 + 2c4 + s (s = 0, 1)
+        const bool mrow[2] = {i0 + 2 * c4 < n && p.M[(size_t)b * n + i0 + 2 * c4] != 0,
+                              i0 + 2 * c4 + 1 < n && p.M[(size_t)b * n + i0 + 2 * c4 + 1] != 0};
+        float rm[2][2], rl[2][2];               // running max / sum [s][hh]
+        float fm[2][2], fl[2][2];               // final max, 1/sum [s][hh]
+        float oacc[2][2][4];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            valid[e] = mcol && mrow[e];
-            float gm[2], bt[2];
-            tmem_ld2(tl + FS_TM_FILM + 16 * e + 2 * hq, gm[0], gm[1]);
-            tmem_ld2(tl + FS_TM_FILM + 16 * e + NH + 2 * hq, bt[0], bt[1]);
-            tmem_ld_wait();
+        for (int s = 0; s < 2; ++s)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int h = 2 * hq + hh;
-                const float gam = gm[hh] + g[h], bet = bt[hh] + g[NH + h];
-                const float sv = sacc[hh][e] * rs * (1.f + gam) + bet;
-                sacc[hh][e] = valid[e] ? sv : -INFINITY;
+                rm[s][hh] = -INFINITY;
+                rl[s][hh] = 0.f;
+                fm[s][hh] = -INFINITY;
+                fl[s][hh] = 0.f;
             }
-        }
-
-        if (!pass2) {
-            // running statistics (online softmax): one value per (row, head) and chunk
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) oacc[hh][mt][x] = 0.f;
+
+        for (int it = 0; it < nit; ++it) {
+            const int j0 = 32 * chunk_of(it);
+            const bool pass2 = it >= nch;
+
+            if (it == nch) {
+                // ---------------- end of pass 1: statistics over lanes, then quadrants
+                tmem_st_wait();
+                float *wst = reinterpret_cast<float *>(sp + S::WST);
+                float *fin = reinterpret_cast<float *>(sp + S::FIN);
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float m = rm[s2][hh], l = rl[s2][hh];
+#pragma unroll
+                        for (int o = 4; o < 32; o <<= 1) {
+                            const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+                            const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+                            const float mn = fmaxf(m, mo);
+                            l = (mn == -INFINITY) ? 0.f
+                                                  : l * exp2f((m - mn) * LOG2E) + lo * exp2f((mo - mn) * LOG2E);
+                            m = mn;
+                        }
+                        if (g8 == 0) {
+                            const int il = 2 * c4 + s2, h = 2 * hq + hh;
+                            wst[((q * 8 + il) * 8 + h) * 2 + 0] = m;
+                            wst[((q * 8 + il) * 8 + h) * 2 + 1] = l;
+                        }
+                    }
+                named_bar_sync(1, NTHR);
+                if (tid < 64) {
+                    float m = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) m = fmaxf(m, wst[(k * 64 + tid) * 2]);
+                    float l = 0.f;
+                    if (m != -INFINITY)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float mk = wst[(k * 64 + tid) * 2];
+                            if (mk != -INFINITY) l += wst[(k * 64 + tid) * 2 + 1] * exp2f((mk - m) * LOG2E);
+                        }
+                    fin[tid * 2] = m;
+                    fin[tid * 2 + 1] = (l > 0.f) ? 1.f / l : 0.f;
+                    const int il = tid >> 3, h = tid & 7;
+                    if (i0 + il < n)
+                        p.LSE[((size_t)b * NH + h) * n + i0 + il] = (m == -INFINITY) ? -INFINITY : m + logf(l);
+                }
+                named_bar_sync(1, NTHR);
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int il = 2 * c4 + s2, h = 2 * hq + hh;
+                        fm[s2][hh] = fin[(il * 8 + h) * 2];
+                        fl[s2][hh] = fin[(il * 8 + h) * 2 + 1];
+                    }
+            }
+
+            // ---------------- scores S^T = K Q^T on warp MMAs (2 heads per warp)
+            if (!mbar_wait(bar(FB_FULL + it % FS_NFULL), (it / FS_NFULL) & 1)) flag_timeout(p.status);
+            float sacc[2][4];
+            const uint32_t scol = tl + FS_TM_S + 16 * chunk_of(it) + 2 * hq;
+            if (pass2 && keep_s) {
+                tmem_ld2(scol, sacc[0][0], sacc[1][0]);
+                tmem_ld2(scol + 8, sacc[0][1], sacc[1][1]);
+                tmem_ld_wait();
+            } else {
+                warp_scores2<1>(slot_addr(it, 2), q, t, hq, qf, sacc);
+                if (keep_s) {
+                    tmem_st2(scol, sacc[0][0], sacc[1][0]);
+                    tmem_st2(scol + 8, sacc[0][1], sacc[1][1]);
+                }
+            }
+
+            // ---------------- combine with FiLM: s' = s(1+gamma)+beta, masked
+            if (!mbar_wait(bar(FB_FILM_FULL + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
+            tc_fence_after();
+            float gm[2][2], bt[2][2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const uint32_t fcol = FS_TM_FILM + 32 * (it & 1) + 16 * e;
+                tmem_ld2(tl + fcol + 2 * hq, gm[e][0], gm[e][1]);
+                tmem_ld2(tl + fcol + NH + 2 * hq, bt[e][0], bt[e][1]);
+            }
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (t == 0) mbar_arrive(bar(FB_FILM_EMPTY + (it & 1)));
+            const bool mcol = mj[j0 + 8 * q + g8] != 0;
+            bool valid[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                valid[e] = mcol && mrow[e];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const float x = sacc[hh][e];
-                    const float mn = fmaxf(rm[e][hh], x);
-                    if (mn != -INFINITY) {
-                        rl[e][hh] = rl[e][hh] * exp2f((rm[e][hh] - mn) * LOG2E) + exp2f((x - mn) * LOG2E);
-                        rm[e][hh] = mn;
-                    }
+                    const int h = 2 * hq + hh;
+                    const float gam = gm[e][hh] + g[h], bet = bt[e][hh] + g[NH + h];
+                    const float sv = sacc[hh][e] * rs * (1.f + gam) + bet;
+                    sacc[hh][e] = valid[e] ? sv : -INFINITY;
                 }
-            tc_fence_before();
-            __syncthreads();   // stage s and the FiLM columns are free again
-            if (tid == 0 && it + 2 < nit) issue_load(it + 2);
-            continue;
-        }
+            }
 
-        // ---------------- pass 2: normalised coefficients, edge-update A operand
+            if (!pass2) {
+                // running statistics (online softmax): one value per (row, head) and chunk
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
+                for (int e = 0; e < 2; ++e)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                sacc[hh][e] = valid[e] ? exp2f((sacc[hh][e] - fm[e][hh]) * LOG2E) * fl[e][hh] : 0.f;
-            *reinterpret_cast<uint32_t *>(sp + S::A + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(sacc[0][e], sacc[1][e]);
-        }
-        sacc[0][2] = sacc[0][3] = sacc[1][2] = sacc[1][3] = 0.f;
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const float x = sacc[hh][e];
+                        const float mn = fmaxf(rm[e][hh], x);
+                        if (mn != -INFINITY) {
+                            rl[e][hh] = rl[e][hh] * exp2f((rm[e][hh] - mn) * LOG2E) + exp2f((x - mn) * LOG2E);
+                            rm[e][hh] = mn;
+                        }
+                    }
+                __syncwarp();
+                if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 1)));
+                continue;
+            }
+
+            // ---------------- pass 2: normalised coefficients, edge-update A operand
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    sacc[hh][e] = valid[e] ? exp2f((sacc[hh][e] - fm[e][hh]) * LOG2E) * fl[e][hh] : 0.f;
+                *reinterpret_cast<uint32_t *>(sp + S::A + e * 4096 + ns16(L, 2 * hq)) =
+                    pack_bf16(sacc[0][e], sacc[1][e]);
+            }
+            sacc[0][2] = sacc[0][3] = sacc[1][2] = sacc[1][3] = 0.f;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (t == 0) mbar_arrive(bar(FB_A_FULL));
+
+            // ---------------- O += a V on warp MMAs (overlaps the edge MMAs)
+            warp_contract2<1, true>(slot_addr(it, vslot), q, t, hq, sacc, oacc);
+
+            // ---------------- E' = E + a We, in place (the producer stores it)
+            if (!mbar_wait(bar(FB_EDGE_FULL), (it - nch) & 1)) flag_timeout(p.status);
             tc_fence_after();
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
-                mma_bf16_ss(tmem + FS_TM_EDGE + 64 * e, smem_desc(sbase + S::A + e * 4096, 128, 256, LAYOUT_NONE),
-                            smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
-            mma_commit(bar_edge);
-            // stage (it+2) % 3 held iteration it-1, whose E' store may still be reading it
-            if (it + 2 < nit) {
-                tma_store_wait_read0();
-                issue_load(it + 2);
+            for (int e = 0; e < 2; ++e) {
+                float dv[16];
+                tmem_ld16(tl + FS_TM_EDGE + 64 * e + 16 * hq, dv);
+                tmem_ld_wait();
+                add_residual16(sp + (slot_addr(it, e) - sbase) + L * 128, L, hq, dv);
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 1)));
         }
-        __syncwarp();
 
-        // ---------------- O += a V on warp MMAs (overlaps the edge MMAs)
-        warp_contract2<1, true>(st + S::SV, q, t, hq, sacc, oacc);
-
-        // ---------------- E' = E + a We, in place, then TMA store
-        if (!mbar_wait(bar_edge, (it - nch) & 1)) flag_timeout(p.status);
-        tc_fence_after();
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            float dv[16];
-            tmem_ld16(tl + FS_TM_EDGE + 64 * e + 16 * hq, dv);
-            tmem_ld_wait();
-            add_residual16(sp + (st - sbase) + S::SE + tile_off<1>(e) + L * 128, L, hq, dv);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_5d(&tmEo, st + S::SE, 0, i0 / 2, j0, 0, b);
-            tma_store_commit();
-        }
-    }
-
-    // ---------------- O: sum over the quadrant warps
-    if (tid == 0) tma_store_wait_read0();
-    __syncthreads();   // every stage is free
-    store_quadrant_part(sp, S::OPART, oacc, q, hq, t);
-    __syncthreads();
-    {
+        // ---------------- O: sum over the quadrant warps (in the drained ring)
+        named_bar_sync(2, FS_THR);
+        store_quadrant_part(sp, S::OPART, oacc, q, hq, t);
+        named_bar_sync(1, NTHR);
         const float *part = reinterpret_cast<const float *>(sp + S::OPART);
         for (int x = tid; x < TB * HD / 2; x += NTHR) {
             const int il = (2 * x) / HD, d = (2 * x) % HD;
@@ -359,7 +440,7 @@ cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t
         attr_done = true;
     }
     CUtensorMap mE, mEo, mK, mV;
-    if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32) || !encode_pair_map(&mEo, a.Eout, d.B, d.n, false, 32) ||
+    if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mEo, a.Eout, d.B, d.n, false, 32, 1) ||
         !encode_node_map(&mK, a.K, d.B, d.n, 32) || !encode_node_map(&mV, a.V, d.B, d.n, 32))
         return cudaErrorInvalidValue;
     FwdParams p;
@@ -372,7 +453,7 @@ cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t
     p.status = a.status;
     p.n = d.n;
     p.prefetch_ahead = (uint32_t)sm_count();
-    k_fwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), NTHR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
+    k_fwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), FS_THR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
     return cudaGetLastError();
 }
 

@@ -22,12 +22,13 @@ static EncodeTiledFn get_encode() {
     return fn;
 }
 
-// A [B, n, n, 64] bf16 pair tensor viewed as 5-D with a box of 8 x box_rows pairs.
+// A [B, n, n, 64] bf16 pair tensor viewed as 5-D with a box of 8 x box_rows
+// pairs (box_s = 2) or of the 4 x box_rows pairs of one parity s (box_s = 1).
 // Row tile (transposed = false): dims (c, ic, j, s, b) with i = 2ic + s, so the
 // box lands in shared memory as [s][j box_rows][ic 4][c 64].  Column tile
 // (transposed = true): dims (c, jc, i, s, b) with j = 2jc + s, landing as
 // [s][i box_rows][jc 4][c 64].  Requires n even (i = 2ic + s stays inside the graph).
-bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transposed, int box_rows) {
+bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transposed, int box_rows, int box_s) {
     auto enc = get_encode();
     if (!enc) return false;
     const cuuint64_t rowb = DE * 2;                       // one pair: 128 bytes
@@ -43,7 +44,7 @@ bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transp
         strides[2] = rowb;                                  // s -> one column j
     }
     strides[3] = (cuuint64_t)n * n * rowb;                  // b
-    const cuuint32_t box[5] = {64, 4, (cuuint32_t)box_rows, 2, 1};
+    const cuuint32_t box[5] = {64, 4, (cuuint32_t)box_rows, (cuuint32_t)box_s, 1};
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
