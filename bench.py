@@ -35,6 +35,12 @@ METRIC = "edge-pairs/sec (B·n²) fwd and fwd+bwd on 1 B200; % of HBM roofline"
 UNIT = "edge-pairs/s"
 FALLBACK_HBM_GBS = 6650.0
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the dominant kernels on this workload, from the ncu capture summarised in
+# profiles/ (k_bwd_rows_sbm.md, k_fwd_stream_sbm.md).  They describe the
+# kernels as captured; a changed kernel reports null until it is re-captured.
+NCU_TRAFFIC = {("sbm", "k_bwd_rows"): 477439232, ("sbm", "k_fwd_stream"): 269294592}
+
 
 def env_rank():
     return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
@@ -161,8 +167,9 @@ def run_ours(args):
     K = args.steps
     ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for a, b in ev_f + ev_b:          # torch creates the CUDA event on first record
+    for a, b in ev_f + ev_b + ev_r:   # torch creates the CUDA event on first record
         a.record(stream)
         b.record(stream)
     clocks = ClockSampler(local)
@@ -174,6 +181,7 @@ def run_ours(args):
     for k in range(K):
         eaga.set_profile_events(0, *ev_f[k])
         eaga.set_profile_events(1, *ev_b[k])
+        eaga.set_profile_events(2, *ev_r[k])
         step()
     t1.record(stream)
     torch.cuda.synchronize()
@@ -182,9 +190,11 @@ def run_ours(args):
     clk = clocks.stop()
     eaga.set_profile_events(0)
     eaga.set_profile_events(1)
+    eaga.set_profile_events(2)
     ms_total = t0.elapsed_time(t1)
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
     bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_b)
+    rows_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_r)
     if world > 1:
         t = torch.tensor([ms_total], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -209,7 +219,7 @@ def run_ours(args):
     value = world * pairs_step * K / (ms_total / 1e3)
     peak, peak_kind = measured_peaks()
     kb = pair_kernel_bytes(p, "bwd")
-    achieved = kb / (bwd_ms / 1e3) / 1e9
+    achieved = kb / (rows_ms / 1e3) / 1e9
     kf = pair_kernel_bytes(p, "fwd")
     step_bytes = compulsory_bytes(p)
     out = {
@@ -220,11 +230,15 @@ def run_ours(args):
                                "dx=256 de=64 dy=64 H=8 dh=32, bf16 storage / fp32 accumulation",
                    "global_batch": p.B * world, "seq_len": p.n, "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (E, dE' 144 MiB each; E', dE written each step)"},
-        "roofline": {"bound": "hbm", "kernel": "backward pair kernels", "achieved": achieved, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
-                     "algorithmic_bytes": kb, "ms_per_launch": bwd_ms},
-        "roofline_fwd": {"bound": "hbm", "kernel": "forward pair kernels", "achieved": kf / (fwd_ms / 1e3) / 1e9,
-                         "peak": peak, "unit": "GB/s", "frac": kf / (fwd_ms / 1e3) / 1e9 / peak,
+        "roofline": {"bound": "hbm", "kernel": "k_bwd_rows (backward row pair kernel)", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": NCU_TRAFFIC.get((WORKLOAD, "k_bwd_rows")),
+                     "algorithmic_bytes": kb, "ms_per_launch": rows_ms,
+                     "backward_pair_kernels_ms": bwd_ms},
+        "roofline_fwd": {"bound": "hbm", "kernel": "k_fwd_stream (forward pair kernel)",
+                         "achieved": kf / (fwd_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": kf / (fwd_ms / 1e3) / 1e9 / peak,
+                         "traffic": NCU_TRAFFIC.get((WORKLOAD, "k_fwd_stream")),
                          "algorithmic_bytes": kf, "ms_per_launch": fwd_ms},
         "step_roofline": {"compulsory_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
                           "frac_of_measured": step_bytes / (ms_step / 1e3) / 1e9 / peak,

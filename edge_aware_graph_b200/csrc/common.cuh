@@ -76,7 +76,7 @@ inline WsLayout ws_layout(const eaga_dims &d) {
 }
 
 // Optional profiling events around the pair kernels (eaga_set_profile_events).
-extern void *g_prof_events[2][2];
+extern void *g_prof_events[3][2];
 inline void prof_mark(int point, int which, cudaStream_t st) {
     void *ev = g_prof_events[point][which];
     if (ev) cudaEventRecord(static_cast<cudaEvent_t>(ev), st);

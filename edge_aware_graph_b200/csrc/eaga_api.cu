@@ -10,7 +10,7 @@
 using namespace eaga;
 
 namespace eaga {
-void *g_prof_events[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+void *g_prof_events[3][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
 }
 
 namespace {
@@ -168,7 +168,7 @@ eaga_status eaga_get_device_status(void *workspace, void *stream) {
 }
 
 eaga_status eaga_set_profile_events(int point, void *before, void *after) {
-    if (point < 0 || point > 1) return EAGA_ERR_INVALID_ARG;
+    if (point < 0 || point > 2) return EAGA_ERR_INVALID_ARG;
     if ((before == nullptr) != (after == nullptr)) return EAGA_ERR_INVALID_ARG;
     g_prof_events[point][0] = before;
     g_prof_events[point][1] = after;

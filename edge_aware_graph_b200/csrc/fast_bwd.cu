@@ -686,8 +686,10 @@ static cudaError_t launch_bwd_nr(const eaga_dims &d, const BwdArgs &a, const Fas
         p.npad = W.npad;
         cfg.gridDim = dim3(nc, (d.n + TB - 1) / TB, d.B);
         cfg.dynamicSmemBytes = RowSmem<NR>::BYTES;
+        prof_mark(2, 0, st);
         cudaError_t e = cudaLaunchKernelEx(&cfg, k_bwd_rows<NR>, mE, mDEp, mDE, mK, mV, p);
         if (e != cudaSuccess) return e;
+        prof_mark(2, 1, st);
     }
     {
         CUtensorMap mPds, mPa, mQ, mDO;

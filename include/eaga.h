@@ -168,10 +168,11 @@ EAGA_API eaga_status eaga_get_device_status(void *workspace, void *stream);
 /* Profiling aid.  After eaga_set_profile_events(point, before, after) with
  * two cudaEvent_t handles, every later eaga_forward (point 0: the pair
  * kernels of the forward) or eaga_backward (point 1: the pair kernels of the
- * backward) records `before` on its stream just before launching those
+ * backward; point 2: the backward's row pair kernel alone, specialised bf16
+ * path only) records `before` on its stream just before launching those
  * kernels and `after` just after them.  NULL events clear the point.  This
  * is a process-wide setting: not for concurrent calls. */
-typedef enum { EAGA_PROF_FWD_PAIR = 0, EAGA_PROF_BWD_PAIR = 1 } eaga_prof_point;
+typedef enum { EAGA_PROF_FWD_PAIR = 0, EAGA_PROF_BWD_PAIR = 1, EAGA_PROF_BWD_ROWS = 2 } eaga_prof_point;
 EAGA_API eaga_status eaga_set_profile_events(int point, void *before, void *after);
 
 /* Number of kernel launches (this library's kernels) that one eaga_forward
