@@ -135,7 +135,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from edge_aware_graph_b200 import eaga
+    from edge_aware_graph_b200 import dp, eaga
     from edge_aware_graph_b200 import inputs as I
     from edge_aware_graph_b200.buffers import LayerBuffers
 
@@ -145,9 +145,9 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    p = I.preset(WORKLOAD)
+    p = I.preset(WORKLOAD, seed=dp.rank_seed(I.preset(WORKLOAD).seed, rank))
     d = I.draw_inputs(p, with_grads=True)
-    W = I.draw_weights(p)
+    W = I.draw_weights(I.preset(WORKLOAD))          # one model: the same weights on every rank
     buf = LayerBuffers(p.B, p.n, p.dx, p.de, p.dy, p.H, p.dh, dtype=p.dtype, backward=True)
     buf.load_inputs(d, W)
     stream = torch.cuda.current_stream()
@@ -156,8 +156,7 @@ def run_ours(args):
     def step():
         buf.forward(stream)
         buf.backward(stream)
-        if world > 1:
-            dist.all_reduce(flat_dw)
+        dp.allreduce_weight_grads(flat_dw)
 
     for _ in range(args.warmup):
         step()
@@ -195,17 +194,11 @@ def run_ours(args):
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
     bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_b)
     rows_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_r)
-    if world > 1:
-        t = torch.tensor([ms_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = dp.max_over_ranks(ms_total, "cuda")
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, buf, d, stream, step)
-    if world > 1:
-        t = torch.tensor([e2e["ms"]], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms"] = float(t.item())
+    e2e["ms"] = dp.max_over_ranks(e2e["ms"], "cuda")
 
     launches = (eaga.kernel_launches(buf.dims, False) + eaga.kernel_launches(buf.dims, True)) * K
     if world > 1:
