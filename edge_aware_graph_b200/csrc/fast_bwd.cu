@@ -628,6 +628,9 @@ __global__ void k_film_grads(const float *dg, int B, int dy, const __nv_bfloat16
 
 // ---------------------------------------------------------------- host side
 
+cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
+                              cudaStream_t st);
+
 template <int NR>
 static cudaError_t launch_bwd_nr(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                                  cudaStream_t st) {
@@ -662,35 +665,12 @@ static cudaError_t launch_bwd_nr(const eaga_dims &d, const BwdArgs &a, const Fas
     cfg.stream = st;
     cfg.attrs = at;
     cfg.numAttrs = 1;
+    prof_mark(2, 0, st);
     {
-        CUtensorMap mE, mDEp, mDE, mK, mV;
-        if (!encode_pair_map(&mE, a.E, d.B, d.n, false, TCN) ||
-            !encode_pair_map(&mDEp, a.dEout, d.B, d.n, false, TCN) ||
-            !encode_pair_map(&mDE, a.dE, d.B, d.n, false, TCN) || !encode_node_map(&mK, a.K, d.B, d.n, TCN) ||
-            !encode_node_map(&mV, a.V, d.B, d.n, TCN))
-            return cudaErrorInvalidValue;
-        BwdRowParams p;
-        p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
-        p.dO = dO;
-        p.LSE = a.LSE;
-        p.g = g;
-        p.img = reinterpret_cast<const uint8_t *>(ws + W.img);
-        p.M = a.M;
-        p.D = D;
-        p.dQ = dQ;
-        p.rparts = reinterpret_cast<float *>(ws + W.rparts);
-        p.Pa = reinterpret_cast<__nv_bfloat16 *>(ws + W.Pa);
-        p.Pds = reinterpret_cast<__nv_bfloat16 *>(ws + W.Pds);
-        p.status = a.status;
-        p.n = d.n;
-        p.npad = W.npad;
-        cfg.gridDim = dim3(nc, (d.n + TB - 1) / TB, d.B);
-        cfg.dynamicSmemBytes = RowSmem<NR>::BYTES;
-        prof_mark(2, 0, st);
-        cudaError_t e = cudaLaunchKernelEx(&cfg, k_bwd_rows<NR>, mE, mDEp, mDE, mK, mV, p);
+        cudaError_t e = launch_bwd_stream(d, a, W, ws, g, st);
         if (e != cudaSuccess) return e;
-        prof_mark(2, 1, st);
     }
+    prof_mark(2, 1, st);
     {
         CUtensorMap mPds, mPa, mQ, mDO;
         if (!encode_p_map(&mPds, ws + W.Pds, d.B, d.n, W.npad) || !encode_p_map(&mPa, ws + W.Pa, d.B, d.n, W.npad) ||

@@ -1,0 +1,553 @@
+// Backward row pair kernel for de = 64, H = 8, dh = 32, bf16 storage (sm_100a).
+//
+// Chain rule of the layer (formulas as in the forward, differentiated):
+//   u_ij^h = We[h,:] . dE'_ij          dA^h_ij = dO_ih . v_jh + u_ij^h
+//   D_ih   = sum_j a_ij dA_ij          dS'_ij  = a_ij (dA_ij - D_ih)
+//   dgamma = dS' s,  dbeta = dS',  ds = dS' (1 + gamma)
+//   dq_i = sum_j ds_ij k_j / sqrt(dh)
+//   dE = dE' + [dgamma|dbeta] Wfe^T,  dWfe = sum E^T [dgamma|dbeta],  dWe = sum a^T dE',  dg = sum [dgamma|dbeta]
+// with a_ij = exp(s'_ij - LSE_i) from the forward's saved row statistics.
+//
+// One CTA owns 8 query rows i of one graph and streams the columns j of those
+// rows in chunks of 32 (256 pairs: two 16 KB E tiles, two 16 KB dE' tiles,
+// the 16 KB K and V chunks), twice, because D needs a whole row before any
+// dS' exists:
+//   pass 1: FiLM f = E Wfe and u = dE' We^T on the tensor cores (tcgen05,
+//           fp32 in TMEM), S = Q K^T and dP = dO V^T on warp MMAs, a, dA,
+//           and a running D per thread; S and dP stay in TMEM for pass 2
+//           (32 columns per chunk, n <= 256; larger n reloads K and V);
+//   pass 2: f and u again (E and dE' come back from L2: the chunks are walked
+//           in reverse), dS', dgamma, dbeta, ds; dE = dE' + df Wfe^T on the
+//           tensor cores, in place in shared memory, stored with TMA;
+//           dq += ds K (warp MMAs); dWfe, dWe, dg partials (warp MMAs); and
+//           a, ds of every pair stored in bf16 for the dk / dv kernel.
+// E and dE' leave HBM once, dE is written once.  No CTA waits for another.
+//
+// Warp roles as in the forward pair kernel: 16 compute warps (warp W reads
+// TMEM quadrant W%4 and handles heads 2(W/4), 2(W/4)+1), one MMA warp (FiLM
+// and u one chunk ahead into double-buffered TMEM ranges, dE when the compute
+// warps have written df), one TMA warp (a ring of twelve 16 KB slots, dE
+// stores).  They meet only on mbarriers.  The pair <-> lane mapping is the
+// forward's: row 4j + ic of E tile s is the pair (j, i = 2ic + s), which lane
+// t of quadrant q = j/8 holds in accumulator register s of its m16n8 tile.
+#include <math.h>
+#include "fast.h"
+#include "fast_common.cuh"
+
+namespace eaga {
+namespace fast {
+
+using namespace sm100;
+using namespace dev;
+
+constexpr int BS_SLOTS = 12;
+constexpr uint32_t BS_SLOT = 16384;
+constexpr int BS_NFULL = 4;
+constexpr int BS_THR = NTHR + 64;
+constexpr int BS_KEEP_MAX_CHUNKS = 8;     // S and dP of up to 8 chunks (n <= 256) stay in TMEM
+
+struct BsSmem {
+    static constexpr uint32_t IMG = BS_SLOTS * BS_SLOT;       // Wfe^T sw (FiLM), We sw (u), Wfe ns (dE): 2 KB each
+    static constexpr uint32_t DF = IMG + 6144;                // 2 tiles [128][16] ns: [dgamma | dbeta]
+    static constexpr uint32_t AT = DF + 8192;                 // 2 tiles [128][16] ns: a (h >= 8 zero)
+    static constexpr uint32_t WD = AT + 8192;                 // per-quadrant D [4][8 i][8 h]
+    static constexpr uint32_t WDG = WD + 1024;                // per-warp dg [16][4]
+    static constexpr uint32_t G = WDG + 256;                  // g_b [16]
+    static constexpr uint32_t MJ = G + 64;                    // node mask [n <= 1024]
+    static constexpr uint32_t BAR = MJ + 1024;
+    static constexpr uint32_t TM = BAR + 8 * 12;
+    static constexpr uint32_t STAB = TM + 16;                 // slot table [4 iterations][8] u8
+    static constexpr uint32_t BYTES = STAB + 32 + 1024;
+    // in the drained ring at the end: dq quadrant sums [4][8][256] f32 (32 KB),
+    // then dWfe partials [4 kr][64 c][16 k] (16 KB) and dWe partials [4 kr][8 h][64 c] (8 KB)
+    static constexpr uint32_t QPART = 0, WFP = 32768, WEP = WFP + 16384;
+};
+constexpr int BB_FULL = 0, BB_FILM_FULL = 4, BB_FILM_EMPTY = 6, BB_DF_FULL = 8, BB_DE_FULL = 9,
+              BB_STAGE_DONE = 10;
+
+// TMEM: FiLM 0..63 and u 64..127 (two buffers each), dE 128..255, kept S / dP from 256 (32 per chunk)
+constexpr uint32_t BS_TM_COLS = 512, BS_TM_FILM = 0, BS_TM_U = 64, BS_TM_DE = 128, BS_TM_KEEP = 256;
+
+struct BwdStreamParams {
+    const __nv_bfloat16 *Q, *dO;
+    const float *LSE, *g;
+    const uint8_t *img, *M;
+    __nv_bfloat16 *dQ;       // [B,n,256] out (scaled)
+    float *rparts;           // [graph * row block][RPART] out
+    __nv_bfloat16 *Pa, *Pds; // [B,H,n,npad] out: a and ds (unscaled) of every pair
+    int *status;
+    int n, npad;
+};
+
+__global__ void __launch_bounds__(BS_THR, 1)
+k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmDEp,
+             const __grid_constant__ CUtensorMap tmDE, const __grid_constant__ CUtensorMap tmK,
+             const __grid_constant__ CUtensorMap tmV, BwdStreamParams p) {
+    using S = BsSmem;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
+    const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = (W >> 2) & 3, t = tid & 31, c4 = t & 3, g8 = t >> 2;
+    const int n = p.n, nch = (n + 31) / 32, nit = 2 * nch;
+    const int b = blockIdx.y, i0 = blockIdx.x * TB;
+    const uint32_t bars = sbase + S::BAR;
+    auto bar = [&](int k) { return bars + 8 * k; };
+    float *g = reinterpret_cast<float *>(sp + S::G);
+    uint8_t *mj = sp + S::MJ;
+
+    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0.  Its
+    // tiles: E(s=0), E(s=1), dE'(s=0), dE'(s=1), K, then V in pass 1 (and in
+    // pass 2 when S, dP are not kept).  The TMA warp places each tile in any
+    // free slot and records the slot in the table entry it % 4, which the
+    // other warps read after the iteration's load barrier.
+    const bool keep = nch <= BS_KEEP_MAX_CHUNKS;
+    const int ns1 = 6, ns2 = keep ? 5 : 6;
+    auto chunk_of = [&](int it) { return it < nch ? it : nit - 1 - it; };
+    auto nslots = [&](int it) { return it < nch ? ns1 : ns2; };
+    volatile uint8_t *stab = sp + S::STAB;
+    auto slot_addr = [&](int it, int k) { return sbase + (uint32_t)stab[(it % BS_NFULL) * 8 + k] * BS_SLOT; };
+
+    // ---------------- setup: barriers, TMEM, operands
+    if (tid == 0) {
+        for (int k = 0; k < BS_NFULL; ++k) mbar_init(bar(BB_FULL + k), 1);
+        mbar_init(bar(BB_FILM_FULL), 1);
+        mbar_init(bar(BB_FILM_FULL + 1), 1);
+        mbar_init(bar(BB_FILM_EMPTY), NWARP);
+        mbar_init(bar(BB_FILM_EMPTY + 1), NWARP);
+        mbar_init(bar(BB_DF_FULL), NWARP);
+        mbar_init(bar(BB_DE_FULL), 1);
+        mbar_init(bar(BB_STAGE_DONE), NWARP);
+        mbar_init(bar(BB_STAGE_DONE + 1), NWARP);
+        fence_mbar_init();
+    }
+    if (W == 0) {
+        tmem_alloc(sbase + S::TM, BS_TM_COLS);
+        tmem_relinquish();
+    }
+    if (tid < 384) {
+        const uint32_t img_off = (tid >> 7) == 0 ? IMG_WFE_T_SW : (tid >> 7) == 1 ? IMG_WE_SW : IMG_WFE_NS;
+        reinterpret_cast<uint4 *>(sp + S::IMG)[tid] = reinterpret_cast<const uint4 *>(p.img)[(img_off >> 4) + (tid & 127)];
+    }
+    // a tiles: the K half h >= 8 stays zero
+    for (int e = tid; e < 8192 / 16; e += BS_THR) reinterpret_cast<uint4 *>(sp + S::AT)[e] = make_uint4(0, 0, 0, 0);
+    if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
+    for (int j = tid; j < 32 * nch; j += BS_THR) mj[j] = j < n ? p.M[(size_t)b * n + j] : 0;
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+
+    if (W == NWARP) {
+        // ================= MMA issuer
+        if (t == 0) {
+            const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_d = idesc_bf16_f32(128, DE);
+            auto issue_fu = [&](int it) {
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    const uint32_t ae = slot_addr(it, s), ad = slot_addr(it, 2 + s);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        mma_bf16_ss(tmem + BS_TM_FILM + 32 * (it & 1) + 16 * s,
+                                    smem_desc(ae + kk * 32, 16, 1024, LAYOUT_SW128),
+                                    smem_desc(sbase + S::IMG + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f, kk > 0);
+                        mma_bf16_ss(tmem + BS_TM_U + 32 * (it & 1) + 16 * s,
+                                    smem_desc(ad + kk * 32, 16, 1024, LAYOUT_SW128),
+                                    smem_desc(sbase + S::IMG + 2048 + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f,
+                                    kk > 0);
+                    }
+                }
+                mma_commit(bar(BB_FILM_FULL + (it & 1)));
+            };
+            auto issue_de = [&]() {
+                tc_fence_after();
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    mma_bf16_ss(tmem + BS_TM_DE + 64 * e, smem_desc(sbase + S::DF + e * 4096, 128, 256, LAYOUT_NONE),
+                                smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_d, 0);
+                mma_commit(bar(BB_DE_FULL));
+            };
+            // issue whichever product is ready first: FiLM/u of the next chunk
+            // (its tiles landed, its TMEM buffer released) or dE of the chunk
+            // whose df the compute warps have written
+            int next_fu = 0, next_de = nch;
+            uint32_t polls = 0;
+            while (next_fu < nit || next_de < nit) {
+                bool progressed = false;
+                if (next_fu < nit && mbar_try_wait(bar(BB_FULL + next_fu % BS_NFULL), (next_fu / BS_NFULL) & 1) &&
+                    (next_fu < 2 || mbar_try_wait(bar(BB_FILM_EMPTY + (next_fu & 1)), ((next_fu - 2) >> 1) & 1))) {
+                    issue_fu(next_fu++);
+                    progressed = true;
+                }
+                if (next_de < nit && next_de < next_fu && mbar_try_wait(bar(BB_DF_FULL), (next_de - nch) & 1)) {
+                    issue_de();
+                    ++next_de;
+                    progressed = true;
+                }
+                if (!progressed && ++polls > (1u << 26)) {
+                    flag_timeout(p.status);
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+        named_bar_sync(2, BS_THR);
+    } else if (W == NWARP + 1) {
+        // ================= TMA: loads into the slot ring, dE stores
+        if (t == 0) {
+            // E and dE' tiles loaded in pass 1 are read again in pass 2: keep
+            // them in L2; pass-2 reads and the dE stores are not read again
+            const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
+            // a pass-2 chunk's E, K (and V) slots are free once the compute
+            // warps are done with it; its dE' slots once the dE store has read them
+            uint32_t free_mask = (1u << BS_SLOTS) - 1u;
+            uint32_t prev_d = 0;          // dE' slots of the previous pass-2 chunk
+            int next_load = 0;
+            auto release = [&](int it, int k) { free_mask |= 1u << stab[(it % BS_NFULL) * 8 + k]; };
+            auto issue_loads = [&]() {
+                while (next_load < nit && __popc(free_mask) >= nslots(next_load)) {
+                    const int it = next_load, j0 = 32 * chunk_of(it);
+                    const bool pass2 = it >= nch;
+                    const uint32_t fb = bar(BB_FULL + it % BS_NFULL);
+                    for (int k = 0; k < nslots(it); ++k) {
+                        const int sidx = __ffs(free_mask) - 1;
+                        free_mask &= free_mask - 1u;
+                        stab[(it % BS_NFULL) * 8 + k] = (uint8_t)sidx;
+                    }
+                    mbar_expect_tx(fb, nslots(it) * BS_SLOT);   // releases the table entry with the barrier
+#pragma unroll
+                    for (int s = 0; s < 2; ++s) {
+                        const uint64_t pol = pass2 ? drop_l2 : keep_l2;
+                        tma_load_5d_hint(slot_addr(it, s), &tmE, fb, 0, i0 / 2, j0, s, b, pol);
+                        tma_load_5d_hint(slot_addr(it, 2 + s), &tmDEp, fb, 0, i0 / 2, j0, s, b, pol);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        tma_load_3d(slot_addr(it, 4) + k * 4096, &tmK, fb, 64 * k, j0, b);
+                        if (!pass2 || !keep) tma_load_3d(slot_addr(it, 5) + k * 4096, &tmV, fb, 64 * k, j0, b);
+                    }
+                    ++next_load;
+                }
+            };
+            issue_loads();
+            for (int it = 0; it < nit; ++it) {
+                const bool pass2 = it >= nch;
+                if (!mbar_wait(bar(BB_STAGE_DONE + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
+                if (pass2) {
+                    const int j0 = 32 * chunk_of(it);
+                    tma_store_5d_hint(&tmDE, slot_addr(it, 2), 0, i0 / 2, j0, 0, b, drop_l2);
+                    tma_store_5d_hint(&tmDE, slot_addr(it, 3), 0, i0 / 2, j0, 1, b, drop_l2);
+                    tma_store_commit();
+                    release(it, 0);
+                    release(it, 1);
+                    release(it, 4);
+                    if (!keep) release(it, 5);
+                    if (it > nch) {
+                        tma_store_wait_read1();
+                        free_mask |= prev_d;
+                    }
+                    prev_d = (1u << stab[(it % BS_NFULL) * 8 + 2]) | (1u << stab[(it % BS_NFULL) * 8 + 3]);
+                } else {
+                    for (int k = 0; k < ns1; ++k) release(it, k);
+                }
+                issue_loads();
+            }
+            tma_store_wait_read0();
+        }
+        __syncwarp();
+        named_bar_sync(2, BS_THR);   // the ring is drained: the compute warps may reuse it
+    } else {
+        // ================= compute warps
+        const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+        const float rs = rsqrtf((float)DH);
+        const uint32_t L = 32 * q + t;
+        uint32_t qf[2][2][2], of[2][2][2];
+        load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
+        load_frags2(p.dO, b, n, i0, hq, g8, c4, of);
+        bool mrow[2];
+        float lse[2][2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int i = i0 + 2 * c4 + e;
+            mrow[e] = i < n && p.M[(size_t)b * n + i] != 0;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) lse[e][hh] = i < n ? p.LSE[((size_t)b * NH + 2 * hq + hh) * n + i] : 0.f;
+        }
+        float dsum[2][2] = {{0.f, 0.f}, {0.f, 0.f}};     // running D partial, then the final D [e][hh]
+        float qacc[2][2][4];
+        float wf[2][4], we4[4];
+        float dgp[4] = {0.f, 0.f, 0.f, 0.f};              // dgamma h0, h1, dbeta h0, h1
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            wf[0][x] = wf[1][x] = we4[x] = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) qacc[hh][0][x] = qacc[hh][1][x] = 0.f;
+        }
+        const int ct = W & 3, kr = W >> 2;
+
+        for (int it = 0; it < nit; ++it) {
+            const int c = chunk_of(it), j0 = 32 * c;
+            const bool pass2 = it >= nch;
+
+            if (it == nch) {
+                // ---------------- D over lanes, then quadrants
+                tmem_st_wait();
+                float *wd = reinterpret_cast<float *>(sp + S::WD);
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float x = dsum[e][hh];
+                        x += __shfl_xor_sync(0xffffffffu, x, 4);
+                        x += __shfl_xor_sync(0xffffffffu, x, 8);
+                        x += __shfl_xor_sync(0xffffffffu, x, 16);
+                        if (g8 == 0) wd[(q * 8 + 2 * c4 + e) * 8 + 2 * hq + hh] = x;
+                    }
+                named_bar_sync(1, NTHR);
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int o = (2 * c4 + e) * 8 + 2 * hq + hh;
+                        dsum[e][hh] = wd[o] + wd[64 + o] + wd[128 + o] + wd[192 + o];
+                    }
+            }
+
+            if (!mbar_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1)) flag_timeout(p.status);
+            // ---------------- S = Q K^T, dP = dO V^T (warp MMAs), or the kept ones
+            float sv[2][4], da[2][4];
+            const uint32_t kcol = tl + BS_TM_KEEP + 32 * c + 2 * hq;
+            if (pass2 && keep) {
+                tmem_ld2(kcol, sv[0][0], sv[1][0]);
+                tmem_ld2(kcol + 8, sv[0][1], sv[1][1]);
+                tmem_ld2(kcol + 16, da[0][0], da[1][0]);
+                tmem_ld2(kcol + 24, da[0][1], da[1][1]);
+                tmem_ld_wait();
+            } else {
+                warp_scores2<1>(slot_addr(it, 4), q, t, hq, qf, sv);
+                warp_scores2<1>(slot_addr(it, 5), q, t, hq, of, da);
+                if (keep) {
+                    tmem_st2(kcol, sv[0][0], sv[1][0]);
+                    tmem_st2(kcol + 8, sv[0][1], sv[1][1]);
+                    tmem_st2(kcol + 16, da[0][0], da[1][0]);
+                    tmem_st2(kcol + 24, da[0][1], da[1][1]);
+                }
+            }
+
+            // ---------------- FiLM and u from TMEM
+            if (!mbar_wait(bar(BB_FILM_FULL + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
+            tc_fence_after();
+            float fg[2][2], fb[2][2], fu[2][2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const uint32_t fcol = BS_TM_FILM + 32 * (it & 1) + 16 * e, ucol = BS_TM_U + 32 * (it & 1) + 16 * e;
+                tmem_ld2(tl + fcol + 2 * hq, fg[e][0], fg[e][1]);
+                tmem_ld2(tl + fcol + NH + 2 * hq, fb[e][0], fb[e][1]);
+                tmem_ld2(tl + ucol + 2 * hq, fu[e][0], fu[e][1]);
+            }
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (t == 0) mbar_arrive(bar(BB_FILM_EMPTY + (it & 1)));
+            const bool mcol = mj[j0 + 8 * q + g8] != 0;
+            float av[2][4], gm[2][4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const bool valid = mcol && mrow[e];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int h = 2 * hq + hh;
+                    const float s = sv[hh][e] * rs;
+                    const float gam = fg[e][hh] + g[h], bet = fb[e][hh] + g[NH + h];
+                    av[hh][e] = valid ? exp2f((s * (1.f + gam) + bet - lse[e][hh]) * LOG2E) : 0.f;
+                    sv[hh][e] = s;
+                    gm[hh][e] = gam;
+                    da[hh][e] += fu[e][hh];
+                }
+            }
+
+            if (!pass2) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) dsum[e][hh] += av[hh][e] * da[hh][e];
+                __syncwarp();
+                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 1)));
+                continue;
+            }
+
+            // ---------------- pass 2: dS', df and a tiles for the tensor cores / warp MMAs
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float dgam[2], dbet[2];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const float dsp = av[hh][e] * (da[hh][e] - dsum[e][hh]);
+                    dgam[hh] = dsp * sv[hh][e];
+                    dbet[hh] = dsp;
+                    da[hh][e] = dsp * (1.f + gm[hh][e]);     // ds (unscaled)
+                    dgp[hh] += dgam[hh];
+                    dgp[2 + hh] += dbet[hh];
+                }
+                *reinterpret_cast<uint32_t *>(sp + S::DF + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(dgam[0], dgam[1]);
+                *reinterpret_cast<uint32_t *>(sp + S::DF + e * 4096 + ns16(L, NH + 2 * hq)) = pack_bf16(dbet[0], dbet[1]);
+                *reinterpret_cast<uint32_t *>(sp + S::AT + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(av[0][e], av[1][e]);
+            }
+            av[0][2] = av[0][3] = av[1][2] = av[1][3] = 0.f;
+            da[0][2] = da[0][3] = da[1][2] = da[1][3] = 0.f;
+            // a and ds of the chunk's pairs for the dk / dv pass: [b][h][i][j] bf16.
+            // Lanes t and t^4 hold neighbouring columns j; they swap one head so that
+            // each stores two columns of one head in a 4-byte word.
+            {
+                const bool odd = g8 & 1;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float xa = __shfl_xor_sync(0xffffffffu, odd ? av[0][e] : av[1][e], 4);
+                    const float xd = __shfl_xor_sync(0xffffffffu, odd ? da[0][e] : da[1][e], 4);
+                    const int i = i0 + 2 * c4 + e, j = j0 + 8 * q + (g8 & ~1);
+                    if (i < n && j < n) {
+                        const size_t o = (((size_t)b * NH + 2 * hq + (odd ? 1 : 0)) * n + i) * p.npad + j;
+                        // streaming stores: read once, by the dk / dv kernel
+                        __stcs(reinterpret_cast<unsigned int *>(p.Pa + o), odd ? pack_bf16(xa, av[1][e]) : pack_bf16(av[0][e], xa));
+                        __stcs(reinterpret_cast<unsigned int *>(p.Pds + o), odd ? pack_bf16(xd, da[1][e]) : pack_bf16(da[0][e], xd));
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, NTHR);          // df and a tiles complete
+            if (t == 0) mbar_arrive(bar(BB_DF_FULL));
+
+            // ---------------- dq += ds K (warp MMAs; overlaps the dE MMAs)
+            warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, da, qacc);
+
+            // ---------------- dWfe [64 c][16 k] and dWe^T [64 c][8 h] partials: warp W owns
+            // c in [16ct, 16ct+16) over the k-range kr of the chunk's pairs
+#pragma unroll 2
+            for (int kk = 4 * kr; kk < 4 * (kr + 1); ++kk) {
+                const int e = kk >> 3, L0 = 16 * (kk & 7);
+                const uint32_t arow = L0 + (t & 7) + ((t >> 4) & 1) * 8;
+                const uint32_t ach = 2 * ct + ((t >> 3) & 1);
+                uint32_t aE[4], aD[4], bF[4], bA0, bA1;
+                ldsm_x4_t(slot_addr(it, e) + sw128(arow, ach), aE);
+                ldsm_x4_t(slot_addr(it, 2 + e) + sw128(arow, ach), aD);
+                const uint32_t Lr = L0 + (t & 7) + ((t >> 3) & 1) * 8;
+                ldsm_x4_t(sbase + S::DF + e * 4096 + ns16(Lr, 8 * (t >> 4)), bF);
+                ldsm_x2_t(sbase + S::AT + e * 4096 + ns16(Lr, 0), bA0, bA1);
+                mma16816(wf[0], aE, bF[0], bF[1]);
+                mma16816(wf[1], aE, bF[2], bF[3]);
+                mma16816(we4, aD, bA0, bA1);
+            }
+            named_bar_sync(1, NTHR);          // every warp is done reading dE', df, a of this chunk
+
+            // ---------------- dE = dE' + df Wfe^T, in place (the TMA warp stores it)
+            if (!mbar_wait(bar(BB_DE_FULL), (it - nch) & 1)) flag_timeout(p.status);
+            tc_fence_after();
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float dv[16];
+                tmem_ld16(tl + BS_TM_DE + 64 * e + 16 * hq, dv);
+                tmem_ld_wait();
+                add_residual16(sp + (slot_addr(it, 2 + e) - sbase) + L * 128, L, hq, dv);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 1)));
+        }
+
+        // ---------------- end of the row block, in the drained ring
+        named_bar_sync(2, BS_THR);
+        float *wdg = reinterpret_cast<float *>(sp + S::WDG);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float x = dgp[k];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+            if (t == 0) wdg[W * 4 + k] = x;
+        }
+        store_quadrant_part(sp, S::QPART, qacc, q, hq, t);
+        {
+            float *wfp = reinterpret_cast<float *>(sp + S::WFP) + kr * (DE * NF);
+            float *wep = reinterpret_cast<float *>(sp + S::WEP) + kr * (NH * DE);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int cc = 16 * ct + g8 + 8 * (e >> 1);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) wfp[cc * NF + nt * 8 + 2 * c4 + (e & 1)] = wf[nt][e];
+                wep[(2 * c4 + (e & 1)) * DE + cc] = we4[e];
+            }
+        }
+        named_bar_sync(1, NTHR);
+        const float *part = reinterpret_cast<const float *>(sp + S::QPART);
+        for (int x = tid; x < TB * HD / 2; x += NTHR) {
+            const int il = (2 * x) / HD, d = (2 * x) % HD;
+            if (i0 + il >= n) continue;
+            float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                o0 += part[k * TB * HD + il * HD + d];
+                o1 += part[k * TB * HD + il * HD + d + 1];
+            }
+            *reinterpret_cast<uint32_t *>(p.dQ + ((size_t)b * n + i0 + il) * HD + d) = pack_bf16(o0 * rs, o1 * rs);
+        }
+        float *rp = p.rparts + (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * RPART;
+        const float *wfp = reinterpret_cast<const float *>(sp + S::WFP);
+        const float *wep = reinterpret_cast<const float *>(sp + S::WEP);
+        for (int x = tid; x < DE * NF + NH * DE + NF; x += NTHR) {
+            float v = 0.f;
+            if (x < DE * NF) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v += wfp[k * DE * NF + x];
+            } else if (x < DE * NF + NH * DE) {
+                const int y2 = x - DE * NF;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v += wep[k * NH * DE + y2];
+            } else {
+                const int y2 = x - DE * NF - NH * DE, which = y2 >> 3, h = y2 & 7, hq2 = h >> 1, hh = h & 1;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v += wdg[(4 * hq2 + k) * 4 + which * 2 + hh];
+            }
+            rp[x] = v;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (W == 0) tmem_dealloc(tmem, BS_TM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+
+cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
+                              cudaStream_t st) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(k_bwd_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, BsSmem::BYTES);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    CUtensorMap mE, mDEp, mDE, mK, mV;
+    if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mDEp, a.dEout, d.B, d.n, false, 32, 1) ||
+        !encode_pair_map(&mDE, a.dE, d.B, d.n, false, 32, 1) || !encode_node_map(&mK, a.K, d.B, d.n, 32) ||
+        !encode_node_map(&mV, a.V, d.B, d.n, 32))
+        return cudaErrorInvalidValue;
+    BwdStreamParams p;
+    p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
+    p.dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
+    p.LSE = a.LSE;
+    p.g = g;
+    p.img = reinterpret_cast<const uint8_t *>(ws + W.img);
+    p.M = a.M;
+    p.dQ = reinterpret_cast<__nv_bfloat16 *>(ws + W.dQ);
+    p.rparts = reinterpret_cast<float *>(ws + W.rparts);
+    p.Pa = reinterpret_cast<__nv_bfloat16 *>(ws + W.Pa);
+    p.Pds = reinterpret_cast<__nv_bfloat16 *>(ws + W.Pds);
+    p.status = a.status;
+    p.n = d.n;
+    p.npad = W.npad;
+    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, p);
+    return cudaGetLastError();
+}
+
+}  // namespace fast
+}  // namespace eaga

@@ -138,9 +138,6 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         if (t == 0) {
             const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_e = idesc_bf16_f32(128, DE);
             auto issue_film = [&](int it) {
-                const uint32_t fb = bar(FB_FULL + it % FS_NFULL);
-                if (!mbar_wait(fb, (it / FS_NFULL) & 1)) flag_timeout(p.status);
-                if (it >= 2 && !mbar_wait(bar(FB_FILM_EMPTY + (it & 1)), ((it - 2) >> 1) & 1)) flag_timeout(p.status);
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
@@ -153,19 +150,38 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
                 mma_commit(bar(FB_FILM_FULL + (it & 1)));
             };
-            issue_film(0);
-            for (int it = 0; it < nit; ++it) {
-                if (it >= nch) {
-                    if (!mbar_wait(bar(FB_A_FULL), (it - nch) & 1)) flag_timeout(p.status);
-                    tc_fence_after();
+            auto issue_edge = [&]() {
+                tc_fence_after();
 #pragma unroll
-                    for (int e = 0; e < 2; ++e)
-                        mma_bf16_ss(tmem + FS_TM_EDGE + 64 * e,
-                                    smem_desc(sbase + S::A + e * 4096, 128, 256, LAYOUT_NONE),
-                                    smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
-                    mma_commit(bar(FB_EDGE_FULL));
+                for (int e = 0; e < 2; ++e)
+                    mma_bf16_ss(tmem + FS_TM_EDGE + 64 * e, smem_desc(sbase + S::A + e * 4096, 128, 256, LAYOUT_NONE),
+                                smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
+                mma_commit(bar(FB_EDGE_FULL));
+            };
+            // issue whichever product is ready first: FiLM of the next chunk (its
+            // tiles landed, its TMEM buffer released) or the edge update of the
+            // chunk whose a the compute warps have written
+            int next_film = 0, next_edge = nch;
+            uint32_t polls = 0;
+            while (next_film < nit || next_edge < nit) {
+                bool progressed = false;
+                if (next_film < nit &&
+                    mbar_try_wait(bar(FB_FULL + next_film % FS_NFULL), (next_film / FS_NFULL) & 1) &&
+                    (next_film < 2 ||
+                     mbar_try_wait(bar(FB_FILM_EMPTY + (next_film & 1)), ((next_film - 2) >> 1) & 1))) {
+                    issue_film(next_film++);
+                    progressed = true;
                 }
-                if (it + 1 < nit) issue_film(it + 1);
+                if (next_edge < nit && next_edge < next_film &&
+                    mbar_try_wait(bar(FB_A_FULL), (next_edge - nch) & 1)) {
+                    issue_edge();
+                    ++next_edge;
+                    progressed = true;
+                }
+                if (!progressed && ++polls > (1u << 26)) {
+                    flag_timeout(p.status);
+                    break;
+                }
             }
         }
         __syncwarp();
@@ -173,6 +189,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     } else if (W == NWARP + 1) {
         // ================= TMA: loads into the slot ring, E' stores
         if (t == 0) {
+            // E tiles loaded in pass 1 are read again in pass 2: keep them in L2;
+            // pass-2 reads and the E' stores are not read again
+            const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
             int next_load = 0, free_slots = FS_SLOTS;
             auto issue_loads = [&]() {
                 while (next_load < nit && nslots(next_load) <= free_slots) {
@@ -180,8 +199,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     const bool pass2 = it >= nch;
                     const uint32_t fb = bar(FB_FULL + it % FS_NFULL);
                     mbar_expect_tx(fb, nslots(it) * FS_SLOT);
-                    tma_load_5d(slot_addr(it, 0), &tmE, fb, 0, i0 / 2, j0, 0, b);
-                    tma_load_5d(slot_addr(it, 1), &tmE, fb, 0, i0 / 2, j0, 1, b);
+                    const uint64_t pol = pass2 ? drop_l2 : keep_l2;
+                    tma_load_5d_hint(slot_addr(it, 0), &tmE, fb, 0, i0 / 2, j0, 0, b, pol);
+                    tma_load_5d_hint(slot_addr(it, 1), &tmE, fb, 0, i0 / 2, j0, 1, b, pol);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         if (!pass2 || !keep_s) tma_load_3d(slot_addr(it, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
@@ -208,8 +228,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 if (!mbar_wait(bar(FB_STAGE_DONE + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
                 if (pass2) {
                     const int j0 = 32 * chunk_of(it);
-                    tma_store_5d(&tmEo, slot_addr(it, 0), 0, i0 / 2, j0, 0, b);
-                    tma_store_5d(&tmEo, slot_addr(it, 1), 0, i0 / 2, j0, 1, b);
+                    tma_store_5d_hint(&tmEo, slot_addr(it, 0), 0, i0 / 2, j0, 0, b, drop_l2);
+                    tma_store_5d_hint(&tmEo, slot_addr(it, 1), 0, i0 / 2, j0, 1, b, drop_l2);
                     tma_store_commit();
                     // the previous pass-2 chunk's slots are free once its store has read them
                     if (it > nch) {
