@@ -38,7 +38,7 @@ size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, s
 
 int kernel_launches(const eaga_dims &, int for_backward) {
     // forward: prologue, weight images, QKV, pairs, out-proj
-    // backward: prologue, dO, rows, cols, dX, wgrad x2, bias partial, rparts partial, finish, film grads
+    // backward: prologue, dO, row pairs, dk/dv, dX, wgrad x2, bias partial, rparts partial, finish, film grads
     return for_backward ? 11 : 5;
 }
 

@@ -1,22 +1,11 @@
-// Backward pair kernels for de = 64, H = 8, dh = 32, bf16 storage (sm_100a).
-//
-// Chain rule of the layer (same formulas as the forward's, differentiated):
-//   u_ij^h = We[h,:] . dE'_ij          dA^h_ij = dO_ih . v_jh + u_ij^h
-//   D_ih   = sum_j a_ij dA_ij          dS'_ij  = a_ij (dA_ij - D_ih)
-//   dgamma = dS' s,  dbeta = dS',  ds = dS' (1 + gamma)
-//   dq_i = sum_j ds_ij k_j / sqrt(dh),  dk_j = sum_i ds_ij q_i / sqrt(dh),  dv_j = sum_i a_ij dO_i
-//   dE = dE' + [dgamma|dbeta] Wfe^T,  dWfe = sum E^T [dgamma|dbeta],  dWe = sum a^T dE',  dg = sum [dgamma|dbeta]
-// D needs a whole row of pairs before any dS' exists, so the work is split in
-//   k_bwd_rows: clusters along j (like the forward): a, u, dA, cluster-wide D,
-//               dS', dq (cluster-reduced), dE (tensor cores, written in place,
-//               TMA store), dWfe / dWe / dg partials reduced over the cluster,
-//               and a, ds of every pair stored in bf16 (32 bytes per pair);
-//   k_bwd_kv:   dk, dv as sums over rows i of those a, ds times Q, dO (warp
-//               MMAs fed by a TMA pipeline), so E and dE' are read only once.
-// The row kernel loads both pair tiles once with TMA and keeps them in shared memory; the FiLM and
-// u = dE' We^T products run on tcgen05 with the same pair <-> TMEM lane map as
-// the forward.  16 warps: warp W reads TMEM quadrant W%4, heads 2(W/4)+{0,1}.
-// NR selects 32NR cluster rows per CTA (NR = 1: two CTAs share an SM).
+// Backward kernels of the specialised path (de = 64, H = 8, dh = 32, bf16
+// storage) besides the row pair kernel (fast_bwd_stream.cu):
+//   k_bwd_kv:   dk_j = sum_i ds_ij q_i / sqrt(dh) and dv_j = sum_i a_ij dO_i
+//               from the a and ds the row kernel stored (warp MMAs fed by a
+//               TMA pipeline), so E and dE' are read only once;
+//   reductions: bias gradients, the per-(graph, row block) dWfe / dWe / dg
+//               partials, the split-K weight-gradient partials, and the global
+//               FiLM term's dWfy, dbf, dy; all in a fixed order.
 #include <math.h>
 #include "fast.h"
 #include "fast_common.cuh"
@@ -27,375 +16,11 @@ namespace fast {
 using namespace sm100;
 using namespace dev;
 
-struct BwdRowParams {
-    const __nv_bfloat16 *Q, *dO;
-    const float *LSE, *g;
-    const uint8_t *img, *M;
-    float *D;                // [B,H,n] out
-    __nv_bfloat16 *dQ;       // [B,n,256] out (scaled)
-    float *rparts;           // [graph * row block][RPART] out
-    __nv_bfloat16 *Pa, *Pds; // [B,H,n,npad] out: a and ds (unscaled) of every pair
-    int *status;
-    int n, npad;
-};
-
 struct BwdKvParams {
     __nv_bfloat16 *dK, *dV;  // [B,n,256] out (dK scaled)
     int *status;
     int n;
 };
-
-// ---------------------------------------------------------------- row kernel
-
-template <int NR>
-struct RowSmem {
-    static constexpr uint32_t E = 0, DEP = NR * 32768, K = NR * 65536, V = K + NR * 16384;
-    static constexpr uint32_t DF = V, AT = V + NR * 8192;          // reuse of the V chunk after dP
-    static constexpr uint32_t IMG = V + NR * 16384;                // Wfe^T sw, We sw, Wfe ns (2 KB each)
-    static constexpr uint32_t WD = IMG + 6144;                     // per-quadrant D partials [4][8][8]
-    static constexpr uint32_t CD = WD + 1024;                      // CTA D [64] (read by peers)
-    static constexpr uint32_t FD = CD + 256;                       // final D [64]
-    static constexpr uint32_t WDG = FD + 256;                      // per-warp dg [16][4]
-    static constexpr uint32_t G = WDG + 256;
-    static constexpr uint32_t LSE = G + 64;                        // [8 i][8 h]
-    static constexpr uint32_t MI = LSE + 256, MJ = MI + 16;
-    static constexpr uint32_t BAR = MJ + 64;                       // 9 mbarriers
-    static constexpr uint32_t TM = BAR + 72;
-    static constexpr uint32_t RD = TM + 24;                        // received D partials [16][64] f32
-    static constexpr uint32_t BYTES = RD + 4096 + 1024;
-    // in the E tile once it is dead: the CTA weight-grad partial, the pushed
-    // weight-grad slices and the pushed dq slices of the cluster
-    static constexpr uint32_t WP = E, RWP = E + 6400, RQ = E + 13056;
-    static constexpr uint32_t QPART = K;                           // 16 KB two-slot dq sums (K, V dead)
-};
-
-template <int NR>
-__global__ void __launch_bounds__(NTHR, NR == 1 ? 2 : 1)
-k_bwd_rows(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmDEp,
-           const __grid_constant__ CUtensorMap tmDE, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, BwdRowParams p) {
-    using S = RowSmem<NR>;
-    constexpr int TCN = tile_cols(NR), NE = 2 * NR;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
-    const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = W >> 2, t = tid & 31, c4 = t & 3, g8 = t >> 2;
-    const uint32_t rank = cluster_rank(), nclu = gridDim.x;
-    const int n = p.n;
-    const int j0 = blockIdx.x * TCN, i0 = blockIdx.y * TB, b = blockIdx.z;
-    const uint32_t bar_e = sbase + S::BAR, bar_dep = bar_e + 8, bar_kv = bar_e + 16, bar_film = bar_e + 24,
-                   bar_u = bar_e + 32, bar_de = bar_e + 40, bar_d = bar_e + 48, bar_wp = bar_e + 56,
-                   bar_q = bar_e + 64;
-    float *g = reinterpret_cast<float *>(sp + S::G);
-    float *lse = reinterpret_cast<float *>(sp + S::LSE);
-    uint8_t *mi = sp + S::MI, *mj = sp + S::MJ;
-    constexpr uint32_t TM_FILM = 0, TM_U = 64, TM_DE = 128, TM_COLS = 256;
-
-    if (tid == 0) {
-        mbar_init(bar_e, 1); mbar_init(bar_dep, 1); mbar_init(bar_kv, 1);
-        mbar_init(bar_film, 1); mbar_init(bar_u, 1); mbar_init(bar_de, 1);
-        mbar_init(bar_d, 1); mbar_init(bar_wp, 1); mbar_init(bar_q, 1);
-        fence_mbar_init();
-        mbar_expect_tx(bar_d, nclu * 64 * 4);
-        mbar_expect_tx(bar_wp, nclu * flat_slice(RPART, nclu, rank) * 16);
-        mbar_expect_tx(bar_q, nclu * rows_slice(1, nclu, rank) * 16);
-        mbar_expect_tx(bar_e, NR * 32768);
-        tma_load_5d(sbase + S::E, &tmE, bar_e, 0, i0 / 2, j0, 0, b);
-        mbar_expect_tx(bar_dep, NR * 32768);
-        tma_load_5d(sbase + S::DEP, &tmDEp, bar_dep, 0, i0 / 2, j0, 0, b);
-        mbar_expect_tx(bar_kv, NR * 32768);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            tma_load_3d(sbase + S::K + k * NR * 4096, &tmK, bar_kv, 64 * k, j0, b);
-            tma_load_3d(sbase + S::V + k * NR * 4096, &tmV, bar_kv, 64 * k, j0, b);
-        }
-    }
-    if (W == 0) {
-        tmem_alloc(sbase + S::TM, TM_COLS);
-        tmem_relinquish();
-    }
-    if (tid < 384) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.img);
-        const uint32_t img_off = (tid >> 7) == 0 ? IMG_WFE_T_SW : (tid >> 7) == 1 ? IMG_WE_SW : IMG_WFE_NS;
-        reinterpret_cast<uint4 *>(sp + S::IMG)[tid] = src[(img_off >> 4) + (tid & 127)];
-    }
-    if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
-    if (tid >= 32 && tid < 32 + TB) mi[tid - 32] = (i0 + tid - 32 < n) ? p.M[(size_t)b * n + i0 + tid - 32] : 0;
-    if (tid >= 64 && tid < 64 + TCN) mj[tid - 64] = (j0 + tid - 64 < n) ? p.M[(size_t)b * n + j0 + tid - 64] : 0;
-    if (tid >= 128 && tid < 192) {
-        const int x = tid - 128, il = x >> 3, h = x & 7;
-        lse[x] = (i0 + il < n) ? p.LSE[((size_t)b * NH + h) * n + i0 + il] : 0.f;
-    }
-    uint32_t qf[2][2][2], of[2][2][2];
-    load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
-    load_frags2(p.dO, b, n, i0, hq, g8, c4, of);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
-    const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
-    cluster_arrive();   // receive barriers of this CTA are armed
-
-    if (tid == 0) {
-        if (!mbar_wait(bar_e, 0)) flag_timeout(p.status);
-        tc_fence_after();
-        issue_pair_products<NR>(sbase + S::E, sbase + S::IMG, tmem + TM_FILM);
-        mma_commit(bar_film);
-        if (!mbar_wait(bar_dep, 0)) flag_timeout(p.status);
-        tc_fence_after();
-        issue_pair_products<NR>(sbase + S::DEP, sbase + S::IMG + 2048, tmem + TM_U);
-        mma_commit(bar_u);
-    }
-    __syncwarp();
-    if (!mbar_wait(bar_kv, 0)) flag_timeout(p.status);
-    float sv[2][4], da[2][4], av[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    warp_scores2<NR>(sbase + S::K, q, t, hq, qf, sv);
-    warp_scores2<NR>(sbase + S::V, q, t, hq, of, da);
-
-    if (!mbar_wait(bar_film, 0)) flag_timeout(p.status);
-    if (!mbar_wait(bar_u, 0)) flag_timeout(p.status);
-    tc_fence_after();
-    const float rs = rsqrtf((float)DH);
-    float gm[2][4];
-#pragma unroll
-    for (int e = 0; e < NE; ++e) {
-        const int jl = 32 * (e >> 1) + 8 * q + g8, il = 2 * c4 + (e & 1);
-        const bool valid = mi[il] && mj[jl];
-        float f0, f1, b0, b1, u0, u1;
-        tmem_ld2(tl + TM_FILM + 16 * e + 2 * hq, f0, f1);
-        tmem_ld2(tl + TM_FILM + 16 * e + NH + 2 * hq, b0, b1);
-        tmem_ld2(tl + TM_U + 16 * e + 2 * hq, u0, u1);
-        tmem_ld_wait();
-        const float fg[2] = {f0, f1}, fb[2] = {b0, b1}, fu[2] = {u0, u1};
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int h = 2 * hq + hh;
-            const float s = sv[hh][e] * rs;
-            const float gam = fg[hh] + g[h], bet = fb[hh] + g[NH + h];
-            av[hh][e] = valid ? exp2f((s * (1.f + gam) + bet - lse[il * 8 + h]) * LOG2E) : 0.f;
-            sv[hh][e] = s;
-            gm[hh][e] = gam;
-            da[hh][e] += fu[hh];
-        }
-    }
-    // D_ih = sum_j a dA: warp, CTA, cluster
-    float *wd = reinterpret_cast<float *>(sp + S::WD);
-    float *cd = reinterpret_cast<float *>(sp + S::CD);
-    float *fd = reinterpret_cast<float *>(sp + S::FD);
-#pragma unroll
-    for (int s = 0; s < 2; ++s)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float x = av[hh][s] * da[hh][s];
-            if (NR == 2) x += av[hh][2 + s] * da[hh][2 + s];
-            x += __shfl_xor_sync(0xffffffffu, x, 4);
-            x += __shfl_xor_sync(0xffffffffu, x, 8);
-            x += __shfl_xor_sync(0xffffffffu, x, 16);
-            if (g8 == 0) wd[(q * 8 + 2 * c4 + s) * 8 + 2 * hq + hh] = x;
-        }
-    __syncthreads();
-    if (tid < 64) cd[tid] = wd[tid] + wd[64 + tid] + wd[128 + tid] + wd[192 + tid];
-    __syncthreads();
-    cluster_wait();     // every peer's receive barriers are armed
-    push_rowvals_f32(sp, sbase, S::CD, S::RD, bar_d, tid, rank, nclu);
-    if (!mbar_wait(bar_d, 0)) flag_timeout(p.status);
-    combine_rowvals_f32(sp, S::RD, S::FD, tid, nclu);
-    __syncthreads();
-    if (tid < 64) {
-        const int il = tid >> 3, h = tid & 7;
-        if (rank == 0 && i0 + il < n) p.D[((size_t)b * NH + h) * n + i0 + il] = fd[tid];
-    }
-
-    // dS', df = [dgamma | dbeta], ds = dS'(1+gamma); df and a tiles for the tensor cores
-    float dgp[4] = {0.f, 0.f, 0.f, 0.f};   // dgamma h0, h1, dbeta h0, h1
-    const uint32_t L = 32 * q + t;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        if (e >= NE) {
-            da[0][e] = da[1][e] = 0.f;
-            continue;
-        }
-        const int il = 2 * c4 + (e & 1);
-        float dgam[2], dbet[2];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const float dsp = av[hh][e] * (da[hh][e] - fd[il * 8 + 2 * hq + hh]);
-            dgam[hh] = dsp * sv[hh][e];
-            dbet[hh] = dsp;
-            da[hh][e] = dsp * (1.f + gm[hh][e]);     // ds (unscaled)
-            dgp[hh] += dgam[hh];
-            dgp[2 + hh] += dbet[hh];
-        }
-        *reinterpret_cast<uint32_t *>(sp + S::DF + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(dgam[0], dgam[1]);
-        *reinterpret_cast<uint32_t *>(sp + S::DF + e * 4096 + ns16(L, NH + 2 * hq)) = pack_bf16(dbet[0], dbet[1]);
-        *reinterpret_cast<uint32_t *>(sp + S::AT + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(av[0][e], av[1][e]);
-        if (hq == 0) *reinterpret_cast<uint4 *>(sp + S::AT + e * 4096 + ns16(L, 8)) = make_uint4(0, 0, 0, 0);
-    }
-    // a and ds of the tile's pairs for the dk / dv pass: [b][h][i][j] bf16.
-    // Lanes t and t^4 hold neighbouring columns j; they swap one head so that
-    // each stores two columns of one head in a 4-byte word.
-    {
-        const bool odd = g8 & 1;
-#pragma unroll
-        for (int e = 0; e < NE; ++e) {
-            const float xa = __shfl_xor_sync(0xffffffffu, odd ? av[0][e] : av[1][e], 4);
-            const float xd = __shfl_xor_sync(0xffffffffu, odd ? da[0][e] : da[1][e], 4);
-            const int i = i0 + 2 * c4 + (e & 1), j = j0 + 32 * (e >> 1) + 8 * q + (g8 & ~1);
-            if (i < n && j < n) {
-                const size_t o = (((size_t)b * NH + 2 * hq + (odd ? 1 : 0)) * n + i) * p.npad + j;
-                *reinterpret_cast<uint32_t *>(p.Pa + o) = odd ? pack_bf16(xa, av[1][e]) : pack_bf16(av[0][e], xa);
-                *reinterpret_cast<uint32_t *>(p.Pds + o) = odd ? pack_bf16(xd, da[1][e]) : pack_bf16(da[0][e], xd);
-            }
-        }
-    }
-    float *wdg = reinterpret_cast<float *>(sp + S::WDG);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        float x = dgp[k];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        if (t == 0) wdg[W * 4 + k] = x;
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    const uint32_t idesc_de = idesc_bf16_f32(128, DE);
-    if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int ee = 0; ee < 2; ++ee)
-            mma_bf16_ss(tmem + TM_DE + 64 * ee, smem_desc(sbase + S::DF + ee * 4096, 128, 256, LAYOUT_NONE),
-                        smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_de, 0);
-        mma_commit(bar_de);
-    }
-    __syncwarp();
-
-    // dq partial = K^T ds^T (warp MMAs)
-    float qacc[2][2][4];
-    warp_contract2<NR>(sbase + S::K, q, t, hq, da, qacc);
-
-    // dWfe [64 c][16 k] and dWe^T [64 c][8 h] partials: warp W owns c in
-    // [16ct, 16ct+16) (ct = W%4) over k-range kr = W/4 of the CTA's pairs; the
-    // four k-ranges are added in a fixed order.
-    {
-        const int ct = W & 3, kr = W >> 2;
-        float wf[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        float we4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-        for (int kk = 4 * NR * kr; kk < 4 * NR * (kr + 1); ++kk) {
-            const int e = kk >> 3, L0 = 16 * (kk & 7);
-            const uint32_t row0 = tile_off<NR>(e) / 128 + L0;
-            const uint32_t arow = row0 + (t & 7) + ((t >> 4) & 1) * 8;
-            const uint32_t ach = 2 * ct + ((t >> 3) & 1);
-            uint32_t aE[4], aD[4], bF[4], bA0, bA1;
-            ldsm_x4_t(sbase + S::E + sw128(arow, ach), aE);
-            ldsm_x4_t(sbase + S::DEP + sw128(arow, ach), aD);
-            const uint32_t Lr = L0 + (t & 7) + ((t >> 3) & 1) * 8;
-            ldsm_x4_t(sbase + S::DF + e * 4096 + ns16(Lr, 8 * (t >> 4)), bF);
-            ldsm_x2_t(sbase + S::AT + e * 4096 + ns16(Lr, 0), bA0, bA1);
-            mma16816(wf[0], aE, bF[0], bF[1]);
-            mma16816(wf[1], aE, bF[2], bF[3]);
-            mma16816(we4, aD, bA0, bA1);
-        }
-        __syncthreads();   // the E tile is dead from here on
-        cluster_arrive();  // peers may now push into this CTA's E tile space
-        float *rp = reinterpret_cast<float *>(sp + S::WP);
-        for (int phase = 0; phase < 4; ++phase) {
-            if (kr == phase) {
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = 16 * ct + g8 + 8 * (e >> 1), k = nt * 8 + 2 * c4 + (e & 1);
-                        rp[c * NF + k] = (phase ? rp[c * NF + k] : 0.f) + wf[nt][e];
-                    }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = 16 * ct + g8 + 8 * (e >> 1), h = 2 * c4 + (e & 1);
-                    float *dst = rp + DE * NF + h * DE + c;
-                    *dst = (phase ? *dst : 0.f) + we4[e];
-                }
-            }
-            __syncthreads();
-        }
-        if (tid < NF) {
-            const int which = tid >> 3, h = tid & 7, hq2 = h >> 1, hh = h & 1;
-            float x = 0.f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) x += wdg[(4 * hq2 + k) * 4 + which * 2 + hh];
-            rp[DE * NF + NH * DE + tid] = x;
-        }
-    }
-    // sum the CTA partials over the cluster: one partial per (graph, row block)
-    __syncthreads();
-    cluster_wait();
-    push_flat(sp, sbase, S::WP, RPART, S::RWP, bar_wp, tid, rank, nclu);
-
-    // dE = dE' + df Wfe^T, written in place over the dE' tile, NR rounds of two MMAs
-    for (int round = 0; round < NR; ++round) {
-        if (!mbar_wait(bar_de, round)) flag_timeout(p.status);
-        tc_fence_after();
-#pragma unroll
-        for (int ee = 0; ee < 2; ++ee) {
-            const int e = 2 * round + ee;
-            float dv[16];
-            tmem_ld16(tl + TM_DE + 64 * ee + 16 * hq, dv);
-            tmem_ld_wait();
-            add_residual16(sp + S::DEP + tile_off<NR>(e) + L * 128, L, hq, dv);
-        }
-        if (round + 1 < NR) {
-            tc_fence_before();
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int ee = 0; ee < 2; ++ee)
-                    mma_bf16_ss(tmem + TM_DE + 64 * ee,
-                                smem_desc(sbase + S::DF + (2 * (round + 1) + ee) * 4096, 128, 256, LAYOUT_NONE),
-                                smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_de, 0);
-                mma_commit(bar_de);
-            }
-            __syncwarp();
-        }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-        tma_store_5d(&tmDE, sbase + S::DEP, 0, i0 / 2, j0, 0, b);
-        tma_store_commit();
-    }
-    // weight-grad partial of the cluster: this CTA's slice of the sum over peers
-    if (!mbar_wait(bar_wp, 0)) flag_timeout(p.status);
-    {
-        float *rp = p.rparts + (size_t)(blockIdx.z * gridDim.y + blockIdx.y) * RPART;
-        const uint32_t per4 = (RPART / 4 + nclu - 1) / nclu, slice = flat_slice(RPART, nclu, rank);
-        const float4 *rv = reinterpret_cast<const float4 *>(sp + S::RWP);
-        for (uint32_t k0 = tid; k0 < slice; k0 += NTHR) {
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (uint32_t pp = 0; pp < nclu; ++pp) {
-                const float4 v = rv[pp * per4 + k0];
-                a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
-            }
-            reinterpret_cast<float4 *>(rp)[rank * per4 + k0] = a;
-        }
-    }
-    // dq: reduce over the quadrant warps and the cluster
-    store_quadrant_part_2ph(sp, S::QPART, qacc, q, hq, t);
-    {
-        const uint32_t parts[1] = {S::QPART};
-        push_rows_partials<1, 2>(sp, sbase, parts, S::RQ, bar_q, tid, rank, nclu);
-        if (!mbar_wait(bar_q, 0)) flag_timeout(p.status);
-        __nv_bfloat16 *const outs[1] = {p.dQ};
-        const float sc[1] = {rs};
-        finish_rows_partials<1>(sp, S::RQ, tid, rank, nclu, outs, b, n, i0, sc);
-    }
-    if (tid == 0) tma_store_wait_read0();
-    tc_fence_before();
-    __syncthreads();
-    if (W == 0) tmem_dealloc(tmem, TM_COLS);
-}
 
 // ---------------------------------------------------------------- dk, dv pass
 // dk_j = sum_i ds_ij q_i / sqrt(dh) and dv_j = sum_i a_ij dO_i from the a and
@@ -631,66 +256,33 @@ __global__ void k_film_grads(const float *dg, int B, int dy, const __nv_bfloat16
 cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                               cudaStream_t st);
 
-template <int NR>
-static cudaError_t launch_bwd_nr(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
-                                 cudaStream_t st) {
-    constexpr int TCN = tile_cols(NR);
+// Row pair kernel, then dk / dv from its a and ds.
+cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
+                             cudaStream_t st) {
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e;
-        if ((e = cudaFuncSetAttribute(k_bwd_rows<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      RowSmem<NR>::BYTES)) != cudaSuccess)
-            return e;
-        if ((e = cudaFuncSetAttribute(k_bwd_rows<NR>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
-            cudaSuccess)
-            return e;
-        if ((e = cudaFuncSetAttribute(k_bwd_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, KvSmem::BYTES)) !=
-            cudaSuccess)
-            return e;
+        cudaError_t e = cudaFuncSetAttribute(k_bwd_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, KvSmem::BYTES);
+        if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    __nv_bfloat16 *dO = reinterpret_cast<__nv_bfloat16 *>(ws + W.dO);
-    __nv_bfloat16 *dQ = reinterpret_cast<__nv_bfloat16 *>(ws + W.dQ);
-    __nv_bfloat16 *dK = reinterpret_cast<__nv_bfloat16 *>(ws + W.dK);
-    __nv_bfloat16 *dV = reinterpret_cast<__nv_bfloat16 *>(ws + W.dV);
-    float *D = reinterpret_cast<float *>(ws + W.D);
-    const int nc = (d.n + TCN - 1) / TCN;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = nc;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(NTHR);
-    cfg.stream = st;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
     prof_mark(2, 0, st);
     {
         cudaError_t e = launch_bwd_stream(d, a, W, ws, g, st);
         if (e != cudaSuccess) return e;
     }
     prof_mark(2, 1, st);
-    {
-        CUtensorMap mPds, mPa, mQ, mDO;
-        if (!encode_p_map(&mPds, ws + W.Pds, d.B, d.n, W.npad) || !encode_p_map(&mPa, ws + W.Pa, d.B, d.n, W.npad) ||
-            !encode_node_map(&mQ, a.Q, d.B, d.n, KV_I) || !encode_node_map(&mDO, dO, d.B, d.n, KV_I))
-            return cudaErrorInvalidValue;
-        BwdKvParams p;
-        p.dK = dK;
-        p.dV = dV;
-        p.status = a.status;
-        p.n = d.n;
-        k_bwd_kv<<<dim3((d.n + KV_J - 1) / KV_J, d.B), KV_THR, KvSmem::BYTES, st>>>(mPds, mPa, mQ, mDO, p);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-}
-
-cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
-                             cudaStream_t st) {
-    return pick_nr(d.n) == 1 ? launch_bwd_nr<1>(d, a, W, ws, g, st) : launch_bwd_nr<2>(d, a, W, ws, g, st);
+    CUtensorMap mPds, mPa, mQ, mDO;
+    const __nv_bfloat16 *dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
+    if (!encode_p_map(&mPds, ws + W.Pds, d.B, d.n, W.npad) || !encode_p_map(&mPa, ws + W.Pa, d.B, d.n, W.npad) ||
+        !encode_node_map(&mQ, a.Q, d.B, d.n, KV_I) || !encode_node_map(&mDO, dO, d.B, d.n, KV_I))
+        return cudaErrorInvalidValue;
+    BwdKvParams p;
+    p.dK = reinterpret_cast<__nv_bfloat16 *>(ws + W.dK);
+    p.dV = reinterpret_cast<__nv_bfloat16 *>(ws + W.dV);
+    p.status = a.status;
+    p.n = d.n;
+    k_bwd_kv<<<dim3((d.n + KV_J - 1) / KV_J, d.B), KV_THR, KvSmem::BYTES, st>>>(mPds, mPa, mQ, mDO, p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_finish(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,

@@ -19,8 +19,10 @@
 //   pass 2: f and u again (E and dE' come back from L2: the chunks are walked
 //           in reverse), dS', dgamma, dbeta, ds; dE = dE' + df Wfe^T on the
 //           tensor cores, in place in shared memory, stored with TMA;
-//           dq += ds K (warp MMAs); dWfe, dWe, dg partials (warp MMAs); and
-//           a, ds of every pair stored in bf16 for the dk / dv kernel.
+//           dWfe += E^T df and dWe^T += dE'^T a on the tensor cores too
+//           (M = 64 channels, MN-major operands straight from the tiles,
+//           accumulated in TMEM over the row block); dq += ds K (warp MMAs);
+//           and a, ds of every pair stored in bf16 for the dk / dv kernel.
 // E and dE' leave HBM once, dE is written once.  No CTA waits for another.
 //
 // Warp roles as in the forward pair kernel: 16 compute warps (warp W reads
@@ -44,7 +46,7 @@ constexpr int BS_SLOTS = 12;
 constexpr uint32_t BS_SLOT = 16384;
 constexpr int BS_NFULL = 4;
 constexpr int BS_THR = NTHR + 64;
-constexpr int BS_KEEP_MAX_CHUNKS = 8;     // S and dP of up to 8 chunks (n <= 256) stay in TMEM
+constexpr int BS_KEEP_MAX_CHUNKS = 7;     // S and dP of up to 7 chunks (n <= 224) stay in TMEM
 
 struct BsSmem {
     static constexpr uint32_t IMG = BS_SLOTS * BS_SLOT;       // Wfe^T sw (FiLM), We sw (u), Wfe ns (dE): 2 KB each
@@ -58,15 +60,17 @@ struct BsSmem {
     static constexpr uint32_t TM = BAR + 8 * 12;
     static constexpr uint32_t STAB = TM + 16;                 // slot table [4 iterations][8] u8
     static constexpr uint32_t BYTES = STAB + 32 + 1024;
-    // in the drained ring at the end: dq quadrant sums [4][8][256] f32 (32 KB),
-    // then dWfe partials [4 kr][64 c][16 k] (16 KB) and dWe partials [4 kr][8 h][64 c] (8 KB)
-    static constexpr uint32_t QPART = 0, WFP = 32768, WEP = WFP + 16384;
+    // in the drained ring at the end: dq quadrant sums [4][8][256] f32 (32 KB)
+    static constexpr uint32_t QPART = 0;
 };
 constexpr int BB_FULL = 0, BB_FILM_FULL = 4, BB_FILM_EMPTY = 6, BB_DF_FULL = 8, BB_DE_FULL = 9,
               BB_STAGE_DONE = 10;
 
-// TMEM: FiLM 0..63 and u 64..127 (two buffers each), dE 128..255, kept S / dP from 256 (32 per chunk)
-constexpr uint32_t BS_TM_COLS = 512, BS_TM_FILM = 0, BS_TM_U = 64, BS_TM_DE = 128, BS_TM_KEEP = 256;
+// TMEM: FiLM 0..63 and u 64..127 (two buffers each), dE 128..255, kept S / dP
+// 256..479 (32 per chunk), dWfe [64 c][16 k] at 480, dWe^T [64 c][16 h] at 496
+// (M = 64 accumulators: row m in lane m%16 + 32(m/16))
+constexpr uint32_t BS_TM_COLS = 512, BS_TM_FILM = 0, BS_TM_U = 64, BS_TM_DE = 128, BS_TM_KEEP = 256,
+                   BS_TM_WFE = 480, BS_TM_WE = 496;
 
 struct BwdStreamParams {
     const __nv_bfloat16 *Q, *dO;
@@ -142,6 +146,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         // ================= MMA issuer
         if (t == 0) {
             const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_d = idesc_bf16_f32(128, DE);
+            const uint32_t idesc_w = idesc_bf16_f32_mn(64, NF);
             auto issue_fu = [&](int it) {
                 tc_fence_after();
 #pragma unroll
@@ -160,12 +165,28 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
                 mma_commit(bar(BB_FILM_FULL + (it & 1)));
             };
-            auto issue_de = [&]() {
+            auto issue_de = [&](int it) {
                 tc_fence_after();
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
                     mma_bf16_ss(tmem + BS_TM_DE + 64 * e, smem_desc(sbase + S::DF + e * 4096, 128, 256, LAYOUT_NONE),
                                 smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_d, 0);
+                // dWfe [c][k] += sum_pairs E[pair][c] df[pair][k], dWe^T [c][h] += sum_pairs dE'[pair][c] a[pair][h]:
+                // A = the pair tile read MN-major (64 c per 128-byte swizzled row, 8-row groups 1024 B
+                // apart), B = the df / a tile read MN-major (8 x 8 core matrices: 128 B along N,
+                // 256 B along K); 16 pairs per MMA
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const uint32_t te = slot_addr(it, e), td = slot_addr(it, 2 + e);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t acc = (it > nch || e > 0 || ks > 0) ? 1u : 0u;
+                        mma_bf16_ss(tmem + BS_TM_WFE, smem_desc(te + ks * 2048, 16, 1024, LAYOUT_SW128),
+                                    smem_desc(sbase + S::DF + e * 4096 + ks * 512, 256, 128, LAYOUT_NONE), idesc_w, acc);
+                        mma_bf16_ss(tmem + BS_TM_WE, smem_desc(td + ks * 2048, 16, 1024, LAYOUT_SW128),
+                                    smem_desc(sbase + S::AT + e * 4096 + ks * 512, 256, 128, LAYOUT_NONE), idesc_w, acc);
+                    }
+                }
                 mma_commit(bar(BB_DE_FULL));
             };
             // issue whichever product is ready first: FiLM/u of the next chunk
@@ -175,17 +196,17 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             uint32_t polls = 0;
             while (next_fu < nit || next_de < nit) {
                 bool progressed = false;
-                if (next_fu < nit && mbar_try_wait(bar(BB_FULL + next_fu % BS_NFULL), (next_fu / BS_NFULL) & 1) &&
-                    (next_fu < 2 || mbar_try_wait(bar(BB_FILM_EMPTY + (next_fu & 1)), ((next_fu - 2) >> 1) & 1))) {
+                if (next_fu < nit && mbar_test_wait(bar(BB_FULL + next_fu % BS_NFULL), (next_fu / BS_NFULL) & 1) &&
+                    (next_fu < 2 || mbar_test_wait(bar(BB_FILM_EMPTY + (next_fu & 1)), ((next_fu - 2) >> 1) & 1))) {
                     issue_fu(next_fu++);
                     progressed = true;
                 }
-                if (next_de < nit && next_de < next_fu && mbar_try_wait(bar(BB_DF_FULL), (next_de - nch) & 1)) {
-                    issue_de();
+                if (next_de < nit && next_de < next_fu && mbar_test_wait(bar(BB_DF_FULL), (next_de - nch) & 1)) {
+                    issue_de(next_de);
                     ++next_de;
                     progressed = true;
                 }
-                if (!progressed && ++polls > (1u << 26)) {
+                if (!progressed && ++polls > (1u << 28)) {
                     flag_timeout(p.status);
                     break;
                 }
@@ -276,15 +297,11 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         }
         float dsum[2][2] = {{0.f, 0.f}, {0.f, 0.f}};     // running D partial, then the final D [e][hh]
         float qacc[2][2][4];
-        float wf[2][4], we4[4];
         float dgp[4] = {0.f, 0.f, 0.f, 0.f};              // dgamma h0, h1, dbeta h0, h1
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            wf[0][x] = wf[1][x] = we4[x] = 0.f;
+        for (int x = 0; x < 4; ++x)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) qacc[hh][0][x] = qacc[hh][1][x] = 0.f;
-        }
-        const int ct = W & 3, kr = W >> 2;
 
         for (int it = 0; it < nit; ++it) {
             const int c = chunk_of(it), j0 = 32 * c;
@@ -396,6 +413,12 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             }
             av[0][2] = av[0][3] = av[1][2] = av[1][3] = 0.f;
             da[0][2] = da[0][3] = da[1][2] = da[1][3] = 0.f;
+            // df and a of this warp's rows are in place: the MMA warp issues dE and
+            // the weight-gradient products once all 16 warps have arrived
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (t == 0) mbar_arrive(bar(BB_DF_FULL));
+
             // a and ds of the chunk's pairs for the dk / dv pass: [b][h][i][j] bf16.
             // Lanes t and t^4 hold neighbouring columns j; they swap one head so that
             // each stores two columns of one head in a 4-byte word.
@@ -414,31 +437,9 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     }
                 }
             }
-            fence_proxy_async_smem();
-            named_bar_sync(1, NTHR);          // df and a tiles complete
-            if (t == 0) mbar_arrive(bar(BB_DF_FULL));
 
-            // ---------------- dq += ds K (warp MMAs; overlaps the dE MMAs)
+            // ---------------- dq += ds K (warp MMAs; overlaps the tensor-core products)
             warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, da, qacc);
-
-            // ---------------- dWfe [64 c][16 k] and dWe^T [64 c][8 h] partials: warp W owns
-            // c in [16ct, 16ct+16) over the k-range kr of the chunk's pairs
-#pragma unroll 2
-            for (int kk = 4 * kr; kk < 4 * (kr + 1); ++kk) {
-                const int e = kk >> 3, L0 = 16 * (kk & 7);
-                const uint32_t arow = L0 + (t & 7) + ((t >> 4) & 1) * 8;
-                const uint32_t ach = 2 * ct + ((t >> 3) & 1);
-                uint32_t aE[4], aD[4], bF[4], bA0, bA1;
-                ldsm_x4_t(slot_addr(it, e) + sw128(arow, ach), aE);
-                ldsm_x4_t(slot_addr(it, 2 + e) + sw128(arow, ach), aD);
-                const uint32_t Lr = L0 + (t & 7) + ((t >> 3) & 1) * 8;
-                ldsm_x4_t(sbase + S::DF + e * 4096 + ns16(Lr, 8 * (t >> 4)), bF);
-                ldsm_x2_t(sbase + S::AT + e * 4096 + ns16(Lr, 0), bA0, bA1);
-                mma16816(wf[0], aE, bF[0], bF[1]);
-                mma16816(wf[1], aE, bF[2], bF[3]);
-                mma16816(we4, aD, bA0, bA1);
-            }
-            named_bar_sync(1, NTHR);          // every warp is done reading dE', df, a of this chunk
 
             // ---------------- dE = dE' + df Wfe^T, in place (the TMA warp stores it)
             if (!mbar_wait(bar(BB_DE_FULL), (it - nch) & 1)) flag_timeout(p.status);
@@ -467,17 +468,6 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             if (t == 0) wdg[W * 4 + k] = x;
         }
         store_quadrant_part(sp, S::QPART, qacc, q, hq, t);
-        {
-            float *wfp = reinterpret_cast<float *>(sp + S::WFP) + kr * (DE * NF);
-            float *wep = reinterpret_cast<float *>(sp + S::WEP) + kr * (NH * DE);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int cc = 16 * ct + g8 + 8 * (e >> 1);
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) wfp[cc * NF + nt * 8 + 2 * c4 + (e & 1)] = wf[nt][e];
-                wep[(2 * c4 + (e & 1)) * DE + cc] = we4[e];
-            }
-        }
         named_bar_sync(1, NTHR);
         const float *part = reinterpret_cast<const float *>(sp + S::QPART);
         for (int x = tid; x < TB * HD / 2; x += NTHR) {
@@ -491,24 +481,32 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             }
             *reinterpret_cast<uint32_t *>(p.dQ + ((size_t)b * n + i0 + il) * HD + d) = pack_bf16(o0 * rs, o1 * rs);
         }
+        // weight-gradient partials of the row block: dWfe [c][k] and dWe^T [c][h]
+        // from the M = 64 TMEM accumulators (row c in lane c%16 of quadrant c/16),
+        // dg from the per-warp sums
         float *rp = p.rparts + (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * RPART;
-        const float *wfp = reinterpret_cast<const float *>(sp + S::WFP);
-        const float *wep = reinterpret_cast<const float *>(sp + S::WEP);
-        for (int x = tid; x < DE * NF + NH * DE + NF; x += NTHR) {
-            float v = 0.f;
-            if (x < DE * NF) {
+        tc_fence_after();
+        if (hq < 2) {
+            float v[16];
+            tmem_ld16(tl + (hq == 0 ? BS_TM_WFE : BS_TM_WE), v);
+            tmem_ld_wait();
+            if (t < 16) {
+                const int c = 16 * q + t;
+                if (hq == 0) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) v += wfp[k * DE * NF + x];
-            } else if (x < DE * NF + NH * DE) {
-                const int y2 = x - DE * NF;
+                    for (int k = 0; k < NF; ++k) rp[c * NF + k] = v[k];
+                } else {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) v += wep[k * NH * DE + y2];
-            } else {
-                const int y2 = x - DE * NF - NH * DE, which = y2 >> 3, h = y2 & 7, hq2 = h >> 1, hh = h & 1;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) v += wdg[(4 * hq2 + k) * 4 + which * 2 + hh];
+                    for (int h = 0; h < NH; ++h) rp[DE * NF + h * DE + c] = v[h];
+                }
             }
-            rp[x] = v;
+        }
+        if (tid < NF) {
+            const int which = tid >> 3, h = tid & 7, hq2 = h >> 1, hh = h & 1;
+            float v = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v += wdg[(4 * hq2 + k) * 4 + which * 2 + hh];
+            rp[DE * NF + NH * DE + tid] = v;
         }
     }
     tc_fence_before();

@@ -9,11 +9,7 @@ namespace eaga {
 namespace fast {
 
 constexpr int DE = 64, NH = 8, DH = 32, HD = 256, NF = 16;
-constexpr int TB = 8;            // pair tile: 8 "own" rows x 32*NR "cluster" rows
-// NR = 1: 32 cluster rows per CTA (n <= 512; two CTAs fit on an SM);
-// NR = 2: 64 cluster rows per CTA (n <= 1024).
-__host__ __device__ constexpr int tile_cols(int NR) { return 32 * NR; }
-inline int pick_nr(int n) { return n <= 512 ? 1 : 2; }
+constexpr int TB = 8;            // query rows per pair-kernel CTA (one row block)
 // Streaming multiprocessors of the current device (cached per process).
 inline int sm_count() {
     static int cached = 0;
@@ -96,34 +92,15 @@ bool encode_p_map(CUtensorMap *m, const void *base, int B, int n, int npad);
 
 
 // ------------------------------------------------------------------ device pieces
-// The pair kernels run 16 warps.  Warp W owns TMEM lane quadrant q = W % 4
-// (the pairs of chunk rows 8q+t/4 (+32 when NR = 2)) and the two heads
-// 2hq, 2hq+1 with hq = W / 4.  Tile (r,s) of an [s][32NR][4][64] pair tile
-// holds 128 pairs: chunk rows 32r..32r+31 with own-row parity s.
+// The pair kernels run 16 compute warps.  Warp W owns TMEM lane quadrant
+// q = W % 4 (the pairs of chunk columns 8q + t/4) and the two heads 2hq,
+// 2hq+1 with hq = W / 4.  A chunk is 32 columns j of the CTA's 8 rows i, held
+// as two [32 j][4 ic][64 c] tiles (i = 2ic + s, one per parity s): 256 pairs.
+// The helpers keep an NR parameter: NR = 1 is the 32-column chunk.
 namespace dev {
 using namespace sm100;
 constexpr int NWARP = 16, NTHR = 512;
 constexpr float LOG2E = 1.4426950408889634f;
-
-template <int NR>
-__device__ __forceinline__ uint32_t tile_off(int e) {   // byte offset of pair group e = 2r + s
-    return (e & 1) * NR * 16384 + (e >> 1) * 16384;
-}
-
-// One thread issues D[e] (+)= tile(e) x B for the 2NR pair groups of a pair
-// tile (FiLM with B = Wfe^T, u with B = We), K = 64 in four steps.
-template <int NR>
-__device__ __forceinline__ void issue_pair_products(uint32_t tile, uint32_t bimg, uint32_t tm_col) {
-    const uint32_t idesc = idesc_bf16_f32(128, NF);
-#pragma unroll
-    for (int e = 0; e < 2 * NR; ++e) {
-        const uint32_t a0 = tile + tile_off<NR>(e);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tm_col + 16 * e, smem_desc(a0 + kk * 32, 16, 1024, LAYOUT_SW128),
-                        smem_desc(bimg + kk * 32, 16, 1024, LAYOUT_SW128), idesc, kk > 0);
-    }
-}
 
 // B-operand fragments of 8 node rows base+g8 for heads 2hq, 2hq+1 (zero past n).
 __device__ __forceinline__ void load_frags2(const __nv_bfloat16 *X, int b, int n, int base, int hq, int g8, int c4,
@@ -212,279 +189,6 @@ __device__ __forceinline__ void store_quadrant_part(uint8_t *sp, uint32_t s_part
                 const int d = (2 * hq + hh) * DH + mt * 16 + g8 + 8 * (e >> 1), il = 2 * c4 + (e & 1);
                 dst[il * HD + d] = acc[hh][mt][e];
             }
-}
-
-// Cluster-wide sum of NB quadrant buffers (each [4][8][256] fp32, written by
-// store_quadrant_part on every CTA of the cluster): this CTA reduces its
-// 1/nclu slice, one quadrant per lane, all peer loads in flight, quadrants
-// combined by shuffles in a fixed order.  Writes rows base+il < n of out[k]
-// ([B,n,256] bf16) times scale[k].  Starts with a cluster barrier; ends with
-// cluster_arrive(): the caller executes cluster_wait() before its shared
-// memory can be reused or the CTA exits.
-template <int NB>
-__device__ __forceinline__ void cluster_reduce_rows(uint32_t sbase, const uint32_t (&s_part)[NB], int tid,
-                                                    uint32_t rank, uint32_t nclu, __nv_bfloat16 *const (&out)[NB],
-                                                    int b, int n, int base, const float (&scale)[NB]) {
-    cluster_sync();
-    constexpr int G = TB * HD / 4;                       // float4 groups per buffer
-    const int per = (NB * G + nclu - 1) / nclu;
-    const int lo = rank * per, hi = min((int)(rank + 1) * per, NB * G);
-    const int q = tid & 3;
-    for (int x0 = lo; x0 < hi; x0 += NTHR / 4) {
-        const int x = x0 + (tid >> 2);
-        const bool act = x < hi;
-        const int k = act ? x / G : 0, gq = act ? x % G : 0;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (act) {
-            const uint32_t off = s_part[k] + (q * G + gq) * 16;
-            for (uint32_t p0 = 0; p0 < nclu; p0 += 4) {
-                float4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    v[u] = (p0 + u < nclu) ? ld_peer_f32x4(map_peer(sbase + off, p0 + u)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    a.x += v[u].x; a.y += v[u].y; a.z += v[u].z; a.w += v[u].w;
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 1; o < 4; o <<= 1) {
-            a.x += __shfl_xor_sync(0xffffffffu, a.x, o);
-            a.y += __shfl_xor_sync(0xffffffffu, a.y, o);
-            a.z += __shfl_xor_sync(0xffffffffu, a.z, o);
-            a.w += __shfl_xor_sync(0xffffffffu, a.w, o);
-        }
-        if (act && q == 0) {
-            const int il = (gq * 4) / HD, d = (gq * 4) % HD;
-            if (base + il < n) {
-                const float sc = scale[k];
-                __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(out[k] + ((size_t)b * n + base + il) * HD + d);
-                o2[0] = __floats2bfloat162_rn(a.x * sc, a.y * sc);
-                o2[1] = __floats2bfloat162_rn(a.z * sc, a.w * sc);
-            }
-        }
-    }
-    cluster_arrive();
-}
-
-// Cluster-wide combine of per-CTA (row, head) values: 64 entries, this CTA
-// reads entry x from every peer (thread = (x, peer group of 8)) and combines
-// in a fixed order.  Mode 0: softmax (max, sum) pairs at s_in (8 bytes per
-// entry) -> (max, 1/sum) at s_out; mode 1: sums of one float at s_in -> s_out.
-template <int MODE>
-__device__ __forceinline__ void cluster_combine64(uint8_t *sp, uint32_t sbase, uint32_t s_in, uint32_t s_out,
-                                                  int tid, uint32_t nclu) {
-    const int x = tid >> 3, p = tid & 7;      // 64 entries x 8 lanes
-    constexpr uint32_t STRIDE = MODE == 0 ? 8 : 4;
-    float m0 = -INFINITY, l0 = 0.f, m1 = -INFINITY, l1 = 0.f;
-    if ((uint32_t)p < nclu) {
-        const uint32_t a = map_peer(sbase + s_in + x * STRIDE, p);
-        if (MODE == 0) { m0 = ld_peer_f32(a); l0 = ld_peer_f32(a + 4); } else { l0 = ld_peer_f32(a); }
-    }
-    if ((uint32_t)(p + 8) < nclu) {
-        const uint32_t a = map_peer(sbase + s_in + x * STRIDE, p + 8);
-        if (MODE == 0) { m1 = ld_peer_f32(a); l1 = ld_peer_f32(a + 4); } else { l1 = ld_peer_f32(a); }
-    }
-    if (MODE == 0) {
-        float m = fmaxf(m0, m1);
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
-        if (m != -INFINITY) {
-            if (m0 != -INFINITY) l += l0 * exp2f((m0 - m) * LOG2E);
-            if (m1 != -INFINITY) l += l1 * exp2f((m1 - m) * LOG2E);
-        }
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (p == 0) {
-            float *fo = reinterpret_cast<float *>(sp + s_out);
-            fo[x * 2] = m;
-            fo[x * 2 + 1] = l;   // sum (the caller turns it into 1/sum)
-        }
-    } else {
-        float l = l0 + l1;
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (p == 0) reinterpret_cast<float *>(sp + s_out)[x] = l;
-    }
-}
-
-// ---- push-based cluster exchanges (no cluster barrier on the critical path)
-// Every CTA initialises its receive mbarriers, arms them with the bytes its
-// peers will send (expect_tx), then cluster_arrive(); the matching
-// cluster_wait() precedes its first push.  Each receiver waits only on its
-// own mbarrier, so no CTA ever reads a peer's shared memory.
-
-constexpr uint32_t RECV_ROWVALS_BYTES = 16 * 64 * 8;             // [16 peers][64 entries][8 bytes]
-__host__ __device__ constexpr uint32_t recv_rows_bytes(int NB) {  // [nclu][per] float4, per = ceil(NB*512/nclu)
-    return (uint32_t)(NB * 512 + 16) * 16;
-}
-__host__ __device__ inline uint32_t rows_per(int NB, uint32_t nclu) { return (NB * 512 + nclu - 1) / nclu; }
-__host__ __device__ inline uint32_t rows_slice(int NB, uint32_t nclu, uint32_t r) {
-    const int per = (int)rows_per(NB, nclu), lo = (int)r * per, hi = min(NB * 512, lo + per);
-    return hi > lo ? (uint32_t)(hi - lo) : 0u;
-}
-
-// Push this CTA's 64 (row, head) values (v0, v1) from s_src ([64][2] f32) to
-// slot `rank` of every CTA's receive buffer s_recv.
-__device__ __forceinline__ void push_rowvals(uint8_t *sp, uint32_t sbase, uint32_t s_src, uint32_t s_recv,
-                                             uint32_t bar, int tid, uint32_t rank, uint32_t nclu) {
-    const int x = tid >> 3, p0 = tid & 7;
-    const float *src = reinterpret_cast<const float *>(sp + s_src);
-    const float v0 = src[x * 2], v1 = src[x * 2 + 1];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const uint32_t p = p0 + 8 * u;
-        if (p < nclu)
-            st_async_v2(map_peer(sbase + s_recv + (rank * 64 + x) * 8, p), v0, v1, map_peer(bar, p));
-    }
-}
-
-// Combine the nclu received copies of the 64 entries in a fixed order.
-// MODE 0: softmax (max, sum) pairs -> (max, sum) at s_out; MODE 1: sums of v0.
-template <int MODE>
-__device__ __forceinline__ void combine_rowvals(uint8_t *sp, uint32_t s_recv, uint32_t s_out, int tid,
-                                                uint32_t nclu) {
-    const int x = tid >> 3, p = tid & 7;
-    const float *rv = reinterpret_cast<const float *>(sp + s_recv);
-    float m0 = -INFINITY, l0 = 0.f, m1 = -INFINITY, l1 = 0.f;
-    if ((uint32_t)p < nclu) { m0 = rv[(p * 64 + x) * 2]; l0 = rv[(p * 64 + x) * 2 + 1]; }
-    if ((uint32_t)(p + 8) < nclu) { m1 = rv[((p + 8) * 64 + x) * 2]; l1 = rv[((p + 8) * 64 + x) * 2 + 1]; }
-    float *fo = reinterpret_cast<float *>(sp + s_out);
-    if (MODE == 0) {
-        float m = fmaxf(m0, m1);
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
-        if (m != -INFINITY) {
-            if (m0 != -INFINITY) l += l0 * exp2f((m0 - m) * LOG2E);
-            if (m1 != -INFINITY) l += l1 * exp2f((m1 - m) * LOG2E);
-        }
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (p == 0) { fo[x * 2] = m; fo[x * 2 + 1] = l; }
-    } else {
-        float l = ((uint32_t)p < nclu ? m0 : 0.f) + ((uint32_t)(p + 8) < nclu ? m1 : 0.f);
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (p == 0) fo[x] = l;
-    }
-}
-
-// Sum the NSLOT slot partials of NB [NSLOT][8][256] fp32 buffers and push
-// float4 group gg (over the NB buffers) to its owner rank gg / per, slot
-// rank * per + (gg - owner * per) of the owner's receive buffer.
-template <int NB, int NSLOT = 4>
-__device__ __forceinline__ void push_rows_partials(uint8_t *sp, uint32_t sbase, const uint32_t (&s_part)[NB],
-                                                   uint32_t s_recv, uint32_t bar, int tid, uint32_t rank,
-                                                   uint32_t nclu) {
-    constexpr int G = TB * HD / 4;
-    const uint32_t per = rows_per(NB, nclu);
-    for (int gg = tid; gg < NB * G; gg += NTHR) {
-        const int k = gg / G, g = gg % G;
-        const float4 *pt = reinterpret_cast<const float4 *>(sp + s_part[k]);
-        float4 v = pt[g];
-#pragma unroll
-        for (int qq = 1; qq < NSLOT; ++qq) {
-            const float4 w = pt[qq * G + g];
-            v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-        }
-        const uint32_t owner = gg / per, slot = rank * per + (gg - owner * per);
-        st_async_v4(map_peer(sbase + s_recv + slot * 16, owner), v, map_peer(bar, owner));
-    }
-}
-
-// The warps' [8 i][256 d] contributions summed over the 4 quadrants in two
-// fixed-order phases into a [2][8][256] fp32 buffer (16 KB): quadrants 0,1
-// write slots 0,1, then quadrants 2,3 add into them.  All threads call it.
-__device__ __forceinline__ void store_quadrant_part_2ph(uint8_t *sp, uint32_t s_part, const float (&acc)[2][2][4],
-                                                        int q, int hq, int t) {
-    const int c4 = t & 3, g8 = t >> 2;
-    float *dst = reinterpret_cast<float *>(sp + s_part) + (q & 1) * TB * HD;
-    for (int phase = 0; phase < 2; ++phase) {
-        if ((q >> 1) == phase) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int d = (2 * hq + hh) * DH + mt * 16 + g8 + 8 * (e >> 1), il = 2 * c4 + (e & 1);
-                        float *x = dst + il * HD + d;
-                        *x = (phase ? *x : 0.f) + acc[hh][mt][e];
-                    }
-        }
-        __syncthreads();
-    }
-}
-
-// Push 64 per-(row, head) floats src[x] to slot `rank` of every CTA's
-// receive buffer s_recv ([16][64] f32).
-__device__ __forceinline__ void push_rowvals_f32(uint8_t *sp, uint32_t sbase, uint32_t s_src, uint32_t s_recv,
-                                                 uint32_t bar, int tid, uint32_t rank, uint32_t nclu) {
-    const int x = tid >> 3, p0 = tid & 7;
-    const float v = reinterpret_cast<const float *>(sp + s_src)[x];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const uint32_t pp = p0 + 8 * u;
-        if (pp < nclu) st_async_f32(map_peer(sbase + s_recv + (rank * 64 + x) * 4, pp), v, map_peer(bar, pp));
-    }
-}
-
-// Sum of the nclu received copies of 64 floats ([16][64] f32), fixed order.
-__device__ __forceinline__ void combine_rowvals_f32(uint8_t *sp, uint32_t s_recv, uint32_t s_out, int tid,
-                                                    uint32_t nclu) {
-    const int x = tid >> 3, pp = tid & 7;
-    const float *rv = reinterpret_cast<const float *>(sp + s_recv);
-    float l = ((uint32_t)pp < nclu ? rv[pp * 64 + x] : 0.f) + ((uint32_t)(pp + 8) < nclu ? rv[(pp + 8) * 64 + x] : 0.f);
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (pp == 0) reinterpret_cast<float *>(sp + s_out)[x] = l;
-}
-
-// Push a flat fp32 array of `count` floats (count % 4 == 0) to its owners:
-// float4 group g goes to rank g / per4 (per4 = ceil(count/4 / nclu)), slot
-// rank * per4 + (g - owner * per4) of the owner's receive buffer.
-__device__ __forceinline__ void push_flat(uint8_t *sp, uint32_t sbase, uint32_t s_src, int count, uint32_t s_recv,
-                                          uint32_t bar, int tid, uint32_t rank, uint32_t nclu) {
-    const int g4 = count / 4;
-    const uint32_t per = (g4 + nclu - 1) / nclu;
-    const float4 *src = reinterpret_cast<const float4 *>(sp + s_src);
-    for (int g = tid; g < g4; g += NTHR) {
-        const uint32_t owner = g / per, slot = rank * per + (g - owner * per);
-        st_async_v4(map_peer(sbase + s_recv + slot * 16, owner), src[g], map_peer(bar, owner));
-    }
-}
-__host__ __device__ inline uint32_t flat_slice(int count, uint32_t nclu, uint32_t r) {
-    const int g4 = count / 4, per = (g4 + (int)nclu - 1) / (int)nclu, lo = (int)r * per, hi = min(g4, lo + per);
-    return hi > lo ? (uint32_t)(hi - lo) : 0u;
-}
-
-// Owner side: after its receive mbarrier completed, sum the nclu pushed
-// copies of its groups (fixed order) and write rows base+il < n of out[k].
-template <int NB>
-__device__ __forceinline__ void finish_rows_partials(uint8_t *sp, uint32_t s_recv, int tid, uint32_t rank,
-                                                     uint32_t nclu, __nv_bfloat16 *const (&out)[NB], int b, int n,
-                                                     int base, const float (&scale)[NB]) {
-    constexpr int G = TB * HD / 4;
-    const uint32_t per = rows_per(NB, nclu), slice = rows_slice(NB, nclu, rank);
-    const float4 *rv = reinterpret_cast<const float4 *>(sp + s_recv);
-    for (uint32_t k0 = tid; k0 < slice; k0 += NTHR) {
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (uint32_t p = 0; p < nclu; ++p) {
-            const float4 v = rv[p * per + k0];
-            a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
-        }
-        const int gg = rank * per + k0, k = gg / G, g = gg % G;
-        const int il = (g * 4) / HD, d = (g * 4) % HD;
-        if (base + il < n) {
-            const float sc = scale[k];
-            __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(out[k] + ((size_t)b * n + base + il) * HD + d);
-            o2[0] = __floats2bfloat162_rn(a.x * sc, a.y * sc);
-            o2[1] = __floats2bfloat162_rn(a.z * sc, a.w * sc);
-        }
-    }
 }
 
 // In-place residual on a 128-byte swizzled pair row: row[c] += dv[c - 16hq]

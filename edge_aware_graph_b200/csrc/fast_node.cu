@@ -1,12 +1,9 @@
-// Node-side matrix products of the layer on the tensor cores (bf16 operands,
-// fp32 accumulation), one kernel template for all of them:
-//   QKV      [Q|K|V] = X [Wq|Wk|Wv] + b; rows of masked nodes written as zero
-//   out-proj X' = X + M (O Wo + bo)
-//   dO       dO = M (dX' Wo^T)
-//   dX       dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T
-//   dW       X^T dQ, X^T dK, X^T dV, O^T dX' as split-K fp32 partials
-// 64x64 output tile per CTA, 4 warps of 32x32, K in steps of 32 through a
-// two-stage cp.async pipeline, 16-byte swizzled shared-memory rows.
+// Weight gradients of the node projections on warp MMAs (bf16 operands, fp32
+// accumulation): X^T dQ, X^T dK, X^T dV and O^T dX' (O is zero on masked
+// rows) as split-K fp32 partials over row chunks, summed in a fixed order by
+// the finishing kernel.  64x64 output tile per CTA, 4 warps of 32x32, K (the
+// node rows) in steps of 32 through a two-stage cp.async pipeline, 16-byte
+// swizzled shared-memory rows.
 #include "fast.h"
 #include "fast_common.cuh"
 
@@ -16,18 +13,11 @@ namespace fast {
 using namespace sm100;
 
 constexpr int GBM = 64, GBN = 64, GBK = 32, GTHR = 128;
-enum GemmMode { GM_QKV = 0, GM_OUT = 1, GM_DO = 2, GM_DX = 3, GM_WGRAD = 4 };
-
 struct GemmParams {
     const __nv_bfloat16 *A[3];       // per K-segment; [M,K] (or [K,M] when A is transposed)
-    const __nv_bfloat16 *B[3];       // per output matrix (QKV, wgrad) or per K-segment (dX)
-    const __nv_bfloat16 *bias[3];
-    __nv_bfloat16 *C[3];             // bf16 outputs [M, Nb]
+    const __nv_bfloat16 *B[3];       // per output matrix
     float *P[3];                     // fp32 split-K partials [splits][M, Nb]
-    const __nv_bfloat16 *R;          // residual [M, Nb]
-    const uint8_t *mask;             // [M] (rows)
     int M, K, Nb, lda, ldb, nseg, kchunk;
-    int mode;
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool pred) {
@@ -52,8 +42,8 @@ __global__ void __launch_bounds__(GTHR) k_node_gemm(GemmParams p) {
     const int n0g = blockIdx.x * GBN, m0 = blockIdx.y * GBM;
     const int which = n0g / p.Nb, n0 = n0g % p.Nb;
     const int wm = (w >> 1) * 32, wn = (w & 1) * 32;
-    const int kbeg = p.mode == GM_WGRAD ? blockIdx.z * p.kchunk : 0;
-    const int kend = p.mode == GM_WGRAD ? min(p.K, kbeg + p.kchunk) : p.K;
+    const int kbeg = blockIdx.z * p.kchunk;
+    const int kend = min(p.K, kbeg + p.kchunk);
     float acc[2][4][4];
 #pragma unroll
     for (int a = 0; a < 2; ++a)
@@ -150,91 +140,13 @@ __global__ void __launch_bounds__(GTHR) k_node_gemm(GemmParams p) {
                 const int row = m0 + wm + mt * 16 + (t >> 2) + hh * 8;
                 const int col = n0 + wn + nt * 8 + (t & 3) * 2;
                 if (row >= p.M) continue;
-                float v0 = acc[mt][nt][hh * 2], v1 = acc[mt][nt][hh * 2 + 1];
                 const size_t o = (size_t)row * p.Nb + col;
-                if (p.mode == GM_WGRAD) {
-                    float *P = p.P[which] + (size_t)blockIdx.z * p.M * p.Nb;
-                    *reinterpret_cast<float2 *>(P + o) = make_float2(v0, v1);
-                    continue;
-                }
-                const bool mk = p.mask[row] != 0;
-                __nv_bfloat162 out;
-                if (p.mode == GM_QKV || p.mode == GM_OUT) {
-                    const float2 bb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p.bias[which] + col));
-                    v0 += bb.x;
-                    v1 += bb.y;
-                }
-                if (p.mode == GM_QKV || p.mode == GM_DO) {
-                    out = mk ? __floats2bfloat162_rn(v0, v1) : __floats2bfloat162_rn(0.f, 0.f);
-                } else if (p.mode == GM_OUT) {
-                    const __nv_bfloat162 rr = *reinterpret_cast<const __nv_bfloat162 *>(p.R + o);
-                    const float2 x = __bfloat1622float2(rr);
-                    out = mk ? __floats2bfloat162_rn(x.x + v0, x.y + v1) : rr;
-                } else {   // GM_DX
-                    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p.R + o));
-                    out = __floats2bfloat162_rn(x.x + v0, x.y + v1);
-                }
-                *reinterpret_cast<__nv_bfloat162 *>(p.C[which] + o) = out;
+                float *P = p.P[which] + (size_t)blockIdx.z * p.M * p.Nb;
+                *reinterpret_cast<float2 *>(P + o) = make_float2(acc[mt][nt][hh * 2], acc[mt][nt][hh * 2 + 1]);
             }
 }
 
 static inline const __nv_bfloat16 *bf(const void *p) { return static_cast<const __nv_bfloat16 *>(p); }
-
-cudaError_t launch_qkv(const eaga_dims &d, const FwdArgs &a, cudaStream_t st) {
-    GemmParams p = {};
-    p.A[0] = bf(a.X);
-    for (int q = 0; q < 3; ++q) {
-        p.B[q] = bf(a.w[2 * q]);
-        p.bias[q] = bf(a.w[2 * q + 1]);
-    }
-    p.C[0] = static_cast<__nv_bfloat16 *>(a.Q);
-    p.C[1] = static_cast<__nv_bfloat16 *>(a.K);
-    p.C[2] = static_cast<__nv_bfloat16 *>(a.V);
-    p.mask = a.M;
-    p.M = d.B * d.n; p.K = d.dx; p.Nb = HD; p.lda = d.dx; p.ldb = HD; p.nseg = 1; p.mode = GM_QKV;
-    k_node_gemm<false, false><<<dim3(3 * HD / GBN, (p.M + GBM - 1) / GBM), GTHR, 0, st>>>(p);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_out_proj(const eaga_dims &d, const FwdArgs &a, cudaStream_t st) {
-    GemmParams p = {};
-    p.A[0] = bf(a.O);
-    p.B[0] = bf(a.w[10]);
-    p.bias[0] = bf(a.w[11]);
-    p.C[0] = static_cast<__nv_bfloat16 *>(a.Xout);
-    p.R = bf(a.X);
-    p.mask = a.M;
-    p.M = d.B * d.n; p.K = HD; p.Nb = d.dx; p.lda = HD; p.ldb = d.dx; p.nseg = 1; p.mode = GM_OUT;
-    k_node_gemm<false, false><<<dim3(d.dx / GBN, (p.M + GBM - 1) / GBM), GTHR, 0, st>>>(p);
-    return cudaGetLastError();
-}
-
-// dO = M (dX' Wo^T): A = dX' [rows, dx], B = Wo stored [N=256, K=dx].
-cudaError_t launch_dO(const eaga_dims &d, const BwdArgs &a, __nv_bfloat16 *dO, cudaStream_t st) {
-    GemmParams p = {};
-    p.A[0] = bf(a.dXout);
-    p.B[0] = bf(a.w[10]);
-    p.C[0] = dO;
-    p.mask = a.M;
-    p.M = d.B * d.n; p.K = d.dx; p.Nb = HD; p.lda = d.dx; p.ldb = d.dx; p.nseg = 1; p.mode = GM_DO;
-    k_node_gemm<false, true><<<dim3(HD / GBN, (p.M + GBM - 1) / GBM), GTHR, 0, st>>>(p);
-    return cudaGetLastError();
-}
-
-// dX = dX' + sum_q dN_q Wq^T over the three projections: B_q stored [N=dx, K=256].
-cudaError_t launch_dX(const eaga_dims &d, const BwdArgs &a, const __nv_bfloat16 *dN[3], cudaStream_t st) {
-    GemmParams p = {};
-    for (int q = 0; q < 3; ++q) {
-        p.A[q] = dN[q];
-        p.B[q] = bf(a.w[2 * q]);
-    }
-    p.C[0] = static_cast<__nv_bfloat16 *>(a.dX);
-    p.R = bf(a.dXout);
-    p.mask = a.M;
-    p.M = d.B * d.n; p.K = HD; p.Nb = d.dx; p.lda = HD; p.ldb = HD; p.nseg = 3; p.mode = GM_DX;
-    k_node_gemm<false, true><<<dim3(d.dx / GBN, (p.M + GBM - 1) / GBM), GTHR, 0, st>>>(p);
-    return cudaGetLastError();
-}
 
 // Split-K weight-gradient partials: P_q[z] = (rows of chunk z of A)^T B_q.
 //   X^T [dQ|dK|dV] -> 3 matrices [dx, 256];  O^T dX' -> [256, dx]
@@ -248,13 +160,13 @@ cudaError_t launch_wgrad(const eaga_dims &d, const BwdArgs &a, const __nv_bfloat
         p.B[q] = dN[q];
         p.P[q] = parts + q * msz;
     }
-    p.M = d.dx; p.K = rows; p.Nb = HD; p.lda = d.dx; p.ldb = HD; p.nseg = 1; p.kchunk = kchunk; p.mode = GM_WGRAD;
+    p.M = d.dx; p.K = rows; p.Nb = HD; p.lda = d.dx; p.ldb = HD; p.nseg = 1; p.kchunk = kchunk;
     k_node_gemm<true, false><<<dim3(3 * HD / GBN, (d.dx + GBM - 1) / GBM, splits), GTHR, 0, st>>>(p);
     GemmParams o = {};
     o.A[0] = bf(a.O);
     o.B[0] = bf(a.dXout);
     o.P[0] = parts + 3 * msz;
-    o.M = HD; o.K = rows; o.Nb = d.dx; o.lda = HD; o.ldb = d.dx; o.nseg = 1; o.kchunk = kchunk; o.mode = GM_WGRAD;
+    o.M = HD; o.K = rows; o.Nb = d.dx; o.lda = HD; o.ldb = d.dx; o.nseg = 1; o.kchunk = kchunk;
     k_node_gemm<true, false><<<dim3(d.dx / GBN, HD / GBM, splits), GTHR, 0, st>>>(o);
     return cudaGetLastError();
 }
