@@ -33,7 +33,8 @@ struct TcSmem {
     static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
     static constexpr uint32_t BAR = TSTAGES * STAGE;        // full[S], empty[S], done
     static constexpr uint32_t TM = BAR + (2 * TSTAGES + 1) * 8;
-    static constexpr uint32_t BYTES = TM + 16 + 1024;
+    static constexpr uint32_t BIAS = TM + 16;                // the tile's BN bias values, fp32
+    static constexpr uint32_t BYTES = BIAS + BN * 4 + 1024;
 };
 
 template <int BN>
@@ -64,6 +65,12 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
     if (w == 0) {
         tmem_alloc(sbase + S::TM, BN);
         tmem_relinquish();
+    }
+    float *sbias = reinterpret_cast<float *>(sp + S::BIAS);
+    const bool has_bias = p.mode == TC_QKV || p.mode == TC_OUT;
+    for (int c = tid; c < BN; c += TTHR) {
+        const int ng = n0 + c;
+        sbias[c] = has_bias ? __bfloat162float(p.bias[ng / p.Nb][ng % p.Nb]) : 0.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -102,55 +109,45 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
         mma_commit(done);
     }
     __syncwarp();
-    if (!mbar_wait(done, 0)) atomicExch(p.status, DEV_TIMEOUT);
-    tc_fence_after();
-
-    // epilogue: warp w holds rows m0 + 32w + t, 16 columns per TMEM load
+    // epilogue: warp w holds rows m0 + 32w + t.  The residual row segment is
+    // loaded into registers before the accumulator is ready.
     const int row = m0 + 32 * w + t;
     const bool in = row < p.M;
     const bool mk = in && p.mask[in ? row : 0] != 0;
-#pragma unroll 1
+    const bool has_res = p.mode == TC_OUT || p.mode == TC_DX;
+    const int which0 = n0 / p.Nb, col0 = n0 % p.Nb;     // BN divides Nb: one output per tile
+    const size_t obase = (size_t)(in ? row : 0) * p.Nb + col0;
+    uint4 res[BN / 8];
+#pragma unroll
+    for (int u = 0; u < BN / 8; ++u)
+        res[u] = (has_res && in) ? reinterpret_cast<const uint4 *>(p.R + obase)[u] : make_uint4(0, 0, 0, 0);
+    if (!mbar_wait(done, 0)) atomicExch(p.status, DEV_TIMEOUT);
+    tc_fence_after();
+#pragma unroll
     for (int c0 = 0; c0 < BN; c0 += 16) {
         float v[16];
         tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + c0, v);
         tmem_ld_wait();
         if (!in) continue;
-        const int ng = n0 + c0, which = ng / p.Nb, col = ng % p.Nb;
-        const size_t o = (size_t)row * p.Nb + col;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] += sbias[c0 + u];
         uint4 outv[2];
         __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(outv);
-        if (p.mode == TC_QKV || p.mode == TC_OUT) {
-            const uint4 *bb = reinterpret_cast<const uint4 *>(p.bias[which] + col);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 bv = bb[h];
-                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&bv);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 f = __bfloat1622float2(b2[u]);
-                    v[8 * h + 2 * u] += f.x;
-                    v[8 * h + 2 * u + 1] += f.y;
-                }
-            }
-        }
         if (p.mode == TC_QKV || p.mode == TC_DO) {
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 o2[u] = mk ? __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]) : __floats2bfloat162_rn(0.f, 0.f);
         } else {
-            const uint4 *rr = reinterpret_cast<const uint4 *>(p.R + o);
-            const uint4 r0 = rr[0], r1 = rr[1];
-            const __nv_bfloat162 *x2[2] = {reinterpret_cast<const __nv_bfloat162 *>(&r0),
-                                           reinterpret_cast<const __nv_bfloat162 *>(&r1)};
             const bool add = p.mode == TC_DX || mk;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const __nv_bfloat162 xr = x2[u >> 2][u & 3];
+                const uint4 r4 = res[c0 / 8 + (u >> 2)];
+                const __nv_bfloat162 xr = reinterpret_cast<const __nv_bfloat162 *>(&r4)[u & 3];
                 const float2 x = __bfloat1622float2(xr);
                 o2[u] = add ? __floats2bfloat162_rn(x.x + v[2 * u], x.y + v[2 * u + 1]) : xr;
             }
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(p.C[which] + o);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.C[which0] + obase + c0);
         dst[0] = outv[0];
         dst[1] = outv[1];
     }
@@ -183,7 +180,8 @@ cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A
                     const void *const bias[3], void *const C[3], int Nb, const void *R, const uint8_t *mask,
                     int *status, cudaStream_t st) {
     CUtensorMap am[3], bm[3];
-    const int BN = N >= 512 ? 128 : 64;
+    // N is a multiple of 64; the wider tile only where it divides N
+    const int BN = (N >= 512 && N % 128 == 0) ? 128 : 64;
     for (int s = 0; s < 3; ++s) {
         const int ss = s < nseg ? s : 0;
         if (!encode_2d(&am[s], A[ss], M, K, TBM) || !encode_2d(&bm[s], Bt[ss], N, K, BN))

@@ -85,6 +85,9 @@ CASES = [
     (2, 200, 64, 32, 8, 4, 16, "bf16", "prefix"),
     (5, 1, 16, 8, 8, 2, 8, "fp32", "full"),
     (2, 257, 256, 64, 64, 8, 32, "bf16", "random"),
+    (2, 96, 576, 64, 64, 8, 32, "bf16", "random"),     # node GEMMs: N a multiple of 64 only
+    (3, 64, 64, 64, 64, 8, 32, "bf16", "prefix"),      # narrowest node width of the fast path
+    (2, 250, 256, 64, 64, 8, 32, "bf16", "random"),    # backward: S, dP reloaded instead of kept
 ]
 
 
