@@ -14,8 +14,8 @@ cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A
                     int *status, cudaStream_t st);
 cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
                              cudaStream_t st);
-cudaError_t launch_wgrad(const eaga_dims &d, const BwdArgs &a, const __nv_bfloat16 *dN[3], float *parts,
-                         int splits, cudaStream_t st);
+cudaError_t tc_wgrad(int M, int Nb, int nout, int K, int splits, const void *A, const void *const B[3],
+                     float *const P[3], int *status, cudaStream_t st);
 cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                              cudaStream_t st);
 cudaError_t launch_bwd_finish(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
@@ -96,7 +96,14 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         void *C[3] = {a.dX, a.dX, a.dX};
         FAST_TRY(tc_gemm(3, rows, d.dx, HD, 3, A, Bt, nullptr, C, d.dx, a.dXout, a.M, a.status, st));
     }
-    FAST_TRY(launch_wgrad(d, a, dN, reinterpret_cast<float *>(ws + W.wparts), W.wsplits, st));
+    {   // split-K partials of dW{q,k,v} = X^T d{Q,K,V} and dWo = O^T dX' (O is zero on masked rows)
+        float *parts = reinterpret_cast<float *>(ws + W.wparts);
+        const size_t msz = (size_t)W.wsplits * d.dx * HD;
+        const void *Bq[3] = {dN[0], dN[1], dN[2]}, *Bo[3] = {a.dXout, a.dXout, a.dXout};
+        float *const Pq[3] = {parts, parts + msz, parts + 2 * msz}, *const Po[3] = {parts + 3 * msz, nullptr, nullptr};
+        FAST_TRY(tc_wgrad(d.dx, HD, 3, rows, W.wsplits, a.X, Bq, Pq, a.status, st));
+        FAST_TRY(tc_wgrad(HD, d.dx, 1, rows, W.wsplits, a.O, Bo, Po, a.status, st));
+    }
     return launch_bwd_finish(d, a, W, ws, reinterpret_cast<float *>(ws + W.dg), st);
 }
 

@@ -172,15 +172,28 @@ __global__ void __launch_bounds__(256) k_bias_partial(const __nv_bfloat16 *dQ, c
     }
 }
 
+// sum_{z < count} src[z * stride] with four independent accumulators (loads in
+// flight together), combined in a fixed order: deterministic.
+__device__ __forceinline__ float strided_sum(const float *src, int count, size_t stride) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int z = 0;
+    for (; z + 4 <= count; z += 4) {
+        a0 += src[(size_t)z * stride];
+        a1 += src[(size_t)(z + 1) * stride];
+        a2 += src[(size_t)(z + 2) * stride];
+        a3 += src[(size_t)(z + 3) * stride];
+    }
+    for (; z < count; ++z) a0 += src[(size_t)z * stride];
+    return (a0 + a1) + (a2 + a3);
+}
+
 // Row-kernel partials: out[z][e] = sum over CTAs of segment z of rparts[cta][e], e < dWfe+dWe.
 __global__ void k_rparts_partial(const float *rparts, int ctas, int seg, float *out) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     constexpr int NE = DE * NF + NH * DE;
     if (e >= NE) return;
     const int c0 = blockIdx.y * seg, c1 = min(ctas, c0 + seg);
-    float acc = 0.f;
-    for (int c = c0; c < c1; ++c) acc += rparts[(size_t)c * RPART + e];
-    out[(size_t)blockIdx.y * NE + e] = acc;
+    out[(size_t)blockIdx.y * NE + e] = c1 > c0 ? strided_sum(rparts + (size_t)c0 * RPART + e, c1 - c0, RPART) : 0.f;
 }
 
 struct DWPtrs {
@@ -201,32 +214,26 @@ __global__ void k_bwd_finish(const float *wparts, int wsplits, const float *bpar
     if (e < 4 * msz) {
         const int q = e / msz, o = e % msz;
         const float *src = wparts + (size_t)q * wsplits * msz + o;
-        float acc = 0.f;
-        for (int z = 0; z < wsplits; ++z) acc += src[(size_t)z * msz];
-        dW.p[q == 0 ? 0 : q == 1 ? 2 : q == 2 ? 4 : 10][o] = acc;
+        dW.p[q == 0 ? 0 : q == 1 ? 2 : q == 2 ? 4 : 10][o] = strided_sum(src, wsplits, msz);
         return;
     }
     int x = e - 4 * msz;
     if (x < ncol) {
-        float acc = 0.f;
-        for (int z = 0; z < bsplits; ++z) acc += bparts[(size_t)z * ncol + x];
+        const float acc = strided_sum(bparts + x, bsplits, ncol);
         if (x < 3 * HD) dW.p[1 + 2 * (x / HD)][x % HD] = acc;
         else dW.p[11][x - 3 * HD] = acc;
         return;
     }
     x -= ncol;
     if (x < NE) {
-        float acc = 0.f;
-        for (int z = 0; z < rsplits; ++z) acc += r2[(size_t)z * NE + x];
+        const float acc = strided_sum(r2 + x, rsplits, NE);
         if (x < DE * NF) dW.p[6][x] = acc; else dW.p[9][x - DE * NF] = acc;
         return;
     }
     x -= NE;
     if (x < B * NF) {
         const int b = x / NF, k = x % NF;
-        float acc = 0.f;
-        for (int c = 0; c < ctas_per_graph; ++c) acc += rparts[((size_t)b * ctas_per_graph + c) * RPART + NE + k];
-        dg[x] = acc;
+        dg[x] = strided_sum(rparts + (size_t)b * ctas_per_graph * RPART + NE + k, ctas_per_graph, RPART);
     }
 }
 

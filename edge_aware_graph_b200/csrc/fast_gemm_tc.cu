@@ -7,6 +7,9 @@
 //   dO       dO = M (dX' Wo^T)                              (Bt = Wo)
 //   dX       dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T          (three segments, Bt = W)
 // One thread issues TMA and MMAs; the four warps run the epilogue from TMEM.
+// k_tc_wgrad computes the weight gradients A^T B over node rows (split-K fp32
+// partials) with both operands read MN-major straight from the row-major
+// node tensors.
 #include "fast.h"
 #include "fast_common.cuh"
 
@@ -15,7 +18,9 @@ namespace fast {
 
 using namespace sm100;
 
-constexpr int TBM = 128, TBK = 64, TSTAGES = 4, TTHR = 128;
+constexpr int TBM = 128, TBK = 64, TTHR = 128;
+// pipeline stages: 4 for 64-wide tiles, 3 for 128-wide (two CTAs fit an SM either way)
+template <int BN> constexpr int tc_stages() { return BN == 128 ? 3 : 4; }
 enum TcMode { TC_QKV = 0, TC_OUT = 1, TC_DO = 2, TC_DX = 3 };
 
 struct TcParams {
@@ -27,7 +32,7 @@ struct TcParams {
     int M, K, Nb, nseg, mode;
 };
 
-template <int BN>
+template <int BN, int TSTAGES = tc_stages<BN>()>
 struct TcSmem {
     static constexpr uint32_t A_BYTES = TBM * TBK * 2, B_BYTES = BN * TBK * 2;
     static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
@@ -43,6 +48,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
           const __grid_constant__ CUtensorMap a2, const __grid_constant__ CUtensorMap b0,
           const __grid_constant__ CUtensorMap b1, const __grid_constant__ CUtensorMap b2, TcParams p) {
     using S = TcSmem<BN>;
+    constexpr int TSTAGES = tc_stages<BN>();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
@@ -156,6 +162,121 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
     if (w == 0) tmem_dealloc(tmem, BN);
 }
 
+// ------------------------------------------------------------------ weight gradients
+// P[z] = A[rows of split z]^T B[rows of split z]: A [K rows][M] and B [K rows][N]
+// row-major (K = node rows), i.e. both MN-major for the product.  TMA boxes of
+// 64 rows x 64 columns land as 64 swizzled 128-byte rows: one MN atom of 64
+// elements by 8 atoms of 8 rows along K.  An M (or N) tile of 128 is two such
+// boxes 8 KB apart (the descriptor's leading offset); 8-row groups are 1 KB
+// apart (stride offset); each MMA consumes 16 rows.
+struct WgParams {
+    float *P[3];                 // [splits][M][Nb] fp32 per output matrix
+    int *status;
+    int M, K, Nb, kchunk;
+};
+
+template <int BN>
+struct WgSmem {
+    static constexpr uint32_t A_BYTES = TBM * TBK * 2, B_BYTES = BN * TBK * 2;
+    static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+    static constexpr int ST = 3;
+    static constexpr uint32_t BAR = ST * STAGE;
+    static constexpr uint32_t TM = BAR + (2 * ST + 1) * 8;
+    static constexpr uint32_t BYTES = TM + 16 + 1024;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(TTHR, 1)
+k_tc_wgrad(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtensorMap b0,
+           const __grid_constant__ CUtensorMap b1, const __grid_constant__ CUtensorMap b2, WgParams p) {
+    using S = WgSmem<BN>;
+    constexpr int ST = S::ST;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
+    const int tid = threadIdx.x, w = tid >> 5, t = tid & 31;
+    const int n0g = blockIdx.x * BN, m0 = blockIdx.y * TBM;
+    const int which = n0g / p.Nb, n0 = n0g % p.Nb;
+    const int kbeg = blockIdx.z * p.kchunk, kend = min(p.K, kbeg + p.kchunk);
+    const int nk = kend > kbeg ? (kend - kbeg + TBK - 1) / TBK : 0;
+    const CUtensorMap *bm = which == 0 ? &b0 : which == 1 ? &b1 : &b2;
+    const uint32_t bar0 = sbase + S::BAR;
+    auto full = [&](int s) { return bar0 + 8 * s; };
+    auto empty = [&](int s) { return bar0 + 8 * (ST + s); };
+    const uint32_t done = bar0 + 16 * ST;
+
+    if (tid == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    if (w == 0) {
+        tmem_alloc(sbase + S::TM, BN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+
+    if (tid == 0) {
+        auto issue_load = [&](int kt) {
+            const int s = kt % ST, k0 = kbeg + kt * TBK;
+            const uint32_t st = sbase + s * S::STAGE;
+            mbar_expect_tx(full(s), S::STAGE);
+#pragma unroll
+            for (int h = 0; h < TBM / 64; ++h) tma_load_2d(st + h * 8192, &a0, full(s), m0 + 64 * h, k0);
+#pragma unroll
+            for (int h = 0; h < BN / 64; ++h) tma_load_2d(st + S::A_BYTES + h * 8192, bm, full(s), n0 + 64 * h, k0);
+        };
+        for (int kt = 0; kt < ST && kt < nk; ++kt) issue_load(kt);
+        const uint32_t idesc = idesc_bf16_f32_mn(TBM, BN);
+        for (int kt = 0; kt < nk; ++kt) {
+            const int s = kt % ST;
+            const uint32_t ph = (kt / ST) & 1;
+            if (!mbar_wait(full(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
+            tc_fence_after();
+            const uint32_t st = sbase + s * S::STAGE;
+#pragma unroll
+            for (int kk = 0; kk < TBK / 16; ++kk)
+                mma_bf16_ss(tmem, smem_desc(st + kk * 2048, 8192, 1024, LAYOUT_SW128),
+                            smem_desc(st + S::A_BYTES + kk * 2048, 8192, 1024, LAYOUT_SW128), idesc,
+                            (kt > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(empty(s));
+            if (kt + ST < nk) {
+                if (!mbar_wait(empty(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
+                issue_load(kt + ST);
+            }
+        }
+        mma_commit(done);
+    }
+    __syncwarp();
+    if (!mbar_wait(done, 0)) atomicExch(p.status, DEV_TIMEOUT);
+    tc_fence_after();
+    const int row = m0 + 32 * w + t;
+    float *P = p.P[which] + (size_t)blockIdx.z * p.M * p.Nb + (size_t)row * p.Nb + n0;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + c0, v);
+        tmem_ld_wait();
+        if (row >= p.M) continue;
+        if (nk == 0) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = 0.f;
+        }
+        float4 *dst = reinterpret_cast<float4 *>(P + c0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tmem, BN);
+}
+
 // ------------------------------------------------------------------ host side
 
 bool encode_2d(CUtensorMap *m, const void *base, int rows, int cols, int box_rows);
@@ -197,6 +318,42 @@ cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A
     p.status = status;
     p.M = M; p.K = K; p.Nb = Nb; p.nseg = nseg; p.mode = mode;
     return BN == 128 ? tc_launch<128>(am, bm, p, N, st) : tc_launch<64>(am, bm, p, N, st);
+}
+
+// A [K][M] row-major with 64 x 64 boxes (one MN atom of 64 columns by 64 rows).
+static bool encode_mn(CUtensorMap *m, const void *base, int rows, int cols) { return encode_2d(m, base, rows, cols, 64); }
+
+template <int BN>
+static cudaError_t wg_launch(const CUtensorMap &am, const CUtensorMap (&bm)[3], const WgParams &p, int N, int splits,
+                             cudaStream_t st) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(k_tc_wgrad<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             WgSmem<BN>::BYTES);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    dim3 grid(N / BN, (p.M + TBM - 1) / TBM, splits);
+    k_tc_wgrad<BN><<<grid, TTHR, WgSmem<BN>::BYTES, st>>>(am, bm[0], bm[1], bm[2], p);
+    return cudaGetLastError();
+}
+
+// Split-K weight-gradient partials P_q[z] = A[rows of split z]^T B_q[rows of split z]
+// for q < nout: A [K][M], B_q [K][Nb] row-major bf16, outputs [splits][M][Nb] fp32.
+cudaError_t tc_wgrad(int M, int Nb, int nout, int K, int splits, const void *A, const void *const B[3],
+                     float *const P[3], int *status, cudaStream_t st) {
+    CUtensorMap am, bm[3];
+    if (!encode_mn(&am, A, K, M)) return cudaErrorInvalidValue;
+    for (int q = 0; q < 3; ++q)
+        if (!encode_mn(&bm[q], B[q < nout ? q : 0], K, Nb)) return cudaErrorInvalidValue;
+    WgParams p = {};
+    for (int q = 0; q < 3; ++q) p.P[q] = P[q < nout ? q : 0];
+    p.status = status;
+    p.M = M; p.K = K; p.Nb = Nb;
+    p.kchunk = ((K + splits - 1) / splits + TBK - 1) / TBK * TBK;
+    const int N = Nb * nout;
+    const int BN = (N % 128 == 0 && Nb % 128 == 0) ? 128 : 64;
+    return BN == 128 ? wg_launch<128>(am, bm, p, N, splits, st) : wg_launch<64>(am, bm, p, N, splits, st);
 }
 
 }  // namespace fast
