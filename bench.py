@@ -37,9 +37,9 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the dominant kernels on this workload, from the ncu capture summarised in
-# profiles/ (k_bwd_rows_sbm.md, k_fwd_stream_sbm.md).  They describe the
+# profiles/ (k_bwd_stream_sbm.md, k_fwd_stream_sbm.md).  They describe the
 # kernels as captured; a changed kernel reports null until it is re-captured.
-NCU_TRAFFIC = {("sbm", "k_bwd_rows"): 477439232, ("sbm", "k_fwd_stream"): 269294592}
+NCU_TRAFFIC = {}
 
 
 def env_rank():
@@ -67,7 +67,7 @@ class ClockSampler:
                0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples, self.reasons = [], set()
         self.period = period_s
         self.max_mhz = None
@@ -153,24 +153,66 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     flat_dw = buf.dW_flat
 
+    def layer(s):
+        buf.forward(s)
+        buf.backward(s)
+
     def step():
-        buf.forward(stream)
-        buf.backward(stream)
+        layer(torch.cuda.current_stream())
         dp.allreduce_weight_grads(flat_dw)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, events per step around the pair kernels
-    K = args.steps
-    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- per-kernel times: eager steps with CUDA events around the pair kernels
+    nk = min(args.steps, 20)
+    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+    ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+    ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
     for a, b in ev_f + ev_b + ev_r:   # torch creates the CUDA event on first record
         a.record(stream)
         b.record(stream)
+    torch.cuda.synchronize()
+    for k in range(nk):
+        eaga.set_profile_events(0, *ev_f[k])
+        eaga.set_profile_events(1, *ev_b[k])
+        eaga.set_profile_events(2, *ev_r[k])
+        step()
+    torch.cuda.synchronize()
+    eaga.set_profile_events(0)
+    eaga.set_profile_events(1)
+    eaga.set_profile_events(2)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
+    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_b)
+    rows_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_r)
+
+    # ---- the step's kernels as one CUDA graph (launch gaps removed); the
+    # weight-gradient all-reduce (N > 1) stays outside the graph
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            layer(cap)                     # warm the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=cap):
+            layer(cap)
+        torch.cuda.synchronize()
+
+    def timed_step():
+        if graph is not None:
+            graph.replay()
+            dp.allreduce_weight_grads(flat_dw)
+        else:
+            step()
+
+    for _ in range(3):
+        timed_step()
+    # ---- timed region: K steps
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
@@ -178,23 +220,17 @@ def run_ours(args):
     clocks.start()
     t0.record(stream)
     for k in range(K):
-        eaga.set_profile_events(0, *ev_f[k])
-        eaga.set_profile_events(1, *ev_b[k])
-        eaga.set_profile_events(2, *ev_r[k])
-        step()
+        timed_step()
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    eaga.set_profile_events(0)
-    eaga.set_profile_events(1)
-    eaga.set_profile_events(2)
     ms_total = t0.elapsed_time(t1)
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
-    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_b)
-    rows_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_r)
     ms_total = dp.max_over_ranks(ms_total, "cuda")
+    if graph is not None:
+        torch.cuda.synchronize()
+        del graph
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, buf, d, stream, step)
@@ -222,10 +258,11 @@ def run_ours(args):
         "config": {"workload": "sbm-shaped training step (fwd+bwd): B=32, n=192 padded, n_real~U[44,187], "
                                "dx=256 de=64 dy=64 H=8 dh=32, bf16 storage / fp32 accumulation",
                    "global_batch": p.B * world, "seq_len": p.n, "parallelism": f"dp{world}",
-                   "l2": "inputs larger than L2 (E, dE' 144 MiB each; E', dE written each step)"},
-        "roofline": {"bound": "hbm", "kernel": "k_bwd_rows (backward row pair kernel)", "achieved": achieved,
+                   "l2": "inputs larger than L2 (E, dE' 144 MiB each; E', dE written each step)",
+                   "launch": "CUDA graph of the step's kernels" if not args.no_graph else "eager"},
+        "roofline": {"bound": "hbm", "kernel": "k_bwd_stream (backward row pair kernel)", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": NCU_TRAFFIC.get((WORKLOAD, "k_bwd_rows")),
+                     "traffic": NCU_TRAFFIC.get((WORKLOAD, "k_bwd_stream")),
                      "algorithmic_bytes": kb, "ms_per_launch": rows_ms,
                      "backward_pair_kernels_ms": bwd_ms},
         "roofline_fwd": {"bound": "hbm", "kernel": "k_fwd_stream (forward pair kernel)",
@@ -340,6 +377,7 @@ def main():
     ap.add_argument("--cpu-graphs", type=int, default=16)
     ap.add_argument("--ref-graphs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the step's kernels one by one")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -5,10 +5,9 @@
 // clients that link this library but no device allocator, or code running
 // under a framework whose memory pool must not be bypassed and that only
 // hands out the tensors it owns (inputs, outputs, the saved state).  For them
-// the forward's scratch (the status word, the per-graph global FiLM term, the
-// tensor-core operand images of the FiLM and edge weights and the transposed
-// node weights) lives in a fixed device array inside this library instead of
-// a caller buffer.
+// the forward's small scratch (the status word, the per-graph global FiLM
+// term and the tensor-core operand images of the FiLM and edge weights) lives
+// in a fixed device array inside this library instead of a caller buffer.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds NOALLOC_SCRATCH_BYTES of it until the process exits.  All
@@ -24,7 +23,7 @@ using namespace eaga;
 
 namespace {
 
-constexpr size_t NOALLOC_SCRATCH_BYTES = 4u << 20;   // status word + g [B,2H] fp32 + weight images
+constexpr size_t NOALLOC_SCRATCH_BYTES = 64 * 1024;   // status word + g [B,2H] fp32 + 8 KB of operand images
 constexpr size_t NOALLOC_STATUS = 0, NOALLOC_G = 256;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];

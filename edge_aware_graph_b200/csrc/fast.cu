@@ -8,10 +8,9 @@ namespace fast {
 
 cudaError_t launch_prologue(const eaga_dims &d, const void *const w[12], const void *y, float *g, uint8_t *img,
                             cudaStream_t st);
-cudaError_t launch_weight_images(const eaga_dims &d, const void *const w[12], uint8_t *wimg, cudaStream_t st);
-cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A[3], const void *const Bt[3],
+cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A[3], const void *const B[3],
                     const void *const bias[3], void *const C[3], int Nb, const void *R, const uint8_t *mask,
-                    int *status, cudaStream_t st);
+                    int *status, cudaStream_t st, bool b_mn);
 cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
                              cudaStream_t st);
 cudaError_t tc_wgrad(int M, int Nb, int nout, int K, int splits, const void *A, const void *const B[3],
@@ -26,20 +25,18 @@ bool supports(const eaga_dims &d) {
            d.n <= 1024 && d.dx % 64 == 0 && d.dx >= 64;
 }
 
-// Forward: the small operand images, then the transposed node weights
-// (W{q,k,v}^T [768][dx], Wo^T [dx][256]) after the common workspace;
-// backward: the whole FastWs.
-static size_t wimg_bytes(const eaga_dims &d) { return align256(size_t(4) * HD * d.dx * 2); }
-size_t forward_scratch_bytes(const eaga_dims &d) { return align256(IMG_BYTES) + wimg_bytes(d); }
+// Forward: the small operand images after the common workspace; backward:
+// the whole FastWs.
+size_t forward_scratch_bytes(const eaga_dims &) { return align256(IMG_BYTES); }
 size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, size_t common_head) {
-    if (!for_backward) return align256(common_fwd + IMG_BYTES) + wimg_bytes(d);
+    if (!for_backward) return align256(common_fwd + IMG_BYTES);
     return fast_ws(d, common_head).total;
 }
 
 int kernel_launches(const eaga_dims &, int for_backward) {
-    // forward: prologue, weight images, QKV, pairs, out-proj
+    // forward: prologue, QKV, pairs, out-proj
     // backward: prologue, dO, row pairs, dk/dv, dX, wgrad x2, bias partial, rparts partial, finish, film grads
-    return for_backward ? 11 : 5;
+    return for_backward ? 11 : 4;
 }
 
 #define FAST_TRY(x)                               \
@@ -50,26 +47,22 @@ int kernel_launches(const eaga_dims &, int for_backward) {
 
 cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st) {
     uint8_t *img = reinterpret_cast<uint8_t *>(ws_after_common);
-    uint8_t *wimg = img + align256(IMG_BYTES);
-    const __nv_bfloat16 *WqkvT = reinterpret_cast<const __nv_bfloat16 *>(wimg);
-    const __nv_bfloat16 *WoT = WqkvT + (size_t)3 * HD * d.dx;
     const int rows = d.B * d.n;
     FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, st));
-    FAST_TRY(launch_weight_images(d, a.w, wimg, st));
     {   // [Q|K|V] = X [Wq|Wk|Wv] + b
-        const void *A[3] = {a.X, a.X, a.X}, *Bt[3] = {WqkvT, WqkvT, WqkvT};
+        const void *A[3] = {a.X, a.X, a.X}, *B[3] = {a.w[0], a.w[2], a.w[4]};
         const void *bias[3] = {a.w[1], a.w[3], a.w[5]};
         void *C[3] = {a.Q, a.K, a.V};
-        FAST_TRY(tc_gemm(0, rows, 3 * HD, d.dx, 1, A, Bt, bias, C, HD, nullptr, a.M, a.status, st));
+        FAST_TRY(tc_gemm(0, rows, 3 * HD, d.dx, 1, A, B, bias, C, HD, nullptr, a.M, a.status, st, true));
     }
     prof_mark(0, 0, st);
     FAST_TRY(launch_fwd_pairs(d, a, img, a.g, st));
     prof_mark(0, 1, st);
     {   // X' = X + M (O Wo + bo)
-        const void *A[3] = {a.O, a.O, a.O}, *Bt[3] = {WoT, WoT, WoT};
+        const void *A[3] = {a.O, a.O, a.O}, *B[3] = {a.w[10], a.w[10], a.w[10]};
         const void *bias[3] = {a.w[11], a.w[11], a.w[11]};
         void *C[3] = {a.Xout, a.Xout, a.Xout};
-        FAST_TRY(tc_gemm(1, rows, d.dx, HD, 1, A, Bt, bias, C, d.dx, a.X, a.M, a.status, st));
+        FAST_TRY(tc_gemm(1, rows, d.dx, HD, 1, A, B, bias, C, d.dx, a.X, a.M, a.status, st, true));
     }
     return cudaSuccess;
 }
@@ -83,7 +76,7 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
     {   // dO = M (dX' Wo^T)
         const void *A[3] = {a.dXout, a.dXout, a.dXout}, *Bt[3] = {a.w[10], a.w[10], a.w[10]};
         void *C[3] = {dO, dO, dO};
-        FAST_TRY(tc_gemm(2, rows, HD, d.dx, 1, A, Bt, nullptr, C, HD, nullptr, a.M, a.status, st));
+        FAST_TRY(tc_gemm(2, rows, HD, d.dx, 1, A, Bt, nullptr, C, HD, nullptr, a.M, a.status, st, false));
     }
     prof_mark(1, 0, st);
     FAST_TRY(launch_bwd_pairs(d, a, W, ws, a.g, st));
@@ -94,7 +87,7 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
     {   // dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T
         const void *A[3] = {dN[0], dN[1], dN[2]}, *Bt[3] = {a.w[0], a.w[2], a.w[4]};
         void *C[3] = {a.dX, a.dX, a.dX};
-        FAST_TRY(tc_gemm(3, rows, d.dx, HD, 3, A, Bt, nullptr, C, d.dx, a.dXout, a.M, a.status, st));
+        FAST_TRY(tc_gemm(3, rows, d.dx, HD, 3, A, Bt, nullptr, C, d.dx, a.dXout, a.M, a.status, st, false));
     }
     {   // split-K partials of dW{q,k,v} = X^T d{Q,K,V} and dWo = O^T dX' (O is zero on masked rows)
         float *parts = reinterpret_cast<float *>(ws + W.wparts);

@@ -1,9 +1,10 @@
-// Node-side GEMMs on tcgen05: C[M, N] = sum_seg A_seg[M, K] Bt_seg[N, K]^T,
-// both operands K-major (row-major with K contiguous), 128B-swizzled tiles
+// Node-side GEMMs on tcgen05: C[M, N] = sum_seg A_seg[M, K] B_seg[K, N], A
+// K-major (row-major [M, K]); B either K-major (stored [N, K]) or MN-major
+// (stored [K, N], one matrix per output when the outputs are several); 128B-swizzled tiles
 // loaded by TMA through a 4-stage mbarrier pipeline, the 128 x BN fp32
 // accumulator in TMEM, and the layer's epilogues fused:
-//   QKV      [Q|K|V] = X [Wq|Wk|Wv] + b, masked rows zero   (Bt = the three W^T stacked)
-//   out-proj X' = X + M (O Wo + bo)                         (Bt = Wo^T)
+//   QKV      [Q|K|V] = X [Wq|Wk|Wv] + b, masked rows zero   (B = Wq, Wk, Wv, MN-major)
+//   out-proj X' = X + M (O Wo + bo)                         (B = Wo, MN-major)
 //   dO       dO = M (dX' Wo^T)                              (Bt = Wo)
 //   dX       dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T          (three segments, Bt = W)
 // One thread issues TMA and MMAs; the four warps run the epilogue from TMEM.
@@ -30,6 +31,7 @@ struct TcParams {
     const uint8_t *mask;         // [M]
     int *status;
     int M, K, Nb, nseg, mode;
+    int b_mn;                    // B stored [K, N] (MN-major), map chosen by output matrix
 };
 
 template <int BN, int TSTAGES = tc_stages<BN>()>
@@ -59,6 +61,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
     auto empty = [&](int s) { return bar0 + 8 * (TSTAGES + s); };
     const uint32_t done = bar0 + 16 * TSTAGES;
     const int kt_seg = p.K / TBK, nk = kt_seg * p.nseg;
+    const int which_n = n0 / p.Nb, ncol0 = n0 % p.Nb;
 
     if (tid == 0) {
         for (int s = 0; s < TSTAGES; ++s) {
@@ -87,14 +90,21 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
         auto issue_load = [&](int kt) {
             const int s = kt % TSTAGES, seg = kt / kt_seg, k0 = (kt % kt_seg) * TBK;
             const CUtensorMap *am = seg == 0 ? &a0 : seg == 1 ? &a1 : &a2;
-            const CUtensorMap *bm = seg == 0 ? &b0 : seg == 1 ? &b1 : &b2;
+            const int bsel = p.b_mn ? which_n : seg;
+            const CUtensorMap *bm = bsel == 0 ? &b0 : bsel == 1 ? &b1 : &b2;
             const uint32_t st = sbase + s * S::STAGE;
             mbar_expect_tx(full(s), S::STAGE);
             tma_load_2d(st, am, full(s), k0, m0);
-            tma_load_2d(st + S::A_BYTES, bm, full(s), k0, n0);
+            if (p.b_mn) {
+                // [64 k rows][64 n] boxes, 8 KB apart along N
+#pragma unroll
+                for (int h = 0; h < BN / 64; ++h) tma_load_2d(st + S::A_BYTES + h * 8192, bm, full(s), ncol0 + 64 * h, k0);
+            } else {
+                tma_load_2d(st + S::A_BYTES, bm, full(s), k0, n0);
+            }
         };
         for (int kt = 0; kt < TSTAGES && kt < nk; ++kt) issue_load(kt);
-        const uint32_t idesc = idesc_bf16_f32(TBM, BN);
+        const uint32_t idesc = idesc_bf16_f32(TBM, BN) | (p.b_mn ? (1u << 16) : 0u);
         for (int kt = 0; kt < nk; ++kt) {
             const int s = kt % TSTAGES;
             const uint32_t ph = (kt / TSTAGES) & 1;
@@ -104,8 +114,9 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
 #pragma unroll
             for (int kk = 0; kk < TBK / 16; ++kk)
                 mma_bf16_ss(tmem, smem_desc(st + kk * 32, 16, 1024, LAYOUT_SW128),
-                            smem_desc(st + S::A_BYTES + kk * 32, 16, 1024, LAYOUT_SW128), idesc,
-                            (kt > 0 || kk > 0) ? 1u : 0u);
+                            p.b_mn ? smem_desc(st + S::A_BYTES + kk * 2048, 8192, 1024, LAYOUT_SW128)
+                                   : smem_desc(st + S::A_BYTES + kk * 32, 16, 1024, LAYOUT_SW128),
+                            idesc, (kt > 0 || kk > 0) ? 1u : 0u);
             mma_commit(empty(s));
             if (kt + TSTAGES < nk) {
                 if (!mbar_wait(empty(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
@@ -296,16 +307,19 @@ static cudaError_t tc_launch(const CUtensorMap (&am)[3], const CUtensorMap (&bm)
     return cudaGetLastError();
 }
 
-// Out = epilogue(sum_seg A[seg] Bt[seg]^T): A[seg] [M, K], Bt[seg] [N, K] row-major bf16.
-cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A[3], const void *const Bt[3],
+// Out = epilogue(sum_seg A[seg] B[seg]): A[seg] [M, K] row-major bf16; B[seg] stored
+// [N, K] (b_mn = false), or, with b_mn, B[q] stored [K, Nb] for output matrix q.
+cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A[3], const void *const B[3],
                     const void *const bias[3], void *const C[3], int Nb, const void *R, const uint8_t *mask,
-                    int *status, cudaStream_t st) {
+                    int *status, cudaStream_t st, bool b_mn) {
     CUtensorMap am[3], bm[3];
-    // N is a multiple of 64; the wider tile only where it divides N
-    const int BN = (N >= 512 && N % 128 == 0) ? 128 : 64;
+    // N is a multiple of 64; the wider tile only where it divides N (and each output)
+    const int BN = (N >= 512 && N % 128 == 0 && Nb % 128 == 0) ? 128 : 64;
+    const int nb_maps = b_mn ? N / Nb : nseg;
     for (int s = 0; s < 3; ++s) {
-        const int ss = s < nseg ? s : 0;
-        if (!encode_2d(&am[s], A[ss], M, K, TBM) || !encode_2d(&bm[s], Bt[ss], N, K, BN))
+        const int sa = s < nseg ? s : 0, sb = s < nb_maps ? s : 0;
+        if (!encode_2d(&am[s], A[sa], M, K, TBM)) return cudaErrorInvalidValue;
+        if (!(b_mn ? encode_2d(&bm[s], B[sb], K, Nb, 64) : encode_2d(&bm[s], B[sb], N, K, BN)))
             return cudaErrorInvalidValue;
     }
     TcParams p = {};
@@ -316,7 +330,7 @@ cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A
     p.R = static_cast<const __nv_bfloat16 *>(R);
     p.mask = mask;
     p.status = status;
-    p.M = M; p.K = K; p.Nb = Nb; p.nseg = nseg; p.mode = mode;
+    p.M = M; p.K = K; p.Nb = Nb; p.nseg = nseg; p.mode = mode; p.b_mn = b_mn ? 1 : 0;
     return BN == 128 ? tc_launch<128>(am, bm, p, N, st) : tc_launch<64>(am, bm, p, N, st);
 }
 

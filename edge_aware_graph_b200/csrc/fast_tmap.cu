@@ -91,35 +91,6 @@ bool encode_p_map(CUtensorMap *m, const void *base, int B, int n, int npad) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Transposed weight images for the K-major tcgen05 GEMMs of the forward:
-// WqkvT [3*256][dx] (row n = column n%256 of W{q,k,v}[n/256]) and WoT [dx][256].
-__global__ void k_weight_images(const __nv_bfloat16 *Wq, const __nv_bfloat16 *Wk, const __nv_bfloat16 *Wv,
-                                const __nv_bfloat16 *Wo, __nv_bfloat16 *WqkvT, __nv_bfloat16 *WoT, int dx) {
-    __shared__ __nv_bfloat16 tile[32][33];
-    // block (bx, by, bz): bz < 3 -> W{q,k,v} [dx][256] tile; bz == 3 -> Wo [256][dx] tile
-    const int bz = blockIdx.z;
-    const __nv_bfloat16 *src = bz == 0 ? Wq : bz == 1 ? Wk : bz == 2 ? Wv : Wo;
-    const int rows = bz < 3 ? dx : HD, cols = bz < 3 ? HD : dx;
-    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-    if (r0 >= rows || c0 >= cols) return;
-    for (int k = threadIdx.y; k < 32; k += blockDim.y)
-        tile[k][threadIdx.x] = src[(size_t)(r0 + k) * cols + c0 + threadIdx.x];
-    __syncthreads();
-    __nv_bfloat16 *dst = bz < 3 ? WqkvT + (size_t)bz * HD * dx : WoT;
-    for (int k = threadIdx.y; k < 32; k += blockDim.y)
-        dst[(size_t)(c0 + k) * rows + r0 + threadIdx.x] = tile[threadIdx.x][k];
-}
-
-cudaError_t launch_weight_images(const eaga_dims &d, const void *const w[12], uint8_t *wimg, cudaStream_t st) {
-    __nv_bfloat16 *WqkvT = reinterpret_cast<__nv_bfloat16 *>(wimg);
-    __nv_bfloat16 *WoT = WqkvT + (size_t)3 * HD * d.dx;
-    const int big = d.dx > HD ? d.dx : HD;
-    k_weight_images<<<dim3(big / 32, big / 32, 4), dim3(32, 8), 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(w[0]), static_cast<const __nv_bfloat16 *>(w[2]),
-        static_cast<const __nv_bfloat16 *>(w[4]), static_cast<const __nv_bfloat16 *>(w[10]), WqkvT, WoT, d.dx);
-    return cudaGetLastError();
-}
-
 // g_b = y_b Wfy + bf (fp32) for every graph: one warp per graph, lanes split
 // the dy terms and add their 16 sums with shuffles in a fixed order.  The last
 // block writes the four operand images from Wfe and We staged in shared memory.

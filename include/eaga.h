@@ -131,13 +131,11 @@ EAGA_API eaga_status eaga_backward(const eaga_dims *dims,
  * same arguments minus the workspace; `saved` is required (it is an output
  * as large as the node tensors).
  *
- * The forward's scratch (status word, global FiLM term g [B,2H] fp32 and,
- * on the specialised bf16 path, the tensor-core images of Wfe, We and of
- * the transposed node weights) lives in a 4 MiB array in the library's
- * device memory, held by every GPU that loads the library until the process
- * exits.  Limit: 256 + roundup256(8*H*B) [+ 8192 + 2048*dx on the bf16
- * path with de = 64, H = 8, dh = 32] bytes must fit in 4 MiB (for example
- * B <= 57,000 graphs at H = 8, dx = 256); larger problems return
+ * The forward's small scratch (status word, global FiLM term g [B,2H] fp32,
+ * 8 KB of tensor-core operand images on the bf16 path) lives in a 64 KiB
+ * array in the library's device memory, held by every GPU that loads the
+ * library until the process exits.  Limit: 256 + roundup256(8*H*B) + 8192
+ * bytes must fit in 64 KiB, so B <= 892 graphs at H = 8; larger B returns
  * EAGA_ERR_UNSUPPORTED without launching.  No device memory is allocated or
  * freed by this call.
  *

@@ -79,7 +79,7 @@ def test_noalloc_forward_matches_forward_twice(name):
 
 def test_noalloc_rejects_too_many_graphs():
     L = eaga.lib()
-    d = eaga.dims(100000, 8, 64, 64, 64, 8, 32, "bf16")   # g alone needs 6.4 MB > 4 MiB
+    d = eaga.dims(100000, 8, 64, 64, 64, 8, 32, "bf16")   # g alone needs 6.4 MB > 64 KiB
     fake = ctypes.c_void_p(0x100000)
     w = eaga.Weights(*([0x100000] * 12))
     rc = L.eaga_forward_noalloc(ctypes.byref(d), fake, fake, fake, fake, ctypes.byref(w), fake, fake, fake, None)
