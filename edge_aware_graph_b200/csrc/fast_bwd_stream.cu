@@ -57,7 +57,7 @@ struct BsSmem {
     static constexpr uint32_t G = WDG + 256;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // node mask [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;
-    static constexpr uint32_t TM = BAR + 8 * 12;
+    static constexpr uint32_t TM = BAR + 8 * 14;
     static constexpr uint32_t STAB = TM + 16;                 // slot table [4 iterations][8] u8
     static constexpr uint32_t BYTES = STAB + 32 + 1024;
     // in the drained ring at the end: dq quadrant sums [4][8][256] f32 (32 KB)
@@ -120,8 +120,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         mbar_init(bar(BB_FILM_EMPTY + 1), NWARP);
         mbar_init(bar(BB_DF_FULL), NWARP);
         mbar_init(bar(BB_DE_FULL), 1);
-        mbar_init(bar(BB_STAGE_DONE), NWARP);
-        mbar_init(bar(BB_STAGE_DONE + 1), NWARP);
+        for (int k = 0; k < 4; ++k) mbar_init(bar(BB_STAGE_DONE + k), NWARP);
         fence_mbar_init();
     }
     if (W == 0) {
@@ -254,7 +253,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             issue_loads();
             for (int it = 0; it < nit; ++it) {
                 const bool pass2 = it >= nch;
-                if (!mbar_wait(bar(BB_STAGE_DONE + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
+                if (!mbar_wait(bar(BB_STAGE_DONE + (it & 3)), (it >> 2) & 1)) flag_timeout(p.status);
                 if (pass2) {
                     const int j0 = 32 * chunk_of(it);
                     tma_store_5d_hint(&tmDE, slot_addr(it, 2), 0, i0 / 2, j0, 0, b, drop_l2);
@@ -390,7 +389,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) dsum[e][hh] += av[hh][e] * da[hh][e];
                 __syncwarp();
-                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 1)));
+                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
                 continue;
             }
 
@@ -454,7 +453,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 1)));
+            if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
         }
 
         // ---------------- end of the row block, in the drained ring

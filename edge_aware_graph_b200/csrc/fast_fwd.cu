@@ -53,11 +53,11 @@ struct FsSmem {
     static constexpr uint32_t G = FIN + 512;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // mask of the graph's nodes [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;                // mbarriers, see below
-    static constexpr uint32_t TM = BAR + 8 * 12;              // TMEM base address
+    static constexpr uint32_t TM = BAR + 8 * 14;              // TMEM base address
     static constexpr uint32_t BYTES = TM + 16 + 1024;         // + alignment slack
     static constexpr uint32_t OPART = 0;                      // [4][8][256] f32 O partials (ring drained)
 };
-// mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full, edge_full, stage_done[2]
+// mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full, edge_full, stage_done[4]
 constexpr int FB_FULL = 0, FB_FILM_FULL = 4, FB_FILM_EMPTY = 6, FB_A_FULL = 8, FB_EDGE_FULL = 9,
               FB_STAGE_DONE = 10;
 
@@ -113,8 +113,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         mbar_init(bar(FB_FILM_EMPTY + 1), NWARP);
         mbar_init(bar(FB_A_FULL), NWARP);
         mbar_init(bar(FB_EDGE_FULL), 1);
-        mbar_init(bar(FB_STAGE_DONE), NWARP);
-        mbar_init(bar(FB_STAGE_DONE + 1), NWARP);
+        for (int k = 0; k < 4; ++k) mbar_init(bar(FB_STAGE_DONE + k), NWARP);
         fence_mbar_init();
     }
     if (W == 0) {
@@ -166,19 +165,19 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             while (next_film < nit || next_edge < nit) {
                 bool progressed = false;
                 if (next_film < nit &&
-                    mbar_try_wait(bar(FB_FULL + next_film % FS_NFULL), (next_film / FS_NFULL) & 1) &&
+                    mbar_test_wait(bar(FB_FULL + next_film % FS_NFULL), (next_film / FS_NFULL) & 1) &&
                     (next_film < 2 ||
-                     mbar_try_wait(bar(FB_FILM_EMPTY + (next_film & 1)), ((next_film - 2) >> 1) & 1))) {
+                     mbar_test_wait(bar(FB_FILM_EMPTY + (next_film & 1)), ((next_film - 2) >> 1) & 1))) {
                     issue_film(next_film++);
                     progressed = true;
                 }
                 if (next_edge < nit && next_edge < next_film &&
-                    mbar_try_wait(bar(FB_A_FULL), (next_edge - nch) & 1)) {
+                    mbar_test_wait(bar(FB_A_FULL), (next_edge - nch) & 1)) {
                     issue_edge();
                     ++next_edge;
                     progressed = true;
                 }
-                if (!progressed && ++polls > (1u << 26)) {
+                if (!progressed && ++polls > (1u << 28)) {
                     flag_timeout(p.status);
                     break;
                 }
@@ -225,7 +224,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                             tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
                     }
                 }
-                if (!mbar_wait(bar(FB_STAGE_DONE + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
+                if (!mbar_wait(bar(FB_STAGE_DONE + (it & 3)), (it >> 2) & 1)) flag_timeout(p.status);
                 if (pass2) {
                     const int j0 = 32 * chunk_of(it);
                     tma_store_5d_hint(&tmEo, slot_addr(it, 0), 0, i0 / 2, j0, 0, b, drop_l2);
@@ -390,7 +389,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         }
                     }
                 __syncwarp();
-                if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 1)));
+                if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
                 continue;
             }
 
@@ -424,7 +423,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 1)));
+            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
         }
 
         // ---------------- O: sum over the quadrant warps (in the drained ring)
