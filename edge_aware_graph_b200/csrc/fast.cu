@@ -1,5 +1,6 @@
 // Host glue of the specialised sm_100a path (de = 64, H = 8, dh = 32, bf16):
 // which dims it covers, its workspace, its launch sequence and launch count.
+#include <mutex>
 #include "fast.h"
 #include "fast_common.cuh"
 
@@ -17,8 +18,9 @@ cudaError_t tc_wgrad(int M, int Nb, int nout, int K, int splits, const void *A, 
                      float *const P[3], int *status, cudaStream_t st);
 cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                              cudaStream_t st);
-cudaError_t launch_bwd_finish(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
-                              cudaStream_t st);
+cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
+cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
+                             cudaStream_t st);
 
 bool supports(const eaga_dims &d) {
     return d.dtype == EAGA_BF16 && d.de == DE && d.H == NH && d.dh == DH && d.n % 2 == 0 && d.n >= 2 &&
@@ -67,23 +69,80 @@ cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common,
     return cudaSuccess;
 }
 
+// Two auxiliary streams and a pool of events per device, created on first
+// use: the backward runs independent kernels side by side (fork / join on
+// events), which a CUDA graph captured around the call keeps as parallel
+// branches.  The lock is held while a call enqueues, so concurrent calls on
+// one device never share an event between a record and its wait.
+namespace {
+constexpr int kMaxDevices = 64, kEvents = 6;
+struct DeviceAux {
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t s[2] = {nullptr, nullptr};
+    cudaEvent_t ev[kEvents] = {};
+};
+DeviceAux g_aux[kMaxDevices];
+
+cudaError_t device_aux(DeviceAux **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    *out = &g_aux[dev];
+    return cudaSuccess;
+}
+
+cudaError_t aux_init(DeviceAux &x) {   // called with x.mu held
+    if (x.ready) return cudaSuccess;
+    cudaError_t e;
+    for (int k = 0; k < 2; ++k)
+        if ((e = cudaStreamCreateWithFlags(&x.s[k], cudaStreamNonBlocking)) != cudaSuccess) return e;
+    for (int k = 0; k < kEvents; ++k)
+        if ((e = cudaEventCreateWithFlags(&x.ev[k], cudaEventDisableTiming)) != cudaSuccess) return e;
+    x.ready = true;
+    return cudaSuccess;
+}
+
+// `to` waits for everything enqueued on `from` so far
+cudaError_t stream_after(cudaStream_t to, cudaStream_t from, cudaEvent_t ev) {
+    cudaError_t e = cudaEventRecord(ev, from);
+    return e == cudaSuccess ? cudaStreamWaitEvent(to, ev, 0) : e;
+}
+}  // namespace
+
 cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head, cudaStream_t st) {
     const FastWs W = fast_ws(d, head);
     uint8_t *img = reinterpret_cast<uint8_t *>(ws + W.img);
     __nv_bfloat16 *dO = reinterpret_cast<__nv_bfloat16 *>(ws + W.dO);
     const int rows = d.B * d.n;
-    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, st));
-    {   // dO = M (dX' Wo^T)
+    DeviceAux *aux = nullptr;
+    FAST_TRY(device_aux(&aux));
+    std::lock_guard<std::mutex> lock(aux->mu);
+    FAST_TRY(aux_init(*aux));
+    cudaStream_t s1 = aux->s[0], s2 = aux->s[1];
+    cudaEvent_t *ev = aux->ev;
+
+    // prologue (g, operand images) beside dO = M (dX' Wo^T)
+    FAST_TRY(stream_after(s1, st, ev[0]));
+    {
         const void *A[3] = {a.dXout, a.dXout, a.dXout}, *Bt[3] = {a.w[10], a.w[10], a.w[10]};
         void *C[3] = {dO, dO, dO};
-        FAST_TRY(tc_gemm(2, rows, HD, d.dx, 1, A, Bt, nullptr, C, HD, nullptr, a.M, a.status, st, false));
+        FAST_TRY(tc_gemm(2, rows, HD, d.dx, 1, A, Bt, nullptr, C, HD, nullptr, a.M, a.status, s1, false));
     }
+    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, st));
+    FAST_TRY(stream_after(st, s1, ev[1]));
+
     prof_mark(1, 0, st);
     FAST_TRY(launch_bwd_pairs(d, a, W, ws, a.g, st));
     prof_mark(1, 1, st);
+
+    // dX, the weight-gradient partials and the reductions' first level side by side
     const __nv_bfloat16 *dN[3] = {reinterpret_cast<const __nv_bfloat16 *>(ws + W.dQ),
                                   reinterpret_cast<const __nv_bfloat16 *>(ws + W.dK),
                                   reinterpret_cast<const __nv_bfloat16 *>(ws + W.dV)};
+    FAST_TRY(stream_after(s1, st, ev[2]));
+    FAST_TRY(stream_after(s2, st, ev[3]));
     {   // dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T
         const void *A[3] = {dN[0], dN[1], dN[2]}, *Bt[3] = {a.w[0], a.w[2], a.w[4]};
         void *C[3] = {a.dX, a.dX, a.dX};
@@ -94,10 +153,13 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         const size_t msz = (size_t)W.wsplits * d.dx * HD;
         const void *Bq[3] = {dN[0], dN[1], dN[2]}, *Bo[3] = {a.dXout, a.dXout, a.dXout};
         float *const Pq[3] = {parts, parts + msz, parts + 2 * msz}, *const Po[3] = {parts + 3 * msz, nullptr, nullptr};
-        FAST_TRY(tc_wgrad(d.dx, HD, 3, rows, W.wsplits, a.X, Bq, Pq, a.status, st));
-        FAST_TRY(tc_wgrad(HD, d.dx, 1, rows, W.wsplits, a.O, Bo, Po, a.status, st));
+        FAST_TRY(tc_wgrad(d.dx, HD, 3, rows, W.wsplits, a.X, Bq, Pq, a.status, s1));
+        FAST_TRY(tc_wgrad(HD, d.dx, 1, rows, W.wsplits, a.O, Bo, Po, a.status, s1));
     }
-    return launch_bwd_finish(d, a, W, ws, reinterpret_cast<float *>(ws + W.dg), st);
+    FAST_TRY(launch_bwd_partials(d, a, W, ws, s2));
+    FAST_TRY(stream_after(st, s1, ev[4]));
+    FAST_TRY(stream_after(st, s2, ev[5]));
+    return launch_bwd_final(d, a, W, ws, reinterpret_cast<float *>(ws + W.dg), st);
 }
 
 }  // namespace fast

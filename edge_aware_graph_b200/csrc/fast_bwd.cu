@@ -292,12 +292,13 @@ cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs 
     return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_finish(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
-                              cudaStream_t st) {
+// Column sums for the bias gradients and the first level of the row-block
+// partials of dWfe / dWe (both read only what the pair kernels wrote).
+cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st) {
     const __nv_bfloat16 *dQ = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dQ);
     const __nv_bfloat16 *dK = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dK);
     const __nv_bfloat16 *dV = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dV);
-    const int rows = d.B * d.n, ncol = 3 * HD + d.dx;
+    const int rows = d.B * d.n;
     float *bparts = reinterpret_cast<float *>(ws + W.bparts);
     const int seg_rows = (rows + W.bsplits - 1) / W.bsplits;
     k_bias_partial<<<dim3(3 + (d.dx + 255) / 256, W.bsplits), 256, 0, st>>>(
@@ -307,15 +308,24 @@ cudaError_t launch_bwd_finish(const eaga_dims &d, const BwdArgs &a, const FastWs
     constexpr int NE = DE * NF + NH * DE;
     const float *rparts = reinterpret_cast<const float *>(ws + W.rparts);
     k_rparts_partial<<<dim3((NE + 255) / 256, W.rsplits), 256, 0, st>>>(rparts, ctas, seg, r2);
+    return cudaGetLastError();
+}
+
+// Final sums of every weight gradient and the global FiLM term's gradients.
+cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
+                             cudaStream_t st) {
+    const int ncol = 3 * HD + d.dx;
+    constexpr int NE = DE * NF + NH * DE;
     DWPtrs dWdev;
     for (int q = 0; q < 12; ++q) dWdev.p[q] = a.dW[q];
     const int total = 4 * d.dx * HD + ncol + NE + d.B * NF;
     const int cpg = (d.n + TB - 1) / TB;
-    k_bwd_finish<<<(total + 255) / 256, 256, 0, st>>>(reinterpret_cast<const float *>(ws + W.wparts), W.wsplits,
-                                                      bparts, W.bsplits, r2, W.rsplits, rparts, cpg, d.B, d.dx,
-                                                      d.dy, static_cast<const __nv_bfloat16 *>(a.y),
-                                                      static_cast<const __nv_bfloat16 *>(a.w[7]), dWdev,
-                                                      static_cast<__nv_bfloat16 *>(a.dy), dg);
+    k_bwd_finish<<<(total + 255) / 256, 256, 0, st>>>(
+        reinterpret_cast<const float *>(ws + W.wparts), W.wsplits, reinterpret_cast<const float *>(ws + W.bparts),
+        W.bsplits, reinterpret_cast<const float *>(ws + W.r2), W.rsplits,
+        reinterpret_cast<const float *>(ws + W.rparts), cpg, d.B, d.dx, d.dy,
+        static_cast<const __nv_bfloat16 *>(a.y), static_cast<const __nv_bfloat16 *>(a.w[7]), dWdev,
+        static_cast<__nv_bfloat16 *>(a.dy), dg);
     const int tf = NF + d.dy * NF + d.B * d.dy;
     k_film_grads<<<(tf + 255) / 256, 256, 0, st>>>(dg, d.B, d.dy, static_cast<const __nv_bfloat16 *>(a.y),
                                                    static_cast<const __nv_bfloat16 *>(a.w[7]), a.dW[8], a.dW[7],

@@ -115,7 +115,12 @@ EAGA_API eaga_status eaga_forward(const eaga_dims *dims,
  * the upstream gradients dXout, dEout, writes dX, dE, dy and every weight
  * gradient (fp32).  `workspace` must hold eaga_workspace_size(dims, 1) bytes.
  * Gradients of masked nodes / invalid pairs are the residual ones
- * (dX_i = dX'_i, dE_ij = dE'_ij). */
+ * (dX_i = dX'_i, dE_ij = dE'_ij).
+ * On the specialised bf16 path some independent kernels run on two streams
+ * the library creates once per device; they start after the work already
+ * on `stream` and `stream` waits for them before the call's last kernels,
+ * so the call is ordered on `stream` as a whole (and a CUDA graph captured
+ * around it keeps them as parallel branches). */
 EAGA_API eaga_status eaga_backward(const eaga_dims *dims,
                           const void *X, const void *E, const void *y, const uint8_t *M,
                           const eaga_weights *w, const void *saved,
