@@ -81,6 +81,7 @@ struct BwdStreamParams {
     __nv_bfloat16 *Pa, *Pds; // [B,H,n,npad] out: a and ds (unscaled) of every pair
     int *status;
     int n, npad;
+    uint32_t prefetch_ahead;   // CTAs between this one and the one whose first tiles it prefetches
 };
 
 __global__ void __launch_bounds__(BS_THR, 1)
@@ -253,6 +254,19 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             issue_loads();
             for (int it = 0; it < nit; ++it) {
                 const bool pass2 = it >= nch;
+                if (it == nch && p.prefetch_ahead) {
+                    // L2 prefetch of the first tiles of the CTA that runs about one wave later
+                    const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
+                    if (cid < gridDim.x * gridDim.y) {
+                        const int prb = cid % gridDim.x, pb = cid / gridDim.x;
+                        for (int cc = 0; cc < nch && cc < 2; ++cc) {
+                            tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
+                            tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 1, pb);
+                            tma_prefetch_5d(&tmDEp, 0, prb * TB / 2, 32 * cc, 0, pb);
+                            tma_prefetch_5d(&tmDEp, 0, prb * TB / 2, 32 * cc, 1, pb);
+                        }
+                    }
+                }
                 if (!mbar_wait(bar(BB_STAGE_DONE + (it & 3)), (it >> 2) & 1)) flag_timeout(p.status);
                 if (pass2) {
                     const int j0 = 32 * chunk_of(it);
@@ -542,6 +556,7 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
     p.status = a.status;
     p.n = d.n;
     p.npad = W.npad;
+    p.prefetch_ahead = (uint32_t)sm_count();
     k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, p);
     return cudaGetLastError();
 }

@@ -206,12 +206,14 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         if (!pass2 || !keep_s) tma_load_3d(slot_addr(it, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
                         if (pass2) tma_load_3d(slot_addr(it, vslot) + k * 4096, &tmV, fb, 64 * k, j0, b);
                     }
-                    if (!pass2 && it + FS_PF < nch) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (it + FS_PF), 0, b);
+                    if (!pass2 && it + FS_PF < nch)
+                        for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (it + FS_PF), s, b);
                     free_slots -= nslots(it);
                     ++next_load;
                 }
             };
-            for (int c = 0; c < nch && c < FS_PF; ++c) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * c, 0, b);
+            for (int c = 0; c < nch && c < FS_PF; ++c)
+                for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * c, s, b);
             issue_loads();
             for (int it = 0; it < nit; ++it) {
                 const bool pass2 = it >= nch;
@@ -221,7 +223,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     if (cid < gridDim.x * gridDim.y) {
                         const int prb = cid % gridDim.x, pb = cid / gridDim.x;
                         for (int cc = 0; cc < nch && cc < 2; ++cc)
-                            tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
+                            for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, s, pb);
                     }
                 }
                 if (!mbar_wait(bar(FB_STAGE_DONE + (it & 3)), (it >> 2) & 1)) flag_timeout(p.status);
