@@ -47,25 +47,25 @@ constexpr int FS_THR = NTHR + 64;         // 16 compute warps, the MMA warp, the
 struct FsSmem {
     static constexpr uint32_t WFE = FS_SLOTS * FS_SLOT;       // Wfe^T [16][64] swizzled (FiLM B)
     static constexpr uint32_t WE = WFE + 2048;                // We^T [64][16] no swizzle (edge-update B)
-    static constexpr uint32_t A = WE + 2048;                  // 2 tiles [128][16] no swizzle (edge-update A)
-    static constexpr uint32_t WST = A + 8192;                 // per-quadrant stats [4][8 i][8 h][2] f32
+    static constexpr uint32_t A = WE + 2048;                  // 2 buffers x 2 tiles [128][16] no swizzle (edge-update A)
+    static constexpr uint32_t WST = A + 16384;                // per-quadrant stats [4][8 i][8 h][2] f32
     static constexpr uint32_t FIN = WST + 2048;               // final m, 1/l [8][8][2]
     static constexpr uint32_t G = FIN + 512;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // mask of the graph's nodes [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;                // mbarriers, see below
-    static constexpr uint32_t TM = BAR + 8 * 14;              // TMEM base address
+    static constexpr uint32_t TM = BAR + 8 * 16;              // TMEM base address
     static constexpr uint32_t BYTES = TM + 16 + 1024;         // + alignment slack
     static constexpr uint32_t OPART = 0;                      // [4][8][256] f32 O partials (ring drained)
 };
-// mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full, edge_full, stage_done[4]
-constexpr int FB_FULL = 0, FB_FILM_FULL = 4, FB_FILM_EMPTY = 6, FB_A_FULL = 8, FB_EDGE_FULL = 9,
-              FB_STAGE_DONE = 10;
+// mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full[2], edge_full[2], stage_done[4]
+constexpr int FB_FULL = 0, FB_FILM_FULL = 4, FB_FILM_EMPTY = 6, FB_A_FULL = 8, FB_EDGE_FULL = 10,
+              FB_STAGE_DONE = 12;
 
-// TMEM columns: FiLM 0..63 (two buffers), edge update 64..191, pass-1 scores
-// from 192 on (16 per chunk, kept when nch <= 20 so pass 2 needs no K)
+// TMEM columns: FiLM 0..63 (two buffers), edge update 64..319 (two buffers),
+// pass-1 scores from 320 on (16 per chunk, kept when nch <= 12 so pass 2 needs no K)
 constexpr uint32_t FS_TM_COLS = 512;
-constexpr uint32_t FS_TM_FILM = 0, FS_TM_EDGE = 64, FS_TM_S = 192;
-constexpr int FS_KEEP_S_MAX_CHUNKS = (512 - 192) / 16;
+constexpr uint32_t FS_TM_FILM = 0, FS_TM_EDGE = 64, FS_TM_S = 320;
+constexpr int FS_KEEP_S_MAX_CHUNKS = (512 - 320) / 16;
 
 struct FwdParams {
     const __nv_bfloat16 *Q;
@@ -112,7 +112,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         mbar_init(bar(FB_FILM_EMPTY), NWARP);
         mbar_init(bar(FB_FILM_EMPTY + 1), NWARP);
         mbar_init(bar(FB_A_FULL), NWARP);
+        mbar_init(bar(FB_A_FULL + 1), NWARP);
         mbar_init(bar(FB_EDGE_FULL), 1);
+        mbar_init(bar(FB_EDGE_FULL + 1), 1);
         for (int k = 0; k < 4; ++k) mbar_init(bar(FB_STAGE_DONE + k), NWARP);
         fence_mbar_init();
     }
@@ -123,7 +125,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     // operand images: Wfe^T (FiLM B, swizzled) and We^T (edge-update B, no swizzle), 2 KB each
     if (tid < 256) reinterpret_cast<uint4 *>(sp + S::WFE)[tid] = reinterpret_cast<const uint4 *>(p.img)[tid];
     // edge-update A tiles: zero (the K half h >= 8 stays zero)
-    for (int e = tid; e < 8192 / 16; e += FS_THR) reinterpret_cast<uint4 *>(sp + S::A)[e] = make_uint4(0, 0, 0, 0);
+    for (int e = tid; e < 16384 / 16; e += FS_THR) reinterpret_cast<uint4 *>(sp + S::A)[e] = make_uint4(0, 0, 0, 0);
     if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
     for (int j = tid; j < 32 * nch; j += FS_THR) mj[j] = j < n ? p.M[(size_t)b * n + j] : 0;
     fence_proxy_async_smem();
@@ -149,13 +151,14 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
                 mma_commit(bar(FB_FILM_FULL + (it & 1)));
             };
-            auto issue_edge = [&]() {
+            auto issue_edge = [&](int p2) {   // pass-2 chunk p2: a buffer and TMEM buffer p2 & 1
                 tc_fence_after();
+                const uint32_t ab = S::A + (p2 & 1) * 8192, eb = FS_TM_EDGE + 128 * (p2 & 1);
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
-                    mma_bf16_ss(tmem + FS_TM_EDGE + 64 * e, smem_desc(sbase + S::A + e * 4096, 128, 256, LAYOUT_NONE),
+                    mma_bf16_ss(tmem + eb + 64 * e, smem_desc(sbase + ab + e * 4096, 128, 256, LAYOUT_NONE),
                                 smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
-                mma_commit(bar(FB_EDGE_FULL));
+                mma_commit(bar(FB_EDGE_FULL + (p2 & 1)));
             };
             // issue whichever product is ready first: FiLM of the next chunk (its
             // tiles landed, its TMEM buffer released) or the edge update of the
@@ -172,8 +175,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     progressed = true;
                 }
                 if (next_edge < nit && next_edge < next_film &&
-                    mbar_test_wait(bar(FB_A_FULL), (next_edge - nch) & 1)) {
-                    issue_edge();
+                    mbar_test_wait(bar(FB_A_FULL + ((next_edge - nch) & 1)), ((next_edge - nch) >> 1) & 1)) {
+                    issue_edge(next_edge - nch);
                     ++next_edge;
                     progressed = true;
                 }
@@ -275,6 +278,23 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 #pragma unroll
                 for (int x = 0; x < 4; ++x) oacc[hh][mt][x] = 0.f;
 
+        // E' = E + a We of pass-2 chunk it, in place (the TMA warp stores it)
+        auto edge_residual = [&](int it) {
+            const int p2 = it - nch;
+            if (!mbar_wait(bar(FB_EDGE_FULL + (p2 & 1)), (p2 >> 1) & 1)) flag_timeout(p.status);
+            tc_fence_after();
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float dv[16];
+                tmem_ld16(tl + FS_TM_EDGE + 128 * (p2 & 1) + 64 * e + 16 * hq, dv);
+                tmem_ld_wait();
+                add_residual16(sp + (slot_addr(it, e) - sbase) + L * 128, L, hq, dv);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
+        };
         for (int it = 0; it < nit; ++it) {
             const int j0 = 32 * chunk_of(it);
             const bool pass2 = it >= nch;
@@ -395,38 +415,29 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 continue;
             }
 
-            // ---------------- pass 2: normalised coefficients, edge-update A operand
+            // ---------------- pass 2, front of this chunk: normalised coefficients, a buffer p2 & 1
+            const int p2 = it - nch;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh)
                     sacc[hh][e] = valid[e] ? exp2f((sacc[hh][e] - fm[e][hh]) * LOG2E) * fl[e][hh] : 0.f;
-                *reinterpret_cast<uint32_t *>(sp + S::A + e * 4096 + ns16(L, 2 * hq)) =
+                *reinterpret_cast<uint32_t *>(sp + S::A + (p2 & 1) * 8192 + e * 4096 + ns16(L, 2 * hq)) =
                     pack_bf16(sacc[0][e], sacc[1][e]);
             }
             sacc[0][2] = sacc[0][3] = sacc[1][2] = sacc[1][3] = 0.f;
             fence_proxy_async_smem();
+            tc_fence_before();
             __syncwarp();
-            if (t == 0) mbar_arrive(bar(FB_A_FULL));
+            if (t == 0) mbar_arrive(bar(FB_A_FULL + (p2 & 1)));
 
             // ---------------- O += a V on warp MMAs (overlaps the edge MMAs)
             warp_contract2<1, true>(slot_addr(it, vslot), q, t, hq, sacc, oacc);
 
-            // ---------------- E' = E + a We, in place (the producer stores it)
-            if (!mbar_wait(bar(FB_EDGE_FULL), (it - nch) & 1)) flag_timeout(p.status);
-            tc_fence_after();
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float dv[16];
-                tmem_ld16(tl + FS_TM_EDGE + 64 * e + 16 * hq, dv);
-                tmem_ld_wait();
-                add_residual16(sp + (slot_addr(it, e) - sbase) + L * 128, L, hq, dv);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
+            // ---------------- back of the previous chunk, whose edge update ran meanwhile
+            if (p2 > 0) edge_residual(it - 1);
         }
+        if (nit > nch) edge_residual(nit - 1);
 
         // ---------------- O: sum over the quadrant warps (in the drained ring)
         named_bar_sync(2, FS_THR);
