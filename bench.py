@@ -39,7 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 # the dominant kernels on this workload, from the ncu capture summarised in
 # profiles/ (k_bwd_stream_sbm.md, k_fwd_stream_sbm.md).  They describe the
 # kernels as captured; a changed kernel reports null until it is re-captured.
-NCU_TRAFFIC = {("sbm", "k_bwd_stream"): 473985024, ("sbm", "k_fwd_stream"): 258154496}
+NCU_TRAFFIC = {("sbm", "k_bwd_stream"): 485526528, ("sbm", "k_fwd_stream"): 258202880}
 
 
 def env_rank():
@@ -279,7 +279,7 @@ def run_ours(args):
         "gpu_launches": launches,
     }
     if world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(p, d, W, args.cpu_graphs)
+        out["cpu_baseline"] = cpu_baseline(p, d, W, args.cpu_graphs, args.cpu_reps)
     return out
 
 
@@ -322,20 +322,22 @@ def run_e2e(args, buf, d, stream, step):
 # ------------------------------------------------------------------ oracle arm
 
 
-def cpu_baseline(p, d, W, graphs):
+def cpu_baseline(p, d, W, graphs, reps=1):
     """The fp64 oracle, as it stands, on a bounded sample: the first `graphs`
-    graphs of the batch, forward + backward, all usable host cores."""
+    graphs of the batch, forward + backward, `reps` times, all usable host cores."""
     import oracle
     oracle.build()
     sl = {k: d[k][:graphs] for k in ("X", "E", "y", "M", "dXout", "dEout")}
     dims = dict(H=p.H, dh=p.dh)
     t = time.perf_counter()
-    oracle.forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W)
-    oracle.backward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, sl["dXout"], sl["dEout"])
+    for _ in range(reps):
+        oracle.forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W)
+        oracle.backward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, sl["dXout"], sl["dEout"])
     dt = time.perf_counter() - t
-    pairs = graphs * p.n * p.n
+    pairs = reps * graphs * p.n * p.n
     return {"value": pairs / dt, "unit": UNIT, "cores": oracle.threads_used(), "kind": "oracle",
-            "sample": f"{graphs} of {p.B} graphs of the workload (n={p.n}), forward + backward, fp64",
+            "sample": f"{graphs} of {p.B} graphs of the workload (n={p.n}), forward + backward, fp64, "
+                      f"{reps} time(s)",
             "seconds": dt}
 
 
@@ -374,7 +376,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--cpu-graphs", type=int, default=16)
+    ap.add_argument("--cpu-graphs", type=int, default=32)
+    ap.add_argument("--cpu-reps", type=int, default=3)
     ap.add_argument("--ref-graphs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the step's kernels one by one")
