@@ -6,6 +6,8 @@
 #include "common.cuh"
 #include "generic.h"
 #include "fast.h"
+#include "sm100.cuh"
+#include <nvtx3/nvToolsExt.h>
 
 using namespace eaga;
 
@@ -65,9 +67,16 @@ size_t eaga_saved_size(const eaga_dims *d) {
     return saved_layout(*d).saved_total;
 }
 
+// NVTX range around an API call (visible to profilers that attach; inert otherwise).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+
 eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
                          const eaga_weights *w, void *Xout, void *Eout, void *saved, void *workspace,
                          size_t ws_bytes, void *stream) {
+    NvtxRange range("eaga_forward");
     eaga_status s = check_dims(d);
     if (s != EAGA_OK) return s;
     if ((s = check_weights(w)) != EAGA_OK) return s;
@@ -98,6 +107,7 @@ eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, cons
                           const eaga_weights *w, const void *saved, const void *dXout, const void *dEout,
                           void *dX, void *dE, void *dy, const eaga_weight_grads *dW, void *workspace,
                           size_t ws_bytes, void *stream) {
+    NvtxRange range("eaga_backward");
     eaga_status s = check_dims(d);
     if (s != EAGA_OK) return s;
     if ((s = check_weights(w)) != EAGA_OK) return s;
@@ -154,6 +164,27 @@ eaga_status eaga_debug_attention_map(const eaga_dims *d, const void *E, const ui
     a.A = A;
     a.g = A + (size_t)d->B * d->H * d->n * d->n;
     return launch_status(generic::attention_map(*d, a, static_cast<cudaStream_t>(stream)));
+}
+
+// One thread waits, with the pair kernels' bounded poll loop, on phase 0 of an
+// mbarrier that expects one arrival nobody makes.
+__global__ void k_wait_probe(int *status, unsigned limit) {
+    __shared__ __align__(8) unsigned long long bar;
+    const uint32_t b = sm100::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(b, 1);
+        sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !sm100::mbar_wait(b, 0, limit)) atomicExch(status, DEV_TIMEOUT);
+}
+
+eaga_status eaga_debug_wait_probe(void *workspace, unsigned limit, void *stream) {
+    if (!workspace || limit < 1 || limit > (1u << 24)) return EAGA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return EAGA_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    k_wait_probe<<<1, 32, 0, st>>>(static_cast<int *>(workspace), limit);
+    return cudaGetLastError() == cudaSuccess ? EAGA_OK : EAGA_ERR_CUDA;
 }
 
 eaga_status eaga_get_device_status(void *workspace, void *stream) {

@@ -46,7 +46,7 @@ __host__ __device__ __forceinline__ uint32_t ns16(uint32_t row, uint32_t k) {
 
 // Workspace of the fast path (after the common status word and g).
 struct FastWs {
-    size_t img, dO, dQ, dK, dV, D, Pa, Pds, rparts, wparts, bparts, r2, dg, total;
+    size_t img, dO, dQ, dK, dV, Pa, Pds, rparts, wparts, bparts, r2, dg, total;
     int n_rparts, wsplits, bsplits, rsplits, npad;
 };
 
@@ -67,7 +67,6 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
     W.dQ = off; off = align256(off + rows * HD * 2);
     W.dK = off; off = align256(off + rows * HD * 2);
     W.dV = off; off = align256(off + rows * HD * 2);
-    W.D = off; off = align256(off + size_t(d.B) * NH * d.n * 4);
     // a and ds of every pair, [B][H][n][npad] bf16, for the dk / dv pass
     W.npad = (d.n + 7) / 8 * 8;
     W.Pa = off; off = align256(off + size_t(d.B) * NH * d.n * W.npad * 2);

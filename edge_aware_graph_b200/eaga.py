@@ -21,7 +21,7 @@ STATUS = {0: "EAGA_OK", 1: "EAGA_ERR_INVALID_ARG", 2: "EAGA_ERR_UNSUPPORTED", 3:
           4: "EAGA_ERR_WORKSPACE", 5: "EAGA_ERR_CUDA", 6: "EAGA_ERR_TIMEOUT"}
 EXPORTED = ("eaga_workspace_size", "eaga_saved_size", "eaga_forward", "eaga_backward",
             "eaga_debug_attention_map", "eaga_get_device_status", "eaga_strerror",
-            "eaga_set_profile_events", "eaga_kernel_launches", "eaga_forward_noalloc")
+            "eaga_set_profile_events", "eaga_kernel_launches", "eaga_forward_noalloc", "eaga_debug_wait_probe")
 
 
 class Dims(ctypes.Structure):
@@ -67,6 +67,8 @@ def lib():
         L.eaga_debug_attention_map.restype = i32
         L.eaga_get_device_status.argtypes = [vp, vp]
         L.eaga_get_device_status.restype = i32
+        L.eaga_debug_wait_probe.argtypes = [vp, ctypes.c_uint, vp]
+        L.eaga_debug_wait_probe.restype = i32
         L.eaga_set_profile_events.argtypes = [i32, vp, vp]
         L.eaga_set_profile_events.restype = i32
         L.eaga_kernel_launches.argtypes = [ctypes.POINTER(Dims), i32]
@@ -140,6 +142,12 @@ def debug_attention_map(d: Dims, E, M, W: dict, y, saved, A, stream=None):
 
 def get_device_status(workspace, stream=None) -> int:
     return int(lib().eaga_get_device_status(_p(workspace), _stream(stream)))
+
+
+def debug_wait_probe(workspace, limit: int, stream=None):
+    """Run the bounded-wait failure path once (test aid): a wait that never
+    completes gives up after `limit` polls and records a timeout."""
+    _check(lib().eaga_debug_wait_probe(_p(workspace), int(limit), _stream(stream)), "eaga_debug_wait_probe")
 
 
 def set_profile_events(point: int, before=None, after=None):

@@ -183,6 +183,16 @@ EAGA_API eaga_status eaga_set_profile_events(int point, void *before, void *afte
  * these dims; -1 for invalid or unsupported dims. */
 EAGA_API int eaga_kernel_launches(const eaga_dims *dims, int for_backward);
 
+/* Test aid for the failure path of the bounded device waits.  Launches one
+ * small kernel that waits on an mbarrier nothing will ever complete, with the
+ * same bounded poll loop the pair kernels use, for `limit` polls
+ * (1 <= limit <= 2^24); when the limit runs out the kernel records the
+ * timeout in the status word at the start of `workspace` and returns, the
+ * way a pair kernel does (no trap, the context stays usable).  A following
+ * eaga_get_device_status on that workspace returns EAGA_ERR_TIMEOUT.  The
+ * pages have no counterpart. */
+EAGA_API eaga_status eaga_debug_wait_probe(void *workspace, unsigned limit, void *stream);
+
 /* Static, human-readable name of a status code. */
 EAGA_API const char *eaga_strerror(eaga_status s);
 

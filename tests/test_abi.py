@@ -95,3 +95,12 @@ def test_strerror(L):
     for code in range(7):
         assert eaga.strerror(code)
     assert eaga.strerror(99) == "unknown status"
+
+
+def test_wait_probe_arguments(L):
+    # argument checks happen on the host, before any launch
+    assert L.eaga_debug_wait_probe(None, 100, None) == 1           # EAGA_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(0x100000)
+    assert L.eaga_debug_wait_probe(fake, 0, None) == 1
+    assert L.eaga_debug_wait_probe(fake, (1 << 24) + 1, None) == 1
+    assert L.eaga_debug_wait_probe(ctypes.c_void_p(0x100008), 100, None) == 3   # misaligned

@@ -214,3 +214,39 @@ def test_device_status_ok():
     buf = make(p, d, W, backward=False)
     buf.forward()
     assert eaga.get_device_status(buf.ws_fwd) == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(oracle_lib):
+    """A device wait that can never complete gives up after its poll limit,
+    the status word reports EAGA_ERR_TIMEOUT, and the next calls run normally."""
+    from edge_aware_graph_b200 import eaga
+    p, d, W = custom_case(2, 64, 256, 64, 64, 8, 32, "bf16", seed=5, mask="random", with_grads=False)
+    buf = make(p, d, W, backward=False)
+    eaga.debug_wait_probe(buf.ws_fwd, 2000)
+    torch.cuda.synchronize()
+    assert eaga.get_device_status(buf.ws_fwd) == 6            # EAGA_ERR_TIMEOUT
+    assert eaga.get_device_status(buf.ws_fwd) == 0            # reading it cleared it
+    buf.forward()
+    torch.cuda.synchronize()
+    assert eaga.get_device_status(buf.ws_fwd) == 0
+    check_forward(buf, oracle_forward(oracle_lib, p, d, W), TOL["bf16"])
+
+
+def test_calls_allocate_no_device_memory():
+    """After the first calls (library load, streams), forward and backward
+    leave the device's free memory and torch's allocations unchanged."""
+    p = I.preset("sbm", B=4)
+    d = I.draw_inputs(p, with_grads=True)
+    W = I.draw_weights(p)
+    buf = make(p, d, W, backward=True)
+    for _ in range(2):
+        buf.forward()
+        buf.backward()
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    for _ in range(3):
+        buf.forward()
+        buf.backward()
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
