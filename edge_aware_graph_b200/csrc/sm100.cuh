@@ -1,7 +1,7 @@
 // Inline-PTX building blocks for sm_100a: mbarriers with bounded waits, TMA
 // tile loads/stores (no multicast), tcgen05 (TMEM allocation, MMA with shared
-// memory descriptors, loads), thread-block-cluster barriers and distributed
-// shared memory, and the warp-level bf16 MMA used for the attention core.
+// memory descriptors, loads and stores), named CTA barriers, and the
+// warp-level bf16 MMA used for the attention core.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -80,14 +80,6 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
         "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
-__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1,
-                                            int c2, int c3, int c4) {
-    asm volatile(
-        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, "
-        "%6, %7}], [%2];" ::"r"(dst),
-        "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-        : "memory");
-}
 // L2 eviction policies for the cache-hinted TMA copies below.
 __device__ __forceinline__ uint64_t l2_evict_last() {
     uint64_t pol;
@@ -121,18 +113,6 @@ __device__ __forceinline__ void tma_prefetch_5d(const CUtensorMap *map, int c0, 
                  "r"(c1), "r"(c2), "r"(c3), "r"(c4)
                  : "memory");
 }
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(c0), "r"(c1),
-                 "r"(c2)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, int c3,
-                                             int c4) {
-    asm volatile("cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(
-                     map),
-                 "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-                 : "memory");
-}
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void tma_store_wait_read0() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
@@ -140,12 +120,8 @@ __device__ __forceinline__ void tma_store_wait_read0() {
 __device__ __forceinline__ void tma_store_wait_read1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
-__device__ __forceinline__ void tma_store_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -231,61 +207,11 @@ __device__ __forceinline__ void tmem_st2(uint32_t taddr, float v0, float v1) {
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// ------------------------------------------------------------------ cluster
+// ------------------------------------------------------------------ CTA barriers
 
 // Barrier `id` (1..15) among `nthreads` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Asynchronous store into a (possibly remote) CTA's shared memory; the bytes
-// are counted on that CTA's mbarrier `cbar` (both shared::cluster addresses).
-__device__ __forceinline__ void st_async_v2(uint32_t caddr, float a, float b, uint32_t cbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(caddr),
-                 "f"(a), "f"(b), "r"(cbar)
-                 : "memory");
-}
-__device__ __forceinline__ void st_async_f32(uint32_t caddr, float a, uint32_t cbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(caddr),
-                 "r"(__float_as_uint(a)), "r"(cbar)
-                 : "memory");
-}
-__device__ __forceinline__ void st_async_v4(uint32_t caddr, float4 v, uint32_t cbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     caddr),
-                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cbar)
-                 : "memory");
-}
-// Split cluster barrier: arrive now (after the last read of a peer's shared
-// memory), wait later (before this CTA's shared memory may disappear).
-__device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-__device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ float ld_peer_f32(uint32_t caddr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr) : "memory");
-    return v;
-}
-__device__ __forceinline__ float4 ld_peer_f32x4(uint32_t caddr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(caddr)
-                 : "memory");
-    return v;
 }
 
 // ------------------------------------------------------------------ warp MMA
@@ -297,12 +223,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ void mma1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(b0));
-}
 __device__ __forceinline__ void ldsm_x4(uint32_t saddr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -312,14 +232,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t saddr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(saddr));
-}
-__device__ __forceinline__ void ldsm_x2_t(uint32_t saddr, uint32_t &r0, uint32_t &r1) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-                 : "=r"(r0), "=r"(r1)
-                 : "r"(saddr));
-}
-__device__ __forceinline__ void ldsm_x2(uint32_t saddr, uint32_t &r0, uint32_t &r1) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(saddr));
 }
 // Transpose of an 8x8 b16 matrix held in the mma fragment layout.
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
