@@ -50,9 +50,8 @@ constexpr int BS_KEEP_MAX_CHUNKS = 7;     // S and dP of up to 7 chunks (n <= 22
 
 struct BsSmem {
     static constexpr uint32_t IMG = BS_SLOTS * BS_SLOT;       // Wfe^T sw (FiLM), We sw (u), Wfe ns (dE): 2 KB each
-    static constexpr uint32_t DF = IMG + 6144;                // 2 tiles [128][16] ns: [dgamma | dbeta]
-    static constexpr uint32_t AT = DF + 8192;                 // 2 tiles [128][16] ns: a (h >= 8 zero)
-    static constexpr uint32_t WD = AT + 8192;                 // per-quadrant D [4][8 i][8 h]
+    static constexpr uint32_t DA = IMG + 6144;                // 2 tiles [128][32] ns: [dgamma | dbeta | a | 0]
+    static constexpr uint32_t WD = DA + 16384;                // per-quadrant D [4][8 i][8 h]
     static constexpr uint32_t WDG = WD + 1024;                // per-warp dg [16][4]
     static constexpr uint32_t G = WDG + 256;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // node mask [n <= 1024]
@@ -67,10 +66,18 @@ constexpr int BB_FULL = 0, BB_FILM_FULL = 4, BB_FILM_EMPTY = 6, BB_DF_FULL = 8, 
               BB_STAGE_DONE = 10;
 
 // TMEM: FiLM 0..63 and u 64..127 (two buffers each), dE 128..255, kept S / dP
-// 256..479 (32 per chunk), dWfe [64 c][16 k] at 480, dWe^T [64 c][16 h] at 496
-// (M = 64 accumulators: row m in lane m%16 + 32(m/16))
+// 256..479 (32 per chunk), and at 480 the weight-gradient accumulator
+// [E | dE']^T [df | a]: lanes 0..63 the E channels, 64..127 the dE' channels,
+// columns 0..31 the df and a columns; its blocks E^T df = dWfe [c][k] and
+// dE'^T a = dWe^T [c][h] are the ones used
 constexpr uint32_t BS_TM_COLS = 512, BS_TM_FILM = 0, BS_TM_U = 64, BS_TM_DE = 128, BS_TM_KEEP = 256,
-                   BS_TM_WFE = 480, BS_TM_WE = 496;
+                   BS_TM_W = 480;
+
+// Byte offset of element (row, col) of a [128][32] bf16 tile in 8 x 8 core
+// matrices: 128 B apart along the columns, 512 B along the rows.
+__device__ __forceinline__ uint32_t ns32(uint32_t row, uint32_t col) {
+    return (row >> 3) * 512u + (col >> 3) * 128u + (row & 7u) * 16u + (col & 7u) * 2u;
+}
 
 struct BwdStreamParams {
     const __nv_bfloat16 *Q, *dO;
@@ -132,8 +139,8 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         const uint32_t img_off = (tid >> 7) == 0 ? IMG_WFE_T_SW : (tid >> 7) == 1 ? IMG_WE_SW : IMG_WFE_NS;
         reinterpret_cast<uint4 *>(sp + S::IMG)[tid] = reinterpret_cast<const uint4 *>(p.img)[(img_off >> 4) + (tid & 127)];
     }
-    // a tiles: the K half h >= 8 stays zero
-    for (int e = tid; e < 8192 / 16; e += BS_THR) reinterpret_cast<uint4 *>(sp + S::AT)[e] = make_uint4(0, 0, 0, 0);
+    // [df | a] tiles: columns 24..31 (a of h >= 8) stay zero
+    for (int e = tid; e < 16384 / 16; e += BS_THR) reinterpret_cast<uint4 *>(sp + S::DA)[e] = make_uint4(0, 0, 0, 0);
     if (tid < NF) g[tid] = p.g[(size_t)b * NF + tid];
     for (int j = tid; j < 32 * nch; j += BS_THR) mj[j] = j < n ? p.M[(size_t)b * n + j] : 0;
     fence_proxy_async_smem();
@@ -146,7 +153,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         // ================= MMA issuer
         if (t == 0) {
             const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_d = idesc_bf16_f32(128, DE);
-            const uint32_t idesc_w = idesc_bf16_f32_mn(64, NF);
+            const uint32_t idesc_w = idesc_bf16_f32_mn(128, 2 * NF);
             auto issue_fu = [&](int it) {
                 tc_fence_after();
 #pragma unroll
@@ -169,22 +176,22 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 tc_fence_after();
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
-                    mma_bf16_ss(tmem + BS_TM_DE + 64 * e, smem_desc(sbase + S::DF + e * 4096, 128, 256, LAYOUT_NONE),
+                    mma_bf16_ss(tmem + BS_TM_DE + 64 * e, smem_desc(sbase + S::DA + e * 8192, 128, 512, LAYOUT_NONE),
                                 smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_d, 0);
-                // dWfe [c][k] += sum_pairs E[pair][c] df[pair][k], dWe^T [c][h] += sum_pairs dE'[pair][c] a[pair][h]:
-                // A = the pair tile read MN-major (64 c per 128-byte swizzled row, 8-row groups 1024 B
-                // apart), B = the df / a tile read MN-major (8 x 8 core matrices: 128 B along N,
-                // 256 B along K); 16 pairs per MMA
+                // [dWfe | .] and [. | dWe^T] in one product: A = the E tile and the dE' tile read
+                // MN-major as the two 64-channel atoms of M = 128 (64 c per 128-byte swizzled row,
+                // 8-row groups 1024 B apart; the second atom one slot distance further: the
+                // TMA warp hands out slots in increasing order, so the dE' slot of a parity
+                // half lies above its E slot); B = the [df | a] tile read MN-major (8 x 8 core
+                // matrices: 128 B along N, 512 B along K); 16 pairs per MMA
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const uint32_t te = slot_addr(it, e), td = slot_addr(it, 2 + e);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t acc = (it > nch || e > 0 || ks > 0) ? 1u : 0u;
-                        mma_bf16_ss(tmem + BS_TM_WFE, smem_desc(te + ks * 2048, 16, 1024, LAYOUT_SW128),
-                                    smem_desc(sbase + S::DF + e * 4096 + ks * 512, 256, 128, LAYOUT_NONE), idesc_w, acc);
-                        mma_bf16_ss(tmem + BS_TM_WE, smem_desc(td + ks * 2048, 16, 1024, LAYOUT_SW128),
-                                    smem_desc(sbase + S::AT + e * 4096 + ks * 512, 256, 128, LAYOUT_NONE), idesc_w, acc);
+                        mma_bf16_ss(tmem + BS_TM_W, smem_desc(te + ks * 2048, td - te, 1024, LAYOUT_SW128),
+                                    smem_desc(sbase + S::DA + e * 8192 + ks * 1024, 512, 128, LAYOUT_NONE), idesc_w, acc);
                     }
                 }
                 mma_commit(bar(BB_DE_FULL));
@@ -420,9 +427,9 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     dgp[hh] += dgam[hh];
                     dgp[2 + hh] += dbet[hh];
                 }
-                *reinterpret_cast<uint32_t *>(sp + S::DF + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(dgam[0], dgam[1]);
-                *reinterpret_cast<uint32_t *>(sp + S::DF + e * 4096 + ns16(L, NH + 2 * hq)) = pack_bf16(dbet[0], dbet[1]);
-                *reinterpret_cast<uint32_t *>(sp + S::AT + e * 4096 + ns16(L, 2 * hq)) = pack_bf16(av[0][e], av[1][e]);
+                *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, 2 * hq)) = pack_bf16(dgam[0], dgam[1]);
+                *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, NH + 2 * hq)) = pack_bf16(dbet[0], dbet[1]);
+                *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, NF + 2 * hq)) = pack_bf16(av[0][e], av[1][e]);
             }
             av[0][2] = av[0][3] = av[1][2] = av[1][3] = 0.f;
             da[0][2] = da[0][3] = da[1][2] = da[1][3] = 0.f;
@@ -494,24 +501,23 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             }
             *reinterpret_cast<uint32_t *>(p.dQ + ((size_t)b * n + i0 + il) * HD + d) = pack_bf16(o0 * rs, o1 * rs);
         }
-        // weight-gradient partials of the row block: dWfe [c][k] and dWe^T [c][h]
-        // from the M = 64 TMEM accumulators (row c in lane c%16 of quadrant c/16),
-        // dg from the per-warp sums
+        // weight-gradient partials of the row block: dWfe [c][k] from lanes 0..63,
+        // columns 0..15 of the accumulator, dWe^T [c][h] from lanes 64..127,
+        // columns 16..23; dg from the per-warp sums
         float *rp = p.rparts + (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * RPART;
         tc_fence_after();
-        if (hq < 2) {
+        if (hq == 0) {
             float v[16];
-            tmem_ld16(tl + (hq == 0 ? BS_TM_WFE : BS_TM_WE), v);
+            tmem_ld16(tl + BS_TM_W + (q < 2 ? 0 : NF), v);
             tmem_ld_wait();
-            if (t < 16) {
-                const int c = 16 * q + t;
-                if (hq == 0) {
+            if (q < 2) {
+                const int c = 32 * q + t;
 #pragma unroll
-                    for (int k = 0; k < NF; ++k) rp[c * NF + k] = v[k];
-                } else {
+                for (int k = 0; k < NF; ++k) rp[c * NF + k] = v[k];
+            } else {
+                const int c = 32 * (q - 2) + t;
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) rp[DE * NF + h * DE + c] = v[h];
-                }
+                for (int h = 0; h < NH; ++h) rp[DE * NF + h * DE + c] = v[h];
             }
         }
         if (tid < NF) {
