@@ -31,6 +31,10 @@ if ROOT not in sys.path:
 import numpy as np
 
 WORKLOAD = "sbm"
+# --workload: the training step (default), or the sampling-time forward on
+# Planar- / Tree-shaped batches (forward only, many calls per model)
+WORKLOADS = {"sbm-train": "sbm", "planar-sample": "planar", "tree-sample": "tree"}
+SAMPLE_ROTATION = 6     # batches cycled by the sampling workload: 6 x ~77 MB > L2
 METRIC = "edge-pairs/sec (B·n²) fwd and fwd+bwd on 1 B200; % of HBM roofline"
 UNIT = "edge-pairs/s"
 FALLBACK_HBM_GBS = 6650.0
@@ -134,6 +138,8 @@ def pair_kernel_bytes(p, which):
 
 
 def run_ours(args):
+    if args.workload != "sbm-train":
+        return run_sample(args, WORKLOADS[args.workload])
     import torch
     import torch.distributed as dist
 
@@ -285,6 +291,172 @@ def run_ours(args):
     return out
 
 
+def run_sample(args, name):
+    """Sampling-time forward: the forward alone, called once per step on one of
+    SAMPLE_ROTATION resident batches in turn (inputs larger than L2), the
+    rotation's calls replayed as one CUDA graph."""
+    import torch
+    import torch.distributed as dist
+
+    from edge_aware_graph_b200 import dp, eaga
+    from edge_aware_graph_b200 import inputs as I
+    from edge_aware_graph_b200.buffers import LayerBuffers, host_to_storage_tensor
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    p0 = I.preset(name)
+    R = SAMPLE_ROTATION
+    W = I.draw_weights(p0)                          # one model on every rank
+    bufs, ds = [], []
+    for r in range(R):
+        p = I.preset(name, seed=dp.rank_seed(p0.seed, rank * R + r))
+        d = I.draw_inputs(p, with_grads=False)
+        buf = LayerBuffers(p.B, p.n, p.dx, p.de, p.dy, p.H, p.dh, dtype=p.dtype, backward=False)
+        buf.load_inputs(d, W)
+        bufs.append(buf)
+        ds.append(d)
+    stream = torch.cuda.current_stream()
+
+    def call(r, s):
+        bufs[r].forward(s)
+
+    for k in range(max(args.warmup, R)):
+        call(k % R, stream)
+    torch.cuda.synchronize()
+
+    # ---- forward pair kernel times: eager calls with CUDA events around it
+    nk = min(args.steps, 24)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+    for a, b in ev:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    for k in range(nk):
+        eaga.set_profile_events(0, *ev[k])
+        call(k % R, stream)
+    torch.cuda.synchronize()
+    eaga.set_profile_events(0)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            for r in range(R):
+                call(r, cap)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=cap):
+            for r in range(R):
+                call(r, cap)
+        torch.cuda.synchronize()
+
+    def rotation():
+        if graph is not None:
+            graph.replay()
+        else:
+            for r in range(R):
+                call(r, stream)
+
+    rotation()
+    reps = max(1, (args.steps + R - 1) // R)
+    K = reps * R
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for _ in range(reps):
+        rotation()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms_total = dp.max_over_ranks(t0.elapsed_time(t1), "cuda")
+    if graph is not None:
+        del graph
+
+    # ---- end to end through the public API: inputs from pinned host memory,
+    # X' and E' read back, every call
+    host_in = [{k: host_to_storage_tensor(d[k], bufs[0].dtype).pin_memory() for k in ("X", "E", "y")}
+               for d in ds]
+    host_M = [torch.from_numpy(np.ascontiguousarray(d["M"])).pin_memory() for d in ds]
+    host_out = [(torch.empty(b.Xout.shape, dtype=b.Xout.dtype).pin_memory(),
+                 torch.empty(b.Eout.shape, dtype=b.Eout.dtype).pin_memory()) for b in bufs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in[0].values()) + host_M[0].numel()
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
+
+    def e2e_call(r):
+        b = bufs[r]
+        for k in ("X", "E", "y"):
+            getattr(b, k).copy_(host_in[r][k], non_blocking=True)
+        b.M.copy_(host_M[r], non_blocking=True)
+        call(r, stream)
+        host_out[r][0].copy_(b.Xout, non_blocking=True)
+        host_out[r][1].copy_(b.Eout, non_blocking=True)
+
+    for r in range(R):
+        e2e_call(r)
+    torch.cuda.synchronize()
+    ne = max(args.e2e_steps, R)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(ne):
+        e2e_call(k % R)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1) / ne, "cuda")
+
+    launches = eaga.kernel_launches(bufs[0].dims, False) * K
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    pairs_call = p0.B * p0.n * p0.n
+    value = world * pairs_call * K / (ms_total / 1e3)
+    peak, peak_kind = measured_peaks()
+    kf = pair_kernel_bytes(p0, "fwd")
+    achieved = kf / (fwd_ms / 1e3) / 1e9
+    call_bytes = compulsory_bytes(p0, training=False)
+    ms_call = ms_total / K
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_call, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": f"synthetic (seeded {name.capitalize()}-shaped graphs; edge_aware_graph_b200/inputs.py)",
+        "config": {"workload": f"{name}-shaped sampling-time forward: B={p0.B}, n={p0.n} (all nodes real), "
+                               f"dx={p0.dx} de={p0.de} dy={p0.dy} H={p0.H} dh={p0.dh}, bf16 storage / fp32 "
+                               "accumulation, saved state written",
+                   "global_batch": p0.B * world, "seq_len": p0.n, "parallelism": f"dp{world}",
+                   "l2": f"inputs larger than L2: {R} resident batches called in turn "
+                         f"(E {p0.B * p0.n * p0.n * p0.de * 2 / 2**20:.0f} MiB each)",
+                   "launch": (f"CUDA graph of {R} forward calls" if not args.no_graph else "eager")},
+        "roofline": {"bound": "hbm", "kernel": "k_fwd_stream (forward pair kernel)", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": NCU_TRAFFIC.get((name, "k_fwd_stream")),
+                     "algorithmic_bytes": kf, "ms_per_launch": fwd_ms},
+        "step_roofline": {"compulsory_bytes": call_bytes, "achieved_gbs": call_bytes / (ms_call / 1e3) / 1e9,
+                          "frac_of_measured": call_bytes / (ms_call / 1e3) / 1e9 / peak,
+                          "frac_of_8tbs": call_bytes / (ms_call / 1e3) / 1e9 / 8000.0},
+        "clocks": clk,
+        "e2e": {"value": world * pairs_call / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ne},
+        "gpu_launches": launches,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_forward(p0, ds[0], W, args.cpu_seconds)
+    return out
+
+
 def run_e2e(args, buf, d, stream, step):
     """Steps whose timed region includes the pinned-host -> device copy of the
     step's inputs and the device -> host read of its results."""
@@ -343,11 +515,32 @@ def cpu_baseline(p, d, W, graphs, reps=1):
             "seconds": dt}
 
 
+def cpu_baseline_forward(p, d, W, min_seconds):
+    """The fp64 oracle, as it stands, on the forward of the whole batch,
+    repeated until `min_seconds` have passed (a bounded sample)."""
+    import oracle
+    oracle.build()
+    dims = dict(H=p.H, dh=p.dh)
+    reps, t = 0, time.perf_counter()
+    while True:
+        oracle.forward(dims, d["X"], d["E"], d["y"], d["M"], W)
+        reps += 1
+        dt = time.perf_counter() - t
+        if dt >= min_seconds or reps >= 1000:
+            break
+    pairs = reps * p.B * p.n * p.n
+    return {"value": pairs / dt, "unit": UNIT, "cores": oracle.threads_used(), "kind": "oracle",
+            "sample": f"the forward of all {p.B} graphs of the batch (n={p.n}), fp64, {reps} time(s)",
+            "seconds": dt}
+
+
 def run_reference(args):
     rank, world, _ = env_rank()
     if rank != 0:
         return None
     from edge_aware_graph_b200 import inputs as I
+    if args.workload != "sbm-train":
+        return run_reference_sample(args, WORKLOADS[args.workload], world)
     p = I.preset(WORKLOAD)
     d = I.draw_inputs(p, with_grads=True)
     W = I.draw_weights(p)
@@ -371,6 +564,36 @@ def run_reference(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_reference_sample(args, name, world):
+    """The oracle arm of the sampling workload: the oracle's forward on
+    --ref-graphs graphs of the batch per step."""
+    from edge_aware_graph_b200 import inputs as I
+    p = I.preset(name)
+    d = I.draw_inputs(p, with_grads=False)
+    W = I.draw_weights(p)
+    import oracle
+    oracle.build()
+    g = max(1, min(args.ref_graphs, p.B))
+    sl = {k: d[k][:g] for k in ("X", "E", "y", "M")}
+    dims = dict(H=p.H, dh=p.dh)
+    for _ in range(args.warmup):
+        oracle.forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W)
+    secs = time.perf_counter() - t
+    value = args.steps * g * p.n * p.n / secs
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": f"synthetic (seeded {name.capitalize()}-shaped graphs)",
+            "config": {"workload": f"{name}-shaped sampling-time forward, bounded sample of {g} graph(s) "
+                                   "per step", "global_batch": g, "seq_len": p.n, "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads_used(), "kind": "oracle",
+                             "sample": f"the forward of {g} of {p.B} graphs (n={p.n}), fp64, per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,6 +606,11 @@ def main():
     ap.add_argument("--ref-graphs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the step's kernels one by one")
+    ap.add_argument("--workload", default="sbm-train", choices=list(WORKLOADS),
+                    help="sbm-train: the training step (default); planar-sample / tree-sample: the "
+                         "sampling-time forward on Planar- / Tree-shaped batches")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="sampling workloads: seconds of oracle forward calls in cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
