@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <atomic>
 #include "eaga.h"
 
 namespace eaga {
@@ -76,10 +77,26 @@ inline WsLayout ws_layout(const eaga_dims &d) {
 }
 
 // Optional profiling events around the pair kernels (eaga_set_profile_events).
-extern void *g_prof_events[3][2];
+extern std::atomic<void *> g_prof_events[3][2];
 inline void prof_mark(int point, int which, cudaStream_t st) {
-    void *ev = g_prof_events[point][which];
+    void *ev = g_prof_events[point][which].load(std::memory_order_acquire);
     if (ev) cudaEventRecord(static_cast<cudaEvent_t>(ev), st);
+}
+
+// Opt `kernel` in to `bytes` of dynamic shared memory on the current device,
+// once per device (function attributes are per device).  `done` is the
+// caller's per-kernel mask of devices already set; concurrent callers may both
+// set the attribute, which is harmless.
+template <typename K>
+inline cudaError_t ensure_smem_attr(K kernel, int bytes, std::atomic<uint32_t> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint32_t bit = dev < 32 ? 1u << dev : 0u;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
 }
 
 // Device status word values (first int of the workspace).

@@ -12,7 +12,7 @@
 using namespace eaga;
 
 namespace eaga {
-void *g_prof_events[3][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+std::atomic<void *> g_prof_events[3][2] = {};
 }
 
 namespace {
@@ -201,8 +201,8 @@ eaga_status eaga_get_device_status(void *workspace, void *stream) {
 eaga_status eaga_set_profile_events(int point, void *before, void *after) {
     if (point < 0 || point > 2) return EAGA_ERR_INVALID_ARG;
     if ((before == nullptr) != (after == nullptr)) return EAGA_ERR_INVALID_ARG;
-    g_prof_events[point][0] = before;
-    g_prof_events[point][1] = after;
+    g_prof_events[point][0].store(before, std::memory_order_release);
+    g_prof_events[point][1].store(after, std::memory_order_release);
     return EAGA_OK;
 }
 

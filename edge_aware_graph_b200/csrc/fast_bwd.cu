@@ -266,12 +266,8 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
 // Row pair kernel, then dk / dv from its a and ds.
 cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                              cudaStream_t st) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_bwd_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, KvSmem::BYTES);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    static std::atomic<uint32_t> attr_set{0};
+    if (cudaError_t e = ensure_smem_attr(k_bwd_kv, KvSmem::BYTES, attr_set); e != cudaSuccess) return e;
     prof_mark(2, 0, st);
     {
         cudaError_t e = launch_bwd_stream(d, a, W, ws, g, st);

@@ -10,17 +10,13 @@ namespace fast {
 
 constexpr int DE = 64, NH = 8, DH = 32, HD = 256, NF = 16;
 constexpr int TB = 8;            // query rows per pair-kernel CTA (one row block)
-// Streaming multiprocessors of the current device (cached per process).
+// Streaming multiprocessors of the current device.
 inline int sm_count() {
-    static int cached = 0;
-    if (!cached) {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-            cached = v;
-        else
-            cached = 148;
-    }
-    return cached;
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        v > 0)
+        return v;
+    return 148;
 }
 
 // Operand images prepared once per call by the prologue kernel (bf16, in the

@@ -465,12 +465,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 
 cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
                              cudaStream_t st) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_fwd_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, FsSmem::BYTES);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    static std::atomic<uint32_t> attr_set{0};
+    if (cudaError_t e = ensure_smem_attr(k_fwd_stream, FsSmem::BYTES, attr_set); e != cudaSuccess) return e;
     CUtensorMap mE, mEo, mK, mV;
     if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mEo, a.Eout, d.B, d.n, false, 32, 1) ||
         !encode_node_map(&mK, a.K, d.B, d.n, 32) || !encode_node_map(&mV, a.V, d.B, d.n, 32))

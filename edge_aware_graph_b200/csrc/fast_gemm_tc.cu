@@ -295,13 +295,8 @@ bool encode_2d(CUtensorMap *m, const void *base, int rows, int cols, int box_row
 template <int BN>
 static cudaError_t tc_launch(const CUtensorMap (&am)[3], const CUtensorMap (&bm)[3], const TcParams &p, int N,
                              cudaStream_t st) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             TcSmem<BN>::BYTES);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    static std::atomic<uint32_t> attr_set{0};
+    if (cudaError_t e = ensure_smem_attr(k_tc_gemm<BN>, TcSmem<BN>::BYTES, attr_set); e != cudaSuccess) return e;
     dim3 grid(N / BN, (p.M + TBM - 1) / TBM);
     k_tc_gemm<BN><<<grid, TTHR, TcSmem<BN>::BYTES, st>>>(am[0], am[1], am[2], bm[0], bm[1], bm[2], p);
     return cudaGetLastError();
@@ -340,13 +335,8 @@ static bool encode_mn(CUtensorMap *m, const void *base, int rows, int cols) { re
 template <int BN>
 static cudaError_t wg_launch(const CUtensorMap &am, const CUtensorMap (&bm)[3], const WgParams &p, int N, int splits,
                              cudaStream_t st) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_tc_wgrad<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             WgSmem<BN>::BYTES);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    static std::atomic<uint32_t> attr_set{0};
+    if (cudaError_t e = ensure_smem_attr(k_tc_wgrad<BN>, WgSmem<BN>::BYTES, attr_set); e != cudaSuccess) return e;
     dim3 grid(N / BN, (p.M + TBM - 1) / TBM, splits);
     k_tc_wgrad<BN><<<grid, TTHR, WgSmem<BN>::BYTES, st>>>(am, bm[0], bm[1], bm[2], p);
     return cudaGetLastError();

@@ -38,9 +38,10 @@
  *     launch errors only; device-side conditions (a bounded wait that ran out)
  *     are recorded in the workspace status word and read by
  *     eaga_get_device_status.
- *   - No global state besides cached kernel attributes and the optional
- *     profiling events; calls on distinct streams with distinct workspaces
- *     are thread-safe.
+ *   - No global state besides per-device cached kernel attributes, the
+ *     backward's per-device auxiliary streams and the optional profiling
+ *     events; calls on distinct streams with distinct workspaces are
+ *     thread-safe, also across devices of one process.
  */
 #ifndef EAGA_H
 #define EAGA_H
