@@ -85,8 +85,38 @@ def dims(B, n, dx, de, dy, H, dh, dtype) -> Dims:
     return Dims(B, n, dx, de, dy, H, dh, dtype)
 
 
-def _p(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+def _p(t, name="tensor", dtype=None):
+    """Data pointer of a tensor handed to the library: a contiguous CUDA tensor
+    on the current device (and of `dtype`, when given); None passes NULL.  A
+    host tensor or one on another GPU would reach the kernels as a bad device
+    pointer, so it is refused here."""
+    if t is None:
+        return None
+    import torch
+    if not t.is_cuda:
+        raise ValueError(f"{name}: a CUDA tensor is required (got {t.device})")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name}: on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _storage(d: Dims):
+    import torch
+    return torch.bfloat16 if d.dtype == EAGA_BF16 else torch.float32
+
+
+def _u8():
+    import torch
+    return torch.uint8
+
+
+def _f32():
+    import torch
+    return torch.float32
 
 
 def _stream(stream):
@@ -96,8 +126,8 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
-def _weights(W: dict) -> Weights:
-    return Weights(*(W[k].data_ptr() for k in WEIGHT_NAMES))
+def _weights(W: dict, dtype=None, what="W") -> Weights:
+    return Weights(*(_p(W[k], f"{what}[{k}]", dtype).value for k in WEIGHT_NAMES))
 
 
 def _check(rc: int, where: str):
@@ -113,41 +143,54 @@ def saved_size(d: Dims) -> int:
     return int(lib().eaga_saved_size(ctypes.byref(d)))
 
 
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def forward(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, workspace, stream=None):
-    rc = lib().eaga_forward(ctypes.byref(d), _p(X), _p(E), _p(y), _p(M), ctypes.byref(_weights(W)),
-                            _p(Xout), _p(Eout), _p(saved), _p(workspace), workspace.numel() * workspace.element_size(),
-                            _stream(stream))
+    sd = _storage(d)
+    rc = lib().eaga_forward(ctypes.byref(d), _p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd), _p(M, "M", _u8()),
+                            ctypes.byref(_weights(W, sd)), _p(Xout, "Xout", sd), _p(Eout, "Eout", sd),
+                            _p(saved, "saved"), _p(workspace, "workspace"), _nbytes(workspace), _stream(stream))
     _check(rc, "eaga_forward")
 
 
 def forward_noalloc(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, stream=None):
     """eaga_forward without a workspace argument (the library's own fixed scratch is used)."""
-    rc = lib().eaga_forward_noalloc(ctypes.byref(d), _p(X), _p(E), _p(y), _p(M), ctypes.byref(_weights(W)),
-                                    _p(Xout), _p(Eout), _p(saved), _stream(stream))
+    sd = _storage(d)
+    rc = lib().eaga_forward_noalloc(ctypes.byref(d), _p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd),
+                                    _p(M, "M", _u8()), ctypes.byref(_weights(W, sd)), _p(Xout, "Xout", sd),
+                                    _p(Eout, "Eout", sd), _p(saved, "saved"), _stream(stream))
     _check(rc, "eaga_forward_noalloc")
 
 
 def backward(d: Dims, X, E, y, M, W: dict, saved, dXout, dEout, dX, dE, dy, dW: dict, workspace, stream=None):
-    rc = lib().eaga_backward(ctypes.byref(d), _p(X), _p(E), _p(y), _p(M), ctypes.byref(_weights(W)), _p(saved),
-                             _p(dXout), _p(dEout), _p(dX), _p(dE), _p(dy), ctypes.byref(_weights(dW)),
-                             _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    sd = _storage(d)
+    rc = lib().eaga_backward(ctypes.byref(d), _p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd), _p(M, "M", _u8()),
+                             ctypes.byref(_weights(W, sd)), _p(saved, "saved"), _p(dXout, "dXout", sd),
+                             _p(dEout, "dEout", sd), _p(dX, "dX", sd), _p(dE, "dE", sd), _p(dy, "dy", sd),
+                             ctypes.byref(_weights(dW, _f32(), "dW")), _p(workspace, "workspace"),
+                             _nbytes(workspace), _stream(stream))
     _check(rc, "eaga_backward")
 
 
 def debug_attention_map(d: Dims, E, M, W: dict, y, saved, A, stream=None):
-    rc = lib().eaga_debug_attention_map(ctypes.byref(d), _p(E), _p(M), ctypes.byref(_weights(W)), _p(y), _p(saved),
-                                        _p(A), _stream(stream))
+    sd = _storage(d)
+    rc = lib().eaga_debug_attention_map(ctypes.byref(d), _p(E, "E", sd), _p(M, "M", _u8()),
+                                        ctypes.byref(_weights(W, sd)), _p(y, "y", sd), _p(saved, "saved"),
+                                        _p(A, "A", _f32()), _stream(stream))
     _check(rc, "eaga_debug_attention_map")
 
 
 def get_device_status(workspace, stream=None) -> int:
-    return int(lib().eaga_get_device_status(_p(workspace), _stream(stream)))
+    return int(lib().eaga_get_device_status(_p(workspace, "workspace"), _stream(stream)))
 
 
 def debug_wait_probe(workspace, limit: int, stream=None):
     """Run the bounded-wait failure path once (test aid): a wait that never
     completes gives up after `limit` polls and records a timeout."""
-    _check(lib().eaga_debug_wait_probe(_p(workspace), int(limit), _stream(stream)), "eaga_debug_wait_probe")
+    _check(lib().eaga_debug_wait_probe(_p(workspace, "workspace"), int(limit), _stream(stream)),
+           "eaga_debug_wait_probe")
 
 
 def set_profile_events(point: int, before=None, after=None):

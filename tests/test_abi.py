@@ -104,3 +104,20 @@ def test_wait_probe_arguments(L):
     assert L.eaga_debug_wait_probe(fake, 0, None) == 1
     assert L.eaga_debug_wait_probe(fake, (1 << 24) + 1, None) == 1
     assert L.eaga_debug_wait_probe(ctypes.c_void_p(0x100008), 100, None) == 3   # misaligned
+
+
+def test_binding_refuses_host_tensors(L):
+    # the binding checks every tensor before a pointer reaches the library: a
+    # host tensor would otherwise be read as device memory
+    import torch
+    d = eaga.dims(2, 12, 16, 8, 8, 2, 8, "fp32")
+    t = lambda *s: torch.zeros(*s, dtype=torch.float32)
+    W = {k: t(4) for k in eaga.WEIGHT_NAMES}
+    M = torch.zeros(2, 12, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        eaga.forward(d, t(2, 12, 16), t(2, 12, 12, 8), t(2, 8), M, W, t(2, 12, 16), t(2, 12, 12, 8),
+                     None, torch.zeros(64, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        eaga.get_device_status(torch.zeros(16, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        eaga.debug_wait_probe(torch.zeros(16, dtype=torch.uint8), 100)
