@@ -97,7 +97,8 @@ def test_v_concat_identity_formulation(oracle_lib):
     s = np.einsum("bhid,bhjd->bhij", Q, K) / math.sqrt(p.dh)
     sp = s * (1 + gam) + bet
     valid = valid_mask(d["M"])[:, None]
-    P = scipy.special.softmax(np.where(valid, sp, -np.inf), axis=-1)
+    with np.errstate(invalid="ignore"):      # a fully masked row gives NaN, zeroed below
+        P = scipy.special.softmax(np.where(valid, sp, -np.inf), axis=-1)
     P = np.where(valid, np.nan_to_num(P), 0.0)
     VI = np.concatenate([V, np.broadcast_to(np.eye(p.n), (p.B, p.H, p.n, p.n))], axis=-1)
     res = P @ VI
