@@ -84,6 +84,44 @@ def test_zero_film_is_masked_sdpa(oracle_lib):
     np.testing.assert_allclose(out["Xout"], Xref, rtol=0, atol=1e-12)
 
 
+def test_light_edge_is_sdpa_with_a_global_temperature(oracle_lib):
+    """Light Edge (no per-edge modulation) is the layer with Wfe = 0: gamma and
+    beta are then constant per graph and head, beta cancels in the softmax, and
+    the map is scaled dot-product attention at scale (1 + gamma_bh) / sqrt(dh)."""
+    p, dims, d, W = tiny(seed=7)
+    W = dict(W)
+    W["Wfe"] = np.zeros_like(W["Wfe"])
+    out = oracle_lib.forward(dims, d["X"], d["E"], d["y"], d["M"], W, want_attention=True)
+    g = d["y"].astype(np.float64) @ W["Wfy"].astype(np.float64) + W["bf"]       # [B, 2H]
+    assert np.abs(g[:, p.H:]).max() > 0.1 and np.abs(g[:, :p.H]).max() > 0.1   # beta and gamma both present
+    Q, K, V = qkv(p, d["X"], W)
+    valid = torch.from_numpy(valid_mask(d["M"]))                                # [B,n,n]
+    rows = d["M"].astype(bool)
+    mask = valid | torch.from_numpy(~rows)[:, :, None]      # dummy keys for masked rows, as above
+    O = np.zeros((p.B, p.n, p.H, p.dh))
+    for b in range(p.B):
+        for h in range(p.H):
+            q, k, v = (torch.from_numpy(np.ascontiguousarray(t[b, h])) for t in (Q, K, V))
+            O[b, :, h] = torch.nn.functional.scaled_dot_product_attention(
+                q, k, v, attn_mask=mask[b], scale=(1.0 + g[b, h]) / math.sqrt(p.dh)).numpy()
+    O = O.reshape(p.B, p.n, p.H * p.dh)
+    np.testing.assert_allclose(out["O"][rows], O[rows], rtol=0, atol=1e-11)
+    # the map no longer depends on E: a different E changes only the residual
+    d2 = dict(d)
+    d2["E"] = d["E"] + np.float32(3.0)
+    out2 = oracle_lib.forward(dims, d2["X"], d2["E"], d2["y"], d2["M"], W, want_attention=True)
+    np.testing.assert_array_equal(out2["A"], out["A"])
+    dE_in = d2["E"].astype(np.float64) - d["E"].astype(np.float64)
+    np.testing.assert_allclose(out2["Eout"] - out["Eout"], dE_in, rtol=0, atol=1e-12)
+    # a key bias adds q_i . bk to every score of row i, times the same (1 + gamma):
+    # the softmax cancels it, so its gradient vanishes (it does not with Wfe != 0)
+    g = oracle_lib.backward(dims, d["X"], d["E"], d["y"], d["M"], W, d["dXout"], d["dEout"])
+    assert np.abs(g["dbk"]).max() <= 1e-12 * np.abs(g["dbq"]).max()
+    p3, dims3, d3, W3 = tiny(seed=7)
+    g3 = oracle_lib.backward(dims3, d3["X"], d3["E"], d3["y"], d3["M"], W3, d3["dXout"], d3["dEout"])
+    assert np.abs(g3["dbk"]).max() > 1e-3 * np.abs(g3["dbq"]).max()
+
+
 def test_v_concat_identity_formulation(oracle_lib):
     """The pages' trick: attention applied to [V | I] returns O and the map."""
     p, dims, d, W = tiny()

@@ -103,6 +103,27 @@ def test_ragged_shapes(oracle_lib, case):
     check_backward(buf, oracle_backward(oracle_lib, p, d, W), TOL[dtype])
 
 
+def test_light_edge_variant(oracle_lib):
+    """Light Edge (no per-edge modulation) is the layer with Wfe = 0; the
+    specialised path computes it like any other weights.  With (1 + gamma)
+    constant over j, a key bias shifts a whole score row, so its gradient dbk
+    is exactly zero: the GPU's value is checked against zero, to the parity
+    tolerance taken on the scale of the query-bias gradient."""
+    p, d, W = custom_case(3, 96, 256, 64, 64, 8, 32, "bf16", seed=21, mask="random")
+    W = dict(W)
+    W["Wfe"] = np.zeros_like(W["Wfe"])
+    buf = make(p, d, W, backward=True)
+    buf.forward()
+    buf.backward()
+    torch.cuda.synchronize()
+    check_forward(buf, oracle_forward(oracle_lib, p, d, W), TOL["bf16"])
+    ref = oracle_backward(oracle_lib, p, d, W)
+    check_backward(buf, ref, TOL["bf16"], loose={"dbk": float("inf")})
+    dbk = buf.dW["bk"].cpu().numpy().astype(np.float64)
+    assert np.abs(ref["dbk"]).max() <= 1e-12 * np.abs(ref["dbq"]).max()
+    assert np.abs(dbk).max() <= TOL["bf16"] * np.abs(ref["dbq"]).max()
+
+
 def test_masked_garbage_is_ignored():
     """Large finite values in masked node rows and invalid pairs leave every
     valid output bitwise unchanged; masked outputs equal their inputs."""
