@@ -29,7 +29,9 @@
  * torch's float64 scaled_dot_product_attention; the gamma = -1 closed form
  * (uniform attention); row sums; masked-entry invariance; permutation
  * equivariance; a brute-force per-pair Python evaluation without max
- * subtraction; the [V | I] formulation; beta-shift invariance; and fp64
+ * subtraction; the [V | I] formulation; beta-shift invariance; the Light
+ * Edge case (Wfe = 0) against scaled dot-product attention at a per-graph,
+ * per-head temperature, with its vanishing key-bias gradient; and fp64
  * central finite differences of orc_forward for every gradient orc_backward
  * returns.
  */
