@@ -9,7 +9,7 @@ bool supports(const eaga_dims &d);
 // status word and g (start of the backward's own regions).
 size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, size_t common_head);
 int kernel_launches(const eaga_dims &d, int for_backward);
-// Bytes the forward uses after the common workspace (operand images, transposed node weights).
+// Bytes the forward uses after the common workspace (the FiLM and edge operand images).
 size_t forward_scratch_bytes(const eaga_dims &d);
 cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st);
 cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head, cudaStream_t st);

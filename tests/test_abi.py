@@ -121,3 +121,29 @@ def test_binding_refuses_host_tensors(L):
         eaga.get_device_status(torch.zeros(16, dtype=torch.uint8))
     with pytest.raises(ValueError, match="CUDA tensor"):
         eaga.debug_wait_probe(torch.zeros(16, dtype=torch.uint8), 100)
+
+
+@pytest.mark.parametrize("dims,fast", [
+    ((32, 192, 256, 64, 64, 8, 32, "bf16"), True),      # the SBM-shaped workload
+    ((64, 64, 256, 64, 64, 8, 32, "bf16"), True),       # Planar / Tree shaped
+    ((4, 1024, 256, 64, 64, 8, 32, "bf16"), True),      # Large shaped
+    ((2, 2, 64, 64, 8, 8, 32, "bf16"), True),           # smallest n, narrowest dx
+    ((2, 96, 576, 64, 64, 8, 32, "bf16"), True),        # dx a multiple of 64 only
+    ((32, 192, 256, 64, 64, 8, 32, "fp32"), False),     # fp32 storage
+    ((2, 191, 256, 64, 64, 8, 32, "bf16"), False),      # odd n
+    ((2, 96, 72, 64, 64, 8, 32, "bf16"), False),        # dx not a multiple of 64
+    ((2, 96, 256, 32, 64, 8, 32, "bf16"), False),       # de != 64
+    ((2, 96, 256, 64, 64, 4, 32, "bf16"), False),       # H != 8
+    ((2, 96, 256, 64, 64, 8, 16, "bf16"), False),       # dh != 32
+])
+def test_dispatch_rule(L, dims, fast):
+    # the tcgen05 path (4 forward, 11 backward launches) takes bf16, de = 64,
+    # H = 8, dh = 32, n even, dx a multiple of 64; every other supported shape
+    # runs the CUDA-core kernels (4 and 10)
+    d = eaga.dims(*dims)
+    assert (eaga.kernel_launches(d, False), eaga.kernel_launches(d, True)) == ((4, 11) if fast else (4, 10))
+
+
+def test_dispatch_rejects_unsupported(L):
+    assert eaga.kernel_launches(eaga.dims(2, 1025, 256, 64, 64, 8, 32, "bf16"), False) == -1
+    assert eaga.kernel_launches(eaga.dims(0, 64, 256, 64, 64, 8, 32, "bf16"), False) == -1
