@@ -99,6 +99,48 @@ inline cudaError_t ensure_smem_attr(K kernel, int bytes, std::atomic<uint32_t> &
     return e;
 }
 
+// Byte extents of the layer's tensors for dims d: inputs in the storage
+// dtype, weight gradients in fp32 (order of the eaga_weights fields).
+struct Extents {
+    size_t X, E, y, M, w[12], wgrad[12];
+};
+inline Extents tensor_extents(const eaga_dims &d) {
+    const size_t s = d.dtype == EAGA_BF16 ? 2 : 4, hd = size_t(d.H) * d.dh, f = 2 * size_t(d.H);
+    const size_t dx = d.dx, de = d.de, dy = d.dy;
+    Extents x;
+    x.X = size_t(d.B) * d.n * dx * s;
+    x.E = size_t(d.B) * d.n * d.n * de * s;
+    x.y = size_t(d.B) * dy * s;
+    x.M = size_t(d.B) * d.n;
+    const size_t count[12] = {dx * hd, hd, dx * hd, hd, dx * hd, hd, de * f, dy * f, f, size_t(d.H) * de, hd * dx, dx};
+    for (int t = 0; t < 12; ++t) {
+        x.w[t] = count[t] * s;
+        x.wgrad[t] = count[t] * 4;
+    }
+    return x;
+}
+
+// A byte range [p, p + n) of device memory; n = 0 for an absent buffer.
+struct Span {
+    const void *p;
+    size_t n;
+};
+inline bool spans_overlap(const Span &a, const Span &b) {
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a.p), pb = reinterpret_cast<uintptr_t>(b.p);
+    return a.n && b.n && pa < pb + b.n && pb < pa + a.n;
+}
+// EAGA_ERR_INVALID_ARG when an output range overlaps an input range or
+// another output range (inputs may share memory: they are only read).
+inline eaga_status check_no_alias(const Span *outs, int n_out, const Span *ins, int n_in) {
+    for (int o = 0; o < n_out; ++o) {
+        for (int i = 0; i < n_in; ++i)
+            if (spans_overlap(outs[o], ins[i])) return EAGA_ERR_INVALID_ARG;
+        for (int o2 = o + 1; o2 < n_out; ++o2)
+            if (spans_overlap(outs[o], outs[o2])) return EAGA_ERR_INVALID_ARG;
+    }
+    return EAGA_OK;
+}
+
 // Device status word values (first int of the workspace).
 enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
 

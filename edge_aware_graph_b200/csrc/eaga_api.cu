@@ -49,6 +49,13 @@ void weight_array(const eaga_weights *w, const void *out[12]) {
     memcpy(out, src, sizeof(src));
 }
 
+// Appends the ranges of twelve weight (or weight-gradient) buffers, with
+// extents `ext`, to `spans` at `k`.
+int weight_spans(const void *const src[12], const size_t ext[12], Span *spans, int k) {
+    for (int t = 0; t < 12; ++t) spans[k++] = {src[t], ext[t]};
+    return k;
+}
+
 eaga_status launch_status(cudaError_t e) { return e == cudaSuccess ? EAGA_OK : EAGA_ERR_CUDA; }
 
 }  // namespace
@@ -82,10 +89,20 @@ eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const
     if ((s = check_weights(w)) != EAGA_OK) return s;
     if ((s = check_ptrs({X, E, y, M, Xout, Eout, workspace})) != EAGA_OK) return s;
     if (saved && !aligned16(saved)) return EAGA_ERR_MISALIGNED;
+    const Layout L = saved_layout(*d);
+    {
+        const Extents x = tensor_extents(*d);
+        const Span outs[4] = {{Xout, x.X}, {Eout, x.E}, {saved, saved ? L.saved_total : 0},
+                              {workspace, eaga_workspace_size(d, 0)}};
+        Span ins[16] = {{X, x.X}, {E, x.E}, {y, x.y}, {M, x.M}};
+        const void *wsrc[12];
+        weight_array(w, wsrc);
+        weight_spans(wsrc, x.w, ins, 4);
+        if ((s = check_no_alias(outs, 4, ins, 16)) != EAGA_OK) return s;
+    }
     if (ws_bytes < eaga_workspace_size(d, 0)) return EAGA_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const WsLayout W = ws_layout(*d);
-    const Layout L = saved_layout(*d);
     char *ws = static_cast<char *>(workspace);
     char *sv = saved ? static_cast<char *>(saved) : ws + W.fwd_saved;
     FwdArgs a;
@@ -116,10 +133,22 @@ eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, cons
     if ((s = check_ptrs({dW->Wq, dW->bq, dW->Wk, dW->bk, dW->Wv, dW->bv, dW->Wfe, dW->Wfy, dW->bf, dW->We, dW->Wo,
                          dW->bo})) != EAGA_OK)
         return s;
+    const Layout L = saved_layout(*d);
+    {
+        const Extents x = tensor_extents(*d);
+        Span outs[16] = {{dX, x.X}, {dE, x.E}, {dy, x.y}, {workspace, eaga_workspace_size(d, 1)}};
+        const void *gsrc[12] = {dW->Wq, dW->bq, dW->Wk, dW->bk, dW->Wv, dW->bv,
+                                dW->Wfe, dW->Wfy, dW->bf, dW->We, dW->Wo, dW->bo};
+        weight_spans(gsrc, x.wgrad, outs, 4);
+        Span ins[19] = {{X, x.X}, {E, x.E}, {y, x.y}, {M, x.M}, {saved, L.saved_total}, {dXout, x.X}, {dEout, x.E}};
+        const void *wsrc[12];
+        weight_array(w, wsrc);
+        weight_spans(wsrc, x.w, ins, 7);
+        if ((s = check_no_alias(outs, 16, ins, 19)) != EAGA_OK) return s;
+    }
     if (ws_bytes < eaga_workspace_size(d, 1)) return EAGA_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const WsLayout W = ws_layout(*d);
-    const Layout L = saved_layout(*d);
     char *ws = static_cast<char *>(workspace);
     const char *sv = static_cast<const char *>(saved);
     BwdArgs a;
@@ -156,6 +185,15 @@ eaga_status eaga_debug_attention_map(const eaga_dims *d, const void *E, const ui
     if ((s = check_ptrs({E, M, y, saved, A})) != EAGA_OK) return s;
     // g [B,2H] lives just past the A map the caller provides room for.
     const Layout L = saved_layout(*d);
+    {
+        const Extents x = tensor_extents(*d);
+        const Span outs[1] = {{A, ((size_t)d->B * d->H * d->n * d->n + 2 * (size_t)d->B * d->H) * sizeof(float)}};
+        Span ins[16] = {{E, x.E}, {M, x.M}, {y, x.y}, {saved, L.saved_total}};
+        const void *wsrc[12];
+        weight_array(w, wsrc);
+        weight_spans(wsrc, x.w, ins, 4);
+        if ((s = check_no_alias(outs, 1, ins, 16)) != EAGA_OK) return s;
+    }
     const char *sv = static_cast<const char *>(saved);
     MapArgs a;
     a.E = E; a.y = y; a.Wfe = w->Wfe; a.Wfy = w->Wfy; a.bf = w->bf; a.M = M;

@@ -72,6 +72,15 @@ eaga_status eaga_forward_noalloc(const eaga_dims *d, const void *X, const void *
     const size_t images = fast::supports(*d) ? fast::forward_scratch_bytes(*d) : 0;
     const size_t needed = NOALLOC_G + g_bytes + images;
     if (needed > NOALLOC_SCRATCH_BYTES) return EAGA_ERR_UNSUPPORTED;   // too large for the fixed array
+    {
+        const Extents x = tensor_extents(*d);
+        const Span outs[3] = {{Xout, x.X}, {Eout, x.E}, {saved, saved_layout(*d).saved_total}};
+        Span ins[16] = {{X, x.X}, {E, x.E}, {y, x.y}, {M, x.M}};
+        const void *wsrc[12] = {w->Wq, w->bq, w->Wk, w->bk, w->Wv, w->bv, w->Wfe, w->Wfy, w->bf, w->We, w->Wo, w->bo};
+        for (int t = 0; t < 12; ++t) ins[4 + t] = {wsrc[t], x.w[t]};
+        const eaga_status s = check_no_alias(outs, 3, ins, 16);
+        if (s != EAGA_OK) return s;
+    }
 
     void *base = nullptr;
     eaga_status s = scratch_address(&base);

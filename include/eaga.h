@@ -32,7 +32,11 @@
  *     Wfe [de, 2H]; Wfy [dy, 2H]; bf [2H] (first H columns gamma, next H
  *     beta); We [H, de] (no bias); Wo [H*dh, dx]; bo [dx].
  *   - Shapes: X, X', dX, dX' [B,n,dx]; E, E', dE, dE' [B,n,n,de]; y, dy [B,dy].
- *   - Every pointer must be 16-byte aligned; outputs must not alias inputs.
+ *   - Every pointer must be 16-byte aligned (else EAGA_ERR_MISALIGNED).
+ *     Outputs (including `saved` in the forward and the workspace) must not
+ *     overlap an input or another output: the byte range of every buffer
+ *     follows from the dims, and an overlap returns EAGA_ERR_INVALID_ARG
+ *     before anything is launched.  Inputs may share memory.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  The return value reports host-side validation and
  *     launch errors only; device-side conditions (a bounded wait that ran out)

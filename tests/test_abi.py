@@ -5,7 +5,9 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
+import torch
 
 from edge_aware_graph_b200 import build as B
 from edge_aware_graph_b200 import eaga
@@ -83,12 +85,15 @@ def test_null_and_misaligned_and_workspace(L):
              None) == 3
     w_bad = eaga.Weights(*([0x100000] * 11 + [0x100004]))
     assert f(ctypes.byref(d), ok, ok, ok, ok, ctypes.byref(w_bad), ok, ok, None, ok, big, None) == 3
-    assert f(ctypes.byref(d), ok, ok, ok, ok, ctypes.byref(w), ok, ok, None, ok, big - 1, None) == 4
     g = L.eaga_backward
     bigb = eaga.workspace_size(d, True)
     assert g(ctypes.byref(d), ok, ok, ok, ok, ctypes.byref(w), ok, ok, ok, ok, ok, ok, None, ok, bigb, None) == 1
-    assert g(ctypes.byref(d), ok, ok, ok, ok, ctypes.byref(w), ok, ok, ok, ok, ok, ok, ctypes.byref(w), ok,
-             bigb - 1, None) == 4
+    # a workspace one byte short (distinct, non-overlapping fake buffers: the
+    # size check comes after the overlap check; both return before any launch)
+    fw = forward_layout(d, far=True)
+    assert f(ctypes.byref(d), *fw.args(ws_bytes=big - 1)) == 4
+    bw = backward_layout(d, far=True)
+    assert g(ctypes.byref(d), *bw.args(ws_bytes=bigb - 1)) == 4
 
 
 def test_strerror(L):
@@ -147,3 +152,155 @@ def test_dispatch_rule(L, dims, fast):
 def test_dispatch_rejects_unsupported(L):
     assert eaga.kernel_launches(eaga.dims(2, 1025, 256, 64, 64, 8, 32, "bf16"), False) == -1
     assert eaga.kernel_launches(eaga.dims(0, 64, 256, 64, 64, 8, 32, "bf16"), False) == -1
+
+# ------------------------------------------------------------ buffer layouts
+
+WSHAPES = lambda d: {"Wq": (d.dx, d.H * d.dh), "bq": (d.H * d.dh,), "Wk": (d.dx, d.H * d.dh),
+                     "bk": (d.H * d.dh,), "Wv": (d.dx, d.H * d.dh), "bv": (d.H * d.dh,),
+                     "Wfe": (d.de, 2 * d.H), "Wfy": (d.dy, 2 * d.H), "bf": (2 * d.H,), "We": (d.H, d.de),
+                     "Wo": (d.H * d.dh, d.dx), "bo": (d.dx,)}
+
+
+def tensor_bytes(d):
+    """Bytes of each buffer as a caller allocates it (the shapes of the C ABI)."""
+    s = 2 if d.dtype == eaga.EAGA_BF16 else 4
+    out = {"X": d.B * d.n * d.dx * s, "E": d.B * d.n * d.n * d.de * s, "y": d.B * d.dy * s, "M": d.B * d.n}
+    for k, sh in WSHAPES(d).items():
+        out["W" + k] = int(np.prod(sh)) * s
+        out["G" + k] = int(np.prod(sh)) * 4
+    return out
+
+
+class Layout:
+    """Named fake device pointers: either tightly packed (each buffer starts at
+    the next 16-byte boundary after the previous one, so that any range the
+    library over-estimates runs into its neighbour) or spread 1 GiB apart.
+    Nothing is ever dereferenced on the host."""
+
+    def __init__(self, sizes: dict, far=False):
+        self.ptr, off = {}, 0x100000000
+        for k, n in sizes.items():
+            self.ptr[k] = off
+            off = off + (1 << 30) if far else (off + n + 15) // 16 * 16
+        self.sizes = sizes
+
+    def p(self, k):
+        return ctypes.c_void_p(self.ptr[k])
+
+    def weights(self, prefix):
+        return eaga.Weights(*(self.ptr[prefix + k] for k in eaga.WEIGHT_NAMES))
+
+
+class FwdLayout(Layout):
+    def args(self, ws_bytes=None, **over):
+        q = lambda k: ctypes.c_void_p(over[k]) if k in over else self.p(k)
+        self._w = self.weights("W")
+        return (q("X"), q("E"), q("y"), q("M"), ctypes.byref(self._w), q("Xout"), q("Eout"), q("saved"),
+                q("ws"), self.sizes["ws"] if ws_bytes is None else ws_bytes, None)
+
+
+class BwdLayout(Layout):
+    def args(self, ws_bytes=None, **over):
+        q = lambda k: ctypes.c_void_p(over[k]) if k in over else self.p(k)
+        self._w = self.weights("W")
+        gp = {k: over.get("G" + k, self.ptr["G" + k]) for k in eaga.WEIGHT_NAMES}
+        self._g = eaga.Weights(*(gp[k] for k in eaga.WEIGHT_NAMES))
+        return (q("X"), q("E"), q("y"), q("M"), ctypes.byref(self._w), q("saved"), q("dXout"), q("dEout"),
+                q("dX"), q("dE"), q("dy"), ctypes.byref(self._g), q("ws"),
+                self.sizes["ws"] if ws_bytes is None else ws_bytes, None)
+
+
+def forward_layout(d, far=False):
+    t = tensor_bytes(d)
+    sizes = {"X": t["X"], "E": t["E"], "y": t["y"], "M": t["M"]}
+    sizes.update({"W" + k: t["W" + k] for k in eaga.WEIGHT_NAMES})
+    sizes.update({"Xout": t["X"], "Eout": t["E"], "saved": eaga.saved_size(d), "ws": eaga.workspace_size(d, False)})
+    return FwdLayout(sizes, far)
+
+
+def backward_layout(d, far=False):
+    t = tensor_bytes(d)
+    sizes = {"X": t["X"], "E": t["E"], "y": t["y"], "M": t["M"]}
+    sizes.update({"W" + k: t["W" + k] for k in eaga.WEIGHT_NAMES})
+    sizes.update({"saved": eaga.saved_size(d), "dXout": t["X"], "dEout": t["E"], "dX": t["X"], "dE": t["E"],
+                  "dy": t["y"]})
+    sizes.update({"G" + k: t["G" + k] for k in eaga.WEIGHT_NAMES})
+    sizes["ws"] = eaga.workspace_size(d, True)
+    return BwdLayout(sizes, far)
+
+
+ALIAS_DIMS = [eaga.dims(2, 64, 256, 64, 64, 8, 32, "bf16"),      # the tcgen05 path
+              eaga.dims(3, 37, 24, 24, 16, 3, 16, "fp32")]       # the CUDA-core path
+no_cuda = pytest.mark.skipif(torch.cuda.is_available(),
+                             reason="a clean call goes on to its first CUDA call, with fake pointers")
+
+
+@no_cuda
+@pytest.mark.parametrize("d", ALIAS_DIMS, ids=["bf16-fast", "fp32-generic"])
+def test_overlap_check_forward(L, d):
+    f = lambda **kw: L.eaga_forward(ctypes.byref(d), *lay.args(**kw))
+    lay = forward_layout(d)
+    # tightly packed, nothing shared: the check passes, and the first CUDA
+    # call fails on this host without a GPU (EAGA_ERR_CUDA)
+    assert f() == 5
+    assert f(Eout=lay.ptr["E"]) == 1                                    # E' in place over E
+    assert f(Xout=lay.ptr["X"] + lay.sizes["X"] - 16) == 1              # last 16 bytes of X
+    assert f(saved=lay.ptr["ws"]) == 1                                  # two outputs
+    assert f(ws=lay.ptr["WWo"]) == 1                                    # workspace over a weight
+    assert f(E=lay.ptr["X"], y=lay.ptr["X"]) == 5                       # inputs may share memory
+
+
+@no_cuda
+@pytest.mark.parametrize("d", ALIAS_DIMS, ids=["bf16-fast", "fp32-generic"])
+def test_overlap_check_backward(L, d):
+    g = lambda **kw: L.eaga_backward(ctypes.byref(d), *lay.args(**kw))
+    lay = backward_layout(d)
+    assert g() == 5
+    assert g(dE=lay.ptr["dEout"]) == 1                                  # dE in place over dE'
+    assert g(dX=lay.ptr["saved"] + 16) == 1                             # inside the saved state
+    assert g(Gbo=lay.ptr["dy"]) == 1                                    # two outputs
+    assert g(ws=lay.ptr["E"] + lay.sizes["E"] - 16) == 1                # workspace over E's tail
+
+
+@no_cuda
+def test_overlap_check_attention_map_and_noalloc(L):
+    d = ALIAS_DIMS[0]
+    t = tensor_bytes(d)
+    sizes = {"E": t["E"], "M": t["M"], "y": t["y"], "saved": eaga.saved_size(d)}
+    sizes.update({"W" + k: t["W" + k] for k in eaga.WEIGHT_NAMES})
+    sizes["A"] = (d.B * d.H * d.n * d.n + 2 * d.B * d.H) * 4
+    lay = Layout(sizes)
+    w = lay.weights("W")
+    m = lambda A: L.eaga_debug_attention_map(ctypes.byref(d), lay.p("E"), lay.p("M"), ctypes.byref(w), lay.p("y"),
+                                             lay.p("saved"), ctypes.c_void_p(A), None)
+    assert m(lay.ptr["A"]) == 5
+    assert m(lay.ptr["saved"]) == 1
+    fw = forward_layout(d)
+    n = lambda **kw: L.eaga_forward_noalloc(ctypes.byref(d), *(fw.args(**kw)[:8]), None)
+    assert n(Eout=fw.ptr["E"]) == 1
+    assert n(saved=fw.ptr["Xout"]) == 1
+
+
+def _before(sizes: dict, k: str, o: str) -> dict:
+    """The same buffers with k placed directly before o, at the end."""
+    out = {key: v for key, v in sizes.items() if key not in (k, o)}
+    out[k] = sizes[k]
+    out[o] = sizes[o]
+    return out
+
+
+@no_cuda
+@pytest.mark.parametrize("d", ALIAS_DIMS, ids=["bf16-fast", "fp32-generic"])
+def test_overlap_check_extents_never_exceed_the_buffers(L, d):
+    # every buffer, followed directly by an output: a range the library
+    # over-estimates by a 16-byte step would reach that output and be refused
+    fw = forward_layout(d)
+    for k in fw.sizes:
+        o = "ws" if k != "ws" else "Xout"
+        lay = FwdLayout(_before(fw.sizes, k, o))
+        assert L.eaga_forward(ctypes.byref(d), *lay.args()) == 5, k
+    bw = backward_layout(d)
+    for k in bw.sizes:
+        o = "ws" if k != "ws" else "dX"
+        lay = BwdLayout(_before(bw.sizes, k, o))
+        assert L.eaga_backward(ctypes.byref(d), *lay.args()) == 5, k
