@@ -102,3 +102,24 @@ def test_two_rank_weight_grads_match_whole_batch():
     whole = np.concatenate([np.asarray(g["d" + k], np.float64).ravel() for k in GRAD_KEYS])
     for _, flat in out:
         np.testing.assert_allclose(flat, whole, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("workload", ["sbm-train", "planar-sample"])
+def test_reference_arm_under_torchrun(workload):
+    """bench.py --impl reference launched as the multi-GPU runs are: rank 0
+    alone runs the oracle arm and prints one JSON line; the other rank exits 0."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(WORLD),
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",
+           "--gpus", str(WORLD), "--steps", "1", "--warmup", "3", "--ref-graphs", "1", "--workload", workload]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=600,
+                       env=dict(os.environ, OMP_NUM_THREADS="2"))
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["n_gpus"] == WORLD and out["value"] > 0
+    assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["cpu_baseline"]["kind"] == "oracle"
