@@ -165,6 +165,38 @@ def test_gamma_minus_one_is_uniform(oracle_lib):
         np.testing.assert_array_equal(out["Eout"][b, :, nr:], d["E"][b, :, nr:])
 
 
+def test_gamma_minus_one_backward_closed_forms(oracle_lib):
+    """gamma = -1, beta = 0: every score is zero and a is uniform over real
+    nodes.  Then ds = dS' (1 + gamma) vanishes, so Q and K receive no
+    gradient; dV_j is the mean of M dX' Wo^T over the real rows; dWe[h] is the
+    per-graph mean of the sum of dE' over valid pairs, the same for every
+    head; and dE = dE'."""
+    p, dims, d, W = tiny()
+    W = zero_film(W, p.H, gamma=-1.0, beta=0.0)
+    g = oracle_lib.backward(dims, d["X"], d["E"], d["y"], d["M"], W, d["dXout"], d["dEout"])
+    for k in ("dWq", "dbq", "dWk", "dbk"):
+        assert np.abs(g[k]).max() <= 1e-13, k
+    np.testing.assert_array_equal(g["dE"], d["dEout"].astype(np.float64))
+    X, dXo = d["X"].astype(np.float64), d["dXout"].astype(np.float64)
+    Wo, Wv = W["Wo"].astype(np.float64), W["Wv"].astype(np.float64)
+    dWv = np.zeros_like(Wv)
+    dbv = np.zeros(Wv.shape[1])
+    dWe = np.zeros((p.H, p.de))
+    dX = dXo.copy()
+    for b in range(p.B):
+        nr = int(d["n_real"][b])
+        dO = dXo[b, :nr] @ Wo.T                               # [nr, H*dh], masked rows contribute nothing
+        dv = dO.mean(0)                                       # the same for every real j
+        dWv += np.outer(X[b, :nr].sum(0), dv)
+        dbv += nr * dv
+        dWe += d["dEout"][b, :nr, :nr].astype(np.float64).sum((0, 1))[None, :] / nr
+        dX[b, :nr] += (dv @ Wv.T)[None, :]
+    np.testing.assert_allclose(g["dWv"], dWv, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(g["dbv"], dbv, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(g["dWe"], dWe, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(g["dX"], dX, rtol=0, atol=1e-11)
+
+
 # --------------------------------------------------------------- invariants
 
 
