@@ -1,0 +1,92 @@
+"""Planted mistakes in the oracle: each edit below makes one plausible error
+in oracle/eaga_oracle.c (a dropped term, a wrong sign, index, column or
+operand), and the oracle's pins (test_oracle_pins.py) must catch every one.
+
+Each mutant is compiled from a copy of the oracle in a temporary directory,
+and the pin suite runs against that copy in a subprocess.  The unmodified
+copy must pass.  Nothing here touches the repository's own oracle build.
+"""
+import concurrent.futures as cf
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# name: (text in eaga_oracle.c, replacement)
+MUTANTS = {
+    # forward
+    "drop_beta": ("sp[j] = s * (1.0 + gam) + bet;", "sp[j] = s * (1.0 + gam);"),
+    "gamma_without_one": ("sp[j] = s * (1.0 + gam) + bet;", "sp[j] = s * gam + bet;"),
+    "no_score_scale": ("return acc / sqrt((double)d->dh);", "return acc;"),
+    "film_wrong_column": ("acc += e[c] * Wfe[(long)c * 2 * d->H + k];",
+                          "acc += e[c] * Wfe[(long)c * 2 * d->H + (k + 1) % (2 * d->H)];"),
+    "edge_update_shifted_index": ("acc += arow[(long)h * n + j] * w->We[(long)h * de + c];",
+                                  "acc += arow[(long)h * n + (j + 1) % n] * w->We[(long)h * de + c];"),
+    "mask_rows_only": ("if (mb[j] && sp[j] > m) m = sp[j];", "if (sp[j] > m) m = sp[j];"),
+    # backward
+    "dS_sign": ("const double dsp = a * (dA[(long)h * n + j] - D);",
+                "const double dsp = a * (dA[(long)h * n + j] + D);"),
+    "dE_missing_film_term": ("acc += df[(long)j * F + k] * w->Wfe[(long)c * F + k];",
+                             "acc += 0 * df[(long)j * F + k];"),
+    "dq_without_film_factor": ("const double ds = dsp * (1.0 + gam);", "const double ds = dsp;"),
+    "dk_without_film_factor": ("const double ds = dsp * (1.0 + f[h]);", "const double ds = dsp;"),
+    "dv_transposed": ("dV[r * hd + h * dh + t] += a * dO[ri * hd + h * dh + t];",
+                      "dV[r * hd + h * dh + t] += a * dO[r * hd + h * dh + t];"),
+    "dWe_wrong_operand": ("pWe[(long)h * de + c] += arow[(long)h * n + j] * dEout[e0 + c];",
+                          "pWe[(long)h * de + c] += arow[(long)h * n + j] * E[e0 + c];"),
+}
+
+
+def _copy_tree(dst, oracle_src):
+    os.makedirs(os.path.join(dst, "oracle"))
+    shutil.copy(os.path.join(ROOT, "oracle", "__init__.py"), os.path.join(dst, "oracle"))
+    with open(os.path.join(dst, "oracle", "eaga_oracle.c"), "w") as f:
+        f.write(oracle_src)
+    os.makedirs(os.path.join(dst, "tests"))
+    for name in ("conftest.py", "test_oracle_pins.py"):
+        shutil.copy(os.path.join(ROOT, "tests", name), os.path.join(dst, "tests"))
+    os.makedirs(os.path.join(dst, "edge_aware_graph_b200"))
+    for name in ("__init__.py", "inputs.py"):
+        shutil.copy(os.path.join(ROOT, "edge_aware_graph_b200", name), os.path.join(dst, "edge_aware_graph_b200"))
+
+
+def _run_pins(dst):
+    env = dict(os.environ, PYTHONPATH=dst, OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "tests/test_oracle_pins.py"],
+                       cwd=dst, env=env, capture_output=True, text=True, timeout=900)
+    lines = r.stdout.strip().splitlines()
+    return r.returncode, (lines[-1] if lines else r.stderr[-500:])
+
+
+@pytest.fixture(scope="module")
+def results(tmp_path_factory):
+    src = open(os.path.join(ROOT, "oracle", "eaga_oracle.c")).read()
+    jobs = {"unmodified": src}
+    for name, (old, new) in MUTANTS.items():
+        assert src.count(old) == 1, f"{name}: the text to mutate is not in the oracle exactly once"
+        jobs[name] = src.replace(old, new)
+    base = tmp_path_factory.mktemp("oracle_mutants")
+    dirs = {}
+    for name, text in jobs.items():
+        dirs[name] = str(base / name)
+        _copy_tree(dirs[name], text)
+    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 2)) as ex:
+        futs = {name: ex.submit(_run_pins, d) for name, d in dirs.items()}
+        return {name: f.result() for name, f in futs.items()}
+
+
+def test_unmodified_copy_passes_the_pins(results):
+    rc, summary = results["unmodified"]
+    assert rc == 0, summary
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(results, name):
+    rc, summary = results[name]
+    # exit code 1: the suite ran and at least one pin failed (not a build or
+    # collection error, which would be 2 or more)
+    assert rc == 1 and "failed" in summary, summary
