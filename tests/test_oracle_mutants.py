@@ -16,7 +16,9 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-# name: (text in eaga_oracle.c, replacement)
+# name: (text in eaga_oracle.c, replacement).  Only edits that change some
+# output belong here: leaving dO of a masked row unzeroed, for instance, does
+# not (its row has a = 0, so that dO reaches nothing), and no pin could catch it.
 MUTANTS = {
     # forward
     "drop_beta": ("sp[j] = s * (1.0 + gam) + bet;", "sp[j] = s * (1.0 + gam);"),
@@ -38,6 +40,25 @@ MUTANTS = {
                       "dV[r * hd + h * dh + t] += a * dO[r * hd + h * dh + t];"),
     "dWe_wrong_operand": ("pWe[(long)h * de + c] += arow[(long)h * n + j] * dEout[e0 + c];",
                           "pWe[(long)h * de + c] += arow[(long)h * n + j] * E[e0 + c];"),
+    "lse_without_log": ("lse[h] = valid ? m + log(l) : -INFINITY;", "lse[h] = valid ? m + l : -INFINITY;"),
+    # node residual and output projection
+    "out_proj_not_masked": ("Xout[r * dx + o] = X[r * dx + o] + (mi != 0.0 ? acc : 0.0);",
+                            "Xout[r * dx + o] = X[r * dx + o] + acc;"),
+    "out_proj_no_residual": ("Xout[r * dx + o] = X[r * dx + o] + (mi != 0.0 ? acc : 0.0);",
+                             "Xout[r * dx + o] = (mi != 0.0 ? acc : 0.0);"),
+    "dWo_dbo_not_masked": ("if (!M[r]) continue;", "if (0) continue;"),
+    "dWo_wrong_operand": ("gr->Wo[(long)k * dx + o] += O[r * hd + k] * dXout[r * dx + o];",
+                          "gr->Wo[(long)k * dx + o] += V[r * hd + k] * dXout[r * dx + o];"),
+    # gradients of the FiLM maps and of y
+    "dWfe_wrong_operand": ("pWfe[(long)c * F + k] += E[e0 + c] * df[(long)j * F + k];",
+                           "pWfe[(long)c * F + k] += dEout[e0 + c] * df[(long)j * F + k];"),
+    "dWfy_shifted_column": ("gr->Wfy[(long)c * F + k] += y[(long)b * dyd + c] * dg[(long)b * F + k];",
+                            "gr->Wfy[(long)c * F + k] += y[(long)b * dyd + c] * dg[(long)b * F + (k + 1) % F];"),
+    "dbf_missing": ("gr->bf[k] += dg[(long)b * F + k];", "gr->bf[k] += 0.0 * dg[(long)b * F + k];"),
+    "dy_shifted_column": ("acc += dg[(long)b * F + k] * w->Wfy[(long)c * F + k];",
+                          "acc += dg[(long)b * F + k] * w->Wfy[(long)c * F + (k + 1) % F];"),
+    "dX_without_dK_term": ("for (int p = 0; p < 3; ++p)\n                for (int k = 0; k < hd; ++k) acc += dN[p]",
+                           "for (int p = 0; p < 3; p += 2)\n                for (int k = 0; k < hd; ++k) acc += dN[p]"),
 }
 
 
