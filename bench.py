@@ -4,6 +4,8 @@ Workload (one step): one forward and one backward of the layer over one
 batch of the SBM-shaped training preset (B=32 graphs, n=192 padded nodes,
 n_real ~ U[44,187], dx=256, de=64, dy=64, H=8, dh=32, bf16 storage, fp32
 accumulation), synthetic seeded inputs (edge_aware_graph_b200/inputs.py).
+`--workload large-train` runs the Large-shaped training step (B=4, n=1024)
+instead; `planar-sample` / `tree-sample` the sampling-time forward.
 Metric: edge pairs (B*n^2, padded) per second, and the fraction of the HBM
 roofline of the dominant kernel.
 
@@ -30,10 +32,17 @@ if ROOT not in sys.path:
 
 import numpy as np
 
-WORKLOAD = "sbm"
-# --workload: the training step (default), or the sampling-time forward on
-# Planar- / Tree-shaped batches (forward only, many calls per model)
-WORKLOADS = {"sbm-train": "sbm", "planar-sample": "planar", "tree-sample": "tree"}
+# --workload: the SBM-shaped training step (default), the Large-shaped
+# training step (B=4, n=1024), or the sampling-time forward on Planar- /
+# Tree-shaped batches (forward only, many calls per model)
+WORKLOADS = {"sbm-train": "sbm", "large-train": "large", "planar-sample": "planar", "tree-sample": "tree"}
+TRAINING = ("sbm-train", "large-train")
+DESCRIBE = {
+    "sbm": "sbm-shaped training step (fwd+bwd): B=32, n=192 padded, n_real~U[44,187], 2-5 blocks, "
+           "dx=256 de=64 dy=64 H=8 dh=32, bf16 storage / fp32 accumulation",
+    "large": "large-shaped training step (fwd+bwd): B=4, n=1024 padded, n_real~U[768,1024], 8 blocks, "
+             "dx=256 de=64 dy=64 H=8 dh=32, bf16 storage / fp32 accumulation",
+}
 SAMPLE_ROTATION = 6     # batches cycled by the sampling workload: 6 x ~77 MB > L2
 METRIC = "edge-pairs/sec (B·n²) fwd and fwd+bwd on 1 B200; % of HBM roofline"
 UNIT = "edge-pairs/s"
@@ -137,9 +146,28 @@ def pair_kernel_bytes(p, which):
 # ------------------------------------------------------------------ our arm
 
 
+def memory_report(buf, step, torch):
+    """Device memory of the step: what the buffers hold (inputs, outputs,
+    saved state, the two workspaces) and the allocation peak over one step
+    above what was allocated before it (the library allocates nothing)."""
+    torch.cuda.synchronize()
+    before = torch.cuda.memory_allocated()
+    torch.cuda.reset_peak_memory_stats()
+    step()
+    torch.cuda.synchronize()
+    peak_delta = torch.cuda.max_memory_allocated() - before
+    mib = lambda b: b / 2**20
+    E = buf.E.numel() * buf.E.element_size()
+    return {"peak_mib_delta_per_step": mib(peak_delta), "held_mib": mib(before),
+            "workspace_fwd_mib": mib(buf.ws_fwd.numel()), "workspace_bwd_mib": mib(buf.ws_bwd.numel()),
+            "saved_mib": mib(buf.saved.numel()), "edge_tensor_mib": mib(E),
+            "workspace_bwd_per_pair_bytes": buf.ws_bwd.numel() / (buf.E.shape[0] * buf.E.shape[1] ** 2)}
+
+
 def run_ours(args):
-    if args.workload != "sbm-train":
+    if args.workload not in TRAINING:
         return run_sample(args, WORKLOADS[args.workload])
+    WORKLOAD = WORKLOADS[args.workload]
     import torch
     import torch.distributed as dist
 
@@ -245,6 +273,7 @@ def run_ours(args):
     e2e["ms"] = dp.max_over_ranks(e2e["ms"], "cuda")
 
     launches = (eaga.kernel_launches(buf.dims, False) + eaga.kernel_launches(buf.dims, True)) * K
+    mem = memory_report(buf, step, torch)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -262,11 +291,12 @@ def run_ours(args):
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded SBM-shaped graphs; edge_aware_graph_b200/inputs.py)",
-        "config": {"workload": "sbm-shaped training step (fwd+bwd): B=32, n=192 padded, n_real~U[44,187], "
-                               "dx=256 de=64 dy=64 H=8 dh=32, bf16 storage / fp32 accumulation",
+        "dtype": "bf16",
+        "data": "synthetic (seeded SBM-shaped graphs; edge_aware_graph_b200/inputs.py)",
+        "config": {"workload": DESCRIBE[WORKLOAD],
                    "global_batch": p.B * world, "seq_len": p.n, "parallelism": f"dp{world}",
-                   "l2": "inputs larger than L2 (E, dE' 144 MiB each; E', dE written each step)",
+                   "l2": f"inputs larger than L2 (E, dE' {p.B * p.n * p.n * p.de * 2 / 2**20:.0f} MiB each; "
+                         "E', dE written each step)",
                    "launch": "CUDA graph of the step's kernels" if not args.no_graph else "eager"},
         "roofline": {"bound": "hbm", "kernel": "k_bwd_stream (backward row pair kernel)", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
@@ -285,9 +315,13 @@ def run_ours(args):
         "e2e": {"value": world * pairs_step / (e2e["ms"] / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"]},
         "gpu_launches": launches,
+        "memory": mem,
     }
     if world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(p, d, W, args.cpu_graphs, args.cpu_reps)
+        graphs = min(args.cpu_graphs, p.B) if WORKLOAD == "sbm" else 1
+        reps = args.cpu_reps if WORKLOAD == "sbm" else 1
+        out["cpu_baseline"] = cpu_baseline(p, d, W, graphs, reps)
+        out["cpu_baseline_1thread"] = cpu_baseline(p, d, W, 1, 1, threads=1)
     return out
 
 
@@ -496,11 +530,13 @@ def run_e2e(args, buf, d, stream, step):
 # ------------------------------------------------------------------ oracle arm
 
 
-def cpu_baseline(p, d, W, graphs, reps=1):
+def cpu_baseline(p, d, W, graphs, reps=1, threads=None):
     """The fp64 oracle, as it stands, on a bounded sample: the first `graphs`
-    graphs of the batch, forward + backward, `reps` times, all usable host cores."""
+    graphs of the batch, forward + backward, `reps` times, on all usable host
+    cores (or on `threads` threads)."""
     import oracle
     oracle.build()
+    oracle.set_threads(threads)
     sl = {k: d[k][:graphs] for k in ("X", "E", "y", "M", "dXout", "dEout")}
     dims = dict(H=p.H, dh=p.dh)
     t = time.perf_counter()
@@ -508,8 +544,10 @@ def cpu_baseline(p, d, W, graphs, reps=1):
         oracle.forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W)
         oracle.backward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, sl["dXout"], sl["dEout"])
     dt = time.perf_counter() - t
+    cores = oracle.threads_used()
+    oracle.set_threads(None)
     pairs = reps * graphs * p.n * p.n
-    return {"value": pairs / dt, "unit": UNIT, "cores": oracle.threads_used(), "kind": "oracle",
+    return {"value": pairs / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{graphs} of {p.B} graphs of the workload (n={p.n}), forward + backward, fp64, "
                       f"{reps} time(s)",
             "seconds": dt}
@@ -539,9 +577,12 @@ def run_reference(args):
     if rank != 0:
         return None
     from edge_aware_graph_b200 import inputs as I
-    if args.workload != "sbm-train":
+    if args.workload not in TRAINING:
         return run_reference_sample(args, WORKLOADS[args.workload], world)
+    WORKLOAD = WORKLOADS[args.workload]
     p = I.preset(WORKLOAD)
+    if WORKLOAD == "large":
+        args.ref_graphs = 1
     d = I.draw_inputs(p, with_grads=True)
     W = I.draw_weights(p)
     for _ in range(args.warmup):
@@ -557,8 +598,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded SBM-shaped graphs)",
-            "config": {"workload": "sbm-shaped training step (fwd+bwd), bounded sample of "
-                                   f"{args.ref_graphs} graph(s) per step", "global_batch": args.ref_graphs,
+            "config": {"workload": DESCRIBE[WORKLOAD] + f"; bounded sample of {args.ref_graphs} graph(s) per step",
+                       "global_batch": args.ref_graphs,
                        "seq_len": p.n, "parallelism": "cpu"},
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

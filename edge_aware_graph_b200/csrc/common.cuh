@@ -24,6 +24,25 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// EAGA_ERR_INVALID_ARG for a null dims pointer, a non-positive dim or an
+// unknown dtype; EAGA_ERR_UNSUPPORTED for dims outside the limits of eaga.h.
+inline eaga_status check_dims(const eaga_dims *d) {
+    if (!d) return EAGA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->n < 1 || d->dx < 1 || d->de < 1 || d->dy < 1 || d->H < 1 || d->dh < 1)
+        return EAGA_ERR_INVALID_ARG;
+    if (d->dtype != EAGA_FP32 && d->dtype != EAGA_BF16) return EAGA_ERR_INVALID_ARG;
+    if (d->n > 1024 || d->H * d->dh > 256 || d->dh % 8 || d->de % 8 || d->de > 128 || d->dx % 8 ||
+        d->dx > 1024 || d->dy % 8 || d->dy > 1024 || 2 * d->H > 32 || d->H * d->n > 8192)
+        return EAGA_ERR_UNSUPPORTED;
+    if ((size_t)d->B * d->n > (size_t)1 << 26) return EAGA_ERR_UNSUPPORTED;
+    return EAGA_OK;
+}
+
+// Device address of the no-allocation forward's fixed scratch array on the
+// current device (looked up once per device; eaga_noalloc.cu).  Its first
+// int is that call's status word.
+eaga_status noalloc_scratch_address(void **out);
+
 // Byte layout of the forward's saved state and of the workspaces.
 struct Layout {
     size_t lse, q, k, v, o, saved_total;        // offsets inside `saved`

@@ -19,18 +19,6 @@ namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-eaga_status check_dims(const eaga_dims *d) {
-    if (!d) return EAGA_ERR_INVALID_ARG;
-    if (d->B < 1 || d->n < 1 || d->dx < 1 || d->de < 1 || d->dy < 1 || d->H < 1 || d->dh < 1)
-        return EAGA_ERR_INVALID_ARG;
-    if (d->dtype != EAGA_FP32 && d->dtype != EAGA_BF16) return EAGA_ERR_INVALID_ARG;
-    if (d->n > 1024 || d->H * d->dh > 256 || d->dh % 8 || d->de % 8 || d->de > 128 || d->dx % 8 ||
-        d->dx > 1024 || d->dy % 8 || d->dy > 1024 || 2 * d->H > 32 || d->H * d->n > 8192)
-        return EAGA_ERR_UNSUPPORTED;
-    if ((size_t)d->B * d->n > (size_t)1 << 26) return EAGA_ERR_UNSUPPORTED;
-    return EAGA_OK;
-}
-
 eaga_status check_ptrs(std::initializer_list<const void *> ps) {
     for (const void *p : ps) {
         if (!p) return EAGA_ERR_INVALID_ARG;
@@ -217,21 +205,40 @@ __global__ void k_wait_probe(int *status, unsigned limit) {
     if (threadIdx.x == 0 && !sm100::mbar_wait(b, 0, limit)) atomicExch(status, DEV_TIMEOUT);
 }
 
+// The status word a call reports through: the workspace's first int, or, for
+// workspace == NULL, that of the no-allocation forward's fixed scratch array
+// on the current device.
+static eaga_status status_word(void *workspace, int **out) {
+    if (workspace) {
+        if (reinterpret_cast<uintptr_t>(workspace) & 15u) return EAGA_ERR_MISALIGNED;
+        *out = static_cast<int *>(workspace);
+        return EAGA_OK;
+    }
+    void *base = nullptr;
+    const eaga_status s = noalloc_scratch_address(&base);
+    *out = static_cast<int *>(base);
+    return s;
+}
+
 eaga_status eaga_debug_wait_probe(void *workspace, unsigned limit, void *stream) {
-    if (!workspace || limit < 1 || limit > (1u << 24)) return EAGA_ERR_INVALID_ARG;
-    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return EAGA_ERR_MISALIGNED;
+    if (limit < 1 || limit > (1u << 24)) return EAGA_ERR_INVALID_ARG;
+    int *word = nullptr;
+    const eaga_status s = status_word(workspace, &word);
+    if (s != EAGA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    k_wait_probe<<<1, 32, 0, st>>>(static_cast<int *>(workspace), limit);
+    k_wait_probe<<<1, 32, 0, st>>>(word, limit);
     return cudaGetLastError() == cudaSuccess ? EAGA_OK : EAGA_ERR_CUDA;
 }
 
 eaga_status eaga_get_device_status(void *workspace, void *stream) {
-    if (!workspace) return EAGA_ERR_INVALID_ARG;
+    int *word = nullptr;
+    const eaga_status s = status_word(workspace, &word);
+    if (s != EAGA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int h = 0;
-    if (cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (cudaMemcpyAsync(&h, word, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return EAGA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return EAGA_ERR_CUDA;
-    if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (cudaMemsetAsync(word, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return EAGA_ERR_CUDA;
     return h == DEV_OK ? EAGA_OK : EAGA_ERR_TIMEOUT;
 }

@@ -32,10 +32,16 @@ constexpr int MAX_DEVICES = 64;
 std::mutex g_setup_mutex;
 void *g_scratch_addr[MAX_DEVICES] = {};
 
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+namespace eaga {
+
 // The device address of the array on the current device.  In host code the
 // variable's name only stands for it, so the address is looked up once per
 // device (with that device current) and cached.
-eaga_status scratch_address(void **out) {
+eaga_status noalloc_scratch_address(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return EAGA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
@@ -48,9 +54,7 @@ eaga_status scratch_address(void **out) {
     return EAGA_OK;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-}  // namespace
+}  // namespace eaga
 
 extern "C" {
 
@@ -59,8 +63,8 @@ eaga_status eaga_forward_noalloc(const eaga_dims *d, const void *X, const void *
     // The same argument checks as eaga_forward, with `saved` required: the
     // forward's saved state is as large as the node tensors and stays the
     // caller's buffer.
-    const size_t ws = eaga_workspace_size(d, 0);
-    if (ws == 0) return d ? EAGA_ERR_UNSUPPORTED : EAGA_ERR_INVALID_ARG;
+    const eaga_status ds = check_dims(d);
+    if (ds != EAGA_OK) return ds;
     if (!w) return EAGA_ERR_INVALID_ARG;
     const void *ptrs[] = {X, E, y, M, Xout, Eout, saved, w->Wq, w->bq, w->Wk, w->bk, w->Wv,
                           w->bv, w->Wfe, w->Wfy, w->bf, w->We, w->Wo, w->bo};
@@ -83,7 +87,7 @@ eaga_status eaga_forward_noalloc(const eaga_dims *d, const void *X, const void *
     }
 
     void *base = nullptr;
-    eaga_status s = scratch_address(&base);
+    eaga_status s = noalloc_scratch_address(&base);
     if (s != EAGA_OK) return s;
     char *scratch = static_cast<char *>(base);
     cudaStream_t st = static_cast<cudaStream_t>(stream);

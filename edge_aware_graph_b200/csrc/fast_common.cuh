@@ -205,6 +205,28 @@ __device__ __forceinline__ void add_residual16(uint8_t *row, uint32_t L, int hq,
 }
 
 __device__ __forceinline__ void flag_timeout(int *status) { atomicExch(status, DEV_TIMEOUT); }
+
+// Bounded wait on phase `parity` of mbarrier `bar` that gives up for the
+// whole CTA.  `fail` is a flag in shared memory, zero at the start.  The
+// first wait of the CTA that runs out of polls sets it and records
+// DEV_TIMEOUT in the status word; from then on every wait returns false at
+// once (a thread already waiting notices within 256 polls), the issuing
+// threads stop issuing TMA copies and MMAs, and the CTA runs its remaining
+// control flow (the same named barriers, in-bounds addresses) to the end,
+// where it waits, again with a bound, for what it already issued and frees
+// its tensor memory.  A stalled CTA therefore costs about one bound, not one
+// bound per wait.
+__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, volatile int *fail, int *status,
+                                         uint32_t limit = (1u << 24)) {
+    if (*fail) return false;
+    for (uint32_t it = 0; it < limit; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 255u && *fail) return false;
+    }
+    *fail = 1;
+    flag_timeout(status);
+    return false;
+}
 }  // namespace dev
 }  // namespace fast
 }  // namespace eaga

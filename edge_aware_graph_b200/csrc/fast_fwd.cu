@@ -53,13 +53,15 @@ struct FsSmem {
     static constexpr uint32_t G = FIN + 512;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // mask of the graph's nodes [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;                // mbarriers, see below
-    static constexpr uint32_t TM = BAR + 8 * 16;              // TMEM base address
+    static constexpr uint32_t TM = BAR + 8 * 17;              // TMEM base address
+    static constexpr uint32_t FAIL = TM + 8;                  // CTA failure flag (a wait ran out)
     static constexpr uint32_t BYTES = TM + 16 + 1024;         // + alignment slack
     static constexpr uint32_t OPART = 0;                      // [4][8][256] f32 O partials (ring drained)
 };
-// mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full[2], edge_full[2], stage_done[4]
+// mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full[2], edge_full[2], stage_done[4],
+// mma_final (all MMAs of the CTA complete)
 constexpr int FB_FULL = 0, FB_FILM_FULL = 4, FB_FILM_EMPTY = 6, FB_A_FULL = 8, FB_EDGE_FULL = 10,
-              FB_STAGE_DONE = 12;
+              FB_STAGE_DONE = 12, FB_MMA_FINAL = 16;
 
 // TMEM columns: FiLM 0..63 (two buffers), edge update 64..319 (two buffers),
 // pass-1 scores from 320 on (16 per chunk, kept when nch <= 12 so pass 2 needs no K)
@@ -93,6 +95,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     auto bar = [&](int k) { return bars + 8 * k; };
     float *g = reinterpret_cast<float *>(sp + S::G);
     uint8_t *mj = sp + S::MJ;
+    volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
 
     // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0.  Its
     // slots, from slot_base(it) on: pass 1 E(s=0), E(s=1), K; pass 2 E(s=0),
@@ -116,7 +119,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         mbar_init(bar(FB_EDGE_FULL), 1);
         mbar_init(bar(FB_EDGE_FULL + 1), 1);
         for (int k = 0; k < 4; ++k) mbar_init(bar(FB_STAGE_DONE + k), NWARP);
+        mbar_init(bar(FB_MMA_FINAL), 1);
         fence_mbar_init();
+        *fail = 0;
     }
     if (W == 0) {
         tmem_alloc(sbase + S::TM, FS_TM_COLS);
@@ -165,7 +170,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             // chunk whose a the compute warps have written
             int next_film = 0, next_edge = nch;
             uint32_t polls = 0;
-            while (next_film < nit || next_edge < nit) {
+            while ((next_film < nit || next_edge < nit) && !*fail) {
                 bool progressed = false;
                 if (next_film < nit &&
                     mbar_test_wait(bar(FB_FULL + next_film % FS_NFULL), (next_film / FS_NFULL) & 1) &&
@@ -181,10 +186,14 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     progressed = true;
                 }
                 if (!progressed && ++polls > (1u << 28)) {
+                    *fail = 1;
                     flag_timeout(p.status);
                     break;
                 }
             }
+            // every product issued has completed before the tensor memory is freed
+            mma_commit(bar(FB_MMA_FINAL));
+            if (!mbar_wait(bar(FB_MMA_FINAL), 0)) flag_timeout(p.status);
         }
         __syncwarp();
         named_bar_sync(2, FS_THR);
@@ -196,7 +205,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
             int next_load = 0, free_slots = FS_SLOTS;
             auto issue_loads = [&]() {
-                while (next_load < nit && nslots(next_load) <= free_slots) {
+                while (next_load < nit && nslots(next_load) <= free_slots && !*fail) {
                     const int it = next_load, j0 = 32 * chunk_of(it);
                     const bool pass2 = it >= nch;
                     const uint32_t fb = bar(FB_FULL + it % FS_NFULL);
@@ -229,7 +238,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                             for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, s, pb);
                     }
                 }
-                if (!mbar_wait(bar(FB_STAGE_DONE + (it & 3)), (it >> 2) & 1)) flag_timeout(p.status);
+                if (!cta_wait(bar(FB_STAGE_DONE + (it & 3)), (it >> 2) & 1, fail, p.status)) continue;
                 if (pass2) {
                     const int j0 = 32 * chunk_of(it);
                     tma_store_5d_hint(&tmEo, slot_addr(it, 0), 0, i0 / 2, j0, 0, b, drop_l2);
@@ -246,6 +255,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 issue_loads();
             }
             tma_store_wait_read0();
+            if (*fail)   // loads already issued land before the CTA's shared memory is released
+                for (int it = max(next_load - FS_NFULL, 0); it < next_load; ++it)
+                    mbar_wait(bar(FB_FULL + it % FS_NFULL), (it / FS_NFULL) & 1);
         }
         __syncwarp();
         named_bar_sync(2, FS_THR);   // the ring is drained: the compute warps may reuse it
@@ -281,7 +293,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         // E' = E + a We of pass-2 chunk it, in place (the TMA warp stores it)
         auto edge_residual = [&](int it) {
             const int p2 = it - nch;
-            if (!mbar_wait(bar(FB_EDGE_FULL + (p2 & 1)), (p2 >> 1) & 1)) flag_timeout(p.status);
+            cta_wait(bar(FB_EDGE_FULL + (p2 & 1)), (p2 >> 1) & 1, fail, p.status);
             tc_fence_after();
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -354,7 +366,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             }
 
             // ---------------- scores S^T = K Q^T on warp MMAs (2 heads per warp)
-            if (!mbar_wait(bar(FB_FULL + it % FS_NFULL), (it / FS_NFULL) & 1)) flag_timeout(p.status);
+            cta_wait(bar(FB_FULL + it % FS_NFULL), (it / FS_NFULL) & 1, fail, p.status);
             float sacc[2][4];
             const uint32_t scol = tl + FS_TM_S + 16 * chunk_of(it) + 2 * hq;
             if (pass2 && keep_s) {
@@ -370,7 +382,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             }
 
             // ---------------- combine with FiLM: s' = s(1+gamma)+beta, masked
-            if (!mbar_wait(bar(FB_FILM_FULL + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
+            cta_wait(bar(FB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
             tc_fence_after();
             float gm[2][2], bt[2][2];
 #pragma unroll

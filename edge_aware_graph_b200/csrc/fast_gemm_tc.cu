@@ -18,6 +18,7 @@ namespace eaga {
 namespace fast {
 
 using namespace sm100;
+using dev::cta_wait;
 
 constexpr int TBM = 128, TBK = 64, TTHR = 128;
 // pipeline stages: 4 for 64-wide tiles, 3 for 128-wide (two CTAs fit an SM either way)
@@ -40,6 +41,7 @@ struct TcSmem {
     static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
     static constexpr uint32_t BAR = TSTAGES * STAGE;        // full[S], empty[S], done
     static constexpr uint32_t TM = BAR + (2 * TSTAGES + 1) * 8;
+    static constexpr uint32_t FAIL = TM + 4;                 // CTA failure flag (a wait ran out)
     static constexpr uint32_t BIAS = TM + 16;                // the tile's BN bias values, fp32
     static constexpr uint32_t BYTES = BIAS + BN * 4 + 1024;
 };
@@ -56,6 +58,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
     const int tid = threadIdx.x, w = tid >> 5, t = tid & 31;
     const int n0 = blockIdx.x * BN, m0 = blockIdx.y * TBM;
+    volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
     const uint32_t bar0 = sbase + S::BAR;
     auto full = [&](int s) { return bar0 + 8 * s; };
     auto empty = [&](int s) { return bar0 + 8 * (TSTAGES + s); };
@@ -70,6 +73,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
         }
         mbar_init(done, 1);
         fence_mbar_init();
+        *reinterpret_cast<volatile int *>(sp + S::FAIL) = 0;
     }
     if (w == 0) {
         tmem_alloc(sbase + S::TM, BN);
@@ -103,12 +107,13 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
                 tma_load_2d(st + S::A_BYTES, bm, full(s), k0, n0);
             }
         };
-        for (int kt = 0; kt < TSTAGES && kt < nk; ++kt) issue_load(kt);
+        int issued = 0;
+        for (; issued < TSTAGES && issued < nk; ++issued) issue_load(issued);
         const uint32_t idesc = idesc_bf16_f32(TBM, BN) | (p.b_mn ? (1u << 16) : 0u);
         for (int kt = 0; kt < nk; ++kt) {
             const int s = kt % TSTAGES;
             const uint32_t ph = (kt / TSTAGES) & 1;
-            if (!mbar_wait(full(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
+            if (!cta_wait(full(s), ph, fail, p.status)) break;
             tc_fence_after();
             const uint32_t st = sbase + s * S::STAGE;
 #pragma unroll
@@ -119,11 +124,15 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
                             idesc, (kt > 0 || kk > 0) ? 1u : 0u);
             mma_commit(empty(s));
             if (kt + TSTAGES < nk) {
-                if (!mbar_wait(empty(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
-                issue_load(kt + TSTAGES);
+                if (!cta_wait(empty(s), ph, fail, p.status)) break;
+                issue_load(issued++);
             }
         }
         mma_commit(done);
+        if (*fail) {   // what was issued completes before the CTA's memory is released
+            for (int kt = max(issued - TSTAGES, 0); kt < issued; ++kt) mbar_wait(full(kt % TSTAGES), (kt / TSTAGES) & 1);
+            mbar_wait(done, 0);
+        }
     }
     __syncwarp();
     // epilogue: warp w holds rows m0 + 32w + t.  The residual row segment is
@@ -138,7 +147,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
 #pragma unroll
     for (int u = 0; u < BN / 8; ++u)
         res[u] = (has_res && in) ? reinterpret_cast<const uint4 *>(p.R + obase)[u] : make_uint4(0, 0, 0, 0);
-    if (!mbar_wait(done, 0)) atomicExch(p.status, DEV_TIMEOUT);
+    cta_wait(done, 0, fail, p.status);
     tc_fence_after();
 #pragma unroll
     for (int c0 = 0; c0 < BN; c0 += 16) {
@@ -193,6 +202,7 @@ struct WgSmem {
     static constexpr int ST = 3;
     static constexpr uint32_t BAR = ST * STAGE;
     static constexpr uint32_t TM = BAR + (2 * ST + 1) * 8;
+    static constexpr uint32_t FAIL = TM + 4;                 // CTA failure flag (a wait ran out)
     static constexpr uint32_t BYTES = TM + 16 + 1024;
 };
 
@@ -207,6 +217,7 @@ k_tc_wgrad(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUten
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
     const int tid = threadIdx.x, w = tid >> 5, t = tid & 31;
     const int n0g = blockIdx.x * BN, m0 = blockIdx.y * TBM;
+    volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
     const int which = n0g / p.Nb, n0 = n0g % p.Nb;
     const int kbeg = blockIdx.z * p.kchunk, kend = min(p.K, kbeg + p.kchunk);
     const int nk = kend > kbeg ? (kend - kbeg + TBK - 1) / TBK : 0;
@@ -223,6 +234,7 @@ k_tc_wgrad(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUten
         }
         mbar_init(done, 1);
         fence_mbar_init();
+        *reinterpret_cast<volatile int *>(sp + S::FAIL) = 0;
     }
     if (w == 0) {
         tmem_alloc(sbase + S::TM, BN);
@@ -243,12 +255,13 @@ k_tc_wgrad(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUten
 #pragma unroll
             for (int h = 0; h < BN / 64; ++h) tma_load_2d(st + S::A_BYTES + h * 8192, bm, full(s), n0 + 64 * h, k0);
         };
-        for (int kt = 0; kt < ST && kt < nk; ++kt) issue_load(kt);
+        int issued = 0;
+        for (; issued < ST && issued < nk; ++issued) issue_load(issued);
         const uint32_t idesc = idesc_bf16_f32_mn(TBM, BN);
         for (int kt = 0; kt < nk; ++kt) {
             const int s = kt % ST;
             const uint32_t ph = (kt / ST) & 1;
-            if (!mbar_wait(full(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
+            if (!cta_wait(full(s), ph, fail, p.status)) break;
             tc_fence_after();
             const uint32_t st = sbase + s * S::STAGE;
 #pragma unroll
@@ -258,14 +271,18 @@ k_tc_wgrad(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUten
                             (kt > 0 || kk > 0) ? 1u : 0u);
             mma_commit(empty(s));
             if (kt + ST < nk) {
-                if (!mbar_wait(empty(s), ph)) atomicExch(p.status, DEV_TIMEOUT);
-                issue_load(kt + ST);
+                if (!cta_wait(empty(s), ph, fail, p.status)) break;
+                issue_load(issued++);
             }
         }
         mma_commit(done);
+        if (*fail) {   // what was issued completes before the CTA's memory is released
+            for (int kt = max(issued - ST, 0); kt < issued; ++kt) mbar_wait(full(kt % ST), (kt / ST) & 1);
+            mbar_wait(done, 0);
+        }
     }
     __syncwarp();
-    if (!mbar_wait(done, 0)) atomicExch(p.status, DEV_TIMEOUT);
+    cta_wait(done, 0, fail, p.status);
     tc_fence_after();
     const int row = m0 + 32 * w + t;
     float *P = p.P[which] + (size_t)blockIdx.z * p.M * p.Nb + (size_t)row * p.Nb + n0;

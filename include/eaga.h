@@ -141,20 +141,25 @@ EAGA_API eaga_status eaga_backward(const eaga_dims *dims,
  * same arguments minus the workspace; `saved` is required (it is an output
  * as large as the node tensors).
  *
+ * Argument checks and error codes are those of eaga_forward (invalid dims
+ * give EAGA_ERR_INVALID_ARG, dims outside the limits EAGA_ERR_UNSUPPORTED).
+ *
  * The forward's small scratch (status word, global FiLM term g [B,2H] fp32,
- * 8 KB of tensor-core operand images on the bf16 path) lives in a 64 KiB
- * array in the library's device memory, held by every GPU that loads the
- * library until the process exits.  Limit: 256 + roundup256(8*H*B) + 8192
- * bytes must fit in 64 KiB, so B <= 892 graphs at H = 8; larger B returns
- * EAGA_ERR_UNSUPPORTED without launching.  No device memory is allocated or
- * freed by this call.
+ * and on the specialised bf16 path of de = 64, H = 8, dh = 32 also 8 KiB of
+ * tensor-core operand images) lives in a 64 KiB array in the library's
+ * device memory, held by every GPU that loads the library until the process
+ * exits.  Limit: 256 + roundup256(8*H*B) bytes, plus 8192 on the specialised
+ * path, must fit in 64 KiB: B <= 892 graphs on the specialised path, B <= 4080
+ * at H = 2 on the CUDA-core path; larger B returns EAGA_ERR_UNSUPPORTED
+ * without launching.  No device memory is allocated or freed by this call.
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
  * capture.  Every call on a device shares the array and leaves its contents
  * behind: calls that overlap on the GPU (other streams, other host threads)
  * race on it and must be serialised by the caller.  The status word is
- * cleared at the start of each call. */
+ * cleared at the start of each call; eaga_get_device_status(NULL, stream)
+ * reads it (EAGA_ERR_TIMEOUT if a bounded device wait of the call ran out). */
 EAGA_API eaga_status eaga_forward_noalloc(const eaga_dims *dims,
                                           const void *X, const void *E, const void *y, const uint8_t *M,
                                           const eaga_weights *w, void *Xout, void *Eout, void *saved,
@@ -170,7 +175,9 @@ EAGA_API eaga_status eaga_debug_attention_map(const eaga_dims *dims, const void 
 
 /* Synchronises `stream`, then reads and clears the device status word kept at
  * the start of `workspace`: EAGA_OK, or EAGA_ERR_TIMEOUT if a bounded
- * device-side wait ran out during a call that used this workspace. */
+ * device-side wait ran out during a call that used this workspace.  With
+ * workspace == NULL it reads the status word of eaga_forward_noalloc (the
+ * first int of the library's fixed scratch array on the current device). */
 EAGA_API eaga_status eaga_get_device_status(void *workspace, void *stream);
 
 /* Profiling aid.  After eaga_set_profile_events(point, before, after) with
@@ -194,8 +201,9 @@ EAGA_API int eaga_kernel_launches(const eaga_dims *dims, int for_backward);
  * (1 <= limit <= 2^24); when the limit runs out the kernel records the
  * timeout in the status word at the start of `workspace` and returns, the
  * way a pair kernel does (no trap, the context stays usable).  A following
- * eaga_get_device_status on that workspace returns EAGA_ERR_TIMEOUT.  The
- * pages have no counterpart. */
+ * eaga_get_device_status on that workspace returns EAGA_ERR_TIMEOUT.  With
+ * workspace == NULL the probe reports into the status word of
+ * eaga_forward_noalloc instead.  The pages have no counterpart. */
 EAGA_API eaga_status eaga_debug_wait_probe(void *workspace, unsigned limit, void *stream);
 
 /* Static, human-readable name of a status code. */

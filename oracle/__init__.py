@@ -116,8 +116,23 @@ def backward(dims: dict, X, E, y, M, W: dict, dXout, dEout):
     return out
 
 
+_threads = None
+
+
+def set_threads(n: int | None) -> None:
+    """Run the oracle's OpenMP loops on n threads (None: back to all usable
+    cores).  Only the thread count changes, never the arithmetic."""
+    global _threads
+    _load()
+    gomp = ctypes.CDLL("libgomp.so.1")
+    gomp.omp_set_num_threads(int(n) if n else len(os.sched_getaffinity(0)))
+    _threads = int(n) if n else None
+
+
 def threads_used() -> int:
-    """OpenMP threads the oracle runs with (OMP_NUM_THREADS, else all usable cores)."""
+    """OpenMP threads the oracle runs with (set_threads, OMP_NUM_THREADS, else all usable cores)."""
+    if _threads:
+        return _threads
     env = os.environ.get("OMP_NUM_THREADS")
     if env:
         return int(env)

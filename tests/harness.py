@@ -16,6 +16,34 @@ def rel_err(gpu, ref) -> float:
     return float(np.abs(g - ref).max() / scale)
 
 
+def _half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Half a unit in the last place of the storage dtype at each value of x."""
+    bits = 8 if dtype == "bf16" else 24              # significand bits incl. the implicit one
+    ax = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - bits), 0.0)
+
+
+def increment_err(gpu_out, base, ref_out, dtype: str) -> float:
+    """Error of a residual output's increment, on the increment's own scale.
+
+    A residual output (X' = X + ..., E' = E + ..., dE = dE' + ..., dX = dX' + ...)
+    is compared as out - base against the oracle's out - base, relative to
+    max |oracle increment|, so that a small update is not hidden under the
+    scale of the input it is added to.  The GPU output is stored in `dtype`
+    (round to nearest): its unrounded increment lies within half an ulp of
+    the stored output, so that half ulp (the storage rounding, not arithmetic
+    of the layer) is allowed on top of the parity tolerance."""
+    g = gpu_out.detach().float().cpu().numpy().astype(np.float64) if hasattr(gpu_out, "detach") else np.asarray(gpu_out, np.float64)
+    b = base.detach().float().cpu().numpy().astype(np.float64) if hasattr(base, "detach") else np.asarray(base, np.float64)
+    inc_ref = np.asarray(ref_out, np.float64) - b
+    scale = np.abs(inc_ref).max()
+    dev = np.maximum(np.abs((g - b) - inc_ref) - _half_ulp(g, dtype), 0.0)
+    if scale == 0:
+        return float(dev.max())
+    return float(dev.max() / scale)
+
+
 def custom_case(B, n, dx, de, dy, H, dh, dtype, seed, mask="random", with_grads=True):
     """Dense-family case of arbitrary dims with a chosen mask pattern.
 

@@ -104,7 +104,7 @@ def test_strerror(L):
 
 def test_wait_probe_arguments(L):
     # argument checks happen on the host, before any launch
-    assert L.eaga_debug_wait_probe(None, 100, None) == 1           # EAGA_ERR_INVALID_ARG
+    assert L.eaga_debug_wait_probe(None, 0, None) == 1             # EAGA_ERR_INVALID_ARG
     fake = ctypes.c_void_p(0x100000)
     assert L.eaga_debug_wait_probe(fake, 0, None) == 1
     assert L.eaga_debug_wait_probe(fake, (1 << 24) + 1, None) == 1

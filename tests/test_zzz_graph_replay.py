@@ -11,7 +11,7 @@ import torch
 from edge_aware_graph_b200 import inputs as I
 from edge_aware_graph_b200.buffers import LayerBuffers
 
-from harness import TOL, oracle_backward, oracle_forward, rel_err
+from harness import TOL, increment_err, oracle_backward, oracle_forward, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -49,6 +49,10 @@ def test_sbm_training_step_replayed_from_a_cuda_graph(oracle_lib):
     errs = {"Xout": rel_err(buf.Xout, rf["Xout"]), "Eout": rel_err(buf.Eout, rf["Eout"]),
             "O": rel_err(buf.saved_parts()["O"], rf["O"]),
             "dX": rel_err(buf.dX, rb["dX"]), "dE": rel_err(buf.dE, rb["dE"]), "dy": rel_err(buf.dy, rb["dy"])}
+    errs["Xinc"] = increment_err(buf.Xout, buf.X, rf["Xout"], p.dtype)
+    errs["Einc"] = increment_err(buf.Eout, buf.E, rf["Eout"], p.dtype)
+    errs["dXinc"] = increment_err(buf.dX, buf.dXout, rb["dX"], p.dtype)
+    errs["dEinc"] = increment_err(buf.dE, buf.dEout, rb["dE"], p.dtype)
     for k in I.WEIGHT_NAMES:
         errs["d" + k] = rel_err(buf.dW[k], rb["d" + k])
     bad = {k: v for k, v in errs.items() if not v <= tol}       # NaN fails this test too
