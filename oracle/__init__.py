@@ -17,6 +17,10 @@ _SRC = os.path.join(_HERE, "eaga_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 WEIGHT_NAMES = ("Wq", "bq", "Wk", "bk", "Wv", "bv", "Wfe", "Wfy", "bf", "We", "Wo", "bo")
+# layer variants (eaga_oracle.c): the layer, and the two ablations of the
+# AI-summary page (Light Edge: no per-edge modulation; unnormalised: the edge
+# update from the modulated scores instead of the normalised coefficients)
+VARIANTS = {"layer": 0, "light_edge": 1, "unnormalised": 2}
 
 
 class _Dims(ctypes.Structure):
@@ -42,7 +46,7 @@ def _load():
     global _lib
     if _lib is None:
         _lib = ctypes.CDLL(build())
-        for fn in (_lib.orc_forward, _lib.orc_backward):
+        for fn in (_lib.orc_forward, _lib.orc_backward, _lib.orc_forward_variant, _lib.orc_backward_variant):
             fn.restype = ctypes.c_int
     return _lib
 
@@ -66,11 +70,11 @@ def _shapes_of(X, E, y):
     return B, n, dx, E.shape[-1], y.shape[-1]
 
 
-def forward(dims: dict, X, E, y, M, W: dict, want_attention: bool = False):
+def forward(dims: dict, X, E, y, M, W: dict, want_attention: bool = False, variant: str = "layer"):
     """fp64 forward.  dims needs H and dh; B, n, dx, de, dy come from shapes.
 
     Returns dict with Xout, Eout, O [B,n,H*dh], LSE [B,H,n] and, if asked,
-    A [B,H,n,n].
+    A [B,H,n,n].  `variant` is one of VARIANTS.
     """
     lib = _load()
     B, n, dx, de, dyd = _shapes_of(X, E, y)
@@ -86,15 +90,15 @@ def forward(dims: dict, X, E, y, M, W: dict, want_attention: bool = False):
     }
     if want_attention:
         out["A"] = np.empty((B, d["H"], n, n))
-    rc = lib.orc_forward(ctypes.byref(_dims(d)), _ptr(X), _ptr(E), _ptr(y), _ptr(M),
-                         ctypes.byref(wst), _ptr(out["Xout"]), _ptr(out["Eout"]),
-                         _ptr(out.get("A")), _ptr(out["O"]), _ptr(out["LSE"]))
+    rc = lib.orc_forward_variant(ctypes.byref(_dims(d)), VARIANTS[variant], _ptr(X), _ptr(E), _ptr(y), _ptr(M),
+                                 ctypes.byref(wst), _ptr(out["Xout"]), _ptr(out["Eout"]),
+                                 _ptr(out.get("A")), _ptr(out["O"]), _ptr(out["LSE"]))
     if rc != 0:
         raise RuntimeError(f"orc_forward failed: {rc}")
     return out
 
 
-def backward(dims: dict, X, E, y, M, W: dict, dXout, dEout):
+def backward(dims: dict, X, E, y, M, W: dict, dXout, dEout, variant: str = "layer"):
     """fp64 backward.  Returns dict with dX, dE, dy and d<weight> for each weight."""
     lib = _load()
     B, n, dx, de, dyd = _shapes_of(X, E, y)
@@ -106,8 +110,8 @@ def backward(dims: dict, X, E, y, M, W: dict, dXout, dEout):
     grads = {k: np.zeros_like(Wd[k]) for k in WEIGHT_NAMES}
     gst = _Weights(*(_ptr(grads[k]) for k in WEIGHT_NAMES))
     out = {"dX": np.empty_like(X), "dE": np.empty_like(E), "dy": np.empty_like(y)}
-    rc = lib.orc_backward(ctypes.byref(_dims(d)), _ptr(X), _ptr(E), _ptr(y), _ptr(M),
-                          ctypes.byref(wst), _ptr(dXout), _ptr(dEout),
+    rc = lib.orc_backward_variant(ctypes.byref(_dims(d)), VARIANTS[variant], _ptr(X), _ptr(E), _ptr(y), _ptr(M),
+                                  ctypes.byref(wst), _ptr(dXout), _ptr(dEout),
                           _ptr(out["dX"]), _ptr(out["dE"]), _ptr(out["dy"]), ctypes.byref(gst))
     if rc != 0:
         raise RuntimeError(f"orc_backward failed: {rc}")

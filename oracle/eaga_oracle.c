@@ -25,6 +25,15 @@
  * Weights are [in, out] row-major (Y = X W).  Every loop below follows these
  * formulas in the order written; there is no blocking or reordering.
  *
+ * Two ablation variants of the layer (AI summary page: the method
+ * paragraph's ablation of unnormalised coefficients, and the "Light Edge"
+ * bullet), selected by `variant`:
+ *   ORC_LIGHT_EDGE   no per-edge modulation: gamma, beta = y_b Wfy + bf (Wfe
+ *                    is not used and its gradient is zero);
+ *   ORC_UNNORMALISED the edge update takes the unnormalised coefficients, the
+ *                    modulated scores themselves: E' = E + sum_h s'^h We[h,:]
+ *                    on valid pairs (invalid pairs keep E); nodes unchanged.
+ *
  * Parity pins (tests/test_oracle_pins.py): zero-FiLM special case against
  * torch's float64 scaled_dot_product_attention; the gamma = -1 closed form
  * (uniform attention); row sums; masked-entry invariance; permutation
@@ -40,6 +49,7 @@
 #include <string.h>
 
 typedef struct { int B, n, dx, de, dy, H, dh; } orc_dims;
+enum { ORC_LAYER = 0, ORC_LIGHT_EDGE = 1, ORC_UNNORMALISED = 2 };
 typedef struct {
     const double *Wq, *bq, *Wk, *bk, *Wv, *bv, *Wfe, *Wfy, *bf, *We, *Wo, *bo;
 } orc_weights;
@@ -153,12 +163,15 @@ static void row_attention(const orc_dims *d, const double *E, const unsigned cha
  *   LSE [B,H,n]   (nullable) m + log l per valid row, -inf on masked rows
  * Returns 0.
  */
-int orc_forward(const orc_dims *d, const double *X, const double *E, const double *y,
-                const unsigned char *M, const orc_weights *w,
-                double *Xout, double *Eout, double *A, double *O, double *LSE)
+int orc_forward_variant(const orc_dims *d, int variant, const double *X, const double *E, const double *y,
+                        const unsigned char *M, const orc_weights *w,
+                        double *Xout, double *Eout, double *A, double *O, double *LSE)
 {
     const int B = d->B, n = d->n, H = d->H, dh = d->dh, hd = H * dh, de = d->de, dx = d->dx;
     const long rows = (long)B * n;
+    /* Light Edge: the per-edge FiLM map is absent (zero) */
+    double *Wfe0 = (double *)calloc((size_t)de * 2 * H, sizeof(double));
+    const double *Wfe = variant == ORC_LIGHT_EDGE ? Wfe0 : w->Wfe;
     double *Q = (double *)malloc(sizeof(double) * rows * hd);
     double *K = (double *)malloc(sizeof(double) * rows * hd);
     double *V = (double *)malloc(sizeof(double) * rows * hd);
@@ -173,7 +186,7 @@ int orc_forward(const orc_dims *d, const double *X, const double *E, const doubl
         double *srow = (double *)malloc(sizeof(double) * H * n);
         double *frow = (double *)malloc(sizeof(double) * n * 2 * H);
         double lse[64];
-        row_attention(d, E, M, Q, K, w->Wfe, g, b, i, arow, srow, frow, lse);
+        row_attention(d, E, M, Q, K, Wfe, g, b, i, arow, srow, frow, lse);
         /* node aggregation O_ih = sum_j a_ij v_jh */
         for (int h = 0; h < H; ++h)
             for (int t = 0; t < dh; ++t) {
@@ -182,12 +195,22 @@ int orc_forward(const orc_dims *d, const double *X, const double *E, const doubl
                     acc += arow[(long)h * n + j] * V[((long)b * n + j) * hd + h * dh + t];
                 Ob[r * hd + h * dh + t] = acc;
             }
-        /* edge residual E'_ij = E_ij + sum_h a^h_ij We[h,:] */
+        /* edge residual E'_ij = E_ij + sum_h coef^h_ij We[h,:], coef = a (the layer) or,
+           unnormalised, the modulated score s' on valid pairs and 0 elsewhere */
         for (int j = 0; j < n; ++j) {
             const long e0 = (((long)b * n + i) * n + j) * de;
+            const int valid = M[(long)b * n + i] && M[(long)b * n + j];
             for (int c = 0; c < de; ++c) {
                 double acc = E[e0 + c];
-                for (int h = 0; h < H; ++h) acc += arow[(long)h * n + j] * w->We[(long)h * de + c];
+                for (int h = 0; h < H; ++h) {
+                    double coef = arow[(long)h * n + j];
+                    if (variant == ORC_UNNORMALISED) {
+                        const double sp = srow[(long)h * n + j] * (1.0 + frow[(long)j * 2 * H + h]) +
+                                          frow[(long)j * 2 * H + H + h];
+                        coef = valid ? sp : 0.0;
+                    }
+                    acc += coef * w->We[(long)h * de + c];
+                }
                 Eout[e0 + c] = acc;
             }
         }
@@ -211,8 +234,15 @@ int orc_forward(const orc_dims *d, const double *X, const double *E, const doubl
         }
     }
     if (O) memcpy(O, Ob, sizeof(double) * rows * hd);
-    free(Q); free(K); free(V); free(g); free(Ob);
+    free(Q); free(K); free(V); free(g); free(Ob); free(Wfe0);
     return 0;
+}
+
+int orc_forward(const orc_dims *d, const double *X, const double *E, const double *y,
+                const unsigned char *M, const orc_weights *w,
+                double *Xout, double *Eout, double *A, double *O, double *LSE)
+{
+    return orc_forward_variant(d, ORC_LAYER, X, E, y, M, w, Xout, Eout, A, O, LSE);
 }
 
 /*
@@ -234,15 +264,25 @@ int orc_forward(const orc_dims *d, const double *X, const double *E, const doubl
  * Row work (D, dq, dE, per-row weight-gradient parts) runs per (b,i); column
  * work (dk, dv) per (b,j), recomputing a_ij; per-row parts are summed in row
  * order afterwards.
+ *
+ * Variants.  Light Edge: Wfe is zero in every formula above and its gradient
+ * dWfe is zero (the map is not a parameter of that layer).  Unnormalised: the
+ * edge update reads s' itself, so the edge path reaches s' without the
+ * softmax:  D_ih = sum_j a_ij dO_ih . v_jh  (node path only),
+ *   dS'_ij = a_ij (dO_ih . v_jh - D_ih) + [valid_ij] u_ij,
+ *   dWe = sum_ij [valid_ij] s'_ij^T dE'_ij;  everything downstream of dS' as above.
  */
-int orc_backward(const orc_dims *d, const double *X, const double *E, const double *y,
-                 const unsigned char *M, const orc_weights *w,
-                 const double *dXout, const double *dEout,
-                 double *dX, double *dE, double *dy, orc_grads *gr)
+int orc_backward_variant(const orc_dims *d, int variant, const double *X, const double *E, const double *y,
+                         const unsigned char *M, const orc_weights *w,
+                         const double *dXout, const double *dEout,
+                         double *dX, double *dE, double *dy, orc_grads *gr)
 {
     const int B = d->B, n = d->n, H = d->H, dh = d->dh, hd = H * dh, de = d->de;
     const int dx = d->dx, dyd = d->dy, F = 2 * H;
     const long rows = (long)B * n;
+    const int unnorm = variant == ORC_UNNORMALISED;
+    double *Wfe0 = (double *)calloc((size_t)de * F, sizeof(double));
+    const double *Wfe = variant == ORC_LIGHT_EDGE ? Wfe0 : w->Wfe;
     const double rs = 1.0 / sqrt((double)dh);
     double *Q = (double *)malloc(sizeof(double) * rows * hd);
     double *K = (double *)malloc(sizeof(double) * rows * hd);
@@ -271,7 +311,7 @@ int orc_backward(const orc_dims *d, const double *X, const double *E, const doub
         double *dA = (double *)malloc(sizeof(double) * H * n);
         double *df = (double *)calloc((size_t)n * F, sizeof(double));
         double lse[64];
-        row_attention(d, E, M, Q, K, w->Wfe, g, b, i, arow, srow, frow, lse);
+        row_attention(d, E, M, Q, K, Wfe, g, b, i, arow, srow, frow, lse);
         for (int h = 0; h < H; ++h) LSE[r * H + h] = lse[h];
         for (int h = 0; h < H; ++h)
             for (int t = 0; t < dh; ++t) {
@@ -286,7 +326,8 @@ int orc_backward(const orc_dims *d, const double *X, const double *E, const doub
             for (int o = 0; o < dx; ++o) acc += dXout[r * dx + o] * w->Wo[(long)k * dx + o];
             dO[r * hd + k] = mi * acc;
         }
-        /* dA and D */
+        /* dA and D (the unnormalised variant: the node term only in dA and D, u added to dS') */
+        double *urow = (double *)malloc(sizeof(double) * n);
         for (int h = 0; h < H; ++h) {
             double D = 0.0;
             for (int j = 0; j < n; ++j) {
@@ -296,13 +337,14 @@ int orc_backward(const orc_dims *d, const double *X, const double *E, const doub
                 double dov = 0.0;
                 for (int t = 0; t < dh; ++t)
                     dov += dO[r * hd + h * dh + t] * V[((long)b * n + j) * hd + h * dh + t];
-                dA[(long)h * n + j] = dov + u;
+                urow[j] = (M[r] && M[(long)b * n + j]) ? u : 0.0;
+                dA[(long)h * n + j] = unnorm ? dov : dov + u;
                 D += arow[(long)h * n + j] * dA[(long)h * n + j];
             }
             Dst[r * H + h] = D;
             for (int j = 0; j < n; ++j) {
                 const double a = arow[(long)h * n + j];
-                const double dsp = a * (dA[(long)h * n + j] - D);
+                const double dsp = a * (dA[(long)h * n + j] - D) + (unnorm ? urow[j] : 0.0);
                 const double gam = frow[(long)j * F + h];
                 const double s = srow[(long)h * n + j];
                 df[(long)j * F + h] = dsp * s;          /* dgamma */
@@ -318,16 +360,24 @@ int orc_backward(const orc_dims *d, const double *X, const double *E, const doub
         double *pg = pWe + (long)H * de;
         for (int j = 0; j < n; ++j) {
             const long e0 = (((long)b * n + i) * n + j) * de;
+            const int valid = M[r] && M[(long)b * n + j];
             for (int c = 0; c < de; ++c) {
                 double acc = dEout[e0 + c];
-                for (int k = 0; k < F; ++k) acc += df[(long)j * F + k] * w->Wfe[(long)c * F + k];
+                for (int k = 0; k < F; ++k) acc += df[(long)j * F + k] * Wfe[(long)c * F + k];
                 dE[e0 + c] = acc;
                 for (int k = 0; k < F; ++k) pWfe[(long)c * F + k] += E[e0 + c] * df[(long)j * F + k];
-                for (int h = 0; h < H; ++h) pWe[(long)h * de + c] += arow[(long)h * n + j] * dEout[e0 + c];
+                for (int h = 0; h < H; ++h) {
+                    double coef = arow[(long)h * n + j];
+                    if (unnorm) {
+                        const double sp = srow[(long)h * n + j] * (1.0 + frow[(long)j * F + h]) + frow[(long)j * F + H + h];
+                        coef = valid ? sp : 0.0;
+                    }
+                    pWe[(long)h * de + c] += coef * dEout[e0 + c];
+                }
             }
             for (int k = 0; k < F; ++k) pg[k] += df[(long)j * F + k];
         }
-        free(arow); free(srow); free(frow); free(dA); free(df);
+        free(arow); free(srow); free(frow); free(dA); free(df); free(urow);
     }
 
     /* ---- column pass: dk_j, dv_j (recompute a_ij, dS'_ij over all i) ---- */
@@ -340,7 +390,7 @@ int orc_backward(const orc_dims *d, const double *X, const double *E, const doub
         for (int i = 0; i < n; ++i) {
             if (!mb[i]) continue;
             const long ri = (long)b * n + i;
-            film(d, E, w->Wfe, g, b, i, j, f);
+            film(d, E, Wfe, g, b, i, j, f);
             const double *dep = dEout + ((ri * n) + j) * de;
             for (int h = 0; h < H; ++h) {
                 const double s = raw_score(d, Q, K, b, h, i, j);
@@ -350,7 +400,7 @@ int orc_backward(const orc_dims *d, const double *X, const double *E, const doub
                 for (int c = 0; c < de; ++c) u += w->We[(long)h * de + c] * dep[c];
                 double dov = 0.0;
                 for (int t = 0; t < dh; ++t) dov += dO[ri * hd + h * dh + t] * V[r * hd + h * dh + t];
-                const double dsp = a * (dov + u - Dst[ri * H + h]);
+                const double dsp = unnorm ? a * (dov - Dst[ri * H + h]) + u : a * (dov + u - Dst[ri * H + h]);
                 const double ds = dsp * (1.0 + f[h]);
                 for (int t = 0; t < dh; ++t) {
                     dK[r * hd + h * dh + t] += ds * Q[ri * hd + h * dh + t] * rs;
@@ -418,7 +468,16 @@ int orc_backward(const orc_dims *d, const double *X, const double *E, const doub
             dX[r * dx + c] = acc;
         }
     /* padded / invalid pairs: dE = dE' was written by the row pass for every pair */
+    if (variant == ORC_LIGHT_EDGE) memset(gr->Wfe, 0, sizeof(double) * de * F);
     free(Q); free(K); free(V); free(g); free(O); free(dO); free(dQ); free(dK); free(dV);
-    free(Dst); free(LSE); free(parts); free(dg);
+    free(Dst); free(LSE); free(parts); free(dg); free(Wfe0);
     return 0;
+}
+
+int orc_backward(const orc_dims *d, const double *X, const double *E, const double *y,
+                 const unsigned char *M, const orc_weights *w,
+                 const double *dXout, const double *dEout,
+                 double *dX, double *dE, double *dy, orc_grads *gr)
+{
+    return orc_backward_variant(d, ORC_LAYER, X, E, y, M, w, dXout, dEout, dX, dE, dy, gr);
 }

@@ -26,20 +26,20 @@ MUTANTS = {
     "no_score_scale": ("return acc / sqrt((double)d->dh);", "return acc;"),
     "film_wrong_column": ("acc += e[c] * Wfe[(long)c * 2 * d->H + k];",
                           "acc += e[c] * Wfe[(long)c * 2 * d->H + (k + 1) % (2 * d->H)];"),
-    "edge_update_shifted_index": ("acc += arow[(long)h * n + j] * w->We[(long)h * de + c];",
-                                  "acc += arow[(long)h * n + (j + 1) % n] * w->We[(long)h * de + c];"),
+    "edge_update_shifted_index": ("double coef = arow[(long)h * n + j];\n                    if (variant == ORC_UNNORMALISED) {\n                        const double sp = srow[(long)h * n + j] * (1.0 + frow[(long)j * 2 * H + h]) +",
+                                  "double coef = arow[(long)h * n + (j + 1) % n];\n                    if (variant == ORC_UNNORMALISED) {\n                        const double sp = srow[(long)h * n + j] * (1.0 + frow[(long)j * 2 * H + h]) +"),
     "mask_rows_only": ("if (mb[j] && sp[j] > m) m = sp[j];", "if (sp[j] > m) m = sp[j];"),
     # backward
-    "dS_sign": ("const double dsp = a * (dA[(long)h * n + j] - D);",
-                "const double dsp = a * (dA[(long)h * n + j] + D);"),
-    "dE_missing_film_term": ("acc += df[(long)j * F + k] * w->Wfe[(long)c * F + k];",
+    "dS_sign": ("const double dsp = a * (dA[(long)h * n + j] - D)",
+                "const double dsp = a * (dA[(long)h * n + j] + D)"),
+    "dE_missing_film_term": ("acc += df[(long)j * F + k] * Wfe[(long)c * F + k];",
                              "acc += 0 * df[(long)j * F + k];"),
     "dq_without_film_factor": ("const double ds = dsp * (1.0 + gam);", "const double ds = dsp;"),
     "dk_without_film_factor": ("const double ds = dsp * (1.0 + f[h]);", "const double ds = dsp;"),
     "dv_transposed": ("dV[r * hd + h * dh + t] += a * dO[ri * hd + h * dh + t];",
                       "dV[r * hd + h * dh + t] += a * dO[r * hd + h * dh + t];"),
-    "dWe_wrong_operand": ("pWe[(long)h * de + c] += arow[(long)h * n + j] * dEout[e0 + c];",
-                          "pWe[(long)h * de + c] += arow[(long)h * n + j] * E[e0 + c];"),
+    "dWe_wrong_operand": ("pWe[(long)h * de + c] += coef * dEout[e0 + c];",
+                          "pWe[(long)h * de + c] += coef * E[e0 + c];"),
     "lse_without_log": ("lse[h] = valid ? m + log(l) : -INFINITY;", "lse[h] = valid ? m + l : -INFINITY;"),
     # node residual and output projection
     "out_proj_not_masked": ("Xout[r * dx + o] = X[r * dx + o] + (mi != 0.0 ? acc : 0.0);",
@@ -57,6 +57,20 @@ MUTANTS = {
     "dbf_missing": ("gr->bf[k] += dg[(long)b * F + k];", "gr->bf[k] += 0.0 * dg[(long)b * F + k];"),
     "dy_shifted_column": ("acc += dg[(long)b * F + k] * w->Wfy[(long)c * F + k];",
                           "acc += dg[(long)b * F + k] * w->Wfy[(long)c * F + (k + 1) % F];"),
+    # ablation variants (unnormalised edge update, Light Edge)
+    "unnormalised_update_uses_a": ("coef = valid ? sp : 0.0;\n                    }\n                    acc += coef",
+                                   "coef = arow[(long)h * n + j];\n                    }\n                    acc += coef"),
+    "unnormalised_update_unmasked": ("coef = valid ? sp : 0.0;\n                    }\n                    acc += coef",
+                                     "coef = sp;\n                    }\n                    acc += coef"),
+    "unnormalised_D_keeps_edge_term": ("dA[(long)h * n + j] = unnorm ? dov : dov + u;",
+                                       "dA[(long)h * n + j] = dov + u;"),
+    "unnormalised_row_dS_without_u": ("+ (unnorm ? urow[j] : 0.0);", "+ 0.0;"),
+    "unnormalised_column_dS_without_u": ("a * (dov - Dst[ri * H + h]) + u :", "a * (dov - Dst[ri * H + h]) :"),
+    "unnormalised_dWe_uses_a": ("coef = valid ? sp : 0.0;\n                    }\n                    pWe",
+                                "coef = arow[(long)h * n + j];\n                    }\n                    pWe"),
+    "light_edge_keeps_Wfe": ("const double *Wfe = variant == ORC_LIGHT_EDGE ? Wfe0 : w->Wfe;\n    double *Q",
+                             "const double *Wfe = w->Wfe;\n    double *Q"),
+    "light_edge_dWfe_not_zeroed": ("if (variant == ORC_LIGHT_EDGE) memset(gr->Wfe", "if (0) memset(gr->Wfe"),
     "dX_without_dK_term": ("for (int p = 0; p < 3; ++p)\n                for (int k = 0; k < hd; ++k) acc += dN[p]",
                            "for (int p = 0; p < 3; p += 2)\n                for (int k = 0; k < hd; ++k) acc += dN[p]"),
 }

@@ -386,3 +386,135 @@ def test_masked_gradients_are_residual_only(oracle_lib):
     valid = valid_mask(d["M"])
     np.testing.assert_array_equal(g["dX"][~rows], d["dXout"][~rows])
     np.testing.assert_array_equal(g["dE"][~valid], d["dEout"][~valid])
+
+
+# --------------------------------------------------------------- ablation variants
+# AI-summary page, method paragraph (the ablation of unnormalised coefficients)
+# and its "Light Edge" bullet (no per-edge modulation).  Readings:
+#   unnormalised: E' = E + sum_h s'^h We[h,:] on valid pairs, s' the modulated
+#                 score (the coefficients before the softmax); nodes as the layer;
+#   light edge:   gamma, beta from y alone (Wfe absent, its gradient zero).
+
+
+def test_unnormalised_closed_form(oracle_lib):
+    """gamma = -1 and beta = c_h: every modulated score equals c_h, so the
+    unnormalised edge update adds sum_h c_h We[h] to each valid pair; node
+    outputs stay those of uniform attention."""
+    p, dims, d, W = tiny(seed=3)
+    c = np.array([0.7, -1.3], dtype=np.float32)[: p.H]
+    W = zero_film(W, p.H, gamma=-1.0)
+    W["bf"] = np.concatenate([np.full(p.H, -1.0), c]).astype(np.float32)
+    out = oracle_lib.forward(dims, d["X"], d["E"], d["y"], d["M"], W, variant="unnormalised")
+    lay = oracle_lib.forward(dims, d["X"], d["E"], d["y"], d["M"], W)
+    valid = valid_mask(d["M"])
+    shift = (c.astype(np.float64)[:, None] * W["We"].astype(np.float64)).sum(0)      # [de]
+    E = d["E"].astype(np.float64)
+    np.testing.assert_allclose(out["Eout"][valid], (E + shift)[valid], rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(out["Eout"][~valid], E[~valid])
+    for k in ("Xout", "O"):
+        np.testing.assert_array_equal(out[k], lay[k])
+
+
+def test_unnormalised_brute_force(oracle_lib):
+    """Per-pair pure-Python modulated scores and the edge update they give."""
+    p, dims, d, W = tiny()
+    out = oracle_lib.forward(dims, d["X"], d["E"], d["y"], d["M"], W, variant="unnormalised")
+    H, dh, de = p.H, p.dh, p.de
+    Wd = {k: W[k].astype(float).tolist() for k in WN}
+    Eref = d["E"].astype(np.float64).copy()
+    for b in range(p.B):
+        X = d["X"][b].tolist()
+        y = d["y"][b].tolist()
+        lin = lambda x, Wm, bm: [sum(x[k] * Wm[k][o] for k in range(len(x))) + bm[o] for o in range(len(bm))]
+        q = [lin(X[i], Wd["Wq"], Wd["bq"]) for i in range(p.n)]
+        k_ = [lin(X[i], Wd["Wk"], Wd["bk"]) for i in range(p.n)]
+        gy = lin(y, Wd["Wfy"], Wd["bf"])
+        for i in range(p.n):
+            for j in range(p.n):
+                if not (d["M"][b, i] and d["M"][b, j]):
+                    continue
+                e = d["E"][b, i, j].tolist()
+                for h in range(H):
+                    gam = sum(e[c] * Wd["Wfe"][c][h] for c in range(de)) + gy[h]
+                    bet = sum(e[c] * Wd["Wfe"][c][H + h] for c in range(de)) + gy[H + h]
+                    s = sum(q[i][h * dh + t] * k_[j][h * dh + t] for t in range(dh)) / math.sqrt(dh)
+                    sp = s * (1 + gam) + bet
+                    for c in range(de):
+                        Eref[b, i, j, c] += sp * Wd["We"][h][c]
+    np.testing.assert_allclose(out["Eout"], Eref, rtol=1e-12, atol=1e-12)
+
+
+def test_unnormalised_backward_closed_forms(oracle_lib):
+    """gamma = -1, beta = c_h: ds vanishes (no Q, K gradient); the edge path
+    reaches beta directly, so dbf[H+h] = sum over valid pairs of We[h] . dE'
+    (the softmax alone would give zero) and dWe[h] = c_h times the sum of dE'
+    over valid pairs; dE = dE'."""
+    p, dims, d, W = tiny(seed=4)
+    c = np.array([0.5, -2.0], dtype=np.float32)[: p.H]
+    W = zero_film(W, p.H, gamma=-1.0)
+    W["bf"] = np.concatenate([np.full(p.H, -1.0), c]).astype(np.float32)
+    g = oracle_lib.backward(dims, d["X"], d["E"], d["y"], d["M"], W, d["dXout"], d["dEout"], variant="unnormalised")
+    for k in ("dWq", "dbq", "dWk", "dbk"):
+        assert np.abs(g[k]).max() <= 1e-13, k
+    valid = valid_mask(d["M"])
+    sum_dE = d["dEout"].astype(np.float64)[valid].sum(0)                               # [de]
+    We = W["We"].astype(np.float64)
+    np.testing.assert_allclose(g["dbf"][p.H:], We @ sum_dE, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(g["dWe"], c.astype(np.float64)[:, None] * sum_dE[None, :], rtol=0, atol=1e-11)
+    np.testing.assert_array_equal(g["dE"], d["dEout"].astype(np.float64))
+
+
+def test_variant_backward_finite_differences(oracle_lib):
+    """Every gradient of both variants against fp64 central differences of their forward."""
+    p, dims, d, W = tiny(seed=9)
+    X, E, y = (d[k].astype(np.float64) for k in ("X", "E", "y"))
+    Wd = {k: W[k].astype(np.float64) for k in WN}
+    dXo, dEo = d["dXout"].astype(np.float64), d["dEout"].astype(np.float64)
+    h = 1e-6
+    rng = np.random.default_rng(12)
+    for variant in ("unnormalised", "light_edge"):
+        g = oracle_lib.backward(dims, X, E, y, d["M"], Wd, dXo, dEo, variant=variant)
+
+        def L(X=X, E=E, y=y, W=Wd):
+            o = oracle_lib.forward(dims, X, E, y, d["M"], W, variant=variant)
+            return float((o["Xout"] * dXo).sum() + (o["Eout"] * dEo).sum())
+
+        def check(name, arr, setter, grad, max_entries=None):
+            idx = np.arange(arr.size)
+            if max_entries and arr.size > max_entries:
+                idx = rng.choice(arr.size, max_entries, replace=False)
+            fd = np.empty(len(idx))
+            for t, flat in enumerate(idx):
+                plus = arr.copy().reshape(-1); plus[flat] += h
+                minus = arr.copy().reshape(-1); minus[flat] -= h
+                fd[t] = (setter(plus.reshape(arr.shape)) - setter(minus.reshape(arr.shape))) / (2 * h)
+            an = grad.reshape(-1)[idx]
+            # relative 1e-6, plus an absolute 1e-7 for the difference quotients'
+            # own rounding (a gradient that is exactly zero, as dbk of Light Edge)
+            assert np.abs(fd - an).max() <= 1e-6 * np.abs(an).max() + 1e-7, f"{variant} {name}"
+
+        check("X", X, lambda a: L(X=a), g["dX"])
+        check("E", E, lambda a: L(E=a), g["dE"], max_entries=400)
+        check("y", y, lambda a: L(y=a), g["dy"])
+        for k in WN:
+            if variant == "light_edge" and k == "Wfe":
+                continue                       # not a parameter of that layer
+            def setk(a, k=k):
+                W2 = dict(Wd); W2[k] = a
+                return L(W=W2)
+            check(k, Wd[k], setk, g["d" + k], max_entries=150)
+
+
+def test_light_edge_variant_ignores_wfe(oracle_lib):
+    """Light Edge ignores Wfe: equal to the layer at Wfe = 0 (pinned above
+    against scaled dot-product attention), its dWfe is zero and dE = dE'."""
+    p, dims, d, W = tiny(seed=6)
+    W0 = dict(W)
+    W0["Wfe"] = np.zeros_like(W["Wfe"])
+    lv = oracle_lib.forward(dims, d["X"], d["E"], d["y"], d["M"], W, variant="light_edge")
+    l0 = oracle_lib.forward(dims, d["X"], d["E"], d["y"], d["M"], W0)
+    for k in ("Xout", "Eout", "O", "LSE"):
+        np.testing.assert_array_equal(lv[k], l0[k])
+    gv = oracle_lib.backward(dims, d["X"], d["E"], d["y"], d["M"], W, d["dXout"], d["dEout"], variant="light_edge")
+    assert np.all(gv["dWfe"] == 0)
+    np.testing.assert_array_equal(gv["dE"], d["dEout"].astype(np.float64))
