@@ -190,8 +190,8 @@ def run_ours(args):
     flat_dw = buf.dW_flat
 
     def layer(s):
-        buf.forward(s)
-        buf.backward(s)
+        buf.forward(s, variant=args.variant)
+        buf.backward(s, variant=args.variant)
 
     def step():
         layer(torch.cuda.current_stream())
@@ -293,7 +293,8 @@ def run_ours(args):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded SBM-shaped graphs; edge_aware_graph_b200/inputs.py)",
-        "config": {"workload": DESCRIBE[WORKLOAD],
+        "config": {"workload": DESCRIBE[WORKLOAD] + ("" if args.variant == "layer" else
+                                                     f"; ablation variant: {args.variant}"),
                    "global_batch": p.B * world, "seq_len": p.n, "parallelism": f"dp{world}",
                    "l2": f"inputs larger than L2 (E, dE' {p.B * p.n * p.n * p.de * 2 / 2**20:.0f} MiB each; "
                          "E', dE written each step)",
@@ -320,8 +321,8 @@ def run_ours(args):
     if world == 1 and not args.no_cpu_baseline:
         graphs = min(args.cpu_graphs, p.B) if WORKLOAD == "sbm" else 1
         reps = args.cpu_reps if WORKLOAD == "sbm" else 1
-        out["cpu_baseline"] = cpu_baseline(p, d, W, graphs, reps)
-        out["cpu_baseline_1thread"] = cpu_baseline(p, d, W, 1, 1, threads=1)
+        out["cpu_baseline"] = cpu_baseline(p, d, W, graphs, reps, variant=args.variant)
+        out["cpu_baseline_1thread"] = cpu_baseline(p, d, W, 1, 1, threads=1, variant=args.variant)
     return out
 
 
@@ -530,7 +531,7 @@ def run_e2e(args, buf, d, stream, step):
 # ------------------------------------------------------------------ oracle arm
 
 
-def cpu_baseline(p, d, W, graphs, reps=1, threads=None):
+def cpu_baseline(p, d, W, graphs, reps=1, threads=None, variant="layer"):
     """The fp64 oracle, as it stands, on a bounded sample: the first `graphs`
     graphs of the batch, forward + backward, `reps` times, on all usable host
     cores (or on `threads` threads)."""
@@ -541,8 +542,8 @@ def cpu_baseline(p, d, W, graphs, reps=1, threads=None):
     dims = dict(H=p.H, dh=p.dh)
     t = time.perf_counter()
     for _ in range(reps):
-        oracle.forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W)
-        oracle.backward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, sl["dXout"], sl["dEout"])
+        oracle.forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, variant=variant)
+        oracle.backward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, sl["dXout"], sl["dEout"], variant=variant)
     dt = time.perf_counter() - t
     cores = oracle.threads_used()
     oracle.set_threads(None)
@@ -650,6 +651,8 @@ def main():
     ap.add_argument("--workload", default="sbm-train", choices=list(WORKLOADS),
                     help="sbm-train: the training step (default); planar-sample / tree-sample: the "
                          "sampling-time forward on Planar- / Tree-shaped batches")
+    ap.add_argument("--variant", default="layer", choices=["layer", "light_edge", "unnormalised"],
+                    help="training workloads: the layer (default) or one of its ablation variants")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="sampling workloads: seconds of oracle forward calls in cpu_baseline")
     args = ap.parse_args()

@@ -72,13 +72,13 @@ class LayerBuffers:
 
     # ------------------------------------------------------------ calls
 
-    def forward(self, stream=None, saved=True):
+    def forward(self, stream=None, saved=True, variant="layer"):
         eaga.forward(self.dims, self.X, self.E, self.y, self.M, self.W, self.Xout, self.Eout,
-                     self.saved if saved else None, self.ws_fwd, stream)
+                     self.saved if saved else None, self.ws_fwd, stream, variant=variant)
 
-    def backward(self, stream=None):
+    def backward(self, stream=None, variant="layer"):
         eaga.backward(self.dims, self.X, self.E, self.y, self.M, self.W, self.saved, self.dXout, self.dEout,
-                      self.dX, self.dE, self.dy, self.dW, self.ws_bwd, stream)
+                      self.dX, self.dE, self.dy, self.dW, self.ws_bwd, stream, variant=variant)
 
     def attention_map(self, stream=None):
         B, n, H = self.shape["B"], self.shape["n"], self.shape["H"]

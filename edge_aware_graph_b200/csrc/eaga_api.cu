@@ -53,7 +53,8 @@ extern "C" {
 size_t eaga_workspace_size(const eaga_dims *d, int for_backward) {
     if (check_dims(d) != EAGA_OK) return 0;
     const WsLayout W = ws_layout(*d);
-    if (fast::supports(*d)) return fast::workspace_size(*d, for_backward, W.total_fwd, W.fwd_saved);
+    if (for_backward ? fast::supports_backward(*d) : fast::supports(*d))
+        return fast::workspace_size(*d, for_backward, W.total_fwd, W.fwd_saved);
     return for_backward ? W.total_bwd : W.total_fwd;
 }
 
@@ -68,12 +69,17 @@ struct NvtxRange {
     ~NvtxRange() { nvtxRangePop(); }
 };
 
-eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
-                         const eaga_weights *w, void *Xout, void *Eout, void *saved, void *workspace,
-                         size_t ws_bytes, void *stream) {
+static bool known_variant(int v) {
+    return v == EAGA_VARIANT_LAYER || v == EAGA_VARIANT_LIGHT_EDGE || v == EAGA_VARIANT_UNNORMALISED;
+}
+
+eaga_status eaga_forward_variant(const eaga_dims *d, int variant, const void *X, const void *E, const void *y,
+                                 const uint8_t *M, const eaga_weights *w, void *Xout, void *Eout, void *saved,
+                                 void *workspace, size_t ws_bytes, void *stream) {
     NvtxRange range("eaga_forward");
     eaga_status s = check_dims(d);
     if (s != EAGA_OK) return s;
+    if (!known_variant(variant)) return EAGA_ERR_INVALID_ARG;
     if ((s = check_weights(w)) != EAGA_OK) return s;
     if ((s = check_ptrs({X, E, y, M, Xout, Eout, workspace})) != EAGA_OK) return s;
     if (saved && !aligned16(saved)) return EAGA_ERR_MISALIGNED;
@@ -94,6 +100,7 @@ eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const
     char *ws = static_cast<char *>(workspace);
     char *sv = saved ? static_cast<char *>(saved) : ws + W.fwd_saved;
     FwdArgs a;
+    a.variant = variant;
     a.X = X; a.E = E; a.y = y; a.M = M;
     weight_array(w, a.w);
     a.Xout = Xout; a.Eout = Eout;
@@ -108,13 +115,21 @@ eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const
     return launch_status(generic::forward(*d, a, st));
 }
 
-eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
-                          const eaga_weights *w, const void *saved, const void *dXout, const void *dEout,
-                          void *dX, void *dE, void *dy, const eaga_weight_grads *dW, void *workspace,
-                          size_t ws_bytes, void *stream) {
+eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
+                         const eaga_weights *w, void *Xout, void *Eout, void *saved, void *workspace,
+                         size_t ws_bytes, void *stream) {
+    return eaga_forward_variant(d, EAGA_VARIANT_LAYER, X, E, y, M, w, Xout, Eout, saved, workspace, ws_bytes,
+                                stream);
+}
+
+eaga_status eaga_backward_variant(const eaga_dims *d, int variant, const void *X, const void *E, const void *y,
+                                  const uint8_t *M, const eaga_weights *w, const void *saved, const void *dXout,
+                                  const void *dEout, void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
+                                  void *workspace, size_t ws_bytes, void *stream) {
     NvtxRange range("eaga_backward");
     eaga_status s = check_dims(d);
     if (s != EAGA_OK) return s;
+    if (!known_variant(variant)) return EAGA_ERR_INVALID_ARG;
     if ((s = check_weights(w)) != EAGA_OK) return s;
     if ((s = check_ptrs({X, E, y, M, saved, dXout, dEout, dX, dE, dy, workspace})) != EAGA_OK) return s;
     if (!dW) return EAGA_ERR_INVALID_ARG;
@@ -140,6 +155,7 @@ eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, cons
     char *ws = static_cast<char *>(workspace);
     const char *sv = static_cast<const char *>(saved);
     BwdArgs a;
+    a.variant = variant;
     a.X = X; a.E = E; a.y = y; a.M = M;
     weight_array(w, a.w);
     a.Q = sv + L.q; a.K = sv + L.k; a.V = sv + L.v; a.O = sv + L.o;
@@ -159,10 +175,18 @@ eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, cons
     a.part_stride = W.part_stride;
     a.status = reinterpret_cast<int *>(ws + W.status);
     if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
-    if (fast::supports(*d)) {
+    if (fast::supports_backward(*d)) {
         return launch_status(fast::backward(*d, a, ws, W.fwd_saved, st));
     }
     return launch_status(generic::backward(*d, a, st));
+}
+
+eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
+                          const eaga_weights *w, const void *saved, const void *dXout, const void *dEout,
+                          void *dX, void *dE, void *dy, const eaga_weight_grads *dW, void *workspace,
+                          size_t ws_bytes, void *stream) {
+    return eaga_backward_variant(d, EAGA_VARIANT_LAYER, X, E, y, M, w, saved, dXout, dEout, dX, dE, dy, dW,
+                                 workspace, ws_bytes, stream);
 }
 
 eaga_status eaga_debug_attention_map(const eaga_dims *d, const void *E, const uint8_t *M, const eaga_weights *w,
@@ -253,7 +277,7 @@ eaga_status eaga_set_profile_events(int point, void *before, void *after) {
 
 int eaga_kernel_launches(const eaga_dims *d, int for_backward) {
     if (check_dims(d) != EAGA_OK) return -1;
-    if (fast::supports(*d)) return fast::kernel_launches(*d, for_backward);
+    if (for_backward ? fast::supports_backward(*d) : fast::supports(*d)) return fast::kernel_launches(*d, for_backward);
     return generic::kernel_launches(*d, for_backward);
 }
 

@@ -8,7 +8,7 @@ namespace eaga {
 namespace fast {
 
 cudaError_t launch_prologue(const eaga_dims &d, const void *const w[12], const void *y, float *g, uint8_t *img,
-                            cudaStream_t st);
+                            int *zero, int nzero, cudaStream_t st);
 cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A[3], const void *const B[3],
                     const void *const bias[3], void *const C[3], int Nb, const void *R, const uint8_t *mask,
                     int *status, cudaStream_t st, bool b_mn);
@@ -27,18 +27,23 @@ bool supports(const eaga_dims &d) {
            d.n <= 1024 && d.dx % 64 == 0 && d.dx >= 64;
 }
 
+// The backward pair kernel's CTAs of one graph wait for each other (bounded),
+// so the device must hold the row blocks of one graph at once, one CTA per SM.
+bool supports_backward(const eaga_dims &d) { return supports(d) && sm_count() >= (d.n + TB - 1) / TB; }
+
 // Forward: the small operand images after the common workspace; backward:
 // the whole FastWs.
 size_t forward_scratch_bytes(const eaga_dims &) { return align256(IMG_BYTES); }
 size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, size_t common_head) {
+    // (callers check supports(d), and supports_backward(d) for the backward)
     if (!for_backward) return align256(common_fwd + IMG_BYTES);
     return fast_ws(d, common_head).total;
 }
 
 int kernel_launches(const eaga_dims &, int for_backward) {
     // forward: prologue, QKV, pairs, out-proj
-    // backward: prologue, dO, row pairs, dk/dv, dX, wgrad x2, bias partial, rparts partial, finish, film grads
-    return for_backward ? 11 : 4;
+    // backward: prologue, dO, pairs, dX, wgrad x2, bias partial, rparts partial, finish, film grads
+    return for_backward ? 10 : 4;
 }
 
 #define FAST_TRY(x)                               \
@@ -50,7 +55,7 @@ int kernel_launches(const eaga_dims &, int for_backward) {
 cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st) {
     uint8_t *img = reinterpret_cast<uint8_t *>(ws_after_common);
     const int rows = d.B * d.n;
-    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, st));
+    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, st));
     {   // [Q|K|V] = X [Wq|Wk|Wv] + b
         const void *A[3] = {a.X, a.X, a.X}, *B[3] = {a.w[0], a.w[2], a.w[4]};
         const void *bias[3] = {a.w[1], a.w[3], a.w[5]};
@@ -130,7 +135,7 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         void *C[3] = {dO, dO, dO};
         FAST_TRY(tc_gemm(2, rows, HD, d.dx, 1, A, Bt, nullptr, C, HD, nullptr, a.M, a.status, s1, false));
     }
-    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, st));
+    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, reinterpret_cast<int *>(ws + W.flags), W.n_rparts + 1, st));
     FAST_TRY(stream_after(st, s1, ev[1]));
 
     prof_mark(1, 0, st);

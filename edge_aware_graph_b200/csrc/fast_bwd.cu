@@ -1,11 +1,8 @@
-// Backward kernels of the specialised path (de = 64, H = 8, dh = 32, bf16
-// storage) besides the row pair kernel (fast_bwd_stream.cu):
-//   k_bwd_kv:   dk_j = sum_i ds_ij q_i / sqrt(dh) and dv_j = sum_i a_ij dO_i
-//               from the a and ds the row kernel stored (warp MMAs fed by a
-//               TMA pipeline), so E and dE' are read only once;
-//   reductions: bias gradients, the per-(graph, row block) dWfe / dWe / dg
-//               partials, the split-K weight-gradient partials, and the global
-//               FiLM term's dWfy, dbf, dy; all in a fixed order.
+// Backward reductions of the specialised path (de = 64, H = 8, dh = 32, bf16
+// storage), after the pair kernel (fast_bwd_stream.cu): bias gradients, the
+// per-(graph, row block) dWfe / dWe / dg partials, the split-K
+// weight-gradient partials, and the global FiLM term's dWfy, dbf, dy; all in
+// a fixed order.
 #include <math.h>
 #include "fast.h"
 #include "fast_common.cuh"
@@ -15,116 +12,6 @@ namespace fast {
 
 using namespace sm100;
 using namespace dev;
-
-struct BwdKvParams {
-    __nv_bfloat16 *dK, *dV;  // [B,n,256] out (dK scaled)
-    int *status;
-    int n;
-};
-
-// ---------------------------------------------------------------- dk, dv pass
-// dk_j = sum_i ds_ij q_i / sqrt(dh) and dv_j = sum_i a_ij dO_i from the a and
-// ds the row kernel stored.  CTA = (32 columns j, graph), warp = head; each
-// pipeline stage brings 16 rows i of a, ds (all heads), Q and dO with TMA and
-// every warp adds their products on warp MMAs (M = j, N = d, K = i).
-constexpr int KV_J = 32, KV_I = 16, KV_STAGES = 3, KV_THR = 256;
-struct KvSmem {
-    static constexpr uint32_t PDS = 0, PA = 8192, QT = 16384, DOT = 24576, STAGE = 32768;
-    static constexpr uint32_t BAR = KV_STAGES * STAGE;            // full[S], empty[S]
-    static constexpr uint32_t BYTES = BAR + 2 * KV_STAGES * 8 + 1024;
-};
-
-__global__ void __launch_bounds__(KV_THR, 2)
-k_bwd_kv(const __grid_constant__ CUtensorMap tmPds, const __grid_constant__ CUtensorMap tmPa,
-         const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO, BwdKvParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const int tid = threadIdx.x, h = tid >> 5, t = tid & 31, g8 = t >> 2, c4 = t & 3;
-    const int n = p.n, j0 = blockIdx.x * KV_J, b = blockIdx.y;
-    const int nsteps = (n + KV_I - 1) / KV_I;
-    const uint32_t bar0 = sbase + KvSmem::BAR;
-    auto full = [&](int s) { return bar0 + 8 * s; };
-    auto empty = [&](int s) { return bar0 + 8 * (KV_STAGES + s); };
-    auto issue = [&](int k) {
-        const int s = k % KV_STAGES, i0 = k * KV_I;
-        const uint32_t st = sbase + s * KvSmem::STAGE;
-        mbar_expect_tx(full(s), KvSmem::STAGE);
-        tma_load_4d(st + KvSmem::PDS, &tmPds, full(s), j0, i0, 0, b);
-        tma_load_4d(st + KvSmem::PA, &tmPa, full(s), j0, i0, 0, b);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            tma_load_3d(st + KvSmem::QT + c * 2048, &tmQ, full(s), 64 * c, i0, b);
-            tma_load_3d(st + KvSmem::DOT + c * 2048, &tmDO, full(s), 64 * c, i0, b);
-        }
-    };
-    if (tid == 0) {
-        for (int s = 0; s < KV_STAGES; ++s) {
-            mbar_init(full(s), 1);
-            mbar_init(empty(s), KV_THR / 32);
-        }
-        fence_mbar_init();
-        for (int k = 0; k < KV_STAGES && k < nsteps; ++k) issue(k);
-    }
-    __syncthreads();
-
-    float kacc[2][4][4], vacc[2][4][4];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int x = 0; x < 4; ++x) kacc[mt][nt][x] = vacc[mt][nt][x] = 0.f;
-    // ldmatrix lanes: A = P^T (stored [i][j]) and B = Q, dO (stored [i][d]), both transposed loads
-    const int arow = (t & 7) + ((t >> 4) & 1) * 8, ach = (t >> 3) & 1;
-    const int brow = (t & 7) + ((t >> 3) & 1) * 8, bch = t >> 4;
-    for (int k = 0; k < nsteps; ++k) {
-        const int s = k % KV_STAGES;
-        const uint32_t ph = (k / KV_STAGES) & 1;
-        if (!mbar_wait(full(s), ph)) flag_timeout(p.status);
-        const uint32_t st = sbase + s * KvSmem::STAGE;
-        uint32_t bq[2][4], bo[2][4];
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-            const uint32_t off = (h >> 1) * 2048 + sw128(brow, (h & 1) * 4 + 2 * np + bch);
-            ldsm_x4_t(st + KvSmem::QT + off, bq[np]);
-            ldsm_x4_t(st + KvSmem::DOT + off, bo[np]);
-        }
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-            const uint32_t off = h * 1024 + sw64(arow, 2 * mt + ach);
-            uint32_t ad[4], aa[4];
-            ldsm_x4_t(st + KvSmem::PDS + off, ad);
-            ldsm_x4_t(st + KvSmem::PA + off, aa);
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                mma16816(kacc[mt][nt], ad, bq[nt >> 1][2 * (nt & 1)], bq[nt >> 1][2 * (nt & 1) + 1]);
-                mma16816(vacc[mt][nt], aa, bo[nt >> 1][2 * (nt & 1)], bo[nt >> 1][2 * (nt & 1) + 1]);
-            }
-        }
-        __syncwarp();
-        if (t == 0) mbar_arrive(empty(s));
-        if (tid == 0 && k + KV_STAGES < nsteps) {
-            if (!mbar_wait(empty(s), ph)) flag_timeout(p.status);
-            issue(k + KV_STAGES);
-        }
-        __syncwarp();
-    }
-    const float rs = rsqrtf((float)DH);
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const int j = j0 + 16 * mt + 8 * hf + g8;
-            if (j >= n) continue;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const size_t o = ((size_t)b * n + j) * HD + h * DH + nt * 8 + 2 * c4;
-                *reinterpret_cast<uint32_t *>(p.dK + o) =
-                    pack_bf16(kacc[mt][nt][2 * hf] * rs, kacc[mt][nt][2 * hf + 1] * rs);
-                *reinterpret_cast<uint32_t *>(p.dV + o) = pack_bf16(vacc[mt][nt][2 * hf], vacc[mt][nt][2 * hf + 1]);
-            }
-        }
-}
 
 // ---------------------------------------------------------------- reductions
 // All sums run in a fixed order (deterministic): first over segments of rows
@@ -206,7 +93,7 @@ struct DWPtrs {
 __global__ void k_bwd_finish(const float *wparts, int wsplits, const float *bparts, int bsplits,
                              const float *r2, int rsplits, const float *rparts, int ctas_per_graph, int B, int dx,
                              int dy, const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy, DWPtrs dW,
-                             __nv_bfloat16 *dyo, float *dg) {
+                             __nv_bfloat16 *dyo, float *dg, int zero_wfe) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const int msz = dx * HD;
     const int ncol = 3 * HD + dx;
@@ -227,7 +114,8 @@ __global__ void k_bwd_finish(const float *wparts, int wsplits, const float *bpar
     x -= ncol;
     if (x < NE) {
         const float acc = strided_sum(r2 + x, rsplits, NE);
-        if (x < DE * NF) dW.p[6][x] = acc; else dW.p[9][x - DE * NF] = acc;
+        // (Light Edge: Wfe is not a parameter, its gradient is zero)
+        if (x < DE * NF) dW.p[6][x] = zero_wfe ? 0.f : acc; else dW.p[9][x - DE * NF] = acc;
         return;
     }
     x -= NE;
@@ -263,29 +151,13 @@ __global__ void k_film_grads(const float *dg, int B, int dy, const __nv_bfloat16
 cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                               cudaStream_t st);
 
-// Row pair kernel, then dk / dv from its a and ds.
+// The backward pair kernel (profile point 2 brackets it alone).
 cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                              cudaStream_t st) {
-    static std::atomic<uint32_t> attr_set{0};
-    if (cudaError_t e = ensure_smem_attr(k_bwd_kv, KvSmem::BYTES, attr_set); e != cudaSuccess) return e;
     prof_mark(2, 0, st);
-    {
-        cudaError_t e = launch_bwd_stream(d, a, W, ws, g, st);
-        if (e != cudaSuccess) return e;
-    }
+    const cudaError_t e = launch_bwd_stream(d, a, W, ws, g, st);
     prof_mark(2, 1, st);
-    CUtensorMap mPds, mPa, mQ, mDO;
-    const __nv_bfloat16 *dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
-    if (!encode_p_map(&mPds, ws + W.Pds, d.B, d.n, W.npad) || !encode_p_map(&mPa, ws + W.Pa, d.B, d.n, W.npad) ||
-        !encode_node_map(&mQ, a.Q, d.B, d.n, KV_I) || !encode_node_map(&mDO, dO, d.B, d.n, KV_I))
-        return cudaErrorInvalidValue;
-    BwdKvParams p;
-    p.dK = reinterpret_cast<__nv_bfloat16 *>(ws + W.dK);
-    p.dV = reinterpret_cast<__nv_bfloat16 *>(ws + W.dV);
-    p.status = a.status;
-    p.n = d.n;
-    k_bwd_kv<<<dim3((d.n + KV_J - 1) / KV_J, d.B), KV_THR, KvSmem::BYTES, st>>>(mPds, mPa, mQ, mDO, p);
-    return cudaGetLastError();
+    return e;
 }
 
 // Column sums for the bias gradients and the first level of the row-block
@@ -321,7 +193,7 @@ cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs 
         W.bsplits, reinterpret_cast<const float *>(ws + W.r2), W.rsplits,
         reinterpret_cast<const float *>(ws + W.rparts), cpg, d.B, d.dx, d.dy,
         static_cast<const __nv_bfloat16 *>(a.y), static_cast<const __nv_bfloat16 *>(a.w[7]), dWdev,
-        static_cast<__nv_bfloat16 *>(a.dy), dg);
+        static_cast<__nv_bfloat16 *>(a.dy), dg, a.variant == EAGA_VARIANT_LIGHT_EDGE);
     const int tf = NF + d.dy * NF + d.B * d.dy;
     k_film_grads<<<(tf + 255) / 256, 256, 0, st>>>(dg, d.B, d.dy, static_cast<const __nv_bfloat16 *>(a.y),
                                                    static_cast<const __nv_bfloat16 *>(a.w[7]), a.dW[8], a.dW[7],

@@ -1,37 +1,53 @@
-// Backward row pair kernel for de = 64, H = 8, dh = 32, bf16 storage (sm_100a).
+// Backward pair kernel for de = 64, H = 8, dh = 32, bf16 storage (sm_100a).
 //
 // Chain rule of the layer (formulas as in the forward, differentiated):
 //   u_ij^h = We[h,:] . dE'_ij          dA^h_ij = dO_ih . v_jh + u_ij^h
 //   D_ih   = sum_j a_ij dA_ij          dS'_ij  = a_ij (dA_ij - D_ih)
 //   dgamma = dS' s,  dbeta = dS',  ds = dS' (1 + gamma)
-//   dq_i = sum_j ds_ij k_j / sqrt(dh)
+//   dq_i = sum_j ds_ij k_j / sqrt(dh),  dk_j = sum_i ds_ij q_i / sqrt(dh),  dv_j = sum_i a_ij dO_i
 //   dE = dE' + [dgamma|dbeta] Wfe^T,  dWfe = sum E^T [dgamma|dbeta],  dWe = sum a^T dE',  dg = sum [dgamma|dbeta]
 // with a_ij = exp(s'_ij - LSE_i) from the forward's saved row statistics.
 //
-// One CTA owns 8 query rows i of one graph and streams the columns j of those
-// rows in chunks of 32 (256 pairs: two 16 KB E tiles, two 16 KB dE' tiles,
-// the 16 KB K and V chunks), twice, because D needs a whole row before any
-// dS' exists:
-//   pass 1: FiLM f = E Wfe and u = dE' We^T on the tensor cores (tcgen05,
-//           fp32 in TMEM), S = Q K^T and dP = dO V^T on warp MMAs, a, dA,
-//           and a running D per thread; S and dP stay in TMEM for pass 2
-//           (32 columns per chunk, n <= 256; larger n reloads K and V);
-//   pass 2: f and u again (E and dE' come back from L2: the chunks are walked
-//           in reverse), dS', dgamma, dbeta, ds; dE = dE' + df Wfe^T on the
-//           tensor cores, in place in shared memory, stored with TMA;
-//           dWfe += E^T df and dWe^T += dE'^T a on the tensor cores too
-//           (M = 64 channels, MN-major operands straight from the tiles,
-//           accumulated in TMEM over the row block); dq += ds K (warp MMAs);
-//           and a, ds of every pair stored in bf16 for the dk / dv kernel.
-// E and dE' leave HBM once, dE is written once.  No CTA waits for another.
+// One CTA owns the 8 nodes of one row block of one graph and makes three
+// passes over 32-wide chunks (256 pairs: two 16 KB E tiles, two 16 KB dE'
+// tiles and two 16 KB node chunks each):
+//   pass 1 (its rows i, all columns j): FiLM f = E Wfe and u = dE' We^T on the
+//           tensor cores (tcgen05, fp32 in TMEM), S = Q K^T and dP = dO V^T
+//           on warp MMAs, a, dA and a running D per thread; S and dP stay in
+//           TMEM for pass 2 (32 columns per chunk, n <= 224; larger n reloads
+//           K and V).  At its end the CTA publishes D of its rows (global
+//           memory, then a release flag per row block).
+//   pass 2 (its rows, the chunks in reverse so that E and dE' come back from
+//           L2): dS', dgamma, dbeta, ds; dE = dE' + df Wfe^T on the tensor
+//           cores, in place in shared memory, stored with TMA; dWfe += E^T df
+//           and dWe^T += dE'^T a on the tensor cores (MN-major operands
+//           straight from the tiles, accumulated in TMEM over the row block);
+//           dq += ds K (warp MMAs).
+//   pass 3 (its nodes as the columns j, all rows i): the column tiles of E and
+//           dE' (pairs (i, j) with j among the CTA's 8 nodes), FiLM and u
+//           again, S and dP against the chunk's Q and dO rows, a and ds from
+//           LSE_i and the D_i the other CTAs of the graph published, then
+//           dk += ds^T Q and dv += a^T dO on warp MMAs.
+// E and dE' leave HBM once in passes 1 and 2, dE is written once; pass 3
+// reads the column tiles again (from L2 where the graph's tiles are still
+// there).  Nothing per pair is written besides dE: no [B,H,n,n] array.
+//
+// Pass 3 waits for other CTAs (the D of the rows of its chunk).  CTAs take
+// their (graph, row block) from a counter in the order they start, so the
+// row blocks a waiting CTA needs are held by CTAs already running, whose
+// passes 1 and 2 wait for nobody; every wait is bounded.  The wait needs the
+// row blocks of one graph (n/8 <= 128) to fit on the GPU at once, one CTA per
+// SM (148 on B200).
 //
 // Warp roles as in the forward pair kernel: 16 compute warps (warp W reads
 // TMEM quadrant W%4 and handles heads 2(W/4), 2(W/4)+1), one MMA warp (FiLM
-// and u one chunk ahead into double-buffered TMEM ranges, dE when the compute
-// warps have written df), one TMA warp (a ring of twelve 16 KB slots, dE
-// stores).  They meet only on mbarriers.  The pair <-> lane mapping is the
-// forward's: row 4j + ic of E tile s is the pair (j, i = 2ic + s), which lane
-// t of quadrant q = j/8 holds in accumulator register s of its m16n8 tile.
+// and u one chunk ahead into double-buffered TMEM ranges, dE and the weight
+// gradients when the compute warps have written df), one TMA warp (a ring of
+// twelve 16 KB slots, dE stores).  They meet only on mbarriers.  The pair <->
+// lane mapping is the forward's: row 4x + yc of a tile of parity s is the pair
+// of chunk index x and fixed-side index 2yc + s, which lane t of quadrant
+// q = x/8 holds in accumulator register s of its m16n8 tile (rows: the
+// chunk's nodes; columns: the CTA's 8 nodes).
 #include <math.h>
 #include "fast.h"
 #include "fast_common.cuh"
@@ -49,6 +65,7 @@ constexpr int BS_THR = NTHR + 64;
 constexpr int BS_KEEP_MAX_CHUNKS = 7;     // S and dP of up to 7 chunks (n <= 224) stay in TMEM
 
 struct BsSmem {
+    // offsets from a 1024-aligned base; the TMA destinations (slots, LD) are 1024-aligned
     static constexpr uint32_t IMG = BS_SLOTS * BS_SLOT;       // Wfe^T sw (FiLM), We sw (u), Wfe ns (dE): 2 KB each
     static constexpr uint32_t DA = IMG + 6144;                // 2 tiles [128][32] ns: [dgamma | dbeta | a | 0]
     static constexpr uint32_t WD = DA + 16384;                // per-quadrant D [4][8 i][8 h]
@@ -56,14 +73,19 @@ struct BsSmem {
     static constexpr uint32_t G = WDG + 256;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // node mask [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;
-    static constexpr uint32_t TM = BAR + 8 * 14;
+    static constexpr uint32_t TM = BAR + 8 * 16;              // TMEM base address
+    static constexpr uint32_t FAIL = TM + 4;                  // CTA failure flag (a wait ran out)
+    static constexpr uint32_t ITEM = TM + 8;                  // this CTA's work item
     static constexpr uint32_t STAB = TM + 16;                 // slot table [4 iterations][8] u8
-    static constexpr uint32_t BYTES = STAB + 32 + 1024;
-    // in the drained ring at the end: dq quadrant sums [4][8][256] f32 (32 KB)
-    static constexpr uint32_t QPART = 0;
+    static constexpr uint32_t LD = (STAB + 32 + 1023) / 1024 * 1024;   // pass 3: [2 buffers][LSE, D][8 h][32 i] f32
+    static constexpr uint32_t BYTES = LD + 4096 + 1024;
+    // after pass 2, in the DA tiles: dq quadrant sums of four heads [4][8][128] f32 (16 KB);
+    // at the end, in the drained ring: dk and dv quadrant sums [4][8][256] f32 (32 KB each)
+    static constexpr uint32_t KPART = 0, VPART = 32768;
 };
+// mbarriers: full[4], film_full[2], film_empty[2], df_full, de_full, stage_done[4], mma_final
 constexpr int BB_FULL = 0, BB_FILM_FULL = 4, BB_FILM_EMPTY = 6, BB_DF_FULL = 8, BB_DE_FULL = 9,
-              BB_STAGE_DONE = 10;
+              BB_STAGE_DONE = 10, BB_MMA_FINAL = 14;
 
 // TMEM: FiLM 0..63 and u 64..127 (two buffers each), dE 128..255, kept S / dP
 // 256..479 (32 per chunk), and at 480 the weight-gradient accumulator
@@ -79,43 +101,74 @@ __device__ __forceinline__ uint32_t ns32(uint32_t row, uint32_t col) {
     return (row >> 3) * 512u + (col >> 3) * 128u + (row & 7u) * 16u + (col & 7u) * 2u;
 }
 
+__device__ __forceinline__ void st_release_gpu(int *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 struct BwdStreamParams {
-    const __nv_bfloat16 *Q, *dO;
+    const __nv_bfloat16 *Q, *K, *V, *dO;
     const float *LSE, *g;
     const uint8_t *img, *M;
-    __nv_bfloat16 *dQ;       // [B,n,256] out (scaled)
+    __nv_bfloat16 *dQ, *dK, *dV;   // [B,n,256] out (dQ and dK scaled by 1/sqrt(dh))
     float *rparts;           // [graph * row block][RPART] out
-    __nv_bfloat16 *Pa, *Pds; // [B,H,n,npad] out: a and ds (unscaled) of every pair
+    float *DL;               // [B][LSE, D][H][n4]: LSE and D of every row, published by its row block
+    int *flags;              // [graph * row block]: 1 once that row block's D is published (0 at launch)
+    int *ticket;             // work-item counter (0 at launch)
     int *status;
-    int n, npad;
+    int n, n4;               // n4: n rounded up to a multiple of 4 (the DL row length)
+    int light;               // Light Edge variant: no per-edge FiLM map; E is not read, dE = dE'
+    int unnorm;              // unnormalised variant: the edge path reaches s' directly
     uint32_t prefetch_ahead;   // CTAs between this one and the one whose first tiles it prefetches
 };
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 __global__ void __launch_bounds__(BS_THR, 1)
 k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmDEp,
              const __grid_constant__ CUtensorMap tmDE, const __grid_constant__ CUtensorMap tmK,
-             const __grid_constant__ CUtensorMap tmV, BwdStreamParams p) {
+             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmEt,
+             const __grid_constant__ CUtensorMap tmDEpt, const __grid_constant__ CUtensorMap tmQ,
+             const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmDL,
+             BwdStreamParams p) {
     using S = BsSmem;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
     const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = (W >> 2) & 3, t = tid & 31, c4 = t & 3, g8 = t >> 2;
-    const int n = p.n, nch = (n + 31) / 32, nit = 2 * nch;
-    const int b = blockIdx.y, i0 = blockIdx.x * TB;
+    const int n = p.n, nch = (n + 31) / 32, nit = 3 * nch, nrb = (n + TB - 1) / TB;
     const uint32_t bars = sbase + S::BAR;
     auto bar = [&](int k) { return bars + 8 * k; };
     float *g = reinterpret_cast<float *>(sp + S::G);
     uint8_t *mj = sp + S::MJ;
+    volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
 
-    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0.  Its
-    // tiles: E(s=0), E(s=1), dE'(s=0), dE'(s=1), K, then V in pass 1 (and in
-    // pass 2 when S, dP are not kept).  The TMA warp places each tile in any
-    // free slot and records the slot in the table entry it % 4, which the
-    // other warps read after the iteration's load barrier.
+    // work item (graph b, row block rb) in the order the CTAs start
+    if (tid == 0) *reinterpret_cast<volatile int *>(sp + S::ITEM) = atomicAdd(p.ticket, 1);
+    __syncthreads();
+    const int item = *reinterpret_cast<volatile int *>(sp + S::ITEM);
+    const int b = item / nrb, i0 = (item % nrb) * TB;
+
+    // iteration it: pass 1 walks chunks 0..nch-1 of the rows, pass 2 the same
+    // chunks in reverse, pass 3 the row chunks 0..nch-1 of the CTA's columns.
+    // Tiles (slot table entries 0..5): passes 1, 2: E(s=0), E(s=1), dE'(s=0),
+    // dE'(s=1), K, then V (in pass 2 only when S, dP are not kept); pass 3: the
+    // column tiles of E and dE' in the same order, then Q and dO of the chunk's
+    // rows.  The TMA warp places each tile in any free slot and records the
+    // slot in the table entry it % 4, which the other warps read after the
+    // iteration's load barrier.
     const bool keep = nch <= BS_KEEP_MAX_CHUNKS;
-    const int ns1 = 6, ns2 = keep ? 5 : 6;
-    auto chunk_of = [&](int it) { return it < nch ? it : nit - 1 - it; };
-    auto nslots = [&](int it) { return it < nch ? ns1 : ns2; };
+    const bool light = p.light != 0, unnorm = p.unnorm != 0;
+    const int ns2 = keep ? 5 : 6;
+    auto pass_of = [&](int it) { return it < nch ? 1 : it < 2 * nch ? 2 : 3; };
+    auto chunk_of = [&](int it) { return it < nch ? it : it < 2 * nch ? 2 * nch - 1 - it : it - 2 * nch; };
+    auto nslots = [&](int it) { return pass_of(it) == 2 ? ns2 : 6; };
     volatile uint8_t *stab = sp + S::STAB;
     auto slot_addr = [&](int it, int k) { return sbase + (uint32_t)stab[(it % BS_NFULL) * 8 + k] * BS_SLOT; };
 
@@ -129,7 +182,9 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         mbar_init(bar(BB_DF_FULL), NWARP);
         mbar_init(bar(BB_DE_FULL), 1);
         for (int k = 0; k < 4; ++k) mbar_init(bar(BB_STAGE_DONE + k), NWARP);
+        mbar_init(bar(BB_MMA_FINAL), 1);
         fence_mbar_init();
+        *fail = 0;
     }
     if (W == 0) {
         tmem_alloc(sbase + S::TM, BS_TM_COLS);
@@ -161,9 +216,10 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     const uint32_t ae = slot_addr(it, s), ad = slot_addr(it, 2 + s);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        mma_bf16_ss(tmem + BS_TM_FILM + 32 * (it & 1) + 16 * s,
-                                    smem_desc(ae + kk * 32, 16, 1024, LAYOUT_SW128),
-                                    smem_desc(sbase + S::IMG + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f, kk > 0);
+                        if (!light)   // Light Edge: no FiLM product (its E tiles are not loaded)
+                            mma_bf16_ss(tmem + BS_TM_FILM + 32 * (it & 1) + 16 * s,
+                                        smem_desc(ae + kk * 32, 16, 1024, LAYOUT_SW128),
+                                        smem_desc(sbase + S::IMG + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f, kk > 0);
                         mma_bf16_ss(tmem + BS_TM_U + 32 * (it & 1) + 16 * s,
                                     smem_desc(ad + kk * 32, 16, 1024, LAYOUT_SW128),
                                     smem_desc(sbase + S::IMG + 2048 + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f,
@@ -174,10 +230,12 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             };
             auto issue_de = [&](int it) {
                 tc_fence_after();
+                if (!light)   // Light Edge: df Wfe^T = 0, dE = dE'
 #pragma unroll
-                for (int e = 0; e < 2; ++e)
-                    mma_bf16_ss(tmem + BS_TM_DE + 64 * e, smem_desc(sbase + S::DA + e * 8192, 128, 512, LAYOUT_NONE),
-                                smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_d, 0);
+                    for (int e = 0; e < 2; ++e)
+                        mma_bf16_ss(tmem + BS_TM_DE + 64 * e,
+                                    smem_desc(sbase + S::DA + e * 8192, 128, 512, LAYOUT_NONE),
+                                    smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_d, 0);
                 // [dWfe | .] and [. | dWe^T] in one product: A = the E tile and the dE' tile read
                 // MN-major as the two 64-channel atoms of M = 128 (64 c per 128-byte swizzled row,
                 // 8-row groups 1024 B apart; the second atom one slot distance further: the
@@ -197,27 +255,39 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 mma_commit(bar(BB_DE_FULL));
             };
             // issue whichever product is ready first: FiLM/u of the next chunk
-            // (its tiles landed, its TMEM buffer released) or dE of the chunk
-            // whose df the compute warps have written
+            // (its tiles landed, its TMEM buffer released) or dE of the pass-2
+            // chunk whose df the compute warps have written
             int next_fu = 0, next_de = nch;
             uint32_t polls = 0;
-            while (next_fu < nit || next_de < nit) {
+            while ((next_fu < nit || next_de < 2 * nch) && !*fail) {
                 bool progressed = false;
                 if (next_fu < nit && mbar_test_wait(bar(BB_FULL + next_fu % BS_NFULL), (next_fu / BS_NFULL) & 1) &&
                     (next_fu < 2 || mbar_test_wait(bar(BB_FILM_EMPTY + (next_fu & 1)), ((next_fu - 2) >> 1) & 1))) {
                     issue_fu(next_fu++);
                     progressed = true;
                 }
-                if (next_de < nit && next_de < next_fu && mbar_test_wait(bar(BB_DF_FULL), (next_de - nch) & 1)) {
+                if (next_de < 2 * nch && next_de < next_fu && mbar_test_wait(bar(BB_DF_FULL), (next_de - nch) & 1)) {
                     issue_de(next_de);
                     ++next_de;
                     progressed = true;
                 }
-                if (!progressed && ++polls > (1u << 28)) {
-                    flag_timeout(p.status);
-                    break;
+                // idle: back off after a few polls, so that this thread does not
+                // take issue slots from the compute warps of its SM sub-partition;
+                // a wait that makes no progress for 2^24 polls gives up
+                if (progressed) {
+                    polls = 0;
+                } else {
+                    if (++polls > (1u << 24)) {
+                        *fail = 1;
+                        flag_timeout(p.status);
+                        break;
+                    }
+                    if (polls > 8) __nanosleep(64);
                 }
             }
+            // every product issued has completed before the tensor memory is freed
+            mma_commit(bar(BB_MMA_FINAL));
+            if (!mbar_wait(bar(BB_MMA_FINAL), 0)) flag_timeout(p.status);
         }
         __syncwarp();
         named_bar_sync(2, BS_THR);
@@ -225,7 +295,9 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         // ================= TMA: loads into the slot ring, dE stores
         if (t == 0) {
             // E and dE' tiles loaded in pass 1 are read again in pass 2: keep
-            // them in L2; pass-2 reads and the dE stores are not read again
+            // them in L2; pass-2 reads stay at the normal priority (the column
+            // pass of other CTAs reads the same pairs); pass-3 reads and the dE
+            // stores are not read again
             const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
             // a pass-2 chunk's E, K (and V) slots are free once the compute
             // warps are done with it; its dE' slots once the dE store has read them
@@ -233,49 +305,98 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             uint32_t prev_d = 0;          // dE' slots of the previous pass-2 chunk
             int next_load = 0;
             auto release = [&](int it, int k) { free_mask |= 1u << stab[(it % BS_NFULL) * 8 + k]; };
-            auto issue_loads = [&]() {
-                while (next_load < nit && __popc(free_mask) >= nslots(next_load)) {
-                    const int it = next_load, j0 = 32 * chunk_of(it);
-                    const bool pass2 = it >= nch;
+            // D of the row blocks of pass-3 chunk c published by their CTAs?
+            // With `block`, wait for them (bounded).
+            auto rows_ready = [&](int c, bool block) -> bool {
+                const int r1 = min(4 * c + 4, nrb);
+                for (int r = 4 * c; r < r1; ++r) {
+                    const int *f = p.flags + (size_t)b * nrb + r;
+                    if (ld_acquire_gpu(f)) continue;
+                    if (!block) return false;
+                    uint32_t polls = 0;
+                    while (!ld_acquire_gpu(f) && !*fail) {
+                        if (++polls > (1u << 22)) {
+                            *fail = 1;
+                            flag_timeout(p.status);
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                }
+                // the published LSE, D (generic stores of other CTAs, acquired
+                // above) are read next by this thread's TMA copy
+                fence_proxy_async_global();
+                return true;
+            };
+            // issue loads while slots are free; iteration `must` (and only it)
+            // may wait for the rows its pass-3 chunk needs
+            auto issue_loads = [&](int must) {
+                while (next_load < nit && __popc(free_mask) >= nslots(next_load) && !*fail) {
+                    const int it = next_load, ps = pass_of(it), c = chunk_of(it), x0 = 32 * c;
+                    if (ps == 3 && !rows_ready(c, it <= must)) return;
                     const uint32_t fb = bar(BB_FULL + it % BS_NFULL);
                     for (int k = 0; k < nslots(it); ++k) {
                         const int sidx = __ffs(free_mask) - 1;
                         free_mask &= free_mask - 1u;
                         stab[(it % BS_NFULL) * 8 + k] = (uint8_t)sidx;
                     }
-                    mbar_expect_tx(fb, nslots(it) * BS_SLOT);   // releases the table entry with the barrier
+                    // (Light Edge: the E tiles' slots are taken but not loaded)
+                    mbar_expect_tx(fb, (nslots(it) - (light ? 2 : 0)) * BS_SLOT + (ps == 3 ? 2048u : 0u));
+                    if (ps < 3) {
 #pragma unroll
-                    for (int s = 0; s < 2; ++s) {
-                        const uint64_t pol = pass2 ? drop_l2 : keep_l2;
-                        tma_load_5d_hint(slot_addr(it, s), &tmE, fb, 0, i0 / 2, j0, s, b, pol);
-                        tma_load_5d_hint(slot_addr(it, 2 + s), &tmDEp, fb, 0, i0 / 2, j0, s, b, pol);
-                    }
+                        for (int s = 0; s < 2; ++s) {
+                            if (ps == 1) {
+                                if (!light) tma_load_5d_hint(slot_addr(it, s), &tmE, fb, 0, i0 / 2, x0, s, b, keep_l2);
+                                tma_load_5d_hint(slot_addr(it, 2 + s), &tmDEp, fb, 0, i0 / 2, x0, s, b, keep_l2);
+                            } else {
+                                if (!light) tma_load_5d(slot_addr(it, s), &tmE, fb, 0, i0 / 2, x0, s, b);
+                                tma_load_5d(slot_addr(it, 2 + s), &tmDEp, fb, 0, i0 / 2, x0, s, b);
+                            }
+                        }
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        tma_load_3d(slot_addr(it, 4) + k * 4096, &tmK, fb, 64 * k, j0, b);
-                        if (!pass2 || !keep) tma_load_3d(slot_addr(it, 5) + k * 4096, &tmV, fb, 64 * k, j0, b);
+                        for (int k = 0; k < 4; ++k) {
+                            tma_load_3d(slot_addr(it, 4) + k * 4096, &tmK, fb, 64 * k, x0, b);
+                            if (ps == 1 || !keep) tma_load_3d(slot_addr(it, 5) + k * 4096, &tmV, fb, 64 * k, x0, b);
+                        }
+                    } else {
+#pragma unroll
+                        for (int s = 0; s < 2; ++s) {
+                            if (!light) tma_load_5d_hint(slot_addr(it, s), &tmEt, fb, 0, i0 / 2, x0, s, b, drop_l2);
+                            tma_load_5d_hint(slot_addr(it, 2 + s), &tmDEpt, fb, 0, i0 / 2, x0, s, b, drop_l2);
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            tma_load_3d(slot_addr(it, 4) + k * 4096, &tmQ, fb, 64 * k, x0, b);
+                            tma_load_3d(slot_addr(it, 5) + k * 4096, &tmDO, fb, 64 * k, x0, b);
+                        }
+                        // LSE and D of the chunk's rows; buffer c & 1 is free: chunk
+                        // c - 2 released its slots before these could be taken
+                        tma_load_4d(sbase + S::LD + (c & 1) * 2048, &tmDL, fb, x0, 0, 0, b);
                     }
                     ++next_load;
                 }
             };
-            issue_loads();
+            issue_loads(-1);
             for (int it = 0; it < nit; ++it) {
-                const bool pass2 = it >= nch;
+                const int ps = pass_of(it);
+                while (next_load <= it && !*fail) issue_loads(it);
                 if (it == nch && p.prefetch_ahead) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
-                    const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
+                    const uint32_t cid = (uint32_t)item + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
-                        const int prb = cid % gridDim.x, pb = cid / gridDim.x;
+                        const int prb = cid % nrb, pb = cid / nrb;
                         for (int cc = 0; cc < nch && cc < 2; ++cc) {
-                            tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
-                            tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 1, pb);
+                            if (!light) {
+                                tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
+                                tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 1, pb);
+                            }
                             tma_prefetch_5d(&tmDEp, 0, prb * TB / 2, 32 * cc, 0, pb);
                             tma_prefetch_5d(&tmDEp, 0, prb * TB / 2, 32 * cc, 1, pb);
                         }
                     }
                 }
-                if (!mbar_wait(bar(BB_STAGE_DONE + (it & 3)), (it >> 2) & 1)) flag_timeout(p.status);
-                if (pass2) {
+                if (!cta_wait(bar(BB_STAGE_DONE + (it & 3)), (it >> 2) & 1, fail, p.status)) continue;
+                if (ps == 2) {
                     const int j0 = 32 * chunk_of(it);
                     tma_store_5d_hint(&tmDE, slot_addr(it, 2), 0, i0 / 2, j0, 0, b, drop_l2);
                     tma_store_5d_hint(&tmDE, slot_addr(it, 3), 0, i0 / 2, j0, 1, b, drop_l2);
@@ -289,12 +410,20 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         free_mask |= prev_d;
                     }
                     prev_d = (1u << stab[(it % BS_NFULL) * 8 + 2]) | (1u << stab[(it % BS_NFULL) * 8 + 3]);
+                    if (it == 2 * nch - 1) {   // the last dE store: its slots come back for pass 3
+                        tma_store_wait_read0();
+                        free_mask |= prev_d;
+                        prev_d = 0;
+                    }
                 } else {
-                    for (int k = 0; k < ns1; ++k) release(it, k);
+                    for (int k = 0; k < 6; ++k) release(it, k);
                 }
-                issue_loads();
+                issue_loads(-1);
             }
             tma_store_wait_read0();
+            if (*fail)   // loads already issued land before the CTA's shared memory is released
+                for (int it = max(next_load - BS_NFULL, 0); it < next_load; ++it)
+                    mbar_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1);
         }
         __syncwarp();
         named_bar_sync(2, BS_THR);   // the ring is drained: the compute warps may reuse it
@@ -303,229 +432,358 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
         const float rs = rsqrtf((float)DH);
         const uint32_t L = 32 * q + t;
-        uint32_t qf[2][2][2], of[2][2][2];
-        load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
-        load_frags2(p.dO, b, n, i0, hq, g8, c4, of);
-        bool mrow[2];
-        float lse[2][2];
+        bool mrow[2];            // the CTA's own nodes i0 + 2c4 + e: rows in passes 1-2, columns in pass 3
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int i = i0 + 2 * c4 + e;
             mrow[e] = i < n && p.M[(size_t)b * n + i] != 0;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) lse[e][hh] = i < n ? p.LSE[((size_t)b * NH + 2 * hq + hh) * n + i] : 0.f;
         }
-        float dsum[2][2] = {{0.f, 0.f}, {0.f, 0.f}};     // running D partial, then the final D [e][hh]
-        float qacc[2][2][4];
-        float dgp[4] = {0.f, 0.f, 0.f, 0.f};              // dgamma h0, h1, dbeta h0, h1
+        {
+            // ======== passes 1 and 2: the CTA's rows
+            uint32_t qf[2][2][2], of[2][2][2];
+            load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
+            load_frags2(p.dO, b, n, i0, hq, g8, c4, of);
+            float lse[2][2];
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
+            for (int e = 0; e < 2; ++e) {
+                const int i = i0 + 2 * c4 + e;
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) qacc[hh][0][x] = qacc[hh][1][x] = 0.f;
+                for (int hh = 0; hh < 2; ++hh) lse[e][hh] = i < n ? p.LSE[((size_t)b * NH + 2 * hq + hh) * n + i] : 0.f;
+            }
+            float dsum[2][2] = {{0.f, 0.f}, {0.f, 0.f}};     // running D partial, then the final D [e][hh]
+            float qacc[2][2][4];
+            float dgp[4] = {0.f, 0.f, 0.f, 0.f};              // dgamma h0, h1, dbeta h0, h1
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) qacc[hh][0][x] = qacc[hh][1][x] = 0.f;
 
-        for (int it = 0; it < nit; ++it) {
-            const int c = chunk_of(it), j0 = 32 * c;
-            const bool pass2 = it >= nch;
+            for (int it = 0; it < 2 * nch; ++it) {
+                const int c = chunk_of(it), j0 = 32 * c;
+                const bool pass2 = it >= nch;
 
-            if (it == nch) {
-                // ---------------- D over lanes, then quadrants
-                tmem_st_wait();
-                float *wd = reinterpret_cast<float *>(sp + S::WD);
+                if (it == nch) {
+                    // ---------------- D over lanes, then quadrants
+                    tmem_st_wait();
+                    float *wd = reinterpret_cast<float *>(sp + S::WD);
 #pragma unroll
-                for (int e = 0; e < 2; ++e)
+                    for (int e = 0; e < 2; ++e)
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float x = dsum[e][hh];
-                        x += __shfl_xor_sync(0xffffffffu, x, 4);
-                        x += __shfl_xor_sync(0xffffffffu, x, 8);
-                        x += __shfl_xor_sync(0xffffffffu, x, 16);
-                        if (g8 == 0) wd[(q * 8 + 2 * c4 + e) * 8 + 2 * hq + hh] = x;
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float x = dsum[e][hh];
+                            x += __shfl_xor_sync(0xffffffffu, x, 4);
+                            x += __shfl_xor_sync(0xffffffffu, x, 8);
+                            x += __shfl_xor_sync(0xffffffffu, x, 16);
+                            if (g8 == 0) wd[(q * 8 + 2 * c4 + e) * 8 + 2 * hq + hh] = x;
+                        }
+                    named_bar_sync(1, NTHR);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int o = (2 * c4 + e) * 8 + 2 * hq + hh;
+                            dsum[e][hh] = wd[o] + wd[64 + o] + wd[128 + o] + wd[192 + o];
+                        }
+                    // publish LSE and D of the row block for the column pass of the graph's CTAs
+                    if (q == 0 && g8 == 0) {
+#pragma unroll
+                        for (int e = 0; e < 2; ++e)
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const int i = i0 + 2 * c4 + e;
+                                const size_t o = ((size_t)b * 2 * NH + 2 * hq + hh) * p.n4 + i;
+                                if (i < n) {
+                                    p.DL[o] = lse[e][hh];
+                                    p.DL[o + (size_t)NH * p.n4] = dsum[e][hh];
+                                }
+                            }
+                        __threadfence();
                     }
-                named_bar_sync(1, NTHR);
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int o = (2 * c4 + e) * 8 + 2 * hq + hh;
-                        dsum[e][hh] = wd[o] + wd[64 + o] + wd[128 + o] + wd[192 + o];
+                    named_bar_sync(1, NTHR);
+                    if (tid == 0) st_release_gpu(p.flags + item, 1);
+                }
+
+                cta_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1, fail, p.status);
+                // ---------------- S = Q K^T, dP = dO V^T (warp MMAs), or the kept ones
+                float sv[2][4], da[2][4];
+                const uint32_t kcol = tl + BS_TM_KEEP + 32 * c + 2 * hq;
+                if (pass2 && keep) {
+                    tmem_ld2(kcol, sv[0][0], sv[1][0]);
+                    tmem_ld2(kcol + 8, sv[0][1], sv[1][1]);
+                    tmem_ld2(kcol + 16, da[0][0], da[1][0]);
+                    tmem_ld2(kcol + 24, da[0][1], da[1][1]);
+                    tmem_ld_wait();
+                } else {
+                    warp_scores2<1>(slot_addr(it, 4), q, t, hq, qf, sv);
+                    warp_scores2<1>(slot_addr(it, 5), q, t, hq, of, da);
+                    if (keep) {
+                        tmem_st2(kcol, sv[0][0], sv[1][0]);
+                        tmem_st2(kcol + 8, sv[0][1], sv[1][1]);
+                        tmem_st2(kcol + 16, da[0][0], da[1][0]);
+                        tmem_st2(kcol + 24, da[0][1], da[1][1]);
                     }
-            }
-
-            if (!mbar_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1)) flag_timeout(p.status);
-            // ---------------- S = Q K^T, dP = dO V^T (warp MMAs), or the kept ones
-            float sv[2][4], da[2][4];
-            const uint32_t kcol = tl + BS_TM_KEEP + 32 * c + 2 * hq;
-            if (pass2 && keep) {
-                tmem_ld2(kcol, sv[0][0], sv[1][0]);
-                tmem_ld2(kcol + 8, sv[0][1], sv[1][1]);
-                tmem_ld2(kcol + 16, da[0][0], da[1][0]);
-                tmem_ld2(kcol + 24, da[0][1], da[1][1]);
-                tmem_ld_wait();
-            } else {
-                warp_scores2<1>(slot_addr(it, 4), q, t, hq, qf, sv);
-                warp_scores2<1>(slot_addr(it, 5), q, t, hq, of, da);
-                if (keep) {
-                    tmem_st2(kcol, sv[0][0], sv[1][0]);
-                    tmem_st2(kcol + 8, sv[0][1], sv[1][1]);
-                    tmem_st2(kcol + 16, da[0][0], da[1][0]);
-                    tmem_st2(kcol + 24, da[0][1], da[1][1]);
                 }
-            }
 
-            // ---------------- FiLM and u from TMEM
-            if (!mbar_wait(bar(BB_FILM_FULL + (it & 1)), (it >> 1) & 1)) flag_timeout(p.status);
-            tc_fence_after();
-            float fg[2][2], fb[2][2], fu[2][2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const uint32_t fcol = BS_TM_FILM + 32 * (it & 1) + 16 * e, ucol = BS_TM_U + 32 * (it & 1) + 16 * e;
-                tmem_ld2(tl + fcol + 2 * hq, fg[e][0], fg[e][1]);
-                tmem_ld2(tl + fcol + NH + 2 * hq, fb[e][0], fb[e][1]);
-                tmem_ld2(tl + ucol + 2 * hq, fu[e][0], fu[e][1]);
-            }
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (t == 0) mbar_arrive(bar(BB_FILM_EMPTY + (it & 1)));
-            const bool mcol = mj[j0 + 8 * q + g8] != 0;
-            float av[2][4], gm[2][4];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const bool valid = mcol && mrow[e];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int h = 2 * hq + hh;
-                    const float s = sv[hh][e] * rs;
-                    const float gam = fg[e][hh] + g[h], bet = fb[e][hh] + g[NH + h];
-                    av[hh][e] = valid ? exp2f((s * (1.f + gam) + bet - lse[e][hh]) * LOG2E) : 0.f;
-                    sv[hh][e] = s;
-                    gm[hh][e] = gam;
-                    da[hh][e] += fu[e][hh];
-                }
-            }
-
-            if (!pass2) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) dsum[e][hh] += av[hh][e] * da[hh][e];
-                __syncwarp();
-                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
-                continue;
-            }
-
-            // ---------------- pass 2: dS', df and a tiles for the tensor cores / warp MMAs
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float dgam[2], dbet[2];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const float dsp = av[hh][e] * (da[hh][e] - dsum[e][hh]);
-                    dgam[hh] = dsp * sv[hh][e];
-                    dbet[hh] = dsp;
-                    da[hh][e] = dsp * (1.f + gm[hh][e]);     // ds (unscaled)
-                    dgp[hh] += dgam[hh];
-                    dgp[2 + hh] += dbet[hh];
-                }
-                *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, 2 * hq)) = pack_bf16(dgam[0], dgam[1]);
-                *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, NH + 2 * hq)) = pack_bf16(dbet[0], dbet[1]);
-                *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, NF + 2 * hq)) = pack_bf16(av[0][e], av[1][e]);
-            }
-            av[0][2] = av[0][3] = av[1][2] = av[1][3] = 0.f;
-            da[0][2] = da[0][3] = da[1][2] = da[1][3] = 0.f;
-            // df and a of this warp's rows are in place: the MMA warp issues dE and
-            // the weight-gradient products once all 16 warps have arrived
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (t == 0) mbar_arrive(bar(BB_DF_FULL));
-
-            // a and ds of the chunk's pairs for the dk / dv pass: [b][h][i][j] bf16.
-            // Lanes t and t^4 hold neighbouring columns j; they swap one head so that
-            // each stores two columns of one head in a 4-byte word.
-            {
-                const bool odd = g8 & 1;
+                // ---------------- FiLM and u from TMEM
+                cta_wait(bar(BB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
+                tc_fence_after();
+                float fg[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, fb[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, fu[2][2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float xa = __shfl_xor_sync(0xffffffffu, odd ? av[0][e] : av[1][e], 4);
-                    const float xd = __shfl_xor_sync(0xffffffffu, odd ? da[0][e] : da[1][e], 4);
-                    const int i = i0 + 2 * c4 + e, j = j0 + 8 * q + (g8 & ~1);
-                    if (i < n && j < n) {
-                        const size_t o = (((size_t)b * NH + 2 * hq + (odd ? 1 : 0)) * n + i) * p.npad + j;
-                        // streaming stores: read once, by the dk / dv kernel
-                        __stcs(reinterpret_cast<unsigned int *>(p.Pa + o), odd ? pack_bf16(xa, av[1][e]) : pack_bf16(av[0][e], xa));
-                        __stcs(reinterpret_cast<unsigned int *>(p.Pds + o), odd ? pack_bf16(xd, da[1][e]) : pack_bf16(da[0][e], xd));
+                    const uint32_t fcol = BS_TM_FILM + 32 * (it & 1) + 16 * e, ucol = BS_TM_U + 32 * (it & 1) + 16 * e;
+                    if (!light) {   // Light Edge: gamma, beta from y alone
+                        tmem_ld2(tl + fcol + 2 * hq, fg[e][0], fg[e][1]);
+                        tmem_ld2(tl + fcol + NH + 2 * hq, fb[e][0], fb[e][1]);
+                    }
+                    tmem_ld2(tl + ucol + 2 * hq, fu[e][0], fu[e][1]);
+                }
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (t == 0) mbar_arrive(bar(BB_FILM_EMPTY + (it & 1)));
+                const bool mcol = mj[j0 + 8 * q + g8] != 0;
+                // av: a; sv: s; gm: gamma; da: dA (the layer) or dP with the edge
+                // term u in fu (the unnormalised variant: u enters dS' directly)
+                // and the modulated score in fb (for dWe)
+                float av[2][4], gm[2][4];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const bool valid = mcol && mrow[e];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int h = 2 * hq + hh;
+                        const float s = sv[hh][e] * rs;
+                        const float gam = fg[e][hh] + g[h], bet = fb[e][hh] + g[NH + h];
+                        const float spv = s * (1.f + gam) + bet;
+                        av[hh][e] = valid ? exp2f((spv - lse[e][hh]) * LOG2E) : 0.f;
+                        sv[hh][e] = s;
+                        gm[hh][e] = gam;
+                        if (unnorm) {
+                            fu[e][hh] = valid ? fu[e][hh] : 0.f;
+                            fb[e][hh] = valid ? spv : 0.f;
+                        } else {
+                            da[hh][e] += fu[e][hh];
+                        }
                     }
                 }
+
+                if (!pass2) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) dsum[e][hh] += av[hh][e] * da[hh][e];
+                    __syncwarp();
+                    if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
+                    continue;
+                }
+
+                // ---------------- pass 2: dS', df and a tiles for the tensor cores / warp MMAs
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float dgam[2], dbet[2];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const float dsp = av[hh][e] * (da[hh][e] - dsum[e][hh]) + (unnorm ? fu[e][hh] : 0.f);
+                        dgam[hh] = dsp * sv[hh][e];
+                        dbet[hh] = dsp;
+                        da[hh][e] = dsp * (1.f + gm[hh][e]);     // ds (unscaled)
+                        dgp[hh] += dgam[hh];
+                        dgp[2 + hh] += dbet[hh];
+                    }
+                    *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, 2 * hq)) = pack_bf16(dgam[0], dgam[1]);
+                    *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, NH + 2 * hq)) = pack_bf16(dbet[0], dbet[1]);
+                    // the coefficients the edge update used: a, or s' (unnormalised)
+                    *reinterpret_cast<uint32_t *>(sp + S::DA + e * 8192 + ns32(L, NF + 2 * hq)) =
+                        unnorm ? pack_bf16(fb[e][0], fb[e][1]) : pack_bf16(av[0][e], av[1][e]);
+                }
+                da[0][2] = da[0][3] = da[1][2] = da[1][3] = 0.f;
+                // df and a of this warp's rows are in place: the MMA warp issues dE and
+                // the weight-gradient products once all 16 warps have arrived
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (t == 0) mbar_arrive(bar(BB_DF_FULL));
+
+                // ---------------- dq += ds K (warp MMAs; overlaps the tensor-core products)
+                warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, da, qacc);
+
+                // ---------------- dE = dE' + df Wfe^T, in place (the TMA warp stores it)
+                cta_wait(bar(BB_DE_FULL), (it - nch) & 1, fail, p.status);
+                tc_fence_after();
+                if (!light)   // Light Edge: dE = dE', the tile is stored as loaded
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float dv[16];
+                        tmem_ld16(tl + BS_TM_DE + 64 * e + 16 * hq, dv);
+                        tmem_ld_wait();
+                        add_residual16(sp + (slot_addr(it, 2 + e) - sbase) + L * 128, L, hq, dv);
+                    }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
             }
 
-            // ---------------- dq += ds K (warp MMAs; overlaps the tensor-core products)
-            warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, da, qacc);
-
-            // ---------------- dE = dE' + df Wfe^T, in place (the TMA warp stores it)
-            if (!mbar_wait(bar(BB_DE_FULL), (it - nch) & 1)) flag_timeout(p.status);
-            tc_fence_after();
+            // ---------------- row-block results: dq through the (now idle) DA tiles,
+            // four heads at a time; dg and the weight-gradient partials
+            float *part = reinterpret_cast<float *>(sp + S::DA);
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                if ((hq >> 1) == half) {
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float dv[16];
-                tmem_ld16(tl + BS_TM_DE + 64 * e + 16 * hq, dv);
-                tmem_ld_wait();
-                add_residual16(sp + (slot_addr(it, 2 + e) - sbase) + L * 128, L, hq, dv);
+                    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int d = (2 * (hq & 1) + hh) * DH + mt * 16 + g8 + 8 * (e >> 1), il = 2 * c4 + (e & 1);
+                                part[(q * TB + il) * 128 + d] = qacc[hh][mt][e];
+                            }
+                }
+                named_bar_sync(1, NTHR);
+                {
+                    const int x = tid, il = (2 * x) / 128, d = (2 * x) % 128;   // 512 threads: 8 rows x 64 pairs
+                    if (i0 + il < n) {
+                        float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            o0 += part[(k * TB + il) * 128 + d];
+                            o1 += part[(k * TB + il) * 128 + d + 1];
+                        }
+                        *reinterpret_cast<uint32_t *>(p.dQ + ((size_t)b * n + i0 + il) * HD + 128 * half + d) =
+                            pack_bf16(o0 * rs, o1 * rs);
+                    }
+                }
+                named_bar_sync(1, NTHR);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
-        }
-
-        // ---------------- end of the row block, in the drained ring
-        named_bar_sync(2, BS_THR);
-        float *wdg = reinterpret_cast<float *>(sp + S::WDG);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float x = dgp[k];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-            if (t == 0) wdg[W * 4 + k] = x;
-        }
-        store_quadrant_part(sp, S::QPART, qacc, q, hq, t);
-        named_bar_sync(1, NTHR);
-        const float *part = reinterpret_cast<const float *>(sp + S::QPART);
-        for (int x = tid; x < TB * HD / 2; x += NTHR) {
-            const int il = (2 * x) / HD, d = (2 * x) % HD;
-            if (i0 + il >= n) continue;
-            float o0 = 0.f, o1 = 0.f;
+            float *wdg = reinterpret_cast<float *>(sp + S::WDG);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                o0 += part[k * TB * HD + il * HD + d];
-                o1 += part[k * TB * HD + il * HD + d + 1];
+                float x = dgp[k];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                if (t == 0) wdg[W * 4 + k] = x;
             }
-            *reinterpret_cast<uint32_t *>(p.dQ + ((size_t)b * n + i0 + il) * HD + d) = pack_bf16(o0 * rs, o1 * rs);
-        }
-        // weight-gradient partials of the row block: dWfe [c][k] from lanes 0..63,
-        // columns 0..15 of the accumulator, dWe^T [c][h] from lanes 64..127,
-        // columns 16..23; dg from the per-warp sums
-        float *rp = p.rparts + (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * RPART;
-        tc_fence_after();
-        if (hq == 0) {
-            float v[16];
-            tmem_ld16(tl + BS_TM_W + (q < 2 ? 0 : NF), v);
-            tmem_ld_wait();
-            if (q < 2) {
-                const int c = 32 * q + t;
+            named_bar_sync(1, NTHR);
+            // weight-gradient partials of the row block: dWfe [c][k] from lanes 0..63,
+            // columns 0..15 of the accumulator, dWe^T [c][h] from lanes 64..127,
+            // columns 16..23; dg from the per-warp sums
+            float *rp = p.rparts + (size_t)item * RPART;
+            tc_fence_after();
+            if (hq == 0) {
+                float v[16];
+                tmem_ld16(tl + BS_TM_W + (q < 2 ? 0 : NF), v);
+                tmem_ld_wait();
+                if (q < 2) {
+                    const int c = 32 * q + t;
 #pragma unroll
-                for (int k = 0; k < NF; ++k) rp[c * NF + k] = v[k];
-            } else {
-                const int c = 32 * (q - 2) + t;
+                    for (int k = 0; k < NF; ++k) rp[c * NF + k] = v[k];
+                } else {
+                    const int c = 32 * (q - 2) + t;
 #pragma unroll
-                for (int h = 0; h < NH; ++h) rp[DE * NF + h * DE + c] = v[h];
+                    for (int h = 0; h < NH; ++h) rp[DE * NF + h * DE + c] = v[h];
+                }
+            }
+            if (tid < NF) {
+                const int which = tid >> 3, h = tid & 7, hq2 = h >> 1, hh = h & 1;
+                float v = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v += wdg[(4 * hq2 + k) * 4 + which * 2 + hh];
+                rp[DE * NF + NH * DE + tid] = v;
             }
         }
-        if (tid < NF) {
-            const int which = tid >> 3, h = tid & 7, hq2 = h >> 1, hh = h & 1;
-            float v = 0.f;
+
+        // ======== pass 3: the CTA's nodes as columns j, rows i in chunks of 32
+        {
+            uint32_t kf[2][2][2], vf[2][2][2];
+            load_frags2(p.K, b, n, i0, hq, g8, c4, kf);
+            load_frags2(p.V, b, n, i0, hq, g8, c4, vf);
+            float kacc[2][2][4], vacc[2][2][4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) v += wdg[(4 * hq2 + k) * 4 + which * 2 + hh];
-            rp[DE * NF + NH * DE + tid] = v;
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) kacc[hh][mt][x] = vacc[hh][mt][x] = 0.f;
+            for (int it = 2 * nch; it < nit; ++it) {
+                const int ir = 32 * (it - 2 * nch) + 8 * q + g8;   // this lane's row i
+                cta_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1, fail, p.status);
+                // LSE_i and D_i as the row blocks published them (TMA-loaded with the chunk)
+                float lse3[2], d3[2];
+                {
+                    const float *ld = reinterpret_cast<const float *>(sp + S::LD + ((it - 2 * nch) & 1) * 2048);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        lse3[hh] = ld[(2 * hq + hh) * 32 + 8 * q + g8];
+                        d3[hh] = ld[(NH + 2 * hq + hh) * 32 + 8 * q + g8];
+                    }
+                }
+                float sv[2][4], dp[2][4];
+                warp_scores2<1>(slot_addr(it, 4), q, t, hq, kf, sv);    // q_i . k_j
+                warp_scores2<1>(slot_addr(it, 5), q, t, hq, vf, dp);    // dO_i . v_j
+                cta_wait(bar(BB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
+                tc_fence_after();
+                float fg[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, fb[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, fu[2][2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const uint32_t fcol = BS_TM_FILM + 32 * (it & 1) + 16 * e, ucol = BS_TM_U + 32 * (it & 1) + 16 * e;
+                    if (!light) {   // Light Edge: gamma, beta from y alone
+                        tmem_ld2(tl + fcol + 2 * hq, fg[e][0], fg[e][1]);
+                        tmem_ld2(tl + fcol + NH + 2 * hq, fb[e][0], fb[e][1]);
+                    }
+                    tmem_ld2(tl + ucol + 2 * hq, fu[e][0], fu[e][1]);
+                }
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (t == 0) mbar_arrive(bar(BB_FILM_EMPTY + (it & 1)));
+                const bool mi = mj[ir] != 0;   // mj covers 32 * nch nodes, zero past n
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const bool valid = mi && mrow[e];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int h = 2 * hq + hh;
+                        const float s = sv[hh][e] * rs;
+                        const float gam = fg[e][hh] + g[h], bet = fb[e][hh] + g[NH + h];
+                        const float a = valid ? exp2f((s * (1.f + gam) + bet - lse3[hh]) * LOG2E) : 0.f;
+                        const float dsp = unnorm ? a * (dp[hh][e] - d3[hh]) + (valid ? fu[e][hh] : 0.f)
+                                                 : a * (dp[hh][e] + fu[e][hh] - d3[hh]);
+                        sv[hh][e] = a;                       // a_ij
+                        dp[hh][e] = dsp * (1.f + gam);       // ds_ij (unscaled)
+                    }
+                }
+                sv[0][2] = sv[0][3] = sv[1][2] = sv[1][3] = 0.f;
+                dp[0][2] = dp[0][3] = dp[1][2] = dp[1][3] = 0.f;
+                // dk_j += sum_i ds_ij q_i, dv_j += sum_i a_ij dO_i (warp MMAs over the chunk's rows)
+                warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, dp, kacc);
+                warp_contract2<1, true>(slot_addr(it, 5), q, t, hq, sv, vacc);
+                __syncwarp();
+                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
+            }
+
+            // ---------------- dk, dv: sum over the quadrant warps, in the drained ring
+            named_bar_sync(2, BS_THR);
+            store_quadrant_part(sp, S::KPART, kacc, q, hq, t);
+            store_quadrant_part(sp, S::VPART, vacc, q, hq, t);
+            named_bar_sync(1, NTHR);
+            const float *kp = reinterpret_cast<const float *>(sp + S::KPART);
+            const float *vp = reinterpret_cast<const float *>(sp + S::VPART);
+            for (int x = tid; x < TB * HD / 2; x += NTHR) {
+                const int il = (2 * x) / HD, d = (2 * x) % HD;
+                if (i0 + il >= n) continue;
+                float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int o = k * TB * HD + il * HD + d;
+                    k0 += kp[o];
+                    k1 += kp[o + 1];
+                    v0 += vp[o];
+                    v1 += vp[o + 1];
+                }
+                const size_t o = ((size_t)b * n + i0 + il) * HD + d;
+                *reinterpret_cast<uint32_t *>(p.dK + o) = pack_bf16(k0 * rs, k1 * rs);
+                *reinterpret_cast<uint32_t *>(p.dV + o) = pack_bf16(v0, v1);
+            }
         }
     }
     tc_fence_before();
@@ -539,27 +797,39 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
                               cudaStream_t st) {
     static std::atomic<uint32_t> attr_set{0};
     if (cudaError_t e = ensure_smem_attr(k_bwd_stream, BsSmem::BYTES, attr_set); e != cudaSuccess) return e;
-    CUtensorMap mE, mDEp, mDE, mK, mV;
+    const __nv_bfloat16 *dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
+    CUtensorMap mE, mDEp, mDE, mK, mV, mEt, mDEpt, mQ, mDO, mDL;
+    const int n4 = (d.n + 3) / 4 * 4;
     if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mDEp, a.dEout, d.B, d.n, false, 32, 1) ||
         !encode_pair_map(&mDE, a.dE, d.B, d.n, false, 32, 1) || !encode_node_map(&mK, a.K, d.B, d.n, 32) ||
-        !encode_node_map(&mV, a.V, d.B, d.n, 32))
+        !encode_node_map(&mV, a.V, d.B, d.n, 32) || !encode_pair_map(&mEt, a.E, d.B, d.n, true, 32, 1) ||
+        !encode_pair_map(&mDEpt, a.dEout, d.B, d.n, true, 32, 1) || !encode_node_map(&mQ, a.Q, d.B, d.n, 32) ||
+        !encode_node_map(&mDO, dO, d.B, d.n, 32) || !encode_rowstat_map(&mDL, ws + W.Drow, d.B, d.n, n4))
         return cudaErrorInvalidValue;
     BwdStreamParams p;
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
-    p.dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
+    p.K = static_cast<const __nv_bfloat16 *>(a.K);
+    p.V = static_cast<const __nv_bfloat16 *>(a.V);
+    p.dO = dO;
     p.LSE = a.LSE;
     p.g = g;
     p.img = reinterpret_cast<const uint8_t *>(ws + W.img);
     p.M = a.M;
     p.dQ = reinterpret_cast<__nv_bfloat16 *>(ws + W.dQ);
+    p.dK = reinterpret_cast<__nv_bfloat16 *>(ws + W.dK);
+    p.dV = reinterpret_cast<__nv_bfloat16 *>(ws + W.dV);
     p.rparts = reinterpret_cast<float *>(ws + W.rparts);
-    p.Pa = reinterpret_cast<__nv_bfloat16 *>(ws + W.Pa);
-    p.Pds = reinterpret_cast<__nv_bfloat16 *>(ws + W.Pds);
+    p.DL = reinterpret_cast<float *>(ws + W.Drow);
+    p.flags = reinterpret_cast<int *>(ws + W.flags);
+    p.ticket = p.flags + W.n_rparts;
     p.status = a.status;
     p.n = d.n;
-    p.npad = W.npad;
+    p.n4 = n4;
+    p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
+    p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)sm_count();
-    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, p);
+    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, mEt, mDEpt,
+                                                                                mQ, mDO, mDL, p);
     return cudaGetLastError();
 }
 

@@ -40,10 +40,11 @@ __host__ __device__ __forceinline__ uint32_t ns16(uint32_t row, uint32_t k) {
     return (row >> 3) * 256u + (k >> 3) * 128u + (row & 7u) * 16u + (k & 7u) * 2u;
 }
 
-// Workspace of the fast path (after the common status word and g).
+// Workspace of the fast path (after the common status word and g).  Every
+// region grows with the node count B*n (or is fixed): no per-pair buffer.
 struct FastWs {
-    size_t img, dO, dQ, dK, dV, Pa, Pds, rparts, wparts, bparts, r2, dg, total;
-    int n_rparts, wsplits, bsplits, rsplits, npad;
+    size_t img, dO, dQ, dK, dV, Drow, flags, rparts, wparts, bparts, r2, dg, total;
+    int n_rparts, wsplits, bsplits, rsplits;
 };
 
 inline int row_blocks(const eaga_dims &d) { return ((d.n + TB - 1) / TB) * d.B; }
@@ -63,11 +64,11 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
     W.dQ = off; off = align256(off + rows * HD * 2);
     W.dK = off; off = align256(off + rows * HD * 2);
     W.dV = off; off = align256(off + rows * HD * 2);
-    // a and ds of every pair, [B][H][n][npad] bf16, for the dk / dv pass
-    W.npad = (d.n + 7) / 8 * 8;
-    W.Pa = off; off = align256(off + size_t(d.B) * NH * d.n * W.npad * 2);
-    W.Pds = off; off = align256(off + size_t(d.B) * NH * d.n * W.npad * 2);
+    // LSE and D of every row [B][2][H][roundup4(n)] fp32, published by the pair kernel's row blocks
+    W.Drow = off; off = align256(off + size_t(d.B) * 2 * NH * ((d.n + 3) / 4 * 4) * 4);
     W.n_rparts = row_blocks(d);
+    // one flag per (graph, row block), then the pair kernel's work-item counter: zeroed per call
+    W.flags = off; off = align256(off + size_t(W.n_rparts + 1) * 4);
     W.rparts = off; off = align256(off + size_t(W.n_rparts) * RPART * 4);
     W.wsplits = wgrad_splits(d);
     // split-K partials of dWq, dWk, dWv [dx, 256] and dWo [256, dx]
@@ -83,7 +84,7 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
 
 bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transposed, int box_rows, int box_s = 2);
 bool encode_node_map(CUtensorMap *m, const void *base, int B, int n, int box_rows);
-bool encode_p_map(CUtensorMap *m, const void *base, int B, int n, int npad);
+bool encode_rowstat_map(CUtensorMap *m, const void *base, int B, int n, int n4);
 
 
 // ------------------------------------------------------------------ device pieces
@@ -215,7 +216,8 @@ __device__ __forceinline__ void flag_timeout(int *status) { atomicExch(status, D
 // control flow (the same named barriers, in-bounds addresses) to the end,
 // where it waits, again with a bound, for what it already issued and frees
 // its tensor memory.  A stalled CTA therefore costs about one bound, not one
-// bound per wait.
+// bound per wait.  (Polls without a suspend-time hint: sleeping between
+// polls was measured slower, the wake-up sits on the critical path.)
 __device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, volatile int *fail, int *status,
                                          uint32_t limit = (1u << 24)) {
     if (*fail) return false;

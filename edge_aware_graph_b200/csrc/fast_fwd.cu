@@ -78,6 +78,8 @@ struct FwdParams {
     float *LSE;
     int *status;
     int n;
+    int light;                 // Light Edge variant: no per-edge FiLM map, no E in pass 1, no FiLM products
+    int unnorm;                // unnormalised variant: the edge update takes s' instead of a
     uint32_t prefetch_ahead;   // CTAs between this one and the one whose first tiles it prefetches
 };
 
@@ -98,13 +100,16 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
 
     // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0.  Its
-    // slots, from slot_base(it) on: pass 1 E(s=0), E(s=1), K; pass 2 E(s=0),
-    // E(s=1), V when the pass-1 scores stay in TMEM, else E, E, K, V.
+    // slots, from slot_base(it) on: pass 1 E(s=0), E(s=1), K (Light Edge: K
+    // alone); pass 2 E(s=0), E(s=1), V when the pass-1 scores stay in TMEM,
+    // else E, E, K, V.
+    const bool light = p.light != 0;
     const bool keep_s = nch <= FS_KEEP_S_MAX_CHUNKS;
+    const int ns1 = light ? 1 : 3, ks1 = light ? 0 : 2;
     const int ns2 = keep_s ? 3 : 4, vslot = ns2 - 1;
     auto chunk_of = [&](int it) { return it < nch ? it : nit - 1 - it; };
-    auto nslots = [&](int it) { return it < nch ? 3 : ns2; };
-    auto slot_base = [&](int it) { return (3 * min(it, nch) + ns2 * max(it - nch, 0)) % FS_SLOTS; };
+    auto nslots = [&](int it) { return it < nch ? ns1 : ns2; };
+    auto slot_base = [&](int it) { return (ns1 * min(it, nch) + ns2 * max(it - nch, 0)) % FS_SLOTS; };
     auto slot_addr = [&](int it, int k) { return sbase + (uint32_t)((slot_base(it) + k) % FS_SLOTS) * FS_SLOT; };
 
     // ---------------- setup: barriers, TMEM, operands
@@ -168,7 +173,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             // issue whichever product is ready first: FiLM of the next chunk (its
             // tiles landed, its TMEM buffer released) or the edge update of the
             // chunk whose a the compute warps have written
-            int next_film = 0, next_edge = nch;
+            int next_film = light ? nit : 0, next_edge = nch;   // Light Edge: no FiLM products
             uint32_t polls = 0;
             while ((next_film < nit || next_edge < nit) && !*fail) {
                 bool progressed = false;
@@ -185,10 +190,18 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     ++next_edge;
                     progressed = true;
                 }
-                if (!progressed && ++polls > (1u << 28)) {
-                    *fail = 1;
-                    flag_timeout(p.status);
-                    break;
+                // idle: back off after a few polls, so that this thread does not
+                // take issue slots from the compute warps of its SM sub-partition;
+                // a wait that makes no progress for 2^24 polls gives up
+                if (progressed) {
+                    polls = 0;
+                } else {
+                    if (++polls > (1u << 24)) {
+                        *fail = 1;
+                        flag_timeout(p.status);
+                        break;
+                    }
+                    if (polls > 8) __nanosleep(64);
                 }
             }
             // every product issued has completed before the tensor memory is freed
@@ -211,25 +224,28 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     const uint32_t fb = bar(FB_FULL + it % FS_NFULL);
                     mbar_expect_tx(fb, nslots(it) * FS_SLOT);
                     const uint64_t pol = pass2 ? drop_l2 : keep_l2;
-                    tma_load_5d_hint(slot_addr(it, 0), &tmE, fb, 0, i0 / 2, j0, 0, b, pol);
-                    tma_load_5d_hint(slot_addr(it, 1), &tmE, fb, 0, i0 / 2, j0, 1, b, pol);
+                    if (pass2 || !light) {
+                        tma_load_5d_hint(slot_addr(it, 0), &tmE, fb, 0, i0 / 2, j0, 0, b, pol);
+                        tma_load_5d_hint(slot_addr(it, 1), &tmE, fb, 0, i0 / 2, j0, 1, b, pol);
+                    }
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        if (!pass2 || !keep_s) tma_load_3d(slot_addr(it, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
+                        if (!pass2) tma_load_3d(slot_addr(it, ks1) + k * 4096, &tmK, fb, 64 * k, j0, b);
+                        else if (!keep_s) tma_load_3d(slot_addr(it, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
                         if (pass2) tma_load_3d(slot_addr(it, vslot) + k * 4096, &tmV, fb, 64 * k, j0, b);
                     }
-                    if (!pass2 && it + FS_PF < nch)
+                    if (!pass2 && !light && it + FS_PF < nch)
                         for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (it + FS_PF), s, b);
                     free_slots -= nslots(it);
                     ++next_load;
                 }
             };
-            for (int c = 0; c < nch && c < FS_PF; ++c)
+            for (int c = 0; c < nch && c < FS_PF && !light; ++c)
                 for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * c, s, b);
             issue_loads();
             for (int it = 0; it < nit; ++it) {
                 const bool pass2 = it >= nch;
-                if (it == nch && p.prefetch_ahead) {
+                if (it == nch && p.prefetch_ahead && !light) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
@@ -250,7 +266,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         free_slots += ns2;
                     }
                 } else {
-                    free_slots += 3;
+                    free_slots += ns1;
                 }
                 issue_loads();
             }
@@ -374,7 +390,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 tmem_ld2(scol + 8, sacc[0][1], sacc[1][1]);
                 tmem_ld_wait();
             } else {
-                warp_scores2<1>(slot_addr(it, 2), q, t, hq, qf, sacc);
+                warp_scores2<1>(slot_addr(it, pass2 ? 2 : ks1), q, t, hq, qf, sacc);
                 if (keep_s) {
                     tmem_st2(scol, sacc[0][0], sacc[1][0]);
                     tmem_st2(scol + 8, sacc[0][1], sacc[1][1]);
@@ -382,19 +398,21 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             }
 
             // ---------------- combine with FiLM: s' = s(1+gamma)+beta, masked
-            cta_wait(bar(FB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
-            tc_fence_after();
-            float gm[2][2], bt[2][2];
+            float gm[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, bt[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            if (!light) {
+                cta_wait(bar(FB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
+                tc_fence_after();
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const uint32_t fcol = FS_TM_FILM + 32 * (it & 1) + 16 * e;
-                tmem_ld2(tl + fcol + 2 * hq, gm[e][0], gm[e][1]);
-                tmem_ld2(tl + fcol + NH + 2 * hq, bt[e][0], bt[e][1]);
+                for (int e = 0; e < 2; ++e) {
+                    const uint32_t fcol = FS_TM_FILM + 32 * (it & 1) + 16 * e;
+                    tmem_ld2(tl + fcol + 2 * hq, gm[e][0], gm[e][1]);
+                    tmem_ld2(tl + fcol + NH + 2 * hq, bt[e][0], bt[e][1]);
+                }
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (t == 0) mbar_arrive(bar(FB_FILM_EMPTY + (it & 1)));
             }
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (t == 0) mbar_arrive(bar(FB_FILM_EMPTY + (it & 1)));
             const bool mcol = mj[j0 + 8 * q + g8] != 0;
             bool valid[2];
 #pragma unroll
@@ -427,15 +445,20 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 continue;
             }
 
-            // ---------------- pass 2, front of this chunk: normalised coefficients, a buffer p2 & 1
+            // ---------------- pass 2, front of this chunk: normalised coefficients, a buffer p2 & 1;
+            // the edge update takes a (the layer) or s' (the unnormalised variant)
             const int p2 = it - nch;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
+                float ce[2];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
+                for (int hh = 0; hh < 2; ++hh) {
+                    ce[hh] = valid[e] ? sacc[hh][e] : 0.f;
                     sacc[hh][e] = valid[e] ? exp2f((sacc[hh][e] - fm[e][hh]) * LOG2E) * fl[e][hh] : 0.f;
+                    if (!p.unnorm) ce[hh] = sacc[hh][e];
+                }
                 *reinterpret_cast<uint32_t *>(sp + S::A + (p2 & 1) * 8192 + e * 4096 + ns16(L, 2 * hq)) =
-                    pack_bf16(sacc[0][e], sacc[1][e]);
+                    pack_bf16(ce[0], ce[1]);
             }
             sacc[0][2] = sacc[0][3] = sacc[1][2] = sacc[1][3] = 0.f;
             fence_proxy_async_smem();
@@ -492,6 +515,8 @@ cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t
     p.LSE = a.LSE;
     p.status = a.status;
     p.n = d.n;
+    p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
+    p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)sm_count();
     k_fwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), FS_THR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
     return cudaGetLastError();

@@ -66,6 +66,21 @@ bool encode_node_map(CUtensorMap *m, const void *base, int B, int n, int box_row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The backward's published row statistics [B][2][H][n4] fp32 (LSE, then D;
+// n4 = n rounded up to 4 so that rows are 16-byte multiples); box of 32 rows
+// x 8 heads x both statistics of one graph, no swizzle.
+bool encode_rowstat_map(CUtensorMap *m, const void *base, int B, int n, int n4) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)n, NH, 2, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)n4 * 4, (cuuint64_t)NH * n4 * 4, (cuuint64_t)2 * NH * n4 * 4};
+    const cuuint32_t box[4] = {32, NH, 2, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // A row-major [rows, cols] bf16 matrix; box of 64 columns x box_rows rows, 128B-swizzled.
 bool encode_2d(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
     auto enc = get_encode();
@@ -79,26 +94,15 @@ bool encode_2d(CUtensorMap *m, const void *base, int rows, int cols, int box_row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The per-pair a or ds of the backward, [B][H][n][npad] bf16 (npad = n rounded
-// up to 8); box of 32 columns j x 16 rows i x 8 heads, 64B-swizzled.
-bool encode_p_map(CUtensorMap *m, const void *base, int B, int n, int npad) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)n, (cuuint64_t)n, NH, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)npad * 2, (cuuint64_t)n * npad * 2, (cuuint64_t)NH * n * npad * 2};
-    const cuuint32_t box[4] = {32, 16, NH, 1};
-    const cuuint32_t es[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // g_b = y_b Wfy + bf (fp32) for every graph: one warp per graph, lanes split
 // the dy terms and add their 16 sums with shuffles in a fixed order.  The last
-// block writes the four operand images from Wfe and We staged in shared memory.
+// block writes the four operand images from Wfe and We staged in shared memory
+// and zeroes `nzero` ints at `zero_ints` (the backward pair kernel's row-block
+// flags and work-item counter).
 __global__ void __launch_bounds__(256) k_prologue(const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy,
                                                   const __nv_bfloat16 *bf, const __nv_bfloat16 *Wfe,
-                                                  const __nv_bfloat16 *We, float *g, uint8_t *img, int B, int dy) {
+                                                  const __nv_bfloat16 *We, float *g, uint8_t *img, int B, int dy,
+                                                  int *zero_ints, int nzero) {
     const int w = threadIdx.x >> 5, t = threadIdx.x & 31;
     if (blockIdx.x + 1 < gridDim.x) {
         const int b = blockIdx.x * 8 + w;
@@ -133,6 +137,7 @@ __global__ void __launch_bounds__(256) k_prologue(const __nv_bfloat16 *y, const 
         }
         return;
     }
+    for (int e = threadIdx.x; e < nzero; e += blockDim.x) zero_ints[e] = 0;
     __shared__ __nv_bfloat16 sWfe[DE * NF], sWe[NH * DE];
     for (int e = threadIdx.x; e < DE * NF / 8; e += blockDim.x)
         reinterpret_cast<uint4 *>(sWfe)[e] = reinterpret_cast<const uint4 *>(Wfe)[e];
@@ -166,12 +171,12 @@ __global__ void __launch_bounds__(256) k_prologue(const __nv_bfloat16 *y, const 
 }
 
 cudaError_t launch_prologue(const eaga_dims &d, const void *const w[12], const void *y, float *g, uint8_t *img,
-                            cudaStream_t st) {
+                            int *zero, int nzero, cudaStream_t st) {
     const int blocks = (d.B + 7) / 8 + 1;
     k_prologue<<<blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16 *>(y), static_cast<const __nv_bfloat16 *>(w[7]),
         static_cast<const __nv_bfloat16 *>(w[8]), static_cast<const __nv_bfloat16 *>(w[6]),
-        static_cast<const __nv_bfloat16 *>(w[9]), g, img, d.B, d.dy);
+        static_cast<const __nv_bfloat16 *>(w[9]), g, img, d.B, d.dy, zero, nzero);
     return cudaGetLastError();
 }
 

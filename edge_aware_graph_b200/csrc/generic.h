@@ -8,7 +8,10 @@
 namespace eaga {
 
 // Weight order everywhere: Wq bq Wk bk Wv bv Wfe Wfy bf We Wo bo.
+// `variant` is an eaga_variant: the layer, Light Edge (no per-edge FiLM map)
+// or the unnormalised edge update (from the modulated scores s').
 struct FwdArgs {
+    int variant = 0;
     const void *X, *E, *y;
     const uint8_t *M;
     const void *w[12];
@@ -20,6 +23,7 @@ struct FwdArgs {
 };
 
 struct BwdArgs {
+    int variant = 0;
     const void *X, *E, *y;
     const uint8_t *M;
     const void *w[12];

@@ -108,7 +108,8 @@ __device__ __forceinline__ void load_row_consts(float *q, const T *Qrow, float *
                                                 int hd, int de, int H) {
     const int F = 2 * H;
     for (int t = threadIdx.x; t < hd; t += blockDim.x) q[t] = ldf(Qrow + t);
-    for (int t = threadIdx.x; t < de * F; t += blockDim.x) wfe[t] = ldf(Wfe + t);
+    // Wfe == nullptr: no per-edge FiLM map (the Light Edge variant)
+    for (int t = threadIdx.x; t < de * F; t += blockDim.x) wfe[t] = Wfe ? ldf(Wfe + t) : 0.f;
     for (int t = threadIdx.x; t < H * de; t += blockDim.x) we[t] = ldf(We + t);
     for (int t = threadIdx.x; t < F; t += blockDim.x) gl[t] = g[t];
 }
@@ -128,13 +129,15 @@ __device__ __forceinline__ void film_h(const T *e, const float *wfe, const float
 }
 
 // Forward of one row (b,i): modulated scores, masked softmax, O_i, E'_i*, LSE.
+// unnorm: the edge update takes the modulated scores s' (valid pairs) instead of a.
 template <typename T>
 __global__ void __launch_bounds__(NT) k_attn_fwd_row(const T *E, const uint8_t *M, const T *Q, const T *K,
                                                      const T *V, const T *Wfe, const float *g, const T *We,
-                                                     T *O, float *LSE, T *Eout, int n, int de, int H, int dh) {
+                                                     T *O, float *LSE, T *Eout, int n, int de, int H, int dh,
+                                                     int unnorm) {
     extern __shared__ float sm[];
     const int F = 2 * H, hd = H * dh;
-    float *q = sm, *wfe = q + hd, *we = wfe + de * F, *gl = we + H * de, *a = gl + F;
+    float *q = sm, *wfe = q + hd, *we = wfe + de * F, *gl = we + H * de, *a = gl + F, *sps = a + H * n;
     const int b = blockIdx.y, i = blockIdx.x;
     const size_t row = (size_t)b * n + i;
     const uint8_t *mb = M + (size_t)b * n;
@@ -164,6 +167,7 @@ __global__ void __launch_bounds__(NT) k_attn_fwd_row(const T *E, const uint8_t *
                 sp = s * (1.f + gam) + bet;
             }
             a[h * n + j] = sp;
+            if (unnorm) sps[h * n + j] = vj ? sp : 0.f;
         }
     }
     __syncthreads();
@@ -196,8 +200,9 @@ __global__ void __launch_bounds__(NT) k_attn_fwd_row(const T *E, const uint8_t *
     for (int t = threadIdx.x; t < n * de; t += NT) {
         const int j = t / de, c = t % de;
         float acc = ldf(Erow + t);
+        const float *coef = unnorm ? sps : a;
         if (mb[j])
-            for (int h = 0; h < H; ++h) acc = fmaf(a[h * n + j], we[h * de + c], acc);
+            for (int h = 0; h < H; ++h) acc = fmaf(coef[h * n + j], we[h * de + c], acc);
         stf(Eo + t, acc);
     }
 }
@@ -268,17 +273,18 @@ __global__ void __launch_bounds__(NT) k_bwd_dO(const T *dXout, const T *Wo, cons
 }
 
 // Row pass of the backward for row (b,i): a, dA, D_ih, dS', dq_i, dE_i*, and the
-// row's parts of dWfe [de,2H], dWe [H,de], dg [2H].
+// row's parts of dWfe [de,2H], dWe [H,de], dg [2H].  unnorm: the edge path
+// reaches s' directly (D from the node term only, u added to dS', dWe from s').
 template <typename T>
 __global__ void __launch_bounds__(NT) k_attn_bwd_row(const T *E, const uint8_t *M, const T *Q, const T *K,
                                                      const T *V, const float *LSE, const float *dO,
                                                      const T *dEout, const T *Wfe, const float *g, const T *We,
                                                      float *dQ, T *dE, float *Dout, float *parts,
-                                                     size_t part_stride, int n, int de, int H, int dh) {
+                                                     size_t part_stride, int n, int de, int H, int dh, int unnorm) {
     extern __shared__ float sm[];
     const int F = 2 * H, hd = H * dh;
     float *q = sm, *dOi = q + hd, *wfe = dOi + hd, *we = wfe + de * F, *gl = we + H * de;
-    float *A = gl + F, *G = A + H * n, *S = G + H * n, *GM = S + H * n, *D = GM + H * n;
+    float *A = gl + F, *G = A + H * n, *S = G + H * n, *GM = S + H * n, *D = GM + H * n, *SP = D + H;
     const int b = blockIdx.y, i = blockIdx.x;
     const size_t row = (size_t)b * n + i;
     const uint8_t *mb = M + (size_t)b * n;
@@ -304,18 +310,20 @@ __global__ void __launch_bounds__(NT) k_attn_bwd_row(const T *E, const uint8_t *
         const T *kj = K + ((size_t)b * n + j) * hd;
         const T *vv = V + ((size_t)b * n + j) * hd;
         for (int h = 0; h < H; ++h) {
-            float a = 0.f, dA = 0.f, s = 0.f, gam = 0.f;
+            float a = 0.f, dA = 0.f, s = 0.f, gam = 0.f, spv = 0.f;
             if (vj) {
                 float bet;
                 film_h(e, wfe, gl, de, H, h, gam, bet);
                 for (int t = 0; t < dh; ++t) s = fmaf(q[h * dh + t], ldf(kj + h * dh + t), s);
                 s *= rs;
-                a = expf(s * (1.f + gam) + bet - LSE[((size_t)b * H + h) * n + i]);
+                spv = s * (1.f + gam) + bet;
+                a = expf(spv - LSE[((size_t)b * H + h) * n + i]);
                 float u = 0.f, dov = 0.f;
                 for (int c = 0; c < de; ++c) u = fmaf(we[h * de + c], ldf(dep + c), u);
                 for (int t = 0; t < dh; ++t) dov = fmaf(dOi[h * dh + t], ldf(vv + h * dh + t), dov);
-                dA = dov + u;
+                dA = unnorm ? dov : dov + u;
             }
+            if (unnorm) SP[h * n + j] = spv;
             A[h * n + j] = a;
             G[h * n + j] = dA;
             S[h * n + j] = s;
@@ -336,7 +344,13 @@ __global__ void __launch_bounds__(NT) k_attn_bwd_row(const T *E, const uint8_t *
     __syncthreads();
     for (int t = threadIdx.x; t < H * n; t += NT) {
         const int h = t / n;
-        const float dsp = A[t] * (G[t] - D[h]);
+        float dsp = A[t] * (G[t] - D[h]);
+        if (unnorm && mb[t % n]) {       // + u_ij on valid pairs
+            const T *dep = dEp + (size_t)(t % n) * de;
+            float u = 0.f;
+            for (int c = 0; c < de; ++c) u = fmaf(we[h * de + c], ldf(dep + c), u);
+            dsp += u;
+        }
         G[t] = dsp;                    // dbeta
         S[t] = dsp * S[t];             // dgamma
         GM[t] = dsp * (1.f + GM[t]);   // ds
@@ -367,8 +381,9 @@ __global__ void __launch_bounds__(NT) k_attn_bwd_row(const T *E, const uint8_t *
     }
     for (int t = threadIdx.x; t < H * de; t += NT) {
         const int h = t / de, c = t % de;
+        const float *coef = unnorm ? SP : A;
         float acc = 0.f;
-        for (int j = 0; j < n; ++j) acc = fmaf(A[h * n + j], ldf(dEp + (size_t)j * de + c), acc);
+        for (int j = 0; j < n; ++j) acc = fmaf(coef[h * n + j], ldf(dEp + (size_t)j * de + c), acc);
         pWe[t] = acc;
     }
     for (int k = threadIdx.x; k < F; k += NT) {
@@ -385,7 +400,7 @@ __global__ void __launch_bounds__(NT) k_attn_bwd_col(const T *E, const uint8_t *
                                                      const T *V, const float *LSE, const float *dO,
                                                      const T *dEout, const T *Wfe, const float *g, const T *We,
                                                      const float *Dst, float *dK, float *dV,
-                                                     int n, int de, int H, int dh) {
+                                                     int n, int de, int H, int dh, int unnorm) {
     extern __shared__ float sm[];
     const int F = 2 * H, hd = H * dh;
     float *kj = sm, *vj = kj + hd, *wfe = vj + hd, *we = wfe + de * F, *gl = we + H * de;
@@ -420,7 +435,8 @@ __global__ void __launch_bounds__(NT) k_attn_bwd_col(const T *E, const uint8_t *
                 float u = 0.f, dov = 0.f;
                 for (int c = 0; c < de; ++c) u = fmaf(we[h * de + c], ldf(dep + c), u);
                 for (int t = 0; t < dh; ++t) dov = fmaf(dO[ri * hd + h * dh + t], vj[h * dh + t], dov);
-                const float dsp = a * (dov + u - Dst[((size_t)b * H + h) * n + i]);
+                const float D = Dst[((size_t)b * H + h) * n + i];
+                const float dsp = unnorm ? a * (dov - D) + u : a * (dov + u - D);
                 dsv = dsp * (1.f + gam);
             }
             A[h * n + i] = a;
@@ -518,13 +534,13 @@ __global__ void __launch_bounds__(NT) k_xty(const TA *A, const TB *Bm, float *ou
 
 // dWfe, dWe = sums of the per-row parts (row order); dg[b,:] = sum over the graph's rows.
 __global__ void k_reduce_parts(const float *parts, size_t part_stride, int B, int n, int nWfe, int nWe, int F,
-                               float *dWfe, float *dWe, float *dg) {
+                               float *dWfe, float *dWe, float *dg, int zero_wfe) {
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     const int rows = B * n;
     if (t < nWfe) {
         float acc = 0.f;
         for (int r = 0; r < rows; ++r) acc += parts[(size_t)r * part_stride + t];
-        dWfe[t] = acc;
+        dWfe[t] = zero_wfe ? 0.f : acc;     // Light Edge: Wfe is not a parameter
     } else if (t < nWfe + nWe) {
         float acc = 0.f;
         for (int r = 0; r < rows; ++r) acc += parts[(size_t)r * part_stride + t];
@@ -562,13 +578,14 @@ __global__ void k_film_grads(const T *y, const T *Wfy, const float *dg, float *d
 
 // ------------------------------------------------------------------ host side
 
-static inline size_t row_smem_fwd(const eaga_dims &d) {
+// (the unnormalised variant keeps the modulated scores of the row too: H*n more floats)
+static inline size_t row_smem_fwd(const eaga_dims &d, int unnorm = 1) {
     return sizeof(float) * (size_t(d.H) * d.dh + size_t(d.de) * 2 * d.H + size_t(d.H) * d.de + 2 * d.H +
-                            size_t(d.H) * d.n);
+                            size_t(1 + (unnorm ? 1 : 0)) * d.H * d.n);
 }
-static inline size_t row_smem_bwd(const eaga_dims &d) {
+static inline size_t row_smem_bwd(const eaga_dims &d, int unnorm = 1) {
     return sizeof(float) * (2 * size_t(d.H) * d.dh + size_t(d.de) * 2 * d.H + size_t(d.H) * d.de + 2 * d.H +
-                            4 * size_t(d.H) * d.n + d.H);
+                            size_t(4 + (unnorm ? 1 : 0)) * d.H * d.n + d.H);
 }
 static inline size_t col_smem_bwd(const eaga_dims &d) {
     return sizeof(float) * (2 * size_t(d.H) * d.dh + size_t(d.de) * 2 * d.H + size_t(d.H) * d.de + 2 * d.H +
@@ -606,11 +623,13 @@ static cudaError_t forward_t(const eaga_dims &d, const FwdArgs &a, cudaStream_t 
     k_qkv<T><<<(rows + RB - 1) / RB, NT, sq, st>>>(static_cast<const T *>(a.X), W[0], W[1], W[2], W[3], W[4], W[5],
                                                     a.M, Q, K, V, rows, d.dx, hd);
     k_global_film<T><<<d.B, 32, 0, st>>>(static_cast<const T *>(a.y), W[7], W[8], a.g, d.dy, F);
-    const size_t sr = row_smem_fwd(d);
-    EAGA_TRY(set_smem(k_attn_fwd_row<T>, sr));
+    const int unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
+    const T *Wfe = a.variant == EAGA_VARIANT_LIGHT_EDGE ? nullptr : W[6];
+    const size_t sr = row_smem_fwd(d, unnorm);
+    EAGA_TRY(set_smem(k_attn_fwd_row<T>, row_smem_fwd(d)));
     prof_mark(0, 0, st);
-    k_attn_fwd_row<T><<<dim3(d.n, d.B), NT, sr, st>>>(static_cast<const T *>(a.E), a.M, Q, K, V, W[6], a.g, W[9], O,
-                                                       a.LSE, static_cast<T *>(a.Eout), d.n, d.de, d.H, d.dh);
+    k_attn_fwd_row<T><<<dim3(d.n, d.B), NT, sr, st>>>(static_cast<const T *>(a.E), a.M, Q, K, V, Wfe, a.g, W[9], O,
+                                                       a.LSE, static_cast<T *>(a.Eout), d.n, d.de, d.H, d.dh, unnorm);
     prof_mark(0, 1, st);
     const size_t so = sizeof(float) * RB * hd;
     EAGA_TRY(set_smem(k_out_proj<T>, so));
@@ -632,20 +651,22 @@ static cudaError_t backward_t(const eaga_dims &d, const BwdArgs &a, cudaStream_t
     const size_t sd = sizeof(float) * RB * d.dx;
     EAGA_TRY(set_smem(k_bwd_dO<T>, sd));
     k_bwd_dO<T><<<(rows + RB - 1) / RB, NT, sd, st>>>(dXo, W[10], a.M, a.dO, rows, d.dx, hd);
-    const size_t sr = row_smem_bwd(d);
-    EAGA_TRY(set_smem(k_attn_bwd_row<T>, sr));
+    const int unnorm = a.variant == EAGA_VARIANT_UNNORMALISED, light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
+    const T *Wfe = light ? nullptr : W[6];
+    const size_t sr = row_smem_bwd(d, unnorm);
+    EAGA_TRY(set_smem(k_attn_bwd_row<T>, row_smem_bwd(d)));
     const size_t sc = col_smem_bwd(d);
     EAGA_TRY(set_smem(k_attn_bwd_col<T>, sc));
     prof_mark(1, 0, st);
-    k_attn_bwd_row<T><<<dim3(d.n, d.B), NT, sr, st>>>(E, a.M, Q, K, V, a.LSE, a.dO, dEo, W[6], a.g, W[9], a.dQ,
+    k_attn_bwd_row<T><<<dim3(d.n, d.B), NT, sr, st>>>(E, a.M, Q, K, V, a.LSE, a.dO, dEo, Wfe, a.g, W[9], a.dQ,
                                                        static_cast<T *>(a.dE), a.D, a.parts, a.part_stride, d.n,
-                                                       d.de, d.H, d.dh);
-    k_attn_bwd_col<T><<<dim3(d.n, d.B), NT, sc, st>>>(E, a.M, Q, K, V, a.LSE, a.dO, dEo, W[6], a.g, W[9], a.D,
-                                                       a.dK, a.dV, d.n, d.de, d.H, d.dh);
+                                                       d.de, d.H, d.dh, unnorm);
+    k_attn_bwd_col<T><<<dim3(d.n, d.B), NT, sc, st>>>(E, a.M, Q, K, V, a.LSE, a.dO, dEo, Wfe, a.g, W[9], a.D,
+                                                       a.dK, a.dV, d.n, d.de, d.H, d.dh, unnorm);
     prof_mark(1, 1, st);
     const int nWfe = d.de * F, nWe = d.H * d.de, tot = nWfe + nWe + d.B * F;
     k_reduce_parts<<<(tot + 255) / 256, 256, 0, st>>>(a.parts, a.part_stride, d.B, d.n, nWfe, nWe, F, a.dW[6],
-                                                      a.dW[9], a.dg);
+                                                      a.dW[9], a.dg, light);
     const int tf = d.dy * F + F + d.B * d.dy;
     k_film_grads<T><<<(tf + 255) / 256, 256, 0, st>>>(static_cast<const T *>(a.y), W[7], a.dg, a.dW[7], a.dW[8],
                                                       static_cast<T *>(a.dy), d.B, d.dy, F);

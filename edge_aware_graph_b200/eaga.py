@@ -21,7 +21,10 @@ STATUS = {0: "EAGA_OK", 1: "EAGA_ERR_INVALID_ARG", 2: "EAGA_ERR_UNSUPPORTED", 3:
           4: "EAGA_ERR_WORKSPACE", 5: "EAGA_ERR_CUDA", 6: "EAGA_ERR_TIMEOUT"}
 EXPORTED = ("eaga_workspace_size", "eaga_saved_size", "eaga_forward", "eaga_backward",
             "eaga_debug_attention_map", "eaga_get_device_status", "eaga_strerror",
-            "eaga_set_profile_events", "eaga_kernel_launches", "eaga_forward_noalloc", "eaga_debug_wait_probe")
+            "eaga_set_profile_events", "eaga_kernel_launches", "eaga_forward_noalloc", "eaga_debug_wait_probe",
+            "eaga_forward_variant", "eaga_backward_variant")
+# layer variants (eaga_variant): the layer, Light Edge, the unnormalised edge update
+VARIANTS = {"layer": 0, "light_edge": 1, "unnormalised": 2}
 
 
 class Dims(ctypes.Structure):
@@ -59,6 +62,12 @@ def lib():
         L.eaga_backward.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.POINTER(Weights), vp,
                                     vp, vp, vp, vp, vp, ctypes.POINTER(Weights), vp, sz, vp]
         L.eaga_backward.restype = i32
+        L.eaga_forward_variant.argtypes = [ctypes.POINTER(Dims), i32, vp, vp, vp, vp, ctypes.POINTER(Weights),
+                                           vp, vp, vp, vp, sz, vp]
+        L.eaga_forward_variant.restype = i32
+        L.eaga_backward_variant.argtypes = [ctypes.POINTER(Dims), i32, vp, vp, vp, vp, ctypes.POINTER(Weights), vp,
+                                            vp, vp, vp, vp, vp, ctypes.POINTER(Weights), vp, sz, vp]
+        L.eaga_backward_variant.restype = i32
         L.eaga_forward_noalloc.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.POINTER(Weights),
                                            vp, vp, vp, vp]
         L.eaga_forward_noalloc.restype = i32
@@ -147,12 +156,16 @@ def _nbytes(t):
     return 0 if t is None else t.numel() * t.element_size()
 
 
-def forward(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, workspace, stream=None):
+def forward(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, workspace, stream=None, variant: str = "layer"):
+    """eaga_forward (variant "layer"), else eaga_forward_variant."""
     sd = _storage(d)
-    rc = lib().eaga_forward(ctypes.byref(d), _p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd), _p(M, "M", _u8()),
-                            ctypes.byref(_weights(W, sd)), _p(Xout, "Xout", sd), _p(Eout, "Eout", sd),
-                            _p(saved, "saved"), _p(workspace, "workspace"), _nbytes(workspace), _stream(stream))
-    _check(rc, "eaga_forward")
+    args = (_p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd), _p(M, "M", _u8()),
+            ctypes.byref(_weights(W, sd)), _p(Xout, "Xout", sd), _p(Eout, "Eout", sd),
+            _p(saved, "saved"), _p(workspace, "workspace"), _nbytes(workspace), _stream(stream))
+    if variant == "layer":
+        _check(lib().eaga_forward(ctypes.byref(d), *args), "eaga_forward")
+    else:
+        _check(lib().eaga_forward_variant(ctypes.byref(d), VARIANTS[variant], *args), "eaga_forward_variant")
 
 
 def forward_noalloc(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, stream=None):
@@ -164,14 +177,19 @@ def forward_noalloc(d: Dims, X, E, y, M, W: dict, Xout, Eout, saved, stream=None
     _check(rc, "eaga_forward_noalloc")
 
 
-def backward(d: Dims, X, E, y, M, W: dict, saved, dXout, dEout, dX, dE, dy, dW: dict, workspace, stream=None):
+def backward(d: Dims, X, E, y, M, W: dict, saved, dXout, dEout, dX, dE, dy, dW: dict, workspace, stream=None,
+             variant: str = "layer"):
+    """eaga_backward (variant "layer"), else eaga_backward_variant."""
     sd = _storage(d)
-    rc = lib().eaga_backward(ctypes.byref(d), _p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd), _p(M, "M", _u8()),
-                             ctypes.byref(_weights(W, sd)), _p(saved, "saved"), _p(dXout, "dXout", sd),
-                             _p(dEout, "dEout", sd), _p(dX, "dX", sd), _p(dE, "dE", sd), _p(dy, "dy", sd),
-                             ctypes.byref(_weights(dW, _f32(), "dW")), _p(workspace, "workspace"),
-                             _nbytes(workspace), _stream(stream))
-    _check(rc, "eaga_backward")
+    args = (_p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd), _p(M, "M", _u8()),
+            ctypes.byref(_weights(W, sd)), _p(saved, "saved"), _p(dXout, "dXout", sd),
+            _p(dEout, "dEout", sd), _p(dX, "dX", sd), _p(dE, "dE", sd), _p(dy, "dy", sd),
+            ctypes.byref(_weights(dW, _f32(), "dW")), _p(workspace, "workspace"),
+            _nbytes(workspace), _stream(stream))
+    if variant == "layer":
+        _check(lib().eaga_backward(ctypes.byref(d), *args), "eaga_backward")
+    else:
+        _check(lib().eaga_backward_variant(ctypes.byref(d), VARIANTS[variant], *args), "eaga_backward_variant")
 
 
 def debug_attention_map(d: Dims, E, M, W: dict, y, saved, A, stream=None):

@@ -93,11 +93,9 @@ typedef struct {
 } eaga_weight_grads;
 
 /* Bytes of workspace eaga_forward (for_backward = 0) or eaga_backward
- * (for_backward = 1) needs.  The forward's grows as O(B*n*H*dh) + O(B*H)
- * plus the transposed node weights.  On the specialised bf16 path (de = 64,
- * H = 8, dh = 32) the backward's also holds the attention weights a and the
- * score gradients ds of every pair in bf16, 2*B*H*n*roundup8(n) elements:
- * 32 bytes per pair, a quarter of E, so that E and dE' are read once.
+ * (for_backward = 1) needs.  Both grow with the node count only: O(B*n*H*dh)
+ * + O(B*H*n) + fixed-size partial sums, never a per-pair (B*H*n^2) term; no
+ * attention coefficient of any pair is stored in memory.
  * Returns 0 for invalid or unsupported dims. */
 EAGA_API size_t eaga_workspace_size(const eaga_dims *dims, int for_backward);
 
@@ -132,6 +130,44 @@ EAGA_API eaga_status eaga_backward(const eaga_dims *dims,
                           const void *dXout, const void *dEout,
                           void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
                           void *workspace, size_t ws_bytes, void *stream);
+
+/* Ablation variants of the layer (AI-summary page: the method paragraph's
+ * ablation of unnormalised coefficients, and the "Light Edge" bullet):
+ *   EAGA_VARIANT_LAYER         the layer above (eaga_forward, eaga_backward);
+ *   EAGA_VARIANT_LIGHT_EDGE    no per-edge modulation: gamma, beta = y_b Wfy +
+ *                              bf.  Wfe is not read (pass any valid pointer)
+ *                              and its gradient is written as zero (it is not
+ *                              a parameter of that layer); dE = dE'.  On the
+ *                              specialised bf16 path the forward reads E only
+ *                              once (for the residual) and the backward not
+ *                              at all;
+ *   EAGA_VARIANT_UNNORMALISED  the edge update from the unnormalised
+ *                              coefficients, read as the modulated scores:
+ *                              E'_ij = E_ij + sum_h s'^h_ij We[h,:] on valid
+ *                              pairs (E_ij elsewhere); the node path is the
+ *                              layer's.  Its backward: D_i = sum_j a_ij dO_i.v_j,
+ *                              dS'_ij = a_ij (dO_i.v_j - D_i) + u_ij (u_ij =
+ *                              We . dE'_ij on valid pairs), dWe = sum s'^T dE'.
+ * The pages print neither variant's equations; these are this library's
+ * readings.  Arguments, layouts and errors are those of eaga_forward and
+ * eaga_backward; an unknown variant returns EAGA_ERR_INVALID_ARG. */
+typedef enum {
+    EAGA_VARIANT_LAYER = 0,
+    EAGA_VARIANT_LIGHT_EDGE = 1,
+    EAGA_VARIANT_UNNORMALISED = 2
+} eaga_variant;
+
+EAGA_API eaga_status eaga_forward_variant(const eaga_dims *dims, int variant,
+                                          const void *X, const void *E, const void *y, const uint8_t *M,
+                                          const eaga_weights *w,
+                                          void *Xout, void *Eout, void *saved,
+                                          void *workspace, size_t ws_bytes, void *stream);
+EAGA_API eaga_status eaga_backward_variant(const eaga_dims *dims, int variant,
+                                           const void *X, const void *E, const void *y, const uint8_t *M,
+                                           const eaga_weights *w, const void *saved,
+                                           const void *dXout, const void *dEout,
+                                           void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
+                                           void *workspace, size_t ws_bytes, void *stream);
 
 /* Forward without a caller-provided workspace.  The paper has no counterpart
  * of this call; it exists for callers that cannot allocate device memory
