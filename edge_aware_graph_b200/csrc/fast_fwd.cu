@@ -14,19 +14,24 @@
 // ones pass 1 brought into L2 last: E leaves HBM once, E' is written once and
 // the [B,H,n,n] map never leaves the chip.  No CTA waits for another one.
 //
-// Warp roles.  Warps 0..15 compute.  Warp 17 (one thread) keeps a ring of
-// twelve 16 KB shared-memory slots filled with TMA loads (3 slots per pass-1
-// chunk, 4 per pass-2 chunk, so up to four chunks ahead) and stores E' once
-// the compute warps have written it.  Warp 16 (one thread) issues the FiLM
-// MMAs one chunk ahead into a double-buffered TMEM range and the edge-update
-// MMAs once the compute warps have written a.  They meet only on mbarriers.
+// Warp roles.  Warps 0..15 compute, in two groups of eight that take the
+// chunks in turn (group G = W / 8 takes the iterations it = G, G + 2, ...):
+// while one group waits for its chunk's tensor-core products, the other works
+// on the next chunk, so the per-chunk dependency chain (TMA -> FiLM MMA ->
+// softmax -> edge MMA -> residual -> store) of one group overlaps the other's.
+// Warp 17 (one thread) keeps a ring of twelve 16 KB shared-memory slots
+// filled with TMA loads (3 slots per pass-1 chunk, 3 or 4 per pass-2 chunk)
+// and stores E' once the compute warps have written it.  Warp 16 (one thread)
+// issues the FiLM MMAs into the group's TMEM range as soon as the tiles have
+// landed, and the edge-update MMAs once a group has written its a.  They meet
+// only on mbarriers.
 //
 // Pair <-> lane mapping.  E tile s (i = 2ic + s) is loaded as [j][ic][c] so
 // that its 128 rows, the M rows of FiLM MMA s, are the pairs (j = 8q + t/4,
 // i = 2(t%4) + s) of lane t in the warps of quadrant q: the same pair those
 // lanes hold in accumulator register s of their m16n8 score tile S^T[j,i].
 // TMEM lane 32q+t therefore feeds lane t directly.  Compute warp W reads
-// quadrant q = W%4 and handles heads 2(W/4), 2(W/4)+1.
+// quadrant q = W%4 and handles the four heads 4hp..4hp+3, hp = (W/4)%2.
 #include <math.h>
 #include "fast.h"
 #include "fast_common.cuh"
@@ -48,15 +53,15 @@ struct FsSmem {
     static constexpr uint32_t WFE = FS_SLOTS * FS_SLOT;       // Wfe^T [16][64] swizzled (FiLM B)
     static constexpr uint32_t WE = WFE + 2048;                // We^T [64][16] no swizzle (edge-update B)
     static constexpr uint32_t A = WE + 2048;                  // 2 buffers x 2 tiles [128][16] no swizzle (edge-update A)
-    static constexpr uint32_t WST = A + 16384;                // per-quadrant stats [4][8 i][8 h][2] f32
-    static constexpr uint32_t FIN = WST + 2048;               // final m, 1/l [8][8][2]
+    static constexpr uint32_t WST = A + 16384;                // per-(group, quadrant) stats [2][4][8 i][8 h][2] f32
+    static constexpr uint32_t FIN = WST + 4096;               // final LSE [8 i][8 h]
     static constexpr uint32_t G = FIN + 512;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // mask of the graph's nodes [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;                // mbarriers, see below
     static constexpr uint32_t TM = BAR + 8 * 17;              // TMEM base address
     static constexpr uint32_t FAIL = TM + 8;                  // CTA failure flag (a wait ran out)
     static constexpr uint32_t BYTES = TM + 16 + 1024;         // + alignment slack
-    static constexpr uint32_t OPART = 0;                      // [4][8][256] f32 O partials (ring drained)
+    static constexpr uint32_t OPART = 0;                      // [2][4][8][256] f32 O partials (ring drained)
 };
 // mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full[2], edge_full[2], stage_done[4],
 // mma_final (all MMAs of the CTA complete)
@@ -87,10 +92,12 @@ __global__ void __launch_bounds__(FS_THR, 1)
 k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmEo,
              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, FwdParams p) {
     using S = FsSmem;
+    constexpr int GW = NWARP / 2;       // warps per compute group
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
-    const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = (W >> 2) & 3, t = tid & 31, c4 = t & 3, g8 = t >> 2;
+    const int tid = threadIdx.x, W = tid >> 5, t = tid & 31, c4 = t & 3, g8 = t >> 2;
+    const int G = (W >> 3) & 1, q = W & 3, hp = (W >> 2) & 1;   // group, TMEM quadrant, head quad
     const int n = p.n, nch = (n + 31) / 32, nit = 2 * nch;
     const int b = blockIdx.y, i0 = blockIdx.x * TB;
     const uint32_t bars = sbase + S::BAR;
@@ -99,10 +106,10 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     uint8_t *mj = sp + S::MJ;
     volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
 
-    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0.  Its
-    // slots, from slot_base(it) on: pass 1 E(s=0), E(s=1), K (Light Edge: K
-    // alone); pass 2 E(s=0), E(s=1), V when the pass-1 scores stay in TMEM,
-    // else E, E, K, V.
+    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0;
+    // group it & 1 computes it.  Its slots, from slot_base(it) on: pass 1
+    // E(s=0), E(s=1), K (Light Edge: K alone); pass 2 E(s=0), E(s=1), V when
+    // the pass-1 scores stay in TMEM, else E, E, K, V.
     const bool light = p.light != 0;
     const bool keep_s = nch <= FS_KEEP_S_MAX_CHUNKS;
     const int ns1 = light ? 1 : 3, ks1 = light ? 0 : 2;
@@ -111,19 +118,21 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     auto nslots = [&](int it) { return it < nch ? ns1 : ns2; };
     auto slot_base = [&](int it) { return (ns1 * min(it, nch) + ns2 * max(it - nch, 0)) % FS_SLOTS; };
     auto slot_addr = [&](int it, int k) { return sbase + (uint32_t)((slot_base(it) + k) % FS_SLOTS) * FS_SLOT; };
+    // the first pass-2 iteration of group gg
+    auto first_p2 = [&](int gg) { return nch + ((gg - nch) & 1); };
 
     // ---------------- setup: barriers, TMEM, operands
     if (tid == 0) {
         for (int k = 0; k < FB_FILM_FULL; ++k) mbar_init(bar(FB_FULL + k), 1);
         mbar_init(bar(FB_FILM_FULL), 1);
         mbar_init(bar(FB_FILM_FULL + 1), 1);
-        mbar_init(bar(FB_FILM_EMPTY), NWARP);
-        mbar_init(bar(FB_FILM_EMPTY + 1), NWARP);
-        mbar_init(bar(FB_A_FULL), NWARP);
-        mbar_init(bar(FB_A_FULL + 1), NWARP);
+        mbar_init(bar(FB_FILM_EMPTY), GW);
+        mbar_init(bar(FB_FILM_EMPTY + 1), GW);
+        mbar_init(bar(FB_A_FULL), GW);
+        mbar_init(bar(FB_A_FULL + 1), GW);
         mbar_init(bar(FB_EDGE_FULL), 1);
         mbar_init(bar(FB_EDGE_FULL + 1), 1);
-        for (int k = 0; k < 4; ++k) mbar_init(bar(FB_STAGE_DONE + k), NWARP);
+        for (int k = 0; k < 4; ++k) mbar_init(bar(FB_STAGE_DONE + k), GW);
         mbar_init(bar(FB_MMA_FINAL), 1);
         fence_mbar_init();
         *fail = 0;
@@ -145,10 +154,10 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
 
     if (W == NWARP) {
-        // ================= MMA issuer: FiLM one chunk ahead, edge update on demand
+        // ================= MMA issuer: FiLM as tiles land, edge updates per group on demand
         if (t == 0) {
             const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_e = idesc_bf16_f32(128, DE);
-            auto issue_film = [&](int it) {
+            auto issue_film = [&](int it) {   // into the TMEM range of group it & 1
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
@@ -161,21 +170,22 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
                 mma_commit(bar(FB_FILM_FULL + (it & 1)));
             };
-            auto issue_edge = [&](int p2) {   // pass-2 chunk p2: a buffer and TMEM buffer p2 & 1
+            auto issue_edge = [&](int gg) {   // group gg's a buffer -> its TMEM buffer
                 tc_fence_after();
-                const uint32_t ab = S::A + (p2 & 1) * 8192, eb = FS_TM_EDGE + 128 * (p2 & 1);
+                const uint32_t ab = S::A + gg * 8192, eb = FS_TM_EDGE + 128 * gg;
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
                     mma_bf16_ss(tmem + eb + 64 * e, smem_desc(sbase + ab + e * 4096, 128, 256, LAYOUT_NONE),
                                 smem_desc(sbase + S::WE, 128, 256, LAYOUT_NONE), idesc_e, 0);
-                mma_commit(bar(FB_EDGE_FULL + (p2 & 1)));
+                mma_commit(bar(FB_EDGE_FULL + gg));
             };
-            // issue whichever product is ready first: FiLM of the next chunk (its
-            // tiles landed, its TMEM buffer released) or the edge update of the
-            // chunk whose a the compute warps have written
-            int next_film = light ? nit : 0, next_edge = nch;   // Light Edge: no FiLM products
+            // issue whichever product is ready: FiLM of the next chunk (its tiles
+            // landed, its group's TMEM range released) or the edge update of a
+            // group whose a the compute warps have written
+            int next_film = light ? nit : 0;                 // Light Edge: no FiLM products
+            int next_edge[2] = {first_p2(0), first_p2(1)};
             uint32_t polls = 0;
-            while ((next_film < nit || next_edge < nit) && !*fail) {
+            while ((next_film < nit || next_edge[0] < nit || next_edge[1] < nit) && !*fail) {
                 bool progressed = false;
                 if (next_film < nit &&
                     mbar_test_wait(bar(FB_FULL + next_film % FS_NFULL), (next_film / FS_NFULL) & 1) &&
@@ -184,15 +194,18 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     issue_film(next_film++);
                     progressed = true;
                 }
-                if (next_edge < nit && next_edge < next_film &&
-                    mbar_test_wait(bar(FB_A_FULL + ((next_edge - nch) & 1)), ((next_edge - nch) >> 1) & 1)) {
-                    issue_edge(next_edge - nch);
-                    ++next_edge;
-                    progressed = true;
+#pragma unroll
+                for (int gg = 0; gg < 2; ++gg) {
+                    const int it = next_edge[gg];
+                    if (it < nit && it < next_film &&
+                        mbar_test_wait(bar(FB_A_FULL + gg), ((it - nch) >> 1) & 1)) {
+                        issue_edge(gg);
+                        next_edge[gg] += 2;
+                        progressed = true;
+                    }
                 }
-                // idle: back off after a few polls, so that this thread does not
-                // take issue slots from the compute warps of its SM sub-partition;
-                // a wait that makes no progress for 2^24 polls gives up
+                // idle: back off after a few polls; a wait that makes no progress
+                // for 2^24 polls gives up
                 if (progressed) {
                     polls = 0;
                 } else {
@@ -217,8 +230,13 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             // pass-2 reads and the E' stores are not read again
             const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
             int next_load = 0, free_slots = FS_SLOTS;
+            int consumed = 0;   // iterations whose stage completion this thread has taken
+            // at most FS_NFULL iterations in flight: a load barrier is re-armed
+            // only after its previous iteration completed (Light Edge takes one
+            // slot per pass-1 chunk, so the slots alone would allow twelve)
             auto issue_loads = [&]() {
-                while (next_load < nit && nslots(next_load) <= free_slots && !*fail) {
+                while (next_load < nit && next_load < consumed + FS_NFULL && nslots(next_load) <= free_slots &&
+                       !*fail) {
                     const int it = next_load, j0 = 32 * chunk_of(it);
                     const bool pass2 = it >= nch;
                     const uint32_t fb = bar(FB_FULL + it % FS_NFULL);
@@ -243,6 +261,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             for (int c = 0; c < nch && c < FS_PF && !light; ++c)
                 for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * c, s, b);
             issue_loads();
+            // stage completions arrive in iteration order within each group;
+            // the two groups' iterations interleave, so they are taken in order
+            int pending = 0;                 // pass-2 stores not yet known to have read their slots
             for (int it = 0; it < nit; ++it) {
                 const bool pass2 = it >= nch;
                 if (it == nch && p.prefetch_ahead && !light) {
@@ -255,15 +276,17 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     }
                 }
                 if (!cta_wait(bar(FB_STAGE_DONE + (it & 3)), (it >> 2) & 1, fail, p.status)) continue;
+                consumed = it + 1;
                 if (pass2) {
                     const int j0 = 32 * chunk_of(it);
                     tma_store_5d_hint(&tmEo, slot_addr(it, 0), 0, i0 / 2, j0, 0, b, drop_l2);
                     tma_store_5d_hint(&tmEo, slot_addr(it, 1), 0, i0 / 2, j0, 1, b, drop_l2);
                     tma_store_commit();
                     // the previous pass-2 chunk's slots are free once its store has read them
-                    if (it > nch) {
+                    if (++pending > 1) {
                         tma_store_wait_read1();
                         free_slots += ns2;
+                        --pending;
                     }
                 } else {
                     free_slots += ns1;
@@ -278,135 +301,54 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         __syncwarp();
         named_bar_sync(2, FS_THR);   // the ring is drained: the compute warps may reuse it
     } else {
-        // ================= compute warps
+        // ================= compute warps: group G, quadrant q, heads 4hp..4hp+3
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
         const float rs = rsqrtf((float)DH);
         const uint32_t L = 32 * q + t;
-        uint32_t qf[2][2][2];
-        load_frags2(p.Q, b, n, i0, hq, g8, c4, qf);
-        // the thread's two rows i = i0 + 2c4 + s (s = 0, 1)
+        const int hqa = 2 * hp, hqb = 2 * hp + 1;     // the two head pairs (helpers take pairs)
+        uint32_t qfa[2][2][2], qfb[2][2][2];
+        load_frags2(p.Q, b, n, i0, hqa, g8, c4, qfa);
+        load_frags2(p.Q, b, n, i0, hqb, g8, c4, qfb);
+        // the thread's two rows i = i0 + 2c4 + e (e = 0, 1)
         const bool mrow[2] = {i0 + 2 * c4 < n && p.M[(size_t)b * n + i0 + 2 * c4] != 0,
                               i0 + 2 * c4 + 1 < n && p.M[(size_t)b * n + i0 + 2 * c4 + 1] != 0};
-        float rm[2][2], rl[2][2];               // running max / sum [s][hh]
-        float fm[2][2], fl[2][2];               // final max, 1/sum [s][hh]
-        float oacc[2][2][4];
-#pragma unroll
-        for (int s = 0; s < 2; ++s)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                rm[s][hh] = -INFINITY;
-                rl[s][hh] = 0.f;
-                fm[s][hh] = -INFINITY;
-                fl[s][hh] = 0.f;
-            }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int x = 0; x < 4; ++x) oacc[hh][mt][x] = 0.f;
 
-        // E' = E + a We of pass-2 chunk it, in place (the TMA warp stores it)
-        auto edge_residual = [&](int it) {
-            const int p2 = it - nch;
-            cta_wait(bar(FB_EDGE_FULL + (p2 & 1)), (p2 >> 1) & 1, fail, p.status);
-            tc_fence_after();
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float dv[16];
-                tmem_ld16(tl + FS_TM_EDGE + 128 * (p2 & 1) + 64 * e + 16 * hq, dv);
-                tmem_ld_wait();
-                add_residual16(sp + (slot_addr(it, e) - sbase) + L * 128, L, hq, dv);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
-        };
-        for (int it = 0; it < nit; ++it) {
+        // s' of iteration it for the thread's 2 pairs x 4 heads: sx[k][e] with
+        // k = 2 * pair + hh (heads hqa: k = 0, 1; hqb: k = 2, 3), -inf where invalid
+        auto scores = [&](int it, bool pass2, float (&sx)[4][2], bool (&valid)[2]) {
             const int j0 = 32 * chunk_of(it);
-            const bool pass2 = it >= nch;
-
-            if (it == nch) {
-                // ---------------- end of pass 1: statistics over lanes, then quadrants
-                tmem_st_wait();
-                float *wst = reinterpret_cast<float *>(sp + S::WST);
-                float *fin = reinterpret_cast<float *>(sp + S::FIN);
-#pragma unroll
-                for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float m = rm[s2][hh], l = rl[s2][hh];
-#pragma unroll
-                        for (int o = 4; o < 32; o <<= 1) {
-                            const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-                            const float lo = __shfl_xor_sync(0xffffffffu, l, o);
-                            const float mn = fmaxf(m, mo);
-                            l = (mn == -INFINITY) ? 0.f
-                                                  : l * exp2f((m - mn) * LOG2E) + lo * exp2f((mo - mn) * LOG2E);
-                            m = mn;
-                        }
-                        if (g8 == 0) {
-                            const int il = 2 * c4 + s2, h = 2 * hq + hh;
-                            wst[((q * 8 + il) * 8 + h) * 2 + 0] = m;
-                            wst[((q * 8 + il) * 8 + h) * 2 + 1] = l;
-                        }
-                    }
-                named_bar_sync(1, NTHR);
-                if (tid < 64) {
-                    float m = -INFINITY;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) m = fmaxf(m, wst[(k * 64 + tid) * 2]);
-                    float l = 0.f;
-                    if (m != -INFINITY)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const float mk = wst[(k * 64 + tid) * 2];
-                            if (mk != -INFINITY) l += wst[(k * 64 + tid) * 2 + 1] * exp2f((mk - m) * LOG2E);
-                        }
-                    fin[tid * 2] = m;
-                    fin[tid * 2 + 1] = (l > 0.f) ? 1.f / l : 0.f;
-                    const int il = tid >> 3, h = tid & 7;
-                    if (i0 + il < n)
-                        p.LSE[((size_t)b * NH + h) * n + i0 + il] = (m == -INFINITY) ? -INFINITY : m + logf(l);
-                }
-                named_bar_sync(1, NTHR);
-#pragma unroll
-                for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int il = 2 * c4 + s2, h = 2 * hq + hh;
-                        fm[s2][hh] = fin[(il * 8 + h) * 2];
-                        fl[s2][hh] = fin[(il * 8 + h) * 2 + 1];
-                    }
-            }
-
-            // ---------------- scores S^T = K Q^T on warp MMAs (2 heads per warp)
             cta_wait(bar(FB_FULL + it % FS_NFULL), (it / FS_NFULL) & 1, fail, p.status);
-            float sacc[2][4];
-            const uint32_t scol = tl + FS_TM_S + 16 * chunk_of(it) + 2 * hq;
+            float sa[2][4], sb[2][4];
+            const uint32_t scol = tl + FS_TM_S + 16 * chunk_of(it);
             if (pass2 && keep_s) {
-                tmem_ld2(scol, sacc[0][0], sacc[1][0]);
-                tmem_ld2(scol + 8, sacc[0][1], sacc[1][1]);
+                tmem_ld2(scol + 2 * hqa, sa[0][0], sa[1][0]);
+                tmem_ld2(scol + 2 * hqa + 8, sa[0][1], sa[1][1]);
+                tmem_ld2(scol + 2 * hqb, sb[0][0], sb[1][0]);
+                tmem_ld2(scol + 2 * hqb + 8, sb[0][1], sb[1][1]);
                 tmem_ld_wait();
             } else {
-                warp_scores2<1>(slot_addr(it, pass2 ? 2 : ks1), q, t, hq, qf, sacc);
+                const uint32_t ks = slot_addr(it, pass2 ? 2 : ks1);
+                warp_scores2<1>(ks, q, t, hqa, qfa, sa);
+                warp_scores2<1>(ks, q, t, hqb, qfb, sb);
                 if (keep_s) {
-                    tmem_st2(scol, sacc[0][0], sacc[1][0]);
-                    tmem_st2(scol + 8, sacc[0][1], sacc[1][1]);
+                    tmem_st2(scol + 2 * hqa, sa[0][0], sa[1][0]);
+                    tmem_st2(scol + 2 * hqa + 8, sa[0][1], sa[1][1]);
+                    tmem_st2(scol + 2 * hqb, sb[0][0], sb[1][0]);
+                    tmem_st2(scol + 2 * hqb + 8, sb[0][1], sb[1][1]);
                 }
             }
-
-            // ---------------- combine with FiLM: s' = s(1+gamma)+beta, masked
-            float gm[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, bt[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            // FiLM of the pair: gamma, beta of the four heads
+            float gm[2][4] = {}, bt[2][4] = {};
             if (!light) {
                 cta_wait(bar(FB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
                 tc_fence_after();
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const uint32_t fcol = FS_TM_FILM + 32 * (it & 1) + 16 * e;
-                    tmem_ld2(tl + fcol + 2 * hq, gm[e][0], gm[e][1]);
-                    tmem_ld2(tl + fcol + NH + 2 * hq, bt[e][0], bt[e][1]);
+                    const uint32_t fcol = FS_TM_FILM + 32 * (it & 1) + 16 * e + 4 * hp;
+                    tmem_ld2(tl + fcol, gm[e][0], gm[e][1]);
+                    tmem_ld2(tl + fcol + 2, gm[e][2], gm[e][3]);
+                    tmem_ld2(tl + fcol + NH, bt[e][0], bt[e][1]);
+                    tmem_ld2(tl + fcol + NH + 2, bt[e][2], bt[e][3]);
                 }
                 tmem_ld_wait();
                 tc_fence_before();
@@ -414,69 +356,157 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 if (t == 0) mbar_arrive(bar(FB_FILM_EMPTY + (it & 1)));
             }
             const bool mcol = mj[j0 + 8 * q + g8] != 0;
-            bool valid[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 valid[e] = mcol && mrow[e];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int h = 2 * hq + hh;
-                    const float gam = gm[e][hh] + g[h], bet = bt[e][hh] + g[NH + h];
-                    const float sv = sacc[hh][e] * rs * (1.f + gam) + bet;
-                    sacc[hh][e] = valid[e] ? sv : -INFINITY;
+                for (int k = 0; k < 4; ++k) {
+                    const int h = 4 * hp + k;
+                    const float raw = k < 2 ? sa[k][e] : sb[k - 2][e];
+                    const float sv = raw * rs * (1.f + gm[e][k] + g[h]) + bt[e][k] + g[NH + h];
+                    sx[k][e] = valid[e] ? sv : -INFINITY;
                 }
             }
+        };
 
-            if (!pass2) {
-                // running statistics (online softmax): one value per (row, head) and chunk
+        // ======== pass 1: running (max, sum) per (row, head) over the group's chunks
+        float lse[2][4];        // after pass 1: the row statistics LSE = m + log l, per [e][k]
+        {
+            float rm[2][4], rl[2][4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    rm[e][k] = -INFINITY;
+                    rl[e][k] = 0.f;
+                }
+            for (int it = G; it < nch; it += 2) {
+                float sx[4][2];
+                bool valid[2];
+                scores(it, false, sx, valid);
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const float x = sacc[hh][e];
-                        const float mn = fmaxf(rm[e][hh], x);
+                    for (int k = 0; k < 4; ++k) {
+                        const float x = sx[k][e];
+                        const float mn = fmaxf(rm[e][k], x);
                         if (mn != -INFINITY) {
-                            rl[e][hh] = rl[e][hh] * exp2f((rm[e][hh] - mn) * LOG2E) + exp2f((x - mn) * LOG2E);
-                            rm[e][hh] = mn;
+                            rl[e][k] = rl[e][k] * exp2f((rm[e][k] - mn) * LOG2E) + exp2f((x - mn) * LOG2E);
+                            rm[e][k] = mn;
                         }
                     }
                 __syncwarp();
                 if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
-                continue;
             }
+            // ---------------- end of pass 1: statistics over lanes, then (group, quadrant)
+            tmem_st_wait();
+            float *wst = reinterpret_cast<float *>(sp + S::WST);
+            float *fin = reinterpret_cast<float *>(sp + S::FIN);
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float m = rm[e][k], l = rl[e][k];
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) {
+                        const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+                        const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+                        const float mn = fmaxf(m, mo);
+                        l = (mn == -INFINITY) ? 0.f : l * exp2f((m - mn) * LOG2E) + lo * exp2f((mo - mn) * LOG2E);
+                        m = mn;
+                    }
+                    if (g8 == 0) {
+                        const int il = 2 * c4 + e, h = 4 * hp + k;
+                        wst[(((G * 4 + q) * 8 + il) * 8 + h) * 2 + 0] = m;
+                        wst[(((G * 4 + q) * 8 + il) * 8 + h) * 2 + 1] = l;
+                    }
+                }
+            named_bar_sync(1, NTHR);
+            if (tid < 64) {
+                float m = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) m = fmaxf(m, wst[(k * 64 + tid) * 2]);
+                float l = 0.f;
+                if (m != -INFINITY)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float mk = wst[(k * 64 + tid) * 2];
+                        if (mk != -INFINITY) l += wst[(k * 64 + tid) * 2 + 1] * exp2f((mk - m) * LOG2E);
+                    }
+                const float v = (m == -INFINITY) ? -INFINITY : m + logf(l);
+                fin[tid] = v;
+                const int il = tid >> 3, h = tid & 7;
+                if (i0 + il < n) p.LSE[((size_t)b * NH + h) * n + i0 + il] = v;
+            }
+            named_bar_sync(1, NTHR);
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) lse[e][k] = fin[(2 * c4 + e) * 8 + 4 * hp + k];
+        }
 
-            // ---------------- pass 2, front of this chunk: normalised coefficients, a buffer p2 & 1;
-            // the edge update takes a (the layer) or s' (the unnormalised variant)
-            const int p2 = it - nch;
+        // ======== pass 2: normalised a, O += a V, the edge update, E' = E + a We
+        float oa[2][2][4], ob[2][2][4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) oa[hh][mt][x] = ob[hh][mt][x] = 0.f;
+        for (int it = first_p2(G); it < nit; it += 2) {
+            float sx[4][2];
+            bool valid[2];
+            scores(it, true, sx, valid);
+            // a (for O) and the edge update's coefficient (a, or s' when unnormalised)
+            float pa[2][4], pb[2][4];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                float ce[2];
+                float ce[4];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    ce[hh] = valid[e] ? sacc[hh][e] : 0.f;
-                    sacc[hh][e] = valid[e] ? exp2f((sacc[hh][e] - fm[e][hh]) * LOG2E) * fl[e][hh] : 0.f;
-                    if (!p.unnorm) ce[hh] = sacc[hh][e];
+                for (int k = 0; k < 4; ++k) {
+                    const float a = valid[e] ? exp2f((sx[k][e] - lse[e][k]) * LOG2E) : 0.f;
+                    ce[k] = p.unnorm ? (valid[e] ? sx[k][e] : 0.f) : a;
+                    if (k < 2) pa[k][e] = a; else pb[k - 2][e] = a;
                 }
-                *reinterpret_cast<uint32_t *>(sp + S::A + (p2 & 1) * 8192 + e * 4096 + ns16(L, 2 * hq)) =
-                    pack_bf16(ce[0], ce[1]);
+                uint8_t *arow = sp + S::A + G * 8192 + e * 4096;
+                *reinterpret_cast<uint32_t *>(arow + ns16(L, 4 * hp)) = pack_bf16(ce[0], ce[1]);
+                *reinterpret_cast<uint32_t *>(arow + ns16(L, 4 * hp + 2)) = pack_bf16(ce[2], ce[3]);
             }
-            sacc[0][2] = sacc[0][3] = sacc[1][2] = sacc[1][3] = 0.f;
+            pa[0][2] = pa[0][3] = pa[1][2] = pa[1][3] = 0.f;
+            pb[0][2] = pb[0][3] = pb[1][2] = pb[1][3] = 0.f;
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (t == 0) mbar_arrive(bar(FB_A_FULL + (p2 & 1)));
+            if (t == 0) mbar_arrive(bar(FB_A_FULL + G));
 
-            // ---------------- O += a V on warp MMAs (overlaps the edge MMAs)
-            warp_contract2<1, true>(slot_addr(it, vslot), q, t, hq, sacc, oacc);
+            // O += a V on warp MMAs (overlaps the edge MMA)
+            const uint32_t vs = slot_addr(it, vslot);
+            warp_contract2<1, true>(vs, q, t, hqa, pa, oa);
+            warp_contract2<1, true>(vs, q, t, hqb, pb, ob);
 
-            // ---------------- back of the previous chunk, whose edge update ran meanwhile
-            if (p2 > 0) edge_residual(it - 1);
+            // E' = E + (a We), in place (the TMA warp stores it)
+            cta_wait(bar(FB_EDGE_FULL + G), ((it - nch) >> 1) & 1, fail, p.status);
+            tc_fence_after();
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float dv[16];
+                    tmem_ld16(tl + FS_TM_EDGE + 128 * G + 64 * e + 32 * hp + 16 * half, dv);
+                    tmem_ld_wait();
+                    add_residual16(sp + (slot_addr(it, e) - sbase) + L * 128, L, 2 * hp + half, dv);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
         }
-        if (nit > nch) edge_residual(nit - 1);
 
-        // ---------------- O: sum over the quadrant warps (in the drained ring)
+        // ---------------- O: sum over the (group, quadrant) warps (in the drained ring)
         named_bar_sync(2, FS_THR);
-        store_quadrant_part(sp, S::OPART, oacc, q, hq, t);
+        store_quadrant_part(sp, S::OPART + G * 32768, oa, q, hqa, t);
+        store_quadrant_part(sp, S::OPART + G * 32768, ob, q, hqb, t);
         named_bar_sync(1, NTHR);
         const float *part = reinterpret_cast<const float *>(sp + S::OPART);
         for (int x = tid; x < TB * HD / 2; x += NTHR) {
@@ -484,7 +514,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             if (i0 + il >= n) continue;
             float o0 = 0.f, o1 = 0.f;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 8; ++k) {
                 o0 += part[k * TB * HD + il * HD + d];
                 o1 += part[k * TB * HD + il * HD + d + 1];
             }
