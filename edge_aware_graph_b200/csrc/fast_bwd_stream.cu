@@ -73,7 +73,7 @@ struct BsSmem {
     static constexpr uint32_t G = WDG + 256;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // node mask [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;
-    static constexpr uint32_t TM = BAR + 8 * 16;              // TMEM base address
+    static constexpr uint32_t TM = BAR + 8 * 18;              // TMEM base address
     static constexpr uint32_t FAIL = TM + 4;                  // CTA failure flag (a wait ran out)
     static constexpr uint32_t ITEM = TM + 8;                  // this CTA's work item
     static constexpr uint32_t STAB = TM + 16;                 // slot table [4 iterations][8] u8
@@ -83,9 +83,10 @@ struct BsSmem {
     // at the end, in the drained ring: dk and dv quadrant sums [4][8][256] f32 (32 KB each)
     static constexpr uint32_t KPART = 0, VPART = 32768;
 };
-// mbarriers: full[4], film_full[2], film_empty[2], df_full, de_full, stage_done[4], mma_final
+// mbarriers: full[4], film_full[2], film_empty[2], df_full, de_full, stage_done[4], mma_final,
+// wg_done[2] (the weight-gradient products of pass-2 chunk p2, by p2 & 1)
 constexpr int BB_FULL = 0, BB_FILM_FULL = 4, BB_FILM_EMPTY = 6, BB_DF_FULL = 8, BB_DE_FULL = 9,
-              BB_STAGE_DONE = 10, BB_MMA_FINAL = 14;
+              BB_STAGE_DONE = 10, BB_MMA_FINAL = 14, BB_WG_DONE = 15;
 
 // TMEM: FiLM 0..63 and u 64..127 (two buffers each), dE 128..255, kept S / dP
 // 256..479 (32 per chunk), and at 480 the weight-gradient accumulator
@@ -115,6 +116,7 @@ struct BwdStreamParams {
     const float *LSE, *g;
     const uint8_t *img, *M;
     __nv_bfloat16 *dQ, *dK, *dV;   // [B,n,256] out (dQ and dK scaled by 1/sqrt(dh))
+    __nv_bfloat16 *dE;       // [B,n,n,64] out
     float *rparts;           // [graph * row block][RPART] out
     float *DL;               // [B][LSE, D][H][n4]: LSE and D of every row, published by its row block
     int *flags;              // [graph * row block]: 1 once that row block's D is published (0 at launch)
@@ -132,7 +134,7 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 __global__ void __launch_bounds__(BS_THR, 1)
 k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmDEp,
-             const __grid_constant__ CUtensorMap tmDE, const __grid_constant__ CUtensorMap tmK,
+             const __grid_constant__ CUtensorMap tmK,
              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmEt,
              const __grid_constant__ CUtensorMap tmDEpt, const __grid_constant__ CUtensorMap tmQ,
              const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmDL,
@@ -183,6 +185,8 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         mbar_init(bar(BB_DE_FULL), 1);
         for (int k = 0; k < 4; ++k) mbar_init(bar(BB_STAGE_DONE + k), NWARP);
         mbar_init(bar(BB_MMA_FINAL), 1);
+        mbar_init(bar(BB_WG_DONE), 1);
+        mbar_init(bar(BB_WG_DONE + 1), 1);
         fence_mbar_init();
         *fail = 0;
     }
@@ -236,6 +240,8 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         mma_bf16_ss(tmem + BS_TM_DE + 64 * e,
                                     smem_desc(sbase + S::DA + e * 8192, 128, 512, LAYOUT_NONE),
                                     smem_desc(sbase + S::IMG + 4096, 128, 256, LAYOUT_NONE), idesc_d, 0);
+                // dE alone is on the compute warps' path: its own completion
+                mma_commit(bar(BB_DE_FULL));
                 // [dWfe | .] and [. | dWe^T] in one product: A = the E tile and the dE' tile read
                 // MN-major as the two 64-channel atoms of M = 128 (64 c per 128-byte swizzled row,
                 // 8-row groups 1024 B apart; the second atom one slot distance further: the
@@ -252,7 +258,8 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                                     smem_desc(sbase + S::DA + e * 8192 + ks * 1024, 512, 128, LAYOUT_NONE), idesc_w, acc);
                     }
                 }
-                mma_commit(bar(BB_DE_FULL));
+                // the tiles (E, dE', [df | a]) may be reused once these completed
+                mma_commit(bar(BB_WG_DONE + ((it - nch) & 1)));
             };
             // issue whichever product is ready first: FiLM/u of the next chunk
             // (its tiles landed, its TMEM buffer released) or dE of the pass-2
@@ -296,13 +303,12 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         if (t == 0) {
             // E and dE' tiles loaded in pass 1 are read again in pass 2: keep
             // them in L2; pass-2 reads stay at the normal priority (the column
-            // pass of other CTAs reads the same pairs); pass-3 reads and the dE
-            // stores are not read again
+            // pass of other CTAs reads the same pairs); pass-3 reads are not
+            // read again
             const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
-            // a pass-2 chunk's E, K (and V) slots are free once the compute
-            // warps are done with it; its dE' slots once the dE store has read them
+            // a chunk's slots are free once the compute warps are done with it
+            // (and, in pass 2, its weight-gradient products have read the tiles)
             uint32_t free_mask = (1u << BS_SLOTS) - 1u;
-            uint32_t prev_d = 0;          // dE' slots of the previous pass-2 chunk
             int next_load = 0;
             auto release = [&](int it, int k) { free_mask |= 1u << stab[(it % BS_NFULL) * 8 + k]; };
             // D of the row blocks of pass-3 chunk c published by their CTAs?
@@ -397,30 +403,13 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
                 if (!cta_wait(bar(BB_STAGE_DONE + (it & 3)), (it >> 2) & 1, fail, p.status)) continue;
                 if (ps == 2) {
-                    const int j0 = 32 * chunk_of(it);
-                    tma_store_5d_hint(&tmDE, slot_addr(it, 2), 0, i0 / 2, j0, 0, b, drop_l2);
-                    tma_store_5d_hint(&tmDE, slot_addr(it, 3), 0, i0 / 2, j0, 1, b, drop_l2);
-                    tma_store_commit();
-                    release(it, 0);
-                    release(it, 1);
-                    release(it, 4);
-                    if (!keep) release(it, 5);
-                    if (it > nch) {
-                        tma_store_wait_read1();
-                        free_mask |= prev_d;
-                    }
-                    prev_d = (1u << stab[(it % BS_NFULL) * 8 + 2]) | (1u << stab[(it % BS_NFULL) * 8 + 3]);
-                    if (it == 2 * nch - 1) {   // the last dE store: its slots come back for pass 3
-                        tma_store_wait_read0();
-                        free_mask |= prev_d;
-                        prev_d = 0;
-                    }
-                } else {
-                    for (int k = 0; k < 6; ++k) release(it, k);
+                    // the chunk's tiles are read by its weight-gradient products until these complete
+                    const int p2 = it - nch;
+                    if (!cta_wait(bar(BB_WG_DONE + (p2 & 1)), (p2 >> 1) & 1, fail, p.status)) continue;
                 }
+                for (int k = 0; k < nslots(it); ++k) release(it, k);
                 issue_loads(-1);
             }
-            tma_store_wait_read0();
             if (*fail)   // loads already issued land before the CTA's shared memory is released
                 for (int it = max(next_load - BS_NFULL, 0); it < next_load; ++it)
                     mbar_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1);
@@ -577,7 +566,9 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     continue;
                 }
 
-                // ---------------- pass 2: dS', df and a tiles for the tensor cores / warp MMAs
+                // ---------------- pass 2: dS', df and a tiles for the tensor cores / warp MMAs;
+                // the previous chunk's weight-gradient products read the tile until they complete
+                if (it > nch) cta_wait(bar(BB_WG_DONE + ((it - nch - 1) & 1)), ((it - nch - 1) >> 1) & 1, fail, p.status);
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float dgam[2], dbet[2];
@@ -606,23 +597,33 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 // ---------------- dq += ds K (warp MMAs; overlaps the tensor-core products)
                 warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, da, qacc);
 
-                // ---------------- dE = dE' + df Wfe^T, in place (the TMA warp stores it)
+                // ---------------- dE = dE' + df Wfe^T (Light Edge: dE = dE'), written from registers:
+                // the dE' tile stays as loaded for the weight-gradient product that reads it
                 cta_wait(bar(BB_DE_FULL), (it - nch) & 1, fail, p.status);
                 tc_fence_after();
-                if (!light)   // Light Edge: dE = dE', the tile is stored as loaded
+                {
+                    const int j = j0 + 8 * q + g8;
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         float dv[16];
-                        tmem_ld16(tl + BS_TM_DE + 64 * e + 16 * hq, dv);
-                        tmem_ld_wait();
-                        add_residual16(sp + (slot_addr(it, 2 + e) - sbase) + L * 128, L, hq, dv);
+                        if (!light) {
+                            tmem_ld16(tl + BS_TM_DE + 64 * e + 16 * hq, dv);
+                            tmem_ld_wait();
+                        }
+                        const int i = i0 + 2 * c4 + e;
+                        if (i < n && j < n)
+                            residual16_to_global(sp + (slot_addr(it, 2 + e) - sbase) + L * 128, L, hq, dv, !light,
+                                                 p.dE + ((((size_t)b * n + i) * n + j) * DE + 16 * hq));
                     }
-                fence_proxy_async_smem();
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
             }
 
+            // the last chunk's weight-gradient products complete before the tile and the
+            // accumulator are read
+            cta_wait(bar(BB_WG_DONE + ((nch - 1) & 1)), ((nch - 1) >> 1) & 1, fail, p.status);
             // ---------------- row-block results: dq through the (now idle) DA tiles,
             // four heads at a time; dg and the weight-gradient partials
             float *part = reinterpret_cast<float *>(sp + S::DA);
@@ -798,10 +799,10 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
     static std::atomic<uint32_t> attr_set{0};
     if (cudaError_t e = ensure_smem_attr(k_bwd_stream, BsSmem::BYTES, attr_set); e != cudaSuccess) return e;
     const __nv_bfloat16 *dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
-    CUtensorMap mE, mDEp, mDE, mK, mV, mEt, mDEpt, mQ, mDO, mDL;
+    CUtensorMap mE, mDEp, mK, mV, mEt, mDEpt, mQ, mDO, mDL;
     const int n4 = (d.n + 3) / 4 * 4;
     if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mDEp, a.dEout, d.B, d.n, false, 32, 1) ||
-        !encode_pair_map(&mDE, a.dE, d.B, d.n, false, 32, 1) || !encode_node_map(&mK, a.K, d.B, d.n, 32) ||
+        !encode_node_map(&mK, a.K, d.B, d.n, 32) ||
         !encode_node_map(&mV, a.V, d.B, d.n, 32) || !encode_pair_map(&mEt, a.E, d.B, d.n, true, 32, 1) ||
         !encode_pair_map(&mDEpt, a.dEout, d.B, d.n, true, 32, 1) || !encode_node_map(&mQ, a.Q, d.B, d.n, 32) ||
         !encode_node_map(&mDO, dO, d.B, d.n, 32) || !encode_rowstat_map(&mDL, ws + W.Drow, d.B, d.n, n4))
@@ -818,6 +819,7 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
     p.dQ = reinterpret_cast<__nv_bfloat16 *>(ws + W.dQ);
     p.dK = reinterpret_cast<__nv_bfloat16 *>(ws + W.dK);
     p.dV = reinterpret_cast<__nv_bfloat16 *>(ws + W.dV);
+    p.dE = static_cast<__nv_bfloat16 *>(a.dE);
     p.rparts = reinterpret_cast<float *>(ws + W.rparts);
     p.DL = reinterpret_cast<float *>(ws + W.Drow);
     p.flags = reinterpret_cast<int *>(ws + W.flags);
@@ -828,7 +830,7 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
     p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
     p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)sm_count();
-    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, mEt, mDEpt,
+    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mK, mV, mEt, mDEpt,
                                                                                 mQ, mDO, mDL, p);
     return cudaGetLastError();
 }

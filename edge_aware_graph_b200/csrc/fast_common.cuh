@@ -205,6 +205,27 @@ __device__ __forceinline__ void add_residual16(uint8_t *row, uint32_t L, int hq,
     }
 }
 
+// Residual of a 128-byte swizzled pair row written to global memory: dst[c] =
+// row[c] (+ dv[c - 16hq] when `add`) for the 16 channels c in [16hq, 16hq + 16),
+// rounded to bf16, two 16-byte streaming stores (the row itself is unchanged).
+__device__ __forceinline__ void residual16_to_global(const uint8_t *row, uint32_t L, int hq, const float (&dv)[16],
+                                                     bool add, __nv_bfloat16 *dst) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t ch = 2 * hq + hh;
+        uint4 ev = *reinterpret_cast<const uint4 *>(row + ((ch ^ (L & 7u)) << 4));
+        if (add) {
+            __nv_bfloat162 *e2 = reinterpret_cast<__nv_bfloat162 *>(&ev);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 x = __bfloat1622float2(e2[u]);
+                e2[u] = __floats2bfloat162_rn(x.x + dv[8 * hh + 2 * u], x.y + dv[8 * hh + 2 * u + 1]);
+            }
+        }
+        __stcs(reinterpret_cast<uint4 *>(dst) + hh, ev);
+    }
+}
+
 __device__ __forceinline__ void flag_timeout(int *status) { atomicExch(status, DEV_TIMEOUT); }
 
 // Bounded wait on phase `parity` of mbarrier `bar` that gives up for the
