@@ -53,8 +53,7 @@ extern "C" {
 size_t eaga_workspace_size(const eaga_dims *d, int for_backward) {
     if (check_dims(d) != EAGA_OK) return 0;
     const WsLayout W = ws_layout(*d);
-    if (for_backward ? fast::supports_backward(*d) : fast::supports(*d))
-        return fast::workspace_size(*d, for_backward, W.total_fwd, W.fwd_saved);
+    if (fast::supports(*d)) return fast::workspace_size(*d, for_backward, W.total_fwd, W.fwd_saved);
     return for_backward ? W.total_bwd : W.total_fwd;
 }
 
@@ -175,7 +174,7 @@ eaga_status eaga_backward_variant(const eaga_dims *d, int variant, const void *X
     a.part_stride = W.part_stride;
     a.status = reinterpret_cast<int *>(ws + W.status);
     if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
-    if (fast::supports_backward(*d)) {
+    if (fast::supports(*d)) {
         return launch_status(fast::backward(*d, a, ws, W.fwd_saved, st));
     }
     return launch_status(generic::backward(*d, a, st));
@@ -277,7 +276,7 @@ eaga_status eaga_set_profile_events(int point, void *before, void *after) {
 
 int eaga_kernel_launches(const eaga_dims *d, int for_backward) {
     if (check_dims(d) != EAGA_OK) return -1;
-    if (for_backward ? fast::supports_backward(*d) : fast::supports(*d)) return fast::kernel_launches(*d, for_backward);
+    if (fast::supports(*d)) return fast::kernel_launches(*d, for_backward);
     return generic::kernel_launches(*d, for_backward);
 }
 

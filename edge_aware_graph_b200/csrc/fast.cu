@@ -18,6 +18,7 @@ cudaError_t tc_wgrad(int M, int Nb, int nout, int K, int splits, const void *A, 
                      float *const P[3], int *status, cudaStream_t st);
 cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                              cudaStream_t st);
+cudaError_t launch_kv_convert(const eaga_dims &d, const FastWs &W, char *ws, cudaStream_t st);
 cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
 cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
                              cudaStream_t st);
@@ -26,10 +27,6 @@ bool supports(const eaga_dims &d) {
     return d.dtype == EAGA_BF16 && d.de == DE && d.H == NH && d.dh == DH && d.n % 2 == 0 && d.n >= 2 &&
            d.n <= 1024 && d.dx % 64 == 0 && d.dx >= 64;
 }
-
-// The backward pair kernel's CTAs of one graph wait for each other (bounded),
-// so the device must hold the row blocks of one graph at once, one CTA per SM.
-bool supports_backward(const eaga_dims &d) { return supports(d) && sm_count() >= (d.n + TB - 1) / TB; }
 
 // Forward: the small operand images after the common workspace; backward:
 // the whole FastWs.
@@ -42,8 +39,9 @@ size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, s
 
 int kernel_launches(const eaga_dims &, int for_backward) {
     // forward: prologue, QKV, pairs, out-proj
-    // backward: prologue, dO, pairs, dX, wgrad x2, bias partial, rparts partial, finish, film grads
-    return for_backward ? 10 : 4;
+    // backward: prologue, dO, pairs, dk/dv conversion, dX, wgrad x2, bias partial, rparts partial,
+    // finish, film grads
+    return for_backward ? 11 : 4;
 }
 
 #define FAST_TRY(x)                               \
@@ -135,12 +133,15 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         void *C[3] = {dO, dO, dO};
         FAST_TRY(tc_gemm(2, rows, HD, d.dx, 1, A, Bt, nullptr, C, HD, nullptr, a.M, a.status, s1, false));
     }
-    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, reinterpret_cast<int *>(ws + W.flags), W.n_rparts + 1, st));
+    // the dk, dv accumulators start at zero (beside dO on the auxiliary stream)
+    FAST_TRY(cudaMemsetAsync(ws + W.dK32, 0, (size_t)rows * HD * 4 * 2, s1));
+    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, st));
     FAST_TRY(stream_after(st, s1, ev[1]));
 
     prof_mark(1, 0, st);
     FAST_TRY(launch_bwd_pairs(d, a, W, ws, a.g, st));
     prof_mark(1, 1, st);
+    FAST_TRY(launch_kv_convert(d, W, ws, st));
 
     // dX, the weight-gradient partials and the reductions' first level side by side
     const __nv_bfloat16 *dN[3] = {reinterpret_cast<const __nv_bfloat16 *>(ws + W.dQ),

@@ -5,8 +5,6 @@
 namespace eaga {
 namespace fast {
 bool supports(const eaga_dims &d);
-// supports(d) and the device can hold the row blocks of one graph at once
-bool supports_backward(const eaga_dims &d);
 // common_fwd: end of the common forward workspace; common_head: end of the
 // status word and g (start of the backward's own regions).
 size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, size_t common_head);

@@ -160,6 +160,33 @@ cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs 
     return e;
 }
 
+// dK = bf16(dK32 / sqrt(dh)), dV = bf16(dV32): the pair kernel's fp32 sums over
+// row blocks, for the node GEMMs and the bias sums (four features per thread).
+__global__ void k_kv_convert(const float4 *dK32, const float4 *dV32, size_t n4, __nv_bfloat16 *dK,
+                             __nv_bfloat16 *dV) {
+    const float rs = rsqrtf((float)DH);
+    for (size_t x = blockIdx.x * (size_t)blockDim.x + threadIdx.x; x < n4; x += (size_t)gridDim.x * blockDim.x) {
+        const float4 k = dK32[x], v = dV32[x];
+        uint2 ko, vo;
+        ko.x = sm100::pack_bf16(k.x * rs, k.y * rs);
+        ko.y = sm100::pack_bf16(k.z * rs, k.w * rs);
+        vo.x = sm100::pack_bf16(v.x, v.y);
+        vo.y = sm100::pack_bf16(v.z, v.w);
+        reinterpret_cast<uint2 *>(dK)[x] = ko;
+        reinterpret_cast<uint2 *>(dV)[x] = vo;
+    }
+}
+
+cudaError_t launch_kv_convert(const eaga_dims &d, const FastWs &W, char *ws, cudaStream_t st) {
+    const size_t n4 = (size_t)d.B * d.n * HD / 4;
+    const int blocks = (int)std::min<size_t>((n4 + 255) / 256, (size_t)sm_count() * 8);
+    k_kv_convert<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(ws + W.dK32),
+                                         reinterpret_cast<const float4 *>(ws + W.dV32), n4,
+                                         reinterpret_cast<__nv_bfloat16 *>(ws + W.dK),
+                                         reinterpret_cast<__nv_bfloat16 *>(ws + W.dV));
+    return cudaGetLastError();
+}
+
 // Column sums for the bias gradients and the first level of the row-block
 // partials of dWfe / dWe (both read only what the pair kernels wrote).
 cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st) {

@@ -8,46 +8,36 @@
 //   dE = dE' + [dgamma|dbeta] Wfe^T,  dWfe = sum E^T [dgamma|dbeta],  dWe = sum a^T dE',  dg = sum [dgamma|dbeta]
 // with a_ij = exp(s'_ij - LSE_i) from the forward's saved row statistics.
 //
-// One CTA owns the 8 nodes of one row block of one graph and makes three
-// passes over 32-wide chunks (256 pairs: two 16 KB E tiles, two 16 KB dE'
-// tiles and two 16 KB node chunks each):
-//   pass 1 (its rows i, all columns j): FiLM f = E Wfe and u = dE' We^T on the
-//           tensor cores (tcgen05, fp32 in TMEM), S = Q K^T and dP = dO V^T
-//           on warp MMAs, a, dA and a running D per thread; S and dP stay in
-//           TMEM for pass 2 (32 columns per chunk, n <= 224; larger n reloads
-//           K and V).  At its end the CTA publishes D of its rows (global
-//           memory, then a release flag per row block).
-//   pass 2 (its rows, the chunks in reverse so that E and dE' come back from
-//           L2): dS', dgamma, dbeta, ds; dE = dE' + df Wfe^T on the tensor
-//           cores, in place in shared memory, stored with TMA; dWfe += E^T df
+// One CTA owns the 8 query rows i of one row block of one graph and streams
+// the columns j of those rows in chunks of 32 (256 pairs: two 16 KB E tiles,
+// two 16 KB dE' tiles, the 16 KB K and V chunks), twice, because D needs a
+// whole row before any dS' exists:
+//   pass 1: FiLM f = E Wfe and u = dE' We^T on the tensor cores (tcgen05,
+//           fp32 in TMEM), S = Q K^T and dP = dO V^T on warp MMAs, a, dA, and
+//           a running D per thread; S and dP stay in TMEM for pass 2 (32
+//           columns per chunk, n <= 224; larger n reloads K and V);
+//   pass 2: (the chunks in reverse, so that E and dE' come back from L2) dS',
+//           dgamma, dbeta, ds; dE = dE' + df Wfe^T on the tensor cores, added
+//           to the dE' tile in registers and written from there; dWfe += E^T df
 //           and dWe^T += dE'^T a on the tensor cores (MN-major operands
 //           straight from the tiles, accumulated in TMEM over the row block);
-//           dq += ds K (warp MMAs).
-//   pass 3 (its nodes as the columns j, all rows i): the column tiles of E and
-//           dE' (pairs (i, j) with j among the CTA's 8 nodes), FiLM and u
-//           again, S and dP against the chunk's Q and dO rows, a and ds from
-//           LSE_i and the D_i the other CTAs of the graph published, then
-//           dk += ds^T Q and dv += a^T dO on warp MMAs.
-// E and dE' leave HBM once in passes 1 and 2, dE is written once; pass 3
-// reads the column tiles again (from L2 where the graph's tiles are still
-// there).  Nothing per pair is written besides dE: no [B,H,n,n] array.
-//
-// Pass 3 waits for other CTAs (the D of the rows of its chunk).  CTAs take
-// their (graph, row block) from a counter in the order they start, so the
-// row blocks a waiting CTA needs are held by CTAs already running, whose
-// passes 1 and 2 wait for nobody; every wait is bounded.  The wait needs the
-// row blocks of one graph (n/8 <= 128) to fit on the GPU at once, one CTA per
-// SM (148 on B200).
+//           dq += ds K (warp MMAs); and the row block's share of dk_j, dv_j for
+//           the chunk's columns (warp MMAs over the 8 rows), added into fp32
+//           accumulators [B,n,H*dh] with vector reductions in L2.
+// E and dE' leave HBM once, dE is written once, and no per-pair quantity is
+// written anywhere: no [B,H,n,n] array.  The dk, dv sums over row blocks
+// arrive in whatever order the CTAs run (fp32 additions: the last bits of dk,
+// dv may differ from run to run); everything else is summed in a fixed order.
+// No CTA waits for another.
 //
 // Warp roles as in the forward pair kernel: 16 compute warps (warp W reads
 // TMEM quadrant W%4 and handles heads 2(W/4), 2(W/4)+1), one MMA warp (FiLM
 // and u one chunk ahead into double-buffered TMEM ranges, dE and the weight
 // gradients when the compute warps have written df), one TMA warp (a ring of
 // twelve 16 KB slots, dE stores).  They meet only on mbarriers.  The pair <->
-// lane mapping is the forward's: row 4x + yc of a tile of parity s is the pair
-// of chunk index x and fixed-side index 2yc + s, which lane t of quadrant
-// q = x/8 holds in accumulator register s of its m16n8 tile (rows: the
-// chunk's nodes; columns: the CTA's 8 nodes).
+// lane mapping is the forward's: row 4j + ic of E tile s is the pair (j, i =
+// 2ic + s), which lane t of quadrant q = j/8 holds in accumulator register s
+// of its m16n8 tile S^T[j, i].
 #include <math.h>
 #include "fast.h"
 #include "fast_common.cuh"
@@ -65,7 +55,7 @@ constexpr int BS_THR = NTHR + 64;
 constexpr int BS_KEEP_MAX_CHUNKS = 7;     // S and dP of up to 7 chunks (n <= 224) stay in TMEM
 
 struct BsSmem {
-    // offsets from a 1024-aligned base; the TMA destinations (slots, LD) are 1024-aligned
+    // offsets from a 1024-aligned base
     static constexpr uint32_t IMG = BS_SLOTS * BS_SLOT;       // Wfe^T sw (FiLM), We sw (u), Wfe ns (dE): 2 KB each
     static constexpr uint32_t DA = IMG + 6144;                // 2 tiles [128][32] ns: [dgamma | dbeta | a | 0]
     static constexpr uint32_t WD = DA + 16384;                // per-quadrant D [4][8 i][8 h]
@@ -75,13 +65,9 @@ struct BsSmem {
     static constexpr uint32_t BAR = MJ + 1024;
     static constexpr uint32_t TM = BAR + 8 * 18;              // TMEM base address
     static constexpr uint32_t FAIL = TM + 4;                  // CTA failure flag (a wait ran out)
-    static constexpr uint32_t ITEM = TM + 8;                  // this CTA's work item
     static constexpr uint32_t STAB = TM + 16;                 // slot table [4 iterations][8] u8
-    static constexpr uint32_t LD = (STAB + 32 + 1023) / 1024 * 1024;   // pass 3: [2 buffers][LSE, D][8 h][32 i] f32
-    static constexpr uint32_t BYTES = LD + 4096 + 1024;
-    // after pass 2, in the DA tiles: dq quadrant sums of four heads [4][8][128] f32 (16 KB);
-    // at the end, in the drained ring: dk and dv quadrant sums [4][8][256] f32 (32 KB each)
-    static constexpr uint32_t KPART = 0, VPART = 32768;
+    static constexpr uint32_t BYTES = STAB + 32 + 1024;
+    // after pass 2, in the DA tiles: dq quadrant sums of four heads [4][8][128] f32 (16 KB)
 };
 // mbarriers: full[4], film_full[2], film_empty[2], df_full, de_full, stage_done[4], mma_final,
 // wg_done[2] (the weight-gradient products of pass-2 chunk p2, by p2 & 1)
@@ -102,74 +88,48 @@ __device__ __forceinline__ uint32_t ns32(uint32_t row, uint32_t col) {
     return (row >> 3) * 512u + (col >> 3) * 128u + (row & 7u) * 16u + (col & 7u) * 2u;
 }
 
-__device__ __forceinline__ void st_release_gpu(int *p, int v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 struct BwdStreamParams {
-    const __nv_bfloat16 *Q, *K, *V, *dO;
+    const __nv_bfloat16 *Q, *dO;
     const float *LSE, *g;
     const uint8_t *img, *M;
-    __nv_bfloat16 *dQ, *dK, *dV;   // [B,n,256] out (dQ and dK scaled by 1/sqrt(dh))
+    __nv_bfloat16 *dQ;       // [B,n,256] out (scaled by 1/sqrt(dh))
     __nv_bfloat16 *dE;       // [B,n,n,64] out
     float *rparts;           // [graph * row block][RPART] out
-    float *DL;               // [B][LSE, D][H][n4]: LSE and D of every row, published by its row block
-    int *flags;              // [graph * row block]: 1 once that row block's D is published (0 at launch)
-    int *ticket;             // work-item counter (0 at launch)
+    float *dK32, *dV32;      // [B,n,256] fp32 accumulators of dk (unscaled), dv (zero at launch)
     int *status;
-    int n, n4;               // n4: n rounded up to a multiple of 4 (the DL row length)
+    int n;
     int light;               // Light Edge variant: no per-edge FiLM map; E is not read, dE = dE'
     int unnorm;              // unnormalised variant: the edge path reaches s' directly
     uint32_t prefetch_ahead;   // CTAs between this one and the one whose first tiles it prefetches
 };
 
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-__global__ void __launch_bounds__(BS_THR, 1)
+// 576 threads x 112 registers = 64,512 of the SM's 65,536: one CTA per SM
+__global__ void __maxnreg__(112)
 k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmDEp,
-             const __grid_constant__ CUtensorMap tmK,
-             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmEt,
-             const __grid_constant__ CUtensorMap tmDEpt, const __grid_constant__ CUtensorMap tmQ,
-             const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmDL,
-             BwdStreamParams p) {
+             const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, BwdStreamParams p) {
     using S = BsSmem;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
     const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = (W >> 2) & 3, t = tid & 31, c4 = t & 3, g8 = t >> 2;
-    const int n = p.n, nch = (n + 31) / 32, nit = 3 * nch, nrb = (n + TB - 1) / TB;
+    const int n = p.n, nch = (n + 31) / 32, nit = 2 * nch;
+    const int b = blockIdx.y, i0 = blockIdx.x * TB, item = blockIdx.y * gridDim.x + blockIdx.x;
     const uint32_t bars = sbase + S::BAR;
     auto bar = [&](int k) { return bars + 8 * k; };
     float *g = reinterpret_cast<float *>(sp + S::G);
     uint8_t *mj = sp + S::MJ;
     volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
 
-    // work item (graph b, row block rb) in the order the CTAs start
-    if (tid == 0) *reinterpret_cast<volatile int *>(sp + S::ITEM) = atomicAdd(p.ticket, 1);
-    __syncthreads();
-    const int item = *reinterpret_cast<volatile int *>(sp + S::ITEM);
-    const int b = item / nrb, i0 = (item % nrb) * TB;
-
-    // iteration it: pass 1 walks chunks 0..nch-1 of the rows, pass 2 the same
-    // chunks in reverse, pass 3 the row chunks 0..nch-1 of the CTA's columns.
-    // Tiles (slot table entries 0..5): passes 1, 2: E(s=0), E(s=1), dE'(s=0),
-    // dE'(s=1), K, then V (in pass 2 only when S, dP are not kept); pass 3: the
-    // column tiles of E and dE' in the same order, then Q and dO of the chunk's
-    // rows.  The TMA warp places each tile in any free slot and records the
-    // slot in the table entry it % 4, which the other warps read after the
-    // iteration's load barrier.
+    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0.  Its
+    // tiles: E(s=0), E(s=1), dE'(s=0), dE'(s=1), K, then V in pass 1 (and in
+    // pass 2 when S, dP are not kept).  The TMA warp places each tile in any
+    // free slot and records the slot in the table entry it % 4, which the
+    // other warps read after the iteration's load barrier.
     const bool keep = nch <= BS_KEEP_MAX_CHUNKS;
     const bool light = p.light != 0, unnorm = p.unnorm != 0;
     const int ns2 = keep ? 5 : 6;
-    auto pass_of = [&](int it) { return it < nch ? 1 : it < 2 * nch ? 2 : 3; };
-    auto chunk_of = [&](int it) { return it < nch ? it : it < 2 * nch ? 2 * nch - 1 - it : it - 2 * nch; };
+    auto pass_of = [&](int it) { return it < nch ? 1 : 2; };
+    auto chunk_of = [&](int it) { return it < nch ? it : nit - 1 - it; };
     auto nslots = [&](int it) { return pass_of(it) == 2 ? ns2 : 6; };
     volatile uint8_t *stab = sp + S::STAB;
     auto slot_addr = [&](int it, int k) { return sbase + (uint32_t)stab[(it % BS_NFULL) * 8 + k] * BS_SLOT; };
@@ -302,44 +262,16 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         // ================= TMA: loads into the slot ring, dE stores
         if (t == 0) {
             // E and dE' tiles loaded in pass 1 are read again in pass 2: keep
-            // them in L2; pass-2 reads stay at the normal priority (the column
-            // pass of other CTAs reads the same pairs); pass-3 reads are not
-            // read again
+            // them in L2; pass-2 reads are not read again
             const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
             // a chunk's slots are free once the compute warps are done with it
             // (and, in pass 2, its weight-gradient products have read the tiles)
             uint32_t free_mask = (1u << BS_SLOTS) - 1u;
             int next_load = 0;
             auto release = [&](int it, int k) { free_mask |= 1u << stab[(it % BS_NFULL) * 8 + k]; };
-            // D of the row blocks of pass-3 chunk c published by their CTAs?
-            // With `block`, wait for them (bounded).
-            auto rows_ready = [&](int c, bool block) -> bool {
-                const int r1 = min(4 * c + 4, nrb);
-                for (int r = 4 * c; r < r1; ++r) {
-                    const int *f = p.flags + (size_t)b * nrb + r;
-                    if (ld_acquire_gpu(f)) continue;
-                    if (!block) return false;
-                    uint32_t polls = 0;
-                    while (!ld_acquire_gpu(f) && !*fail) {
-                        if (++polls > (1u << 22)) {
-                            *fail = 1;
-                            flag_timeout(p.status);
-                            break;
-                        }
-                        __nanosleep(128);
-                    }
-                }
-                // the published LSE, D (generic stores of other CTAs, acquired
-                // above) are read next by this thread's TMA copy
-                fence_proxy_async_global();
-                return true;
-            };
-            // issue loads while slots are free; iteration `must` (and only it)
-            // may wait for the rows its pass-3 chunk needs
-            auto issue_loads = [&](int must) {
+            auto issue_loads = [&]() {
                 while (next_load < nit && __popc(free_mask) >= nslots(next_load) && !*fail) {
-                    const int it = next_load, ps = pass_of(it), c = chunk_of(it), x0 = 32 * c;
-                    if (ps == 3 && !rows_ready(c, it <= must)) return;
+                    const int it = next_load, ps = pass_of(it), x0 = 32 * chunk_of(it);
                     const uint32_t fb = bar(BB_FULL + it % BS_NFULL);
                     for (int k = 0; k < nslots(it); ++k) {
                         const int sidx = __ffs(free_mask) - 1;
@@ -347,50 +279,29 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         stab[(it % BS_NFULL) * 8 + k] = (uint8_t)sidx;
                     }
                     // (Light Edge: the E tiles' slots are taken but not loaded)
-                    mbar_expect_tx(fb, (nslots(it) - (light ? 2 : 0)) * BS_SLOT + (ps == 3 ? 2048u : 0u));
-                    if (ps < 3) {
+                    mbar_expect_tx(fb, (nslots(it) - (light ? 2 : 0)) * BS_SLOT);   // releases the table entry too
+                    const uint64_t pol = ps == 1 ? keep_l2 : drop_l2;
 #pragma unroll
-                        for (int s = 0; s < 2; ++s) {
-                            if (ps == 1) {
-                                if (!light) tma_load_5d_hint(slot_addr(it, s), &tmE, fb, 0, i0 / 2, x0, s, b, keep_l2);
-                                tma_load_5d_hint(slot_addr(it, 2 + s), &tmDEp, fb, 0, i0 / 2, x0, s, b, keep_l2);
-                            } else {
-                                if (!light) tma_load_5d(slot_addr(it, s), &tmE, fb, 0, i0 / 2, x0, s, b);
-                                tma_load_5d(slot_addr(it, 2 + s), &tmDEp, fb, 0, i0 / 2, x0, s, b);
-                            }
-                        }
+                    for (int s = 0; s < 2; ++s) {
+                        if (!light) tma_load_5d_hint(slot_addr(it, s), &tmE, fb, 0, i0 / 2, x0, s, b, pol);
+                        tma_load_5d_hint(slot_addr(it, 2 + s), &tmDEp, fb, 0, i0 / 2, x0, s, b, pol);
+                    }
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            tma_load_3d(slot_addr(it, 4) + k * 4096, &tmK, fb, 64 * k, x0, b);
-                            if (ps == 1 || !keep) tma_load_3d(slot_addr(it, 5) + k * 4096, &tmV, fb, 64 * k, x0, b);
-                        }
-                    } else {
-#pragma unroll
-                        for (int s = 0; s < 2; ++s) {
-                            if (!light) tma_load_5d_hint(slot_addr(it, s), &tmEt, fb, 0, i0 / 2, x0, s, b, drop_l2);
-                            tma_load_5d_hint(slot_addr(it, 2 + s), &tmDEpt, fb, 0, i0 / 2, x0, s, b, drop_l2);
-                        }
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            tma_load_3d(slot_addr(it, 4) + k * 4096, &tmQ, fb, 64 * k, x0, b);
-                            tma_load_3d(slot_addr(it, 5) + k * 4096, &tmDO, fb, 64 * k, x0, b);
-                        }
-                        // LSE and D of the chunk's rows; buffer c & 1 is free: chunk
-                        // c - 2 released its slots before these could be taken
-                        tma_load_4d(sbase + S::LD + (c & 1) * 2048, &tmDL, fb, x0, 0, 0, b);
+                    for (int k = 0; k < 4; ++k) {
+                        tma_load_3d(slot_addr(it, 4) + k * 4096, &tmK, fb, 64 * k, x0, b);
+                        if (ps == 1 || !keep) tma_load_3d(slot_addr(it, 5) + k * 4096, &tmV, fb, 64 * k, x0, b);
                     }
                     ++next_load;
                 }
             };
-            issue_loads(-1);
+            issue_loads();
             for (int it = 0; it < nit; ++it) {
                 const int ps = pass_of(it);
-                while (next_load <= it && !*fail) issue_loads(it);
                 if (it == nch && p.prefetch_ahead) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = (uint32_t)item + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
-                        const int prb = cid % nrb, pb = cid / nrb;
+                        const int prb = cid % gridDim.x, pb = cid / gridDim.x;
                         for (int cc = 0; cc < nch && cc < 2; ++cc) {
                             if (!light) {
                                 tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
@@ -408,7 +319,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     if (!cta_wait(bar(BB_WG_DONE + (p2 & 1)), (p2 >> 1) & 1, fail, p.status)) continue;
                 }
                 for (int k = 0; k < nslots(it); ++k) release(it, k);
-                issue_loads(-1);
+                issue_loads();
             }
             if (*fail)   // loads already issued land before the CTA's shared memory is released
                 for (int it = max(next_load - BS_NFULL, 0); it < next_load; ++it)
@@ -473,23 +384,6 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                             const int o = (2 * c4 + e) * 8 + 2 * hq + hh;
                             dsum[e][hh] = wd[o] + wd[64 + o] + wd[128 + o] + wd[192 + o];
                         }
-                    // publish LSE and D of the row block for the column pass of the graph's CTAs
-                    if (q == 0 && g8 == 0) {
-#pragma unroll
-                        for (int e = 0; e < 2; ++e)
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const int i = i0 + 2 * c4 + e;
-                                const size_t o = ((size_t)b * 2 * NH + 2 * hq + hh) * p.n4 + i;
-                                if (i < n) {
-                                    p.DL[o] = lse[e][hh];
-                                    p.DL[o + (size_t)NH * p.n4] = dsum[e][hh];
-                                }
-                            }
-                        __threadfence();
-                    }
-                    named_bar_sync(1, NTHR);
-                    if (tid == 0) st_release_gpu(p.flags + item, 1);
                 }
 
                 cta_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1, fail, p.status);
@@ -597,6 +491,46 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 // ---------------- dq += ds K (warp MMAs; overlaps the tensor-core products)
                 warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, da, qacc);
 
+                // ---------------- the row block's share of dk_j = sum_i ds_ij q_i and dv_j =
+                // sum_i a_ij dO_i for the warp's 8 columns j (two heads): warp MMAs with M = j,
+                // K = i (the 8 rows), N = 8 features.  A is the score tile's own fragment (row
+                // j, columns i), B the transposed Q / dO fragment of the rows; the two lanes of
+                // a pair (c4, c4 ^ 1) swap halves so that each adds four consecutive features
+                // with one vector reduction: even lanes dk, odd lanes dv.
+                {
+                    const int j = j0 + 8 * q + g8;
+                    const bool live = j < n && mj[j];        // masked columns get nothing
+                    const bool even = (c4 & 1) == 0;
+                    float *rowk = p.dK32 + ((size_t)b * n + (live ? j : 0)) * HD;
+                    float *rowv = p.dV32 + ((size_t)b * n + (live ? j : 0)) * HD;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t ak[4] = {pack_bf16(da[hh][0], da[hh][1]), 0u, 0u, 0u};
+                        const uint32_t av4[4] = {pack_bf16(av[hh][0], av[hh][1]), 0u, 0u, 0u};
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                float ck[4] = {0.f, 0.f, 0.f, 0.f}, cv[4] = {0.f, 0.f, 0.f, 0.f};
+                                mma16816(ck, ak, movmatrix_t(qf[hh][kk][half]), 0u);
+                                mma16816(cv, av4, movmatrix_t(of[hh][kk][half]), 0u);
+                                // lane holds features d0 + 2c4, +1 (d0 = the tile's first feature)
+                                const float s0 = even ? cv[0] : ck[0], s1 = even ? cv[1] : ck[1];
+                                const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1);
+                                const float r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+                                const int d0 = (2 * hq + hh) * DH + 16 * kk + 8 * half;
+                                if (live) {
+                                    if (even)
+                                        atomicAdd(reinterpret_cast<float4 *>(rowk + d0 + 2 * c4),
+                                                  make_float4(ck[0], ck[1], r0, r1));
+                                    else
+                                        atomicAdd(reinterpret_cast<float4 *>(rowv + d0 + 2 * c4 - 2),
+                                                  make_float4(r0, r1, cv[0], cv[1]));
+                                }
+                            }
+                    }
+                }
+
                 // ---------------- dE = dE' + df Wfe^T (Light Edge: dE = dE'), written from registers:
                 // the dE' tile stays as loaded for the weight-gradient product that reads it
                 cta_wait(bar(BB_DE_FULL), (it - nch) & 1, fail, p.status);
@@ -693,99 +627,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             }
         }
 
-        // ======== pass 3: the CTA's nodes as columns j, rows i in chunks of 32
-        {
-            uint32_t kf[2][2][2], vf[2][2][2];
-            load_frags2(p.K, b, n, i0, hq, g8, c4, kf);
-            load_frags2(p.V, b, n, i0, hq, g8, c4, vf);
-            float kacc[2][2][4], vacc[2][2][4];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) kacc[hh][mt][x] = vacc[hh][mt][x] = 0.f;
-            for (int it = 2 * nch; it < nit; ++it) {
-                const int ir = 32 * (it - 2 * nch) + 8 * q + g8;   // this lane's row i
-                cta_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1, fail, p.status);
-                // LSE_i and D_i as the row blocks published them (TMA-loaded with the chunk)
-                float lse3[2], d3[2];
-                {
-                    const float *ld = reinterpret_cast<const float *>(sp + S::LD + ((it - 2 * nch) & 1) * 2048);
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        lse3[hh] = ld[(2 * hq + hh) * 32 + 8 * q + g8];
-                        d3[hh] = ld[(NH + 2 * hq + hh) * 32 + 8 * q + g8];
-                    }
-                }
-                float sv[2][4], dp[2][4];
-                warp_scores2<1>(slot_addr(it, 4), q, t, hq, kf, sv);    // q_i . k_j
-                warp_scores2<1>(slot_addr(it, 5), q, t, hq, vf, dp);    // dO_i . v_j
-                cta_wait(bar(BB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
-                tc_fence_after();
-                float fg[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, fb[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, fu[2][2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const uint32_t fcol = BS_TM_FILM + 32 * (it & 1) + 16 * e, ucol = BS_TM_U + 32 * (it & 1) + 16 * e;
-                    if (!light) {   // Light Edge: gamma, beta from y alone
-                        tmem_ld2(tl + fcol + 2 * hq, fg[e][0], fg[e][1]);
-                        tmem_ld2(tl + fcol + NH + 2 * hq, fb[e][0], fb[e][1]);
-                    }
-                    tmem_ld2(tl + ucol + 2 * hq, fu[e][0], fu[e][1]);
-                }
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (t == 0) mbar_arrive(bar(BB_FILM_EMPTY + (it & 1)));
-                const bool mi = mj[ir] != 0;   // mj covers 32 * nch nodes, zero past n
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const bool valid = mi && mrow[e];
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int h = 2 * hq + hh;
-                        const float s = sv[hh][e] * rs;
-                        const float gam = fg[e][hh] + g[h], bet = fb[e][hh] + g[NH + h];
-                        const float a = valid ? exp2f((s * (1.f + gam) + bet - lse3[hh]) * LOG2E) : 0.f;
-                        const float dsp = unnorm ? a * (dp[hh][e] - d3[hh]) + (valid ? fu[e][hh] : 0.f)
-                                                 : a * (dp[hh][e] + fu[e][hh] - d3[hh]);
-                        sv[hh][e] = a;                       // a_ij
-                        dp[hh][e] = dsp * (1.f + gam);       // ds_ij (unscaled)
-                    }
-                }
-                sv[0][2] = sv[0][3] = sv[1][2] = sv[1][3] = 0.f;
-                dp[0][2] = dp[0][3] = dp[1][2] = dp[1][3] = 0.f;
-                // dk_j += sum_i ds_ij q_i, dv_j += sum_i a_ij dO_i (warp MMAs over the chunk's rows)
-                warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, dp, kacc);
-                warp_contract2<1, true>(slot_addr(it, 5), q, t, hq, sv, vacc);
-                __syncwarp();
-                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
-            }
-
-            // ---------------- dk, dv: sum over the quadrant warps, in the drained ring
-            named_bar_sync(2, BS_THR);
-            store_quadrant_part(sp, S::KPART, kacc, q, hq, t);
-            store_quadrant_part(sp, S::VPART, vacc, q, hq, t);
-            named_bar_sync(1, NTHR);
-            const float *kp = reinterpret_cast<const float *>(sp + S::KPART);
-            const float *vp = reinterpret_cast<const float *>(sp + S::VPART);
-            for (int x = tid; x < TB * HD / 2; x += NTHR) {
-                const int il = (2 * x) / HD, d = (2 * x) % HD;
-                if (i0 + il >= n) continue;
-                float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int o = k * TB * HD + il * HD + d;
-                    k0 += kp[o];
-                    k1 += kp[o + 1];
-                    v0 += vp[o];
-                    v1 += vp[o + 1];
-                }
-                const size_t o = ((size_t)b * n + i0 + il) * HD + d;
-                *reinterpret_cast<uint32_t *>(p.dK + o) = pack_bf16(k0 * rs, k1 * rs);
-                *reinterpret_cast<uint32_t *>(p.dV + o) = pack_bf16(v0, v1);
-            }
-        }
+        named_bar_sync(2, BS_THR);   // meets the MMA and TMA warps at their end
     }
     tc_fence_before();
     __syncthreads();
@@ -798,40 +640,28 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
                               cudaStream_t st) {
     static std::atomic<uint32_t> attr_set{0};
     if (cudaError_t e = ensure_smem_attr(k_bwd_stream, BsSmem::BYTES, attr_set); e != cudaSuccess) return e;
-    const __nv_bfloat16 *dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
-    CUtensorMap mE, mDEp, mK, mV, mEt, mDEpt, mQ, mDO, mDL;
-    const int n4 = (d.n + 3) / 4 * 4;
+    CUtensorMap mE, mDEp, mK, mV;
     if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mDEp, a.dEout, d.B, d.n, false, 32, 1) ||
-        !encode_node_map(&mK, a.K, d.B, d.n, 32) ||
-        !encode_node_map(&mV, a.V, d.B, d.n, 32) || !encode_pair_map(&mEt, a.E, d.B, d.n, true, 32, 1) ||
-        !encode_pair_map(&mDEpt, a.dEout, d.B, d.n, true, 32, 1) || !encode_node_map(&mQ, a.Q, d.B, d.n, 32) ||
-        !encode_node_map(&mDO, dO, d.B, d.n, 32) || !encode_rowstat_map(&mDL, ws + W.Drow, d.B, d.n, n4))
+        !encode_node_map(&mK, a.K, d.B, d.n, 32) || !encode_node_map(&mV, a.V, d.B, d.n, 32))
         return cudaErrorInvalidValue;
     BwdStreamParams p;
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
-    p.K = static_cast<const __nv_bfloat16 *>(a.K);
-    p.V = static_cast<const __nv_bfloat16 *>(a.V);
-    p.dO = dO;
+    p.dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
     p.LSE = a.LSE;
     p.g = g;
     p.img = reinterpret_cast<const uint8_t *>(ws + W.img);
     p.M = a.M;
     p.dQ = reinterpret_cast<__nv_bfloat16 *>(ws + W.dQ);
-    p.dK = reinterpret_cast<__nv_bfloat16 *>(ws + W.dK);
-    p.dV = reinterpret_cast<__nv_bfloat16 *>(ws + W.dV);
     p.dE = static_cast<__nv_bfloat16 *>(a.dE);
     p.rparts = reinterpret_cast<float *>(ws + W.rparts);
-    p.DL = reinterpret_cast<float *>(ws + W.Drow);
-    p.flags = reinterpret_cast<int *>(ws + W.flags);
-    p.ticket = p.flags + W.n_rparts;
+    p.dK32 = reinterpret_cast<float *>(ws + W.dK32);
+    p.dV32 = reinterpret_cast<float *>(ws + W.dV32);
     p.status = a.status;
     p.n = d.n;
-    p.n4 = n4;
     p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
     p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)sm_count();
-    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mK, mV, mEt, mDEpt,
-                                                                                mQ, mDO, mDL, p);
+    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mK, mV, p);
     return cudaGetLastError();
 }
 

@@ -43,7 +43,7 @@ __host__ __device__ __forceinline__ uint32_t ns16(uint32_t row, uint32_t k) {
 // Workspace of the fast path (after the common status word and g).  Every
 // region grows with the node count B*n (or is fixed): no per-pair buffer.
 struct FastWs {
-    size_t img, dO, dQ, dK, dV, Drow, flags, rparts, wparts, bparts, r2, dg, total;
+    size_t img, dO, dQ, dK, dV, dK32, dV32, rparts, wparts, bparts, r2, dg, total;
     int n_rparts, wsplits, bsplits, rsplits;
 };
 
@@ -64,11 +64,10 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
     W.dQ = off; off = align256(off + rows * HD * 2);
     W.dK = off; off = align256(off + rows * HD * 2);
     W.dV = off; off = align256(off + rows * HD * 2);
-    // LSE and D of every row [B][2][H][roundup4(n)] fp32, published by the pair kernel's row blocks
-    W.Drow = off; off = align256(off + size_t(d.B) * 2 * NH * ((d.n + 3) / 4 * 4) * 4);
+    // fp32 accumulators of dk (unscaled) and dv [B*n, 256], summed over row blocks in L2
+    W.dK32 = off; off = align256(off + rows * HD * 4);
+    W.dV32 = off; off = align256(off + rows * HD * 4);
     W.n_rparts = row_blocks(d);
-    // one flag per (graph, row block), then the pair kernel's work-item counter: zeroed per call
-    W.flags = off; off = align256(off + size_t(W.n_rparts + 1) * 4);
     W.rparts = off; off = align256(off + size_t(W.n_rparts) * RPART * 4);
     W.wsplits = wgrad_splits(d);
     // split-K partials of dWq, dWk, dWv [dx, 256] and dWo [256, dx]
@@ -84,7 +83,6 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
 
 bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transposed, int box_rows, int box_s = 2);
 bool encode_node_map(CUtensorMap *m, const void *base, int B, int n, int box_rows);
-bool encode_rowstat_map(CUtensorMap *m, const void *base, int B, int n, int n4);
 
 
 // ------------------------------------------------------------------ device pieces

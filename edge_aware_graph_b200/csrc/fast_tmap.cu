@@ -66,21 +66,6 @@ bool encode_node_map(CUtensorMap *m, const void *base, int B, int n, int box_row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The backward's published row statistics [B][2][H][n4] fp32 (LSE, then D;
-// n4 = n rounded up to 4 so that rows are 16-byte multiples); box of 32 rows
-// x 8 heads x both statistics of one graph, no swizzle.
-bool encode_rowstat_map(CUtensorMap *m, const void *base, int B, int n, int n4) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)n, NH, 2, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)n4 * 4, (cuuint64_t)NH * n4 * 4, (cuuint64_t)2 * NH * n4 * 4};
-    const cuuint32_t box[4] = {32, NH, 2, 1};
-    const cuuint32_t es[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // A row-major [rows, cols] bf16 matrix; box of 64 columns x box_rows rows, 128B-swizzled.
 bool encode_2d(CUtensorMap *m, const void *base, int rows, int cols, int box_rows) {
     auto enc = get_encode();
