@@ -32,7 +32,6 @@ bool supports(const eaga_dims &d) {
 // the whole FastWs.
 size_t forward_scratch_bytes(const eaga_dims &) { return align256(IMG_BYTES); }
 size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, size_t common_head) {
-    // (callers check supports(d), and supports_backward(d) for the backward)
     if (!for_backward) return align256(common_fwd + IMG_BYTES);
     return fast_ws(d, common_head).total;
 }
