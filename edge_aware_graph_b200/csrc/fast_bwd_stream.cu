@@ -103,8 +103,9 @@ struct BwdStreamParams {
     uint32_t prefetch_ahead;   // CTAs between this one and the one whose first tiles it prefetches
 };
 
-// 576 threads x 112 registers = 64,512 of the SM's 65,536: one CTA per SM
-__global__ void __maxnreg__(112)
+// 576 threads (18 warps): five warps share one of the four 16K-register sub-partitions,
+// so at most 96 registers a thread
+__global__ void __launch_bounds__(BS_THR, 1)
 k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmDEp,
              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, BwdStreamParams p) {
     using S = BsSmem;
