@@ -155,11 +155,17 @@ def test_masked_garbage_is_ignored():
     rt = torch.from_numpy(rows).cuda()
     assert torch.equal(buf.Xout[rt], base["Xout"][rt])
     assert torch.equal(buf.Eout[vt], base["Eout"][vt])
-    assert torch.equal(buf.dX[rt], base["dX"][rt])
     assert torch.equal(buf.dE[vt], base["dE"][vt])
     assert torch.equal(buf.dy, base["dy"])
+    # dk, dv are fp32 sums over row blocks that arrive in the order the CTAs run,
+    # so what depends on them (dX, dWk, dbk, dWv, dbv) may differ in the last bits
+    # between any two calls; garbage reaching them would show at its 1e3 scale
     for k in base_dw:
-        assert torch.equal(buf.dW[k], base_dw[k]), k
+        if k in ("Wk", "bk", "Wv", "bv"):
+            assert rel_err(buf.dW[k], base_dw[k].cpu().numpy()) <= 1e-3, k
+        else:
+            assert torch.equal(buf.dW[k], base_dw[k]), k
+    assert rel_err(buf.dX[rt], base["dX"][rt].float().cpu().numpy()) <= 1e-3
     assert torch.equal(buf.Xout[~rt], buf.X[~rt])
     assert torch.equal(buf.Eout[~vt], buf.E[~vt])
     assert torch.equal(buf.dE[~vt], buf.dEout[~vt])
