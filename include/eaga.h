@@ -123,7 +123,10 @@ EAGA_API eaga_status eaga_forward(const eaga_dims *dims,
  * the library creates once per device; they start after the work already
  * on `stream` and `stream` waits for them before the call's last kernels,
  * so the call is ordered on `stream` as a whole (and a CUDA graph captured
- * around it keeps them as parallel branches). */
+ * around it keeps them as parallel branches).  On that path the key and
+ * value gradients are fp32 sums over the graph's row blocks added in the
+ * order the blocks run, so dX, dWk, dbk, dWv and dbv may differ in their
+ * last bits between calls; every other output is reproducible bit for bit. */
 EAGA_API eaga_status eaga_backward(const eaga_dims *dims,
                           const void *X, const void *E, const void *y, const uint8_t *M,
                           const eaga_weights *w, const void *saved,
