@@ -82,6 +82,13 @@ def test_light_edge_ignores_wfe():
         buf.forward(variant="light_edge")
         buf.backward(variant="light_edge")
         torch.cuda.synchronize()
-        outs.append([t.clone() for t in (buf.Xout, buf.Eout, buf.dX, buf.dE, buf.dy, buf.dW_flat)])
-    for a, b in zip(*outs):
+        outs.append([t.clone() for t in (buf.Xout, buf.Eout, buf.dE, buf.dy, buf.dX, buf.dW_flat)])
+    # Xout, Eout, dE and dy do not depend on the dk, dv sums over row blocks
+    # (fp32 additions in L2 in no fixed order): bitwise
+    for a, b in zip(outs[0][:4], outs[1][:4]):
         assert torch.equal(a, b)
+    # dX and the flat weight gradients (dWk, dbk, dWv, dbv among them) do:
+    # within 1e-3 of their scale, far below what a seven-fold Wfe would change
+    for a, b in zip(outs[0][4:], outs[1][4:]):
+        a, b = a.float(), b.float()
+        assert float((a - b).abs().max()) <= 1e-3 * float(a.abs().max())
