@@ -30,6 +30,10 @@
 // dv may differ from run to run); everything else is summed in a fixed order.
 // No CTA waits for another.
 //
+// Block sparsity, as in the forward: a chunk with no valid pair adds nothing
+// to D, dq, dk, dv, dg or the weight gradients, and its dE is its dE'.  It
+// skips pass 1 and in pass 2 the TMA warp copies its dE' tiles to dE.
+//
 // Warp roles as in the forward pair kernel: 16 compute warps (warp W reads
 // TMEM quadrant W%4 and handles heads 2(W/4), 2(W/4)+1), one MMA warp (FiLM
 // and u one chunk ahead into double-buffered TMEM ranges, dE and the weight
@@ -63,16 +67,21 @@ struct BsSmem {
     static constexpr uint32_t G = WDG + 256;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // node mask [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;
-    static constexpr uint32_t TM = BAR + 8 * 18;              // TMEM base address
+    static constexpr uint32_t TM = BAR + 8 * 21;              // TMEM base address
     static constexpr uint32_t FAIL = TM + 4;                  // CTA failure flag (a wait ran out)
-    static constexpr uint32_t STAB = TM + 16;                 // slot table [4 iterations][8] u8
-    static constexpr uint32_t BYTES = STAB + 32 + 1024;
+    static constexpr uint32_t STAB = TM + 16;                 // slot table [4 live iterations][8] u8
+    static constexpr uint32_t CTAB = STAB + 32;               // slots of the copies [4][2] u8
+    static constexpr uint32_t LIVE = CTAB + 8;                // live-chunk mask of the row block
+    static constexpr uint32_t LC = LIVE + 8;                  // the live chunks, ascending [32] u8
+    static constexpr uint32_t BYTES = LC + 32 + 1024;
     // after pass 2, in the DA tiles: dq quadrant sums of four heads [4][8][128] f32 (16 KB)
 };
-// mbarriers: full[4], film_full[2], film_empty[2], df_full, de_full, stage_done[4], mma_final,
-// wg_done[2] (the weight-gradient products of pass-2 chunk p2, by p2 & 1)
+// mbarriers: full[4] (loads of live iterations), film_full[2], film_empty[2], df_full, de_full,
+// stage_done[4], mma_final, wg_done[2] (the weight-gradient products of pass-2 live chunk p2,
+// by p2 & 1), copy[4] (loads of dead chunks)
 constexpr int BB_FULL = 0, BB_FILM_FULL = 4, BB_FILM_EMPTY = 6, BB_DF_FULL = 8, BB_DE_FULL = 9,
-              BB_STAGE_DONE = 10, BB_MMA_FINAL = 14, BB_WG_DONE = 15;
+              BB_STAGE_DONE = 10, BB_MMA_FINAL = 14, BB_WG_DONE = 15, BB_COPY = 17;
+constexpr int BS_NCOPY = 4;               // dead-chunk copies in flight
 
 // TMEM: FiLM 0..63 and u 64..127 (two buffers each), dE 128..255, kept S / dP
 // 256..479 (32 per chunk), and at 480 the weight-gradient accumulator
@@ -107,13 +116,14 @@ struct BwdStreamParams {
 // so at most 96 registers a thread
 __global__ void __launch_bounds__(BS_THR, 1)
 k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmDEp,
-             const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, BwdStreamParams p) {
+             const __grid_constant__ CUtensorMap tmDE, const __grid_constant__ CUtensorMap tmK,
+             const __grid_constant__ CUtensorMap tmV, BwdStreamParams p) {
     using S = BsSmem;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
     const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = (W >> 2) & 3, t = tid & 31, c4 = t & 3, g8 = t >> 2;
-    const int n = p.n, nch = (n + 31) / 32, nit = 2 * nch;
+    const int n = p.n, nch = (n + 31) / 32;
     const int b = blockIdx.y, i0 = blockIdx.x * TB, item = blockIdx.y * gridDim.x + blockIdx.x;
     const uint32_t bars = sbase + S::BAR;
     auto bar = [&](int k) { return bars + 8 * k; };
@@ -121,19 +131,21 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     uint8_t *mj = sp + S::MJ;
     volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
 
-    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0.  Its
-    // tiles: E(s=0), E(s=1), dE'(s=0), dE'(s=1), K, then V in pass 1 (and in
-    // pass 2 when S, dP are not kept).  The TMA warp places each tile in any
-    // free slot and records the slot in the table entry it % 4, which the
-    // other warps read after the iteration's load barrier.
+    // Block sparsity: a chunk holding no valid pair (live_chunk_mask) adds
+    // nothing to any sum and its dE is its dE'.  The TMA warp loads iterations
+    // it in order: pass 1 the nl live chunks, ascending; pass 2 all nch chunks,
+    // descending, where a live chunk is computed and a dead one only copied
+    // (its two dE' tiles loaded and stored as dE).  The live iterations li = 0
+    // .. 2 nl - 1 (pass 1, then pass 2's live chunks) are the ones the MMA and
+    // compute warps see.  Tiles of a live iteration: E(s=0), E(s=1), dE'(s=0),
+    // dE'(s=1), K, then V in pass 1 (and in pass 2 when S, dP are not kept).
+    // The TMA warp places each tile in any free slot and records the slot in
+    // table entry li % 4, which the other warps read after the load barrier.
     const bool keep = nch <= BS_KEEP_MAX_CHUNKS;
     const bool light = p.light != 0, unnorm = p.unnorm != 0;
     const int ns2 = keep ? 5 : 6;
-    auto pass_of = [&](int it) { return it < nch ? 1 : 2; };
-    auto chunk_of = [&](int it) { return it < nch ? it : nit - 1 - it; };
-    auto nslots = [&](int it) { return pass_of(it) == 2 ? ns2 : 6; };
     volatile uint8_t *stab = sp + S::STAB;
-    auto slot_addr = [&](int it, int k) { return sbase + (uint32_t)stab[(it % BS_NFULL) * 8 + k] * BS_SLOT; };
+    auto slot_addr = [&](int li, int k) { return sbase + (uint32_t)stab[(li % BS_NFULL) * 8 + k] * BS_SLOT; };
 
     // ---------------- setup: barriers, TMEM, operands
     if (tid == 0) {
@@ -148,12 +160,18 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         mbar_init(bar(BB_MMA_FINAL), 1);
         mbar_init(bar(BB_WG_DONE), 1);
         mbar_init(bar(BB_WG_DONE + 1), 1);
+        for (int k = 0; k < BS_NCOPY; ++k) mbar_init(bar(BB_COPY + k), 1);
         fence_mbar_init();
         *fail = 0;
     }
     if (W == 0) {
         tmem_alloc(sbase + S::TM, BS_TM_COLS);
         tmem_relinquish();
+    }
+    if (W == 1) {
+        const uint32_t lm = live_chunk_mask(p.M, b, n, i0, t);
+        if (t == 0) *reinterpret_cast<volatile uint32_t *>(sp + S::LIVE) = lm;
+        if ((lm >> t) & 1u) sp[S::LC + __popc(lm & ((1u << t) - 1u))] = (uint8_t)t;
     }
     if (tid < 384) {
         const uint32_t img_off = (tid >> 7) == 0 ? IMG_WFE_T_SW : (tid >> 7) == 1 ? IMG_WE_SW : IMG_WFE_NS;
@@ -168,32 +186,38 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+    const uint32_t live = *reinterpret_cast<volatile uint32_t *>(sp + S::LIVE);
+    const int nl = __popc(live), nit = 2 * nl, nload = nl + nch;
+    const volatile uint8_t *lc = sp + S::LC;
+    // chunk of live iteration li; chunk of load iteration it
+    auto chunk_of_li = [&](int li) { return (int)lc[li < nl ? li : nit - 1 - li]; };
+    auto chunk_of_it = [&](int it) { return it < nl ? (int)lc[it] : nch - 1 - (it - nl); };
 
     if (W == NWARP) {
         // ================= MMA issuer
         if (t == 0) {
             const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_d = idesc_bf16_f32(128, DE);
             const uint32_t idesc_w = idesc_bf16_f32_mn(128, 2 * NF);
-            auto issue_fu = [&](int it) {
+            auto issue_fu = [&](int li) {
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    const uint32_t ae = slot_addr(it, s), ad = slot_addr(it, 2 + s);
+                    const uint32_t ae = slot_addr(li, s), ad = slot_addr(li, 2 + s);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         if (!light)   // Light Edge: no FiLM product (its E tiles are not loaded)
-                            mma_bf16_ss(tmem + BS_TM_FILM + 32 * (it & 1) + 16 * s,
+                            mma_bf16_ss(tmem + BS_TM_FILM + 32 * (li & 1) + 16 * s,
                                         smem_desc(ae + kk * 32, 16, 1024, LAYOUT_SW128),
                                         smem_desc(sbase + S::IMG + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f, kk > 0);
-                        mma_bf16_ss(tmem + BS_TM_U + 32 * (it & 1) + 16 * s,
+                        mma_bf16_ss(tmem + BS_TM_U + 32 * (li & 1) + 16 * s,
                                     smem_desc(ad + kk * 32, 16, 1024, LAYOUT_SW128),
                                     smem_desc(sbase + S::IMG + 2048 + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f,
                                     kk > 0);
                     }
                 }
-                mma_commit(bar(BB_FILM_FULL + (it & 1)));
+                mma_commit(bar(BB_FILM_FULL + (li & 1)));
             };
-            auto issue_de = [&](int it) {
+            auto issue_de = [&](int li) {
                 tc_fence_after();
                 if (!light)   // Light Edge: df Wfe^T = 0, dE = dE'
 #pragma unroll
@@ -211,30 +235,30 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 // matrices: 128 B along N, 512 B along K); 16 pairs per MMA
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const uint32_t te = slot_addr(it, e), td = slot_addr(it, 2 + e);
+                    const uint32_t te = slot_addr(li, e), td = slot_addr(li, 2 + e);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t acc = (it > nch || e > 0 || ks > 0) ? 1u : 0u;
+                        const uint32_t acc = (li > nl || e > 0 || ks > 0) ? 1u : 0u;
                         mma_bf16_ss(tmem + BS_TM_W, smem_desc(te + ks * 2048, td - te, 1024, LAYOUT_SW128),
                                     smem_desc(sbase + S::DA + e * 8192 + ks * 1024, 512, 128, LAYOUT_NONE), idesc_w, acc);
                     }
                 }
                 // the tiles (E, dE', [df | a]) may be reused once these completed
-                mma_commit(bar(BB_WG_DONE + ((it - nch) & 1)));
+                mma_commit(bar(BB_WG_DONE + ((li - nl) & 1)));
             };
             // issue whichever product is ready first: FiLM/u of the next chunk
             // (its tiles landed, its TMEM buffer released) or dE of the pass-2
             // chunk whose df the compute warps have written
-            int next_fu = 0, next_de = nch;
+            int next_fu = 0, next_de = nl;
             uint32_t polls = 0;
-            while ((next_fu < nit || next_de < 2 * nch) && !*fail) {
+            while ((next_fu < nit || next_de < nit) && !*fail) {
                 bool progressed = false;
                 if (next_fu < nit && mbar_test_wait(bar(BB_FULL + next_fu % BS_NFULL), (next_fu / BS_NFULL) & 1) &&
                     (next_fu < 2 || mbar_test_wait(bar(BB_FILM_EMPTY + (next_fu & 1)), ((next_fu - 2) >> 1) & 1))) {
                     issue_fu(next_fu++);
                     progressed = true;
                 }
-                if (next_de < 2 * nch && next_de < next_fu && mbar_test_wait(bar(BB_DF_FULL), (next_de - nch) & 1)) {
+                if (next_de < nit && next_de < next_fu && mbar_test_wait(bar(BB_DF_FULL), (next_de - nl) & 1)) {
                     issue_de(next_de);
                     ++next_de;
                     progressed = true;
@@ -260,45 +284,70 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         __syncwarp();
         named_bar_sync(2, BS_THR);
     } else if (W == NWARP + 1) {
-        // ================= TMA: loads into the slot ring, dE stores
+        // ================= TMA: loads into the slot ring, copies of dead chunks
         if (t == 0) {
             // E and dE' tiles loaded in pass 1 are read again in pass 2: keep
             // them in L2; pass-2 reads are not read again
             const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
-            // a chunk's slots are free once the compute warps are done with it
-            // (and, in pass 2, its weight-gradient products have read the tiles)
+            volatile uint8_t *ctab = sp + S::CTAB;
+            // a live chunk's slots are free once the compute warps are done with
+            // it (and, in pass 2, its weight-gradient products have read the
+            // tiles); a copy's once its store has read them
             uint32_t free_mask = (1u << BS_SLOTS) - 1u;
-            int next_load = 0;
-            auto release = [&](int it, int k) { free_mask |= 1u << stab[(it % BS_NFULL) * 8 + k]; };
+            auto take_slot = [&]() {
+                const int sidx = __ffs(free_mask) - 1;
+                free_mask &= free_mask - 1u;
+                return (uint8_t)sidx;
+            };
+            auto is_live = [&](int it) { return it < nl || ((live >> chunk_of_it(it)) & 1u) != 0; };
+            // loads go out in iteration order; a live iteration waits for its
+            // load barrier to be free (at most BS_NFULL live iterations in
+            // flight), a copy likewise for its copy barrier
+            int next_load = 0, load_li = 0, load_dk = 0, done_li = 0, done_dk = 0;
             auto issue_loads = [&]() {
-                while (next_load < nit && __popc(free_mask) >= nslots(next_load) && !*fail) {
-                    const int it = next_load, ps = pass_of(it), x0 = 32 * chunk_of(it);
-                    const uint32_t fb = bar(BB_FULL + it % BS_NFULL);
-                    for (int k = 0; k < nslots(it); ++k) {
-                        const int sidx = __ffs(free_mask) - 1;
-                        free_mask &= free_mask - 1u;
-                        stab[(it % BS_NFULL) * 8 + k] = (uint8_t)sidx;
-                    }
-                    // (Light Edge: the E tiles' slots are taken but not loaded)
-                    mbar_expect_tx(fb, (nslots(it) - (light ? 2 : 0)) * BS_SLOT);   // releases the table entry too
-                    const uint64_t pol = ps == 1 ? keep_l2 : drop_l2;
+                while (next_load < nload && !*fail) {
+                    const int it = next_load, x0 = 32 * chunk_of_it(it);
+                    const bool pass2 = it >= nl;
+                    if (is_live(it)) {
+                        const int li = load_li, ns = pass2 ? ns2 : 6;
+                        if (li >= done_li + BS_NFULL || __popc(free_mask) < ns) break;
+                        // slots in increasing order: each dE' slot lies above the E slot of its parity
+                        for (int k = 0; k < ns; ++k) stab[(li % BS_NFULL) * 8 + k] = take_slot();
+                        const uint32_t fb = bar(BB_FULL + li % BS_NFULL);
+                        // (Light Edge: the E tiles' slots are taken but not loaded)
+                        mbar_expect_tx(fb, (ns - (light ? 2 : 0)) * BS_SLOT);   // releases the table entry too
+                        const uint64_t pol = pass2 ? drop_l2 : keep_l2;
 #pragma unroll
-                    for (int s = 0; s < 2; ++s) {
-                        if (!light) tma_load_5d_hint(slot_addr(it, s), &tmE, fb, 0, i0 / 2, x0, s, b, pol);
-                        tma_load_5d_hint(slot_addr(it, 2 + s), &tmDEp, fb, 0, i0 / 2, x0, s, b, pol);
-                    }
+                        for (int s = 0; s < 2; ++s) {
+                            if (!light) tma_load_5d_hint(slot_addr(li, s), &tmE, fb, 0, i0 / 2, x0, s, b, pol);
+                            tma_load_5d_hint(slot_addr(li, 2 + s), &tmDEp, fb, 0, i0 / 2, x0, s, b, pol);
+                        }
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        tma_load_3d(slot_addr(it, 4) + k * 4096, &tmK, fb, 64 * k, x0, b);
-                        if (ps == 1 || !keep) tma_load_3d(slot_addr(it, 5) + k * 4096, &tmV, fb, 64 * k, x0, b);
+                        for (int k = 0; k < 4; ++k) {
+                            tma_load_3d(slot_addr(li, 4) + k * 4096, &tmK, fb, 64 * k, x0, b);
+                            if (!pass2 || !keep) tma_load_3d(slot_addr(li, 5) + k * 4096, &tmV, fb, 64 * k, x0, b);
+                        }
+                        ++load_li;
+                    } else {
+                        const int dk = load_dk;
+                        if (dk >= done_dk + BS_NCOPY || __popc(free_mask) < 2) break;
+                        const uint32_t cb = bar(BB_COPY + dk % BS_NCOPY);
+                        mbar_expect_tx(cb, 2 * BS_SLOT);
+#pragma unroll
+                        for (int s = 0; s < 2; ++s) {
+                            const uint8_t sl = take_slot();
+                            ctab[(dk % BS_NCOPY) * 2 + s] = sl;
+                            tma_load_5d_hint(sbase + sl * BS_SLOT, &tmDEp, cb, 0, i0 / 2, x0, s, b, drop_l2);
+                        }
+                        ++load_dk;
                     }
                     ++next_load;
                 }
             };
             issue_loads();
-            for (int it = 0; it < nit; ++it) {
-                const int ps = pass_of(it);
-                if (it == nch && p.prefetch_ahead) {
+            uint32_t pend_mask = 0u;   // slots of the last copy store, not yet known to have read them
+            for (int it = 0; it < nload; ++it) {
+                if (it == nl && p.prefetch_ahead) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = (uint32_t)item + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
@@ -313,18 +362,40 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         }
                     }
                 }
-                if (!cta_wait(bar(BB_STAGE_DONE + (it & 3)), (it >> 2) & 1, fail, p.status)) continue;
-                if (ps == 2) {
-                    // the chunk's tiles are read by its weight-gradient products until these complete
-                    const int p2 = it - nch;
-                    if (!cta_wait(bar(BB_WG_DONE + (p2 & 1)), (p2 >> 1) & 1, fail, p.status)) continue;
+                if (is_live(it)) {
+                    const int li = done_li++;
+                    if (!cta_wait(bar(BB_STAGE_DONE + (li & 3)), (li >> 2) & 1, fail, p.status)) continue;
+                    const bool pass2 = it >= nl;
+                    if (pass2) {
+                        // the chunk's tiles are read by its weight-gradient products until these complete
+                        const int p2 = li - nl;
+                        if (!cta_wait(bar(BB_WG_DONE + (p2 & 1)), (p2 >> 1) & 1, fail, p.status)) continue;
+                    }
+                    for (int k = 0; k < (pass2 ? ns2 : 6); ++k) free_mask |= 1u << stab[(li % BS_NFULL) * 8 + k];
+                } else {
+                    const int dk = done_dk++;
+                    if (!cta_wait(bar(BB_COPY + dk % BS_NCOPY), (dk / BS_NCOPY) & 1, fail, p.status)) continue;
+                    const uint32_t s0 = ctab[(dk % BS_NCOPY) * 2], s1 = ctab[(dk % BS_NCOPY) * 2 + 1];
+                    const int x0 = 32 * chunk_of_it(it);
+                    tma_store_5d_hint(&tmDE, sbase + s0 * BS_SLOT, 0, i0 / 2, x0, 0, b, drop_l2);
+                    tma_store_5d_hint(&tmDE, sbase + s1 * BS_SLOT, 0, i0 / 2, x0, 1, b, drop_l2);
+                    tma_store_commit();
+                    // the previous copy's slots are free once its store has read them
+                    if (pend_mask) {
+                        tma_store_wait_read1();
+                        free_mask |= pend_mask;
+                    }
+                    pend_mask = (1u << s0) | (1u << s1);
                 }
-                for (int k = 0; k < nslots(it); ++k) release(it, k);
                 issue_loads();
             }
-            if (*fail)   // loads already issued land before the CTA's shared memory is released
-                for (int it = max(next_load - BS_NFULL, 0); it < next_load; ++it)
-                    mbar_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1);
+            tma_store_wait_read0();
+            if (*fail) {   // loads already issued land before the CTA's shared memory is released
+                for (int li = max(load_li - BS_NFULL, 0); li < load_li; ++li)
+                    mbar_wait(bar(BB_FULL + li % BS_NFULL), (li / BS_NFULL) & 1);
+                for (int dk = max(load_dk - BS_NCOPY, 0); dk < load_dk; ++dk)
+                    mbar_wait(bar(BB_COPY + dk % BS_NCOPY), (dk / BS_NCOPY) & 1);
+            }
         }
         __syncwarp();
         named_bar_sync(2, BS_THR);   // the ring is drained: the compute warps may reuse it
@@ -359,11 +430,11 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) qacc[hh][0][x] = qacc[hh][1][x] = 0.f;
 
-            for (int it = 0; it < 2 * nch; ++it) {
-                const int c = chunk_of(it), j0 = 32 * c;
-                const bool pass2 = it >= nch;
+            for (int li = 0; li < nit; ++li) {
+                const int c = chunk_of_li(li), j0 = 32 * c;
+                const bool pass2 = li >= nl;
 
-                if (it == nch) {
+                if (li == nl) {
                     // ---------------- D over lanes, then quadrants
                     tmem_st_wait();
                     float *wd = reinterpret_cast<float *>(sp + S::WD);
@@ -387,7 +458,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         }
                 }
 
-                cta_wait(bar(BB_FULL + it % BS_NFULL), (it / BS_NFULL) & 1, fail, p.status);
+                cta_wait(bar(BB_FULL + li % BS_NFULL), (li / BS_NFULL) & 1, fail, p.status);
                 // ---------------- S = Q K^T, dP = dO V^T (warp MMAs), or the kept ones
                 float sv[2][4], da[2][4];
                 const uint32_t kcol = tl + BS_TM_KEEP + 32 * c + 2 * hq;
@@ -398,8 +469,8 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     tmem_ld2(kcol + 24, da[0][1], da[1][1]);
                     tmem_ld_wait();
                 } else {
-                    warp_scores2<1>(slot_addr(it, 4), q, t, hq, qf, sv);
-                    warp_scores2<1>(slot_addr(it, 5), q, t, hq, of, da);
+                    warp_scores2<1>(slot_addr(li, 4), q, t, hq, qf, sv);
+                    warp_scores2<1>(slot_addr(li, 5), q, t, hq, of, da);
                     if (keep) {
                         tmem_st2(kcol, sv[0][0], sv[1][0]);
                         tmem_st2(kcol + 8, sv[0][1], sv[1][1]);
@@ -409,12 +480,12 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
 
                 // ---------------- FiLM and u from TMEM
-                cta_wait(bar(BB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
+                cta_wait(bar(BB_FILM_FULL + (li & 1)), (li >> 1) & 1, fail, p.status);
                 tc_fence_after();
                 float fg[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, fb[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, fu[2][2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const uint32_t fcol = BS_TM_FILM + 32 * (it & 1) + 16 * e, ucol = BS_TM_U + 32 * (it & 1) + 16 * e;
+                    const uint32_t fcol = BS_TM_FILM + 32 * (li & 1) + 16 * e, ucol = BS_TM_U + 32 * (li & 1) + 16 * e;
                     if (!light) {   // Light Edge: gamma, beta from y alone
                         tmem_ld2(tl + fcol + 2 * hq, fg[e][0], fg[e][1]);
                         tmem_ld2(tl + fcol + NH + 2 * hq, fb[e][0], fb[e][1]);
@@ -424,7 +495,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (t == 0) mbar_arrive(bar(BB_FILM_EMPTY + (it & 1)));
+                if (t == 0) mbar_arrive(bar(BB_FILM_EMPTY + (li & 1)));
                 const bool mcol = mj[j0 + 8 * q + g8] != 0;
                 // av: a; sv: s; gm: gamma; da: dA (the layer) or dP with the edge
                 // term u in fu (the unnormalised variant: u enters dS' directly)
@@ -457,13 +528,13 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) dsum[e][hh] += av[hh][e] * da[hh][e];
                     __syncwarp();
-                    if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
+                    if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (li & 3)));
                     continue;
                 }
 
                 // ---------------- pass 2: dS', df and a tiles for the tensor cores / warp MMAs;
                 // the previous chunk's weight-gradient products read the tile until they complete
-                if (it > nch) cta_wait(bar(BB_WG_DONE + ((it - nch - 1) & 1)), ((it - nch - 1) >> 1) & 1, fail, p.status);
+                if (li > nl) cta_wait(bar(BB_WG_DONE + ((li - nl - 1) & 1)), ((li - nl - 1) >> 1) & 1, fail, p.status);
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float dgam[2], dbet[2];
@@ -490,7 +561,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 if (t == 0) mbar_arrive(bar(BB_DF_FULL));
 
                 // ---------------- dq += ds K (warp MMAs; overlaps the tensor-core products)
-                warp_contract2<1, true>(slot_addr(it, 4), q, t, hq, da, qacc);
+                warp_contract2<1, true>(slot_addr(li, 4), q, t, hq, da, qacc);
 
                 // ---------------- the row block's share of dk_j = sum_i ds_ij q_i and dv_j =
                 // sum_i a_ij dO_i for the warp's 8 columns j (two heads): warp MMAs with M = j,
@@ -534,7 +605,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 
                 // ---------------- dE = dE' + df Wfe^T (Light Edge: dE = dE'), written from registers:
                 // the dE' tile stays as loaded for the weight-gradient product that reads it
-                cta_wait(bar(BB_DE_FULL), (it - nch) & 1, fail, p.status);
+                cta_wait(bar(BB_DE_FULL), (li - nl) & 1, fail, p.status);
                 tc_fence_after();
                 {
                     const int j = j0 + 8 * q + g8;
@@ -547,18 +618,18 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         }
                         const int i = i0 + 2 * c4 + e;
                         if (i < n && j < n)
-                            residual16_to_global(sp + (slot_addr(it, 2 + e) - sbase) + L * 128, L, hq, dv, !light,
+                            residual16_to_global(sp + (slot_addr(li, 2 + e) - sbase) + L * 128, L, hq, dv, !light,
                                                  p.dE + ((((size_t)b * n + i) * n + j) * DE + 16 * hq));
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (it & 3)));
+                if (t == 0) mbar_arrive(bar(BB_STAGE_DONE + (li & 3)));
             }
 
             // the last chunk's weight-gradient products complete before the tile and the
             // accumulator are read
-            cta_wait(bar(BB_WG_DONE + ((nch - 1) & 1)), ((nch - 1) >> 1) & 1, fail, p.status);
+            if (nl > 0) cta_wait(bar(BB_WG_DONE + ((nl - 1) & 1)), ((nl - 1) >> 1) & 1, fail, p.status);
             // ---------------- row-block results: dq through the (now idle) DA tiles,
             // four heads at a time; dg and the weight-gradient partials
             float *part = reinterpret_cast<float *>(sp + S::DA);
@@ -607,8 +678,13 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             tc_fence_after();
             if (hq == 0) {
                 float v[16];
-                tmem_ld16(tl + BS_TM_W + (q < 2 ? 0 : NF), v);
-                tmem_ld_wait();
+                if (nl > 0) {
+                    tmem_ld16(tl + BS_TM_W + (q < 2 ? 0 : NF), v);
+                    tmem_ld_wait();
+                } else {   // no live chunk: no product was accumulated
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) v[k] = 0.f;
+                }
                 if (q < 2) {
                     const int c = 32 * q + t;
 #pragma unroll
@@ -641,9 +717,10 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
                               cudaStream_t st) {
     static std::atomic<uint32_t> attr_set{0};
     if (cudaError_t e = ensure_smem_attr(k_bwd_stream, BsSmem::BYTES, attr_set); e != cudaSuccess) return e;
-    CUtensorMap mE, mDEp, mK, mV;
+    CUtensorMap mE, mDEp, mDE, mK, mV;
     if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mDEp, a.dEout, d.B, d.n, false, 32, 1) ||
-        !encode_node_map(&mK, a.K, d.B, d.n, 32) || !encode_node_map(&mV, a.V, d.B, d.n, 32))
+        !encode_pair_map(&mDE, a.dE, d.B, d.n, false, 32, 1) || !encode_node_map(&mK, a.K, d.B, d.n, 32) ||
+        !encode_node_map(&mV, a.V, d.B, d.n, 32))
         return cudaErrorInvalidValue;
     BwdStreamParams p;
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
@@ -662,7 +739,7 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
     p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
     p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)sm_count();
-    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mK, mV, p);
+    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, p);
     return cudaGetLastError();
 }
 

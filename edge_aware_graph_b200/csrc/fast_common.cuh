@@ -226,6 +226,32 @@ __device__ __forceinline__ void residual16_to_global(const uint8_t *row, uint32_
 
 __device__ __forceinline__ void flag_timeout(int *status) { atomicExch(status, DEV_TIMEOUT); }
 
+// Block sparsity of a row block (the rows i0 .. i0+TB-1 of graph b): bit c is
+// set when chunk c (columns 32c .. 32c+31) holds at least one valid pair, i.e.
+// some row of the block and some column of the chunk are nodes of the graph.
+// Every other pair of the chunk has a = 0, so its outputs are its inputs (E' =
+// E, dE = dE') and it adds nothing to any sum.  One warp; every lane returns
+// the mask.  n is even, so the mask row is 2-byte aligned.
+__device__ __forceinline__ uint32_t live_chunk_mask(const uint8_t *M, int b, int n, int i0, int t) {
+    const uint8_t *mb = M + (size_t)b * n;
+    const bool row = t < TB && i0 + t < n && mb[i0 + t] != 0;
+    if (!__any_sync(0xffffffffu, row)) return 0u;
+    const uint16_t *m2 = reinterpret_cast<const uint16_t *>(mb);
+    uint32_t any = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int j = 32 * t + 2 * k;
+        if (j < n) any |= m2[j >> 1];
+    }
+    return __ballot_sync(0xffffffffu, any != 0);
+}
+
+// Position of the k-th (from 0) set bit of m; m has more than k bits set.
+__device__ __forceinline__ int nth_set_bit(uint32_t m, int k) {
+    for (int x = 0; x < k; ++x) m &= m - 1u;
+    return __ffs(m) - 1;
+}
+
 // Bounded wait on phase `parity` of mbarrier `bar` that gives up for the
 // whole CTA.  `fail` is a flag in shared memory, zero at the start.  The
 // first wait of the CTA that runs out of polls sets it and records

@@ -14,6 +14,13 @@
 // ones pass 1 brought into L2 last: E leaves HBM once, E' is written once and
 // the [B,H,n,n] map never leaves the chip.  No CTA waits for another one.
 //
+// Block sparsity (as a block mask lets FlexAttention skip whole blocks): a
+// chunk with no valid pair (no node among the CTA's rows, or none among the
+// chunk's columns: padding of a smaller graph) has a = 0 everywhere, so E' = E
+// there.  Such a chunk skips pass 1 and in pass 2 is only copied by the TMA
+// warp (loaded and stored back, bit for bit); the compute and MMA warps never
+// see it.  A CTA whose rows are all padding copies its whole slice.
+//
 // Warp roles.  Warps 0..15 compute, in two groups of eight that take the
 // chunks in turn (group G = W / 8 takes the iterations it = G, G + 2, ...):
 // while one group waits for its chunk's tensor-core products, the other works
@@ -58,15 +65,21 @@ struct FsSmem {
     static constexpr uint32_t G = FIN + 512;                  // g_b [16]
     static constexpr uint32_t MJ = G + 64;                    // mask of the graph's nodes [n <= 1024]
     static constexpr uint32_t BAR = MJ + 1024;                // mbarriers, see below
-    static constexpr uint32_t TM = BAR + 8 * 17;              // TMEM base address
+    static constexpr uint32_t TM = BAR + 8 * 21;              // TMEM base address
     static constexpr uint32_t FAIL = TM + 8;                  // CTA failure flag (a wait ran out)
-    static constexpr uint32_t BYTES = TM + 16 + 1024;         // + alignment slack
+    static constexpr uint32_t STAB = TM + 16;                 // slot table [4 live iterations][4] u8
+    static constexpr uint32_t CTAB = STAB + 16;               // slots of the copies [4][2] u8
+    static constexpr uint32_t LIVE = CTAB + 8;                // live-chunk mask of the row block
+    static constexpr uint32_t LC = LIVE + 8;                  // the live chunks, ascending [32] u8
+    static constexpr uint32_t BYTES = LC + 32 + 1024;         // + alignment slack
     static constexpr uint32_t OPART = 0;                      // [2][4][8][256] f32 O partials (ring drained)
 };
-// mbarriers: full[4] (loads), film_full[2], film_empty[2], a_full[2], edge_full[2], stage_done[4],
-// mma_final (all MMAs of the CTA complete)
+// mbarriers: full[4] (loads of live iterations), film_full[2], film_empty[2], a_full[2],
+// edge_full[2], stage_done[4], mma_final (all MMAs of the CTA complete), copy[4] (loads of
+// dead chunks)
 constexpr int FB_FULL = 0, FB_FILM_FULL = 4, FB_FILM_EMPTY = 6, FB_A_FULL = 8, FB_EDGE_FULL = 10,
-              FB_STAGE_DONE = 12, FB_MMA_FINAL = 16;
+              FB_STAGE_DONE = 12, FB_MMA_FINAL = 16, FB_COPY = 17;
+constexpr int FS_NCOPY = 4;               // dead-chunk copies in flight
 
 // TMEM columns: FiLM 0..63 (two buffers), edge update 64..319 (two buffers),
 // pass-1 scores from 320 on (16 per chunk, kept when nch <= 12 so pass 2 needs no K)
@@ -100,7 +113,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
     const int tid = threadIdx.x, W = tid >> 5, t = tid & 31, c4 = t & 3, g8 = t >> 2;
     const int G = (W >> 3) & 1, q = W & 3, hp = (W >> 2) & 1;   // group, TMEM quadrant, head quad
-    const int n = p.n, nch = (n + 31) / 32, nit = 2 * nch;
+    const int n = p.n, nch = (n + 31) / 32;
     const int b = blockIdx.y, i0 = blockIdx.x * TB;
     const uint32_t bars = sbase + S::BAR;
     auto bar = [&](int k) { return bars + 8 * k; };
@@ -108,20 +121,23 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     uint8_t *mj = sp + S::MJ;
     volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
 
-    // iteration it: pass 1 walks chunks 0..nch-1, pass 2 walks nch-1..0;
-    // group it & 1 computes it.  Its slots, from slot_base(it) on: pass 1
+    // Block sparsity: a chunk holding no valid pair (live_chunk_mask) needs no
+    // arithmetic, its E' is its E.  The TMA warp loads iterations it in order:
+    // pass 1 the nl live chunks, ascending; pass 2 all nch chunks, descending,
+    // where a live chunk is computed and a dead one only copied (its two E
+    // tiles loaded and stored back).  The live iterations, numbered li = 0 ..
+    // 2 nl - 1 (pass 1, then pass 2's live chunks), are the ones the MMA warp
+    // and the compute groups see: group li & 1 computes li.  Slots: pass 1
     // E(s=0), E(s=1), K (Light Edge: K alone); pass 2 E(s=0), E(s=1), V when
-    // the pass-1 scores stay in TMEM, else E, E, K, V.
+    // the pass-1 scores stay in TMEM, else E, E, K, V; a dead chunk E, E.  The
+    // TMA warp takes any free slots and records them in table entry li % 4
+    // (load barrier li % 4), which the other warps read after that barrier.
     const bool light = p.light != 0;
     const bool keep_s = nch <= FS_KEEP_S_MAX_CHUNKS;
     const int ns1 = light ? 1 : 3, ks1 = light ? 0 : 2;
     const int ns2 = keep_s ? 3 : 4, vslot = ns2 - 1;
-    auto chunk_of = [&](int it) { return it < nch ? it : nit - 1 - it; };
-    auto nslots = [&](int it) { return it < nch ? ns1 : ns2; };
-    auto slot_base = [&](int it) { return (ns1 * min(it, nch) + ns2 * max(it - nch, 0)) % FS_SLOTS; };
-    auto slot_addr = [&](int it, int k) { return sbase + (uint32_t)((slot_base(it) + k) % FS_SLOTS) * FS_SLOT; };
-    // the first pass-2 iteration of group gg
-    auto first_p2 = [&](int gg) { return nch + ((gg - nch) & 1); };
+    volatile uint8_t *stab = sp + S::STAB;
+    auto slot_addr = [&](int li, int k) { return sbase + (uint32_t)stab[(li % FS_NFULL) * 4 + k] * FS_SLOT; };
 
     // ---------------- setup: barriers, TMEM, operands
     if (tid == 0) {
@@ -136,12 +152,18 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         mbar_init(bar(FB_EDGE_FULL + 1), 1);
         for (int k = 0; k < 4; ++k) mbar_init(bar(FB_STAGE_DONE + k), GW);
         mbar_init(bar(FB_MMA_FINAL), 1);
+        for (int k = 0; k < FS_NCOPY; ++k) mbar_init(bar(FB_COPY + k), 1);
         fence_mbar_init();
         *fail = 0;
     }
     if (W == 0) {
         tmem_alloc(sbase + S::TM, FS_TM_COLS);
         tmem_relinquish();
+    }
+    if (W == 1) {
+        const uint32_t lm = live_chunk_mask(p.M, b, n, i0, t);
+        if (t == 0) *reinterpret_cast<volatile uint32_t *>(sp + S::LIVE) = lm;
+        if ((lm >> t) & 1u) sp[S::LC + __popc(lm & ((1u << t) - 1u))] = (uint8_t)t;
     }
     // operand images: Wfe^T (FiLM B, swizzled) and We^T (edge-update B, no swizzle), 2 KB each
     if (tid < 256) reinterpret_cast<uint4 *>(sp + S::WFE)[tid] = reinterpret_cast<const uint4 *>(p.img)[tid];
@@ -154,23 +176,31 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+    const uint32_t live = *reinterpret_cast<volatile uint32_t *>(sp + S::LIVE);
+    const int nl = __popc(live), nit = 2 * nl, nload = nl + nch;
+    // chunk of live iteration li; chunk of load iteration it
+    const volatile uint8_t *lc = sp + S::LC;
+    auto chunk_of_li = [&](int li) { return (int)lc[li < nl ? li : nit - 1 - li]; };
+    auto chunk_of_it = [&](int it) { return it < nl ? (int)lc[it] : nch - 1 - (it - nl); };
+    // the first pass-2 live iteration of group gg
+    auto first_p2 = [&](int gg) { return nl + ((gg - nl) & 1); };
 
     if (W == NWARP) {
         // ================= MMA issuer: FiLM as tiles land, edge updates per group on demand
         if (t == 0) {
             const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_e = idesc_bf16_f32(128, DE);
-            auto issue_film = [&](int it) {   // into the TMEM range of group it & 1
+            auto issue_film = [&](int li) {   // into the TMEM range of group li & 1
                 tc_fence_after();
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    const uint32_t a0 = slot_addr(it, s);
+                    const uint32_t a0 = slot_addr(li, s);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tmem + FS_TM_FILM + 32 * (it & 1) + 16 * s,
+                        mma_bf16_ss(tmem + FS_TM_FILM + 32 * (li & 1) + 16 * s,
                                     smem_desc(a0 + kk * 32, 16, 1024, LAYOUT_SW128),
                                     smem_desc(sbase + S::WFE + kk * 32, 16, 1024, LAYOUT_SW128), idesc_f, kk > 0);
                 }
-                mma_commit(bar(FB_FILM_FULL + (it & 1)));
+                mma_commit(bar(FB_FILM_FULL + (li & 1)));
             };
             auto issue_edge = [&](int gg) {   // group gg's a buffer -> its TMEM buffer
                 tc_fence_after();
@@ -198,9 +228,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
 #pragma unroll
                 for (int gg = 0; gg < 2; ++gg) {
-                    const int it = next_edge[gg];
-                    if (it < nit && it < next_film &&
-                        mbar_test_wait(bar(FB_A_FULL + gg), ((it - nch) >> 1) & 1)) {
+                    const int li = next_edge[gg];
+                    if (li < nit && li < next_film &&
+                        mbar_test_wait(bar(FB_A_FULL + gg), ((li - nl) >> 1) & 1)) {
                         issue_edge(gg);
                         next_edge[gg] += 2;
                         progressed = true;
@@ -226,49 +256,76 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         __syncwarp();
         named_bar_sync(2, FS_THR);
     } else if (W == NWARP + 1) {
-        // ================= TMA: loads into the slot ring, E' stores
+        // ================= TMA: loads into the slot ring, E' stores, copies of dead chunks
         if (t == 0) {
             // E tiles loaded in pass 1 are read again in pass 2: keep them in L2;
             // pass-2 reads and the E' stores are not read again
             const uint64_t keep_l2 = l2_evict_last(), drop_l2 = l2_evict_first();
-            int next_load = 0, free_slots = FS_SLOTS;
-            int consumed = 0;   // iterations whose stage completion this thread has taken
-            // at most FS_NFULL iterations in flight: a load barrier is re-armed
-            // only after its previous iteration completed (Light Edge takes one
-            // slot per pass-1 chunk, so the slots alone would allow twelve)
+            volatile uint8_t *ctab = sp + S::CTAB;
+            uint32_t free_mask = (1u << FS_SLOTS) - 1u;
+            auto take_slot = [&]() {
+                const int sidx = __ffs(free_mask) - 1;
+                free_mask &= free_mask - 1u;
+                return (uint8_t)sidx;
+            };
+            auto is_live = [&](int it) { return it < nl || ((live >> chunk_of_it(it)) & 1u) != 0; };
+            // loads go out in iteration order; a live iteration waits for its
+            // load barrier to be free (at most FS_NFULL live iterations in
+            // flight: a barrier is re-armed only after its previous iteration
+            // was taken off the ring), a copy likewise for its copy barrier
+            int next_load = 0, load_li = 0, load_dk = 0, done_li = 0, done_dk = 0;
             auto issue_loads = [&]() {
-                while (next_load < nit && next_load < consumed + FS_NFULL && nslots(next_load) <= free_slots &&
-                       !*fail) {
-                    const int it = next_load, j0 = 32 * chunk_of(it);
-                    const bool pass2 = it >= nch;
-                    const uint32_t fb = bar(FB_FULL + it % FS_NFULL);
-                    mbar_expect_tx(fb, nslots(it) * FS_SLOT);
-                    const uint64_t pol = pass2 ? drop_l2 : keep_l2;
-                    if (pass2 || !light) {
-                        tma_load_5d_hint(slot_addr(it, 0), &tmE, fb, 0, i0 / 2, j0, 0, b, pol);
-                        tma_load_5d_hint(slot_addr(it, 1), &tmE, fb, 0, i0 / 2, j0, 1, b, pol);
-                    }
+                while (next_load < nload && !*fail) {
+                    const int it = next_load, j0 = 32 * chunk_of_it(it);
+                    const bool pass2 = it >= nl;
+                    if (is_live(it)) {
+                        const int li = load_li, ns = pass2 ? ns2 : ns1;
+                        if (li >= done_li + FS_NFULL || __popc(free_mask) < ns) break;
+                        for (int k = 0; k < ns; ++k) stab[(li % FS_NFULL) * 4 + k] = take_slot();
+                        const uint32_t fb = bar(FB_FULL + li % FS_NFULL);
+                        mbar_expect_tx(fb, ns * FS_SLOT);   // releases the table entry too
+                        const uint64_t pol = pass2 ? drop_l2 : keep_l2;
+                        if (pass2 || !light) {
+                            tma_load_5d_hint(slot_addr(li, 0), &tmE, fb, 0, i0 / 2, j0, 0, b, pol);
+                            tma_load_5d_hint(slot_addr(li, 1), &tmE, fb, 0, i0 / 2, j0, 1, b, pol);
+                        }
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        if (!pass2) tma_load_3d(slot_addr(it, ks1) + k * 4096, &tmK, fb, 64 * k, j0, b);
-                        else if (!keep_s) tma_load_3d(slot_addr(it, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
-                        if (pass2) tma_load_3d(slot_addr(it, vslot) + k * 4096, &tmV, fb, 64 * k, j0, b);
+                        for (int k = 0; k < 4; ++k) {
+                            if (!pass2) tma_load_3d(slot_addr(li, ks1) + k * 4096, &tmK, fb, 64 * k, j0, b);
+                            else if (!keep_s) tma_load_3d(slot_addr(li, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
+                            if (pass2) tma_load_3d(slot_addr(li, vslot) + k * 4096, &tmV, fb, 64 * k, j0, b);
+                        }
+                        if (!pass2 && !light && li + FS_PF < nl)
+                            for (int s = 0; s < 2; ++s)
+                                tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * lc[li + FS_PF], s, b);
+                        ++load_li;
+                    } else {
+                        const int dk = load_dk;
+                        if (dk >= done_dk + FS_NCOPY || __popc(free_mask) < 2) break;
+                        const uint32_t cb = bar(FB_COPY + dk % FS_NCOPY);
+                        mbar_expect_tx(cb, 2 * FS_SLOT);
+#pragma unroll
+                        for (int s = 0; s < 2; ++s) {
+                            const uint8_t sl = take_slot();
+                            ctab[(dk % FS_NCOPY) * 2 + s] = sl;
+                            tma_load_5d_hint(sbase + sl * FS_SLOT, &tmE, cb, 0, i0 / 2, j0, s, b, drop_l2);
+                        }
+                        ++load_dk;
                     }
-                    if (!pass2 && !light && it + FS_PF < nch)
-                        for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (it + FS_PF), s, b);
-                    free_slots -= nslots(it);
                     ++next_load;
                 }
             };
-            for (int c = 0; c < nch && c < FS_PF && !light; ++c)
-                for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * c, s, b);
+            for (int c = 0; c < nl && c < FS_PF && !light; ++c)
+                for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * lc[c], s, b);
             issue_loads();
-            // stage completions arrive in iteration order within each group;
-            // the two groups' iterations interleave, so they are taken in order
-            int pending = 0;                 // pass-2 stores not yet known to have read their slots
-            for (int it = 0; it < nit; ++it) {
-                const bool pass2 = it >= nch;
-                if (it == nch && p.prefetch_ahead && !light) {
+            // iterations are taken off the ring in order: a live one once its
+            // group is done with it (stage_done), a copy once its tiles landed;
+            // a pass-2 chunk's E tiles (E' in place, or the copy) are stored
+            // and their slots are free once the store has read them
+            uint32_t pend_mask = 0u;   // slots of the last store, not yet known to have read them
+            for (int it = 0; it < nload; ++it) {
+                const bool pass2 = it >= nl;
+                if (it == nl && p.prefetch_ahead && !light) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
@@ -277,28 +334,41 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                             for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, s, pb);
                     }
                 }
-                if (!cta_wait(bar(FB_STAGE_DONE + (it & 3)), (it >> 2) & 1, fail, p.status)) continue;
-                consumed = it + 1;
-                if (pass2) {
-                    const int j0 = 32 * chunk_of(it);
-                    tma_store_5d_hint(&tmEo, slot_addr(it, 0), 0, i0 / 2, j0, 0, b, drop_l2);
-                    tma_store_5d_hint(&tmEo, slot_addr(it, 1), 0, i0 / 2, j0, 1, b, drop_l2);
-                    tma_store_commit();
-                    // the previous pass-2 chunk's slots are free once its store has read them
-                    if (++pending > 1) {
-                        tma_store_wait_read1();
-                        free_slots += ns2;
-                        --pending;
-                    }
+                const int j0 = 32 * chunk_of_it(it);
+                uint32_t s0, s1;        // the slots of the E tiles a pass-2 store reads
+                if (is_live(it)) {
+                    const int li = done_li++;
+                    if (!cta_wait(bar(FB_STAGE_DONE + (li & 3)), (li >> 2) & 1, fail, p.status)) continue;
+                    const int ns = pass2 ? ns2 : ns1;
+                    for (int k = pass2 ? 2 : 0; k < ns; ++k) free_mask |= 1u << stab[(li % FS_NFULL) * 4 + k];
+                    s0 = stab[(li % FS_NFULL) * 4];
+                    s1 = stab[(li % FS_NFULL) * 4 + 1];
                 } else {
-                    free_slots += ns1;
+                    const int dk = done_dk++;
+                    if (!cta_wait(bar(FB_COPY + dk % FS_NCOPY), (dk / FS_NCOPY) & 1, fail, p.status)) continue;
+                    s0 = ctab[(dk % FS_NCOPY) * 2];
+                    s1 = ctab[(dk % FS_NCOPY) * 2 + 1];
+                }
+                if (pass2) {
+                    tma_store_5d_hint(&tmEo, sbase + s0 * FS_SLOT, 0, i0 / 2, j0, 0, b, drop_l2);
+                    tma_store_5d_hint(&tmEo, sbase + s1 * FS_SLOT, 0, i0 / 2, j0, 1, b, drop_l2);
+                    tma_store_commit();
+                    // the previous store's slots are free once it has read them
+                    if (pend_mask) {
+                        tma_store_wait_read1();
+                        free_mask |= pend_mask;
+                    }
+                    pend_mask = (1u << s0) | (1u << s1);
                 }
                 issue_loads();
             }
             tma_store_wait_read0();
-            if (*fail)   // loads already issued land before the CTA's shared memory is released
-                for (int it = max(next_load - FS_NFULL, 0); it < next_load; ++it)
-                    mbar_wait(bar(FB_FULL + it % FS_NFULL), (it / FS_NFULL) & 1);
+            if (*fail) {   // loads already issued land before the CTA's shared memory is released
+                for (int li = max(load_li - FS_NFULL, 0); li < load_li; ++li)
+                    mbar_wait(bar(FB_FULL + li % FS_NFULL), (li / FS_NFULL) & 1);
+                for (int dk = max(load_dk - FS_NCOPY, 0); dk < load_dk; ++dk)
+                    mbar_wait(bar(FB_COPY + dk % FS_NCOPY), (dk / FS_NCOPY) & 1);
+            }
         }
         __syncwarp();
         named_bar_sync(2, FS_THR);   // the ring is drained: the compute warps may reuse it
@@ -315,13 +385,13 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         const bool mrow[2] = {i0 + 2 * c4 < n && p.M[(size_t)b * n + i0 + 2 * c4] != 0,
                               i0 + 2 * c4 + 1 < n && p.M[(size_t)b * n + i0 + 2 * c4 + 1] != 0};
 
-        // s' of iteration it for the thread's 2 pairs x 4 heads: sx[k][e] with
+        // s' of live iteration li for the thread's 2 pairs x 4 heads: sx[k][e] with
         // k = 2 * pair + hh (heads hqa: k = 0, 1; hqb: k = 2, 3), -inf where invalid
-        auto scores = [&](int it, bool pass2, float (&sx)[4][2], bool (&valid)[2]) {
-            const int j0 = 32 * chunk_of(it);
-            cta_wait(bar(FB_FULL + it % FS_NFULL), (it / FS_NFULL) & 1, fail, p.status);
+        auto scores = [&](int li, bool pass2, float (&sx)[4][2], bool (&valid)[2]) {
+            const int c = chunk_of_li(li), j0 = 32 * c;
+            cta_wait(bar(FB_FULL + li % FS_NFULL), (li / FS_NFULL) & 1, fail, p.status);
             float sa[2][4], sb[2][4];
-            const uint32_t scol = tl + FS_TM_S + 16 * chunk_of(it);
+            const uint32_t scol = tl + FS_TM_S + 16 * c;
             if (pass2 && keep_s) {
                 tmem_ld2(scol + 2 * hqa, sa[0][0], sa[1][0]);
                 tmem_ld2(scol + 2 * hqa + 8, sa[0][1], sa[1][1]);
@@ -329,7 +399,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 tmem_ld2(scol + 2 * hqb + 8, sb[0][1], sb[1][1]);
                 tmem_ld_wait();
             } else {
-                const uint32_t ks = slot_addr(it, pass2 ? 2 : ks1);
+                const uint32_t ks = slot_addr(li, pass2 ? 2 : ks1);
                 warp_scores2<1>(ks, q, t, hqa, qfa, sa);
                 warp_scores2<1>(ks, q, t, hqb, qfb, sb);
                 if (keep_s) {
@@ -342,11 +412,11 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             // FiLM of the pair: gamma, beta of the four heads
             float gm[2][4] = {}, bt[2][4] = {};
             if (!light) {
-                cta_wait(bar(FB_FILM_FULL + (it & 1)), (it >> 1) & 1, fail, p.status);
+                cta_wait(bar(FB_FILM_FULL + (li & 1)), (li >> 1) & 1, fail, p.status);
                 tc_fence_after();
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const uint32_t fcol = FS_TM_FILM + 32 * (it & 1) + 16 * e + 4 * hp;
+                    const uint32_t fcol = FS_TM_FILM + 32 * (li & 1) + 16 * e + 4 * hp;
                     tmem_ld2(tl + fcol, gm[e][0], gm[e][1]);
                     tmem_ld2(tl + fcol + 2, gm[e][2], gm[e][3]);
                     tmem_ld2(tl + fcol + NH, bt[e][0], bt[e][1]);
@@ -355,7 +425,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (t == 0) mbar_arrive(bar(FB_FILM_EMPTY + (it & 1)));
+                if (t == 0) mbar_arrive(bar(FB_FILM_EMPTY + (li & 1)));
             }
             const bool mcol = mj[j0 + 8 * q + g8] != 0;
 #pragma unroll
@@ -382,10 +452,10 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     rm[e][k] = -INFINITY;
                     rl[e][k] = 0.f;
                 }
-            for (int it = G; it < nch; it += 2) {
+            for (int li = G; li < nl; li += 2) {
                 float sx[4][2];
                 bool valid[2];
-                scores(it, false, sx, valid);
+                scores(li, false, sx, valid);
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
 #pragma unroll
@@ -398,7 +468,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         }
                     }
                 __syncwarp();
-                if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
+                if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (li & 3)));
             }
             // ---------------- end of pass 1: statistics over lanes, then (group, quadrant)
             tmem_st_wait();
@@ -455,10 +525,10 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                 for (int x = 0; x < 4; ++x) oa[hh][mt][x] = ob[hh][mt][x] = 0.f;
-        for (int it = first_p2(G); it < nit; it += 2) {
+        for (int li = first_p2(G); li < nit; li += 2) {
             float sx[4][2];
             bool valid[2];
-            scores(it, true, sx, valid);
+            scores(li, true, sx, valid);
             // a (for O) and the edge update's coefficient (a, or s' when unnormalised)
             float pa[2][4], pb[2][4];
 #pragma unroll
@@ -482,12 +552,12 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             if (t == 0) mbar_arrive(bar(FB_A_FULL + G));
 
             // O += a V on warp MMAs (overlaps the edge MMA)
-            const uint32_t vs = slot_addr(it, vslot);
+            const uint32_t vs = slot_addr(li, vslot);
             warp_contract2<1, true>(vs, q, t, hqa, pa, oa);
             warp_contract2<1, true>(vs, q, t, hqb, pb, ob);
 
             // E' = E + (a We), in place (the TMA warp stores it)
-            cta_wait(bar(FB_EDGE_FULL + G), ((it - nch) >> 1) & 1, fail, p.status);
+            cta_wait(bar(FB_EDGE_FULL + G), ((li - nl) >> 1) & 1, fail, p.status);
             tc_fence_after();
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -496,13 +566,13 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     float dv[16];
                     tmem_ld16(tl + FS_TM_EDGE + 128 * G + 64 * e + 32 * hp + 16 * half, dv);
                     tmem_ld_wait();
-                    add_residual16(sp + (slot_addr(it, e) - sbase) + L * 128, L, 2 * hp + half, dv);
+                    add_residual16(sp + (slot_addr(li, e) - sbase) + L * 128, L, 2 * hp + half, dv);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (it & 3)));
+            if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (li & 3)));
         }
 
         // ---------------- O: sum over the (group, quadrant) warps (in the drained ring)

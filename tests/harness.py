@@ -48,7 +48,9 @@ def custom_case(B, n, dx, de, dy, H, dh, dtype, seed, mask="random", with_grads=
     """Dense-family case of arbitrary dims with a chosen mask pattern.
 
     mask: "prefix" (random real counts), "random" (non-prefix, includes one
-    fully masked graph and one single-node graph when B >= 3), "full".
+    fully masked graph and one single-node graph when B >= 3), "blocks" (node
+    spans that leave whole 32-column chunks and 8-row blocks without a valid
+    pair between live ones, an empty graph, a single-node graph), "full".
     """
     p = I.Preset("custom", seed, dtype, B=B, n=n, dx=dx, de=de, dy=dy, H=H, dh=dh, family="dense",
                  training=with_grads, n_real=(n,))
@@ -61,6 +63,12 @@ def custom_case(B, n, dx, de, dy, H, dh, dtype, seed, mask="random", with_grads=
             M[1] = 0
             M[2] = 0
             M[2, n // 2] = 1
+    elif mask == "blocks":
+        M = np.zeros((B, n), np.uint8)
+        for b in range(B):
+            spans = ([(0, 20), (70, 90), (n - 10, n)], [(40, 50)], [], [(n // 2, n // 2 + 1)])[b % 4]
+            for lo, hi in spans:
+                M[b, lo:min(hi, n)] = 1
     elif mask == "prefix":
         nr = rng.integers(1, n + 1, size=B)
         M = (np.arange(n)[None] < nr[:, None]).astype(np.uint8)

@@ -98,6 +98,10 @@ CASES = [
     (4, 16, 256, 64, 64, 8, 32, "bf16", "random"),
     (4, 30, 256, 64, 64, 8, 32, "bf16", "random"),
     (3, 64, 1024, 64, 64, 8, 32, "bf16", "random"),    # widest node features
+    # block sparsity: chunks and row blocks without a valid pair between live
+    # ones (copied, not computed), with S, dP kept and reloaded
+    (4, 160, 256, 64, 64, 8, 32, "bf16", "blocks"),
+    (4, 250, 256, 64, 64, 8, 32, "bf16", "blocks"),
 ]
 
 
@@ -134,10 +138,12 @@ def test_light_edge_variant(oracle_lib):
     assert np.abs(dbk).max() <= TOL["bf16"] * np.abs(ref["dbq"]).max()
 
 
-def test_masked_garbage_is_ignored():
+@pytest.mark.parametrize("mask", ["random", "blocks"])
+def test_masked_garbage_is_ignored(mask):
     """Large finite values in masked node rows and invalid pairs leave every
-    valid output bitwise unchanged; masked outputs equal their inputs."""
-    p, d, W = custom_case(4, 96, 256, 64, 64, 8, 32, "bf16", seed=3, mask="random")
+    valid output bitwise unchanged; masked outputs equal their inputs (also
+    where whole chunks hold no valid pair and are copied)."""
+    p, d, W = custom_case(4, 96, 256, 64, 64, 8, 32, "bf16", seed=3, mask=mask)
     buf = make(p, d, W, backward=True)
     buf.forward(); buf.backward()
     base = {k: getattr(buf, k).clone() for k in ("Xout", "Eout", "dX", "dE", "dy")}
