@@ -165,13 +165,15 @@ def test_masked_garbage_is_ignored(mask):
     assert torch.equal(buf.dy, base["dy"])
     # dk, dv are fp32 sums over row blocks that arrive in the order the CTAs run,
     # so what depends on them (dX, dWk, dbk, dWv, dbv) may differ in the last bits
-    # between any two calls; garbage reaching them would show at its 1e3 scale
+    # between any two calls (fp32: 1e-3 of the scale; bf16 dX: such a difference
+    # can move a rounding by one bf16 step, at most 2^-7 of the element); garbage
+    # reaching them would show at its 1e3 scale
     for k in base_dw:
         if k in ("Wk", "bk", "Wv", "bv"):
             assert rel_err(buf.dW[k], base_dw[k].cpu().numpy()) <= 1e-3, k
         else:
             assert torch.equal(buf.dW[k], base_dw[k]), k
-    assert rel_err(buf.dX[rt], base["dX"][rt].float().cpu().numpy()) <= 1e-3
+    assert rel_err(buf.dX[rt], base["dX"][rt].float().cpu().numpy()) <= 2.0 ** -7
     assert torch.equal(buf.Xout[~rt], buf.X[~rt])
     assert torch.equal(buf.Eout[~vt], buf.E[~vt])
     assert torch.equal(buf.dE[~vt], buf.dEout[~vt])

@@ -88,8 +88,9 @@ def test_light_edge_ignores_wfe():
     # (fp32 additions in L2 in no fixed order): bitwise
     for a, b in zip(outs[0][:4], outs[1][:4]):
         assert torch.equal(a, b)
-    # dX and the flat weight gradients (dWk, dbk, dWv, dbv among them) do:
-    # within 1e-3 of their scale, far below what a seven-fold Wfe would change
-    for a, b in zip(outs[0][4:], outs[1][4:]):
+    # dX (bf16: one rounding step, at most 2^-7 of an element) and the flat fp32
+    # weight gradients (dWk, dbk, dWv, dbv among them: 1e-3) do, far below what a
+    # seven-fold Wfe would change
+    for (a, b), bound in zip(zip(outs[0][4:], outs[1][4:]), (2.0 ** -7, 1e-3)):
         a, b = a.float(), b.float()
-        assert float((a - b).abs().max()) <= 1e-3 * float(a.abs().max())
+        assert float((a - b).abs().max()) <= bound * float(a.abs().max())
