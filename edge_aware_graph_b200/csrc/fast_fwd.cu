@@ -17,9 +17,9 @@
 // Block sparsity (as a block mask lets FlexAttention skip whole blocks): a
 // chunk with no valid pair (no node among the CTA's rows, or none among the
 // chunk's columns: padding of a smaller graph) has a = 0 everywhere, so E' = E
-// there.  Such a chunk skips pass 1 and in pass 2 is only copied by the TMA
-// warp (loaded and stored back, bit for bit); the compute and MMA warps never
-// see it.  A CTA whose rows are all padding copies its whole slice.
+// there.  Such a chunk is only copied by the TMA warp (loaded and stored back,
+// bit for bit, while pass 1 runs); the compute and MMA warps never see it.  A
+// CTA whose rows are all padding copies its whole slice.
 //
 // Warp roles.  Warps 0..15 compute, in two groups of eight that take the
 // chunks in turn (group G = W / 8 takes the iterations it = G, G + 2, ...):
@@ -71,7 +71,8 @@ struct FsSmem {
     static constexpr uint32_t CTAB = STAB + 16;               // slots of the copies [4][2] u8
     static constexpr uint32_t LIVE = CTAB + 8;                // live-chunk mask of the row block
     static constexpr uint32_t LC = LIVE + 8;                  // the live chunks, ascending [32] u8
-    static constexpr uint32_t BYTES = LC + 32 + 1024;         // + alignment slack
+    static constexpr uint32_t DC = LC + 32;                   // the dead chunks, ascending [32] u8
+    static constexpr uint32_t BYTES = DC + 32 + 1024;         // + alignment slack
     static constexpr uint32_t OPART = 0;                      // [2][4][8][256] f32 O partials (ring drained)
 };
 // mbarriers: full[4] (loads of live iterations), film_full[2], film_empty[2], a_full[2],
@@ -123,13 +124,13 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 
     // Block sparsity: a chunk holding no valid pair (live_chunk_mask) needs no
     // arithmetic, its E' is its E.  The TMA warp loads iterations it in order:
-    // pass 1 the nl live chunks, ascending; pass 2 all nch chunks, descending,
-    // where a live chunk is computed and a dead one only copied (its two E
-    // tiles loaded and stored back).  The live iterations, numbered li = 0 ..
+    // in pass 1 the nl live chunks, ascending, and the copies of the dead ones
+    // (two E tiles loaded and stored back); in pass 2 the live chunks,
+    // descending (the load order is below).  The live iterations, numbered li = 0 ..
     // 2 nl - 1 (pass 1, then pass 2's live chunks), are the ones the MMA warp
     // and the compute groups see: group li & 1 computes li.  Slots: pass 1
     // E(s=0), E(s=1), K (Light Edge: K alone); pass 2 E(s=0), E(s=1), V when
-    // the pass-1 scores stay in TMEM, else E, E, K, V; a dead chunk E, E.  The
+    // the pass-1 scores stay in TMEM, else E, E, K, V; a copy E, E.  The
     // TMA warp takes any free slots and records them in table entry li % 4
     // (load barrier li % 4), which the other warps read after that barrier.
     const bool light = p.light != 0;
@@ -163,7 +164,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     if (W == 1) {
         const uint32_t lm = live_chunk_mask(p.M, b, n, i0, t);
         if (t == 0) *reinterpret_cast<volatile uint32_t *>(sp + S::LIVE) = lm;
-        if ((lm >> t) & 1u) sp[S::LC + __popc(lm & ((1u << t) - 1u))] = (uint8_t)t;
+        const int below = __popc(lm & ((1u << t) - 1u));   // live chunks below chunk t
+        if ((lm >> t) & 1u) sp[S::LC + below] = (uint8_t)t;
+        else if (t < nch) sp[S::DC + t - below] = (uint8_t)t;
     }
     // operand images: Wfe^T (FiLM B, swizzled) and We^T (edge-update B, no swizzle), 2 KB each
     if (tid < 256) reinterpret_cast<uint4 *>(sp + S::WFE)[tid] = reinterpret_cast<const uint4 *>(p.img)[tid];
@@ -181,7 +184,17 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     // chunk of live iteration li; chunk of load iteration it
     const volatile uint8_t *lc = sp + S::LC;
     auto chunk_of_li = [&](int li) { return (int)lc[li < nl ? li : nit - 1 - li]; };
-    auto chunk_of_it = [&](int it) { return it < nl ? (int)lc[it] : nch - 1 - (it - nl); };
+    // Load order: pass 1 takes the live chunks and the copies of the dead ones
+    // in turn (live 0, dead 0, live 1, dead 1, ..., then the rest of the longer
+    // list), so the copies fill the memory system while pass 1 computes; pass 2
+    // (it >= nch) takes the live chunks in reverse.
+    const volatile uint8_t *dc = sp + S::DC;
+    const int nmix = min(nl, nch - nl);
+    auto is_live = [&](int it) { return it >= nch || (it < 2 * nmix ? (it & 1) == 0 : 2 * nl > nch); };
+    auto p1_index = [&](int it) { return it < 2 * nmix ? it >> 1 : it - nmix; };
+    auto chunk_of_it = [&](int it) {
+        return it >= nch ? (int)lc[nch - 1 - it + nl] : is_live(it) ? (int)lc[p1_index(it)] : (int)dc[p1_index(it)];
+    };
     // the first pass-2 live iteration of group gg
     auto first_p2 = [&](int gg) { return nl + ((gg - nl) & 1); };
 
@@ -268,7 +281,6 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 free_mask &= free_mask - 1u;
                 return (uint8_t)sidx;
             };
-            auto is_live = [&](int it) { return it < nl || ((live >> chunk_of_it(it)) & 1u) != 0; };
             // loads go out in iteration order; a live iteration waits for its
             // load barrier to be free (at most FS_NFULL live iterations in
             // flight: a barrier is re-armed only after its previous iteration
@@ -277,7 +289,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             auto issue_loads = [&]() {
                 while (next_load < nload && !*fail) {
                     const int it = next_load, j0 = 32 * chunk_of_it(it);
-                    const bool pass2 = it >= nl;
+                    const bool pass2 = it >= nch;
                     if (is_live(it)) {
                         const int li = load_li, ns = pass2 ? ns2 : ns1;
                         if (li >= done_li + FS_NFULL || __popc(free_mask) < ns) break;
@@ -320,12 +332,12 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             issue_loads();
             // iterations are taken off the ring in order: a live one once its
             // group is done with it (stage_done), a copy once its tiles landed;
-            // a pass-2 chunk's E tiles (E' in place, or the copy) are stored
-            // and their slots are free once the store has read them
+            // the E tiles of a pass-2 chunk (E' in place) or of a copy are
+            // stored, and their slots are free once the store has read them
             uint32_t pend_mask = 0u;   // slots of the last store, not yet known to have read them
             for (int it = 0; it < nload; ++it) {
-                const bool pass2 = it >= nl;
-                if (it == nl && p.prefetch_ahead && !light) {
+                const bool pass2 = it >= nch;
+                if (it == nch && p.prefetch_ahead && !light) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
@@ -335,8 +347,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     }
                 }
                 const int j0 = 32 * chunk_of_it(it);
-                uint32_t s0, s1;        // the slots of the E tiles a pass-2 store reads
-                if (is_live(it)) {
+                const bool lv = is_live(it);
+                uint32_t s0, s1;        // the slots of the E tiles a store reads
+                if (lv) {
                     const int li = done_li++;
                     if (!cta_wait(bar(FB_STAGE_DONE + (li & 3)), (li >> 2) & 1, fail, p.status)) continue;
                     const int ns = pass2 ? ns2 : ns1;
@@ -349,7 +362,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     s0 = ctab[(dk % FS_NCOPY) * 2];
                     s1 = ctab[(dk % FS_NCOPY) * 2 + 1];
                 }
-                if (pass2) {
+                if (pass2 || !lv) {
                     tma_store_5d_hint(&tmEo, sbase + s0 * FS_SLOT, 0, i0 / 2, j0, 0, b, drop_l2);
                     tma_store_5d_hint(&tmEo, sbase + s1 * FS_SLOT, 0, i0 / 2, j0, 1, b, drop_l2);
                     tma_store_commit();
