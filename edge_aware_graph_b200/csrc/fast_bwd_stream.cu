@@ -32,7 +32,7 @@
 //
 // Block sparsity, as in the forward: a chunk with no valid pair adds nothing
 // to D, dq, dk, dv, dg or the weight gradients, and its dE is its dE'.  The
-// TMA warp copies its dE' tiles to dE while pass 1 runs; no other warp sees it.
+// TMA warp copies its dE' tiles to dE; no other warp sees it.
 //
 // Warp roles as in the forward pair kernel: 16 compute warps (warp W reads
 // TMEM quadrant W%4 and handles heads 2(W/4), 2(W/4)+1), one MMA warp (FiLM
@@ -134,9 +134,9 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 
     // Block sparsity: a chunk holding no valid pair (live_chunk_mask) adds
     // nothing to any sum and its dE is its dE'.  The TMA warp loads iterations
-    // it in order: in pass 1 the nl live chunks, ascending, and the copies of
-    // the dead ones (two dE' tiles loaded and stored as dE); in pass 2 the live
-    // chunks, descending (the load order is below).  The live iterations li = 0
+    // it in order: pass 1 the nl live chunks, ascending; pass 2 the live
+    // chunks, descending; then the copies of the dead ones (two dE' tiles
+    // loaded and stored as dE).  The live iterations li = 0
     // .. 2 nl - 1 (pass 1, then pass 2's live chunks) are the ones the MMA and
     // compute warps see.  Tiles of a live iteration: E(s=0), E(s=1), dE'(s=0),
     // dE'(s=1), K, then V in pass 1 (and in pass 2 when S, dP are not kept).
@@ -194,17 +194,13 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     const volatile uint8_t *lc = sp + S::LC;
     // chunk of live iteration li; chunk of load iteration it
     auto chunk_of_li = [&](int li) { return (int)lc[li < nl ? li : nit - 1 - li]; };
-    // Load order: pass 1 takes the live chunks and the copies of the dead ones
-    // in turn (live 0, dead 0, live 1, dead 1, ..., then the rest of the longer
-    // list), so the copies fill the memory system while pass 1 computes; pass 2
-    // (it >= nch) takes the live chunks in reverse.
+    // Load order: pass 1 (the live chunks, ascending), pass 2 (the live chunks,
+    // descending), then the copies of the dead chunks, which stream at the CTA's
+    // end while the last live chunks are computed (measured faster than copies
+    // taken between the pass-1 chunks, which hold ring slots that pass 1 needs).
     const volatile uint8_t *dc = sp + S::DC;
-    const int nmix = min(nl, nch - nl);
-    auto is_live = [&](int it) { return it >= nch || (it < 2 * nmix ? (it & 1) == 0 : 2 * nl > nch); };
-    auto p1_index = [&](int it) { return it < 2 * nmix ? it >> 1 : it - nmix; };
-    auto chunk_of_it = [&](int it) {
-        return it >= nch ? (int)lc[nch - 1 - it + nl] : is_live(it) ? (int)lc[p1_index(it)] : (int)dc[p1_index(it)];
-    };
+    auto is_live = [&](int it) { return it < nit; };
+    auto chunk_of_it = [&](int it) { return it < nl ? (int)lc[it] : it < nit ? (int)lc[nit - 1 - it] : (int)dc[it - nit]; };
 
     if (W == NWARP) {
         // ================= MMA issuer
@@ -319,7 +315,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             auto issue_loads = [&]() {
                 while (next_load < nload && !*fail) {
                     const int it = next_load, x0 = 32 * chunk_of_it(it);
-                    const bool pass2 = it >= nch;
+                    const bool pass2 = it >= nl && it < nit;
                     if (is_live(it)) {
                         const int li = load_li, ns = pass2 ? ns2 : 6;
                         if (li >= done_li + BS_NFULL || __popc(free_mask) < ns) break;
@@ -359,7 +355,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             issue_loads();
             uint32_t pend_mask = 0u;   // slots of the last copy store, not yet known to have read them
             for (int it = 0; it < nload; ++it) {
-                if (it == nch && p.prefetch_ahead) {
+                if (it == nl && p.prefetch_ahead) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = (uint32_t)item + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
@@ -377,7 +373,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 if (is_live(it)) {
                     const int li = done_li++;
                     if (!cta_wait(bar(BB_STAGE_DONE + (li & 3)), (li >> 2) & 1, fail, p.status)) continue;
-                    const bool pass2 = it >= nch;
+                    const bool pass2 = it >= nl && it < nit;
                     if (pass2) {
                         // the chunk's tiles are read by its weight-gradient products until these complete
                         const int p2 = li - nl;

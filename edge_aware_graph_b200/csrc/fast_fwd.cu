@@ -18,8 +18,8 @@
 // chunk with no valid pair (no node among the CTA's rows, or none among the
 // chunk's columns: padding of a smaller graph) has a = 0 everywhere, so E' = E
 // there.  Such a chunk is only copied by the TMA warp (loaded and stored back,
-// bit for bit, while pass 1 runs); the compute and MMA warps never see it.  A
-// CTA whose rows are all padding copies its whole slice.
+// bit for bit); the compute and MMA warps never see it.  A CTA whose rows are
+// all padding copies its whole slice.
 //
 // Warp roles.  Warps 0..15 compute, in two groups of eight that take the
 // chunks in turn (group G = W / 8 takes the iterations it = G, G + 2, ...):
@@ -124,21 +124,24 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 
     // Block sparsity: a chunk holding no valid pair (live_chunk_mask) needs no
     // arithmetic, its E' is its E.  The TMA warp loads iterations it in order:
-    // in pass 1 the nl live chunks, ascending, and the copies of the dead ones
-    // (two E tiles loaded and stored back); in pass 2 the live chunks,
-    // descending (the load order is below).  The live iterations, numbered li = 0 ..
-    // 2 nl - 1 (pass 1, then pass 2's live chunks), are the ones the MMA warp
-    // and the compute groups see: group li & 1 computes li.  Slots: pass 1
-    // E(s=0), E(s=1), K (Light Edge: K alone); pass 2 E(s=0), E(s=1), V when
-    // the pass-1 scores stay in TMEM, else E, E, K, V; a copy E, E.  The
-    // TMA warp takes any free slots and records them in table entry li % 4
-    // (load barrier li % 4), which the other warps read after that barrier.
+    // pass 1 the nl live chunks, ascending; pass 2 the live chunks, descending;
+    // then the copies of the dead ones (two E tiles loaded and stored back).
+    // The live iterations, numbered li = 0 .. 2 nl - 1 (pass 1, then pass 2),
+    // are the ones the MMA warp and the compute groups see: group li & 1
+    // computes li.  Slots: pass 1 E(s=0), E(s=1), K (Light Edge: K alone);
+    // pass 2 E(s=0), E(s=1), V when the pass-1 scores stay in TMEM, else E, E,
+    // K, V; a copy E, E.  The TMA warp takes any free slots and records them
+    // in table entry li % 4 (load barrier li % 4), which the other warps read
+    // after that barrier.
     const bool light = p.light != 0;
     const bool keep_s = nch <= FS_KEEP_S_MAX_CHUNKS;
     const int ns1 = light ? 1 : 3, ks1 = light ? 0 : 2;
     const int ns2 = keep_s ? 3 : 4, vslot = ns2 - 1;
-    volatile uint8_t *stab = sp + S::STAB;
-    auto slot_addr = [&](int li, int k) { return sbase + (uint32_t)stab[(li % FS_NFULL) * 4 + k] * FS_SLOT; };
+    // the slots of live iteration li: one word of the table (slot k in byte k),
+    // written once by the TMA warp and read once after the load barrier
+    volatile uint32_t *stab = reinterpret_cast<volatile uint32_t *>(sp + S::STAB);
+    auto slot_word = [&](int li) { return stab[li % FS_NFULL]; };
+    auto slot_at = [&](uint32_t sw, int k) { return sbase + ((sw >> (8 * k)) & 0xffu) * FS_SLOT; };
 
     // ---------------- setup: barriers, TMEM, operands
     if (tid == 0) {
@@ -184,17 +187,13 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     // chunk of live iteration li; chunk of load iteration it
     const volatile uint8_t *lc = sp + S::LC;
     auto chunk_of_li = [&](int li) { return (int)lc[li < nl ? li : nit - 1 - li]; };
-    // Load order: pass 1 takes the live chunks and the copies of the dead ones
-    // in turn (live 0, dead 0, live 1, dead 1, ..., then the rest of the longer
-    // list), so the copies fill the memory system while pass 1 computes; pass 2
-    // (it >= nch) takes the live chunks in reverse.
+    // Load order: pass 1 (the live chunks, ascending), pass 2 (the live chunks,
+    // descending), then the copies of the dead chunks, which stream at the CTA's
+    // end while the last live chunks are computed (measured faster than copies
+    // taken between the pass-1 chunks, which hold ring slots that pass 1 needs).
     const volatile uint8_t *dc = sp + S::DC;
-    const int nmix = min(nl, nch - nl);
-    auto is_live = [&](int it) { return it >= nch || (it < 2 * nmix ? (it & 1) == 0 : 2 * nl > nch); };
-    auto p1_index = [&](int it) { return it < 2 * nmix ? it >> 1 : it - nmix; };
-    auto chunk_of_it = [&](int it) {
-        return it >= nch ? (int)lc[nch - 1 - it + nl] : is_live(it) ? (int)lc[p1_index(it)] : (int)dc[p1_index(it)];
-    };
+    auto is_live = [&](int it) { return it < nit; };
+    auto chunk_of_it = [&](int it) { return it < nl ? (int)lc[it] : it < nit ? (int)lc[nit - 1 - it] : (int)dc[it - nit]; };
     // the first pass-2 live iteration of group gg
     auto first_p2 = [&](int gg) { return nl + ((gg - nl) & 1); };
 
@@ -204,9 +203,10 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             const uint32_t idesc_f = idesc_bf16_f32(128, NF), idesc_e = idesc_bf16_f32(128, DE);
             auto issue_film = [&](int li) {   // into the TMEM range of group li & 1
                 tc_fence_after();
+                const uint32_t sw = slot_word(li);
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
-                    const uint32_t a0 = slot_addr(li, s);
+                    const uint32_t a0 = slot_at(sw, s);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16_ss(tmem + FS_TM_FILM + 32 * (li & 1) + 16 * s,
@@ -289,23 +289,25 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             auto issue_loads = [&]() {
                 while (next_load < nload && !*fail) {
                     const int it = next_load, j0 = 32 * chunk_of_it(it);
-                    const bool pass2 = it >= nch;
+                    const bool pass2 = it >= nl && it < nit;
                     if (is_live(it)) {
                         const int li = load_li, ns = pass2 ? ns2 : ns1;
                         if (li >= done_li + FS_NFULL || __popc(free_mask) < ns) break;
-                        for (int k = 0; k < ns; ++k) stab[(li % FS_NFULL) * 4 + k] = take_slot();
+                        uint32_t sw = 0;
+                        for (int k = 0; k < ns; ++k) sw |= (uint32_t)take_slot() << (8 * k);
+                        stab[li % FS_NFULL] = sw;
                         const uint32_t fb = bar(FB_FULL + li % FS_NFULL);
                         mbar_expect_tx(fb, ns * FS_SLOT);   // releases the table entry too
                         const uint64_t pol = pass2 ? drop_l2 : keep_l2;
                         if (pass2 || !light) {
-                            tma_load_5d_hint(slot_addr(li, 0), &tmE, fb, 0, i0 / 2, j0, 0, b, pol);
-                            tma_load_5d_hint(slot_addr(li, 1), &tmE, fb, 0, i0 / 2, j0, 1, b, pol);
+                            tma_load_5d_hint(slot_at(sw, 0), &tmE, fb, 0, i0 / 2, j0, 0, b, pol);
+                            tma_load_5d_hint(slot_at(sw, 1), &tmE, fb, 0, i0 / 2, j0, 1, b, pol);
                         }
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            if (!pass2) tma_load_3d(slot_addr(li, ks1) + k * 4096, &tmK, fb, 64 * k, j0, b);
-                            else if (!keep_s) tma_load_3d(slot_addr(li, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
-                            if (pass2) tma_load_3d(slot_addr(li, vslot) + k * 4096, &tmV, fb, 64 * k, j0, b);
+                            if (!pass2) tma_load_3d(slot_at(sw, ks1) + k * 4096, &tmK, fb, 64 * k, j0, b);
+                            else if (!keep_s) tma_load_3d(slot_at(sw, 2) + k * 4096, &tmK, fb, 64 * k, j0, b);
+                            if (pass2) tma_load_3d(slot_at(sw, vslot) + k * 4096, &tmV, fb, 64 * k, j0, b);
                         }
                         if (!pass2 && !light && li + FS_PF < nl)
                             for (int s = 0; s < 2; ++s)
@@ -336,8 +338,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             // stored, and their slots are free once the store has read them
             uint32_t pend_mask = 0u;   // slots of the last store, not yet known to have read them
             for (int it = 0; it < nload; ++it) {
-                const bool pass2 = it >= nch;
-                if (it == nch && p.prefetch_ahead && !light) {
+                const bool pass2 = it >= nl && it < nit;
+                if (it == nl && p.prefetch_ahead && !light) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
@@ -353,9 +355,10 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     const int li = done_li++;
                     if (!cta_wait(bar(FB_STAGE_DONE + (li & 3)), (li >> 2) & 1, fail, p.status)) continue;
                     const int ns = pass2 ? ns2 : ns1;
-                    for (int k = pass2 ? 2 : 0; k < ns; ++k) free_mask |= 1u << stab[(li % FS_NFULL) * 4 + k];
-                    s0 = stab[(li % FS_NFULL) * 4];
-                    s1 = stab[(li % FS_NFULL) * 4 + 1];
+                    const uint32_t sw = slot_word(li);
+                    for (int k = pass2 ? 2 : 0; k < ns; ++k) free_mask |= 1u << ((sw >> (8 * k)) & 0xffu);
+                    s0 = sw & 0xffu;
+                    s1 = (sw >> 8) & 0xffu;
                 } else {
                     const int dk = done_dk++;
                     if (!cta_wait(bar(FB_COPY + dk % FS_NCOPY), (dk / FS_NCOPY) & 1, fail, p.status)) continue;
@@ -400,9 +403,10 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 
         // s' of live iteration li for the thread's 2 pairs x 4 heads: sx[k][e] with
         // k = 2 * pair + hh (heads hqa: k = 0, 1; hqb: k = 2, 3), -inf where invalid
-        auto scores = [&](int li, bool pass2, float (&sx)[4][2], bool (&valid)[2]) {
+        auto scores = [&](int li, bool pass2, float (&sx)[4][2], bool (&valid)[2], uint32_t &sw) {
             const int c = chunk_of_li(li), j0 = 32 * c;
             cta_wait(bar(FB_FULL + li % FS_NFULL), (li / FS_NFULL) & 1, fail, p.status);
+            sw = slot_word(li);
             float sa[2][4], sb[2][4];
             const uint32_t scol = tl + FS_TM_S + 16 * c;
             if (pass2 && keep_s) {
@@ -412,7 +416,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 tmem_ld2(scol + 2 * hqb + 8, sb[0][1], sb[1][1]);
                 tmem_ld_wait();
             } else {
-                const uint32_t ks = slot_addr(li, pass2 ? 2 : ks1);
+                const uint32_t ks = slot_at(sw, pass2 ? 2 : ks1);
                 warp_scores2<1>(ks, q, t, hqa, qfa, sa);
                 warp_scores2<1>(ks, q, t, hqb, qfb, sb);
                 if (keep_s) {
@@ -468,7 +472,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             for (int li = G; li < nl; li += 2) {
                 float sx[4][2];
                 bool valid[2];
-                scores(li, false, sx, valid);
+                uint32_t sw;
+                scores(li, false, sx, valid, sw);
 #pragma unroll
                 for (int e = 0; e < 2; ++e)
 #pragma unroll
@@ -541,7 +546,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         for (int li = first_p2(G); li < nit; li += 2) {
             float sx[4][2];
             bool valid[2];
-            scores(li, true, sx, valid);
+            uint32_t sw;
+            scores(li, true, sx, valid, sw);
             // a (for O) and the edge update's coefficient (a, or s' when unnormalised)
             float pa[2][4], pb[2][4];
 #pragma unroll
@@ -565,7 +571,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             if (t == 0) mbar_arrive(bar(FB_A_FULL + G));
 
             // O += a V on warp MMAs (overlaps the edge MMA)
-            const uint32_t vs = slot_addr(li, vslot);
+            const uint32_t vs = slot_at(sw, vslot);
             warp_contract2<1, true>(vs, q, t, hqa, pa, oa);
             warp_contract2<1, true>(vs, q, t, hqb, pb, ob);
 
@@ -579,7 +585,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     float dv[16];
                     tmem_ld16(tl + FS_TM_EDGE + 128 * G + 64 * e + 32 * hp + 16 * half, dv);
                     tmem_ld_wait();
-                    add_residual16(sp + (slot_addr(li, e) - sbase) + L * 128, L, 2 * hp + half, dv);
+                    add_residual16(sp + (slot_at(sw, e) - sbase) + L * 128, L, 2 * hp + half, dv);
                 }
             }
             fence_proxy_async_smem();
