@@ -49,12 +49,16 @@ UNIT = "edge-pairs/s"
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
-# the dominant kernels on this workload, from the ncu capture summarised in
-# profiles/ (k_bwd_stream_sbm.md, k_fwd_stream_sbm.md).  They describe the
-# kernels as captured; a changed kernel reports null until it is re-captured.
-# k_bwd_stream has changed since its capture (weight-gradient products
-# stacked into M = 128 MMAs): null until it is re-captured.
-NCU_TRAFFIC = {("sbm", "k_fwd_stream"): 258202880}
+# the dominant kernels on each workload, from one ncu capture of the kernels as
+# they are (the summaries under profiles/ give the commands).  A kernel that
+# changes reports null until it is captured again.  Large: the counters come
+# in GB with three digits (1.78 GB read by k_bwd_stream).
+NCU_TRAFFIC = {
+    ("sbm", "k_fwd_stream"): 158565888 + 98265856,
+    ("sbm", "k_bwd_stream"): 254333696 + 115731712,
+    ("large", "k_fwd_stream"): 807830000 + 482330000,
+    ("large", "k_bwd_stream"): 1780000000 + 504840000,
+}
 
 
 def env_rank():
