@@ -6,10 +6,11 @@
 // need two passes", AI-summary page, method paragraph):
 //   pass 1: FiLM coefficients f = E Wfe on the tensor cores (tcgen05, fp32 in
 //           TMEM), scores S = Q K^T with warp MMAs, s' = S(1+gamma)+beta,
-//           running masked row max / sum per thread (online softmax);
-//   pass 2: the same f and s' again, normalised a, O += a V (warp MMAs), edge
-//           update dE = a We on the tensor cores, E' = E + dE written in place
-//           and stored with TMA.
+//           running masked row max / sum per thread (online softmax); s' is
+//           kept in TMEM (16 columns per chunk, n <= 384);
+//   pass 2: s' from TMEM (larger graphs compute f and S again), normalised a,
+//           O += a V (warp MMAs), edge update dE = a We on the tensor cores,
+//           E' = E + dE written in place and stored with TMA.
 // Pass 2 walks the chunks in reverse, so the E tiles it reads again are the
 // ones pass 1 brought into L2 last: E leaves HBM once, E' is written once and
 // the [B,H,n,n] map never leaves the chip.  No CTA waits for another one.
@@ -83,7 +84,8 @@ constexpr int FB_FULL = 0, FB_FILM_FULL = 4, FB_FILM_EMPTY = 6, FB_A_FULL = 8, F
 constexpr int FS_NCOPY = 4;               // dead-chunk copies in flight
 
 // TMEM columns: FiLM 0..63 (two buffers), edge update 64..319 (two buffers),
-// pass-1 scores from 320 on (16 per chunk, kept when nch <= 12 so pass 2 needs no K)
+// pass-1 modulated scores s' from 320 on (16 per chunk, kept when nch <= 12, so
+// that pass 2 needs neither K nor the FiLM product)
 constexpr uint32_t FS_TM_COLS = 512;
 constexpr uint32_t FS_TM_FILM = 0, FS_TM_EDGE = 64, FS_TM_S = 320;
 constexpr int FS_KEEP_S_MAX_CHUNKS = (512 - 320) / 16;
@@ -103,7 +105,10 @@ struct FwdParams {
 };
 
 // 576 threads (18 warps): five warps share one of the four 16K-register sub-partitions,
-// so at most 96 registers a thread
+// so at most 96 registers a thread.  KEEP_S: s' stays in tensor memory between
+// the passes (nch <= 12); the instance without it holds the Q fragments through
+// pass 2, the one with it frees them after pass 1.
+template <bool KEEP_S>
 __global__ void __launch_bounds__(FS_THR, 1)
 k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmEo,
              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, FwdParams p) {
@@ -134,7 +139,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     // in table entry li % 4 (load barrier li % 4), which the other warps read
     // after that barrier.
     const bool light = p.light != 0;
-    const bool keep_s = nch <= FS_KEEP_S_MAX_CHUNKS;
+    constexpr bool keep_s = KEEP_S;
     const int ns1 = light ? 1 : 3, ks1 = light ? 0 : 2;
     const int ns2 = keep_s ? 3 : 4, vslot = ns2 - 1;
     // the slots of live iteration li: one word of the table (slot k in byte k),
@@ -227,12 +232,15 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             // issue whichever product is ready: FiLM of the next chunk (its tiles
             // landed, its group's TMEM range released) or the edge update of a
             // group whose a the compute warps have written
-            int next_film = light ? nit : 0;                 // Light Edge: no FiLM products
+            // FiLM products: every live iteration, or pass 1 only when s' stays in
+            // tensor memory; none for Light Edge
+            const int nfilm = light ? 0 : keep_s ? nl : nit;
+            int next_film = 0;
             int next_edge[2] = {first_p2(0), first_p2(1)};
             uint32_t polls = 0;
-            while ((next_film < nit || next_edge[0] < nit || next_edge[1] < nit) && !*fail) {
+            while ((next_film < nfilm || next_edge[0] < nit || next_edge[1] < nit) && !*fail) {
                 bool progressed = false;
-                if (next_film < nit &&
+                if (next_film < nfilm &&
                     mbar_test_wait(bar(FB_FULL + next_film % FS_NFULL), (next_film / FS_NFULL) & 1) &&
                     (next_film < 2 ||
                      mbar_test_wait(bar(FB_FILM_EMPTY + (next_film & 1)), ((next_film - 2) >> 1) & 1))) {
@@ -242,7 +250,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 #pragma unroll
                 for (int gg = 0; gg < 2; ++gg) {
                     const int li = next_edge[gg];
-                    if (li < nit && li < next_film &&
+                    if (li < nit && (li < next_film || next_film == nfilm) &&
                         mbar_test_wait(bar(FB_A_FULL + gg), ((li - nl) >> 1) & 1)) {
                         issue_edge(gg);
                         next_edge[gg] += 2;
@@ -407,25 +415,24 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             const int c = chunk_of_li(li), j0 = 32 * c;
             cta_wait(bar(FB_FULL + li % FS_NFULL), (li / FS_NFULL) & 1, fail, p.status);
             sw = slot_word(li);
-            float sa[2][4], sb[2][4];
             const uint32_t scol = tl + FS_TM_S + 16 * c;
+            const bool mcol = mj[j0 + 8 * q + g8] != 0;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) valid[e] = mcol && mrow[e];
             if (pass2 && keep_s) {
-                tmem_ld2(scol + 2 * hqa, sa[0][0], sa[1][0]);
-                tmem_ld2(scol + 2 * hqa + 8, sa[0][1], sa[1][1]);
-                tmem_ld2(scol + 2 * hqb, sb[0][0], sb[1][0]);
-                tmem_ld2(scol + 2 * hqb + 8, sb[0][1], sb[1][1]);
+                // s' as pass 1 left it in tensor memory (-inf where invalid):
+                // no K, no FiLM product in pass 2
+                tmem_ld2(scol + 2 * hqa, sx[0][0], sx[1][0]);
+                tmem_ld2(scol + 2 * hqa + 8, sx[0][1], sx[1][1]);
+                tmem_ld2(scol + 2 * hqb, sx[2][0], sx[3][0]);
+                tmem_ld2(scol + 2 * hqb + 8, sx[2][1], sx[3][1]);
                 tmem_ld_wait();
-            } else {
-                const uint32_t ks = slot_at(sw, pass2 ? 2 : ks1);
-                warp_scores2<1>(ks, q, t, hqa, qfa, sa);
-                warp_scores2<1>(ks, q, t, hqb, qfb, sb);
-                if (keep_s) {
-                    tmem_st2(scol + 2 * hqa, sa[0][0], sa[1][0]);
-                    tmem_st2(scol + 2 * hqa + 8, sa[0][1], sa[1][1]);
-                    tmem_st2(scol + 2 * hqb, sb[0][0], sb[1][0]);
-                    tmem_st2(scol + 2 * hqb + 8, sb[0][1], sb[1][1]);
-                }
+                return;
             }
+            float sa[2][4], sb[2][4];
+            const uint32_t ks = slot_at(sw, pass2 ? 2 : ks1);
+            warp_scores2<1>(ks, q, t, hqa, qfa, sa);
+            warp_scores2<1>(ks, q, t, hqb, qfb, sb);
             // FiLM of the pair: gamma, beta of the four heads
             float gm[2][4] = {}, bt[2][4] = {};
             if (!light) {
@@ -444,10 +451,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 __syncwarp();
                 if (t == 0) mbar_arrive(bar(FB_FILM_EMPTY + (li & 1)));
             }
-            const bool mcol = mj[j0 + 8 * q + g8] != 0;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                valid[e] = mcol && mrow[e];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int h = 4 * hp + k;
@@ -455,6 +460,12 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     const float sv = raw * rs * (1.f + gm[e][k] + g[h]) + bt[e][k] + g[NH + h];
                     sx[k][e] = valid[e] ? sv : -INFINITY;
                 }
+            }
+            if (keep_s) {   // pass 1: s' for pass 2
+                tmem_st2(scol + 2 * hqa, sx[0][0], sx[1][0]);
+                tmem_st2(scol + 2 * hqa + 8, sx[0][1], sx[1][1]);
+                tmem_st2(scol + 2 * hqb, sx[2][0], sx[3][0]);
+                tmem_st2(scol + 2 * hqb + 8, sx[2][1], sx[3][1]);
             }
         };
 
@@ -488,8 +499,11 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 __syncwarp();
                 if (t == 0) mbar_arrive(bar(FB_STAGE_DONE + (li & 3)));
             }
-            // ---------------- end of pass 1: statistics over lanes, then (group, quadrant)
+            // ---------------- end of pass 1: statistics over lanes, then (group, quadrant);
+            // the kept s' (read in pass 2 by whichever group takes the chunk) is
+            // complete before the barrier
             tmem_st_wait();
+            tc_fence_before();
             float *wst = reinterpret_cast<float *>(sp + S::WST);
             float *fin = reinterpret_cast<float *>(sp + S::FIN);
 #pragma unroll
@@ -512,6 +526,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     }
                 }
             named_bar_sync(1, NTHR);
+            tc_fence_after();
             if (tid < 64) {
                 float m = -INFINITY;
 #pragma unroll
@@ -621,8 +636,12 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
 
 cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
                              cudaStream_t st) {
-    static std::atomic<uint32_t> attr_set{0};
-    if (cudaError_t e = ensure_smem_attr(k_fwd_stream, FsSmem::BYTES, attr_set); e != cudaSuccess) return e;
+    const bool keep_s = (d.n + 31) / 32 <= FS_KEEP_S_MAX_CHUNKS;
+    static std::atomic<uint32_t> attr_set[2] = {{0}, {0}};
+    if (cudaError_t e = ensure_smem_attr(keep_s ? k_fwd_stream<true> : k_fwd_stream<false>, FsSmem::BYTES,
+                                         attr_set[keep_s]);
+        e != cudaSuccess)
+        return e;
     CUtensorMap mE, mEo, mK, mV;
     if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mEo, a.Eout, d.B, d.n, false, 32, 1) ||
         !encode_node_map(&mK, a.K, d.B, d.n, 32) || !encode_node_map(&mV, a.V, d.B, d.n, 32))
@@ -639,7 +658,11 @@ cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t
     p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
     p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)sm_count();
-    k_fwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), FS_THR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
+    const dim3 grid((d.n + TB - 1) / TB, d.B);
+    if (keep_s)
+        k_fwd_stream<true><<<grid, FS_THR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
+    else
+        k_fwd_stream<false><<<grid, FS_THR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
     return cudaGetLastError();
 }
 
