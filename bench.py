@@ -54,7 +54,9 @@ FALLBACK_HBM_GBS = 6650.0
 # changes reports null until it is captured again.  Large: the counters come
 # in GB with three digits (1.78 GB read by k_bwd_stream).
 NCU_TRAFFIC = {
+    ("sbm", "k_fwd_stream"): 158670000 + 96130000,
     ("sbm", "k_bwd_stream"): 254333696 + 115731712,
+    ("large", "k_fwd_stream"): 809080000 + 481850000,
     ("large", "k_bwd_stream"): 1780000000 + 504840000,
 }
 
