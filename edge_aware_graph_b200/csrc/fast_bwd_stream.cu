@@ -407,6 +407,17 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         }
         __syncwarp();
         named_bar_sync(2, BS_THR);   // the ring is drained: the compute warps may reuse it
+    } else if (nl == 0) {
+        // ================= compute warps of a row block without a valid pair: dq of
+        // its rows and its weight-gradient partials are zero, no passes
+        for (int x = tid; x < TB * HD / 8; x += NTHR) {
+            const int il = x / (HD / 8), d = (x % (HD / 8)) * 8;
+            if (i0 + il < n)
+                *reinterpret_cast<uint4 *>(p.dQ + ((size_t)b * n + i0 + il) * HD + d) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        float *rp = p.rparts + (size_t)item * RPART;
+        for (int x = tid; x < RPART; x += NTHR) rp[x] = 0.f;
+        named_bar_sync(2, BS_THR);   // the TMA warp has stored the copies
     } else {
         // ================= compute warps
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);

@@ -396,6 +396,19 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
         }
         __syncwarp();
         named_bar_sync(2, FS_THR);   // the ring is drained: the compute warps may reuse it
+    } else if (nl == 0) {
+        // ================= compute warps of a row block without a valid pair: its
+        // rows get LSE = -inf and O = 0 (what the passes would give), no passes
+        for (int x = tid; x < TB * NH; x += NTHR) {
+            const int il = x >> 3, h = x & 7;
+            if (i0 + il < n) p.LSE[((size_t)b * NH + h) * n + i0 + il] = -INFINITY;
+        }
+        for (int x = tid; x < TB * HD / 8; x += NTHR) {
+            const int il = x / (HD / 8), d = (x % (HD / 8)) * 8;
+            if (i0 + il < n)
+                *reinterpret_cast<uint4 *>(p.O + ((size_t)b * n + i0 + il) * HD + d) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        named_bar_sync(2, FS_THR);   // the TMA warp has stored the copies
     } else {
         // ================= compute warps: group G, quadrant q, heads 4hp..4hp+3
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
