@@ -20,8 +20,7 @@ cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs 
                              cudaStream_t st);
 cudaError_t launch_kv_convert(const eaga_dims &d, const FastWs &W, char *ws, cudaStream_t st);
 cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
-cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
-                             cudaStream_t st);
+cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
 
 bool supports(const eaga_dims &d) {
     return d.dtype == EAGA_BF16 && d.de == DE && d.H == NH && d.dh == DH && d.n % 2 == 0 && d.n >= 2 &&
@@ -49,32 +48,10 @@ int kernel_launches(const eaga_dims &, int for_backward) {
         if (e_ != cudaSuccess) return e_;         \
     } while (0)
 
-cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st) {
-    uint8_t *img = reinterpret_cast<uint8_t *>(ws_after_common);
-    const int rows = d.B * d.n;
-    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, st));
-    {   // [Q|K|V] = X [Wq|Wk|Wv] + b
-        const void *A[3] = {a.X, a.X, a.X}, *B[3] = {a.w[0], a.w[2], a.w[4]};
-        const void *bias[3] = {a.w[1], a.w[3], a.w[5]};
-        void *C[3] = {a.Q, a.K, a.V};
-        FAST_TRY(tc_gemm(0, rows, 3 * HD, d.dx, 1, A, B, bias, C, HD, nullptr, a.M, a.status, st, true));
-    }
-    prof_mark(0, 0, st);
-    FAST_TRY(launch_fwd_pairs(d, a, img, a.g, st));
-    prof_mark(0, 1, st);
-    {   // X' = X + M (O Wo + bo)
-        const void *A[3] = {a.O, a.O, a.O}, *B[3] = {a.w[10], a.w[10], a.w[10]};
-        const void *bias[3] = {a.w[11], a.w[11], a.w[11]};
-        void *C[3] = {a.Xout, a.Xout, a.Xout};
-        FAST_TRY(tc_gemm(1, rows, d.dx, HD, 1, A, B, bias, C, d.dx, a.X, a.M, a.status, st, true));
-    }
-    return cudaSuccess;
-}
-
 // Two auxiliary streams and a pool of events per device, created on first
-// use: the backward runs independent kernels side by side (fork / join on
-// events), which a CUDA graph captured around the call keeps as parallel
-// branches.  The lock is held while a call enqueues, so concurrent calls on
+// use: the forward and the backward run independent kernels side by side
+// (fork / join on events), which a CUDA graph captured around the call keeps
+// as parallel branches.  The lock is held while a call enqueues, so concurrent calls on
 // one device never share an event between a record and its wait.
 namespace {
 constexpr int kMaxDevices = 64, kEvents = 6;
@@ -112,6 +89,35 @@ cudaError_t stream_after(cudaStream_t to, cudaStream_t from, cudaEvent_t ev) {
     return e == cudaSuccess ? cudaStreamWaitEvent(to, ev, 0) : e;
 }
 }  // namespace
+
+cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st) {
+    uint8_t *img = reinterpret_cast<uint8_t *>(ws_after_common);
+    const int rows = d.B * d.n;
+    DeviceAux *aux = nullptr;
+    FAST_TRY(device_aux(&aux));
+    std::lock_guard<std::mutex> lock(aux->mu);
+    FAST_TRY(aux_init(*aux));
+    // the prologue (g, operand images) beside the QKV projection
+    FAST_TRY(stream_after(aux->s[0], st, aux->ev[0]));
+    FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, aux->s[0]));
+    {   // [Q|K|V] = X [Wq|Wk|Wv] + b
+        const void *A[3] = {a.X, a.X, a.X}, *B[3] = {a.w[0], a.w[2], a.w[4]};
+        const void *bias[3] = {a.w[1], a.w[3], a.w[5]};
+        void *C[3] = {a.Q, a.K, a.V};
+        FAST_TRY(tc_gemm(0, rows, 3 * HD, d.dx, 1, A, B, bias, C, HD, nullptr, a.M, a.status, st, true));
+    }
+    FAST_TRY(stream_after(st, aux->s[0], aux->ev[1]));
+    prof_mark(0, 0, st);
+    FAST_TRY(launch_fwd_pairs(d, a, img, a.g, st));
+    prof_mark(0, 1, st);
+    {   // X' = X + M (O Wo + bo)
+        const void *A[3] = {a.O, a.O, a.O}, *B[3] = {a.w[10], a.w[10], a.w[10]};
+        const void *bias[3] = {a.w[11], a.w[11], a.w[11]};
+        void *C[3] = {a.Xout, a.Xout, a.Xout};
+        FAST_TRY(tc_gemm(1, rows, d.dx, HD, 1, A, B, bias, C, d.dx, a.X, a.M, a.status, st, true));
+    }
+    return cudaSuccess;
+}
 
 cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head, cudaStream_t st) {
     const FastWs W = fast_ws(d, head);
@@ -161,10 +167,10 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         FAST_TRY(tc_wgrad(d.dx, HD, 3, rows, W.wsplits, a.X, Bq, Pq, a.status, s1));
         FAST_TRY(tc_wgrad(HD, d.dx, 1, rows, W.wsplits, a.O, Bo, Po, a.status, s1));
     }
-    FAST_TRY(launch_bwd_partials(d, a, W, ws, s2));
+    FAST_TRY(launch_bwd_partials(d, a, W, ws, s2));   // bias and row-block partials, dg, dbf, dWfy, dy
     FAST_TRY(stream_after(st, s1, ev[4]));
     FAST_TRY(stream_after(st, s2, ev[5]));
-    return launch_bwd_final(d, a, W, ws, reinterpret_cast<float *>(ws + W.dg), st);
+    return launch_bwd_final(d, a, W, ws, st);
 }
 
 }  // namespace fast

@@ -74,10 +74,20 @@ __device__ __forceinline__ float strided_sum(const float *src, int count, size_t
     return (a0 + a1) + (a2 + a3);
 }
 
-// Row-kernel partials: out[z][e] = sum over CTAs of segment z of rparts[cta][e], e < dWfe+dWe.
-__global__ void k_rparts_partial(const float *rparts, int ctas, int seg, float *out) {
+// Row-kernel partials: out[z][e] = sum over CTAs of segment z of rparts[cta][e], e < dWfe+dWe
+// (blockIdx.y = z < gridDim.y - 1); the last row of blocks sums each graph's
+// dg_b = sum over its row blocks of their dg partials.
+__global__ void k_rparts_partial(const float *rparts, int ctas, int seg, float *out, float *dg, int B,
+                                 int ctas_per_graph) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     constexpr int NE = DE * NF + NH * DE;
+    if (blockIdx.y + 1 == gridDim.y) {
+        if (e < B * NF) {
+            const int b = e / NF, k = e % NF;
+            dg[e] = strided_sum(rparts + (size_t)b * ctas_per_graph * RPART + NE + k, ctas_per_graph, RPART);
+        }
+        return;
+    }
     if (e >= NE) return;
     const int c0 = blockIdx.y * seg, c1 = min(ctas, c0 + seg);
     out[(size_t)blockIdx.y * NE + e] = c1 > c0 ? strided_sum(rparts + (size_t)c0 * RPART + e, c1 - c0, RPART) : 0.f;
@@ -88,12 +98,9 @@ struct DWPtrs {
 };
 
 // Final sums: weight gradients of the four node projections (split-K
-// partials), bias gradients, dWfe / dWe, and the global FiLM term's dg_b,
-// dWfy, dbf, dy.
+// partials), bias gradients, dWfe / dWe.
 __global__ void k_bwd_finish(const float *wparts, int wsplits, const float *bparts, int bsplits,
-                             const float *r2, int rsplits, const float *rparts, int ctas_per_graph, int B, int dx,
-                             int dy, const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy, DWPtrs dW,
-                             __nv_bfloat16 *dyo, float *dg, int zero_wfe) {
+                             const float *r2, int rsplits, int dx, DWPtrs dW, int zero_wfe) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const int msz = dx * HD;
     const int ncol = 3 * HD + dx;
@@ -116,16 +123,10 @@ __global__ void k_bwd_finish(const float *wparts, int wsplits, const float *bpar
         const float acc = strided_sum(r2 + x, rsplits, NE);
         // (Light Edge: Wfe is not a parameter, its gradient is zero)
         if (x < DE * NF) dW.p[6][x] = zero_wfe ? 0.f : acc; else dW.p[9][x - DE * NF] = acc;
-        return;
-    }
-    x -= NE;
-    if (x < B * NF) {
-        const int b = x / NF, k = x % NF;
-        dg[x] = strided_sum(rparts + (size_t)b * ctas_per_graph * RPART + NE + k, ctas_per_graph, RPART);
     }
 }
 
-// dbf, dWfy, dy from dg (after k_bwd_finish).
+// dbf, dWfy, dy from dg (after k_rparts_partial).
 __global__ void k_film_grads(const float *dg, int B, int dy, const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy,
                              float *dbf, float *dWfy, __nv_bfloat16 *dyo) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -199,32 +200,32 @@ cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const Fast
     k_bias_partial<<<dim3(3 + (d.dx + 255) / 256, W.bsplits), 256, 0, st>>>(
         dQ, dK, dV, static_cast<const __nv_bfloat16 *>(a.dXout), a.M, rows, d.dx, seg_rows, bparts);
     float *r2 = reinterpret_cast<float *>(ws + W.r2);
+    float *dg = reinterpret_cast<float *>(ws + W.dg);
     const int ctas = W.n_rparts, seg = (ctas + W.rsplits - 1) / W.rsplits;
     constexpr int NE = DE * NF + NH * DE;
     const float *rparts = reinterpret_cast<const float *>(ws + W.rparts);
-    k_rparts_partial<<<dim3((NE + 255) / 256, W.rsplits), 256, 0, st>>>(rparts, ctas, seg, r2);
-    return cudaGetLastError();
-}
-
-// Final sums of every weight gradient and the global FiLM term's gradients.
-cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, float *dg,
-                             cudaStream_t st) {
-    const int ncol = 3 * HD + d.dx;
-    constexpr int NE = DE * NF + NH * DE;
-    DWPtrs dWdev;
-    for (int q = 0; q < 12; ++q) dWdev.p[q] = a.dW[q];
-    const int total = 4 * d.dx * HD + ncol + NE + d.B * NF;
-    const int cpg = (d.n + TB - 1) / TB;
-    k_bwd_finish<<<(total + 255) / 256, 256, 0, st>>>(
-        reinterpret_cast<const float *>(ws + W.wparts), W.wsplits, reinterpret_cast<const float *>(ws + W.bparts),
-        W.bsplits, reinterpret_cast<const float *>(ws + W.r2), W.rsplits,
-        reinterpret_cast<const float *>(ws + W.rparts), cpg, d.B, d.dx, d.dy,
-        static_cast<const __nv_bfloat16 *>(a.y), static_cast<const __nv_bfloat16 *>(a.w[7]), dWdev,
-        static_cast<__nv_bfloat16 *>(a.dy), dg, a.variant == EAGA_VARIANT_LIGHT_EDGE);
+    const int xblocks = (std::max(NE, d.B * NF) + 255) / 256;
+    k_rparts_partial<<<dim3(xblocks, W.rsplits + 1), 256, 0, st>>>(rparts, ctas, seg, r2, dg, d.B,
+                                                                   (d.n + TB - 1) / TB);
+    // dbf, dWfy, dy from dg (on the same stream, off the path of dX and dW)
     const int tf = NF + d.dy * NF + d.B * d.dy;
     k_film_grads<<<(tf + 255) / 256, 256, 0, st>>>(dg, d.B, d.dy, static_cast<const __nv_bfloat16 *>(a.y),
                                                    static_cast<const __nv_bfloat16 *>(a.w[7]), a.dW[8], a.dW[7],
                                                    static_cast<__nv_bfloat16 *>(a.dy));
+    return cudaGetLastError();
+}
+
+// Final sums of the node projections' weight and bias gradients and of dWfe, dWe.
+cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st) {
+    const int ncol = 3 * HD + d.dx;
+    constexpr int NE = DE * NF + NH * DE;
+    DWPtrs dWdev;
+    for (int q = 0; q < 12; ++q) dWdev.p[q] = a.dW[q];
+    const int total = 4 * d.dx * HD + ncol + NE;
+    k_bwd_finish<<<(total + 255) / 256, 256, 0, st>>>(
+        reinterpret_cast<const float *>(ws + W.wparts), W.wsplits, reinterpret_cast<const float *>(ws + W.bparts),
+        W.bsplits, reinterpret_cast<const float *>(ws + W.r2), W.rsplits, d.dx, dWdev,
+        a.variant == EAGA_VARIANT_LIGHT_EDGE);
     return cudaGetLastError();
 }
 

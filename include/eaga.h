@@ -43,9 +43,9 @@
  *     are recorded in the workspace status word and read by
  *     eaga_get_device_status.
  *   - No global state besides per-device cached kernel attributes, the
- *     backward's per-device auxiliary streams and the optional profiling
- *     events; calls on distinct streams with distinct workspaces are
- *     thread-safe, also across devices of one process.
+ *     per-device auxiliary streams of the specialised path and the optional
+ *     profiling events; calls on distinct streams with distinct workspaces
+ *     are thread-safe, also across devices of one process.
  */
 #ifndef EAGA_H
 #define EAGA_H
@@ -107,7 +107,10 @@ EAGA_API size_t eaga_saved_size(const eaga_dims *dims);
 /* Forward of the layer (the formulas above).  Writes Xout and Eout.  `saved`
  * (nullable; eaga_saved_size bytes) receives the state eaga_backward needs;
  * with saved == NULL that state lives in the workspace and is discarded.
- * `workspace` must hold eaga_workspace_size(dims, 0) bytes. */
+ * `workspace` must hold eaga_workspace_size(dims, 0) bytes.  On the
+ * specialised bf16 path the small prologue kernel runs beside the Q/K/V
+ * projection on one of the library's per-device streams, ordered on `stream`
+ * like the backward's (below). */
 EAGA_API eaga_status eaga_forward(const eaga_dims *dims,
                          const void *X, const void *E, const void *y, const uint8_t *M,
                          const eaga_weights *w,
