@@ -102,6 +102,11 @@ CASES = [
     # ones (copied, not computed), with S, dP kept and reloaded
     (4, 160, 256, 64, 64, 8, 32, "bf16", "blocks"),
     (4, 250, 256, 64, 64, 8, 32, "bf16", "blocks"),
+    # a row block's columns over a cluster of CTAs (more than 8 chunks): 2 CTAs
+    # of 5 and 4 chunks; 4 CTAs of 5, 5, 5 and 2 chunks; 4 CTAs of 8 chunks
+    (2, 288, 256, 64, 64, 8, 32, "bf16", "blocks"),
+    (2, 544, 256, 64, 64, 8, 32, "bf16", "random"),
+    (1, 1024, 256, 64, 64, 8, 32, "bf16", "prefix"),
 ]
 
 

@@ -28,6 +28,7 @@ CASES = [
     (4, 30, 256, 64, 64, 8, 32, "bf16", "random"),      # tcgen05 path, one partial chunk
     (2, 250, 256, 64, 64, 8, 32, "bf16", "prefix"),     # tcgen05 path, S and dP reloaded
     (4, 160, 256, 64, 64, 8, 32, "bf16", "blocks"),     # tcgen05 path, chunks without a valid pair
+    (2, 288, 256, 64, 64, 8, 32, "bf16", "blocks"),     # tcgen05 path, a row block over 2 CTAs
     (3, 37, 24, 24, 16, 3, 16, "fp32", "random"),       # CUDA-core path, fp32
     (2, 70, 64, 32, 8, 4, 16, "bf16", "prefix"),        # CUDA-core path, bf16
 ]
