@@ -56,7 +56,7 @@ constexpr int FS_THR = FS_CTHR + 64;      // + the MMA warp and the TMA warp
 constexpr int FS_SLOTS = 6;               // 16 KB slots of the load ring
 constexpr uint32_t FS_SLOT = 16384;
 constexpr int FS_NFULL = 4;               // load barriers of live iterations
-constexpr int FS_NCOPY = 2;               // dead-chunk copies in flight
+constexpr int FS_NCOPY = 3;               // dead-chunk copies in flight
 constexpr int FS_PF = 4;                  // pass-1 chunks prefetched into L2 beyond the loads
 constexpr int FS_MAX_CPC = 8;             // chunks per CTA (their s' fills the upper half of TMEM)
 constexpr int FS_MAX_CS = 4;              // CTAs per row block
@@ -71,10 +71,10 @@ struct FsSmem {
     static constexpr uint32_t XST = FIN + 512;                // the cluster's partial statistics [4 ranks][64][2]
     static constexpr uint32_t G = XST + 2048;                 // g_b [16]
     static constexpr uint32_t BAR = G + 64;                   // mbarriers, see below
-    static constexpr uint32_t TM = BAR + 8 * 18;              // TMEM base address
+    static constexpr uint32_t TM = BAR + 8 * 19;              // TMEM base address
     static constexpr uint32_t FAIL = TM + 8;                  // CTA failure flag (a wait ran out)
     static constexpr uint32_t STAB = TM + 16;                 // slot table [4 live iterations] u32
-    static constexpr uint32_t CTAB = STAB + 16;               // slots of the copies [2][2] u8
+    static constexpr uint32_t CTAB = STAB + 16;               // slots of the copies [3][2] u8
     static constexpr uint32_t LIVE = CTAB + 8;                // live-chunk mask of the CTA's chunks
     static constexpr uint32_t LC = LIVE + 8;                  // the live chunks, ascending [8] u8 (+ slack)
     static constexpr uint32_t DC = LC + 32;                   // the dead chunks, ascending [8] u8 (+ slack)
@@ -84,10 +84,10 @@ struct FsSmem {
 };
 static_assert(FsSmem::BYTES <= 115712, "two CTAs per SM");
 // mbarriers: full[4] (loads of live iterations), film_full[2], film_empty[2], a_full,
-// edge_full, stage_done[4], mma_final, copy[2] (loads of dead chunks), stats (the
+// edge_full, stage_done[4], mma_final, copy[3] (loads of dead chunks), stats (the
 // cluster's partial row statistics have arrived)
 constexpr int FB_FULL = 0, FB_FILM_FULL = 4, FB_FILM_EMPTY = 6, FB_A_FULL = 8, FB_EDGE_FULL = 9,
-              FB_STAGE_DONE = 10, FB_MMA_FINAL = 14, FB_COPY = 15, FB_STATS = 17;
+              FB_STAGE_DONE = 10, FB_MMA_FINAL = 14, FB_COPY = 15, FB_STATS = 18;
 
 // TMEM columns: FiLM 0..63 (two buffers, pass 1), edge update 0..127 (pass 2),
 // s' of the CTA's chunks 128..255 (16 per chunk)
