@@ -72,22 +72,39 @@ static bool known_variant(int v) {
     return v == EAGA_VARIANT_LAYER || v == EAGA_VARIANT_LIGHT_EDGE || v == EAGA_VARIANT_UNNORMALISED;
 }
 
-eaga_status eaga_forward_variant(const eaga_dims *d, int variant, const void *X, const void *E, const void *y,
-                                 const uint8_t *M, const eaga_weights *w, void *Xout, void *Eout, void *saved,
-                                 void *workspace, size_t ws_bytes, void *stream) {
+// A slab of each graph's rows, row0 .. row0+rows-1 (rows < 0: the whole graph):
+// the specialised path only; row0 and rows whole row blocks of 8 (the last
+// slab may end at n).  Returns EAGA_OK or the reason it is refused.
+static eaga_status check_slab(const eaga_dims &d, int row0, int rows) {
+    if (rows < 0) return EAGA_OK;
+    if (row0 < 0 || rows < 2 || (rows & 1) || row0 + rows > d.n || (row0 % 8) || ((rows % 8) && row0 + rows != d.n))
+        return EAGA_ERR_INVALID_ARG;
+    return fast::supports(d) ? EAGA_OK : EAGA_ERR_UNSUPPORTED;
+}
+// Bytes of an E-sized tensor of the slab.
+static size_t slab_bytes(const eaga_dims &d, int rows) {
+    const Extents x = tensor_extents(d);
+    return rows < 0 ? x.E : x.E / d.n * rows;
+}
+
+static eaga_status forward_impl(const eaga_dims *d, int variant, int row0, int rows, const void *X, const void *E,
+                                const void *y, const uint8_t *M, const eaga_weights *w, void *Xout, void *Eout,
+                                void *saved, void *workspace, size_t ws_bytes, void *stream) {
     NvtxRange range("eaga_forward");
     eaga_status s = check_dims(d);
     if (s != EAGA_OK) return s;
     if (!known_variant(variant)) return EAGA_ERR_INVALID_ARG;
+    if ((s = check_slab(*d, row0, rows)) != EAGA_OK) return s;
     if ((s = check_weights(w)) != EAGA_OK) return s;
     if ((s = check_ptrs({X, E, y, M, Xout, Eout, workspace})) != EAGA_OK) return s;
     if (saved && !aligned16(saved)) return EAGA_ERR_MISALIGNED;
     const Layout L = saved_layout(*d);
     {
         const Extents x = tensor_extents(*d);
-        const Span outs[4] = {{Xout, x.X}, {Eout, x.E}, {saved, saved ? L.saved_total : 0},
+        const size_t xe = slab_bytes(*d, rows);
+        const Span outs[4] = {{Xout, x.X}, {Eout, xe}, {saved, saved ? L.saved_total : 0},
                               {workspace, eaga_workspace_size(d, 0)}};
-        Span ins[16] = {{X, x.X}, {E, x.E}, {y, x.y}, {M, x.M}};
+        Span ins[16] = {{X, x.X}, {E, xe}, {y, x.y}, {M, x.M}};
         const void *wsrc[12];
         weight_array(w, wsrc);
         weight_spans(wsrc, x.w, ins, 4);
@@ -100,6 +117,8 @@ eaga_status eaga_forward_variant(const eaga_dims *d, int variant, const void *X,
     char *sv = saved ? static_cast<char *>(saved) : ws + W.fwd_saved;
     FwdArgs a;
     a.variant = variant;
+    a.row0 = rows < 0 ? 0 : row0;
+    a.rows = rows;
     a.X = X; a.E = E; a.y = y; a.M = M;
     weight_array(w, a.w);
     a.Xout = Xout; a.Eout = Eout;
@@ -114,6 +133,20 @@ eaga_status eaga_forward_variant(const eaga_dims *d, int variant, const void *X,
     return launch_status(generic::forward(*d, a, st));
 }
 
+eaga_status eaga_forward_variant(const eaga_dims *d, int variant, const void *X, const void *E, const void *y,
+                                 const uint8_t *M, const eaga_weights *w, void *Xout, void *Eout, void *saved,
+                                 void *workspace, size_t ws_bytes, void *stream) {
+    return forward_impl(d, variant, 0, -1, X, E, y, M, w, Xout, Eout, saved, workspace, ws_bytes, stream);
+}
+
+eaga_status eaga_forward_rows(const eaga_dims *d, int variant, int row0, int rows, const void *X, const void *E_rows,
+                              const void *y, const uint8_t *M, const eaga_weights *w, void *Xout, void *Eout_rows,
+                              void *saved, void *workspace, size_t ws_bytes, void *stream) {
+    if (rows < 0) return EAGA_ERR_INVALID_ARG;
+    return forward_impl(d, variant, row0, rows, X, E_rows, y, M, w, Xout, Eout_rows, saved, workspace, ws_bytes,
+                        stream);
+}
+
 eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
                          const eaga_weights *w, void *Xout, void *Eout, void *saved, void *workspace,
                          size_t ws_bytes, void *stream) {
@@ -121,14 +154,15 @@ eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const
                                 stream);
 }
 
-eaga_status eaga_backward_variant(const eaga_dims *d, int variant, const void *X, const void *E, const void *y,
-                                  const uint8_t *M, const eaga_weights *w, const void *saved, const void *dXout,
-                                  const void *dEout, void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
-                                  void *workspace, size_t ws_bytes, void *stream) {
+static eaga_status backward_impl(const eaga_dims *d, int variant, int row0, int rows, const void *X, const void *E,
+                                 const void *y, const uint8_t *M, const eaga_weights *w, const void *saved,
+                                 const void *dXout, const void *dEout, void *dX, void *dE, void *dy,
+                                 const eaga_weight_grads *dW, void *workspace, size_t ws_bytes, void *stream) {
     NvtxRange range("eaga_backward");
     eaga_status s = check_dims(d);
     if (s != EAGA_OK) return s;
     if (!known_variant(variant)) return EAGA_ERR_INVALID_ARG;
+    if ((s = check_slab(*d, row0, rows)) != EAGA_OK) return s;
     if ((s = check_weights(w)) != EAGA_OK) return s;
     if ((s = check_ptrs({X, E, y, M, saved, dXout, dEout, dX, dE, dy, workspace})) != EAGA_OK) return s;
     if (!dW) return EAGA_ERR_INVALID_ARG;
@@ -138,11 +172,12 @@ eaga_status eaga_backward_variant(const eaga_dims *d, int variant, const void *X
     const Layout L = saved_layout(*d);
     {
         const Extents x = tensor_extents(*d);
-        Span outs[16] = {{dX, x.X}, {dE, x.E}, {dy, x.y}, {workspace, eaga_workspace_size(d, 1)}};
+        const size_t xe = slab_bytes(*d, rows);
+        Span outs[16] = {{dX, x.X}, {dE, xe}, {dy, x.y}, {workspace, eaga_workspace_size(d, 1)}};
         const void *gsrc[12] = {dW->Wq, dW->bq, dW->Wk, dW->bk, dW->Wv, dW->bv,
                                 dW->Wfe, dW->Wfy, dW->bf, dW->We, dW->Wo, dW->bo};
         weight_spans(gsrc, x.wgrad, outs, 4);
-        Span ins[19] = {{X, x.X}, {E, x.E}, {y, x.y}, {M, x.M}, {saved, L.saved_total}, {dXout, x.X}, {dEout, x.E}};
+        Span ins[19] = {{X, x.X}, {E, xe}, {y, x.y}, {M, x.M}, {saved, L.saved_total}, {dXout, x.X}, {dEout, xe}};
         const void *wsrc[12];
         weight_array(w, wsrc);
         weight_spans(wsrc, x.w, ins, 7);
@@ -155,6 +190,8 @@ eaga_status eaga_backward_variant(const eaga_dims *d, int variant, const void *X
     const char *sv = static_cast<const char *>(saved);
     BwdArgs a;
     a.variant = variant;
+    a.row0 = rows < 0 ? 0 : row0;
+    a.rows = rows;
     a.X = X; a.E = E; a.y = y; a.M = M;
     weight_array(w, a.w);
     a.Q = sv + L.q; a.K = sv + L.k; a.V = sv + L.v; a.O = sv + L.o;
@@ -178,6 +215,23 @@ eaga_status eaga_backward_variant(const eaga_dims *d, int variant, const void *X
         return launch_status(fast::backward(*d, a, ws, W.fwd_saved, st));
     }
     return launch_status(generic::backward(*d, a, st));
+}
+
+eaga_status eaga_backward_variant(const eaga_dims *d, int variant, const void *X, const void *E, const void *y,
+                                  const uint8_t *M, const eaga_weights *w, const void *saved, const void *dXout,
+                                  const void *dEout, void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
+                                  void *workspace, size_t ws_bytes, void *stream) {
+    return backward_impl(d, variant, 0, -1, X, E, y, M, w, saved, dXout, dEout, dX, dE, dy, dW, workspace, ws_bytes,
+                         stream);
+}
+
+eaga_status eaga_backward_rows(const eaga_dims *d, int variant, int row0, int rows, const void *X, const void *E_rows,
+                               const void *y, const uint8_t *M, const eaga_weights *w, const void *saved,
+                               const void *dXout, const void *dEout_rows, void *dX, void *dE_rows, void *dy,
+                               const eaga_weight_grads *dW, void *workspace, size_t ws_bytes, void *stream) {
+    if (rows < 0) return EAGA_ERR_INVALID_ARG;
+    return backward_impl(d, variant, row0, rows, X, E_rows, y, M, w, saved, dXout, dEout_rows, dX, dE_rows, dy, dW,
+                         workspace, ws_bytes, stream);
 }
 
 eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,

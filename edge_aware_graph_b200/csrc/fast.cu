@@ -107,6 +107,9 @@ cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common,
         FAST_TRY(tc_gemm(0, rows, 3 * HD, d.dx, 1, A, B, bias, C, HD, nullptr, a.M, a.status, st, true));
     }
     FAST_TRY(stream_after(st, aux->s[0], aux->ev[1]));
+    // a slab of rows: O of the rows outside it is zero (the out-projection and,
+    // in the backward, dWo read every row)
+    if (a.rows >= 0 && a.rows < d.n) FAST_TRY(cudaMemsetAsync(a.O, 0, (size_t)rows * HD * 2, st));
     prof_mark(0, 0, st);
     FAST_TRY(launch_fwd_pairs(d, a, img, a.g, st));
     prof_mark(0, 1, st);
@@ -140,6 +143,10 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
     }
     // the dk, dv accumulators start at zero (beside dO on the auxiliary stream)
     FAST_TRY(cudaMemsetAsync(ws + W.dK32, 0, (size_t)rows * HD * 4 * 2, s1));
+    if (a.rows >= 0 && a.rows < d.n) {   // a slab of rows: dq and the row-block partials of the other rows are zero
+        FAST_TRY(cudaMemsetAsync(ws + W.dQ, 0, (size_t)rows * HD * 2, s1));
+        FAST_TRY(cudaMemsetAsync(ws + W.rparts, 0, (size_t)W.n_rparts * RPART * 4, s1));
+    }
     FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, st));
     FAST_TRY(stream_after(st, s1, ev[1]));
 

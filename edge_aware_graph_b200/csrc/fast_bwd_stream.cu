@@ -108,6 +108,7 @@ struct BwdStreamParams {
     float *dK32, *dV32;      // [B,n,256] fp32 accumulators of dk (unscaled), dv (zero at launch)
     int *status;
     int n;
+    int row0, rows;          // the slab of rows this call owns (E, dE', dE hold rows row0 .. row0+rows-1)
     int light;               // Light Edge variant: no per-edge FiLM map; E is not read, dE = dE'
     int unnorm;              // unnormalised variant: the edge path reaches s' directly
     uint32_t prefetch_ahead;   // CTAs between this one and the one whose first tiles it prefetches
@@ -125,7 +126,10 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
     const int tid = threadIdx.x, W = tid >> 5, q = W & 3, hq = (W >> 2) & 3, t = tid & 31, c4 = t & 3, g8 = t >> 2;
     const int n = p.n, nch = (n + 31) / 32;
-    const int b = blockIdx.y, i0 = blockIdx.x * TB, item = blockIdx.y * gridDim.x + blockIdx.x;
+    // i0: the row block's first row in the graph; i0l: in the slab (E, dE', dE
+    // rows); item: the row block's partials, (graph, row block of the graph)
+    const int b = blockIdx.y, i0l = blockIdx.x * TB, i0 = p.row0 + i0l;
+    const int item = blockIdx.y * ((n + TB - 1) / TB) + i0 / TB;
     const uint32_t bars = sbase + S::BAR;
     auto bar = [&](int k) { return bars + 8 * k; };
     float *g = reinterpret_cast<float *>(sp + S::G);
@@ -327,8 +331,8 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         const uint64_t pol = pass2 ? drop_l2 : keep_l2;
 #pragma unroll
                         for (int s = 0; s < 2; ++s) {
-                            if (!light) tma_load_5d_hint(slot_addr(li, s), &tmE, fb, 0, i0 / 2, x0, s, b, pol);
-                            tma_load_5d_hint(slot_addr(li, 2 + s), &tmDEp, fb, 0, i0 / 2, x0, s, b, pol);
+                            if (!light) tma_load_5d_hint(slot_addr(li, s), &tmE, fb, 0, i0l / 2, x0, s, b, pol);
+                            tma_load_5d_hint(slot_addr(li, 2 + s), &tmDEp, fb, 0, i0l / 2, x0, s, b, pol);
                         }
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
@@ -345,7 +349,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         for (int s = 0; s < 2; ++s) {
                             const uint8_t sl = take_slot();
                             ctab[(dk % BS_NCOPY) * 2 + s] = sl;
-                            tma_load_5d_hint(sbase + sl * BS_SLOT, &tmDEp, cb, 0, i0 / 2, x0, s, b, drop_l2);
+                            tma_load_5d_hint(sbase + sl * BS_SLOT, &tmDEp, cb, 0, i0l / 2, x0, s, b, drop_l2);
                         }
                         ++load_dk;
                     }
@@ -357,7 +361,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
             for (int it = 0; it < nload; ++it) {
                 if (it == nl && p.prefetch_ahead) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
-                    const uint32_t cid = (uint32_t)item + p.prefetch_ahead;
+                    const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
                         const int prb = cid % gridDim.x, pb = cid / gridDim.x;
                         for (int cc = 0; cc < nch && cc < 2; ++cc) {
@@ -385,8 +389,8 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     if (!cta_wait(bar(BB_COPY + dk % BS_NCOPY), (dk / BS_NCOPY) & 1, fail, p.status)) continue;
                     const uint32_t s0 = ctab[(dk % BS_NCOPY) * 2], s1 = ctab[(dk % BS_NCOPY) * 2 + 1];
                     const int x0 = 32 * chunk_of_it(it);
-                    tma_store_5d_hint(&tmDE, sbase + s0 * BS_SLOT, 0, i0 / 2, x0, 0, b, drop_l2);
-                    tma_store_5d_hint(&tmDE, sbase + s1 * BS_SLOT, 0, i0 / 2, x0, 1, b, drop_l2);
+                    tma_store_5d_hint(&tmDE, sbase + s0 * BS_SLOT, 0, i0l / 2, x0, 0, b, drop_l2);
+                    tma_store_5d_hint(&tmDE, sbase + s1 * BS_SLOT, 0, i0l / 2, x0, 1, b, drop_l2);
                     tma_store_commit();
                     // the previous copy's slots are free once its store has read them
                     if (pend_mask) {
@@ -638,7 +642,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         const int i = i0 + 2 * c4 + e;
                         if (i < n && j < n)
                             residual16_to_global(sp + (slot_addr(li, 2 + e) - sbase) + L * 128, L, hq, dv, !light,
-                                                 p.dE + ((((size_t)b * n + i) * n + j) * DE + 16 * hq));
+                                                 p.dE + ((((size_t)b * p.rows + i - p.row0) * n + j) * DE + 16 * hq));
                     }
                 }
                 tc_fence_before();
@@ -737,8 +741,9 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
     static std::atomic<uint32_t> attr_set{0};
     if (cudaError_t e = ensure_smem_attr(k_bwd_stream, BsSmem::BYTES, attr_set); e != cudaSuccess) return e;
     CUtensorMap mE, mDEp, mDE, mK, mV;
-    if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mDEp, a.dEout, d.B, d.n, false, 32, 1) ||
-        !encode_pair_map(&mDE, a.dE, d.B, d.n, false, 32, 1) || !encode_node_map(&mK, a.K, d.B, d.n, 32) ||
+    const int rows = a.rows < 0 ? d.n : a.rows;
+    if (!encode_pair_map(&mE, a.E, d.B, rows, d.n, 32, 1) || !encode_pair_map(&mDEp, a.dEout, d.B, rows, d.n, 32, 1) ||
+        !encode_pair_map(&mDE, a.dE, d.B, rows, d.n, 32, 1) || !encode_node_map(&mK, a.K, d.B, d.n, 32) ||
         !encode_node_map(&mV, a.V, d.B, d.n, 32))
         return cudaErrorInvalidValue;
     BwdStreamParams p;
@@ -755,10 +760,12 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
     p.dV32 = reinterpret_cast<float *>(ws + W.dV32);
     p.status = a.status;
     p.n = d.n;
+    p.row0 = a.row0;
+    p.rows = rows;
     p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
     p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)sm_count();
-    k_bwd_stream<<<dim3((d.n + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, p);
+    k_bwd_stream<<<dim3((rows + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, p);
     return cudaGetLastError();
 }
 

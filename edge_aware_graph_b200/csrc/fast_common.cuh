@@ -81,7 +81,7 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
     return W;
 }
 
-bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transposed, int box_rows, int box_s = 2);
+bool encode_pair_map(CUtensorMap *m, const void *base, int B, int rows, int n, int box_rows, int box_s = 2);
 bool encode_node_map(CUtensorMap *m, const void *base, int B, int n, int box_rows);
 
 

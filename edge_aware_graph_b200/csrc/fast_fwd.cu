@@ -103,6 +103,7 @@ struct FwdParams {
     float *LSE;
     int *status;
     int n;
+    int row0, rows;          // the slab of rows this call owns (E, E' hold rows row0 .. row0+rows-1)
     int cs;                  // CTAs per row block (a cluster when > 1)
     int light;               // Light Edge variant: no per-edge FiLM map, no E in pass 1, no FiLM products
     int unnorm;              // unnormalised variant: the edge update takes s' instead of a
@@ -122,7 +123,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     const int q = W & 3, hp = (W >> 2) & 1;   // TMEM quadrant, head quad (compute warps)
     const int n = p.n, nch = (n + 31) / 32, cs = p.cs;
     const int cpc = (nch + cs - 1) / cs;                        // chunks per CTA of the row block
-    const int rank = blockIdx.x % cs, b = blockIdx.y, i0 = (blockIdx.x / cs) * TB;
+    // i0: the row block's first row in the graph; i0l: in the slab (E, E' rows)
+    const int rank = blockIdx.x % cs, b = blockIdx.y, i0l = (blockIdx.x / cs) * TB, i0 = p.row0 + i0l;
     const int c_begin = rank * cpc, nchl = max(0, min(nch, c_begin + cpc) - c_begin);
     const uint32_t bars = sbase + S::BAR;
     auto bar = [&](int k) { return bars + 8 * k; };
@@ -291,8 +293,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         mbar_expect_tx(fb, ns * FS_SLOT);   // releases the table entry too
                         const uint64_t pol = pass2 ? drop_l2 : keep_l2;
                         if (pass2 || !light) {
-                            tma_load_5d_hint(slot_at(sw, 0), &tmE, fb, 0, i0 / 2, j0, 0, b, pol);
-                            tma_load_5d_hint(slot_at(sw, 1), &tmE, fb, 0, i0 / 2, j0, 1, b, pol);
+                            tma_load_5d_hint(slot_at(sw, 0), &tmE, fb, 0, i0l / 2, j0, 0, b, pol);
+                            tma_load_5d_hint(slot_at(sw, 1), &tmE, fb, 0, i0l / 2, j0, 1, b, pol);
                         }
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
@@ -301,7 +303,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         }
                         if (!pass2 && !light && li + FS_PF < nl)
                             for (int s = 0; s < 2; ++s)
-                                tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (c_begin + lc[li + FS_PF]), s, b);
+                                tma_prefetch_5d(&tmE, 0, i0l / 2, 32 * (c_begin + lc[li + FS_PF]), s, b);
                         ++load_li;
                     } else {
                         const int dk = load_dk;
@@ -312,7 +314,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         for (int s = 0; s < 2; ++s) {
                             const uint8_t sl = take_slot();
                             ctab[(dk % FS_NCOPY) * 2 + s] = sl;
-                            tma_load_5d_hint(sbase + sl * FS_SLOT, &tmE, cb, 0, i0 / 2, j0, s, b, drop_l2);
+                            tma_load_5d_hint(sbase + sl * FS_SLOT, &tmE, cb, 0, i0l / 2, j0, s, b, drop_l2);
                         }
                         ++load_dk;
                     }
@@ -320,7 +322,7 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
             };
             for (int c = 0; c < nl && c < FS_PF && !light; ++c)
-                for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0 / 2, 32 * (c_begin + lc[c]), s, b);
+                for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, i0l / 2, 32 * (c_begin + lc[c]), s, b);
             issue_loads();
             // iterations are taken off the ring in order: a live one once the
             // compute warps are done with it (stage_done), a copy once its
@@ -357,8 +359,8 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     s1 = ctab[(dk % FS_NCOPY) * 2 + 1];
                 }
                 if (pass2 || !lv) {
-                    tma_store_5d_hint(&tmEo, sbase + s0 * FS_SLOT, 0, i0 / 2, j0, 0, b, drop_l2);
-                    tma_store_5d_hint(&tmEo, sbase + s1 * FS_SLOT, 0, i0 / 2, j0, 1, b, drop_l2);
+                    tma_store_5d_hint(&tmEo, sbase + s0 * FS_SLOT, 0, i0l / 2, j0, 0, b, drop_l2);
+                    tma_store_5d_hint(&tmEo, sbase + s1 * FS_SLOT, 0, i0l / 2, j0, 1, b, drop_l2);
                     tma_store_commit();
                     // the previous store's slots are free once it has read them
                     if (pend_mask) {
@@ -697,7 +699,8 @@ cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t
         }
     }
     CUtensorMap mE, mEo, mK, mV;
-    if (!encode_pair_map(&mE, a.E, d.B, d.n, false, 32, 1) || !encode_pair_map(&mEo, a.Eout, d.B, d.n, false, 32, 1) ||
+    const int rows = a.rows < 0 ? d.n : a.rows;
+    if (!encode_pair_map(&mE, a.E, d.B, rows, d.n, 32, 1) || !encode_pair_map(&mEo, a.Eout, d.B, rows, d.n, 32, 1) ||
         !encode_node_map(&mK, a.K, d.B, d.n, 32) || !encode_node_map(&mV, a.V, d.B, d.n, 32))
         return cudaErrorInvalidValue;
     const int cs = fwd_cluster_size(d.n);
@@ -711,11 +714,13 @@ cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t
     p.LSE = a.LSE;
     p.status = a.status;
     p.n = d.n;
+    p.row0 = a.row0;
+    p.rows = rows;
     p.cs = cs;
     p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
     p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)(2 * sm_count());   // two CTAs per SM
-    const dim3 grid(((d.n + TB - 1) / TB) * cs, d.B);
+    const dim3 grid(((rows + TB - 1) / TB) * cs, d.B);
     if (cs == 1) {
         k_fwd_stream<<<grid, FS_THR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
         return cudaGetLastError();

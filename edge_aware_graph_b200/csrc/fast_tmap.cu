@@ -24,28 +24,20 @@ static EncodeTiledFn get_encode() {
     return fn;
 }
 
-// A [B, n, n, 64] bf16 pair tensor viewed as 5-D with a box of 8 x box_rows
-// pairs (box_s = 2) or of the 4 x box_rows pairs of one parity s (box_s = 1).
-// Row tile (transposed = false): dims (c, ic, j, s, b) with i = 2ic + s, so the
-// box lands in shared memory as [s][j box_rows][ic 4][c 64].  Column tile
-// (transposed = true): dims (c, jc, i, s, b) with j = 2jc + s, landing as
-// [s][i box_rows][jc 4][c 64].  Requires n even (i = 2ic + s stays inside the graph).
-bool encode_pair_map(CUtensorMap *m, const void *base, int B, int n, bool transposed, int box_rows, int box_s) {
+// A [B, rows, n, 64] bf16 pair tensor (rows = n for a whole graph, fewer for
+// a slab of its rows) viewed as 5-D, dims (c, ic, j, s, b) with i = 2ic + s,
+// and a box of 4 x box_rows pairs of one parity s (box_s = 1) or 8 x box_rows
+// (box_s = 2), landing in shared memory as [s][j box_rows][ic 4][c 64].
+// Requires rows even (i = 2ic + s stays inside the slab).
+bool encode_pair_map(CUtensorMap *m, const void *base, int B, int rows, int n, int box_rows, int box_s) {
     auto enc = get_encode();
     if (!enc) return false;
     const cuuint64_t rowb = DE * 2;                       // one pair: 128 bytes
-    const cuuint64_t dims[5] = {DE, (cuuint64_t)(n / 2), (cuuint64_t)n, 2, (cuuint64_t)B};
-    cuuint64_t strides[4];
-    if (!transposed) {
-        strides[0] = 2 * (cuuint64_t)n * rowb;             // ic -> two rows i
-        strides[1] = rowb;                                  // j
-        strides[2] = (cuuint64_t)n * rowb;                  // s -> one row i
-    } else {
-        strides[0] = 2 * rowb;                              // jc -> two columns j
-        strides[1] = (cuuint64_t)n * rowb;                  // i
-        strides[2] = rowb;                                  // s -> one column j
-    }
-    strides[3] = (cuuint64_t)n * n * rowb;                  // b
+    const cuuint64_t dims[5] = {DE, (cuuint64_t)(rows / 2), (cuuint64_t)n, 2, (cuuint64_t)B};
+    const cuuint64_t strides[4] = {2 * (cuuint64_t)n * rowb,          // ic -> two rows i
+                                   rowb,                              // j
+                                   (cuuint64_t)n * rowb,              // s -> one row i
+                                   (cuuint64_t)rows * n * rowb};      // b
     const cuuint32_t box[5] = {64, 4, (cuuint32_t)box_rows, (cuuint32_t)box_s, 1};
     const cuuint32_t es[5] = {1, 1, 1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, es,

@@ -10,8 +10,11 @@ namespace eaga {
 // Weight order everywhere: Wq bq Wk bk Wv bv Wfe Wfy bf We Wo bo.
 // `variant` is an eaga_variant: the layer, Light Edge (no per-edge FiLM map)
 // or the unnormalised edge update (from the modulated scores s').
+// row0, rows: the slab of each graph's rows the call owns (rows < 0: the
+// whole graph); E, Eout (dEout, dE) then hold those rows only, [B, rows, n, de].
 struct FwdArgs {
     int variant = 0;
+    int row0 = 0, rows = -1;
     const void *X, *E, *y;
     const uint8_t *M;
     const void *w[12];
@@ -24,6 +27,7 @@ struct FwdArgs {
 
 struct BwdArgs {
     int variant = 0;
+    int row0 = 0, rows = -1;
     const void *X, *E, *y;
     const uint8_t *M;
     const void *w[12];

@@ -22,7 +22,7 @@ STATUS = {0: "EAGA_OK", 1: "EAGA_ERR_INVALID_ARG", 2: "EAGA_ERR_UNSUPPORTED", 3:
 EXPORTED = ("eaga_workspace_size", "eaga_saved_size", "eaga_forward", "eaga_backward",
             "eaga_debug_attention_map", "eaga_get_device_status", "eaga_strerror",
             "eaga_set_profile_events", "eaga_kernel_launches", "eaga_forward_noalloc", "eaga_debug_wait_probe",
-            "eaga_forward_variant", "eaga_backward_variant")
+            "eaga_forward_variant", "eaga_backward_variant", "eaga_forward_rows", "eaga_backward_rows")
 # layer variants (eaga_variant): the layer, Light Edge, the unnormalised edge update
 VARIANTS = {"layer": 0, "light_edge": 1, "unnormalised": 2}
 
@@ -68,6 +68,12 @@ def lib():
         L.eaga_backward_variant.argtypes = [ctypes.POINTER(Dims), i32, vp, vp, vp, vp, ctypes.POINTER(Weights), vp,
                                             vp, vp, vp, vp, vp, ctypes.POINTER(Weights), vp, sz, vp]
         L.eaga_backward_variant.restype = i32
+        L.eaga_forward_rows.argtypes = [ctypes.POINTER(Dims), i32, i32, i32, vp, vp, vp, vp, ctypes.POINTER(Weights),
+                                        vp, vp, vp, vp, sz, vp]
+        L.eaga_forward_rows.restype = i32
+        L.eaga_backward_rows.argtypes = [ctypes.POINTER(Dims), i32, i32, i32, vp, vp, vp, vp, ctypes.POINTER(Weights),
+                                         vp, vp, vp, vp, vp, vp, ctypes.POINTER(Weights), vp, sz, vp]
+        L.eaga_backward_rows.restype = i32
         L.eaga_forward_noalloc.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, ctypes.POINTER(Weights),
                                            vp, vp, vp, vp]
         L.eaga_forward_noalloc.restype = i32
@@ -190,6 +196,32 @@ def backward(d: Dims, X, E, y, M, W: dict, saved, dXout, dEout, dX, dE, dy, dW: 
         _check(lib().eaga_backward(ctypes.byref(d), *args), "eaga_backward")
     else:
         _check(lib().eaga_backward_variant(ctypes.byref(d), VARIANTS[variant], *args), "eaga_backward_variant")
+
+
+def forward_rows(d: Dims, row0: int, rows: int, X, E_rows, y, M, W: dict, Xout, Eout_rows, saved, workspace,
+                 stream=None, variant: str = "layer"):
+    """eaga_forward_rows: the rows row0 .. row0+rows-1 of every graph, E_rows and
+    Eout_rows [B, rows, n, de] slabs."""
+    sd = _storage(d)
+    rc = lib().eaga_forward_rows(ctypes.byref(d), VARIANTS[variant], int(row0), int(rows), _p(X, "X", sd),
+                                 _p(E_rows, "E_rows", sd), _p(y, "y", sd), _p(M, "M", _u8()),
+                                 ctypes.byref(_weights(W, sd)), _p(Xout, "Xout", sd), _p(Eout_rows, "Eout_rows", sd),
+                                 _p(saved, "saved"), _p(workspace, "workspace"), _nbytes(workspace), _stream(stream))
+    _check(rc, "eaga_forward_rows")
+
+
+def backward_rows(d: Dims, row0: int, rows: int, X, E_rows, y, M, W: dict, saved, dXout, dEout_rows, dX, dE_rows,
+                  dy, dW: dict, workspace, stream=None, variant: str = "layer"):
+    """eaga_backward_rows: this slab's part of dX, dy and the weight gradients
+    (dXout zero outside the slab's rows), and the slab's dE."""
+    sd = _storage(d)
+    rc = lib().eaga_backward_rows(ctypes.byref(d), VARIANTS[variant], int(row0), int(rows), _p(X, "X", sd),
+                                  _p(E_rows, "E_rows", sd), _p(y, "y", sd), _p(M, "M", _u8()),
+                                  ctypes.byref(_weights(W, sd)), _p(saved, "saved"), _p(dXout, "dXout", sd),
+                                  _p(dEout_rows, "dEout_rows", sd), _p(dX, "dX", sd), _p(dE_rows, "dE_rows", sd),
+                                  _p(dy, "dy", sd), ctypes.byref(_weights(dW, _f32(), "dW")),
+                                  _p(workspace, "workspace"), _nbytes(workspace), _stream(stream))
+    _check(rc, "eaga_backward_rows")
 
 
 def debug_attention_map(d: Dims, E, M, W: dict, y, saved, A, stream=None):

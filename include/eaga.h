@@ -175,6 +175,37 @@ EAGA_API eaga_status eaga_backward_variant(const eaga_dims *dims, int variant,
                                            void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
                                            void *workspace, size_t ws_bytes, void *stream);
 
+/* Row slabs of one graph (rows split over ranks: the AI-summary page's method
+ * paragraph notes the edge update stays quadratic, so a large graph's pairs
+ * are split by rows i).  The call owns rows row0 .. row0+rows-1 of every
+ * graph: E_rows, Eout_rows, dEout_rows and dE_rows are [B, rows, n, de]
+ * slabs of the pair tensors; X, y, M, Xout, dXout, dX, dy, the weights and
+ * `saved` are whole.  Specialised bf16 path only (EAGA_ERR_UNSUPPORTED
+ * otherwise); row0 a multiple of 8, rows even and a multiple of 8 unless the
+ * slab ends at n (EAGA_ERR_INVALID_ARG otherwise).  Workspace sizes are those
+ * of the whole layer.
+ *
+ * Forward: Q, K, V of every node (each rank computes them: a node GEMM, no
+ * exchange), then the pairs of the slab's rows against all columns.  Writes
+ * Eout_rows, and in Xout and `saved` the slab's rows (O of the other rows is
+ * zero; their Xout rows are left unspecified).
+ *
+ * Backward: the gradients of L_r = <dXout, Xout> + <dEout_rows, Eout_rows>
+ * with dXout zero outside the slab's rows (the caller passes it so).  dE_rows
+ * is final; dX, dy and the weight gradients are this slab's part, and the
+ * sum of the parts over slabs covering every row is the layer's gradient
+ * (the layer is linear in its upstream gradients), e.g. one all-reduce. */
+EAGA_API eaga_status eaga_forward_rows(const eaga_dims *dims, int variant, int row0, int rows,
+                                       const void *X, const void *E_rows, const void *y, const uint8_t *M,
+                                       const eaga_weights *w, void *Xout, void *Eout_rows, void *saved,
+                                       void *workspace, size_t ws_bytes, void *stream);
+EAGA_API eaga_status eaga_backward_rows(const eaga_dims *dims, int variant, int row0, int rows,
+                                        const void *X, const void *E_rows, const void *y, const uint8_t *M,
+                                        const eaga_weights *w, const void *saved,
+                                        const void *dXout, const void *dEout_rows,
+                                        void *dX, void *dE_rows, void *dy, const eaga_weight_grads *dW,
+                                        void *workspace, size_t ws_bytes, void *stream);
+
 /* Forward without a caller-provided workspace.  The paper has no counterpart
  * of this call; it exists for callers that cannot allocate device memory
  * for scratch: plain C clients that link this library but no device
