@@ -330,6 +330,111 @@ def run_ours(args):
     return out
 
 
+def run_rows(args):
+    """Row-sharded training step (edge_aware_graph_b200/rowshard.py): every rank
+    holds the same graphs and owns a slab of each graph's rows; a step is the
+    slab's forward and backward plus one all-reduce of the gradient parts.
+    Under torchrun the N ranks split the rows N ways (total work fixed: strong
+    scaling).  With one GPU, --row-slabs K runs rank 0's slab of a K-way split
+    alone (no exchange), the share one GPU of K would take."""
+    WORKLOAD = WORKLOADS[args.workload]
+    import torch
+    import torch.distributed as dist
+
+    from edge_aware_graph_b200 import dp, eaga, rowshard
+    from edge_aware_graph_b200 import inputs as I
+    from edge_aware_graph_b200.buffers import LayerBuffers
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    ways = world if world > 1 else max(1, args.row_slabs)
+    p = I.preset(WORKLOAD)
+    d = I.draw_inputs(p, with_grads=True)
+    W = I.draw_weights(p)
+    buf = LayerBuffers(p.B, p.n, p.dx, p.de, p.dy, p.H, p.dh, dtype=p.dtype, backward=True)
+    buf.load_inputs(d, W)
+    row0, rows = rowshard.row_slabs(p.n, ways)[rank if world > 1 else 0]
+    E_r = buf.E[:, row0:row0 + rows].contiguous()
+    dEo_r = buf.dEout[:, row0:row0 + rows].contiguous()
+    Eo_r, dE_r = torch.empty_like(E_r), torch.empty_like(E_r)
+    del buf.E, buf.Eout, buf.dEout, buf.dE             # the rank holds slabs only
+    dX32 = torch.zeros(p.B, p.n, p.dx, dtype=torch.float32, device="cuda")
+    dy32 = torch.zeros(p.B, p.dy, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rowshard.forward_rows(buf.dims, row0, rows, buf.X, E_r, buf.y, buf.M, buf.W, buf.Xout, Eo_r, buf.saved,
+                              buf.ws_fwd, stream)
+        rowshard.backward_rows(buf.dims, row0, rows, buf.X, E_r, buf.y, buf.M, buf.W, buf.saved, buf.dXout, dEo_r,
+                               buf.dX, dE_r, buf.dy, buf.dW, buf.ws_bwd, stream)
+        if world > 1:
+            dX32.copy_(buf.dX)
+            dy32.copy_(buf.dy)
+            rowshard.allreduce_parts([dX32, dy32, buf.dW_flat])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    nk = min(args.steps, 20)
+    ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+    for a, b in ev_r:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    for k in range(nk):
+        eaga.set_profile_events(2, *ev_r[k])
+        step()
+    torch.cuda.synchronize()
+    eaga.set_profile_events(2)
+    rows_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_r)
+
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms_total = dp.max_over_ranks(t0.elapsed_time(t1), "cuda")
+    launches = (eaga.kernel_launches(buf.dims, False) + eaga.kernel_launches(buf.dims, True)) * K
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    ms_step = ms_total / K
+    pairs_step = p.B * p.n * p.n if world > 1 else p.B * rows * p.n
+    peak, peak_kind = measured_peaks()
+    kb = 3 * p.B * rows * p.n * p.de * 2          # the slab's E, dE' read and dE written
+    return {
+        "metric": METRIC, "value": pairs_step / (ms_step / 1e3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if world > 1 else "one rank's share", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded graphs; edge_aware_graph_b200/inputs.py)",
+        "config": {"workload": DESCRIBE[WORKLOAD] + f"; rows split {ways} ways (rank 0's slab: rows {row0}.."
+                   f"{row0 + rows - 1} of every graph" + ("" if world > 1 else ", run alone") + ")",
+                   "global_batch": p.B, "seq_len": p.n, "parallelism": f"rows{ways}",
+                   "l2": "inputs larger than L2" if E_r.numel() * 2 > (126 << 20) else "slab smaller than L2",
+                   "launch": "eager"},
+        "roofline": {"bound": "hbm", "kernel": "k_bwd_stream (backward row pair kernel, the slab)",
+                     "achieved": kb / (rows_ms / 1e3) / 1e9, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": kb / (rows_ms / 1e3) / 1e9 / peak, "traffic": None, "algorithmic_bytes": kb,
+                     "ms_per_launch": rows_ms},
+        "clocks": clk, "e2e": None, "gpu_launches": launches,
+    }
+
+
 def run_sample(args, name):
     """Sampling-time forward: the forward alone, called once per step on one of
     SAMPLE_ROTATION resident batches in turn (inputs larger than L2), the
@@ -643,6 +748,10 @@ def run_reference_sample(args, name, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--parallel", default="batch", choices=["batch", "rows"],
+                    help="split graphs over the ranks (batch) or each graph's rows (rows: eaga_*_rows)")
+    ap.add_argument("--row-slabs", type=int, default=2,
+                    help="with --parallel rows on one GPU: rank 0's slab of this many")
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -662,7 +771,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl == "reference":
+        out = run_reference(args)
+    elif args.parallel == "rows" and args.workload in TRAINING:
+        out = run_rows(args)
+    else:
+        out = run_ours(args)
     if out is not None:
         print(json.dumps(out), flush=True)
 
