@@ -17,10 +17,11 @@
 //           a running D per thread; S and dP stay in TMEM for pass 2 (32
 //           columns per chunk, n <= 224; larger n reloads K and V);
 //   pass 2: (the chunks in reverse, so that E and dE' come back from L2) dS',
-//           dgamma, dbeta, ds; dE = dE' + df Wfe^T on the tensor cores, added
-//           to the dE' tile in registers and written from there; dWfe += E^T df
-//           and dWe^T += dE'^T a on the tensor cores (MN-major operands
-//           straight from the tiles, accumulated in TMEM over the row block);
+//           dgamma, dbeta, ds; dWfe += E^T df and dWe^T += dE'^T a on the
+//           tensor cores (MN-major operands straight from the tiles,
+//           accumulated in TMEM over the row block); dE = dE' + df Wfe^T on the
+//           tensor cores, added in place to the dE' tile once those products
+//           have read it, and stored with TMA;
 //           dq += ds K (warp MMAs); and the row block's share of dk_j, dv_j for
 //           the chunk's columns (warp MMAs over the 8 rows), added into fp32
 //           accumulators [B,n,H*dh] with vector reductions in L2.
@@ -357,7 +358,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                 }
             };
             issue_loads();
-            uint32_t pend_mask = 0u;   // slots of the last copy store, not yet known to have read them
+            uint32_t pend_mask = 0u;   // slots of the last dE store, not yet known to have read them
             for (int it = 0; it < nload; ++it) {
                 if (it == nl && p.prefetch_ahead) {
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
@@ -374,30 +375,46 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                         }
                     }
                 }
+                uint32_t s0, s1;   // the slots of the two dE tiles a store reads
+                const bool pass2 = it >= nl && it < nit;
                 if (is_live(it)) {
                     const int li = done_li++;
                     if (!cta_wait(bar(BB_STAGE_DONE + (li & 3)), (li >> 2) & 1, fail, p.status)) continue;
-                    const bool pass2 = it >= nl && it < nit;
                     if (pass2) {
                         // the chunk's tiles are read by its weight-gradient products until these complete
                         const int p2 = li - nl;
                         if (!cta_wait(bar(BB_WG_DONE + (p2 & 1)), (p2 >> 1) & 1, fail, p.status)) continue;
                     }
-                    for (int k = 0; k < (pass2 ? ns2 : 6); ++k) free_mask |= 1u << stab[(li % BS_NFULL) * 8 + k];
+                    // pass 2: the dE' tiles (now dE) are stored first; the other slots are free
+                    for (int k = 0; k < (pass2 ? ns2 : 6); ++k)
+                        if (!pass2 || (k != 2 && k != 3)) free_mask |= 1u << stab[(li % BS_NFULL) * 8 + k];
+                    s0 = stab[(li % BS_NFULL) * 8 + 2];
+                    s1 = stab[(li % BS_NFULL) * 8 + 3];
                 } else {
                     const int dk = done_dk++;
                     if (!cta_wait(bar(BB_COPY + dk % BS_NCOPY), (dk / BS_NCOPY) & 1, fail, p.status)) continue;
-                    const uint32_t s0 = ctab[(dk % BS_NCOPY) * 2], s1 = ctab[(dk % BS_NCOPY) * 2 + 1];
+                    s0 = ctab[(dk % BS_NCOPY) * 2];
+                    s1 = ctab[(dk % BS_NCOPY) * 2 + 1];
+                }
+                if (pass2 || !is_live(it)) {
                     const int x0 = 32 * chunk_of_it(it);
                     tma_store_5d_hint(&tmDE, sbase + s0 * BS_SLOT, 0, i0l / 2, x0, 0, b, drop_l2);
                     tma_store_5d_hint(&tmDE, sbase + s1 * BS_SLOT, 0, i0l / 2, x0, 1, b, drop_l2);
                     tma_store_commit();
-                    // the previous copy's slots are free once its store has read them
-                    if (pend_mask) {
-                        tma_store_wait_read1();
-                        free_mask |= pend_mask;
+                    if (keep) {
+                        // the previous store's slots are free once it has read them
+                        if (pend_mask) {
+                            tma_store_wait_read1();
+                            free_mask |= pend_mask;
+                        }
+                        pend_mask = (1u << s0) | (1u << s1);
+                    } else {
+                        // six slots a pass-2 chunk: two chunks in flight only if this
+                        // store's slots come back before the next loads
+                        tma_store_wait_read0();
+                        free_mask |= pend_mask | (1u << s0) | (1u << s1);
+                        pend_mask = 0u;
                     }
-                    pend_mask = (1u << s0) | (1u << s1);
                 }
                 issue_loads();
             }
@@ -626,24 +643,21 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     }
                 }
 
-                // ---------------- dE = dE' + df Wfe^T (Light Edge: dE = dE'), written from registers:
-                // the dE' tile stays as loaded for the weight-gradient product that reads it
-                cta_wait(bar(BB_DE_FULL), (li - nl) & 1, fail, p.status);
-                tc_fence_after();
-                {
-                    const int j = j0 + 8 * q + g8;
+                // ---------------- dE = dE' + df Wfe^T (Light Edge: dE = dE'), in place in the
+                // dE' tile once this chunk's weight-gradient products (which read the tile)
+                // have completed; the TMA warp stores it
+                if (!light) {
+                    cta_wait(bar(BB_DE_FULL), (li - nl) & 1, fail, p.status);
+                    cta_wait(bar(BB_WG_DONE + ((li - nl) & 1)), ((li - nl) >> 1) & 1, fail, p.status);
+                    tc_fence_after();
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         float dv[16];
-                        if (!light) {
-                            tmem_ld16(tl + BS_TM_DE + 64 * e + 16 * hq, dv);
-                            tmem_ld_wait();
-                        }
-                        const int i = i0 + 2 * c4 + e;
-                        if (i < n && j < n)
-                            residual16_to_global(sp + (slot_addr(li, 2 + e) - sbase) + L * 128, L, hq, dv, !light,
-                                                 p.dE + ((((size_t)b * p.rows + i - p.row0) * n + j) * DE + 16 * hq));
+                        tmem_ld16(tl + BS_TM_DE + 64 * e + 16 * hq, dv);
+                        tmem_ld_wait();
+                        add_residual16(sp + (slot_addr(li, 2 + e) - sbase) + L * 128, L, hq, dv);
                     }
+                    fence_proxy_async_smem();
                 }
                 tc_fence_before();
                 __syncwarp();
