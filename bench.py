@@ -52,12 +52,15 @@ FALLBACK_HBM_GBS = 6650.0
 # the dominant kernels on each workload, from one ncu capture of the kernels as
 # they are (the summaries under profiles/ give the commands).  A kernel that
 # changes reports null until it is captured again.  Large: the counters come
-# in GB with three digits (1.78 GB read by k_bwd_stream).
+# in GB with three digits (1.77 GB read by k_bwd_stream).  Planar: one batch's
+# E' (32 MiB) fits in L2, so within the captured launch its writes stay in L2
+# and reach DRAM later, under the next batch's launch.
 NCU_TRAFFIC = {
-    ("sbm", "k_fwd_stream"): 158670000 + 96130000,
-    ("sbm", "k_bwd_stream"): 254333696 + 115731712,
-    ("large", "k_fwd_stream"): 809080000 + 481850000,
-    ("large", "k_bwd_stream"): 1780000000 + 504840000,
+    ("sbm", "k_fwd_stream"): 167305984 + 97689344,
+    ("sbm", "k_bwd_stream"): 252016128 + 113165824,
+    ("large", "k_fwd_stream"): 736150000 + 481330000,
+    ("large", "k_bwd_stream"): 1770000000 + 501140000,
+    ("planar", "k_fwd_stream"): 39940000 + 848900,
 }
 
 
