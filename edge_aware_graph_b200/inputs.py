@@ -214,6 +214,51 @@ def draw_weights(p: Preset, seed_offset: int = 1000) -> dict:
     return out
 
 
+# parameters of the graph-transformer block around the layer: per sub-block
+# (x node, e edge, y global) LayerNorm 1, the FFN (hidden width twice the
+# feature width) and LayerNorm 2; then the pooling maps of the global update
+BLOCK_SUB_PARAMS = ("ln1_g", "ln1_s", "W1", "b1", "W2", "b2", "ln2_g", "ln2_s")
+BLOCK_WEIGHT_NAMES = tuple(f"{s}_{k}" for s in ("x", "e", "y") for k in BLOCK_SUB_PARAMS) + ("Wyx", "Wye", "by")
+
+
+def block_weight_shapes(p: Preset) -> dict:
+    """[in, out] shapes of the block's parameters and the fan-in of each draw
+    (None for LayerNorm parameters)."""
+    out = {}
+    for s, w in (("x", p.dx), ("e", p.de), ("y", p.dy)):
+        f = 2 * w
+        out.update({f"{s}_ln1_g": ((w,), None), f"{s}_ln1_s": ((w,), None),
+                    f"{s}_W1": ((w, f), w), f"{s}_b1": ((f,), w),
+                    f"{s}_W2": ((f, w), f), f"{s}_b2": ((w,), f),
+                    f"{s}_ln2_g": ((w,), None), f"{s}_ln2_s": ((w,), None)})
+    out.update({"Wyx": ((p.dx, p.dy), p.dx), "Wye": ((p.de, p.dy), p.de), "by": ((p.dy,), p.dx)})
+    return out
+
+
+def draw_block_weights(p: Preset, seed_offset: int = 2000) -> dict:
+    """Block parameters: matrices and biases ~ N(0,1)/sqrt(fan_in); LayerNorm
+    gains 1 + 0.1 N(0,1), shifts 0.1 N(0,1); rounded to the storage dtype."""
+    rng = np.random.default_rng(p.seed + seed_offset)
+    out = {}
+    for name in BLOCK_WEIGHT_NAMES:
+        shape, fan_in = block_weight_shapes(p)[name]
+        r = rng.standard_normal(shape)
+        if fan_in is not None:
+            w = r / math.sqrt(fan_in)
+        elif name.endswith("_g"):
+            w = 1.0 + 0.1 * r
+        else:
+            w = 0.1 * r
+        out[name] = to_storage(w, p.dtype)
+    return out
+
+
+def draw_block_upstream(p: Preset, seed_offset: int = 3000) -> np.ndarray:
+    """Upstream gradient of the block's global output, dyout [B, dy] ~ N(0,1)."""
+    rng = np.random.default_rng(p.seed + seed_offset)
+    return to_storage(rng.standard_normal((p.B, p.dy)), p.dtype)
+
+
 def _symmetric_noise(rng, n, de, std, dtype=np.float32):
     r = rng.standard_normal((n, n, de), dtype=np.float32) * np.float32(std)
     iu = np.triu(np.ones((n, n), bool))
