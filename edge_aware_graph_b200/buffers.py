@@ -102,3 +102,51 @@ class LayerBuffers:
             out[k] = self.saved[off:off + sz].view(torch_dtype(self.dtype)).view(B, n, hd)
             off = al(off + sz)
         return out
+
+
+class BlockBuffers(LayerBuffers):
+    """LayerBuffers plus the graph-transformer block around the layer: the
+    block's parameters, the layer's outputs X', E' (Xmid, Emid), the block's
+    outputs, saved state, workspaces and gradients."""
+
+    def __init__(self, B, n, dx, de, dy, H, dh, dtype="bf16", device="cuda", backward=True):
+        super().__init__(B, n, dx, de, dy, H, dh, dtype, device, backward)
+        td = torch_dtype(dtype)
+        dev = self.device
+        e = lambda *s: torch.empty(*s, dtype=td, device=dev)
+        self.bshapes = {}
+        for s, w in (("x", dx), ("e", de), ("y", dy)):
+            self.bshapes.update({f"{s}_ln1_g": (w,), f"{s}_ln1_s": (w,), f"{s}_W1": (w, 2 * w), f"{s}_b1": (2 * w,),
+                                 f"{s}_W2": (2 * w, w), f"{s}_b2": (w,), f"{s}_ln2_g": (w,), f"{s}_ln2_s": (w,)})
+        self.bshapes.update({"Wyx": (dx, dy), "Wye": (de, dy), "by": (dy,)})
+        self.Wb = {k: e(*self.bshapes[k]) for k in eaga.BLOCK_WEIGHT_NAMES}
+        self.Xmid, self.Emid = e(B, n, dx), e(B, n, n, de)
+        self.yout = e(B, dy)
+        self.bsaved = torch.empty(eaga.block_saved_size(self.dims), dtype=torch.uint8, device=dev)
+        self.bws_fwd = torch.empty(eaga.block_workspace_size(self.dims, False), dtype=torch.uint8, device=dev)
+        if backward:
+            self.dyout = e(B, dy)
+            self.dEmid = e(B, n, n, de)
+            offs, off = {}, 0
+            for k in eaga.BLOCK_WEIGHT_NAMES:
+                offs[k] = off
+                off += (int(np.prod(self.bshapes[k])) + 63) // 64 * 64
+            self.dWb_flat = torch.zeros(off, dtype=torch.float32, device=dev)
+            self.dWb = {k: self.dWb_flat[offs[k]:offs[k] + int(np.prod(self.bshapes[k]))].view(self.bshapes[k])
+                        for k in eaga.BLOCK_WEIGHT_NAMES}
+            self.bws_bwd = torch.empty(eaga.block_workspace_size(self.dims, True), dtype=torch.uint8, device=dev)
+
+    def load_block(self, block_weights: dict, dyout=None):
+        for k in eaga.BLOCK_WEIGHT_NAMES:
+            self.Wb[k].copy_(host_to_storage_tensor(block_weights[k], self.dtype))
+        if dyout is not None and self.has_backward:
+            self.dyout.copy_(host_to_storage_tensor(dyout, self.dtype))
+
+    def block_forward(self, stream=None):
+        eaga.block_forward(self.dims, self.X, self.E, self.y, self.M, self.W, self.Wb, self.Xmid, self.Emid,
+                           self.Xout, self.Eout, self.yout, self.bsaved, self.bws_fwd, stream)
+
+    def block_backward(self, stream=None):
+        eaga.block_backward(self.dims, self.X, self.E, self.y, self.M, self.W, self.Wb, self.Xmid, self.Emid,
+                            self.bsaved, self.dXout, self.dEout, self.dyout, self.dEmid, self.dX, self.dE,
+                            self.dy, self.dW, self.dWb, self.bws_bwd, stream)

@@ -6,6 +6,7 @@
 #include "common.cuh"
 #include "generic.h"
 #include "fast.h"
+#include "fast_block.h"
 #include "sm100.cuh"
 #include <nvtx3/nvToolsExt.h>
 
@@ -89,7 +90,8 @@ static size_t slab_bytes(const eaga_dims &d, int rows) {
 
 static eaga_status forward_impl(const eaga_dims *d, int variant, int row0, int rows, const void *X, const void *E,
                                 const void *y, const uint8_t *M, const eaga_weights *w, void *Xout, void *Eout,
-                                void *saved, void *workspace, size_t ws_bytes, void *stream) {
+                                void *saved, void *workspace, size_t ws_bytes, void *stream,
+                                bool clear_status = true) {
     NvtxRange range("eaga_forward");
     eaga_status s = check_dims(d);
     if (s != EAGA_OK) return s;
@@ -126,7 +128,7 @@ static eaga_status forward_impl(const eaga_dims *d, int variant, int row0, int r
     a.Q = sv + L.q; a.K = sv + L.k; a.V = sv + L.v; a.O = sv + L.o;
     a.g = reinterpret_cast<float *>(ws + W.g);
     a.status = reinterpret_cast<int *>(ws + W.status);
-    if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (clear_status && cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
     if (fast::supports(*d)) {
         return launch_status(fast::forward(*d, a, ws + W.total_fwd, st));
     }
@@ -157,7 +159,8 @@ eaga_status eaga_forward(const eaga_dims *d, const void *X, const void *E, const
 static eaga_status backward_impl(const eaga_dims *d, int variant, int row0, int rows, const void *X, const void *E,
                                  const void *y, const uint8_t *M, const eaga_weights *w, const void *saved,
                                  const void *dXout, const void *dEout, void *dX, void *dE, void *dy,
-                                 const eaga_weight_grads *dW, void *workspace, size_t ws_bytes, void *stream) {
+                                 const eaga_weight_grads *dW, void *workspace, size_t ws_bytes, void *stream,
+                                 bool clear_status = true) {
     NvtxRange range("eaga_backward");
     eaga_status s = check_dims(d);
     if (s != EAGA_OK) return s;
@@ -210,7 +213,7 @@ static eaga_status backward_impl(const eaga_dims *d, int variant, int row0, int 
     a.dg = reinterpret_cast<float *>(ws + W.dg);
     a.part_stride = W.part_stride;
     a.status = reinterpret_cast<int *>(ws + W.status);
-    if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
+    if (clear_status && cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
     if (fast::supports(*d)) {
         return launch_status(fast::backward(*d, a, ws, W.fwd_saved, st));
     }
@@ -240,6 +243,134 @@ eaga_status eaga_backward(const eaga_dims *d, const void *X, const void *E, cons
                           size_t ws_bytes, void *stream) {
     return eaga_backward_variant(d, EAGA_VARIANT_LAYER, X, E, y, M, w, saved, dXout, dEout, dX, dE, dy, dW,
                                  workspace, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------ the block around the layer
+
+static eaga_status check_block_dims(const eaga_dims *d) {
+    eaga_status s = check_dims(d);
+    if (s != EAGA_OK) return s;
+    if (!fast::supports(*d) || !fast::blk::block_supports(d->dx, d->de, d->dy)) return EAGA_ERR_UNSUPPORTED;
+    return EAGA_OK;
+}
+static size_t layer_saved_bytes(const eaga_dims &d) { return align256(saved_layout(d).saved_total); }
+
+size_t eaga_block_saved_size(const eaga_dims *d) {
+    if (check_block_dims(d) != EAGA_OK) return 0;
+    return fast::blk::block_saved_layout(d->B, d->n, d->dx, d->dy, layer_saved_bytes(*d)).total;
+}
+
+size_t eaga_block_workspace_size(const eaga_dims *d, int for_backward) {
+    if (check_block_dims(d) != EAGA_OK) return 0;
+    const size_t base = align256(eaga_workspace_size(d, for_backward ? 1 : 0));
+    return fast::blk::block_ws_layout(d->B, d->n, d->dx, d->dy, base, for_backward).total;
+}
+
+int eaga_block_kernel_launches(const eaga_dims *d, int for_backward) {
+    if (check_block_dims(d) != EAGA_OK) return -1;
+    return eaga_kernel_launches(d, for_backward) + fast::blk::block_kernel_launches(for_backward);
+}
+
+static eaga_status check_block_weights(const eaga_block_weights *wb, const void *out[27]) {
+    if (!wb) return EAGA_ERR_INVALID_ARG;
+    const void *src[27] = {wb->x_ln1_g, wb->x_ln1_s, wb->x_W1, wb->x_b1, wb->x_W2, wb->x_b2, wb->x_ln2_g,
+                           wb->x_ln2_s, wb->e_ln1_g, wb->e_ln1_s, wb->e_W1, wb->e_b1, wb->e_W2, wb->e_b2,
+                           wb->e_ln2_g, wb->e_ln2_s, wb->y_ln1_g, wb->y_ln1_s, wb->y_W1, wb->y_b1, wb->y_W2,
+                           wb->y_b2, wb->y_ln2_g, wb->y_ln2_s, wb->Wyx, wb->Wye, wb->by};
+    for (int k = 0; k < 27; ++k) {
+        if (!src[k]) return EAGA_ERR_INVALID_ARG;
+        if (!aligned16(src[k])) return EAGA_ERR_MISALIGNED;
+        out[k] = src[k];
+    }
+    return EAGA_OK;
+}
+
+eaga_status eaga_block_forward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
+                               const eaga_weights *w, const eaga_block_weights *wb, void *Xmid, void *Emid,
+                               void *Xout, void *Eout, void *yout, void *saved, void *workspace, size_t ws_bytes,
+                               void *stream) {
+    NvtxRange range("eaga_block_forward");
+    eaga_status s = check_block_dims(d);
+    if (s != EAGA_OK) return s;
+    const void *wbs[27];
+    if ((s = check_block_weights(wb, wbs)) != EAGA_OK) return s;
+    if ((s = check_ptrs({Xout, Eout, yout, saved, workspace})) != EAGA_OK) return s;
+    if (ws_bytes < eaga_block_workspace_size(d, 0)) return EAGA_ERR_WORKSPACE;
+    const fast::blk::BlockSaved S =
+        fast::blk::block_saved_layout(d->B, d->n, d->dx, d->dy, layer_saved_bytes(*d));
+    {
+        const Extents x = tensor_extents(*d);
+        const Span outs[4] = {{Xout, x.X}, {Eout, x.E}, {yout, x.y}, {saved, S.total}};
+        const Span ins[7] = {{X, x.X}, {E, x.E}, {y, x.y}, {M, x.M}, {Xmid, x.X}, {Emid, x.E},
+                             {workspace, eaga_block_workspace_size(d, 0)}};
+        if ((s = check_no_alias(outs, 4, ins, 7)) != EAGA_OK) return s;
+    }
+    const size_t base = align256(eaga_workspace_size(d, 0));
+    s = forward_impl(d, EAGA_VARIANT_LAYER, 0, -1, X, E, y, M, w, Xmid, Emid, saved, workspace, base, stream);
+    if (s != EAGA_OK) return s;
+    const fast::blk::BlockWs W = fast::blk::block_ws_layout(d->B, d->n, d->dx, d->dy, base, 0);
+    char *ws = static_cast<char *>(workspace);
+    fast::blk::TailFwd a = {};
+    a.B = d->B; a.n = d->n; a.dx = d->dx; a.dy = d->dy;
+    a.M = M; a.y = y; a.Xmid = Xmid; a.Emid = Emid; a.wb = wbs;
+    a.Xout = Xout; a.Eout = Eout; a.yout = yout;
+    a.status = reinterpret_cast<int *>(ws + ws_layout(*d).status);
+    return launch_status(
+        fast::blk::tail_forward(a, ws, W, static_cast<char *>(saved), S, static_cast<cudaStream_t>(stream)));
+}
+
+eaga_status eaga_block_backward(const eaga_dims *d, const void *X, const void *E, const void *y, const uint8_t *M,
+                                const eaga_weights *w, const eaga_block_weights *wb, const void *Xmid,
+                                const void *Emid, const void *saved, const void *dXout, const void *dEout,
+                                const void *dyout, void *dEmid, void *dX, void *dE, void *dy,
+                                const eaga_weight_grads *dW, const eaga_block_grads *dWb, void *workspace,
+                                size_t ws_bytes, void *stream) {
+    NvtxRange range("eaga_block_backward");
+    eaga_status s = check_block_dims(d);
+    if (s != EAGA_OK) return s;
+    const void *wbs[27];
+    if ((s = check_block_weights(wb, wbs)) != EAGA_OK) return s;
+    if ((s = check_ptrs({Xmid, Emid, saved, dXout, dEout, dyout, dEmid, workspace})) != EAGA_OK) return s;
+    if (!dWb) return EAGA_ERR_INVALID_ARG;
+    float *dwb[27];
+    {
+        void *src[27] = {dWb->x_ln1_g, dWb->x_ln1_s, dWb->x_W1, dWb->x_b1, dWb->x_W2, dWb->x_b2, dWb->x_ln2_g,
+                         dWb->x_ln2_s, dWb->e_ln1_g, dWb->e_ln1_s, dWb->e_W1, dWb->e_b1, dWb->e_W2, dWb->e_b2,
+                         dWb->e_ln2_g, dWb->e_ln2_s, dWb->y_ln1_g, dWb->y_ln1_s, dWb->y_W1, dWb->y_b1, dWb->y_W2,
+                         dWb->y_b2, dWb->y_ln2_g, dWb->y_ln2_s, dWb->Wyx, dWb->Wye, dWb->by};
+        for (int k = 0; k < 27; ++k) {
+            if (!src[k]) return EAGA_ERR_INVALID_ARG;
+            if (!aligned16(src[k])) return EAGA_ERR_MISALIGNED;
+            dwb[k] = static_cast<float *>(src[k]);
+        }
+    }
+    if (ws_bytes < eaga_block_workspace_size(d, 1)) return EAGA_ERR_WORKSPACE;
+    {
+        const Extents x = tensor_extents(*d);
+        const Span outs[2] = {{dEmid, x.E}, {workspace, eaga_block_workspace_size(d, 1)}};
+        const Span ins[11] = {{X, x.X}, {E, x.E}, {y, x.y}, {M, x.M}, {Xmid, x.X}, {Emid, x.E},
+                              {saved, eaga_block_saved_size(d)}, {dXout, x.X}, {dEout, x.E}, {dyout, x.y},
+                              {dE, x.E}};
+        if ((s = check_no_alias(outs, 2, ins, 11)) != EAGA_OK) return s;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t base = align256(eaga_workspace_size(d, 1));
+    const fast::blk::BlockWs W = fast::blk::block_ws_layout(d->B, d->n, d->dx, d->dy, base, 1);
+    const fast::blk::BlockSaved S =
+        fast::blk::block_saved_layout(d->B, d->n, d->dx, d->dy, layer_saved_bytes(*d));
+    char *ws = static_cast<char *>(workspace);
+    int *status = reinterpret_cast<int *>(ws + ws_layout(*d).status);
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
+    fast::blk::TailBwd a = {};
+    a.B = d->B; a.n = d->n; a.dx = d->dx; a.dy = d->dy;
+    a.M = M; a.Xmid = Xmid; a.Emid = Emid; a.dXout = dXout; a.dEout = dEout; a.dyout = dyout;
+    a.wb = wbs; a.dwb = dwb; a.dEmid = dEmid; a.status = status;
+    if ((s = launch_status(fast::blk::tail_backward(a, ws, W, static_cast<const char *>(saved), S, st))) != EAGA_OK)
+        return s;
+    s = backward_impl(d, EAGA_VARIANT_LAYER, 0, -1, X, E, y, M, w, saved, ws + W.dXmid, dEmid, dX, dE, dy, dW,
+                      workspace, base, stream, false);
+    if (s != EAGA_OK) return s;
+    return launch_status(fast::blk::add_dy(dy, reinterpret_cast<const float *>(ws + W.dy1), d->B * d->dy, st));
 }
 
 eaga_status eaga_debug_attention_map(const eaga_dims *d, const void *E, const uint8_t *M, const eaga_weights *w,

@@ -1,0 +1,814 @@
+// Edge sub-block of the graph-transformer block around the layer, fused per
+// tile of 128 pairs (sm_100a, de = 64, FFN width 128, bf16 storage).
+//
+// The layer sits in DeFoG's graph-transformer backbone, which updates node,
+// edge and global features jointly (AI-summary page, method paragraph; paper
+// index page, abstract).  The pages print no equations for the block; the
+// edge part taken here is the plain post-norm one:
+//   Ea   = LN(E'; g1, s1)
+//   Ez   = Ea + relu(Ea W1 + b1) W2 + b2
+//   Eout = valid_ij * LN(Ez; g2, s2)
+// with LN over the 64 channels of a pair (biased variance, eps 1e-5).
+//
+// k_eblk_fwd streams tiles of 4 rows i x 32 columns j (128 pairs, 16 KB) of
+// E' through shared memory: the LayerNorms run per pair in registers (thread
+// r owns pair r, TMEM lane r), the two FFN products run on the tensor cores
+// (tcgen05, M = 128, fp32 in TMEM: Ea W1 is 128 x 128 over K = 64, H W2 is
+// 128 x 64 over K = 128), and the result is written in place into the tile and
+// stored with TMA: E' is read once and Eout written once.  A tile without a
+// valid pair is not read; it is stored as zeros.  The same pass adds the valid
+// pairs' E' into per-graph sums for the global update's edge pooling.
+//
+// k_eblk_bwd recomputes the forward of a tile from E' and runs its chain rule:
+//   dEz = LN^T(valid * dEout; g2)      dg2 += dEout x2, ds2 += dEout
+//   dh  = dEz W2^T [Ea W1 + b1 > 0]    dW2 += h^T dEz,   db2 += dEz
+//   dEa = dEz + dh W1^T                dW1 += Ea^T dh,   db1 += dh
+//   dE' = valid * (LN^T(dEa; g1) + dpE_b)               dg1 += dEa x1, ds1 += dEa
+// (dpE_b: the global update's gradient of the edge pooling, already divided
+// by the pair count).  The four products and the two weight-gradient products
+// (M = 128 over the tile's 128 pairs, accumulated in TMEM over the CTA's
+// tiles) run on the tensor cores; the per-channel sums run per warp with
+// shuffles; each CTA writes its partial sums once.
+//
+// Four warps, one pair row per thread; thread 0 also issues the MMAs (after
+// a named barrier of the CTA) and the TMA loads and stores, and warp 0 computes
+// each tile's validity masks one tile ahead.  The forward double-buffers its
+// tiles (the next tile's load is issued with the current tile's first
+// product); the backward holds one tile pair and prefetches the next into L2.
+// Persistent grid, two CTAs per SM (8 warps: 255 registers a thread), tiles
+// taken in a stride of the grid size.
+#include "fast.h"
+#include "fast_common.cuh"
+#include "fast_block.h"
+
+namespace eaga {
+namespace fast {
+namespace blk {
+
+using namespace sm100;
+using dev::cta_wait;
+
+constexpr int EB_THR = 128;                   // four warps, one pair row per thread
+constexpr int EF = 128;                       // FFN width of the edge sub-block (2 de)
+constexpr uint32_t EB_TILE = 16384;           // 128 pairs x 64 channels bf16
+constexpr float LN_EPS = 1e-5f;
+
+// Forward shared memory (bytes from a 1024-aligned base).
+struct EfSmem {
+    static constexpr uint32_t SLOT = 0;                  // 2 x 16 KB: E' tile -> Ea -> output
+    static constexpr uint32_t H = 2 * EB_TILE;           // 2 x 16 KB: relu(Ea W1 + b1), channels 0..63 | 64..127
+    static constexpr uint32_t W1 = H + 2 * EB_TILE;      // W1 [64][128] as two 64 x 64 boxes (8 KB each)
+    static constexpr uint32_t W2 = W1 + EB_TILE;         // W2 [128][64] as one box
+    static constexpr uint32_t PAR = W2 + EB_TILE;        // fp32: g1, s1 [64], b1 [128], b2, g2, s2 [64]
+    static constexpr uint32_t INFO = PAR + 448 * 4;      // per slot: column mask, row mask | live << 8
+    static constexpr uint32_t BAR = INFO + 16;           // full[2], mma, wts
+    static constexpr uint32_t TM = BAR + 4 * 8;
+    static constexpr uint32_t FAIL = TM + 8;
+    static constexpr uint32_t BYTES = FAIL + 8 + 1024;
+};
+static_assert(EfSmem::BYTES <= 113 * 1024, "two CTAs per SM");
+constexpr int PAR_G1 = 0, PAR_S1 = 64, PAR_B1 = 128, PAR_B2 = 256, PAR_G2 = 320, PAR_S2 = 384;
+
+// Backward shared memory: one E' tile (-> Ea), one dEout tile (-> dEz -> dE'),
+// H (h -> dh), the weights and the parameters.
+struct EbSmem {
+    static constexpr uint32_t SA = 0;
+    static constexpr uint32_t SB = EB_TILE;
+    static constexpr uint32_t H = 2 * EB_TILE;
+    static constexpr uint32_t W1 = H + 2 * EB_TILE;
+    static constexpr uint32_t W2 = W1 + EB_TILE;
+    static constexpr uint32_t PAR = W2 + EB_TILE;
+    static constexpr uint32_t INFO = PAR + 448 * 4;
+    static constexpr uint32_t BAR = INFO + 16;           // full, mma, wts
+    static constexpr uint32_t TM = BAR + 3 * 8;
+    static constexpr uint32_t FAIL = TM + 8;
+    static constexpr uint32_t BYTES = FAIL + 8 + 1024;
+};
+static_assert(EbSmem::BYTES <= 113 * 1024, "two CTAs per SM");
+// TMEM columns of the backward: the tile's products 0..127, dW2 128..191, dW1^T 192..255
+constexpr uint32_t EB_TM_COLS = 256, EB_TM_DW2 = 128, EB_TM_DW1 = 192;
+
+// Sum over the 32 lanes of the warp of f(c) for channels c < N, by halving:
+// the first step pairs channels c and c + N/2 as they are computed, so only
+// N/2 values are live.  On return out[i] of lane l is channel (N/32) l + i.
+template <int N, class F>
+__device__ __forceinline__ void warp_colsum_of(F f, int lane, float (&out)[N / 32]) {
+    float v[N / 2];
+    const bool up = (lane & 16) != 0;
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+        const float a = f(i), b = f(i + N / 2);
+        v[i] = (up ? b : a) + __shfl_xor_sync(0xffffffffu, up ? a : b, 16);
+    }
+#pragma unroll
+    for (int s = 1; s < 5; ++s) {
+        const int o = 16 >> s, h = N >> (s + 1);
+        const bool u2 = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            const float send = u2 ? v[i] : v[i + h];
+            const float keep = u2 ? v[i + h] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < N / 32; ++i) out[i] = v[i];
+}
+
+// Tile t of the grid of (graph, 4-row block, 32-column block).
+struct TileAt {
+    int b, i0, j0;
+};
+__device__ __forceinline__ TileAt tile_at(int t, int ti, int tj) {
+    TileAt r;
+    const int per = ti * tj;
+    r.b = t / per;
+    const int rem = t - r.b * per;
+    r.i0 = (rem / tj) * 4;
+    r.j0 = (rem % tj) * 32;
+    return r;
+}
+
+// Validity masks of a tile (one warp; every lane returns both): bit jj of
+// the column mask is set when column j0 + jj is a node, bit ii of the row mask
+// when row i0 + ii is.
+__device__ __forceinline__ void tile_masks(const uint8_t *M, int n, const TileAt &T, int lane, uint32_t &cm,
+                                           uint32_t &rm) {
+    const uint8_t *mb = M + (size_t)T.b * n;
+    const bool c = T.j0 + lane < n && mb[T.j0 + lane] != 0;
+    const bool r = lane < 4 && T.i0 + lane < n && mb[T.i0 + lane] != 0;
+    cm = __ballot_sync(0xffffffffu, c);
+    rm = __ballot_sync(0xffffffffu, r) & 0xFu;
+}
+
+// Row r of a 128B-swizzled [128][64] bf16 tile <-> 64 fp32 values.
+__device__ __forceinline__ void row_load64(const uint8_t *tile, int r, float (&x)[64]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(tile + sw128(r, c));
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(h[k]);
+            x[8 * c + 2 * k] = f.x;
+            x[8 * c + 2 * k + 1] = f.y;
+        }
+    }
+}
+__device__ __forceinline__ void row_store64(uint8_t *tile, int r, const float (&x)[64]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4 u;
+        u.x = pack_bf16(x[8 * c], x[8 * c + 1]);
+        u.y = pack_bf16(x[8 * c + 2], x[8 * c + 3]);
+        u.z = pack_bf16(x[8 * c + 4], x[8 * c + 5]);
+        u.w = pack_bf16(x[8 * c + 6], x[8 * c + 7]);
+        *reinterpret_cast<uint4 *>(tile + sw128(r, c)) = u;
+    }
+}
+__device__ __forceinline__ void row_zero(uint8_t *tile, int r) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(tile + sw128(r, c)) = make_uint4(0, 0, 0, 0);
+}
+
+// x <- (x - mean) / sqrt(var + eps) over 64 values; returns 1/sqrt(var + eps).
+__device__ __forceinline__ float normalise64(float (&x)[64]) {
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) s += x[c];
+    const float mean = s * (1.f / 64.f);
+    float q = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+        x[c] -= mean;
+        q = fmaf(x[c], x[c], q);
+    }
+    const float r = rsqrtf(q * (1.f / 64.f) + LN_EPS);
+#pragma unroll
+    for (int c = 0; c < 64; ++c) x[c] *= r;
+    return r;
+}
+
+__device__ __forceinline__ void load_params(float *par, const EbParams &p, int tid, int nthr) {
+    for (int c = tid; c < 448; c += nthr) {
+        float v;
+        if (c < 64) v = __bfloat162float(p.g1[c]);
+        else if (c < 128) v = __bfloat162float(p.s1[c - 64]);
+        else if (c < 256) v = __bfloat162float(p.b1[c - 128]);
+        else if (c < 320) v = __bfloat162float(p.b2[c - 256]);
+        else if (c < 384) v = __bfloat162float(p.g2[c - 320]);
+        else v = __bfloat162float(p.s2[c - 384]);
+        par[c] = v;
+    }
+}
+
+// Issue A[128 x K] * B -> TMEM with A K-major 128B-swizzled tiles of 64
+// columns (16 KB apart) and B as the weights' boxes (MN-major: k-steps of 16
+// rows; K-major: 64-column boxes `bstep` apart).
+__device__ __forceinline__ void mma_tile(uint32_t d, uint32_t a, int ksteps, uint32_t b, bool b_mn, uint32_t bstep,
+                                         uint32_t idesc) {
+#pragma unroll 1
+    for (int kk = 0; kk < ksteps; ++kk) {
+        const uint64_t ad = smem_desc(a + (kk >> 2) * EB_TILE + (kk & 3) * 32, 16, 1024, LAYOUT_SW128);
+        const uint64_t bd = b_mn ? smem_desc(b + kk * 2048, 8192, 1024, LAYOUT_SW128)
+                                 : smem_desc(b + (kk >> 2) * bstep + (kk & 3) * 32, 16, 1024, LAYOUT_SW128);
+        mma_bf16_ss(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+// D[M = 128 channels][N = 64] (+)= A^T B over the tile's 128 pairs: A the two
+// 64-channel halves of a [128 pairs][128] tile (16 KB apart), B a [128 pairs][64]
+// tile, both read MN-major.
+__device__ __forceinline__ void mma_wgrad(uint32_t d, uint32_t a, uint32_t b, bool accumulate) {
+    const uint32_t idesc = idesc_bf16_f32_mn(128, 64);
+#pragma unroll 1
+    for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(d, smem_desc(a + kk * 2048, EB_TILE, 1024, LAYOUT_SW128),
+                    smem_desc(b + kk * 2048, 8192, 1024, LAYOUT_SW128), idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// The H epilogue of one pair row: h = relu(T + b1) for the 128 columns,
+// written as bf16 into the two 64-channel halves of the H tile; bit c of
+// `pos` records h_c > 0.
+__device__ __forceinline__ void h_epilogue(uint8_t *Ht, int r, uint32_t tl, const float *b1, uint32_t (&pos)[4]) {
+#pragma unroll
+    for (int c0 = 0; c0 < EF; c0 += 16) {
+        float v[16];
+        tmem_ld16(tl + c0, v);
+        tmem_ld_wait();
+        uint32_t bits = 0;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            v[u] = fmaxf(v[u] + b1[c0 + u], 0.f);
+            bits |= (v[u] > 0.f ? 1u : 0u) << u;
+        }
+        pos[c0 >> 5] |= bits << (c0 & 16);
+        uint8_t *half = Ht + (c0 >> 6) * EB_TILE;
+        const int ch = (c0 & 63) >> 3;
+        uint4 u0, u1;
+        u0.x = pack_bf16(v[0], v[1]); u0.y = pack_bf16(v[2], v[3]);
+        u0.z = pack_bf16(v[4], v[5]); u0.w = pack_bf16(v[6], v[7]);
+        u1.x = pack_bf16(v[8], v[9]); u1.y = pack_bf16(v[10], v[11]);
+        u1.z = pack_bf16(v[12], v[13]); u1.w = pack_bf16(v[14], v[15]);
+        *reinterpret_cast<uint4 *>(half + sw128(r, ch)) = u0;
+        *reinterpret_cast<uint4 *>(half + sw128(r, ch + 1)) = u1;
+    }
+}
+
+// ------------------------------------------------------------------ forward
+
+// Thread 0: load tile t into slot `sl` (or mark it empty when the tile has no
+// valid pair), after the bulk stores issued so far have read their tiles.
+__device__ __forceinline__ void issue_tile(int t, int ntile, uint32_t slot_addr, uint32_t full, uint32_t *info,
+                                           uint32_t cm, uint32_t rm, const CUtensorMap *map, const EbParams &p,
+                                           volatile int *fail) {
+    if (t >= ntile) return;
+    tma_store_wait_read0();
+    const bool live = cm != 0 && rm != 0;
+    info[0] = cm;
+    info[1] = rm | (live ? 0x100u : 0u);
+    if (live && !*fail) {
+        const TileAt T = tile_at(t, p.ti, p.tj);
+        mbar_expect_tx(full, EB_TILE);
+        tma_load_4d(slot_addr, map, full, 0, T.j0, T.i0, T.b);
+    } else {
+        mbar_arrive(full);
+    }
+}
+
+__global__ void __launch_bounds__(EB_THR, 2)
+k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUtensorMap tmOut,
+           const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2, EbParams p) {
+    using S = EfSmem;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
+    const uint32_t bar0 = sbase + S::BAR;
+    auto full = [&](int s) { return bar0 + 8 * s; };
+    const uint32_t mmab = bar0 + 16, wtsb = bar0 + 24;
+    uint32_t *info = reinterpret_cast<uint32_t *>(sp + S::INFO);
+    float *par = reinterpret_cast<float *>(sp + S::PAR);
+
+    if (tid == 0) {
+        mbar_init(full(0), 1);
+        mbar_init(full(1), 1);
+        mbar_init(mmab, 1);
+        mbar_init(wtsb, 1);
+        fence_mbar_init();
+        *fail = 0;
+    }
+    if (w == 0) {
+        tmem_alloc(sbase + S::TM, 128);
+        tmem_relinquish();
+    }
+    load_params(par, p, tid, EB_THR);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+    const int ntile = p.B * p.ti * p.tj, G = gridDim.x;
+    const int r = tid;                           // pair row of the tile, TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(32 * w) << 16);
+    const uint32_t idesc1 = idesc_bf16_f32(128, EF) | (1u << 16);
+    const uint32_t idesc2 = idesc_bf16_f32(128, 64) | (1u << 16);
+
+    if (w == 0 && (int)blockIdx.x < ntile) {
+        uint32_t cm, rm;
+        tile_masks(p.M, p.n, tile_at(blockIdx.x, p.ti, p.tj), lane, cm, rm);
+        if (lane == 0) {
+            mbar_expect_tx(wtsb, 2 * EB_TILE);
+            tma_load_2d(sbase + S::W1, &tmW1, wtsb, 0, 0);
+            tma_load_2d(sbase + S::W1 + 8192, &tmW1, wtsb, 64, 0);
+            tma_load_2d(sbase + S::W2, &tmW2, wtsb, 0, 0);
+            issue_tile(blockIdx.x, ntile, sbase + S::SLOT, full(0), info, cm, rm, &tmIn, p, fail);
+        }
+        __syncwarp();
+    }
+    uint32_t mph = 0;
+    bool wts_ready = false;
+    float pool[2] = {0.f, 0.f};                  // lane's channels 2 lane, 2 lane + 1 of the current graph
+    int pool_b = -1;
+    auto flush_pool = [&]() {
+        if (pool_b >= 0) {
+            atomicAdd(p.pool + (size_t)pool_b * 64 + 2 * lane, pool[0]);
+            atomicAdd(p.pool + (size_t)pool_b * 64 + 2 * lane + 1, pool[1]);
+        }
+        pool[0] = pool[1] = 0.f;
+    };
+    int k = 0;
+    for (int t = blockIdx.x; t < ntile; t += G, ++k) {
+        const int s = k & 1, tn = t + G;
+        const uint32_t slot_a = sbase + S::SLOT + s * EB_TILE, next_a = sbase + S::SLOT + (s ^ 1) * EB_TILE;
+        uint8_t *slot = sp + S::SLOT + s * EB_TILE;
+        uint32_t cmn = 0, rmn = 0;
+        if (w == 0 && tn < ntile) tile_masks(p.M, p.n, tile_at(tn, p.ti, p.tj), lane, cmn, rmn);
+        cta_wait(full(s), (k >> 1) & 1, fail, p.status);
+        const uint32_t cm = info[2 * s], rmw = info[2 * s + 1];
+        const TileAt T = tile_at(t, p.ti, p.tj);
+        const bool live = (rmw & 0x100u) != 0 && !*fail;
+        const bool valid = ((rmw >> (r >> 5)) & 1u) && ((cm >> (r & 31)) & 1u);
+        if (T.b != pool_b) {                     // warp-uniform
+            flush_pool();
+            pool_b = T.b;
+        }
+        if (!live) {
+            row_zero(slot, r);
+            fence_proxy_async_smem();
+            named_bar_sync(1, EB_THR);
+            if (r == 0) {
+                if (!*fail) {
+                    tma_store_4d(&tmOut, slot_a, 0, T.j0, T.i0, T.b);
+                    tma_store_commit();
+                }
+                issue_tile(tn, ntile, next_a, full(s ^ 1), info + 2 * (s ^ 1), cmn, rmn, &tmIn, p, fail);
+            }
+            continue;
+        }
+        if (!wts_ready) {
+            cta_wait(wtsb, 0, fail, p.status);
+            wts_ready = true;
+        }
+        float x[64];
+        row_load64(slot, r, x);
+        {
+            float ps[2];
+            warp_colsum_of<64>([&](int c) { return valid ? x[c] : 0.f; }, lane, ps);
+            pool[0] += ps[0];
+            pool[1] += ps[1];
+        }
+        normalise64(x);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[c] = fmaf(x[c], par[PAR_G1 + c], par[PAR_S1 + c]);
+        row_store64(slot, r, x);
+        fence_proxy_async_smem();
+        named_bar_sync(1, EB_THR);
+        if (r == 0) {
+            if (!*fail) {
+                tc_fence_after();
+                mma_tile(tmem, slot_a, 4, sbase + S::W1, true, 0, idesc1);
+                mma_commit(mmab);
+            }
+            issue_tile(tn, ntile, next_a, full(s ^ 1), info + 2 * (s ^ 1), cmn, rmn, &tmIn, p, fail);
+        }
+        cta_wait(mmab, mph, fail, p.status);
+        mph ^= 1u;
+        tc_fence_after();
+        uint32_t pos[4] = {0, 0, 0, 0};
+        h_epilogue(sp + S::H, r, tl, par + PAR_B1, pos);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(1, EB_THR);
+        if (r == 0 && !*fail) {
+            tc_fence_after();
+            mma_tile(tmem, sbase + S::H, 8, sbase + S::W2, true, 0, idesc2);
+            mma_commit(mmab);
+        }
+        cta_wait(mmab, mph, fail, p.status);
+        mph ^= 1u;
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+            float v[16];
+            tmem_ld16(tl + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) x[c0 + u] += v[u] + par[PAR_B2 + c0 + u];
+        }
+        normalise64(x);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[c] = valid ? fmaf(x[c], par[PAR_G2 + c], par[PAR_S2 + c]) : 0.f;
+        row_store64(slot, r, x);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(1, EB_THR);
+        if (r == 0 && !*fail) {
+            tma_store_4d(&tmOut, slot_a, 0, T.j0, T.i0, T.b);
+            tma_store_commit();
+        }
+    }
+    flush_pool();
+    if (r == 0) tma_store_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tmem, 128);
+}
+
+// ------------------------------------------------------------------ backward
+
+__global__ void __launch_bounds__(EB_THR, 2)
+k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUtensorMap tmDOut,
+           const __grid_constant__ CUtensorMap tmDIn, const __grid_constant__ CUtensorMap tmW1,
+           const __grid_constant__ CUtensorMap tmW2, EbParams p) {
+    using S = EbSmem;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    volatile int *fail = reinterpret_cast<volatile int *>(sp + S::FAIL);
+    const uint32_t bar0 = sbase + S::BAR;
+    const uint32_t fullb = bar0, mmab = bar0 + 8, wtsb = bar0 + 16;
+    uint32_t *info = reinterpret_cast<uint32_t *>(sp + S::INFO);
+    float *par = reinterpret_cast<float *>(sp + S::PAR);
+
+    if (tid == 0) {
+        mbar_init(fullb, 1);
+        mbar_init(mmab, 1);
+        mbar_init(wtsb, 1);
+        fence_mbar_init();
+        *fail = 0;
+    }
+    if (w == 0) {
+        tmem_alloc(sbase + S::TM, EB_TM_COLS);
+        tmem_relinquish();
+    }
+    load_params(par, p, tid, EB_THR);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + S::TM);
+    const int ntile = p.B * p.ti * p.tj, G = gridDim.x;
+    const int r = tid;
+    const uint32_t tl = tmem + ((uint32_t)(32 * w) << 16);
+    const uint32_t idesc_h = idesc_bf16_f32(128, EF) | (1u << 16);    // Ea W1: B MN-major
+    const uint32_t idesc_z = idesc_bf16_f32(128, 64) | (1u << 16);    // h W2: B MN-major
+    const uint32_t idesc_dh = idesc_bf16_f32(128, EF);                // dEz W2^T: B K-major
+    const uint32_t idesc_da = idesc_bf16_f32(128, 64);                // dh W1^T: B K-major
+
+    // thread 0: the loads of tile t (E' and dEout) and an L2 prefetch of the CTA's next tile
+    auto issue = [&](int t, uint32_t cm, uint32_t rm) {
+        if (t >= ntile) return;
+        tma_store_wait_read0();
+        const bool live = cm != 0 && rm != 0;
+        info[0] = cm;
+        info[1] = rm | (live ? 0x100u : 0u);
+        if (live && !*fail) {
+            const TileAt T = tile_at(t, p.ti, p.tj);
+            mbar_expect_tx(fullb, 2 * EB_TILE);
+            tma_load_4d(sbase + S::SA, &tmIn, fullb, 0, T.j0, T.i0, T.b);
+            tma_load_4d(sbase + S::SB, &tmDOut, fullb, 0, T.j0, T.i0, T.b);
+            if (t + G < ntile) {
+                const TileAt N = tile_at(t + G, p.ti, p.tj);
+                tma_prefetch_4d(&tmIn, 0, N.j0, N.i0, N.b);
+                tma_prefetch_4d(&tmDOut, 0, N.j0, N.i0, N.b);
+            }
+        } else {
+            mbar_arrive(fullb);
+        }
+    };
+    if (w == 0 && (int)blockIdx.x < ntile) {
+        uint32_t cm, rm;
+        tile_masks(p.M, p.n, tile_at(blockIdx.x, p.ti, p.tj), lane, cm, rm);
+        if (lane == 0) {
+            mbar_expect_tx(wtsb, 2 * EB_TILE);
+            tma_load_2d(sbase + S::W1, &tmW1, wtsb, 0, 0);
+            tma_load_2d(sbase + S::W1 + 8192, &tmW1, wtsb, 64, 0);
+            tma_load_2d(sbase + S::W2, &tmW2, wtsb, 0, 0);
+            issue(blockIdx.x, cm, rm);
+        }
+        __syncwarp();
+    }
+    uint32_t mph = 0;
+    bool wts_ready = false, any = false;
+    // per-lane channel sums: channels 2l, 2l+1 of dg2, ds2, db2, dg1, ds1 and 4l .. 4l+3 of db1
+    float acc[14];
+#pragma unroll
+    for (int u = 0; u < 14; ++u) acc[u] = 0.f;
+    uint8_t *sa = sp + S::SA, *sb = sp + S::SB;
+    int k = 0;
+    for (int t = blockIdx.x; t < ntile; t += G, ++k) {
+        const int tn = t + G;
+        cta_wait(fullb, k & 1, fail, p.status);
+        const uint32_t cm = info[0], rmw = info[1];
+        const TileAt T = tile_at(t, p.ti, p.tj);
+        const bool live = (rmw & 0x100u) != 0 && !*fail;
+        const bool valid = ((rmw >> (r >> 5)) & 1u) && ((cm >> (r & 31)) & 1u);
+        if (live) {
+            if (!wts_ready) {
+                cta_wait(wtsb, 0, fail, p.status);
+                wts_ready = true;
+            }
+            // LN1 recomputed: x1 = normalised E', Ea = x1 g1 + s1
+            float x1[64], z[64], d[64];
+            row_load64(sa, r, x1);
+            const float r1 = normalise64(x1);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) z[c] = fmaf(x1[c], par[PAR_G1 + c], par[PAR_S1 + c]);
+            row_store64(sa, r, z);
+            fence_proxy_async_smem();
+            named_bar_sync(1, EB_THR);
+            if (r == 0 && !*fail) {
+                tc_fence_after();
+                mma_tile(tmem, sbase + S::SA, 4, sbase + S::W1, true, 0, idesc_h);
+                mma_commit(mmab);
+            }
+            cta_wait(mmab, mph, fail, p.status);
+            mph ^= 1u;
+            tc_fence_after();
+            uint32_t pos[4] = {0, 0, 0, 0};
+            h_epilogue(sp + S::H, r, tl, par + PAR_B1, pos);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(1, EB_THR);
+            if (r == 0 && !*fail) {
+                tc_fence_after();
+                mma_tile(tmem, sbase + S::H, 8, sbase + S::W2, true, 0, idesc_z);
+                mma_commit(mmab);
+            }
+            cta_wait(mmab, mph, fail, p.status);
+            mph ^= 1u;
+            tc_fence_after();
+            // Ez = Ea + h W2 + b2 (z holds Ea), normalised in place (x2)
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+                float v[16];
+                tmem_ld16(tl + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) z[c0 + u] += v[u] + par[PAR_B2 + c0 + u];
+            }
+            const float r2 = normalise64(z);
+            // upstream gradient, masked: dg2, ds2; LN2's input gradient dEz
+            row_load64(sb, r, d);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) d[c] = valid ? d[c] : 0.f;
+            {
+                float o[2];
+                warp_colsum_of<64>([&](int c) { return d[c] * z[c]; }, lane, o);
+                acc[0] += o[0];
+                acc[1] += o[1];
+                warp_colsum_of<64>([&](int c) { return d[c]; }, lane, o);
+                acc[2] += o[0];
+                acc[3] += o[1];
+            }
+            float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                d[c] *= par[PAR_G2 + c];
+                m1 += d[c];
+                m2 = fmaf(d[c], z[c], m2);
+            }
+            m1 *= (1.f / 64.f);
+            m2 *= (1.f / 64.f);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) d[c] = r2 * (d[c] - m1 - z[c] * m2);     // dEz
+            row_store64(sb, r, d);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(1, EB_THR);
+            if (r == 0 && !*fail) {
+                tc_fence_after();
+                // dh' = dEz W2^T (B = W2 read K-major: [N = 128][K = 64]); dW2 += h^T dEz
+                mma_tile(tmem, sbase + S::SB, 4, sbase + S::W2, false, 0, idesc_dh);
+                mma_wgrad(tmem + EB_TM_DW2, sbase + S::H, sbase + S::SB, any);
+                mma_commit(mmab);
+            }
+            {
+                float o[2];
+                warp_colsum_of<64>([&](int c) { return d[c]; }, lane, o);
+                acc[4] += o[0];
+                acc[5] += o[1];
+            }
+            cta_wait(mmab, mph, fail, p.status);
+            mph ^= 1u;
+            tc_fence_after();
+            // dh = dh' [h > 0] into the H tile (h is no longer read); db1 by halving,
+            // channels c and c + 64 together
+            {
+                float v1[64];
+                const bool up = (lane & 16) != 0;
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 16) {
+                    float va[16], vb[16];
+                    tmem_ld16(tl + c0, va);
+                    tmem_ld16(tl + c0 + 64, vb);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int ca = c0 + u, cb = c0 + 64 + u;
+                        va[u] = ((pos[ca >> 5] >> (ca & 31)) & 1u) ? va[u] : 0.f;
+                        vb[u] = ((pos[cb >> 5] >> (cb & 31)) & 1u) ? vb[u] : 0.f;
+                    }
+                    const int ch = c0 >> 3;
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const float *v = hf ? vb : va;
+                        uint8_t *half = sp + S::H + hf * EB_TILE;
+                        uint4 u0, u1;
+                        u0.x = pack_bf16(v[0], v[1]); u0.y = pack_bf16(v[2], v[3]);
+                        u0.z = pack_bf16(v[4], v[5]); u0.w = pack_bf16(v[6], v[7]);
+                        u1.x = pack_bf16(v[8], v[9]); u1.y = pack_bf16(v[10], v[11]);
+                        u1.z = pack_bf16(v[12], v[13]); u1.w = pack_bf16(v[14], v[15]);
+                        *reinterpret_cast<uint4 *>(half + sw128(r, ch)) = u0;
+                        *reinterpret_cast<uint4 *>(half + sw128(r, ch + 1)) = u1;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        v1[c0 + u] = (up ? vb[u] : va[u]) + __shfl_xor_sync(0xffffffffu, up ? va[u] : vb[u], 16);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(1, EB_THR);
+                if (r == 0 && !*fail) {
+                    tc_fence_after();
+                    // dEa' = dh W1^T (B = W1 read K-major: [N = 64][K = 128], two 64-column boxes);
+                    // dW1^T += dh^T Ea
+                    mma_tile(tmem, sbase + S::H, 8, sbase + S::W1, false, 8192, idesc_da);
+                    mma_wgrad(tmem + EB_TM_DW1, sbase + S::H, sbase + S::SA, any);
+                    mma_commit(mmab);
+                }
+#pragma unroll
+                for (int st = 1; st < 5; ++st) {
+                    const int o = 16 >> st, h = 128 >> (st + 1);
+                    const bool u2 = (lane & o) != 0;
+#pragma unroll
+                    for (int i = 0; i < h; ++i) {
+                        const float send = u2 ? v1[i] : v1[i + h];
+                        const float keep = u2 ? v1[i + h] : v1[i];
+                        v1[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[10 + u] += v1[u];
+            }
+            any = true;
+            cta_wait(mmab, mph, fail, p.status);
+            mph ^= 1u;
+            tc_fence_after();
+            // dEa = dEz + dh W1^T (d holds dEz); dg1, ds1; dE' = valid (LN1^T(dEa) + dpE_b)
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+                float v[16];
+                tmem_ld16(tl + c0, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int u = 0; u < 16; ++u) d[c0 + u] += v[u];
+            }
+            {
+                float o[2];
+                warp_colsum_of<64>([&](int c) { return d[c] * x1[c]; }, lane, o);
+                acc[6] += o[0];
+                acc[7] += o[1];
+                warp_colsum_of<64>([&](int c) { return d[c]; }, lane, o);
+                acc[8] += o[0];
+                acc[9] += o[1];
+            }
+            float n1 = 0.f, n2 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                d[c] *= par[PAR_G1 + c];
+                n1 += d[c];
+                n2 = fmaf(d[c], x1[c], n2);
+            }
+            n1 *= (1.f / 64.f);
+            n2 *= (1.f / 64.f);
+            const float4 *dp = reinterpret_cast<const float4 *>(p.dpool + (size_t)T.b * 64);
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 q = __ldg(dp + c4);
+                const float qa[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = 4 * c4 + u;
+                    d[c] = valid ? r1 * (d[c] - n1 - x1[c] * n2) + qa[u] : 0.f;
+                }
+            }
+            row_store64(sb, r, d);
+        } else {
+            row_zero(sb, r);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(1, EB_THR);
+        if (w == 0) {
+            uint32_t cmn = 0, rmn = 0;
+            if (tn < ntile) tile_masks(p.M, p.n, tile_at(tn, p.ti, p.tj), lane, cmn, rmn);
+            if (lane == 0) {
+                if (!*fail) {
+                    tma_store_4d(&tmDIn, sbase + S::SB, 0, T.j0, T.i0, T.b);
+                    tma_store_commit();
+                }
+                issue(tn, cmn, rmn);
+            }
+            __syncwarp();
+        }
+    }
+    // per-warp partial sums: [CTA][warp][448] in the order dg2, ds2, db2, dg1, ds1, db1
+    float *pw = p.parts + ((size_t)blockIdx.x * 4 + w) * EB_PART;
+#pragma unroll
+    for (int q = 0; q < 5; ++q) {
+        pw[64 * q + 2 * lane] = acc[2 * q];
+        pw[64 * q + 2 * lane + 1] = acc[2 * q + 1];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) pw[320 + 4 * lane + u] = acc[10 + u];
+    // the CTA's dW2 [128][64] and dW1^T [128][64] from TMEM (zero without a live
+    // tile); every product was waited for in the loop
+    tc_fence_after();
+    float *pwt = p.wparts + (size_t)blockIdx.x * 2 * EF * 64;
+#pragma unroll 1
+    for (int m = 0; m < 2; ++m) {
+        float *dst = pwt + (size_t)m * EF * 64 + (size_t)r * 64;
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+            float v[16];
+            tmem_ld16(tl + (m == 0 ? EB_TM_DW2 : EB_TM_DW1) + c0, v);
+            tmem_ld_wait();
+            float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                d4[u] = any ? make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3])
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    if (r == 0) tma_store_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tmem, EB_TM_COLS);
+}
+
+// ------------------------------------------------------------------ host
+
+static int grid_ctas(int ntile) {
+    const int g = 2 * sm_count();
+    return ntile < g ? ntile : g;
+}
+
+cudaError_t edge_forward(const EdgeArgs &a, cudaStream_t st) {
+    CUtensorMap tIn, tOut, tW1, tW2;
+    if (!encode_tile_map(&tIn, a.Ein, a.B, a.n) || !encode_tile_map(&tOut, a.Eout, a.B, a.n) ||
+        !encode_2d(&tW1, a.W1, 64, EF, 64) || !encode_2d(&tW2, a.W2, EF, 64, EF))
+        return cudaErrorInvalidValue;
+    EbParams p = a.par;
+    p.ti = (a.n + 3) / 4;
+    p.tj = (a.n + 31) / 32;
+    const int ntile = a.B * p.ti * p.tj;
+    static std::atomic<uint32_t> attr{0};
+    if (cudaError_t e = ensure_smem_attr(k_eblk_fwd, EfSmem::BYTES, attr); e != cudaSuccess) return e;
+    k_eblk_fwd<<<grid_ctas(ntile), EB_THR, EfSmem::BYTES, st>>>(tIn, tOut, tW1, tW2, p);
+    return cudaGetLastError();
+}
+
+int edge_backward_ctas(int B, int n) {
+    return grid_ctas(B * ((n + 3) / 4) * ((n + 31) / 32));
+}
+
+cudaError_t edge_backward(const EdgeArgs &a, cudaStream_t st) {
+    CUtensorMap tIn, tDOut, tDIn, tW1, tW2;
+    if (!encode_tile_map(&tIn, a.Ein, a.B, a.n) || !encode_tile_map(&tDOut, a.dEout, a.B, a.n) ||
+        !encode_tile_map(&tDIn, a.dEin, a.B, a.n) || !encode_2d(&tW1, a.W1, 64, EF, 64) ||
+        !encode_2d(&tW2, a.W2, EF, 64, EF))
+        return cudaErrorInvalidValue;
+    EbParams p = a.par;
+    p.ti = (a.n + 3) / 4;
+    p.tj = (a.n + 31) / 32;
+    const int ntile = a.B * p.ti * p.tj;
+    static std::atomic<uint32_t> attr{0};
+    if (cudaError_t e = ensure_smem_attr(k_eblk_bwd, EbSmem::BYTES, attr); e != cudaSuccess) return e;
+    k_eblk_bwd<<<grid_ctas(ntile), EB_THR, EbSmem::BYTES, st>>>(tIn, tDOut, tDIn, tW1, tW2, p);
+    return cudaGetLastError();
+}
+
+}  // namespace blk
+}  // namespace fast
+}  // namespace eaga

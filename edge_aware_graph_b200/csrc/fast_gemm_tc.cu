@@ -7,6 +7,10 @@
 //   out-proj X' = X + M (O Wo + bo)                         (B = Wo, MN-major)
 //   dO       dO = M (dX' Wo^T)                              (Bt = Wo)
 //   dX       dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T          (three segments, Bt = W)
+// and the node FFN of the graph-transformer block around the layer:
+//   FFN1     H = relu(A W1 + b1)                             (B = W1, MN-major)
+//   FFN2     Z = R + H W2 + b2                               (B = W2, MN-major)
+//   DRELU    dH = (dZ W2^T) [R > 0]   (R = H)                (Bt = W2)
 // One thread issues TMA and MMAs; the four warps run the epilogue from TMEM.
 // k_tc_wgrad computes the weight gradients A^T B over node rows (split-K fp32
 // partials) with both operands read MN-major straight from the row-major
@@ -23,13 +27,13 @@ using dev::cta_wait;
 constexpr int TBM = 128, TBK = 64, TTHR = 128;
 // pipeline stages: 4 for 64-wide tiles, 3 for 128-wide (two CTAs fit an SM either way)
 template <int BN> constexpr int tc_stages() { return BN == 128 ? 3 : 4; }
-enum TcMode { TC_QKV = 0, TC_OUT = 1, TC_DO = 2, TC_DX = 3 };
+enum TcMode { TC_QKV = 0, TC_OUT = 1, TC_DO = 2, TC_DX = 3, TC_FFN1 = 4, TC_FFN2 = 5, TC_DRELU = 6 };
 
 struct TcParams {
     const __nv_bfloat16 *bias[3];
     __nv_bfloat16 *C[3];
     const __nv_bfloat16 *R;      // residual [M, Nb]
-    const uint8_t *mask;         // [M]
+    const uint8_t *mask;         // [M] (QKV, OUT, DO)
     int *status;
     int M, K, Nb, nseg, mode;
     int b_mn;                    // B stored [K, N] (MN-major), map chosen by output matrix
@@ -80,7 +84,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
         tmem_relinquish();
     }
     float *sbias = reinterpret_cast<float *>(sp + S::BIAS);
-    const bool has_bias = p.mode == TC_QKV || p.mode == TC_OUT;
+    const bool has_bias = p.mode == TC_QKV || p.mode == TC_OUT || p.mode == TC_FFN1 || p.mode == TC_FFN2;
     for (int c = tid; c < BN; c += TTHR) {
         const int ng = n0 + c;
         sbias[c] = has_bias ? __bfloat162float(p.bias[ng / p.Nb][ng % p.Nb]) : 0.f;
@@ -139,8 +143,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
     // loaded into registers before the accumulator is ready.
     const int row = m0 + 32 * w + t;
     const bool in = row < p.M;
-    const bool mk = in && p.mask[in ? row : 0] != 0;
-    const bool has_res = p.mode == TC_OUT || p.mode == TC_DX;
+    const bool mk = in && (p.mask == nullptr || p.mask[in ? row : 0] != 0);
+    const bool has_res = p.mode == TC_OUT || p.mode == TC_DX || p.mode == TC_FFN2 || p.mode == TC_DRELU;
     const int which0 = n0 / p.Nb, col0 = n0 % p.Nb;     // BN divides Nb: one output per tile
     const size_t obase = (size_t)(in ? row : 0) * p.Nb + col0;
     uint4 res[BN / 8];
@@ -163,8 +167,18 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 o2[u] = mk ? __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]) : __floats2bfloat162_rn(0.f, 0.f);
+        } else if (p.mode == TC_FFN1) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) o2[u] = __floats2bfloat162_rn(fmaxf(v[2 * u], 0.f), fmaxf(v[2 * u + 1], 0.f));
+        } else if (p.mode == TC_DRELU) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint4 r4 = res[c0 / 8 + (u >> 2)];
+                const float2 h = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162 *>(&r4)[u & 3]);
+                o2[u] = __floats2bfloat162_rn(h.x > 0.f ? v[2 * u] : 0.f, h.y > 0.f ? v[2 * u + 1] : 0.f);
+            }
         } else {
-            const bool add = p.mode == TC_DX || mk;
+            const bool add = p.mode == TC_DX || p.mode == TC_FFN2 || mk;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const uint4 r4 = res[c0 / 8 + (u >> 2)];

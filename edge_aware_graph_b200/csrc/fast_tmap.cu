@@ -71,6 +71,21 @@ bool encode_2d(CUtensorMap *m, const void *base, int rows, int cols, int box_row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A [B, n, n, 64] bf16 pair tensor as 4-D (c, j, i, b) with a box of 4 rows i
+// x 32 columns j (128 pairs, landing as [i 4][j 32][c 64], 128B-swizzled).
+bool encode_tile_map(CUtensorMap *m, const void *base, int B, int n) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t rowb = DE * 2;
+    const cuuint64_t dims[4] = {DE, (cuuint64_t)n, (cuuint64_t)n, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {rowb, (cuuint64_t)n * rowb, (cuuint64_t)n * n * rowb};
+    const cuuint32_t box[4] = {64, 32, 4, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // g_b = y_b Wfy + bf (fp32) for every graph: one warp per graph, lanes split
 // the dy terms and add their 16 sums with shuffles in a fixed order.  The last
 // block writes the four operand images from Wfe and We staged in shared memory

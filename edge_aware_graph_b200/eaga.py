@@ -22,7 +22,12 @@ STATUS = {0: "EAGA_OK", 1: "EAGA_ERR_INVALID_ARG", 2: "EAGA_ERR_UNSUPPORTED", 3:
 EXPORTED = ("eaga_workspace_size", "eaga_saved_size", "eaga_forward", "eaga_backward",
             "eaga_debug_attention_map", "eaga_get_device_status", "eaga_strerror",
             "eaga_set_profile_events", "eaga_kernel_launches", "eaga_forward_noalloc", "eaga_debug_wait_probe",
-            "eaga_forward_variant", "eaga_backward_variant", "eaga_forward_rows", "eaga_backward_rows")
+            "eaga_forward_variant", "eaga_backward_variant", "eaga_forward_rows", "eaga_backward_rows",
+            "eaga_block_saved_size", "eaga_block_workspace_size", "eaga_block_kernel_launches",
+            "eaga_block_forward", "eaga_block_backward")
+# parameters of the graph-transformer block (eaga_block_weights field order)
+BLOCK_SUB_PARAMS = ("ln1_g", "ln1_s", "W1", "b1", "W2", "b2", "ln2_g", "ln2_s")
+BLOCK_WEIGHT_NAMES = tuple(f"{s}_{k}" for s in ("x", "e", "y") for k in BLOCK_SUB_PARAMS) + ("Wyx", "Wye", "by")
 # layer variants (eaga_variant): the layer, Light Edge, the unnormalised edge update
 VARIANTS = {"layer": 0, "light_edge": 1, "unnormalised": 2}
 
@@ -33,6 +38,10 @@ class Dims(ctypes.Structure):
 
 class Weights(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in WEIGHT_NAMES]
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in BLOCK_WEIGHT_NAMES]
 
 
 class EagaError(RuntimeError):
@@ -88,6 +97,19 @@ def lib():
         L.eaga_set_profile_events.restype = i32
         L.eaga_kernel_launches.argtypes = [ctypes.POINTER(Dims), i32]
         L.eaga_kernel_launches.restype = i32
+        L.eaga_block_saved_size.argtypes = [ctypes.POINTER(Dims)]
+        L.eaga_block_saved_size.restype = sz
+        L.eaga_block_workspace_size.argtypes = [ctypes.POINTER(Dims), i32]
+        L.eaga_block_workspace_size.restype = sz
+        L.eaga_block_kernel_launches.argtypes = [ctypes.POINTER(Dims), i32]
+        L.eaga_block_kernel_launches.restype = i32
+        W_, BW_ = ctypes.POINTER(Weights), ctypes.POINTER(BlockWeights)
+        L.eaga_block_forward.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, W_, BW_, vp, vp, vp, vp, vp, vp,
+                                         vp, sz, vp]
+        L.eaga_block_forward.restype = i32
+        L.eaga_block_backward.argtypes = [ctypes.POINTER(Dims), vp, vp, vp, vp, W_, BW_, vp, vp, vp, vp, vp, vp,
+                                          vp, vp, vp, vp, W_, BW_, vp, sz, vp]
+        L.eaga_block_backward.restype = i32
         L.eaga_strerror.argtypes = [i32]
         L.eaga_strerror.restype = ctypes.c_char_p
         _lib = L
@@ -257,3 +279,47 @@ def kernel_launches(d: Dims, for_backward: bool) -> int:
 
 def strerror(code: int) -> str:
     return lib().eaga_strerror(int(code)).decode()
+
+
+# ---------------------------------------------------------------- the block around the layer
+
+def _block_weights(Wb: dict, dtype=None, what="Wb") -> BlockWeights:
+    return BlockWeights(*(_p(Wb[k], f"{what}[{k}]", dtype).value for k in BLOCK_WEIGHT_NAMES))
+
+
+def block_saved_size(d: Dims) -> int:
+    return int(lib().eaga_block_saved_size(ctypes.byref(d)))
+
+
+def block_workspace_size(d: Dims, for_backward: bool) -> int:
+    return int(lib().eaga_block_workspace_size(ctypes.byref(d), int(bool(for_backward))))
+
+
+def block_kernel_launches(d: Dims, for_backward: bool) -> int:
+    return int(lib().eaga_block_kernel_launches(ctypes.byref(d), int(bool(for_backward))))
+
+
+def block_forward(d: Dims, X, E, y, M, W: dict, Wb: dict, Xmid, Emid, Xout, Eout, yout, saved, workspace,
+                  stream=None):
+    """eaga_block_forward."""
+    sd = _storage(d)
+    rc = lib().eaga_block_forward(
+        ctypes.byref(d), _p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd), _p(M, "M", _u8()),
+        ctypes.byref(_weights(W, sd)), ctypes.byref(_block_weights(Wb, sd)), _p(Xmid, "Xmid", sd),
+        _p(Emid, "Emid", sd), _p(Xout, "Xout", sd), _p(Eout, "Eout", sd), _p(yout, "yout", sd),
+        _p(saved, "saved"), _p(workspace, "workspace"), _nbytes(workspace), _stream(stream))
+    _check(rc, "eaga_block_forward")
+
+
+def block_backward(d: Dims, X, E, y, M, W: dict, Wb: dict, Xmid, Emid, saved, dXout, dEout, dyout, dEmid,
+                   dX, dE, dy, dW: dict, dWb: dict, workspace, stream=None):
+    """eaga_block_backward."""
+    sd = _storage(d)
+    rc = lib().eaga_block_backward(
+        ctypes.byref(d), _p(X, "X", sd), _p(E, "E", sd), _p(y, "y", sd), _p(M, "M", _u8()),
+        ctypes.byref(_weights(W, sd)), ctypes.byref(_block_weights(Wb, sd)), _p(Xmid, "Xmid", sd),
+        _p(Emid, "Emid", sd), _p(saved, "saved"), _p(dXout, "dXout", sd), _p(dEout, "dEout", sd),
+        _p(dyout, "dyout", sd), _p(dEmid, "dEmid", sd), _p(dX, "dX", sd), _p(dE, "dE", sd), _p(dy, "dy", sd),
+        ctypes.byref(_weights(dW, _f32(), "dW")), ctypes.byref(_block_weights(dWb, _f32(), "dWb")),
+        _p(workspace, "workspace"), _nbytes(workspace), _stream(stream))
+    _check(rc, "eaga_block_backward")

@@ -280,6 +280,86 @@ EAGA_API int eaga_kernel_launches(const eaga_dims *dims, int for_backward);
 EAGA_API eaga_status eaga_debug_wait_probe(void *workspace, unsigned limit, void *stream);
 
 /* Static, human-readable name of a status code. */
+/* ---------------------------------------------------------------------
+ * The graph-transformer block around the layer.  The pages place the layer
+ * inside DeFoG's graph-transformer backbone, which updates node, edge and
+ * global features jointly (AI-summary page, method paragraph; paper index
+ * page, abstract), but print none of the block's equations; this library's
+ * reading is the plain post-norm block (LN over the last axis, biased
+ * variance, eps 1e-5; relu; cnt_b = sum_i M_bi; valid as above):
+ *
+ *   (X', E') = the layer above on (X, E, y, M)
+ *   pX_b = sum_i M_bi X'_bi / max(cnt_b, 1)
+ *   pE_b = sum_ij valid_bij E'_bij / max(cnt_b^2, 1)
+ *   y1_b = y_b + pX_b Wyx + pE_b Wye + by
+ *   for Z in (X', E', y1):  Za = LN(Z; ln1_g, ln1_s)
+ *                           Zz = Za + relu(Za W1 + b1) W2 + b2
+ *                           Zo = LN(Zz; ln2_g, ln2_s)
+ *   Xout = M Xo,  Eout = valid Eo,  yout = yo
+ *
+ * Parameters per sub-block (x: node, e: edge, y: global), [in, out]:
+ * ln1_g, ln1_s [w]; W1 [w, 2w]; b1 [2w]; W2 [2w, w]; b2 [w]; ln2_g, ln2_s [w]
+ * with w = dx, de, dy; then Wyx [dx, dy], Wye [de, dy], by [dy].  Storage
+ * dtype as the layer's weights; gradients fp32.
+ *
+ * Supported on the specialised bf16 path only (de = 64, H = 8, dh = 32, n
+ * even) with dx = 256 or 512 and dy a multiple of 32 up to 256; other dims
+ * return EAGA_ERR_UNSUPPORTED.  A stack of blocks calls these once per block
+ * with each block's own weights, feeding Xout, Eout, yout on.
+ * --------------------------------------------------------------------- */
+typedef struct {
+    const void *x_ln1_g, *x_ln1_s, *x_W1, *x_b1, *x_W2, *x_b2, *x_ln2_g, *x_ln2_s;
+    const void *e_ln1_g, *e_ln1_s, *e_W1, *e_b1, *e_W2, *e_b2, *e_ln2_g, *e_ln2_s;
+    const void *y_ln1_g, *y_ln1_s, *y_W1, *y_b1, *y_W2, *y_b2, *y_ln2_g, *y_ln2_s;
+    const void *Wyx, *Wye, *by;
+} eaga_block_weights;
+
+/* fp32 gradients of the block's parameters, same shapes; overwritten. */
+typedef struct {
+    void *x_ln1_g, *x_ln1_s, *x_W1, *x_b1, *x_W2, *x_b2, *x_ln2_g, *x_ln2_s;
+    void *e_ln1_g, *e_ln1_s, *e_W1, *e_b1, *e_W2, *e_b2, *e_ln2_g, *e_ln2_s;
+    void *y_ln1_g, *y_ln1_s, *y_W1, *y_b1, *y_W2, *y_b2, *y_ln2_g, *y_ln2_s;
+    void *Wyx, *Wye, *by;
+} eaga_block_grads;
+
+/* Bytes of the block's saved state: the layer's (eaga_saved_size, first),
+ * then the node sub-block's Za, relu(Za W1 + b1), Zz [B,n,dx|2dx|dx] and y1,
+ * pX, pE per graph (fp32).  O(B n dx), no per-pair term.  0 if unsupported. */
+EAGA_API size_t eaga_block_saved_size(const eaga_dims *dims);
+/* Workspace bytes of eaga_block_forward (0) or eaga_block_backward (1): the
+ * layer's workspace, then the block's node-sized buffers and fixed-size
+ * partial sums.  No per-pair term.  0 if unsupported. */
+EAGA_API size_t eaga_block_workspace_size(const eaga_dims *dims, int for_backward);
+/* Kernels one block call launches (the layer's included); -1 if unsupported. */
+EAGA_API int eaga_block_kernel_launches(const eaga_dims *dims, int for_backward);
+
+/* Forward of one block.  Writes the layer's outputs Xmid (X') and Emid (E'),
+ * the block's outputs Xout, Eout [B,n,n,de], yout [B,dy] and `saved`
+ * (eaga_block_saved_size bytes), which eaga_block_backward reads together
+ * with Xmid and Emid.  Same conventions as eaga_forward; the outputs and
+ * `saved` must not overlap the inputs, Xmid, Emid or the workspace. */
+EAGA_API eaga_status eaga_block_forward(const eaga_dims *dims,
+                                const void *X, const void *E, const void *y, const uint8_t *M,
+                                const eaga_weights *w, const eaga_block_weights *wb,
+                                void *Xmid, void *Emid, void *Xout, void *Eout, void *yout, void *saved,
+                                void *workspace, size_t ws_bytes, void *stream);
+
+/* Backward of one block: given the forward's inputs, Xmid, Emid, `saved` and
+ * the upstream gradients dXout, dEout, dyout, writes dX, dE, dy, the layer's
+ * weight gradients dW and the block's dWb.  dEmid [B,n,n,de] (storage dtype)
+ * is caller-provided scratch that receives dE' (the gradient at the layer's
+ * edge output); it must not overlap anything else.  Sums over rows and pairs
+ * run in a fixed order except the layer's key/value gradients and the
+ * block's edge pooling sums, whose fp32 additions follow the order the
+ * CTAs run (see eaga_backward). */
+EAGA_API eaga_status eaga_block_backward(const eaga_dims *dims,
+                                 const void *X, const void *E, const void *y, const uint8_t *M,
+                                 const eaga_weights *w, const eaga_block_weights *wb,
+                                 const void *Xmid, const void *Emid, const void *saved,
+                                 const void *dXout, const void *dEout, const void *dyout, void *dEmid,
+                                 void *dX, void *dE, void *dy, const eaga_weight_grads *dW,
+                                 const eaga_block_grads *dWb, void *workspace, size_t ws_bytes, void *stream);
+
 EAGA_API const char *eaga_strerror(eaga_status s);
 
 #ifdef __cplusplus

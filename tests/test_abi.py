@@ -67,6 +67,27 @@ def test_sizes(L):
         assert w2 <= 2.05 * w1, n
 
 
+def test_block_sizes(L):
+    """The graph-transformer block's saved state and workspaces grow with the
+    node count only: the second difference over n = 256, 512, 768 at fixed B
+    (a per-pair term c B n^2 would leave 2 c B 256^2 there) is alignment only."""
+    f = lambda n, fb: eaga.block_workspace_size(eaga.dims(4, n, 256, 64, 64, 8, 32, "bf16"), fb)
+    s = lambda n: eaga.block_saved_size(eaga.dims(4, n, 256, 64, 64, 8, 32, "bf16"))
+    for g in (lambda n: f(n, False), lambda n: f(n, True), s):
+        a, b, c = g(256), g(512), g(768)
+        assert a > 0 and b > a and c > b
+        assert abs(c - 2 * b + a) < 64 * 1024
+    d = good_dims()
+    assert eaga.block_saved_size(d) > eaga.saved_size(d)
+    assert eaga.block_workspace_size(d, True) > eaga.workspace_size(d, True)
+    # unsupported: fp32, de != 64, dx not 256 or 512, dy not a multiple of 32
+    for bad in (eaga.dims(2, 16, 16, 8, 8, 2, 8, "fp32"), eaga.dims(4, 64, 128, 64, 64, 8, 32, "bf16"),
+                eaga.dims(4, 64, 256, 64, 48, 8, 32, "bf16")):
+        assert eaga.block_workspace_size(bad, False) == 0 and eaga.block_saved_size(bad) == 0
+        assert eaga.block_kernel_launches(bad, True) == -1
+    assert eaga.block_kernel_launches(d, False) > eaga.kernel_launches(d, False)
+
+
 @pytest.mark.parametrize("field,value,code", [
     ("n", 0, 1), ("B", -1, 1), ("dtype", 7, 1),
     ("n", 1025, 2), ("de", 12, 2), ("dh", 12, 2), ("H", 17, 2), ("dx", 1032, 2),
