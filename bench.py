@@ -35,7 +35,9 @@ import numpy as np
 # --workload: the SBM-shaped training step (default), the Large-shaped
 # training step (B=4, n=1024), or the sampling-time forward on Planar- /
 # Tree-shaped batches (forward only, many calls per model)
-WORKLOADS = {"sbm-train": "sbm", "large-train": "large", "planar-sample": "planar", "tree-sample": "tree"}
+WORKLOADS = {"sbm-train": "sbm", "large-train": "large", "planar-sample": "planar", "tree-sample": "tree",
+             "block-sbm-train": "sbm", "block-large-train": "large"}
+BLOCK = ("block-sbm-train", "block-large-train")
 TRAINING = ("sbm-train", "large-train")
 DESCRIBE = {
     "sbm": "sbm-shaped training step (fwd+bwd): B=32, n=192 padded, n_real~U[44,187], 2-5 blocks, "
@@ -172,6 +174,8 @@ def memory_report(buf, step, torch):
 
 
 def run_ours(args):
+    if args.workload in BLOCK:
+        return run_block(args)
     if args.workload not in TRAINING:
         return run_sample(args, WORKLOADS[args.workload])
     WORKLOAD = WORKLOADS[args.workload]
@@ -640,6 +644,257 @@ def run_e2e(args, buf, d, stream, step):
     return {"ms": t0.elapsed_time(t1) / n, "h2d": h2d, "d2h": d2h, "steps": n}
 
 
+# ------------------------------------------------------------------ the block around the layer
+
+
+def block_step_bytes(p):
+    """Algorithmic bytes of one block training step: the layer's (compulsory_bytes)
+    plus the block's edge streams (forward: E' read, Eout write; backward: E',
+    dEout read, dE' write) and node streams (forward: X' read, Xout write;
+    backward: X', dXout read, dX' write)."""
+    s = 2 if p.dtype == "bf16" else 4
+    pairs, nodes = p.B * p.n * p.n, p.B * p.n
+    return compulsory_bytes(p) + pairs * p.de * s * 5 + nodes * p.dx * s * 5
+
+
+def cpu_baseline_block(p, d, W, Wb, dyo, graphs):
+    """The block oracle (fp64: the layer's C oracle and the block's numpy
+    restatement), as it stands, forward + backward of the first `graphs`
+    graphs of the batch."""
+    import oracle
+    from oracle import block as OB
+    oracle.build()
+    sl = {k: d[k][:graphs] for k in ("X", "E", "y", "M", "dXout", "dEout")}
+    dims = dict(H=p.H, dh=p.dh)
+    t = time.perf_counter()
+    OB.block_forward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, Wb)
+    OB.block_backward(dims, sl["X"], sl["E"], sl["y"], sl["M"], W, Wb, sl["dXout"], sl["dEout"], dyo[:graphs])
+    dt = time.perf_counter() - t
+    return {"value": graphs * p.n * p.n / dt, "unit": UNIT, "cores": oracle.threads_used(), "kind": "oracle",
+            "sample": f"{graphs} of {p.B} graphs of the workload (n={p.n}), block forward + backward, fp64",
+            "seconds": dt}
+
+
+def run_block(args):
+    """Training step of the graph-transformer block around the layer (layer,
+    LayerNorms, FFNs, global update; forward + backward) on the SBM- or
+    Large-shaped batch."""
+    name = WORKLOADS[args.workload]
+    import torch
+    import torch.distributed as dist
+
+    from edge_aware_graph_b200 import dp, eaga
+    from edge_aware_graph_b200 import inputs as I
+    from edge_aware_graph_b200.buffers import BlockBuffers, host_to_storage_tensor
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    base = I.preset(name)
+    p = I.preset(name, seed=dp.rank_seed(base.seed, rank))
+    d = I.draw_inputs(p, with_grads=True)
+    W, Wb = I.draw_weights(base), I.draw_block_weights(base)     # one model on every rank
+    dyo = I.draw_block_upstream(p)
+    buf = BlockBuffers(p.B, p.n, p.dx, p.de, p.dy, p.H, p.dh, dtype=p.dtype, backward=True)
+    buf.load_inputs(d, W)
+    buf.load_block(Wb, dyo)
+    stream = torch.cuda.current_stream()
+
+    def block(s):
+        buf.block_forward(s)
+        buf.block_backward(s)
+
+    def step():
+        block(torch.cuda.current_stream())
+        dp.allreduce_weight_grads(buf.dW_flat)
+        dp.allreduce_weight_grads(buf.dWb_flat)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    nk = min(args.steps, 20)
+    points = (0, 2, 3, 4)
+    evs = {q: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+           for q in points}
+    for q in points:
+        for a, b in evs[q]:
+            a.record(stream)
+            b.record(stream)
+    torch.cuda.synchronize()
+    for k in range(nk):
+        for q in points:
+            eaga.set_profile_events(q, *evs[q][k])
+        step()
+    torch.cuda.synchronize()
+    for q in points:
+        eaga.set_profile_events(q)
+    kms = {q: statistics.mean(a.elapsed_time(b) for a, b in evs[q]) for q in points}
+
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            block(cap)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=cap):
+            block(cap)
+        torch.cuda.synchronize()
+
+    def timed_step():
+        if graph is not None:
+            graph.replay()
+            dp.allreduce_weight_grads(buf.dW_flat)
+            dp.allreduce_weight_grads(buf.dWb_flat)
+        else:
+            step()
+
+    for _ in range(3):
+        timed_step()
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for _ in range(K):
+        timed_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms_total = dp.max_over_ranks(t0.elapsed_time(t1), "cuda")
+    if graph is not None:
+        torch.cuda.synchronize()
+        del graph
+
+    # end to end through the public API: inputs from pinned host memory, every
+    # output and gradient read back, inside the timed region
+    names_in = ["X", "E", "y", "dXout", "dEout", "dyout"]
+    src = dict(d)
+    src["dyout"] = dyo
+    host_in = {k: host_to_storage_tensor(src[k], buf.dtype).pin_memory() for k in names_in}
+    host_M = torch.from_numpy(np.ascontiguousarray(d["M"])).pin_memory()
+    outs = [buf.Xout, buf.Eout, buf.yout, buf.dX, buf.dE, buf.dy, buf.dW_flat, buf.dWb_flat]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + host_M.numel()
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    def e2e_step():
+        for k in names_in:
+            getattr(buf, k).copy_(host_in[k], non_blocking=True)
+        buf.M.copy_(host_M, non_blocking=True)
+        step()
+        for h, t in zip(host_out, outs):
+            h.copy_(t, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dp.max_over_ranks(a0.elapsed_time(a1) / args.e2e_steps, "cuda")
+
+    launches = (eaga.block_kernel_launches(buf.dims, False) + eaga.block_kernel_launches(buf.dims, True)) * K
+    torch.cuda.synchronize()
+    before = torch.cuda.memory_allocated()
+    torch.cuda.reset_peak_memory_stats()
+    step()
+    torch.cuda.synchronize()
+    mem = {"peak_mib_delta_per_step": (torch.cuda.max_memory_allocated() - before) / 2**20,
+           "held_mib": before / 2**20, "block_workspace_bwd_mib": buf.bws_bwd.numel() / 2**20,
+           "block_saved_mib": buf.bsaved.numel() / 2**20,
+           "block_workspace_bwd_per_pair_bytes": buf.bws_bwd.numel() / (p.B * p.n * p.n)}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    pairs = p.B * p.n * p.n
+    ms_step = ms_total / K
+    value = world * pairs * K / (ms_total / 1e3)
+    peak, peak_kind = measured_peaks()
+    kern = {
+        "k_eblk_bwd (edge sub-block backward)": (pairs * p.de * 2 * 3, kms[4], None),
+        "k_eblk_fwd (edge sub-block forward)": (pairs * p.de * 2 * 2, kms[3], None),
+        "k_bwd_stream (layer backward row pair kernel)": (pair_kernel_bytes(p, "bwd"), kms[2],
+                                                          NCU_TRAFFIC.get((name, "k_bwd_stream"))),
+        "k_fwd_stream (layer forward pair kernel)": (pair_kernel_bytes(p, "fwd"), kms[0],
+                                                     NCU_TRAFFIC.get((name, "k_fwd_stream"))),
+    }
+    kern["k_eblk_bwd (edge sub-block backward)"] = kern["k_eblk_bwd (edge sub-block backward)"][:2] + (
+        NCU_TRAFFIC.get((name, "k_eblk_bwd")),)
+    kern["k_eblk_fwd (edge sub-block forward)"] = kern["k_eblk_fwd (edge sub-block forward)"][:2] + (
+        NCU_TRAFFIC.get((name, "k_eblk_fwd")),)
+    rl = lambda k: {"bound": "hbm", "kernel": k, "achieved": kern[k][0] / (kern[k][1] / 1e3) / 1e9, "peak": peak,
+                    "peak_kind": peak_kind, "unit": "GB/s",
+                    "frac": kern[k][0] / (kern[k][1] / 1e3) / 1e9 / peak, "traffic": kern[k][2],
+                    "algorithmic_bytes": kern[k][0], "ms_per_launch": kern[k][1]}
+    dominant = max(kern, key=lambda k: kern[k][1])
+    sb = block_step_bytes(p)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": f"synthetic (seeded {name.upper()}-shaped graphs; edge_aware_graph_b200/inputs.py)",
+        "config": {"workload": "graph-transformer block training step (the layer, LayerNorms, node / edge / "
+                               "global FFNs and the global update; fwd+bwd) on the " + DESCRIBE[name],
+                   "global_batch": p.B * world, "seq_len": p.n, "parallelism": f"dp{world}",
+                   "l2": f"inputs larger than L2 (E, E', dE', dEout {pairs * p.de * 2 / 2**20:.0f} MiB each)",
+                   "launch": "CUDA graph of the step's kernels" if not args.no_graph else "eager"},
+        "roofline": rl(dominant),
+        "roofline_kernels": {k: rl(k) for k in kern},
+        "step_roofline": {"compulsory_bytes": sb, "achieved_gbs": sb / (ms_step / 1e3) / 1e9,
+                          "frac_of_measured": sb / (ms_step / 1e3) / 1e9 / peak},
+        "clocks": clk,
+        "e2e": {"value": world * pairs / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+        "gpu_launches": launches,
+        "memory": mem,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_block(p, d, W, Wb, dyo, 2 if name == "sbm" else 1)
+    return out
+
+
+def run_reference_block(args, world):
+    """The oracle arm of the block workloads: the block oracle's forward +
+    backward on --ref-graphs graphs (one at n = 1024) per step."""
+    from edge_aware_graph_b200 import inputs as I
+    name = WORKLOADS[args.workload]
+    p = I.preset(name)
+    d = I.draw_inputs(p, with_grads=True)
+    W, Wb, dyo = I.draw_weights(p), I.draw_block_weights(p), I.draw_block_upstream(p)
+    g = 1 if name == "large" else max(1, min(args.ref_graphs, p.B))
+    for _ in range(args.warmup):
+        cpu_baseline_block(p, d, W, Wb, dyo, 1)
+    res = [cpu_baseline_block(p, d, W, Wb, dyo, g) for _ in range(args.steps)]
+    secs = sum(r["seconds"] for r in res)
+    value = args.steps * g * p.n * p.n / secs
+    cb = dict(res[0])
+    cb["value"] = value
+    cb.pop("seconds", None)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": f"synthetic (seeded {name.upper()}-shaped graphs)",
+            "config": {"workload": "graph-transformer block training step on the " + DESCRIBE[name]
+                                   + f"; bounded sample of {g} graph(s) per step",
+                       "global_batch": g, "seq_len": p.n, "parallelism": "cpu"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 # ------------------------------------------------------------------ oracle arm
 
 
@@ -690,6 +945,8 @@ def run_reference(args):
     if rank != 0:
         return None
     from edge_aware_graph_b200 import inputs as I
+    if args.workload in BLOCK:
+        return run_reference_block(args, world)
     if args.workload not in TRAINING:
         return run_reference_sample(args, WORKLOADS[args.workload], world)
     WORKLOAD = WORKLOADS[args.workload]

@@ -95,8 +95,9 @@ inline WsLayout ws_layout(const eaga_dims &d) {
     return W;
 }
 
-// Optional profiling events around the pair kernels (eaga_set_profile_events).
-extern std::atomic<void *> g_prof_events[3][2];
+// Optional profiling events around the pair kernels and the block's edge kernels
+// (eaga_set_profile_events).
+extern std::atomic<void *> g_prof_events[5][2];
 inline void prof_mark(int point, int which, cudaStream_t st) {
     void *ev = g_prof_events[point][which].load(std::memory_order_acquire);
     if (ev) cudaEventRecord(static_cast<cudaEvent_t>(ev), st);

@@ -13,7 +13,7 @@
 using namespace eaga;
 
 namespace eaga {
-std::atomic<void *> g_prof_events[3][2] = {};
+std::atomic<void *> g_prof_events[5][2] = {};
 }
 
 namespace {
@@ -452,7 +452,7 @@ eaga_status eaga_get_device_status(void *workspace, void *stream) {
 }
 
 eaga_status eaga_set_profile_events(int point, void *before, void *after) {
-    if (point < 0 || point > 2) return EAGA_ERR_INVALID_ARG;
+    if (point < 0 || point > 4) return EAGA_ERR_INVALID_ARG;
     if ((before == nullptr) != (after == nullptr)) return EAGA_ERR_INVALID_ARG;
     g_prof_events[point][0].store(before, std::memory_order_release);
     g_prof_events[point][1].store(after, std::memory_order_release);

@@ -205,27 +205,43 @@ __device__ __forceinline__ float block_ln(const float *z, float *xh, int dy, flo
     return rs;
 }
 
+// out[o] = init(o) + sum_k in[k] w(k, o) for o < nout <= blockDim.x, by every
+// thread of the CTA: the k range split into blockDim.x / nout parts whose
+// partial sums (in `part`, blockDim.x floats) are added in part order.
+template <class W, class Init>
+__device__ __forceinline__ void block_matvec(const float *in, int K, int nout, W w, Init init, float *out,
+                                             float *part) {
+    const int P = blockDim.x / nout;
+    const int t = threadIdx.x, o = t % nout, pi = t / nout;
+    if (pi < P) {
+        const int k0 = pi * K / P, k1 = (pi + 1) * K / P;
+        float a = 0.f;
+        for (int k = k0; k < k1; ++k) a = fmaf(in[k], w(k, o), a);
+        part[pi * nout + o] = a;
+    }
+    __syncthreads();
+    for (int q = t; q < nout; q += blockDim.x) {
+        float a = init(q);
+        for (int pp = 0; pp < P; ++pp) a += part[pp * nout + q];
+        out[q] = a;
+    }
+    __syncthreads();
+}
+
 // Recomputes the global sub-block of graph b from y1 into shared memory:
 // x1 (LN1 normalised), ya, hpre, h, x2 (LN2 normalised); returns r1, r2.
 __device__ void y_sub_forward(const YParams &p, const float *y1, float *x1, float *ya, float *hpre, float *h,
-                              float *yz, float *x2, float *scratch, float &r1, float &r2) {
+                              float *yz, float *x2, float *scratch, float *part, float &r1, float &r2) {
     const int dy = p.dy, fy = 2 * p.dy;
     r1 = block_ln(y1, x1, dy, scratch);
     for (int o = threadIdx.x; o < dy; o += blockDim.x) ya[o] = fmaf(x1[o], bf(p.g1, o), bf(p.s1, o));
     __syncthreads();
-    for (int f = threadIdx.x; f < fy; f += blockDim.x) {
-        float a = bf(p.b1, f);
-        for (int o = 0; o < dy; ++o) a = fmaf(ya[o], bf(p.W1, (size_t)o * fy + f), a);
-        hpre[f] = a;
-        h[f] = fmaxf(a, 0.f);
-    }
+    block_matvec(ya, dy, fy, [&](int k, int f) { return bf(p.W1, (size_t)k * fy + f); },
+                 [&](int f) { return bf(p.b1, f); }, hpre, part);
+    for (int f = threadIdx.x; f < fy; f += blockDim.x) h[f] = fmaxf(hpre[f], 0.f);
     __syncthreads();
-    for (int o = threadIdx.x; o < dy; o += blockDim.x) {
-        float a = ya[o] + bf(p.b2, o);
-        for (int f = 0; f < fy; ++f) a = fmaf(h[f], bf(p.W2, (size_t)f * dy + o), a);
-        yz[o] = a;
-    }
-    __syncthreads();
+    block_matvec(h, fy, dy, [&](int k, int o) { return bf(p.W2, (size_t)k * dy + o); },
+                 [&](int o) { return ya[o] + bf(p.b2, o); }, yz, part);
     r2 = block_ln(yz, x2, dy, scratch);
 }
 
@@ -261,7 +277,7 @@ __global__ void __launch_bounds__(256) k_y_fwd(YParams p) {
     extern __shared__ float sm[];
     const int b = blockIdx.x, dx = p.dx, dy = p.dy, fy = 2 * p.dy, n = p.n;
     float *pX = sm, *pE = pX + dx, *y1 = pE + 64, *x1 = y1 + dy, *ya = x1 + dy, *hpre = ya + dy, *h = hpre + fy,
-          *yz = h + fy, *x2 = yz + dy, *scratch = x2 + dy;
+          *yz = h + fy, *x2 = yz + dy, *part = x2 + dy, *y1b = part + 256, *scratch = y1b + dy;
     float c = 0.f;
     for (int i = threadIdx.x; i < n; i += blockDim.x) c += p.M[(size_t)b * n + i] ? 1.f : 0.f;
     const float cnt = block_sum(c, scratch);
@@ -275,16 +291,15 @@ __global__ void __launch_bounds__(256) k_y_fwd(YParams p) {
         p.pE[(size_t)b * 64 + k] = pE[k];
     }
     __syncthreads();
-    for (int o = threadIdx.x; o < dy; o += blockDim.x) {
-        float a = bf(p.y, (size_t)b * dy + o) + bf(p.by, o);
-        for (int k = 0; k < dx; ++k) a = fmaf(pX[k], bf(p.Wyx, (size_t)k * dy + o), a);
-        for (int k = 0; k < 64; ++k) a = fmaf(pE[k], bf(p.Wye, (size_t)k * dy + o), a);
-        y1[o] = a;
-        p.y1[(size_t)b * dy + o] = a;
-    }
+    // y1 = y + pX Wyx + pE Wye + by
+    block_matvec(pX, dx, dy, [&](int k, int o) { return bf(p.Wyx, (size_t)k * dy + o); },
+                 [&](int o) { return bf(p.y, (size_t)b * dy + o) + bf(p.by, o); }, y1b, part);
+    block_matvec(pE, 64, dy, [&](int k, int o) { return bf(p.Wye, (size_t)k * dy + o); },
+                 [&](int o) { return y1b[o]; }, y1, part);
+    for (int o = threadIdx.x; o < dy; o += blockDim.x) p.y1[(size_t)b * dy + o] = y1[o];
     __syncthreads();
     float r1, r2;
-    y_sub_forward(p, y1, x1, ya, hpre, h, yz, x2, scratch, r1, r2);
+    y_sub_forward(p, y1, x1, ya, hpre, h, yz, x2, scratch, part, r1, r2);
     for (int o = threadIdx.x; o < dy; o += blockDim.x)
         p.yout[(size_t)b * dy + o] = __float2bfloat16_rn(fmaf(x2[o], bf(p.g2, o), bf(p.s2, o)));
 }
@@ -296,11 +311,11 @@ __global__ void __launch_bounds__(256) k_y_bwd(YParams p) {
     extern __shared__ float sm[];
     const int b = blockIdx.x, dx = p.dx, dy = p.dy, fy = 2 * p.dy, n = p.n;
     float *y1 = sm, *x1 = y1 + dy, *ya = x1 + dy, *hpre = ya + dy, *h = hpre + fy, *yz = h + fy, *x2 = yz + dy,
-          *dyz = x2 + dy, *dh = dyz + dy, *dya = dh + fy, *dy1 = dya + dy, *scratch = dy1 + dy;
+          *dyz = x2 + dy, *dh = dyz + dy, *dya = dh + fy, *dy1 = dya + dy, *part = dy1 + dy, *scratch = part + 256;
     for (int o = threadIdx.x; o < dy; o += blockDim.x) y1[o] = p.y1[(size_t)b * dy + o];
     __syncthreads();
     float r1, r2;
-    y_sub_forward(p, y1, x1, ya, hpre, h, yz, x2, scratch, r1, r2);
+    y_sub_forward(p, y1, x1, ya, hpre, h, yz, x2, scratch, part, r1, r2);
     // dyz = LN2^T(dyout)
     float m1 = 0.f, m2 = 0.f;
     for (int o = threadIdx.x; o < dy; o += blockDim.x) {
@@ -315,18 +330,14 @@ __global__ void __launch_bounds__(256) k_y_bwd(YParams p) {
         dyz[o] = r2 * (dg - m1 - x2[o] * m2);
     }
     __syncthreads();
-    for (int f = threadIdx.x; f < fy; f += blockDim.x) {
-        float a = 0.f;
-        for (int o = 0; o < dy; ++o) a = fmaf(dyz[o], bf(p.W2, (size_t)f * dy + o), a);
-        dh[f] = hpre[f] > 0.f ? a : 0.f;
-    }
+    // dh = dyz W2^T [hpre > 0]
+    block_matvec(dyz, dy, fy, [&](int k, int f) { return bf(p.W2, (size_t)f * dy + k); }, [](int) { return 0.f; },
+                 dh, part);
+    for (int f = threadIdx.x; f < fy; f += blockDim.x) dh[f] = hpre[f] > 0.f ? dh[f] : 0.f;
     __syncthreads();
-    for (int o = threadIdx.x; o < dy; o += blockDim.x) {
-        float a = dyz[o];
-        for (int f = 0; f < fy; ++f) a = fmaf(dh[f], bf(p.W1, (size_t)o * fy + f), a);
-        dya[o] = a;
-    }
-    __syncthreads();
+    // dya = dyz + dh W1^T
+    block_matvec(dh, fy, dy, [&](int k, int o) { return bf(p.W1, (size_t)o * fy + k); },
+                 [&](int o) { return dyz[o]; }, dya, part);
     m1 = 0.f;
     m2 = 0.f;
     for (int o = threadIdx.x; o < dy; o += blockDim.x) {
@@ -424,23 +435,39 @@ __global__ void __launch_bounds__(256) k_y_wgrad(YParams p, YGrads gr) {
 // ------------------------------------------------------------------ reductions
 
 // dst = sum over parts of src (part k at src + k * stride); with trows > 0 the
-// segment is the transpose of a [trows][count / trows] source.
+// segment is the transpose of a [trows][count / trows] source.  One warp per
+// item: a segment of many parts (more than 16) gives one entry to each warp,
+// whose lanes take every 32nd part and add their sums with shuffles; a segment
+// of few parts gives 32 consecutive entries to each warp, one a lane.  Every
+// entry is summed in the same order on every call.
 __global__ void __launch_bounds__(256) k_sum_parts(SumSegs segs) {
-    int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    int item = blockIdx.x * 8 + (threadIdx.x >> 5);
     for (int s = 0; s < segs.n; ++s) {
         const SumSeg &g = segs.seg[s];
-        if (e < g.count) {
-            int src = e;
-            if (g.trows > 0) {
-                const int cols = g.count / g.trows;
-                src = (e % g.trows) * cols + e / g.trows;
-            }
-            float t = 0.f;
+        const bool wide = g.nparts > 16;
+        const int items = wide ? g.count : (g.count + 31) / 32;
+        if (item >= items) {
+            item -= items;
+            continue;
+        }
+        const int e = wide ? item : item * 32 + lane;
+        if (e >= g.count) return;
+        int src = e;
+        if (g.trows > 0) {
+            const int cols = g.count / g.trows;
+            src = (e % g.trows) * cols + e / g.trows;
+        }
+        float t = 0.f;
+        if (wide) {
+            for (int k = lane; k < g.nparts; k += 32) t += g.src[(size_t)k * g.stride + src];
+            t = warp_sum(t);
+            if (lane == 0) g.dst[e] = t;
+        } else {
             for (int k = 0; k < g.nparts; ++k) t += g.src[(size_t)k * g.stride + src];
             g.dst[e] = t;
-            return;
         }
-        e -= g.count;
+        return;
     }
 }
 
@@ -494,7 +521,7 @@ cudaError_t ln_bwd(int D, const void *Z, const void *dOut, const void *g, const 
 }  // namespace
 
 bool block_supports(int dx, int de, int dy) {
-    return de == 64 && (dx == 256 || dx == 512) && dy % 32 == 0 && dy >= 32 && dy <= 256;
+    return de == 64 && (dx == 256 || dx == 512) && dy % 32 == 0 && dy >= 32 && dy <= 128;
 }
 
 BlockSaved block_saved_layout(int B, int n, int dx, int dy, size_t base) {
@@ -537,7 +564,7 @@ BlockWs block_ws_layout(int B, int n, int dx, int dy, size_t base, int for_backw
         L.wg1 = off; off = align256(off + (size_t)L.wsplits * dx * 2 * dx * 4);
         L.wg2 = off; off = align256(off + (size_t)L.wsplits * 2 * dx * dx * 4);
         L.ectas = edge_backward_ctas(B, n);
-        L.eparts = off; off = align256(off + (size_t)L.ectas * 4 * EB_PART * 4);
+        L.eparts = off; off = align256(off + (size_t)L.ectas * EB_PART * 4);
         L.ewparts = off; off = align256(off + (size_t)L.ectas * 2 * 128 * 64 * 4);
     }
     L.total = off;
@@ -597,7 +624,9 @@ cudaError_t tail_forward(const TailFwd &a, char *ws, const BlockWs &W, char *sav
         p.status = a.status;
         p.B = a.B;
         p.n = a.n;
+        prof_mark(3, 0, st);
         BLK_TRY(edge_forward(e, st));
+        prof_mark(3, 1, st);
     }
     void *Xa = saved + S.Xa, *Hx = saved + S.Hx, *Xz = saved + S.Xz;
     BLK_TRY(ln_fwd(dx, a.Xmid, a.wb[BW_X + 0], a.wb[BW_X + 1], nullptr, Xa, R, st));
@@ -627,7 +656,7 @@ cudaError_t tail_forward(const TailFwd &a, char *ws, const BlockWs &W, char *sav
         p.pX = reinterpret_cast<float *>(saved + S.pX);
         p.pE = reinterpret_cast<float *>(saved + S.pE);
         p.yout = static_cast<__nv_bfloat16 *>(a.yout);
-        const size_t smem = (size_t)(a.dx + 64 + 9 * a.dy + 32) * 4;
+        const size_t smem = (size_t)(a.dx + 64 + 10 * a.dy + 256 + 32) * 4;
         k_y_fwd<<<a.B, 256, smem, st>>>(p);
         BLK_TRY(cudaGetLastError());
     }
@@ -647,7 +676,7 @@ cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const ch
     yp.dpE = reinterpret_cast<float *>(ws + W.dpE);
     yp.yv = reinterpret_cast<float *>(ws + W.yv);
     {
-        const size_t smem = (size_t)(15 * a.dy + 32) * 4;
+        const size_t smem = (size_t)(15 * a.dy + 256 + 32) * 4;
         k_y_bwd<<<a.B, 256, smem, st>>>(yp);
         BLK_TRY(cudaGetLastError());
         YGrads g;
@@ -682,7 +711,9 @@ cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const ch
         p.status = a.status;
         p.B = a.B;
         p.n = a.n;
+        prof_mark(4, 0, st);
         BLK_TRY(edge_backward(e, st));
+        prof_mark(4, 1, st);
     }
     void *dXz = ws + W.dXz, *dHx = ws + W.dHx, *dXa = ws + W.dXa, *dXmid = ws + W.dXmid;
     const void *Xa = saved + S.Xa, *Hx = saved + S.Hx, *Xz = saved + S.Xz;
@@ -733,7 +764,7 @@ cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const ch
         add(reinterpret_cast<float *>(ws + W.wg1), dw(BW_X + 2), W.wsplits, dx * 2 * dx, dx * 2 * dx, 0);
         add(reinterpret_cast<float *>(ws + W.wg2), dw(BW_X + 4), W.wsplits, 2 * dx * dx, 2 * dx * dx, 0);
         const float *ep = reinterpret_cast<const float *>(ws + W.eparts);
-        const int np = W.ectas * 4;
+        const int np = W.ectas;
         add(ep + 0, dw(BW_E + 6), np, EB_PART, 64, 0);      // dg2
         add(ep + 64, dw(BW_E + 7), np, EB_PART, 64, 0);     // ds2
         add(ep + 128, dw(BW_E + 5), np, EB_PART, 64, 0);    // db2
@@ -743,9 +774,10 @@ cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const ch
         const float *ew = reinterpret_cast<const float *>(ws + W.ewparts);
         add(ew, dw(BW_E + 4), W.ectas, 2 * 128 * 64, 128 * 64, 0);            // dW2 [128][64]
         add(ew + 128 * 64, dw(BW_E + 2), W.ectas, 2 * 128 * 64, 128 * 64, 128);  // dW1 = (dW1^T)^T
-        int total = 0;
-        for (int s = 0; s < sg.n; ++s) total += sg.seg[s].count;
-        k_sum_parts<<<(total + 255) / 256, 256, 0, st>>>(sg);
+        int items = 0;
+        for (int s = 0; s < sg.n; ++s)
+            items += sg.seg[s].nparts > 16 ? sg.seg[s].count : (sg.seg[s].count + 31) / 32;
+        k_sum_parts<<<(items + 7) / 8, 256, 0, st>>>(sg);
         BLK_TRY(cudaGetLastError());
     }
     return cudaSuccess;

@@ -14,7 +14,7 @@ bool encode_tile_map(CUtensorMap *m, const void *base, int B, int n);
 
 namespace blk {
 
-constexpr int EB_PART = 448;     // per-warp channel sums of the edge backward: dg2, ds2, db2, dg1, ds1 [64], db1 [128]
+constexpr int EB_PART = 448;     // per-CTA channel sums of the edge backward: dg2, ds2, db2, dg1, ds1 [64], db1 [128]
 
 // Parameters of the edge kernels (device pointers; bf16 parameters).
 struct EbParams {
@@ -22,7 +22,7 @@ struct EbParams {
     const __nv_bfloat16 *g1, *s1, *b1, *b2, *g2, *s2;
     float *pool;            // forward: [B, 64] sums of E' over valid pairs (added to)
     const float *dpool;     // backward: [B, 64] gradient of the edge pooling, divided by the pair count
-    float *parts;           // backward: [CTAs * 4][EB_PART]
+    float *parts;           // backward: [CTAs][EB_PART]
     float *wparts;          // backward: [CTAs][2][128][64]: dW2, dW1^T
     int *status;
     int B, n, ti, tj;

@@ -189,6 +189,39 @@ __device__ __forceinline__ float normalise64(float (&x)[64]) {
     return r;
 }
 
+// Parameters from shared memory four at a time (the arrays are 16-byte aligned).
+__device__ __forceinline__ float4 par4(const float *par, int i) { return *reinterpret_cast<const float4 *>(par + i); }
+// x = x g + s over 64 channels (g, s at par offsets), or 0 where !keep.
+__device__ __forceinline__ void affine64(float (&x)[64], const float *par, int g, int s, bool keep = true) {
+#pragma unroll
+    for (int c = 0; c < 64; c += 4) {
+        const float4 a = par4(par, g + c), b = par4(par, s + c);
+        x[c] = keep ? fmaf(x[c], a.x, b.x) : 0.f;
+        x[c + 1] = keep ? fmaf(x[c + 1], a.y, b.y) : 0.f;
+        x[c + 2] = keep ? fmaf(x[c + 2], a.z, b.z) : 0.f;
+        x[c + 3] = keep ? fmaf(x[c + 3], a.w, b.w) : 0.f;
+    }
+}
+// Four 16-column TMEM loads of the thread's lane into v[64], one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(v));
+    tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+    tmem_ld16(taddr + 32, *reinterpret_cast<float(*)[16]>(v + 32));
+    tmem_ld16(taddr + 48, *reinterpret_cast<float(*)[16]>(v + 48));
+    tmem_ld_wait();
+}
+// x += v + b over 64 channels (b at a par offset).
+__device__ __forceinline__ void add_bias64(float (&x)[64], const float (&v)[64], const float *par, int b) {
+#pragma unroll
+    for (int c = 0; c < 64; c += 4) {
+        const float4 q = par4(par, b + c);
+        x[c] += v[c] + q.x;
+        x[c + 1] += v[c + 1] + q.y;
+        x[c + 2] += v[c + 2] + q.z;
+        x[c + 3] += v[c + 3] + q.w;
+    }
+}
+
 __device__ __forceinline__ void load_params(float *par, const EbParams &p, int tid, int nthr) {
     for (int c = tid; c < 448; c += nthr) {
         float v;
@@ -231,26 +264,35 @@ __device__ __forceinline__ void mma_wgrad(uint32_t d, uint32_t a, uint32_t b, bo
 // `pos` records h_c > 0.
 __device__ __forceinline__ void h_epilogue(uint8_t *Ht, int r, uint32_t tl, const float *b1, uint32_t (&pos)[4]) {
 #pragma unroll
-    for (int c0 = 0; c0 < EF; c0 += 16) {
-        float v[16];
-        tmem_ld16(tl + c0, v);
-        tmem_ld_wait();
-        uint32_t bits = 0;
+    for (int hf = 0; hf < 2; ++hf) {
+        float v[64];
+        tmem_ld64(tl + 64 * hf, v);
+        uint8_t *half = Ht + hf * EB_TILE;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            v[u] = fmaxf(v[u] + b1[c0 + u], 0.f);
-            bits |= (v[u] > 0.f ? 1u : 0u) << u;
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+            uint32_t bits = 0;
+#pragma unroll
+            for (int u = 0; u < 16; u += 4) {
+                const float4 q = par4(b1, 64 * hf + c0 + u);
+                v[c0 + u] = fmaxf(v[c0 + u] + q.x, 0.f);
+                v[c0 + u + 1] = fmaxf(v[c0 + u + 1] + q.y, 0.f);
+                v[c0 + u + 2] = fmaxf(v[c0 + u + 2] + q.z, 0.f);
+                v[c0 + u + 3] = fmaxf(v[c0 + u + 3] + q.w, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) bits |= (v[c0 + u] > 0.f ? 1u : 0u) << u;
+            const int cg = 64 * hf + c0;
+            pos[cg >> 5] |= bits << (cg & 16);
+            const int ch = c0 >> 3;
+            const float *w = v + c0;
+            uint4 u0, u1;
+            u0.x = pack_bf16(w[0], w[1]); u0.y = pack_bf16(w[2], w[3]);
+            u0.z = pack_bf16(w[4], w[5]); u0.w = pack_bf16(w[6], w[7]);
+            u1.x = pack_bf16(w[8], w[9]); u1.y = pack_bf16(w[10], w[11]);
+            u1.z = pack_bf16(w[12], w[13]); u1.w = pack_bf16(w[14], w[15]);
+            *reinterpret_cast<uint4 *>(half + sw128(r, ch)) = u0;
+            *reinterpret_cast<uint4 *>(half + sw128(r, ch + 1)) = u1;
         }
-        pos[c0 >> 5] |= bits << (c0 & 16);
-        uint8_t *half = Ht + (c0 >> 6) * EB_TILE;
-        const int ch = (c0 & 63) >> 3;
-        uint4 u0, u1;
-        u0.x = pack_bf16(v[0], v[1]); u0.y = pack_bf16(v[2], v[3]);
-        u0.z = pack_bf16(v[4], v[5]); u0.w = pack_bf16(v[6], v[7]);
-        u1.x = pack_bf16(v[8], v[9]); u1.y = pack_bf16(v[10], v[11]);
-        u1.z = pack_bf16(v[12], v[13]); u1.w = pack_bf16(v[14], v[15]);
-        *reinterpret_cast<uint4 *>(half + sw128(r, ch)) = u0;
-        *reinterpret_cast<uint4 *>(half + sw128(r, ch + 1)) = u1;
     }
 }
 
@@ -379,7 +421,7 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         }
         normalise64(x);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = fmaf(x[c], par[PAR_G1 + c], par[PAR_S1 + c]);
+        affine64(x, par, PAR_G1, PAR_S1);
         row_store64(slot, r, x);
         fence_proxy_async_smem();
         named_bar_sync(1, EB_THR);
@@ -407,17 +449,13 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         cta_wait(mmab, mph, fail, p.status);
         mph ^= 1u;
         tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 16) {
-            float v[16];
-            tmem_ld16(tl + c0, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int u = 0; u < 16; ++u) x[c0 + u] += v[u] + par[PAR_B2 + c0 + u];
+        {
+            float v[64];
+            tmem_ld64(tl, v);
+            add_bias64(x, v, par, PAR_B2);
         }
         normalise64(x);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = valid ? fmaf(x[c], par[PAR_G2 + c], par[PAR_S2 + c]) : 0.f;
+        affine64(x, par, PAR_G2, PAR_S2, valid);
         row_store64(slot, r, x);
         fence_proxy_async_smem();
         tc_fence_before();
@@ -533,7 +571,8 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             row_load64(sa, r, x1);
             const float r1 = normalise64(x1);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) z[c] = fmaf(x1[c], par[PAR_G1 + c], par[PAR_S1 + c]);
+            for (int c = 0; c < 64; ++c) z[c] = x1[c];
+            affine64(z, par, PAR_G1, PAR_S1);
             row_store64(sa, r, z);
             fence_proxy_async_smem();
             named_bar_sync(1, EB_THR);
@@ -559,13 +598,10 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             mph ^= 1u;
             tc_fence_after();
             // Ez = Ea + h W2 + b2 (z holds Ea), normalised in place (x2)
-#pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) {
-                float v[16];
-                tmem_ld16(tl + c0, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int u = 0; u < 16; ++u) z[c0 + u] += v[u] + par[PAR_B2 + c0 + u];
+            {
+                float v[64];
+                tmem_ld64(tl, v);
+                add_bias64(z, v, par, PAR_B2);
             }
             const float r2 = normalise64(z);
             // upstream gradient, masked: dg2, ds2; LN2's input gradient dEz
@@ -583,8 +619,12 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             }
             float m1 = 0.f, m2 = 0.f;
 #pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+                const float4 g = par4(par, PAR_G2 + c);
+                d[c] *= g.x; d[c + 1] *= g.y; d[c + 2] *= g.z; d[c + 3] *= g.w;
+            }
+#pragma unroll
             for (int c = 0; c < 64; ++c) {
-                d[c] *= par[PAR_G2 + c];
                 m1 += d[c];
                 m2 = fmaf(d[c], z[c], m2);
             }
@@ -676,13 +716,11 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             mph ^= 1u;
             tc_fence_after();
             // dEa = dEz + dh W1^T (d holds dEz); dg1, ds1; dE' = valid (LN1^T(dEa) + dpE_b)
+            {
+                float v[64];
+                tmem_ld64(tl, v);
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 16) {
-                float v[16];
-                tmem_ld16(tl + c0, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int u = 0; u < 16; ++u) d[c0 + u] += v[u];
+                for (int c = 0; c < 64; ++c) d[c] += v[c];
             }
             {
                 float o[2];
@@ -695,8 +733,12 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             }
             float n1 = 0.f, n2 = 0.f;
 #pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+                const float4 g = par4(par, PAR_G1 + c);
+                d[c] *= g.x; d[c + 1] *= g.y; d[c + 2] *= g.z; d[c + 3] *= g.w;
+            }
+#pragma unroll
             for (int c = 0; c < 64; ++c) {
-                d[c] *= par[PAR_G1 + c];
                 n1 += d[c];
                 n2 = fmaf(d[c], x1[c], n2);
             }
@@ -733,15 +775,25 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             __syncwarp();
         }
     }
-    // per-warp partial sums: [CTA][warp][448] in the order dg2, ds2, db2, dg1, ds1, db1
-    float *pw = p.parts + ((size_t)blockIdx.x * 4 + w) * EB_PART;
+    // the CTA's partial sums [CTA][448] in the order dg2, ds2, db2, dg1, ds1, db1:
+    // the four warps' sums added in warp order through shared memory (the H tile)
+    {
+        float *red = reinterpret_cast<float *>(sp + S::H);
+        tc_fence_before();
+        __syncthreads();
+        float *pw = red + w * EB_PART;
 #pragma unroll
-    for (int q = 0; q < 5; ++q) {
-        pw[64 * q + 2 * lane] = acc[2 * q];
-        pw[64 * q + 2 * lane + 1] = acc[2 * q + 1];
+        for (int q = 0; q < 5; ++q) {
+            pw[64 * q + 2 * lane] = acc[2 * q];
+            pw[64 * q + 2 * lane + 1] = acc[2 * q + 1];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) pw[320 + 4 * lane + u] = acc[10 + u];
+        __syncthreads();
+        for (int c = tid; c < EB_PART; c += EB_THR)
+            p.parts[(size_t)blockIdx.x * EB_PART + c] = red[c] + red[EB_PART + c] + red[2 * EB_PART + c] +
+                                                        red[3 * EB_PART + c];
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) pw[320 + 4 * lane + u] = acc[10 + u];
     // the CTA's dW2 [128][64] and dW1^T [128][64] from TMEM (zero without a live
     // tile); every product was waited for in the loop
     tc_fence_after();

@@ -267,7 +267,8 @@ def debug_wait_probe(workspace, limit: int, stream=None):
 
 def set_profile_events(point: int, before=None, after=None):
     """point 0: forward pair kernels, 1: backward pair kernels, 2: the backward's
-    row pair kernel alone; torch.cuda.Event or None."""
+    row pair kernel alone, 3 / 4: the edge kernel of the block's forward /
+    backward; torch.cuda.Event or None."""
     b = ctypes.c_void_p(before.cuda_event) if before is not None else None
     a = ctypes.c_void_p(after.cuda_event) if after is not None else None
     _check(lib().eaga_set_profile_events(int(point), b, a), "eaga_set_profile_events")

@@ -258,9 +258,13 @@ EAGA_API eaga_status eaga_get_device_status(void *workspace, void *stream);
  * kernels of the forward) or eaga_backward (point 1: the pair kernels of the
  * backward; point 2: the backward's row pair kernel alone, specialised bf16
  * path only) records `before` on its stream just before launching those
- * kernels and `after` just after them.  NULL events clear the point.  This
- * is a process-wide setting: not for concurrent calls. */
-typedef enum { EAGA_PROF_FWD_PAIR = 0, EAGA_PROF_BWD_PAIR = 1, EAGA_PROF_BWD_ROWS = 2 } eaga_prof_point;
+ * kernels and `after` just after them; points 3 and 4 do the same around the
+ * edge kernel of eaga_block_forward and eaga_block_backward.  NULL events
+ * clear the point.  This is a process-wide setting: not for concurrent calls. */
+typedef enum {
+    EAGA_PROF_FWD_PAIR = 0, EAGA_PROF_BWD_PAIR = 1, EAGA_PROF_BWD_ROWS = 2,
+    EAGA_PROF_BLOCK_EDGE_FWD = 3, EAGA_PROF_BLOCK_EDGE_BWD = 4
+} eaga_prof_point;
 EAGA_API eaga_status eaga_set_profile_events(int point, void *before, void *after);
 
 /* Number of kernel launches (this library's kernels) that one eaga_forward
@@ -303,7 +307,7 @@ EAGA_API eaga_status eaga_debug_wait_probe(void *workspace, unsigned limit, void
  * dtype as the layer's weights; gradients fp32.
  *
  * Supported on the specialised bf16 path only (de = 64, H = 8, dh = 32, n
- * even) with dx = 256 or 512 and dy a multiple of 32 up to 256; other dims
+ * even) with dx = 256 or 512 and dy a multiple of 32 up to 128; other dims
  * return EAGA_ERR_UNSUPPORTED.  A stack of blocks calls these once per block
  * with each block's own weights, feeding Xout, Eout, yout on.
  * --------------------------------------------------------------------- */
