@@ -260,9 +260,8 @@ __device__ __forceinline__ void mma_wgrad(uint32_t d, uint32_t a, uint32_t b, bo
 }
 
 // The H epilogue of one pair row: h = relu(T + b1) for the 128 columns,
-// written as bf16 into the two 64-channel halves of the H tile; bit c of
-// `pos` records h_c > 0.
-__device__ __forceinline__ void h_epilogue(uint8_t *Ht, int r, uint32_t tl, const float *b1, uint32_t (&pos)[4]) {
+// written as bf16 into the two 64-channel halves of the H tile.
+__device__ __forceinline__ void h_epilogue(uint8_t *Ht, int r, uint32_t tl, const float *b1) {
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
         float v[64];
@@ -270,7 +269,6 @@ __device__ __forceinline__ void h_epilogue(uint8_t *Ht, int r, uint32_t tl, cons
         uint8_t *half = Ht + hf * EB_TILE;
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 16) {
-            uint32_t bits = 0;
 #pragma unroll
             for (int u = 0; u < 16; u += 4) {
                 const float4 q = par4(b1, 64 * hf + c0 + u);
@@ -279,10 +277,6 @@ __device__ __forceinline__ void h_epilogue(uint8_t *Ht, int r, uint32_t tl, cons
                 v[c0 + u + 2] = fmaxf(v[c0 + u + 2] + q.z, 0.f);
                 v[c0 + u + 3] = fmaxf(v[c0 + u + 3] + q.w, 0.f);
             }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) bits |= (v[c0 + u] > 0.f ? 1u : 0u) << u;
-            const int cg = 64 * hf + c0;
-            pos[cg >> 5] |= bits << (cg & 16);
             const int ch = c0 >> 3;
             const float *w = v + c0;
             uint4 u0, u1;
@@ -294,6 +288,22 @@ __device__ __forceinline__ void h_epilogue(uint8_t *Ht, int r, uint32_t tl, cons
             *reinterpret_cast<uint4 *>(half + sw128(r, ch + 1)) = u1;
         }
     }
+}
+
+// dh = dh' where the stored h > 0 (relu(x) > 0 exactly when x > 0), for 8
+// channels held as one 16-byte chunk of the H tile.
+__device__ __forceinline__ void relu_gate8(const uint4 hq, float *v) {
+    const uint32_t w[4] = {hq.x, hq.y, hq.z, hq.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        v[2 * k] = (int16_t)(w[k] & 0xFFFFu) > 0 ? v[2 * k] : 0.f;        // a positive bf16, as int16
+        v[2 * k + 1] = (int16_t)(w[k] >> 16) > 0 ? v[2 * k + 1] : 0.f;
+    }
+}
+
+// Packed bf16 pairs <-> floats of a 64-channel row kept in 32 registers.
+__device__ __forceinline__ float pk_get(const uint32_t (&p)[32], int c) {
+    return __uint_as_float((c & 1) ? (p[c >> 1] & 0xFFFF0000u) : (p[c >> 1] << 16));
 }
 
 // ------------------------------------------------------------------ forward
@@ -436,8 +446,7 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         cta_wait(mmab, mph, fail, p.status);
         mph ^= 1u;
         tc_fence_after();
-        uint32_t pos[4] = {0, 0, 0, 0};
-        h_epilogue(sp + S::H, r, tl, par + PAR_B1, pos);
+        h_epilogue(sp + S::H, r, tl, par + PAR_B1);
         fence_proxy_async_smem();
         tc_fence_before();
         named_bar_sync(1, EB_THR);
@@ -567,11 +576,12 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                 wts_ready = true;
             }
             // LN1 recomputed: x1 = normalised E', Ea = x1 g1 + s1
-            float x1[64], z[64], d[64];
-            row_load64(sa, r, x1);
-            const float r1 = normalise64(x1);
+            float z[64], d[64];
+            uint32_t x1[32];                 // normalised E' (LN1's x), bf16 pairs
+            row_load64(sa, r, z);
+            const float r1 = normalise64(z);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) z[c] = x1[c];
+            for (int c = 0; c < 32; ++c) x1[c] = pack_bf16(z[2 * c], z[2 * c + 1]);
             affine64(z, par, PAR_G1, PAR_S1);
             row_store64(sa, r, z);
             fence_proxy_async_smem();
@@ -584,8 +594,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             cta_wait(mmab, mph, fail, p.status);
             mph ^= 1u;
             tc_fence_after();
-            uint32_t pos[4] = {0, 0, 0, 0};
-            h_epilogue(sp + S::H, r, tl, par + PAR_B1, pos);
+            h_epilogue(sp + S::H, r, tl, par + PAR_B1);
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(1, EB_THR);
@@ -663,13 +672,11 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                     tmem_ld16(tl + c0, va);
                     tmem_ld16(tl + c0 + 64, vb);
                     tmem_ld_wait();
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int ca = c0 + u, cb = c0 + 64 + u;
-                        va[u] = ((pos[ca >> 5] >> (ca & 31)) & 1u) ? va[u] : 0.f;
-                        vb[u] = ((pos[cb >> 5] >> (cb & 31)) & 1u) ? vb[u] : 0.f;
-                    }
                     const int ch = c0 >> 3;
+                    relu_gate8(*reinterpret_cast<const uint4 *>(sp + S::H + sw128(r, ch)), va);
+                    relu_gate8(*reinterpret_cast<const uint4 *>(sp + S::H + sw128(r, ch + 1)), va + 8);
+                    relu_gate8(*reinterpret_cast<const uint4 *>(sp + S::H + EB_TILE + sw128(r, ch)), vb);
+                    relu_gate8(*reinterpret_cast<const uint4 *>(sp + S::H + EB_TILE + sw128(r, ch + 1)), vb + 8);
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
                         const float *v = hf ? vb : va;
@@ -724,7 +731,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             }
             {
                 float o[2];
-                warp_colsum_of<64>([&](int c) { return d[c] * x1[c]; }, lane, o);
+                warp_colsum_of<64>([&](int c) { return d[c] * pk_get(x1, c); }, lane, o);
                 acc[6] += o[0];
                 acc[7] += o[1];
                 warp_colsum_of<64>([&](int c) { return d[c]; }, lane, o);
@@ -740,7 +747,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
                 n1 += d[c];
-                n2 = fmaf(d[c], x1[c], n2);
+                n2 = fmaf(d[c], pk_get(x1, c), n2);
             }
             n1 *= (1.f / 64.f);
             n2 *= (1.f / 64.f);
@@ -752,7 +759,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int c = 4 * c4 + u;
-                    d[c] = valid ? r1 * (d[c] - n1 - x1[c] * n2) + qa[u] : 0.f;
+                    d[c] = valid ? r1 * (d[c] - n1 - pk_get(x1, c) * n2) + qa[u] : 0.f;
                 }
             }
             row_store64(sb, r, d);
