@@ -115,6 +115,54 @@ __device__ __forceinline__ void warp_colsum_of(F f, int lane, float (&out)[N / 3
     for (int i = 0; i < N / 32; ++i) out[i] = v[i];
 }
 
+// Column sums over the warp's 32 rows (32 w .. 32 w + 31) of a 128B-swizzled
+// [128][64] bf16 tile, on the warp's tensor cores: D = ones(16 x 16) B with B
+// the tile's rows (pairs, K) by channels (N), 8 channel groups of 8, the two
+// 16-row halves accumulated; every row of D is the column sum.  Lane l
+// returns channels 2l, 2l + 1 (the D row's columns 2(l%4), 2(l%4)+1 of
+// channel group l/4).
+__device__ __forceinline__ float2 warp_tile_colsum(uint32_t tile, int w, int lane) {
+    const uint32_t ones[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};
+    const int j = lane >> 2;
+    float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+            const uint32_t row = 32 * w + 16 * kb + (lane & 7) + 8 * ((lane >> 3) & 1);
+            const uint32_t chunk = 2 * g + (lane >> 4);
+            uint32_t q[4];
+            ldsm_x4_t(tile + sw128(row, chunk), q);
+            mma16816(da, ones, q[0], q[1]);
+            mma16816(db, ones, q[2], q[3]);
+        }
+        if (j == 2 * g) {
+            v0 = da[0];
+            v1 = da[1];
+        }
+        if (j == 2 * g + 1) {
+            v0 = db[0];
+            v1 = db[1];
+        }
+    }
+    return make_float2(v0, v1);
+}
+
+// Row r of a 128B-swizzled [128][64] bf16 tile from f(c), c = 0..63.
+template <class F>
+__device__ __forceinline__ void row_store_fn(uint8_t *tile, int r, F f) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4 u;
+        u.x = pack_bf16(f(8 * c), f(8 * c + 1));
+        u.y = pack_bf16(f(8 * c + 2), f(8 * c + 3));
+        u.z = pack_bf16(f(8 * c + 4), f(8 * c + 5));
+        u.w = pack_bf16(f(8 * c + 6), f(8 * c + 7));
+        *reinterpret_cast<uint4 *>(tile + sw128(r, c)) = u;
+    }
+}
+
 // Tile t of the grid of (graph, 4-row block, 32-column block).
 struct TileAt {
     int b, i0, j0;
@@ -423,11 +471,13 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         }
         float x[64];
         row_load64(slot, r, x);
-        {
-            float ps[2];
-            warp_colsum_of<64>([&](int c) { return valid ? x[c] : 0.f; }, lane, ps);
-            pool[0] += ps[0];
-            pool[1] += ps[1];
+        {   // the warp's valid E' rows summed on the tensor cores (invalid rows zeroed first)
+            if (!valid) row_zero(slot, r);
+            __syncwarp();
+            const float2 ps = warp_tile_colsum(slot_a, w, lane);
+            pool[0] += ps.x;
+            pool[1] += ps.y;
+            __syncwarp();
         }
         normalise64(x);
 #pragma unroll
@@ -557,7 +607,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
     }
     uint32_t mph = 0;
     bool wts_ready = false, any = false;
-    // per-lane channel sums: channels 2l, 2l+1 of dg2, ds2, db2, dg1, ds1 and 4l .. 4l+3 of db1
+    // per-lane channel sums: channels 2l, 2l+1 of dg2, ds2, db2, dg1, ds1 and of both halves of db1
     float acc[14];
 #pragma unroll
     for (int u = 0; u < 14; ++u) acc[u] = 0.f;
@@ -617,14 +667,19 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             row_load64(sb, r, d);
 #pragma unroll
             for (int c = 0; c < 64; ++c) d[c] = valid ? d[c] : 0.f;
-            {
-                float o[2];
-                warp_colsum_of<64>([&](int c) { return d[c] * z[c]; }, lane, o);
-                acc[0] += o[0];
-                acc[1] += o[1];
-                warp_colsum_of<64>([&](int c) { return d[c]; }, lane, o);
-                acc[2] += o[0];
-                acc[3] += o[1];
+            {   // dg2 = sum dEout x2, ds2 = sum dEout: rows staged in the dEout tile (read already)
+                row_store_fn(sb, r, [&](int c) { return d[c] * z[c]; });
+                __syncwarp();
+                float2 o = warp_tile_colsum(sbase + S::SB, w, lane);
+                acc[0] += o.x;
+                acc[1] += o.y;
+                __syncwarp();
+                row_store_fn(sb, r, [&](int c) { return d[c]; });
+                __syncwarp();
+                o = warp_tile_colsum(sbase + S::SB, w, lane);
+                acc[2] += o.x;
+                acc[3] += o.y;
+                __syncwarp();
             }
             float m1 = 0.f, m2 = 0.f;
 #pragma unroll
@@ -652,20 +707,16 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                 mma_wgrad(tmem + EB_TM_DW2, sbase + S::H, sbase + S::SB, any);
                 mma_commit(mmab);
             }
-            {
-                float o[2];
-                warp_colsum_of<64>([&](int c) { return d[c]; }, lane, o);
-                acc[4] += o[0];
-                acc[5] += o[1];
+            {   // db2 = sum dEz, from the dEz tile the products read
+                const float2 o = warp_tile_colsum(sbase + S::SB, w, lane);
+                acc[4] += o.x;
+                acc[5] += o.y;
             }
             cta_wait(mmab, mph, fail, p.status);
             mph ^= 1u;
             tc_fence_after();
-            // dh = dh' [h > 0] into the H tile (h is no longer read); db1 by halving,
-            // channels c and c + 64 together
+            // dh = dh' [h > 0] into the H tile (h is no longer read); db1 from that tile
             {
-                float v1[64];
-                const bool up = (lane & 16) != 0;
 #pragma unroll
                 for (int c0 = 0; c0 < 64; c0 += 16) {
                     float va[16], vb[16];
@@ -689,9 +740,6 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                         *reinterpret_cast<uint4 *>(half + sw128(r, ch)) = u0;
                         *reinterpret_cast<uint4 *>(half + sw128(r, ch + 1)) = u1;
                     }
-#pragma unroll
-                    for (int u = 0; u < 16; ++u)
-                        v1[c0 + u] = (up ? vb[u] : va[u]) + __shfl_xor_sync(0xffffffffu, up ? va[u] : vb[u], 16);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -704,19 +752,12 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                     mma_wgrad(tmem + EB_TM_DW1, sbase + S::H, sbase + S::SA, any);
                     mma_commit(mmab);
                 }
-#pragma unroll
-                for (int st = 1; st < 5; ++st) {
-                    const int o = 16 >> st, h = 128 >> (st + 1);
-                    const bool u2 = (lane & o) != 0;
-#pragma unroll
-                    for (int i = 0; i < h; ++i) {
-                        const float send = u2 ? v1[i] : v1[i + h];
-                        const float keep = u2 ? v1[i + h] : v1[i];
-                        v1[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) acc[10 + u] += v1[u];
+                const float2 o0 = warp_tile_colsum(sbase + S::H, w, lane);
+                const float2 o1 = warp_tile_colsum(sbase + S::H + EB_TILE, w, lane);
+                acc[10] += o0.x;
+                acc[11] += o0.y;
+                acc[12] += o1.x;
+                acc[13] += o1.y;
             }
             any = true;
             cta_wait(mmab, mph, fail, p.status);
@@ -729,14 +770,19 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
 #pragma unroll
                 for (int c = 0; c < 64; ++c) d[c] += v[c];
             }
-            {
-                float o[2];
-                warp_colsum_of<64>([&](int c) { return d[c] * pk_get(x1, c); }, lane, o);
-                acc[6] += o[0];
-                acc[7] += o[1];
-                warp_colsum_of<64>([&](int c) { return d[c]; }, lane, o);
-                acc[8] += o[0];
-                acc[9] += o[1];
+            {   // dg1 = sum dEa x1, ds1 = sum dEa: rows staged in the dEz tile (its products are done)
+                row_store_fn(sb, r, [&](int c) { return d[c] * pk_get(x1, c); });
+                __syncwarp();
+                float2 o = warp_tile_colsum(sbase + S::SB, w, lane);
+                acc[6] += o.x;
+                acc[7] += o.y;
+                __syncwarp();
+                row_store_fn(sb, r, [&](int c) { return d[c]; });
+                __syncwarp();
+                o = warp_tile_colsum(sbase + S::SB, w, lane);
+                acc[8] += o.x;
+                acc[9] += o.y;
+                __syncwarp();
             }
             float n1 = 0.f, n2 = 0.f;
 #pragma unroll
@@ -794,8 +840,10 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             pw[64 * q + 2 * lane] = acc[2 * q];
             pw[64 * q + 2 * lane + 1] = acc[2 * q + 1];
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) pw[320 + 4 * lane + u] = acc[10 + u];
+        pw[320 + 2 * lane] = acc[10];
+        pw[320 + 2 * lane + 1] = acc[11];
+        pw[384 + 2 * lane] = acc[12];
+        pw[384 + 2 * lane + 1] = acc[13];
         __syncthreads();
         for (int c = tid; c < EB_PART; c += EB_THR)
             p.parts[(size_t)blockIdx.x * EB_PART + c] = red[c] + red[EB_PART + c] + red[2 * EB_PART + c] +
