@@ -56,8 +56,7 @@ constexpr float LN_EPS = 1e-5f;
 // Forward shared memory (bytes from a 1024-aligned base).
 struct EfSmem {
     static constexpr uint32_t SLOT = 0;                  // 2 x 16 KB: E' tile -> Ea -> output
-    static constexpr uint32_t H = 2 * EB_TILE;           // 2 x 16 KB: relu(Ea W1 + b1), channels 0..63 | 64..127
-    static constexpr uint32_t W1 = H + 2 * EB_TILE;      // W1 [64][128] as two 64 x 64 boxes (8 KB each)
+    static constexpr uint32_t W1 = 2 * EB_TILE;          // W1 [64][128] as two 64 x 64 boxes (8 KB each)
     static constexpr uint32_t W2 = W1 + EB_TILE;         // W2 [128][64] as one box
     static constexpr uint32_t PAR = W2 + EB_TILE;        // fp32: g1, s1 [64], b1 [128], b2, g2, s2 [64]
     static constexpr uint32_t INFO = PAR + 448 * 4;      // per slot: column mask, row mask | live << 8
@@ -66,7 +65,10 @@ struct EfSmem {
     static constexpr uint32_t FAIL = TM + 8;
     static constexpr uint32_t BYTES = FAIL + 8 + 1024;
 };
-static_assert(EfSmem::BYTES <= 113 * 1024, "two CTAs per SM");
+static_assert(EfSmem::BYTES <= 74 * 1024, "three CTAs per SM");
+// TMEM columns of the forward: Ea W1 (fp32) 0..127; then h (bf16 pairs) 0..63
+// as the A operand of h W2, whose result lands in 64..127
+constexpr uint32_t EF_TM_COLS = 128, EF_TM_Z = 64;
 constexpr int PAR_G1 = 0, PAR_S1 = 64, PAR_B1 = 128, PAR_B2 = 256, PAR_G2 = 320, PAR_S2 = 384;
 
 // Backward shared memory: one E' tile (-> Ea), one dEout tile (-> dEz -> dE'),
@@ -338,6 +340,30 @@ __device__ __forceinline__ void h_epilogue(uint8_t *Ht, int r, uint32_t tl, cons
     }
 }
 
+// The forward's H epilogue in tensor memory: h = relu(T + b1) for the 128
+// columns of the thread's lane, stored back as bf16 pairs into columns
+// 0..63 (the A operand of h W2: row = lane, K along the columns).  Columns
+// are read 32 at a time in increasing order, so each store lands on columns
+// already read.
+__device__ __forceinline__ void h_epilogue_tmem(uint32_t tl, const float *b1) {
+#pragma unroll
+    for (int c0 = 0; c0 < EF; c0 += 32) {
+        float v[32];
+        tmem_ld16(tl + c0, *reinterpret_cast<float(*)[16]>(v));
+        tmem_ld16(tl + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; u += 2) {
+            const float4 q = par4(b1, c0 + 2 * u);
+            pk[u] = pack_bf16(fmaxf(v[2 * u] + q.x, 0.f), fmaxf(v[2 * u + 1] + q.y, 0.f));
+            pk[u + 1] = pack_bf16(fmaxf(v[2 * u + 2] + q.z, 0.f), fmaxf(v[2 * u + 3] + q.w, 0.f));
+        }
+        tmem_st16(tl + c0 / 2, pk);
+    }
+    tmem_st_wait();
+}
+
 // dh = dh' where the stored h > 0 (relu(x) > 0 exactly when x > 0), for 8
 // channels held as one 16-byte chunk of the H tile.
 __device__ __forceinline__ void relu_gate8(const uint4 hq, float *v) {
@@ -375,7 +401,7 @@ __device__ __forceinline__ void issue_tile(int t, int ntile, uint32_t slot_addr,
     }
 }
 
-__global__ void __launch_bounds__(EB_THR, 2)
+__global__ void __launch_bounds__(EB_THR, 3)
 k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUtensorMap tmOut,
            const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2, EbParams p) {
     using S = EfSmem;
@@ -399,7 +425,7 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         *fail = 0;
     }
     if (w == 0) {
-        tmem_alloc(sbase + S::TM, 128);
+        tmem_alloc(sbase + S::TM, EF_TM_COLS);
         tmem_relinquish();
     }
     load_params(par, p, tid, EB_THR);
@@ -496,13 +522,15 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         cta_wait(mmab, mph, fail, p.status);
         mph ^= 1u;
         tc_fence_after();
-        h_epilogue(sp + S::H, r, tl, par + PAR_B1);
-        fence_proxy_async_smem();
+        h_epilogue_tmem(tl, par + PAR_B1);
         tc_fence_before();
         named_bar_sync(1, EB_THR);
         if (r == 0 && !*fail) {
             tc_fence_after();
-            mma_tile(tmem, sbase + S::H, 8, sbase + S::W2, true, 0, idesc2);
+#pragma unroll 1
+            for (int kk = 0; kk < 8; ++kk)      // h (TMEM, 8 columns a k-step) x W2 (MN-major)
+                mma_bf16_ts(tmem + EF_TM_Z, tmem + kk * 8, smem_desc(sbase + S::W2 + kk * 2048, 8192, 1024, LAYOUT_SW128),
+                            idesc2, kk > 0 ? 1u : 0u);
             mma_commit(mmab);
         }
         cta_wait(mmab, mph, fail, p.status);
@@ -510,7 +538,7 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         tc_fence_after();
         {
             float v[64];
-            tmem_ld64(tl, v);
+            tmem_ld64(tl + EF_TM_Z, v);
             add_bias64(x, v, par, PAR_B2);
         }
         normalise64(x);
@@ -528,7 +556,7 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
     if (r == 0) tma_store_wait_all();
     tc_fence_before();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tmem, 128);
+    if (w == 0) tmem_dealloc(tmem, EF_TM_COLS);
 }
 
 // ------------------------------------------------------------------ backward
@@ -876,8 +904,8 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
 
 // ------------------------------------------------------------------ host
 
-static int grid_ctas(int ntile) {
-    const int g = 2 * sm_count();
+static int grid_ctas(int ntile, int per_sm) {
+    const int g = per_sm * sm_count();
     return ntile < g ? ntile : g;
 }
 
@@ -892,12 +920,12 @@ cudaError_t edge_forward(const EdgeArgs &a, cudaStream_t st) {
     const int ntile = a.B * p.ti * p.tj;
     static std::atomic<uint32_t> attr{0};
     if (cudaError_t e = ensure_smem_attr(k_eblk_fwd, EfSmem::BYTES, attr); e != cudaSuccess) return e;
-    k_eblk_fwd<<<grid_ctas(ntile), EB_THR, EfSmem::BYTES, st>>>(tIn, tOut, tW1, tW2, p);
+    k_eblk_fwd<<<grid_ctas(ntile, 3), EB_THR, EfSmem::BYTES, st>>>(tIn, tOut, tW1, tW2, p);
     return cudaGetLastError();
 }
 
 int edge_backward_ctas(int B, int n) {
-    return grid_ctas(B * ((n + 3) / 4) * ((n + 31) / 32));
+    return grid_ctas(B * ((n + 3) / 4) * ((n + 31) / 32), 2);
 }
 
 cudaError_t edge_backward(const EdgeArgs &a, cudaStream_t st) {
@@ -912,7 +940,7 @@ cudaError_t edge_backward(const EdgeArgs &a, cudaStream_t st) {
     const int ntile = a.B * p.ti * p.tj;
     static std::atomic<uint32_t> attr{0};
     if (cudaError_t e = ensure_smem_attr(k_eblk_bwd, EbSmem::BYTES, attr); e != cudaSuccess) return e;
-    k_eblk_bwd<<<grid_ctas(ntile), EB_THR, EbSmem::BYTES, st>>>(tIn, tDOut, tDIn, tW1, tW2, p);
+    k_eblk_bwd<<<grid_ctas(ntile, 2), EB_THR, EbSmem::BYTES, st>>>(tIn, tDOut, tDIn, tW1, tW2, p);
     return cudaGetLastError();
 }
 
