@@ -63,6 +63,8 @@ NCU_TRAFFIC = {
     ("large", "k_fwd_stream"): 736150000 + 481330000,
     ("large", "k_bwd_stream"): 1770000000 + 501140000,
     ("planar", "k_fwd_stream"): 39940000 + 848900,
+    ("sbm", "k_eblk_fwd"): 63142912 + 99683840,
+    ("sbm", "k_eblk_bwd"): 182036992 + 124005632,
 }
 
 

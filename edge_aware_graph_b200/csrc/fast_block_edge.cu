@@ -191,6 +191,21 @@ __device__ __forceinline__ void tile_masks(const uint8_t *M, int n, const TileAt
     rm = __ballot_sync(0xffffffffu, r) & 0xFu;
 }
 
+// The lane's node-mask bytes of tile t (column j0 + lane; row i0 + lane for
+// lanes < 4; 0 outside the graph or past the last tile), loaded one tile
+// before the ballot that turns them into the tile's masks, so the load's
+// latency is hidden behind a tile of work.
+__device__ __forceinline__ void mask_bytes(const uint8_t *M, int n, int t, int ti, int tj, int ntile, int lane,
+                                           uint32_t &c, uint32_t &r) {
+    c = 0;
+    r = 0;
+    if (t >= ntile) return;
+    const TileAt T = tile_at(t, ti, tj);
+    const uint8_t *mb = M + (size_t)T.b * n;
+    if (T.j0 + lane < n) c = mb[T.j0 + lane];
+    if (lane < 4 && T.i0 + lane < n) r = mb[T.i0 + lane];
+}
+
 // Row r of a 128B-swizzled [128][64] bf16 tile <-> 64 fp32 values.
 __device__ __forceinline__ void row_load64(const uint8_t *tile, int r, float (&x)[64]) {
 #pragma unroll
@@ -451,6 +466,8 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         }
         __syncwarp();
     }
+    uint32_t mc = 0, mr = 0;                     // warp 0: mask bytes of the tile after the next
+    if (w == 0) mask_bytes(p.M, p.n, blockIdx.x + G, p.ti, p.tj, ntile, lane, mc, mr);
     uint32_t mph = 0;
     bool wts_ready = false;
     float pool[2] = {0.f, 0.f};                  // lane's channels 2 lane, 2 lane + 1 of the current graph
@@ -468,7 +485,11 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         const uint32_t slot_a = sbase + S::SLOT + s * EB_TILE, next_a = sbase + S::SLOT + (s ^ 1) * EB_TILE;
         uint8_t *slot = sp + S::SLOT + s * EB_TILE;
         uint32_t cmn = 0, rmn = 0;
-        if (w == 0 && tn < ntile) tile_masks(p.M, p.n, tile_at(tn, p.ti, p.tj), lane, cmn, rmn);
+        if (w == 0) {
+            cmn = __ballot_sync(0xffffffffu, mc != 0);
+            rmn = __ballot_sync(0xffffffffu, mr != 0) & 0xFu;
+            mask_bytes(p.M, p.n, tn + G, p.ti, p.tj, ntile, lane, mc, mr);
+        }
         cta_wait(full(s), (k >> 1) & 1, fail, p.status);
         const uint32_t cm = info[2 * s], rmw = info[2 * s + 1];
         const TileAt T = tile_at(t, p.ti, p.tj);
@@ -643,6 +664,8 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
     int k = 0;
     for (int t = blockIdx.x; t < ntile; t += G, ++k) {
         const int tn = t + G;
+        uint32_t mc = 0, mr = 0;                 // warp 0: mask bytes of the next tile, used at the end
+        if (w == 0) mask_bytes(p.M, p.n, tn, p.ti, p.tj, ntile, lane, mc, mr);
         cta_wait(fullb, k & 1, fail, p.status);
         const uint32_t cm = info[0], rmw = info[1];
         const TileAt T = tile_at(t, p.ti, p.tj);
@@ -844,8 +867,8 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         tc_fence_before();
         named_bar_sync(1, EB_THR);
         if (w == 0) {
-            uint32_t cmn = 0, rmn = 0;
-            if (tn < ntile) tile_masks(p.M, p.n, tile_at(tn, p.ti, p.tj), lane, cmn, rmn);
+            const uint32_t cmn = __ballot_sync(0xffffffffu, mc != 0);
+            const uint32_t rmn = __ballot_sync(0xffffffffu, mr != 0) & 0xFu;
             if (lane == 0) {
                 if (!*fail) {
                     tma_store_4d(&tmDIn, sbase + S::SB, 0, T.j0, T.i0, T.b);
