@@ -65,6 +65,8 @@ NCU_TRAFFIC = {
     ("planar", "k_fwd_stream"): 39940000 + 848900,
     ("sbm", "k_eblk_fwd"): 63142912 + 99683840,
     ("sbm", "k_eblk_bwd"): 182036992 + 124005632,
+    ("large", "k_eblk_fwd"): 487750000 + 485110000,
+    ("large", "k_eblk_bwd"): 1040000000 + 510180000,
 }
 
 

@@ -383,50 +383,71 @@ __global__ void __launch_bounds__(256) k_y_bwd(YParams p) {
 }
 
 // The global sub-block's weight gradients and those of the pooling maps: one
-// thread per entry, summed over the graphs in order.
+// thread per entry, summed over the graphs in order (each region of entries a
+// plain loop over the graphs, so the loads of consecutive graphs overlap).
 __global__ void __launch_bounds__(256) k_y_wgrad(YParams p, YGrads gr) {
     const int dy = p.dy, fy = 2 * p.dy, dx = p.dx, B = p.B;
     const int nW1 = dy * fy, nW2 = fy * dy, nyx = dx * dy, nye = 64 * dy;
     const int total = nW1 + nW2 + nyx + nye + fy + 6 * dy;
+    const size_t vs = (size_t)YV_PER_DY * dy;                 // per-graph vector stride
+    const float *v0 = p.yv;
+    // offsets inside a graph's vectors: h, dh [fy]; ya, dyz, x1, dya, x2 [dy]
+    const int oh = 0, odh = fy, oya = 2 * fy, odyz = 2 * fy + dy, ox1 = 2 * fy + 2 * dy, odya = 2 * fy + 3 * dy,
+              ox2 = 2 * fy + 4 * dy;
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
         float a = 0.f;
         int q = e;
-        for (int b = 0; b < B; ++b) {
-            const float *v = p.yv + (size_t)b * YV_PER_DY * dy;
-            const float *h = v, *dh = v + fy, *ya = v + 2 * fy, *dyz = ya + dy, *x1 = dyz + dy, *dya = x1 + dy,
-                        *x2 = dya + dy;
-            const float *dy1 = p.dy1 + (size_t)b * dy;
-            q = e;
-            if (q < nW1) { a = fmaf(ya[q / fy], dh[q % fy], a); continue; }
-            q -= nW1;
-            if (q < nW2) { a = fmaf(h[q / dy], dyz[q % dy], a); continue; }
-            q -= nW2;
-            if (q < nyx) { a = fmaf(p.pX[(size_t)b * dx + q / dy], dy1[q % dy], a); continue; }
-            q -= nyx;
-            if (q < nye) { a = fmaf(p.pE[(size_t)b * 64 + q / dy], dy1[q % dy], a); continue; }
-            q -= nye;
-            if (q < fy) { a += dh[q]; continue; }
-            q -= fy;
-            const int k = q / dy, o = q % dy;
-            if (k == 0) a += dyz[o];                                              // b2
-            else if (k == 1) a = fmaf(bf(p.dyout, (size_t)b * dy + o), x2[o], a); // ln2 g
-            else if (k == 2) a += bf(p.dyout, (size_t)b * dy + o);                // ln2 s
-            else if (k == 3) a = fmaf(dya[o], x1[o], a);                          // ln1 g
-            else if (k == 4) a += dya[o];                                         // ln1 s
-            else a += dy1[o];                                                     // by
+        if (q < nW1) {
+            const int o = q / fy, f = q % fy;
+#pragma unroll 4
+            for (int b = 0; b < B; ++b) a = fmaf(v0[b * vs + oya + o], v0[b * vs + odh + f], a);
+            gr.W1[q] = a;
+            continue;
         }
-        q = e;
-        if (q < nW1) { gr.W1[q] = a; continue; }
         q -= nW1;
-        if (q < nW2) { gr.W2[q] = a; continue; }
+        if (q < nW2) {
+            const int f = q / dy, o = q % dy;
+#pragma unroll 4
+            for (int b = 0; b < B; ++b) a = fmaf(v0[b * vs + oh + f], v0[b * vs + odyz + o], a);
+            gr.W2[q] = a;
+            continue;
+        }
         q -= nW2;
-        if (q < nyx) { gr.Wyx[q] = a; continue; }
+        if (q < nyx) {
+            const int k = q / dy, o = q % dy;
+#pragma unroll 4
+            for (int b = 0; b < B; ++b) a = fmaf(p.pX[(size_t)b * dx + k], p.dy1[(size_t)b * dy + o], a);
+            gr.Wyx[q] = a;
+            continue;
+        }
         q -= nyx;
-        if (q < nye) { gr.Wye[q] = a; continue; }
+        if (q < nye) {
+            const int k = q / dy, o = q % dy;
+#pragma unroll 4
+            for (int b = 0; b < B; ++b) a = fmaf(p.pE[(size_t)b * 64 + k], p.dy1[(size_t)b * dy + o], a);
+            gr.Wye[q] = a;
+            continue;
+        }
         q -= nye;
-        if (q < fy) { gr.b1[q] = a; continue; }
+        if (q < fy) {
+#pragma unroll 4
+            for (int b = 0; b < B; ++b) a += v0[b * vs + odh + q];
+            gr.b1[q] = a;
+            continue;
+        }
         q -= fy;
         const int k = q / dy, o = q % dy;
+#pragma unroll 4
+        for (int b = 0; b < B; ++b) {
+            const float *v = v0 + b * vs;
+            const float up = bf(p.dyout, (size_t)b * dy + o);
+            a += k == 0 ? v[odyz + o]                         // b2
+               : k == 1 ? up * v[ox2 + o]                     // ln2 g
+               : k == 2 ? up                                  // ln2 s
+               : k == 3 ? v[odya + o] * v[ox1 + o]            // ln1 g
+               : k == 4 ? v[odya + o]                         // ln1 s
+                        : p.dy1[(size_t)b * dy + o];          // by
+        }
         float *dst = k == 0 ? gr.b2 : k == 1 ? gr.g2 : k == 2 ? gr.s2 : k == 3 ? gr.g1 : k == 4 ? gr.s1 : gr.by;
         dst[o] = a;
     }
@@ -555,7 +576,7 @@ BlockWs block_ws_layout(int B, int n, int dx, int dy, size_t base, int for_backw
         L.ln_grid = 148;
         L.ln2 = off; off = align256(off + (size_t)L.ln_grid * 2 * dx * 4);
         L.ln1 = off; off = align256(off + (size_t)L.ln_grid * 2 * dx * 4);
-        L.cs_rows = 64;
+        L.cs_rows = 16;
         L.cs_grid = (int)((R + L.cs_rows - 1) / L.cs_rows);
         L.cs1 = off; off = align256(off + (size_t)L.cs_grid * 2 * dx * 4);
         L.cs2 = off; off = align256(off + (size_t)L.cs_grid * dx * 4);
