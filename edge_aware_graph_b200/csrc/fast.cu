@@ -20,7 +20,8 @@ cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs 
                              cudaStream_t st);
 cudaError_t launch_kv_convert(const eaga_dims &d, const FastWs &W, char *ws, cudaStream_t st);
 cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
-cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
+cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, int part,
+                             cudaStream_t st);
 
 bool supports(const eaga_dims &d) {
     return d.dtype == EAGA_BF16 && d.de == DE && d.H == NH && d.dh == DH && d.n % 2 == 0 && d.n >= 2 &&
@@ -38,8 +39,8 @@ size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, s
 int kernel_launches(const eaga_dims &, int for_backward) {
     // forward: prologue, QKV, pairs, out-proj
     // backward: prologue, dO, pairs, dk/dv conversion, dX, wgrad x2, bias partial, rparts partial,
-    // finish, film grads
-    return for_backward ? 11 : 4;
+    // finish x2, film grads
+    return for_backward ? 12 : 4;
 }
 
 #define FAST_TRY(x)                               \
@@ -171,13 +172,17 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         const size_t msz = (size_t)W.wsplits * d.dx * HD;
         const void *Bq[3] = {dN[0], dN[1], dN[2]}, *Bo[3] = {a.dXout, a.dXout, a.dXout};
         float *const Pq[3] = {parts, parts + msz, parts + 2 * msz}, *const Po[3] = {parts + 3 * msz, nullptr, nullptr};
+        // dW{q,k,v} and their final sums on one auxiliary stream; dWo, the
+        // bias and row-block partials and the rest of the sums on the other
         FAST_TRY(tc_wgrad(d.dx, HD, 3, rows, W.wsplits, a.X, Bq, Pq, a.status, s1));
-        FAST_TRY(tc_wgrad(HD, d.dx, 1, rows, W.wsplits, a.O, Bo, Po, a.status, s1));
+        FAST_TRY(launch_bwd_final(d, a, W, ws, 0, s1));
+        FAST_TRY(tc_wgrad(HD, d.dx, 1, rows, W.wsplits, a.O, Bo, Po, a.status, s2));
     }
     FAST_TRY(launch_bwd_partials(d, a, W, ws, s2));   // bias and row-block partials, dg, dbf, dWfy, dy
+    FAST_TRY(launch_bwd_final(d, a, W, ws, 1, s2));
     FAST_TRY(stream_after(st, s1, ev[4]));
     FAST_TRY(stream_after(st, s2, ev[5]));
-    return launch_bwd_final(d, a, W, ws, st);
+    return cudaSuccess;
 }
 
 }  // namespace fast

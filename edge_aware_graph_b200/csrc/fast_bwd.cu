@@ -100,8 +100,9 @@ struct DWPtrs {
 // Final sums: weight gradients of the four node projections (split-K
 // partials), bias gradients, dWfe / dWe.
 __global__ void k_bwd_finish(const float *wparts, int wsplits, const float *bparts, int bsplits,
-                             const float *r2, int rsplits, int dx, DWPtrs dW, int zero_wfe) {
-    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+                             const float *r2, int rsplits, int dx, DWPtrs dW, int zero_wfe, int e0, int e1) {
+    const int e = e0 + blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= e1) return;
     const int msz = dx * HD;
     const int ncol = 3 * HD + dx;
     constexpr int NE = DE * NF + NH * DE;
@@ -215,17 +216,22 @@ cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const Fast
     return cudaGetLastError();
 }
 
-// Final sums of the node projections' weight and bias gradients and of dWfe, dWe.
-cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st) {
+// Final sums of the node projections' weight and bias gradients and of dWfe,
+// dWe: entries [e0, e1) of dWq, dWk, dWv, dWo, the biases, dWfe, dWe (in that
+// order; part 0 = dWq, dWk, dWv, part 1 = the rest), so that each part runs
+// on the stream that produced its partials.
+cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, int part,
+                             cudaStream_t st) {
     const int ncol = 3 * HD + d.dx;
     constexpr int NE = DE * NF + NH * DE;
     DWPtrs dWdev;
     for (int q = 0; q < 12; ++q) dWdev.p[q] = a.dW[q];
-    const int total = 4 * d.dx * HD + ncol + NE;
-    k_bwd_finish<<<(total + 255) / 256, 256, 0, st>>>(
+    const int total = 4 * d.dx * HD + ncol + NE, split = 3 * d.dx * HD;
+    const int e0 = part == 0 ? 0 : split, e1 = part == 0 ? split : total;
+    k_bwd_finish<<<(e1 - e0 + 255) / 256, 256, 0, st>>>(
         reinterpret_cast<const float *>(ws + W.wparts), W.wsplits, reinterpret_cast<const float *>(ws + W.bparts),
         W.bsplits, reinterpret_cast<const float *>(ws + W.r2), W.rsplits, d.dx, dWdev,
-        a.variant == EAGA_VARIANT_LIGHT_EDGE);
+        a.variant == EAGA_VARIANT_LIGHT_EDGE, e0, e1);
     return cudaGetLastError();
 }
 
