@@ -20,7 +20,7 @@ So, as for any decision floating point takes, both sides must take it alike:
     whose pre-activation lies inside the rounding band (either side valid).
 
 Cases span several 4 x 32 pair tiles with a ragged tail (n = 30, 96, 100,
-192, 288), masks with empty and single-node graphs, tiles without a valid
+192, 288, 544), masks with empty and single-node graphs, tiles without a valid
 pair between live ones, and the smallest graph (n = 2)."""
 import numpy as np
 import pytest
@@ -84,6 +84,7 @@ CASES = [
     (1, 288, "prefix", 15),     # 9 column tiles, 72 row tiles
     (2, 100, "random", 16),     # ragged rows and columns
     (3, 2, "full", 17),         # the smallest graph
+    (1, 544, "random", 18),     # the layer's columns over clusters of 4 CTAs under the block
 ]
 
 
