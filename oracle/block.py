@@ -23,6 +23,13 @@ LN: LayerNorm over the last axis, biased variance, eps = 1e-5.  FFN widths
 2*dx, 2*de, 2*dy.  Weights are [in, out] (Y = X W).  The backward is the
 chain rule of b0..b4 written out step by step.
 
+Storage: with storage="bf16" the block's inputs X', E' are the layer's
+outputs rounded to bfloat16 (round to nearest even), as a bf16 layer stores
+them; everything after that is fp64.  The pooled means are sensitive to that
+rounding: E' of many pairs shares a few values (the edge features of a graph
+come from few classes), so their rounding errors do not average out, while
+the mean over pairs of unit-size channels can be near zero.
+
 Pins (tests/test_block_oracle.py): the LayerNorm closed form, torch's
 float64 LayerNorm/Linear/ReLU modules and autograd for each sub-block,
 masked outputs, the pooling's independence of padding, and central finite
@@ -46,6 +53,17 @@ BLOCK_WEIGHT_NAMES = tuple(f"{s}_{k}" for s in SUBS for k in SUB_PARAMS) + ("Wyx
 
 def _f64(a):
     return np.asarray(a, dtype=np.float64)
+
+
+def round_bf16(a):
+    """a rounded to the nearest bfloat16 (ties to even), via its float32 bits."""
+    bits = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) & 0xFFFF0000
+    return bits.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _storage(a, storage):
+    return round_bf16(a) if storage == "bf16" else _f64(a)
 
 
 def layer_norm(z, g, s):
@@ -124,11 +142,11 @@ def block_tail_forward(Xm, Em, y, M, Wb):
     return out, dict(x=cx, e=ce, y=cy)
 
 
-def block_forward(dims: dict, X, E, y, M, W: dict, Wb: dict):
+def block_forward(dims: dict, X, E, y, M, W: dict, Wb: dict, storage: str = "fp64"):
     """b0-b4: the layer (C oracle) then the block.  Returns Xout, Eout, yout
     and the intermediates Xmid (X'), Emid (E'), y1, pX, pE."""
     lay = layer_forward(dims, X, E, y, M, W)
-    out, _ = block_tail_forward(lay["Xout"], lay["Eout"], y, M, Wb)
+    out, _ = block_tail_forward(_storage(lay["Xout"], storage), _storage(lay["Eout"], storage), y, M, Wb)
     return out
 
 
@@ -154,11 +172,12 @@ def block_tail_backward(Xm, Em, y, M, Wb, dXout, dEout, dyout):
     return dXm, dEm, dy1, grads
 
 
-def block_backward(dims: dict, X, E, y, M, W: dict, Wb: dict, dXout, dEout, dyout):
+def block_backward(dims: dict, X, E, y, M, W: dict, Wb: dict, dXout, dEout, dyout, storage: str = "fp64"):
     """Gradients of the whole block (layer included): dX, dE, dy, the layer's
     d<weight> and the block's d<name> for every name of BLOCK_WEIGHT_NAMES."""
     lay = layer_forward(dims, X, E, y, M, W)
-    dXm, dEm, dy1, gb = block_tail_backward(lay["Xout"], lay["Eout"], y, M, Wb, dXout, dEout, dyout)
+    dXm, dEm, dy1, gb = block_tail_backward(_storage(lay["Xout"], storage), _storage(lay["Eout"], storage), y, M,
+                                            Wb, dXout, dEout, dyout)
     g = layer_backward(dims, X, E, y, M, W, dXm, dEm)
     out = {"dX": g["dX"], "dE": g["dE"], "dy": g["dy"] + dy1, "dXmid": dXm, "dEmid": dEm, "dy1": dy1}
     for k, v in g.items():

@@ -94,7 +94,7 @@ def test_block_matches_oracle(case):
     B, n, mask, seed = case
     p, d, W, Wb, dyo, buf = _run(B, n, mask, seed)
     dims = dict(H=p.H, dh=p.dh)
-    fwd = OB.block_forward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb)
+    fwd = OB.block_forward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, storage=p.dtype)
     errs, bad = _errs({"Xmid": (buf.Xmid, fwd["Xmid"]), "Emid": (buf.Emid, fwd["Emid"]),
                        "Xout": (buf.Xout, fwd["Xout"]), "Eout": (buf.Eout, fwd["Eout"]),
                        "yout": (buf.yout, fwd["yout"])})
@@ -105,7 +105,8 @@ def test_block_matches_oracle(case):
     valid = M[:, :, None] & M[:, None, :]
     assert torch.all(buf.Eout[~valid] == 0)
 
-    g = OB.block_backward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, d["dXout"], d["dEout"], dyo)
+    g = OB.block_backward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, d["dXout"], d["dEout"], dyo,
+                          storage=p.dtype)
     pairs = {"dEmid": (buf.dEmid, g["dEmid"]), "dX": (buf.dX, g["dX"]), "dE": (buf.dE, g["dE"]),
              "dy": (buf.dy, g["dy"])}
     pairs.update({"d" + k: (buf.dW[k], g["d" + k]) for k in I.WEIGHT_NAMES})
@@ -135,8 +136,9 @@ def test_block_random_weights(case):
     B, n, mask, seed = case
     p, d, W, Wb, dyo, buf = _run(B, n, mask, seed, margins=False)
     dims = dict(H=p.H, dh=p.dh)
-    fwd = OB.block_forward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb)
-    g = OB.block_backward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, d["dXout"], d["dEout"], dyo)
+    fwd = OB.block_forward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, storage=p.dtype)
+    g = OB.block_backward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, d["dXout"], d["dEout"], dyo,
+                          storage=p.dtype)
     pairs = {k: (getattr(buf, k), fwd[k]) for k in ("Xmid", "Emid", "Xout", "Eout", "yout")}
     for s in ("x", "e", "y"):
         for k in ("W2", "b2", "ln2_g", "ln2_s"):
@@ -161,8 +163,9 @@ def test_block_dx512():
     """The node sub-block at dx = 512 (FFN width 1024)."""
     p, d, W, Wb, dyo, buf = _run(2, 64, "random", 21, dx=512)
     dims = dict(H=p.H, dh=p.dh)
-    fwd = OB.block_forward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb)
-    g = OB.block_backward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, d["dXout"], d["dEout"], dyo)
+    fwd = OB.block_forward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, storage=p.dtype)
+    g = OB.block_backward(dims, d["X"], d["E"], d["y"], d["M"], W, Wb, d["dXout"], d["dEout"], dyo,
+                          storage=p.dtype)
     pairs = {"Xout": (buf.Xout, fwd["Xout"]), "yout": (buf.yout, fwd["yout"]), "dX": (buf.dX, g["dX"]),
              "dx_W1": (buf.dWb["x_W1"], g["dx_W1"]), "dx_W2": (buf.dWb["x_W2"], g["dx_W2"]),
              "dx_ln1_g": (buf.dWb["x_ln1_g"], g["dx_ln1_g"])}
@@ -178,7 +181,7 @@ def test_two_block_stack():
     Wl2 = I.draw_weights(p, seed_offset=1500)
     Wb1 = _margin_block_weights(p, d, Wl1, I.draw_block_weights(p))
     dims = dict(H=p.H, dh=p.dh)
-    o1 = OB.block_forward(dims, d["X"], d["E"], d["y"], d["M"], Wl1, Wb1)
+    o1 = OB.block_forward(dims, d["X"], d["E"], d["y"], d["M"], Wl1, Wb1, storage=p.dtype)
     Wb2 = _margin_block_weights(p, d, Wl2, I.draw_block_weights(p, seed_offset=2500),
                                 X=o1["Xout"], E=o1["Eout"], y=o1["yout"])
     dyo = I.draw_block_upstream(p)
@@ -200,9 +203,11 @@ def test_two_block_stack():
     b1.block_backward()
     torch.cuda.synchronize()
 
-    o2 = OB.block_forward(dims, o1["Xout"], o1["Eout"], o1["yout"], d["M"], Wl2, Wb2)
-    g2 = OB.block_backward(dims, o1["Xout"], o1["Eout"], o1["yout"], d["M"], Wl2, Wb2, d["dXout"], d["dEout"], dyo)
-    g1 = OB.block_backward(dims, d["X"], d["E"], d["y"], d["M"], Wl1, Wb1, g2["dX"], g2["dE"], g2["dy"])
+    o2 = OB.block_forward(dims, o1["Xout"], o1["Eout"], o1["yout"], d["M"], Wl2, Wb2, storage=p.dtype)
+    g2 = OB.block_backward(dims, o1["Xout"], o1["Eout"], o1["yout"], d["M"], Wl2, Wb2, d["dXout"], d["dEout"], dyo,
+                           storage=p.dtype)
+    g1 = OB.block_backward(dims, d["X"], d["E"], d["y"], d["M"], Wl1, Wb1, g2["dX"], g2["dE"], g2["dy"],
+                           storage=p.dtype)
     pairs = {"Xout2": (b2.Xout, o2["Xout"]), "Eout2": (b2.Eout, o2["Eout"]), "yout2": (b2.yout, o2["yout"]),
              "dX": (b1.dX, g1["dX"]), "dE": (b1.dE, g1["dE"]), "dy": (b1.dy, g1["dy"]),
              "dWq1": (b1.dW["Wq"], g1["dWq"]), "de_W1_1": (b1.dWb["e_W1"], g1["de_W1"]),

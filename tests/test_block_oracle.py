@@ -39,6 +39,14 @@ def test_block_weight_names_agree_with_the_input_generator():
     assert OB.BLOCK_WEIGHT_NAMES == I.BLOCK_WEIGHT_NAMES
 
 
+def test_round_bf16_against_torch():
+    rng = _rng(2)
+    x = np.concatenate([rng.standard_normal(5000) * 10.0 ** rng.integers(-6, 6, 5000),
+                        [0.0, -0.0, 1.0, 1.00390625, 1.01171875, -3.0078125]])
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(OB.round_bf16(x), ref)
+
+
 def test_layer_norm_closed_form():
     rng = _rng(1)
     z = rng.standard_normal((50, 64)) * rng.uniform(0.01, 5, (50, 1)) + rng.standard_normal((50, 1))
