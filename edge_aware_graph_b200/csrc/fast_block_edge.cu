@@ -27,16 +27,19 @@
 // (dpE_b: the global update's gradient of the edge pooling, already divided
 // by the pair count).  The four products and the two weight-gradient products
 // (M = 128 over the tile's 128 pairs, accumulated in TMEM over the CTA's
-// tiles) run on the tensor cores; the per-channel sums run per warp with
-// shuffles; each CTA writes its partial sums once.
+// tiles) run on the tensor cores; the per-channel sums are column sums on
+// the warps' tensor cores (a ones matrix times the warp's rows staged as bf16
+// in a tile already held); each CTA writes its partial sums once.
 //
 // Four warps, one pair row per thread; thread 0 also issues the MMAs (after
-// a named barrier of the CTA) and the TMA loads and stores, and warp 0 computes
-// each tile's validity masks one tile ahead.  The forward double-buffers its
-// tiles (the next tile's load is issued with the current tile's first
-// product); the backward holds one tile pair and prefetches the next into L2.
-// Persistent grid, two CTAs per SM (8 warps: 255 registers a thread), tiles
-// taken in a stride of the grid size.
+// a named barrier of the CTA) and the TMA loads and stores, and warp 0 loads
+// the node-mask bytes of a tile one tile before its validity masks are
+// needed.  The forward double-buffers its tiles (the next tile's load is
+// issued with the current tile's first product) and keeps h in tensor memory
+// as the A operand of h W2, so three CTAs fit an SM; the backward holds one
+// tile pair, prefetches the next into L2 and runs two CTAs per SM (8 warps:
+// 255 registers a thread).  Persistent grids, tiles taken in a stride of the
+// grid size.
 #include "fast.h"
 #include "fast_common.cuh"
 #include "fast_block.h"
@@ -89,33 +92,6 @@ struct EbSmem {
 static_assert(EbSmem::BYTES <= 113 * 1024, "two CTAs per SM");
 // TMEM columns of the backward: the tile's products 0..127, dW2 128..191, dW1^T 192..255
 constexpr uint32_t EB_TM_COLS = 256, EB_TM_DW2 = 128, EB_TM_DW1 = 192;
-
-// Sum over the 32 lanes of the warp of f(c) for channels c < N, by halving:
-// the first step pairs channels c and c + N/2 as they are computed, so only
-// N/2 values are live.  On return out[i] of lane l is channel (N/32) l + i.
-template <int N, class F>
-__device__ __forceinline__ void warp_colsum_of(F f, int lane, float (&out)[N / 32]) {
-    float v[N / 2];
-    const bool up = (lane & 16) != 0;
-#pragma unroll
-    for (int i = 0; i < N / 2; ++i) {
-        const float a = f(i), b = f(i + N / 2);
-        v[i] = (up ? b : a) + __shfl_xor_sync(0xffffffffu, up ? a : b, 16);
-    }
-#pragma unroll
-    for (int s = 1; s < 5; ++s) {
-        const int o = 16 >> s, h = N >> (s + 1);
-        const bool u2 = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < h; ++i) {
-            const float send = u2 ? v[i] : v[i + h];
-            const float keep = u2 ? v[i + h] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < N / 32; ++i) out[i] = v[i];
-}
 
 // Column sums over the warp's 32 rows (32 w .. 32 w + 31) of a 128B-swizzled
 // [128][64] bf16 tile, on the warp's tensor cores: D = ones(16 x 16) B with B
