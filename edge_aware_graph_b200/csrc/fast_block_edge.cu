@@ -377,8 +377,9 @@ __device__ __forceinline__ float pk_get(const uint32_t (&p)[32], int c) {
 // valid pair), after the bulk stores issued so far have read their tiles.
 __device__ __forceinline__ void issue_tile(int t, int ntile, uint32_t slot_addr, uint32_t full, uint32_t *info,
                                            uint32_t cm, uint32_t rm, const CUtensorMap *map, const EbParams &p,
-                                           volatile int *fail) {
+                                           volatile int *fail, uint32_t &issued) {
     if (t >= ntile) return;
+    ++issued;                                    // one phase of `full` per call
     tma_store_wait_read0();
     const bool live = cm != 0 && rm != 0;
     info[0] = cm;
@@ -430,6 +431,9 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
     const uint32_t idesc1 = idesc_bf16_f32(128, EF) | (1u << 16);
     const uint32_t idesc2 = idesc_bf16_f32(128, 64) | (1u << 16);
 
+    // thread 0's count of the phases it started on each slot's load barrier and
+    // of its MMA commits: on a failed wait, what it issued completes before exit
+    uint32_t nfull[2] = {0u, 0u}, ncommit = 0;
     if (w == 0 && (int)blockIdx.x < ntile) {
         uint32_t cm, rm;
         tile_masks(p.M, p.n, tile_at(blockIdx.x, p.ti, p.tj), lane, cm, rm);
@@ -438,7 +442,7 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
             tma_load_2d(sbase + S::W1, &tmW1, wtsb, 0, 0);
             tma_load_2d(sbase + S::W1 + 8192, &tmW1, wtsb, 64, 0);
             tma_load_2d(sbase + S::W2, &tmW2, wtsb, 0, 0);
-            issue_tile(blockIdx.x, ntile, sbase + S::SLOT, full(0), info, cm, rm, &tmIn, p, fail);
+            issue_tile(blockIdx.x, ntile, sbase + S::SLOT, full(0), info, cm, rm, &tmIn, p, fail, nfull[0]);
         }
         __syncwarp();
     }
@@ -484,7 +488,7 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                     tma_store_4d(&tmOut, slot_a, 0, T.j0, T.i0, T.b);
                     tma_store_commit();
                 }
-                issue_tile(tn, ntile, next_a, full(s ^ 1), info + 2 * (s ^ 1), cmn, rmn, &tmIn, p, fail);
+                issue_tile(tn, ntile, next_a, full(s ^ 1), info + 2 * (s ^ 1), cmn, rmn, &tmIn, p, fail, nfull[s ^ 1]);
             }
             continue;
         }
@@ -513,8 +517,9 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                 tc_fence_after();
                 mma_tile(tmem, slot_a, 4, sbase + S::W1, true, 0, idesc1);
                 mma_commit(mmab);
+                ++ncommit;
             }
-            issue_tile(tn, ntile, next_a, full(s ^ 1), info + 2 * (s ^ 1), cmn, rmn, &tmIn, p, fail);
+            issue_tile(tn, ntile, next_a, full(s ^ 1), info + 2 * (s ^ 1), cmn, rmn, &tmIn, p, fail, nfull[s ^ 1]);
         }
         cta_wait(mmab, mph, fail, p.status);
         mph ^= 1u;
@@ -529,6 +534,7 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                 mma_bf16_ts(tmem + EF_TM_Z, tmem + kk * 8, smem_desc(sbase + S::W2 + kk * 2048, 8192, 1024, LAYOUT_SW128),
                             idesc2, kk > 0 ? 1u : 0u);
             mma_commit(mmab);
+                ++ncommit;
         }
         cta_wait(mmab, mph, fail, p.status);
         mph ^= 1u;
@@ -550,7 +556,15 @@ k_eblk_fwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
         }
     }
     flush_pool();
-    if (r == 0) tma_store_wait_all();
+    if (r == 0) {
+        if (*fail) {   // (bounded) the products and loads already issued land before the memory is released
+            mma_commit(mmab);
+            mbar_wait(mmab, ncommit & 1u);
+            for (int s = 0; s < 2; ++s)
+                if (nfull[s]) mbar_wait(full(s), (nfull[s] - 1u) & 1u);
+        }
+        tma_store_wait_all();
+    }
     tc_fence_before();
     __syncthreads();
     if (w == 0) tmem_dealloc(tmem, EF_TM_COLS);
@@ -597,9 +611,13 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
     const uint32_t idesc_dh = idesc_bf16_f32(128, EF);                // dEz W2^T: B K-major
     const uint32_t idesc_da = idesc_bf16_f32(128, 64);                // dh W1^T: B K-major
 
+    // thread 0's count of the phases it started on the load barrier and of its
+    // MMA commits: on a failed wait, what it issued completes before exit
+    uint32_t nfull = 0, ncommit = 0;
     // thread 0: the loads of tile t (E' and dEout) and an L2 prefetch of the CTA's next tile
     auto issue = [&](int t, uint32_t cm, uint32_t rm) {
         if (t >= ntile) return;
+        ++nfull;
         tma_store_wait_read0();
         const bool live = cm != 0 && rm != 0;
         info[0] = cm;
@@ -667,6 +685,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                 tc_fence_after();
                 mma_tile(tmem, sbase + S::SA, 4, sbase + S::W1, true, 0, idesc_h);
                 mma_commit(mmab);
+                ++ncommit;
             }
             cta_wait(mmab, mph, fail, p.status);
             mph ^= 1u;
@@ -679,6 +698,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                 tc_fence_after();
                 mma_tile(tmem, sbase + S::H, 8, sbase + S::W2, true, 0, idesc_z);
                 mma_commit(mmab);
+                ++ncommit;
             }
             cta_wait(mmab, mph, fail, p.status);
             mph ^= 1u;
@@ -733,6 +753,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                 mma_tile(tmem, sbase + S::SB, 4, sbase + S::W2, false, 0, idesc_dh);
                 mma_wgrad(tmem + EB_TM_DW2, sbase + S::H, sbase + S::SB, any);
                 mma_commit(mmab);
+                ++ncommit;
             }
             {   // db2 = sum dEz, from the dEz tile the products read
                 const float2 o = warp_tile_colsum(sbase + S::SB, w, lane);
@@ -778,6 +799,7 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                     mma_tile(tmem, sbase + S::H, 8, sbase + S::W1, false, 8192, idesc_da);
                     mma_wgrad(tmem + EB_TM_DW1, sbase + S::H, sbase + S::SA, any);
                     mma_commit(mmab);
+                ++ncommit;
                 }
                 const float2 o0 = warp_tile_colsum(sbase + S::H, w, lane);
                 const float2 o1 = warp_tile_colsum(sbase + S::H + EB_TILE, w, lane);
@@ -895,7 +917,14 @@ k_eblk_bwd(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUt
                             : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
-    if (r == 0) tma_store_wait_all();
+    if (r == 0) {
+        if (*fail) {   // (bounded) the products and loads already issued land before the memory is released
+            mma_commit(mmab);
+            mbar_wait(mmab, ncommit & 1u);
+            if (nfull) mbar_wait(fullb, (nfull - 1u) & 1u);
+        }
+        tma_store_wait_all();
+    }
     tc_fence_before();
     __syncthreads();
     if (w == 0) tmem_dealloc(tmem, EB_TM_COLS);
