@@ -19,6 +19,8 @@ cudaError_t tc_wgrad(int M, int Nb, int nout, int K, int splits, const void *A, 
 cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,
                              cudaStream_t st);
 cudaError_t launch_kv_convert(const eaga_dims &d, const FastWs &W, char *ws, cudaStream_t st);
+cudaError_t launch_row_block_order(const eaga_dims &d, const uint8_t *M, int row0, int rows, int *order,
+                                   cudaStream_t st);
 cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
 cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, int part,
                              cudaStream_t st);
@@ -38,9 +40,9 @@ size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, s
 
 int kernel_launches(const eaga_dims &, int for_backward) {
     // forward: prologue, QKV, pairs, out-proj
-    // backward: prologue, dO, pairs, dk/dv conversion, dX, wgrad x2, bias partial, rparts partial,
-    // finish x2, film grads
-    return for_backward ? 12 : 4;
+    // backward: prologue, dO, row-block order, pairs, dk/dv conversion, dX, wgrad x2, bias partial,
+    // rparts partial, finish x2, film grads
+    return for_backward ? 13 : 4;
 }
 
 #define FAST_TRY(x)                               \
@@ -148,6 +150,10 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         FAST_TRY(cudaMemsetAsync(ws + W.dQ, 0, (size_t)rows * HD * 2, s1));
         FAST_TRY(cudaMemsetAsync(ws + W.rparts, 0, (size_t)W.n_rparts * RPART * 4, s1));
     }
+    // the order of the row blocks for the pair kernel (longest first) and the
+    // prologue, beside dO
+    FAST_TRY(launch_row_block_order(d, a.M, a.row0, a.rows < 0 ? d.n : a.rows, reinterpret_cast<int *>(ws + W.order),
+                                    st));
     FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, st));
     FAST_TRY(stream_after(st, s1, ev[1]));
 

@@ -148,6 +148,75 @@ __global__ void k_film_grads(const float *dg, int B, int dy, const __nv_bfloat16
     }
 }
 
+// The order in which a pair kernel's CTAs take the row blocks: longest first
+// (the most chunks with a valid pair), graph-major among equals, so that the
+// short row blocks (few live chunks, or none: only copies) fill the last
+// wave instead of leaving SMs idle behind a long one.  A row block's live
+// chunks are the graph's chunks holding a node when one of its rows is a
+// node, none otherwise (exactly live_chunk_mask's count).  One CTA: per
+// graph the chunks holding a node (a warp a graph), per row block whether a
+// row is a node, then a stable counting sort on the count (bin k: 32 - k live
+// chunks).  Item = graph * row blocks of the slab + row block.
+__global__ void __launch_bounds__(1024) k_row_block_order(const uint8_t *M, int B, int n, int row0, int rows,
+                                                          int *order) {
+    __shared__ uint8_t cost[ORDER_MAX_ITEMS];
+    __shared__ uint8_t gcount[ORDER_MAX_ITEMS];
+    __shared__ int bin_start[33];
+    const int nrb = (rows + TB - 1) / TB, items = B * nrb;
+    const int w = threadIdx.x >> 5, t = threadIdx.x & 31;
+    if (items > ORDER_MAX_ITEMS) {
+        for (int i = threadIdx.x; i < items; i += blockDim.x) order[i] = i;
+        return;
+    }
+    if (threadIdx.x < 33) bin_start[threadIdx.x] = 0;
+    for (int g = w; g < B; g += 32) {   // chunks of graph g holding a node (n even: 2-byte loads)
+        const uint16_t *m2 = reinterpret_cast<const uint16_t *>(M + (size_t)g * n);
+        uint32_t any = 0;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int j = 32 * t + 2 * k;
+            if (j < n) any |= m2[j >> 1];
+        }
+        const uint32_t gm = __ballot_sync(0xffffffffu, any != 0);
+        if (t == 0) gcount[g] = (uint8_t)__popc(gm);
+    }
+    __syncthreads();
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+        const int b = it / nrb, i0 = row0 + (it % nrb) * TB;
+        bool row = false;
+        for (int k = 0; k < TB; ++k) row |= i0 + k < n && M[(size_t)b * n + i0 + k] != 0;
+        const int c = row ? gcount[b] : 0;
+        cost[it] = (uint8_t)c;
+        atomicAdd(&bin_start[32 - c], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {   // counts -> where each bin starts
+        int acc = 0;
+        for (int k = 0; k < 33; ++k) {
+            const int c = bin_start[k];
+            bin_start[k] = acc;
+            acc += c;
+        }
+    }
+    __syncthreads();
+    for (int k = w; k <= 32; k += 32) {
+        int pos = bin_start[k];
+        for (int base = 0; base < items; base += 32) {
+            const int it = base + t;
+            const bool mine = it < items && 32 - cost[it] == k;
+            const uint32_t bal = __ballot_sync(0xffffffffu, mine);
+            if (mine) order[pos + __popc(bal & ((1u << t) - 1u))] = it;
+            pos += __popc(bal);
+        }
+    }
+}
+
+cudaError_t launch_row_block_order(const eaga_dims &d, const uint8_t *M, int row0, int rows, int *order,
+                                   cudaStream_t st) {
+    k_row_block_order<<<1, 1024, 0, st>>>(M, d.B, d.n, row0, rows, order);
+    return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- host side
 
 cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, const float *g,

@@ -100,6 +100,7 @@ __device__ __forceinline__ uint32_t ns32(uint32_t row, uint32_t col) {
 }
 
 struct BwdStreamParams {
+    const int *order;        // [B * row blocks]: the row block each CTA takes (longest first)
     const __nv_bfloat16 *Q, *dO;
     const float *LSE, *g;
     const uint8_t *img, *M;
@@ -129,8 +130,11 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     const int n = p.n, nch = (n + 31) / 32;
     // i0: the row block's first row in the graph; i0l: in the slab (E, dE', dE
     // rows); item: the row block's partials, (graph, row block of the graph)
-    const int b = blockIdx.y, i0l = blockIdx.x * TB, i0 = p.row0 + i0l;
-    const int item = blockIdx.y * ((n + TB - 1) / TB) + i0 / TB;
+    // the row block this CTA takes: longest first (k_row_block_order), so that
+    // the short ones fill the last wave
+    const int nrb = gridDim.x, ord = p.order[blockIdx.y * gridDim.x + blockIdx.x];
+    const int b = ord / nrb, i0l = (ord % nrb) * TB, i0 = p.row0 + i0l;
+    const int item = b * ((n + TB - 1) / TB) + i0 / TB;
     const uint32_t bars = sbase + S::BAR;
     auto bar = [&](int k) { return bars + 8 * k; };
     float *g = reinterpret_cast<float *>(sp + S::G);
@@ -364,7 +368,7 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
-                        const int prb = cid % gridDim.x, pb = cid / gridDim.x;
+                        const int pord = p.order[cid], prb = pord % nrb, pb = pord / nrb;
                         for (int cc = 0; cc < nch && cc < 2; ++cc) {
                             if (!light) {
                                 tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, 0, pb);
@@ -761,6 +765,7 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
         !encode_node_map(&mV, a.V, d.B, d.n, 32))
         return cudaErrorInvalidValue;
     BwdStreamParams p;
+    p.order = reinterpret_cast<const int *>(ws + W.order);
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
     p.dO = reinterpret_cast<const __nv_bfloat16 *>(ws + W.dO);
     p.LSE = a.LSE;

@@ -43,7 +43,7 @@ __host__ __device__ __forceinline__ uint32_t ns16(uint32_t row, uint32_t k) {
 // Workspace of the fast path (after the common status word and g).  Every
 // region grows with the node count B*n (or is fixed): no per-pair buffer.
 struct FastWs {
-    size_t img, dO, dQ, dK, dV, dK32, dV32, rparts, wparts, bparts, r2, dg, total;
+    size_t img, dO, dQ, dK, dV, dK32, dV32, rparts, wparts, bparts, r2, dg, order, total;
     int n_rparts, wsplits, bsplits, rsplits;
 };
 
@@ -77,6 +77,8 @@ inline FastWs fast_ws(const eaga_dims &d, size_t base) {
     W.rsplits = 32;
     W.r2 = off; off = align256(off + size_t(W.rsplits) * (DE * NF + NH * DE) * 4);
     W.dg = off; off = align256(off + size_t(d.B) * NF * 4);
+    // the order in which the backward pair kernel's CTAs take the row blocks
+    W.order = off; off = align256(off + size_t(row_blocks(d)) * 4);
     W.total = off;
     return W;
 }
@@ -245,6 +247,10 @@ __device__ __forceinline__ uint32_t live_chunk_mask(const uint8_t *M, int b, int
     }
     return __ballot_sync(0xffffffffu, any != 0);
 }
+
+// Largest number of row blocks that k_row_block_order sorts (its keys live
+// in 48 KB of shared memory); beyond it the CTAs take the row blocks in order.
+constexpr int ORDER_MAX_ITEMS = 12288;
 
 // Position of the k-th (from 0) set bit of m; m has more than k bits set.
 __device__ __forceinline__ int nth_set_bit(uint32_t m, int k) {
