@@ -73,9 +73,12 @@ eaga_status eaga_forward_noalloc(const eaga_dims *d, const void *X, const void *
         if (!aligned16(p)) return EAGA_ERR_MISALIGNED;
     }
     const size_t g_bytes = align256(size_t(d->B) * 2 * d->H * sizeof(float));
-    const size_t images = fast::supports(*d) ? fast::forward_scratch_bytes(*d) : 0;
+    const bool fast_path = fast::supports(*d);
+    const size_t images = fast_path ? fast::forward_scratch_bytes(*d, false) : 0;
     const size_t needed = NOALLOC_G + g_bytes + images;
     if (needed > NOALLOC_SCRATCH_BYTES) return EAGA_ERR_UNSUPPORTED;   // too large for the fixed array
+    // the pair kernel's row-block order where it still fits (else index order)
+    const bool with_order = fast_path && NOALLOC_G + g_bytes + fast::forward_scratch_bytes(*d) <= NOALLOC_SCRATCH_BYTES;
     {
         const Extents x = tensor_extents(*d);
         const Span outs[3] = {{Xout, x.X}, {Eout, x.E}, {saved, saved_layout(*d).saved_total}};
@@ -105,7 +108,7 @@ eaga_status eaga_forward_noalloc(const eaga_dims *d, const void *X, const void *
     a.g = reinterpret_cast<float *>(scratch + NOALLOC_G);
     // The status word must start at zero; g and the images are rewritten in full by every call.
     if (cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess) return EAGA_ERR_CUDA;
-    cudaError_t e = fast::supports(*d) ? fast::forward(*d, a, scratch + NOALLOC_G + g_bytes, st)
+    cudaError_t e = fast_path ? fast::forward(*d, a, scratch + NOALLOC_G + g_bytes, st, with_order)
                                        : generic::forward(*d, a, st);
     return e == cudaSuccess ? EAGA_OK : EAGA_ERR_CUDA;
 }

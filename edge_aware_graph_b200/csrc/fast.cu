@@ -12,7 +12,7 @@ cudaError_t launch_prologue(const eaga_dims &d, const void *const w[12], const v
 cudaError_t tc_gemm(int mode, int M, int N, int K, int nseg, const void *const A[3], const void *const B[3],
                     const void *const bias[3], void *const C[3], int Nb, const void *R, const uint8_t *mask,
                     int *status, cudaStream_t st, bool b_mn);
-cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
+cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const int *order, const float *g,
                              cudaStream_t st);
 cudaError_t tc_wgrad(int M, int Nb, int nout, int K, int splits, const void *A, const void *const B[3],
                      float *const P[3], int *status, cudaStream_t st);
@@ -32,17 +32,20 @@ bool supports(const eaga_dims &d) {
 
 // Forward: the small operand images after the common workspace; backward:
 // the whole FastWs.
-size_t forward_scratch_bytes(const eaga_dims &) { return align256(IMG_BYTES); }
+// (the operand images, then the order of the row blocks for the pair kernel)
+size_t forward_scratch_bytes(const eaga_dims &d, bool with_order) {
+    return align256(IMG_BYTES) + (with_order ? align256(size_t(row_blocks(d)) * 4) : 0);
+}
 size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, size_t common_head) {
-    if (!for_backward) return align256(common_fwd + IMG_BYTES);
+    if (!for_backward) return align256(common_fwd) + forward_scratch_bytes(d);
     return fast_ws(d, common_head).total;
 }
 
 int kernel_launches(const eaga_dims &, int for_backward) {
-    // forward: prologue, QKV, pairs, out-proj
+    // forward: prologue, row-block order, QKV, pairs, out-proj
     // backward: prologue, dO, row-block order, pairs, dk/dv conversion, dX, wgrad x2, bias partial,
     // rparts partial, finish x2, film grads
-    return for_backward ? 13 : 4;
+    return for_backward ? 13 : 5;
 }
 
 #define FAST_TRY(x)                               \
@@ -93,16 +96,20 @@ cudaError_t stream_after(cudaStream_t to, cudaStream_t from, cudaEvent_t ev) {
 }
 }  // namespace
 
-cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st) {
+cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st,
+                    bool with_order) {
     uint8_t *img = reinterpret_cast<uint8_t *>(ws_after_common);
+    int *order = with_order ? reinterpret_cast<int *>(ws_after_common + align256(IMG_BYTES)) : nullptr;
     const int rows = d.B * d.n;
     DeviceAux *aux = nullptr;
     FAST_TRY(device_aux(&aux));
     std::lock_guard<std::mutex> lock(aux->mu);
     FAST_TRY(aux_init(*aux));
-    // the prologue (g, operand images) beside the QKV projection
+    // the prologue (g, operand images) and the order of the row blocks for the
+    // pair kernel (longest first) beside the QKV projection
     FAST_TRY(stream_after(aux->s[0], st, aux->ev[0]));
     FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, aux->s[0]));
+    if (order) FAST_TRY(launch_row_block_order(d, a.M, a.row0, a.rows < 0 ? d.n : a.rows, order, aux->s[0]));
     {   // [Q|K|V] = X [Wq|Wk|Wv] + b
         const void *A[3] = {a.X, a.X, a.X}, *B[3] = {a.w[0], a.w[2], a.w[4]};
         const void *bias[3] = {a.w[1], a.w[3], a.w[5]};
@@ -114,7 +121,7 @@ cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common,
     // in the backward, dWo read every row)
     if (a.rows >= 0 && a.rows < d.n) FAST_TRY(cudaMemsetAsync(a.O, 0, (size_t)rows * HD * 2, st));
     prof_mark(0, 0, st);
-    FAST_TRY(launch_fwd_pairs(d, a, img, a.g, st));
+    FAST_TRY(launch_fwd_pairs(d, a, img, order, a.g, st));
     prof_mark(0, 1, st);
     {   // X' = X + M (O Wo + bo)
         const void *A[3] = {a.O, a.O, a.O}, *B[3] = {a.w[10], a.w[10], a.w[10]};

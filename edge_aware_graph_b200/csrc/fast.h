@@ -10,8 +10,11 @@ bool supports(const eaga_dims &d);
 size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, size_t common_head);
 int kernel_launches(const eaga_dims &d, int for_backward);
 // Bytes the forward uses after the common workspace (the FiLM and edge operand images).
-size_t forward_scratch_bytes(const eaga_dims &d);
-cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st);
+// with_order: also the pair kernel's row-block order (without it the row
+// blocks run in index order)
+size_t forward_scratch_bytes(const eaga_dims &d, bool with_order = true);
+cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st,
+                    bool with_order = true);
 cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head, cudaStream_t st);
 }  // namespace fast
 }  // namespace eaga

@@ -27,7 +27,9 @@
 // chunk with no valid pair (no node among the CTA's rows, or none among the
 // chunk's columns: padding of a smaller graph) has a = 0 everywhere, so E' = E
 // there.  Such a chunk is only copied by the TMA warp (loaded and stored back,
-// bit for bit); the compute and MMA warps never see it.
+// bit for bit); the compute and MMA warps never see it.  The clusters take
+// the row blocks longest first (most live chunks; k_row_block_order), so
+// that short and copy-only row blocks fill the last wave.
 //
 // Warp roles.  Warps 0..7 compute (warp W reads TMEM quadrant q = W%4 and
 // handles the four heads 4hp..4hp+3, hp = W/4).  Warp 8 (one thread) issues
@@ -95,6 +97,7 @@ constexpr uint32_t FS_TM_COLS = 256;
 constexpr uint32_t FS_TM_FILM = 0, FS_TM_EDGE = 0, FS_TM_S = 128;
 
 struct FwdParams {
+    const int *order;        // [B * row blocks]: the row block each cluster takes, longest first (null: index order)
     const __nv_bfloat16 *Q;
     const uint8_t *img;      // operand images (IMG_*)
     const float *g;          // [B, 16] global FiLM term
@@ -124,7 +127,10 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
     const int n = p.n, nch = (n + 31) / 32, cs = p.cs;
     const int cpc = (nch + cs - 1) / cs;                        // chunks per CTA of the row block
     // i0: the row block's first row in the graph; i0l: in the slab (E, E' rows)
-    const int rank = blockIdx.x % cs, b = blockIdx.y, i0l = (blockIdx.x / cs) * TB, i0 = p.row0 + i0l;
+    // the row block of this CTA's cluster: longest first (k_row_block_order), so
+    // that the short ones fill the last wave
+    const int nrb = gridDim.x / cs, cl = blockIdx.y * nrb + blockIdx.x / cs, ord = p.order ? p.order[cl] : cl;
+    const int rank = blockIdx.x % cs, b = ord / nrb, i0l = (ord % nrb) * TB, i0 = p.row0 + i0l;
     const int c_begin = rank * cpc, nchl = max(0, min(nch, c_begin + cpc) - c_begin);
     const uint32_t bars = sbase + S::BAR;
     auto bar = [&](int k) { return bars + 8 * k; };
@@ -335,8 +341,9 @@ k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
                     // L2 prefetch of the first tiles of the CTA that runs about one wave later
                     const uint32_t cid = blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
                     if (cid < gridDim.x * gridDim.y) {
-                        const int px = cid % gridDim.x, pb = cid / gridDim.x;
-                        const int pc0 = (px % cs) * cpc, prb = px / cs;
+                        const int pord = p.order ? p.order[cid / cs] : int(cid / cs), pb = pord / nrb,
+                                  prb = pord % nrb;
+                        const int pc0 = (cid % cs) * cpc;
                         for (int cc = pc0; cc < nch && cc < pc0 + 2; ++cc)
                             for (int s = 0; s < 2; ++s) tma_prefetch_5d(&tmE, 0, prb * TB / 2, 32 * cc, s, pb);
                     }
@@ -684,7 +691,7 @@ static int fwd_cluster_size(int n) {
     return cs;
 }
 
-cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const float *g,
+cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t *img, const int *order, const float *g,
                              cudaStream_t st) {
     static std::atomic<uint32_t> attr_set{0}, carveout_set{0};
     if (cudaError_t e = ensure_smem_attr(k_fwd_stream, FsSmem::BYTES, attr_set); e != cudaSuccess) return e;
@@ -706,6 +713,7 @@ cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t
     const int cs = fwd_cluster_size(d.n);
     if (cs > FS_MAX_CS) return cudaErrorInvalidValue;
     FwdParams p;
+    p.order = order;
     p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
     p.img = img;
     p.g = g;

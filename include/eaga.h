@@ -224,7 +224,11 @@ EAGA_API eaga_status eaga_backward_rows(const eaga_dims *dims, int variant, int 
  * exits.  Limit: 256 + roundup256(8*H*B) bytes, plus 8192 on the specialised
  * path, must fit in 64 KiB: B <= 892 graphs on the specialised path, B <= 4080
  * at H = 2 on the CUDA-core path; larger B returns EAGA_ERR_UNSUPPORTED
- * without launching.  No device memory is allocated or freed by this call.
+ * without launching.  Where roundup256(4*B*ceil(n/8)) bytes more also fit, the
+ * specialised path keeps there the order in which its pair kernel takes the
+ * row blocks (longest first, one more kernel launch); otherwise it takes them
+ * in index order, with the same results.  No device memory is allocated or
+ * freed by this call.
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
