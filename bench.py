@@ -53,16 +53,15 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the dominant kernels on each workload, from one ncu capture of the kernels as
 # they are (the summaries under profiles/ give the commands).  A kernel that
-# changes reports null until it is captured again.  Large: the counters come
-# in GB with three digits (1.77 GB read by k_bwd_stream).  Planar: one batch's
+# changes reports null until it is captured again.  Planar: one batch's
 # E' (32 MiB) fits in L2, so within the captured launch its writes stay in L2
 # and reach DRAM later, under the next batch's launch.
 NCU_TRAFFIC = {
-    ("sbm", "k_fwd_stream"): 167305984 + 97689344,
-    ("sbm", "k_bwd_stream"): 252016128 + 113165824,
-    ("large", "k_fwd_stream"): 736150000 + 481330000,
-    ("large", "k_bwd_stream"): 1770000000 + 501140000,
-    ("planar", "k_fwd_stream"): 39940000 + 848900,
+    ("sbm", "k_fwd_stream"): 162472448 + 97329664,
+    ("sbm", "k_bwd_stream"): 257099520 + 109985792,
+    ("large", "k_fwd_stream"): 734333184 + 481042944,
+    ("large", "k_bwd_stream"): 1771164416 + 507204608,
+    ("planar", "k_fwd_stream"): 39935744 + 764672,
     ("sbm", "k_eblk_fwd"): 63142912 + 99683840,
     ("sbm", "k_eblk_bwd"): 182036992 + 124005632,
     ("large", "k_eblk_fwd"): 487750000 + 485110000,

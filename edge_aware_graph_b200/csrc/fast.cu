@@ -22,6 +22,7 @@ cudaError_t launch_kv_convert(const eaga_dims &d, const FastWs &W, char *ws, cud
 cudaError_t launch_row_block_order(const eaga_dims &d, const uint8_t *M, int row0, int rows, int *order,
                                    cudaStream_t st);
 cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
+cudaError_t launch_film_grads(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st);
 cudaError_t launch_bwd_final(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, int part,
                              cudaStream_t st);
 
@@ -60,11 +61,11 @@ int kernel_launches(const eaga_dims &, int for_backward) {
 // as parallel branches.  The lock is held while a call enqueues, so concurrent calls on
 // one device never share an event between a record and its wait.
 namespace {
-constexpr int kMaxDevices = 64, kEvents = 6;
+constexpr int kMaxDevices = 64, kEvents = 9, kStreams = 3;
 struct DeviceAux {
     std::mutex mu;
     bool ready = false;
-    cudaStream_t s[2] = {nullptr, nullptr};
+    cudaStream_t s[kStreams] = {};
     cudaEvent_t ev[kEvents] = {};
 };
 DeviceAux g_aux[kMaxDevices];
@@ -81,7 +82,7 @@ cudaError_t device_aux(DeviceAux **out) {
 cudaError_t aux_init(DeviceAux &x) {   // called with x.mu held
     if (x.ready) return cudaSuccess;
     cudaError_t e;
-    for (int k = 0; k < 2; ++k)
+    for (int k = 0; k < kStreams; ++k)
         if ((e = cudaStreamCreateWithFlags(&x.s[k], cudaStreamNonBlocking)) != cudaSuccess) return e;
     for (int k = 0; k < kEvents; ++k)
         if ((e = cudaEventCreateWithFlags(&x.ev[k], cudaEventDisableTiming)) != cudaSuccess) return e;
@@ -106,10 +107,14 @@ cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common,
     std::lock_guard<std::mutex> lock(aux->mu);
     FAST_TRY(aux_init(*aux));
     // the prologue (g, operand images) and the order of the row blocks for the
-    // pair kernel (longest first) beside the QKV projection
+    // pair kernel (longest first) beside the QKV projection, each on a stream
+    // of its own
     FAST_TRY(stream_after(aux->s[0], st, aux->ev[0]));
     FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, aux->s[0]));
-    if (order) FAST_TRY(launch_row_block_order(d, a.M, a.row0, a.rows < 0 ? d.n : a.rows, order, aux->s[0]));
+    if (order) {
+        FAST_TRY(stream_after(aux->s[1], st, aux->ev[2]));
+        FAST_TRY(launch_row_block_order(d, a.M, a.row0, a.rows < 0 ? d.n : a.rows, order, aux->s[1]));
+    }
     {   // [Q|K|V] = X [Wq|Wk|Wv] + b
         const void *A[3] = {a.X, a.X, a.X}, *B[3] = {a.w[0], a.w[2], a.w[4]};
         const void *bias[3] = {a.w[1], a.w[3], a.w[5]};
@@ -117,6 +122,7 @@ cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common,
         FAST_TRY(tc_gemm(0, rows, 3 * HD, d.dx, 1, A, B, bias, C, HD, nullptr, a.M, a.status, st, true));
     }
     FAST_TRY(stream_after(st, aux->s[0], aux->ev[1]));
+    if (order) FAST_TRY(stream_after(st, aux->s[1], aux->ev[3]));
     // a slab of rows: O of the rows outside it is zero (the out-projection and,
     // in the backward, dWo read every row)
     if (a.rows >= 0 && a.rows < d.n) FAST_TRY(cudaMemsetAsync(a.O, 0, (size_t)rows * HD * 2, st));
@@ -141,7 +147,7 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
     FAST_TRY(device_aux(&aux));
     std::lock_guard<std::mutex> lock(aux->mu);
     FAST_TRY(aux_init(*aux));
-    cudaStream_t s1 = aux->s[0], s2 = aux->s[1];
+    cudaStream_t s1 = aux->s[0], s2 = aux->s[1], s3 = aux->s[2];
     cudaEvent_t *ev = aux->ev;
 
     // prologue (g, operand images) beside dO = M (dX' Wo^T)
@@ -175,6 +181,7 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
                                   reinterpret_cast<const __nv_bfloat16 *>(ws + W.dV)};
     FAST_TRY(stream_after(s1, st, ev[2]));
     FAST_TRY(stream_after(s2, st, ev[3]));
+    FAST_TRY(stream_after(s3, st, ev[6]));
     {   // dX = dX' + dQ Wq^T + dK Wk^T + dV Wv^T
         const void *A[3] = {dN[0], dN[1], dN[2]}, *Bt[3] = {a.w[0], a.w[2], a.w[4]};
         void *C[3] = {a.dX, a.dX, a.dX};
@@ -191,10 +198,15 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         FAST_TRY(launch_bwd_final(d, a, W, ws, 0, s1));
         FAST_TRY(tc_wgrad(HD, d.dx, 1, rows, W.wsplits, a.O, Bo, Po, a.status, s2));
     }
-    FAST_TRY(launch_bwd_partials(d, a, W, ws, s2));   // bias and row-block partials, dg, dbf, dWfy, dy
+    // the bias and row-block partials beside dWo (they do not need it), then
+    // dbf, dWfy, dy from dg beside the final sums of the rest
+    FAST_TRY(launch_bwd_partials(d, a, W, ws, s3));
+    FAST_TRY(stream_after(s2, s3, ev[7]));
+    FAST_TRY(launch_film_grads(d, a, W, ws, s3));
     FAST_TRY(launch_bwd_final(d, a, W, ws, 1, s2));
     FAST_TRY(stream_after(st, s1, ev[4]));
     FAST_TRY(stream_after(st, s2, ev[5]));
+    FAST_TRY(stream_after(st, s3, ev[8]));
     return cudaSuccess;
 }
 

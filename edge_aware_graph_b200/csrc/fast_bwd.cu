@@ -277,7 +277,12 @@ cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const Fast
     const int xblocks = (std::max(NE, d.B * NF) + 255) / 256;
     k_rparts_partial<<<dim3(xblocks, W.rsplits + 1), 256, 0, st>>>(rparts, ctas, seg, r2, dg, d.B,
                                                                    (d.n + TB - 1) / TB);
-    // dbf, dWfy, dy from dg (on the same stream, off the path of dX and dW)
+    return cudaGetLastError();
+}
+
+// dbf, dWfy, dy from dg (after launch_bwd_partials; off the path of dX and dW).
+cudaError_t launch_film_grads(const eaga_dims &d, const BwdArgs &a, const FastWs &W, char *ws, cudaStream_t st) {
+    const float *dg = reinterpret_cast<const float *>(ws + W.dg);
     const int tf = NF + d.dy * NF + d.B * d.dy;
     k_film_grads<<<(tf + 255) / 256, 256, 0, st>>>(dg, d.B, d.dy, static_cast<const __nv_bfloat16 *>(a.y),
                                                    static_cast<const __nv_bfloat16 *>(a.w[7]), a.dW[8], a.dW[7],
