@@ -235,6 +235,8 @@ cudaError_t launch_bwd_pairs(const eaga_dims &d, const BwdArgs &a, const FastWs 
 // row blocks, for the node GEMMs and the bias sums (four features per thread).
 __global__ void k_kv_convert(const float4 *dK32, const float4 *dV32, size_t n4, __nv_bfloat16 *dK,
                              __nv_bfloat16 *dV) {
+    griddep_launch_dependents();
+    griddep_wait();
     const float rs = rsqrtf((float)DH);
     for (size_t x = blockIdx.x * (size_t)blockDim.x + threadIdx.x; x < n4; x += (size_t)gridDim.x * blockDim.x) {
         const float4 k = dK32[x], v = dV32[x];
@@ -251,11 +253,9 @@ __global__ void k_kv_convert(const float4 *dK32, const float4 *dV32, size_t n4, 
 cudaError_t launch_kv_convert(const eaga_dims &d, const FastWs &W, char *ws, cudaStream_t st) {
     const size_t n4 = (size_t)d.B * d.n * HD / 4;
     const int blocks = (int)std::min<size_t>((n4 + 255) / 256, (size_t)sm_count() * 8);
-    k_kv_convert<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4 *>(ws + W.dK32),
-                                         reinterpret_cast<const float4 *>(ws + W.dV32), n4,
-                                         reinterpret_cast<__nv_bfloat16 *>(ws + W.dK),
-                                         reinterpret_cast<__nv_bfloat16 *>(ws + W.dV));
-    return cudaGetLastError();
+    return launch_pdl(k_kv_convert, dim3(blocks), dim3(256), 0, st, 1, reinterpret_cast<const float4 *>(ws + W.dK32),
+                      reinterpret_cast<const float4 *>(ws + W.dV32), n4, reinterpret_cast<__nv_bfloat16 *>(ws + W.dK),
+                      reinterpret_cast<__nv_bfloat16 *>(ws + W.dV));
 }
 
 // Column sums for the bias gradients and the first level of the row-block

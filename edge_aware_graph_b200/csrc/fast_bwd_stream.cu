@@ -123,6 +123,8 @@ k_bwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CU
              const __grid_constant__ CUtensorMap tmDE, const __grid_constant__ CUtensorMap tmK,
              const __grid_constant__ CUtensorMap tmV, BwdStreamParams p) {
     using S = BsSmem;
+    griddep_launch_dependents();
+    griddep_wait();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
@@ -784,8 +786,8 @@ cudaError_t launch_bwd_stream(const eaga_dims &d, const BwdArgs &a, const FastWs
     p.light = a.variant == EAGA_VARIANT_LIGHT_EDGE;
     p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)sm_count();
-    k_bwd_stream<<<dim3((rows + TB - 1) / TB, d.B), BS_THR, BsSmem::BYTES, st>>>(mE, mDEp, mDE, mK, mV, p);
-    return cudaGetLastError();
+    return launch_pdl(k_bwd_stream, dim3((rows + TB - 1) / TB, d.B), dim3(BS_THR), BsSmem::BYTES, st, 1, mE, mDEp, mDE,
+                      mK, mV, p);
 }
 
 }  // namespace fast

@@ -2,6 +2,7 @@
 // sm_100a path (de = 64, H = 8, dh = 32, bf16 storage).
 #pragma once
 #include <cuda.h>
+#include <utility>
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -17,6 +18,33 @@ inline int sm_count() {
         v > 0)
         return v;
     return 148;
+}
+
+// Launch of a kernel that may start behind the previous kernel of its stream
+// (programmatic stream serialisation): its CTAs become resident while that
+// kernel's last CTAs finish and wait in griddep_wait before touching global
+// memory.  cluster > 1 adds a cluster dimension.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 1;
+    if (cluster > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    cfg.attrs = attr;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Operand images prepared once per call by the prologue kernel (bf16, in the

@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(FS_THR, 2)
 k_fwd_stream(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmEo,
              const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, FwdParams p) {
     using S = FsSmem;
+    griddep_launch_dependents();
+    griddep_wait();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
@@ -729,23 +731,7 @@ cudaError_t launch_fwd_pairs(const eaga_dims &d, const FwdArgs &a, const uint8_t
     p.unnorm = a.variant == EAGA_VARIANT_UNNORMALISED;
     p.prefetch_ahead = (uint32_t)(2 * sm_count());   // two CTAs per SM
     const dim3 grid(((rows + TB - 1) / TB) * cs, d.B);
-    if (cs == 1) {
-        k_fwd_stream<<<grid, FS_THR, FsSmem::BYTES, st>>>(mE, mEo, mK, mV, p);
-        return cudaGetLastError();
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(FS_THR);
-    cfg.dynamicSmemBytes = FsSmem::BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_fwd_stream, mE, mEo, mK, mV, p);
+    return launch_pdl(k_fwd_stream, grid, dim3(FS_THR), FsSmem::BYTES, st, cs, mE, mEo, mK, mV, p);
 }
 
 }  // namespace fast

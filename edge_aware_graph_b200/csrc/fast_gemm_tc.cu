@@ -57,6 +57,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap a0, const __grid_constant__ CUtens
           const __grid_constant__ CUtensorMap b1, const __grid_constant__ CUtensorMap b2, TcParams p) {
     using S = TcSmem<BN>;
     constexpr int TSTAGES = tc_stages<BN>();
+    griddep_launch_dependents();
+    griddep_wait();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *sp = smem_raw + (sbase - smem_u32(smem_raw));
@@ -329,8 +331,8 @@ static cudaError_t tc_launch(const CUtensorMap (&am)[3], const CUtensorMap (&bm)
     static std::atomic<uint32_t> attr_set{0};
     if (cudaError_t e = ensure_smem_attr(k_tc_gemm<BN>, TcSmem<BN>::BYTES, attr_set); e != cudaSuccess) return e;
     dim3 grid(N / BN, (p.M + TBM - 1) / TBM);
-    k_tc_gemm<BN><<<grid, TTHR, TcSmem<BN>::BYTES, st>>>(am[0], am[1], am[2], bm[0], bm[1], bm[2], p);
-    return cudaGetLastError();
+    return launch_pdl(k_tc_gemm<BN>, grid, dim3(TTHR), TcSmem<BN>::BYTES, st, 1, am[0], am[1], am[2], bm[0], bm[1],
+                      bm[2], p);
 }
 
 // Out = epilogue(sum_seg A[seg] B[seg]): A[seg] [M, K] row-major bf16; B[seg] stored

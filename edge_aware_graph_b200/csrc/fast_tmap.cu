@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(256) k_prologue(const __nv_bfloat16 *y, const 
                                                   const __nv_bfloat16 *bf, const __nv_bfloat16 *Wfe,
                                                   const __nv_bfloat16 *We, float *g, uint8_t *img, int B, int dy,
                                                   int *zero_ints, int nzero) {
+    sm100::griddep_launch_dependents();   // the pair kernel behind it may become resident
     const int w = threadIdx.x >> 5, t = threadIdx.x & 31;
     if (blockIdx.x + 1 < gridDim.x) {
         const int b = blockIdx.x * 8 + w;

@@ -299,6 +299,19 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Wait until the grids this one was launched behind (with programmatic stream
+// serialisation) have completed and their writes are visible; returns at once
+// for a grid launched without it.  A kernel launched that way touches no
+// global memory before this.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the grid launched behind this one (programmatically) start its CTAs
+// once every CTA of this grid has passed here; they wait in griddep_wait.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ warp MMA
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
