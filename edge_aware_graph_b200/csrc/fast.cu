@@ -61,7 +61,7 @@ int kernel_launches(const eaga_dims &, int for_backward) {
 // as parallel branches.  The lock is held while a call enqueues, so concurrent calls on
 // one device never share an event between a record and its wait.
 namespace {
-constexpr int kMaxDevices = 64, kEvents = 9, kStreams = 3;
+constexpr int kMaxDevices = 64, kEvents = 11, kStreams = 3;
 struct DeviceAux {
     std::mutex mu;
     bool ready = false;
@@ -163,12 +163,14 @@ cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head
         FAST_TRY(cudaMemsetAsync(ws + W.dQ, 0, (size_t)rows * HD * 2, s1));
         FAST_TRY(cudaMemsetAsync(ws + W.rparts, 0, (size_t)W.n_rparts * RPART * 4, s1));
     }
-    // the order of the row blocks for the pair kernel (longest first) and the
-    // prologue, beside dO
+    // the order of the row blocks for the pair kernel (longest first) on a
+    // third stream and the prologue, beside dO
+    FAST_TRY(stream_after(s3, st, ev[9]));
     FAST_TRY(launch_row_block_order(d, a.M, a.row0, a.rows < 0 ? d.n : a.rows, reinterpret_cast<int *>(ws + W.order),
-                                    st));
+                                    s3));
     FAST_TRY(launch_prologue(d, a.w, a.y, a.g, img, nullptr, 0, st));
     FAST_TRY(stream_after(st, s1, ev[1]));
+    FAST_TRY(stream_after(st, s3, ev[10]));
 
     prof_mark(1, 0, st);
     FAST_TRY(launch_bwd_pairs(d, a, W, ws, a.g, st));
