@@ -216,6 +216,7 @@ __device__ __forceinline__ void block_matvec(const float *in, int K, int nout, W
     if (pi < P) {
         const int k0 = pi * K / P, k1 = (pi + 1) * K / P;
         float a = 0.f;
+#pragma unroll 8
         for (int k = k0; k < k1; ++k) a = fmaf(in[k], w(k, o), a);
         part[pi * nout + o] = a;
     }
@@ -226,6 +227,25 @@ __device__ __forceinline__ void block_matvec(const float *in, int K, int nout, W
         out[q] = a;
     }
     __syncthreads();
+}
+
+// sum_k v[k] row[k] over a bf16 row of len values (len a multiple of 8, the
+// row 16-byte aligned), read eight values a load, in k order.
+__device__ __forceinline__ float row_dot(const float *v, const __nv_bfloat16 *row, int len) {
+    const uint4 *r4 = reinterpret_cast<const uint4 *>(row);
+    float a = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < len / 8; ++c) {
+        const uint4 u = r4[c];
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(h2[j]);
+            a = fmaf(v[8 * c + 2 * j], f.x, a);
+            a = fmaf(v[8 * c + 2 * j + 1], f.y, a);
+        }
+    }
+    return a;
 }
 
 // Recomputes the global sub-block of graph b from y1 into shared memory:
@@ -330,14 +350,13 @@ __global__ void __launch_bounds__(256) k_y_bwd(YParams p) {
         dyz[o] = r2 * (dg - m1 - x2[o] * m2);
     }
     __syncthreads();
-    // dh = dyz W2^T [hpre > 0]
-    block_matvec(dyz, dy, fy, [&](int k, int f) { return bf(p.W2, (size_t)f * dy + k); }, [](int) { return 0.f; },
-                 dh, part);
-    for (int f = threadIdx.x; f < fy; f += blockDim.x) dh[f] = hpre[f] > 0.f ? dh[f] : 0.f;
+    // dh = dyz W2^T [hpre > 0]: row f of W2 per output
+    for (int f = threadIdx.x; f < fy; f += blockDim.x)
+        dh[f] = hpre[f] > 0.f ? row_dot(dyz, p.W2 + (size_t)f * dy, dy) : 0.f;
     __syncthreads();
-    // dya = dyz + dh W1^T
-    block_matvec(dh, fy, dy, [&](int k, int o) { return bf(p.W1, (size_t)o * fy + k); },
-                 [&](int o) { return dyz[o]; }, dya, part);
+    // dya = dyz + dh W1^T: row o of W1 per output
+    for (int o = threadIdx.x; o < dy; o += blockDim.x) dya[o] = dyz[o] + row_dot(dh, p.W1 + (size_t)o * fy, fy);
+    __syncthreads();
     m1 = 0.f;
     m2 = 0.f;
     for (int o = threadIdx.x; o < dy; o += blockDim.x) {
@@ -357,16 +376,8 @@ __global__ void __launch_bounds__(256) k_y_bwd(YParams p) {
     for (int i = threadIdx.x; i < n; i += blockDim.x) c += p.M[(size_t)b * n + i] ? 1.f : 0.f;
     const float cnt = block_sum(c, scratch);
     const float cx = fmaxf(cnt, 1.f), ce = fmaxf(cnt * cnt, 1.f);
-    for (int k = threadIdx.x; k < dx; k += blockDim.x) {
-        float a = 0.f;
-        for (int o = 0; o < dy; ++o) a = fmaf(dy1[o], bf(p.Wyx, (size_t)k * dy + o), a);
-        p.dpX[(size_t)b * dx + k] = a / cx;
-    }
-    for (int k = threadIdx.x; k < 64; k += blockDim.x) {
-        float a = 0.f;
-        for (int o = 0; o < dy; ++o) a = fmaf(dy1[o], bf(p.Wye, (size_t)k * dy + o), a);
-        p.dpE[(size_t)b * 64 + k] = a / ce;
-    }
+    for (int k = threadIdx.x; k < dx; k += blockDim.x) p.dpX[(size_t)b * dx + k] = row_dot(dy1, p.Wyx + (size_t)k * dy, dy) / cx;
+    for (int k = threadIdx.x; k < 64; k += blockDim.x) p.dpE[(size_t)b * 64 + k] = row_dot(dy1, p.Wye + (size_t)k * dy, dy) / ce;
     // per-graph vectors: h, dh [fy]; ya, dyz, x1, dya, x2 [dy]
     float *v = p.yv + (size_t)b * YV_PER_DY * dy;
     for (int f = threadIdx.x; f < fy; f += blockDim.x) {
@@ -456,38 +467,53 @@ __global__ void __launch_bounds__(256) k_y_wgrad(YParams p, YGrads gr) {
 // ------------------------------------------------------------------ reductions
 
 // dst = sum over parts of src (part k at src + k * stride); with trows > 0 the
-// segment is the transpose of a [trows][count / trows] source.  One warp per
-// item: a segment of many parts (more than 16) gives one entry to each warp,
-// whose lanes take every 32nd part and add their sums with shuffles; a segment
-// of few parts gives 32 consecutive entries to each warp, one a lane.  Every
-// entry is summed in the same order on every call.
+// segment is the transpose of a [trows][count / trows] source.  The lanes of a
+// warp take consecutive source entries, so every load is a coalesced 128-byte
+// row of one part.  A segment of many parts (more than 16) gives 32 entries to
+// a CTA whose eight warps split the parts; a segment of few parts gives 256
+// entries to a CTA, each warp adding all parts of its 32.  Every entry is
+// summed in the same order on every call.
 __global__ void __launch_bounds__(256) k_sum_parts(SumSegs segs) {
-    const int lane = threadIdx.x & 31;
-    int item = blockIdx.x * 8 + (threadIdx.x >> 5);
+    __shared__ float red[8][32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int item = blockIdx.x;
     for (int s = 0; s < segs.n; ++s) {
         const SumSeg &g = segs.seg[s];
+        // a CTA: 32 consecutive source entries of a wide segment (more than 16
+        // parts; warp w adds the parts k = w mod 8, then the eight sums are added
+        // in warp order), or 256 of a narrow one (a warp 32, over every part)
         const bool wide = g.nparts > 16;
-        const int items = wide ? g.count : (g.count + 31) / 32;
-        if (item >= items) {
-            item -= items;
+        const int per = wide ? 32 : 256;
+        const int tiles = (g.count + per - 1) / per;
+        if (item >= tiles) {
+            item -= tiles;
             continue;
         }
-        const int e = wide ? item : item * 32 + lane;
-        if (e >= g.count) return;
-        int src = e;
-        if (g.trows > 0) {
-            const int cols = g.count / g.trows;
-            src = (e % g.trows) * cols + e / g.trows;
-        }
+        const int src = item * per + (wide ? 0 : 32 * w) + lane;   // consecutive lanes: consecutive addresses
+        const bool in = src < g.count;
         float t = 0.f;
         if (wide) {
-            for (int k = lane; k < g.nparts; k += 32) t += g.src[(size_t)k * g.stride + src];
-            t = warp_sum(t);
-            if (lane == 0) g.dst[e] = t;
-        } else {
+            if (in) {
+#pragma unroll 4
+                for (int k = w; k < g.nparts; k += 8) t += g.src[(size_t)k * g.stride + src];
+            }
+            red[w][lane] = t;
+            __syncthreads();
+            if (w != 0) return;
+            t = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t += red[k][lane];
+        } else if (in) {
+#pragma unroll 4
             for (int k = 0; k < g.nparts; ++k) t += g.src[(size_t)k * g.stride + src];
-            g.dst[e] = t;
         }
+        if (!in) return;
+        int e = src;   // the destination entry: source [trows][cols] -> destination [cols][trows]
+        if (g.trows > 0) {
+            const int cols = g.count / g.trows;
+            e = (src % cols) * g.trows + src / cols;
+        }
+        g.dst[e] = t;
         return;
     }
 }
@@ -795,10 +821,10 @@ cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const ch
         const float *ew = reinterpret_cast<const float *>(ws + W.ewparts);
         add(ew, dw(BW_E + 4), W.ectas, 2 * 128 * 64, 128 * 64, 0);            // dW2 [128][64]
         add(ew + 128 * 64, dw(BW_E + 2), W.ectas, 2 * 128 * 64, 128 * 64, 128);  // dW1 = (dW1^T)^T
-        int items = 0;
+        int ctas = 0;
         for (int s = 0; s < sg.n; ++s)
-            items += sg.seg[s].nparts > 16 ? sg.seg[s].count : (sg.seg[s].count + 31) / 32;
-        k_sum_parts<<<(items + 7) / 8, 256, 0, st>>>(sg);
+            ctas += sg.seg[s].nparts > 16 ? (sg.seg[s].count + 31) / 32 : (sg.seg[s].count + 255) / 256;
+        k_sum_parts<<<ctas, 256, 0, st>>>(sg);
         BLK_TRY(cudaGetLastError());
     }
     return cudaSuccess;
