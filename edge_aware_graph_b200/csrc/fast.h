@@ -1,5 +1,6 @@
 // sm_100a kernels specialised for de = 64, H = 8, dh = 32, bf16 storage.
 #pragma once
+#include <functional>
 #include "generic.h"
 
 namespace eaga {
@@ -16,5 +17,9 @@ size_t forward_scratch_bytes(const eaga_dims &d, bool with_order = true);
 cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st,
                     bool with_order = true);
 cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head, cudaStream_t st);
+// Runs `enqueue` with one of the current device's auxiliary streams and two
+// events of its own, the streams' enqueue lock held for the duration (the
+// block around the layer runs its global sub-block there).
+cudaError_t with_side_stream(const std::function<cudaError_t(cudaStream_t side, cudaEvent_t e0, cudaEvent_t e1)> &enqueue);
 }  // namespace fast
 }  // namespace eaga

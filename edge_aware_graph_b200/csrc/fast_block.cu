@@ -648,186 +648,203 @@ YParams y_params(int B, int n, int dx, int dy, const void *const *wb, const uint
 
 cudaError_t tail_forward(const TailFwd &a, char *ws, const BlockWs &W, char *saved, const BlockSaved &S,
                          cudaStream_t st) {
-    const int R = a.B * a.n, dx = a.dx;
-    float *pool = reinterpret_cast<float *>(ws + W.pool), *poolx = pool + (size_t)a.B * 64;
-    BLK_TRY(cudaMemsetAsync(pool, 0, (size_t)a.B * (64 + dx) * 4, st));
-    {   // edge sub-block (and the edge pooling sums)
-        EdgeArgs e = {};
-        e.B = a.B;
-        e.n = a.n;
-        e.Ein = a.Emid;
-        e.Eout = a.Eout;
-        e.W1 = a.wb[BW_E + 2];
-        e.W2 = a.wb[BW_E + 4];
-        EbParams &p = e.par;
-        p.M = a.M;
-        p.g1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 0]);
-        p.s1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 1]);
-        p.b1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 3]);
-        p.b2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 5]);
-        p.g2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 6]);
-        p.s2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 7]);
-        p.pool = pool;
-        p.status = a.status;
-        p.B = a.B;
-        p.n = a.n;
-        prof_mark(3, 0, st);
-        BLK_TRY(edge_forward(e, st));
-        prof_mark(3, 1, st);
-    }
-    void *Xa = saved + S.Xa, *Hx = saved + S.Hx, *Xz = saved + S.Xz;
-    BLK_TRY(ln_fwd(dx, a.Xmid, a.wb[BW_X + 0], a.wb[BW_X + 1], nullptr, Xa, R, st));
-    {   // H = relu(Xa W1 + b1)
-        const void *A[3] = {Xa, Xa, Xa}, *B[3] = {a.wb[BW_X + 2], a.wb[BW_X + 2], a.wb[BW_X + 2]};
-        const void *bias[3] = {a.wb[BW_X + 3], a.wb[BW_X + 3], a.wb[BW_X + 3]};
-        void *C[3] = {Hx, Hx, Hx};
-        BLK_TRY(tc_gemm(4, R, 2 * dx, dx, 1, A, B, bias, C, 2 * dx, nullptr, nullptr, a.status, st, true));
-    }
-    {   // Xz = Xa + H W2 + b2
-        const void *A[3] = {Hx, Hx, Hx}, *B[3] = {a.wb[BW_X + 4], a.wb[BW_X + 4], a.wb[BW_X + 4]};
-        const void *bias[3] = {a.wb[BW_X + 5], a.wb[BW_X + 5], a.wb[BW_X + 5]};
-        void *C[3] = {Xz, Xz, Xz};
-        BLK_TRY(tc_gemm(5, R, dx, 2 * dx, 1, A, B, bias, C, dx, Xa, nullptr, a.status, st, true));
-    }
-    BLK_TRY(ln_fwd(dx, Xz, a.wb[BW_X + 6], a.wb[BW_X + 7], a.M, a.Xout, R, st));
-    k_pool_x<<<dim3(a.B, dx / 64, (a.n + 63) / 64), 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.Xmid), a.M,
-                                                                  poolx, a.n, dx);
-    BLK_TRY(cudaGetLastError());
-    {   // global sub-block
-        YParams p = y_params(a.B, a.n, a.dx, a.dy, a.wb, a.M);
-        p.Xmid = static_cast<const __nv_bfloat16 *>(a.Xmid);
-        p.y = static_cast<const __nv_bfloat16 *>(a.y);
-        p.pool = pool;
-        p.poolx = poolx;
-        p.y1 = reinterpret_cast<float *>(saved + S.y1);
-        p.pX = reinterpret_cast<float *>(saved + S.pX);
-        p.pE = reinterpret_cast<float *>(saved + S.pE);
-        p.yout = static_cast<__nv_bfloat16 *>(a.yout);
-        const size_t smem = (size_t)(a.dx + 64 + 10 * a.dy + 256 + 32) * 4;
-        k_y_fwd<<<a.B, 256, smem, st>>>(p);
+    return with_side_stream([&](cudaStream_t side, cudaEvent_t e0, cudaEvent_t e1) -> cudaError_t {
+        const int R = a.B * a.n, dx = a.dx;
+        float *pool = reinterpret_cast<float *>(ws + W.pool), *poolx = pool + (size_t)a.B * 64;
+        BLK_TRY(cudaMemsetAsync(pool, 0, (size_t)a.B * (64 + dx) * 4, st));
+        {   // edge sub-block (and the edge pooling sums)
+            EdgeArgs e = {};
+            e.B = a.B;
+            e.n = a.n;
+            e.Ein = a.Emid;
+            e.Eout = a.Eout;
+            e.W1 = a.wb[BW_E + 2];
+            e.W2 = a.wb[BW_E + 4];
+            EbParams &p = e.par;
+            p.M = a.M;
+            p.g1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 0]);
+            p.s1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 1]);
+            p.b1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 3]);
+            p.b2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 5]);
+            p.g2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 6]);
+            p.s2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 7]);
+            p.pool = pool;
+            p.status = a.status;
+            p.B = a.B;
+            p.n = a.n;
+            prof_mark(3, 0, st);
+            BLK_TRY(edge_forward(e, st));
+            prof_mark(3, 1, st);
+        }
+        // the global sub-block (its pooling of X' and its update) on a side stream,
+        // beside the node sub-block: it needs the edge pooling sums and X' only
+        BLK_TRY(cudaEventRecord(e0, st));
+        BLK_TRY(cudaStreamWaitEvent(side, e0, 0));
+        k_pool_x<<<dim3(a.B, dx / 64, (a.n + 63) / 64), 256, 0, side>>>(static_cast<const __nv_bfloat16 *>(a.Xmid),
+                                                                        a.M, poolx, a.n, dx);
         BLK_TRY(cudaGetLastError());
-    }
-    return cudaSuccess;
+        {   // global sub-block
+            YParams p = y_params(a.B, a.n, a.dx, a.dy, a.wb, a.M);
+            p.Xmid = static_cast<const __nv_bfloat16 *>(a.Xmid);
+            p.y = static_cast<const __nv_bfloat16 *>(a.y);
+            p.pool = pool;
+            p.poolx = poolx;
+            p.y1 = reinterpret_cast<float *>(saved + S.y1);
+            p.pX = reinterpret_cast<float *>(saved + S.pX);
+            p.pE = reinterpret_cast<float *>(saved + S.pE);
+            p.yout = static_cast<__nv_bfloat16 *>(a.yout);
+            const size_t smem = (size_t)(a.dx + 64 + 10 * a.dy + 256 + 32) * 4;
+            k_y_fwd<<<a.B, 256, smem, side>>>(p);
+            BLK_TRY(cudaGetLastError());
+        }
+        void *Xa = saved + S.Xa, *Hx = saved + S.Hx, *Xz = saved + S.Xz;
+        BLK_TRY(ln_fwd(dx, a.Xmid, a.wb[BW_X + 0], a.wb[BW_X + 1], nullptr, Xa, R, st));
+        {   // H = relu(Xa W1 + b1)
+            const void *A[3] = {Xa, Xa, Xa}, *B[3] = {a.wb[BW_X + 2], a.wb[BW_X + 2], a.wb[BW_X + 2]};
+            const void *bias[3] = {a.wb[BW_X + 3], a.wb[BW_X + 3], a.wb[BW_X + 3]};
+            void *C[3] = {Hx, Hx, Hx};
+            BLK_TRY(tc_gemm(4, R, 2 * dx, dx, 1, A, B, bias, C, 2 * dx, nullptr, nullptr, a.status, st, true));
+        }
+        {   // Xz = Xa + H W2 + b2
+            const void *A[3] = {Hx, Hx, Hx}, *B[3] = {a.wb[BW_X + 4], a.wb[BW_X + 4], a.wb[BW_X + 4]};
+            const void *bias[3] = {a.wb[BW_X + 5], a.wb[BW_X + 5], a.wb[BW_X + 5]};
+            void *C[3] = {Xz, Xz, Xz};
+            BLK_TRY(tc_gemm(5, R, dx, 2 * dx, 1, A, B, bias, C, dx, Xa, nullptr, a.status, st, true));
+        }
+        BLK_TRY(ln_fwd(dx, Xz, a.wb[BW_X + 6], a.wb[BW_X + 7], a.M, a.Xout, R, st));
+        BLK_TRY(cudaEventRecord(e1, side));
+        BLK_TRY(cudaStreamWaitEvent(st, e1, 0));
+        return cudaSuccess;
+    });
 }
 
 cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const char *saved, const BlockSaved &S,
                           cudaStream_t st) {
-    const int R = a.B * a.n, dx = a.dx;
-    YParams yp = y_params(a.B, a.n, a.dx, a.dy, a.wb, a.M);
-    yp.y1 = const_cast<float *>(reinterpret_cast<const float *>(saved + S.y1));
-    yp.pX = const_cast<float *>(reinterpret_cast<const float *>(saved + S.pX));
-    yp.pE = const_cast<float *>(reinterpret_cast<const float *>(saved + S.pE));
-    yp.dyout = static_cast<const __nv_bfloat16 *>(a.dyout);
-    yp.dy1 = reinterpret_cast<float *>(ws + W.dy1);
-    yp.dpX = reinterpret_cast<float *>(ws + W.dpX);
-    yp.dpE = reinterpret_cast<float *>(ws + W.dpE);
-    yp.yv = reinterpret_cast<float *>(ws + W.yv);
-    {
-        const size_t smem = (size_t)(15 * a.dy + 256 + 32) * 4;
-        k_y_bwd<<<a.B, 256, smem, st>>>(yp);
+    return with_side_stream([&](cudaStream_t side, cudaEvent_t e0, cudaEvent_t e1) -> cudaError_t {
+        const int R = a.B * a.n, dx = a.dx;
+        YParams yp = y_params(a.B, a.n, a.dx, a.dy, a.wb, a.M);
+        yp.y1 = const_cast<float *>(reinterpret_cast<const float *>(saved + S.y1));
+        yp.pX = const_cast<float *>(reinterpret_cast<const float *>(saved + S.pX));
+        yp.pE = const_cast<float *>(reinterpret_cast<const float *>(saved + S.pE));
+        yp.dyout = static_cast<const __nv_bfloat16 *>(a.dyout);
+        yp.dy1 = reinterpret_cast<float *>(ws + W.dy1);
+        yp.dpX = reinterpret_cast<float *>(ws + W.dpX);
+        yp.dpE = reinterpret_cast<float *>(ws + W.dpE);
+        yp.yv = reinterpret_cast<float *>(ws + W.yv);
+        {
+            const size_t smem = (size_t)(15 * a.dy + 256 + 32) * 4;
+            k_y_bwd<<<a.B, 256, smem, st>>>(yp);
+            BLK_TRY(cudaGetLastError());
+        }
+        {   // edge sub-block backward: dE' (+ the pooling's gradient), partial sums
+            EdgeArgs e = {};
+            e.B = a.B;
+            e.n = a.n;
+            e.Ein = a.Emid;
+            e.dEout = a.dEout;
+            e.dEin = a.dEmid;
+            e.W1 = a.wb[BW_E + 2];
+            e.W2 = a.wb[BW_E + 4];
+            EbParams &p = e.par;
+            p.M = a.M;
+            p.g1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 0]);
+            p.s1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 1]);
+            p.b1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 3]);
+            p.b2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 5]);
+            p.g2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 6]);
+            p.s2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 7]);
+            p.dpool = reinterpret_cast<const float *>(ws + W.dpE);
+            p.parts = reinterpret_cast<float *>(ws + W.eparts);
+            p.wparts = reinterpret_cast<float *>(ws + W.ewparts);
+            p.status = a.status;
+            p.B = a.B;
+            p.n = a.n;
+            prof_mark(4, 0, st);
+            BLK_TRY(edge_backward(e, st));
+            prof_mark(4, 1, st);
+        }
+        {   // the global sub-block's parameter gradients on a side stream, beside the
+            // node sub-block (after the edge kernel, which fills the GPU)
+            BLK_TRY(cudaEventRecord(e0, st));
+            BLK_TRY(cudaStreamWaitEvent(side, e0, 0));
+            YGrads g;
+            auto d = [&](int i) { return a.dwb[i]; };
+            g.g1 = d(BW_Y + 0); g.s1 = d(BW_Y + 1); g.W1 = d(BW_Y + 2); g.b1 = d(BW_Y + 3);
+            g.W2 = d(BW_Y + 4); g.b2 = d(BW_Y + 5); g.g2 = d(BW_Y + 6); g.s2 = d(BW_Y + 7);
+            g.Wyx = d(BW_YX); g.Wye = d(BW_YE); g.by = d(BW_BY);
+            const int total = 4 * a.dy * a.dy + (dx + 64) * a.dy + 2 * a.dy + 6 * a.dy;
+            k_y_wgrad<<<(total + 255) / 256, 256, 0, side>>>(yp, g);
+            BLK_TRY(cudaGetLastError());
+        }
+        void *dXz = ws + W.dXz, *dHx = ws + W.dHx, *dXa = ws + W.dXa, *dXmid = ws + W.dXmid;
+        const void *Xa = saved + S.Xa, *Hx = saved + S.Hx, *Xz = saved + S.Xz;
+        float *ln2 = reinterpret_cast<float *>(ws + W.ln2), *ln1 = reinterpret_cast<float *>(ws + W.ln1);
+        BLK_TRY(ln_bwd(dx, Xz, a.dXout, a.wb[BW_X + 6], a.M, nullptr, nullptr, a.n, dXz, ln2, R, W.ln_grid, st));
+        {   // dH = (dXz W2^T) [H > 0]
+            const void *A[3] = {dXz, dXz, dXz}, *Bt[3] = {a.wb[BW_X + 4], a.wb[BW_X + 4], a.wb[BW_X + 4]};
+            void *C[3] = {dHx, dHx, dHx};
+            BLK_TRY(tc_gemm(6, R, 2 * dx, dx, 1, A, Bt, nullptr, C, 2 * dx, Hx, nullptr, a.status, st, false));
+        }
+        {   // dXa = dXz + dH W1^T
+            const void *A[3] = {dHx, dHx, dHx}, *Bt[3] = {a.wb[BW_X + 2], a.wb[BW_X + 2], a.wb[BW_X + 2]};
+            void *C[3] = {dXa, dXa, dXa};
+            BLK_TRY(tc_gemm(3, R, dx, 2 * dx, 1, A, Bt, nullptr, C, dx, dXz, nullptr, a.status, st, false));
+        }
+        BLK_TRY(ln_bwd(dx, a.Xmid, dXa, a.wb[BW_X + 0], nullptr, reinterpret_cast<const float *>(ws + W.dpX), a.M,
+                       a.n, dXmid, ln1, R, W.ln_grid, st));
+        {   // dW1 = Xa^T dH, dW2 = H^T dXz (split-K partials)
+            float *g1 = reinterpret_cast<float *>(ws + W.wg1), *g2 = reinterpret_cast<float *>(ws + W.wg2);
+            const void *B1[3] = {dHx, dHx, dHx}, *B2[3] = {dXz, dXz, dXz};
+            float *const P1[3] = {g1, g1, g1}, *const P2[3] = {g2, g2, g2};
+            BLK_TRY(tc_wgrad(dx, 2 * dx, 1, R, W.wsplits, Xa, B1, P1, a.status, st));
+            BLK_TRY(tc_wgrad(2 * dx, dx, 1, R, W.wsplits, Hx, B2, P2, a.status, st));
+        }
+        float *cs1 = reinterpret_cast<float *>(ws + W.cs1), *cs2 = reinterpret_cast<float *>(ws + W.cs2);
+        k_colsum<<<W.cs_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(dHx), cs1, R, 2 * dx, W.cs_rows);
         BLK_TRY(cudaGetLastError());
-        YGrads g;
-        auto d = [&](int i) { return a.dwb[i]; };
-        g.g1 = d(BW_Y + 0); g.s1 = d(BW_Y + 1); g.W1 = d(BW_Y + 2); g.b1 = d(BW_Y + 3);
-        g.W2 = d(BW_Y + 4); g.b2 = d(BW_Y + 5); g.g2 = d(BW_Y + 6); g.s2 = d(BW_Y + 7);
-        g.Wyx = d(BW_YX); g.Wye = d(BW_YE); g.by = d(BW_BY);
-        const int total = 4 * a.dy * a.dy + (dx + 64) * a.dy + 2 * a.dy + 6 * a.dy;
-        k_y_wgrad<<<(total + 255) / 256, 256, 0, st>>>(yp, g);
+        k_colsum<<<W.cs_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(dXz), cs2, R, dx, W.cs_rows);
         BLK_TRY(cudaGetLastError());
-    }
-    {   // edge sub-block backward: dE' (+ the pooling's gradient), partial sums
-        EdgeArgs e = {};
-        e.B = a.B;
-        e.n = a.n;
-        e.Ein = a.Emid;
-        e.dEout = a.dEout;
-        e.dEin = a.dEmid;
-        e.W1 = a.wb[BW_E + 2];
-        e.W2 = a.wb[BW_E + 4];
-        EbParams &p = e.par;
-        p.M = a.M;
-        p.g1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 0]);
-        p.s1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 1]);
-        p.b1 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 3]);
-        p.b2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 5]);
-        p.g2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 6]);
-        p.s2 = static_cast<const __nv_bfloat16 *>(a.wb[BW_E + 7]);
-        p.dpool = reinterpret_cast<const float *>(ws + W.dpE);
-        p.parts = reinterpret_cast<float *>(ws + W.eparts);
-        p.wparts = reinterpret_cast<float *>(ws + W.ewparts);
-        p.status = a.status;
-        p.B = a.B;
-        p.n = a.n;
-        prof_mark(4, 0, st);
-        BLK_TRY(edge_backward(e, st));
-        prof_mark(4, 1, st);
-    }
-    void *dXz = ws + W.dXz, *dHx = ws + W.dHx, *dXa = ws + W.dXa, *dXmid = ws + W.dXmid;
-    const void *Xa = saved + S.Xa, *Hx = saved + S.Hx, *Xz = saved + S.Xz;
-    float *ln2 = reinterpret_cast<float *>(ws + W.ln2), *ln1 = reinterpret_cast<float *>(ws + W.ln1);
-    BLK_TRY(ln_bwd(dx, Xz, a.dXout, a.wb[BW_X + 6], a.M, nullptr, nullptr, a.n, dXz, ln2, R, W.ln_grid, st));
-    {   // dH = (dXz W2^T) [H > 0]
-        const void *A[3] = {dXz, dXz, dXz}, *Bt[3] = {a.wb[BW_X + 4], a.wb[BW_X + 4], a.wb[BW_X + 4]};
-        void *C[3] = {dHx, dHx, dHx};
-        BLK_TRY(tc_gemm(6, R, 2 * dx, dx, 1, A, Bt, nullptr, C, 2 * dx, Hx, nullptr, a.status, st, false));
-    }
-    {   // dXa = dXz + dH W1^T
-        const void *A[3] = {dHx, dHx, dHx}, *Bt[3] = {a.wb[BW_X + 2], a.wb[BW_X + 2], a.wb[BW_X + 2]};
-        void *C[3] = {dXa, dXa, dXa};
-        BLK_TRY(tc_gemm(3, R, dx, 2 * dx, 1, A, Bt, nullptr, C, dx, dXz, nullptr, a.status, st, false));
-    }
-    BLK_TRY(ln_bwd(dx, a.Xmid, dXa, a.wb[BW_X + 0], nullptr, reinterpret_cast<const float *>(ws + W.dpX), a.M,
-                   a.n, dXmid, ln1, R, W.ln_grid, st));
-    {   // dW1 = Xa^T dH, dW2 = H^T dXz (split-K partials)
-        float *g1 = reinterpret_cast<float *>(ws + W.wg1), *g2 = reinterpret_cast<float *>(ws + W.wg2);
-        const void *B1[3] = {dHx, dHx, dHx}, *B2[3] = {dXz, dXz, dXz};
-        float *const P1[3] = {g1, g1, g1}, *const P2[3] = {g2, g2, g2};
-        BLK_TRY(tc_wgrad(dx, 2 * dx, 1, R, W.wsplits, Xa, B1, P1, a.status, st));
-        BLK_TRY(tc_wgrad(2 * dx, dx, 1, R, W.wsplits, Hx, B2, P2, a.status, st));
-    }
-    float *cs1 = reinterpret_cast<float *>(ws + W.cs1), *cs2 = reinterpret_cast<float *>(ws + W.cs2);
-    k_colsum<<<W.cs_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(dHx), cs1, R, 2 * dx, W.cs_rows);
-    BLK_TRY(cudaGetLastError());
-    k_colsum<<<W.cs_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(dXz), cs2, R, dx, W.cs_rows);
-    BLK_TRY(cudaGetLastError());
-    {
-        SumSegs sg = {};
-        auto add = [&](const float *src, float *dst, int nparts, int stride, int count, int trows) {
-            SumSeg &q = sg.seg[sg.n++];
-            q.src = src;
-            q.dst = dst;
-            q.nparts = nparts;
-            q.stride = stride;
-            q.count = count;
-            q.trows = trows;
-        };
-        auto dw = [&](int i) { return a.dwb[i]; };
-        add(ln2, dw(BW_X + 6), W.ln_grid, 2 * dx, dx, 0);
-        add(ln2 + dx, dw(BW_X + 7), W.ln_grid, 2 * dx, dx, 0);
-        add(ln1, dw(BW_X + 0), W.ln_grid, 2 * dx, dx, 0);
-        add(ln1 + dx, dw(BW_X + 1), W.ln_grid, 2 * dx, dx, 0);
-        add(cs1, dw(BW_X + 3), W.cs_grid, 2 * dx, 2 * dx, 0);
-        add(cs2, dw(BW_X + 5), W.cs_grid, dx, dx, 0);
-        add(reinterpret_cast<float *>(ws + W.wg1), dw(BW_X + 2), W.wsplits, dx * 2 * dx, dx * 2 * dx, 0);
-        add(reinterpret_cast<float *>(ws + W.wg2), dw(BW_X + 4), W.wsplits, 2 * dx * dx, 2 * dx * dx, 0);
-        const float *ep = reinterpret_cast<const float *>(ws + W.eparts);
-        const int np = W.ectas;
-        add(ep + 0, dw(BW_E + 6), np, EB_PART, 64, 0);      // dg2
-        add(ep + 64, dw(BW_E + 7), np, EB_PART, 64, 0);     // ds2
-        add(ep + 128, dw(BW_E + 5), np, EB_PART, 64, 0);    // db2
-        add(ep + 192, dw(BW_E + 0), np, EB_PART, 64, 0);    // dg1
-        add(ep + 256, dw(BW_E + 1), np, EB_PART, 64, 0);    // ds1
-        add(ep + 320, dw(BW_E + 3), np, EB_PART, 128, 0);   // db1
-        const float *ew = reinterpret_cast<const float *>(ws + W.ewparts);
-        add(ew, dw(BW_E + 4), W.ectas, 2 * 128 * 64, 128 * 64, 0);            // dW2 [128][64]
-        add(ew + 128 * 64, dw(BW_E + 2), W.ectas, 2 * 128 * 64, 128 * 64, 128);  // dW1 = (dW1^T)^T
-        int ctas = 0;
-        for (int s = 0; s < sg.n; ++s)
-            ctas += sg.seg[s].nparts > 16 ? (sg.seg[s].count + 31) / 32 : (sg.seg[s].count + 255) / 256;
-        k_sum_parts<<<ctas, 256, 0, st>>>(sg);
-        BLK_TRY(cudaGetLastError());
-    }
-    return cudaSuccess;
+        {
+            SumSegs sg = {};
+            auto add = [&](const float *src, float *dst, int nparts, int stride, int count, int trows) {
+                SumSeg &q = sg.seg[sg.n++];
+                q.src = src;
+                q.dst = dst;
+                q.nparts = nparts;
+                q.stride = stride;
+                q.count = count;
+                q.trows = trows;
+            };
+            auto dw = [&](int i) { return a.dwb[i]; };
+            add(ln2, dw(BW_X + 6), W.ln_grid, 2 * dx, dx, 0);
+            add(ln2 + dx, dw(BW_X + 7), W.ln_grid, 2 * dx, dx, 0);
+            add(ln1, dw(BW_X + 0), W.ln_grid, 2 * dx, dx, 0);
+            add(ln1 + dx, dw(BW_X + 1), W.ln_grid, 2 * dx, dx, 0);
+            add(cs1, dw(BW_X + 3), W.cs_grid, 2 * dx, 2 * dx, 0);
+            add(cs2, dw(BW_X + 5), W.cs_grid, dx, dx, 0);
+            add(reinterpret_cast<float *>(ws + W.wg1), dw(BW_X + 2), W.wsplits, dx * 2 * dx, dx * 2 * dx, 0);
+            add(reinterpret_cast<float *>(ws + W.wg2), dw(BW_X + 4), W.wsplits, 2 * dx * dx, 2 * dx * dx, 0);
+            const float *ep = reinterpret_cast<const float *>(ws + W.eparts);
+            const int np = W.ectas;
+            add(ep + 0, dw(BW_E + 6), np, EB_PART, 64, 0);      // dg2
+            add(ep + 64, dw(BW_E + 7), np, EB_PART, 64, 0);     // ds2
+            add(ep + 128, dw(BW_E + 5), np, EB_PART, 64, 0);    // db2
+            add(ep + 192, dw(BW_E + 0), np, EB_PART, 64, 0);    // dg1
+            add(ep + 256, dw(BW_E + 1), np, EB_PART, 64, 0);    // ds1
+            add(ep + 320, dw(BW_E + 3), np, EB_PART, 128, 0);   // db1
+            const float *ew = reinterpret_cast<const float *>(ws + W.ewparts);
+            add(ew, dw(BW_E + 4), W.ectas, 2 * 128 * 64, 128 * 64, 0);            // dW2 [128][64]
+            add(ew + 128 * 64, dw(BW_E + 2), W.ectas, 2 * 128 * 64, 128 * 64, 128);  // dW1 = (dW1^T)^T
+            int ctas = 0;
+            for (int s = 0; s < sg.n; ++s)
+                ctas += sg.seg[s].nparts > 16 ? (sg.seg[s].count + 31) / 32 : (sg.seg[s].count + 255) / 256;
+            k_sum_parts<<<ctas, 256, 0, st>>>(sg);
+            BLK_TRY(cudaGetLastError());
+        }
+        BLK_TRY(cudaEventRecord(e1, side));
+        BLK_TRY(cudaStreamWaitEvent(st, e1, 0));
+        return cudaSuccess;
+    });
 }
 
 cudaError_t add_dy(void *dy, const float *dy1, int count, cudaStream_t st) {
