@@ -108,9 +108,9 @@ EAGA_API size_t eaga_saved_size(const eaga_dims *dims);
  * (nullable; eaga_saved_size bytes) receives the state eaga_backward needs;
  * with saved == NULL that state lives in the workspace and is discarded.
  * `workspace` must hold eaga_workspace_size(dims, 0) bytes.  On the
- * specialised bf16 path the small prologue kernel runs beside the Q/K/V
- * projection on one of the library's per-device streams, ordered on `stream`
- * like the backward's (below). */
+ * specialised bf16 path the small prologue and row-order kernels run beside
+ * the Q/K/V projection on the library's per-device streams, ordered on
+ * `stream` like the backward's (below). */
 EAGA_API eaga_status eaga_forward(const eaga_dims *dims,
                          const void *X, const void *E, const void *y, const uint8_t *M,
                          const eaga_weights *w,
@@ -122,7 +122,7 @@ EAGA_API eaga_status eaga_forward(const eaga_dims *dims,
  * gradient (fp32).  `workspace` must hold eaga_workspace_size(dims, 1) bytes.
  * Gradients of masked nodes / invalid pairs are the residual ones
  * (dX_i = dX'_i, dE_ij = dE'_ij).
- * On the specialised bf16 path some independent kernels run on two streams
+ * On the specialised bf16 path some independent kernels run on three streams
  * the library creates once per device; they start after the work already
  * on `stream` and `stream` waits for them before the call's last kernels,
  * so the call is ordered on `stream` as a whole (and a CUDA graph captured
