@@ -61,7 +61,7 @@ int kernel_launches(const eaga_dims &, int for_backward) {
 // as parallel branches.  The lock is held while a call enqueues, so concurrent calls on
 // one device never share an event between a record and its wait.
 namespace {
-constexpr int kMaxDevices = 64, kEvents = 13, kStreams = 3;
+constexpr int kMaxDevices = 64, kEvents = 16, kStreams = 3;
 struct DeviceAux {
     std::mutex mu;
     bool ready = false;
@@ -138,12 +138,12 @@ cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common,
     return cudaSuccess;
 }
 
-cudaError_t with_side_stream(const std::function<cudaError_t(cudaStream_t, cudaEvent_t, cudaEvent_t)> &enqueue) {
+cudaError_t with_side_streams(const std::function<cudaError_t(const cudaStream_t *, const cudaEvent_t *)> &enqueue) {
     DeviceAux *aux = nullptr;
     FAST_TRY(device_aux(&aux));
     std::lock_guard<std::mutex> lock(aux->mu);
     FAST_TRY(aux_init(*aux));
-    return enqueue(aux->s[2], aux->ev[11], aux->ev[12]);
+    return enqueue(aux->s, aux->ev + 11);   // events 11..15 are the caller's
 }
 
 cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head, cudaStream_t st) {

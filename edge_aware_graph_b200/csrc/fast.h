@@ -17,9 +17,10 @@ size_t forward_scratch_bytes(const eaga_dims &d, bool with_order = true);
 cudaError_t forward(const eaga_dims &d, const FwdArgs &a, char *ws_after_common, cudaStream_t st,
                     bool with_order = true);
 cudaError_t backward(const eaga_dims &d, const BwdArgs &a, char *ws, size_t head, cudaStream_t st);
-// Runs `enqueue` with one of the current device's auxiliary streams and two
-// events of its own, the streams' enqueue lock held for the duration (the
-// block around the layer runs its global sub-block there).
-cudaError_t with_side_stream(const std::function<cudaError_t(cudaStream_t side, cudaEvent_t e0, cudaEvent_t e1)> &enqueue);
+// Runs `enqueue` with the current device's three auxiliary streams and five
+// events of their own, the streams' enqueue lock held for the duration (the
+// block around the layer runs its global sub-block and its node weight
+// gradients there).
+cudaError_t with_side_streams(const std::function<cudaError_t(const cudaStream_t *side, const cudaEvent_t *ev)> &enqueue);
 }  // namespace fast
 }  // namespace eaga

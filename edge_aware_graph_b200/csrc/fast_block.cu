@@ -648,7 +648,9 @@ YParams y_params(int B, int n, int dx, int dy, const void *const *wb, const uint
 
 cudaError_t tail_forward(const TailFwd &a, char *ws, const BlockWs &W, char *saved, const BlockSaved &S,
                          cudaStream_t st) {
-    return with_side_stream([&](cudaStream_t side, cudaEvent_t e0, cudaEvent_t e1) -> cudaError_t {
+    return with_side_streams([&](const cudaStream_t *ss, const cudaEvent_t *ev) -> cudaError_t {
+        cudaStream_t side = ss[2];
+        cudaEvent_t e0 = ev[0], e1 = ev[1];
         const int R = a.B * a.n, dx = a.dx;
         float *pool = reinterpret_cast<float *>(ws + W.pool), *poolx = pool + (size_t)a.B * 64;
         BLK_TRY(cudaMemsetAsync(pool, 0, (size_t)a.B * (64 + dx) * 4, st));
@@ -720,7 +722,9 @@ cudaError_t tail_forward(const TailFwd &a, char *ws, const BlockWs &W, char *sav
 
 cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const char *saved, const BlockSaved &S,
                           cudaStream_t st) {
-    return with_side_stream([&](cudaStream_t side, cudaEvent_t e0, cudaEvent_t e1) -> cudaError_t {
+    return with_side_streams([&](const cudaStream_t *ss, const cudaEvent_t *ev) -> cudaError_t {
+        cudaStream_t side = ss[2];
+        cudaEvent_t e0 = ev[0], e1 = ev[1];
         const int R = a.B * a.n, dx = a.dx;
         YParams yp = y_params(a.B, a.n, a.dx, a.dy, a.wb, a.M);
         yp.y1 = const_cast<float *>(reinterpret_cast<const float *>(saved + S.y1));
@@ -785,6 +789,24 @@ cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const ch
             void *C[3] = {dHx, dHx, dHx};
             BLK_TRY(tc_gemm(6, R, 2 * dx, dx, 1, A, Bt, nullptr, C, 2 * dx, Hx, nullptr, a.status, st, false));
         }
+        // dW1 = Xa^T dH, dW2 = H^T dXz (split-K partials) and the column sums of
+        // dH and dXz (the bias gradients) on two side streams, beside dXa and the
+        // first LayerNorm's backward: they need dH and dXz only
+        float *cs1 = reinterpret_cast<float *>(ws + W.cs1), *cs2 = reinterpret_cast<float *>(ws + W.cs2);
+        BLK_TRY(cudaEventRecord(ev[2], st));
+        BLK_TRY(cudaStreamWaitEvent(ss[0], ev[2], 0));
+        BLK_TRY(cudaStreamWaitEvent(ss[1], ev[2], 0));
+        {
+            float *g1 = reinterpret_cast<float *>(ws + W.wg1), *g2 = reinterpret_cast<float *>(ws + W.wg2);
+            const void *B1[3] = {dHx, dHx, dHx}, *B2[3] = {dXz, dXz, dXz};
+            float *const P1[3] = {g1, g1, g1}, *const P2[3] = {g2, g2, g2};
+            BLK_TRY(tc_wgrad(dx, 2 * dx, 1, R, W.wsplits, Xa, B1, P1, a.status, ss[0]));
+            k_colsum<<<W.cs_grid, 256, 0, ss[0]>>>(static_cast<const __nv_bfloat16 *>(dHx), cs1, R, 2 * dx, W.cs_rows);
+            BLK_TRY(cudaGetLastError());
+            BLK_TRY(tc_wgrad(2 * dx, dx, 1, R, W.wsplits, Hx, B2, P2, a.status, ss[1]));
+            k_colsum<<<W.cs_grid, 256, 0, ss[1]>>>(static_cast<const __nv_bfloat16 *>(dXz), cs2, R, dx, W.cs_rows);
+            BLK_TRY(cudaGetLastError());
+        }
         {   // dXa = dXz + dH W1^T
             const void *A[3] = {dHx, dHx, dHx}, *Bt[3] = {a.wb[BW_X + 2], a.wb[BW_X + 2], a.wb[BW_X + 2]};
             void *C[3] = {dXa, dXa, dXa};
@@ -792,18 +814,10 @@ cudaError_t tail_backward(const TailBwd &a, char *ws, const BlockWs &W, const ch
         }
         BLK_TRY(ln_bwd(dx, a.Xmid, dXa, a.wb[BW_X + 0], nullptr, reinterpret_cast<const float *>(ws + W.dpX), a.M,
                        a.n, dXmid, ln1, R, W.ln_grid, st));
-        {   // dW1 = Xa^T dH, dW2 = H^T dXz (split-K partials)
-            float *g1 = reinterpret_cast<float *>(ws + W.wg1), *g2 = reinterpret_cast<float *>(ws + W.wg2);
-            const void *B1[3] = {dHx, dHx, dHx}, *B2[3] = {dXz, dXz, dXz};
-            float *const P1[3] = {g1, g1, g1}, *const P2[3] = {g2, g2, g2};
-            BLK_TRY(tc_wgrad(dx, 2 * dx, 1, R, W.wsplits, Xa, B1, P1, a.status, st));
-            BLK_TRY(tc_wgrad(2 * dx, dx, 1, R, W.wsplits, Hx, B2, P2, a.status, st));
-        }
-        float *cs1 = reinterpret_cast<float *>(ws + W.cs1), *cs2 = reinterpret_cast<float *>(ws + W.cs2);
-        k_colsum<<<W.cs_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(dHx), cs1, R, 2 * dx, W.cs_rows);
-        BLK_TRY(cudaGetLastError());
-        k_colsum<<<W.cs_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(dXz), cs2, R, dx, W.cs_rows);
-        BLK_TRY(cudaGetLastError());
+        BLK_TRY(cudaEventRecord(ev[3], ss[0]));
+        BLK_TRY(cudaEventRecord(ev[4], ss[1]));
+        BLK_TRY(cudaStreamWaitEvent(st, ev[3], 0));
+        BLK_TRY(cudaStreamWaitEvent(st, ev[4], 0));
         {
             SumSegs sg = {};
             auto add = [&](const float *src, float *dst, int nparts, int stride, int count, int trows) {
