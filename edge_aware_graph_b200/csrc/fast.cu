@@ -44,9 +44,9 @@ size_t workspace_size(const eaga_dims &d, int for_backward, size_t common_fwd, s
 
 int kernel_launches(const eaga_dims &, int for_backward) {
     // forward: prologue, row-block order, QKV, pairs, out-proj
-    // backward: prologue, dO, row-block order, pairs, dk/dv conversion, dX, wgrad x2, bias partial,
-    // rparts partial, finish x2, film grads
-    return for_backward ? 13 : 5;
+    // backward: prologue, dO, row-block order, pairs, dk/dv conversion, dX, wgrad x2, bias and
+    // row-block partials, finish x2, film grads
+    return for_backward ? 12 : 5;
 }
 
 #define FAST_TRY(x)                               \

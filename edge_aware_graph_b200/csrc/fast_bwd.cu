@@ -21,17 +21,17 @@ using namespace dev;
 // [0,256) dQ, [256,512) dK, [512,768) dV, [768,768+dx) M-masked dX'.  Block
 // (256-column strip, row segment): lane = 8 columns (one 16-byte load per
 // row), warp = every 8th row of the segment, warps added in a fixed order.
-__global__ void __launch_bounds__(256) k_bias_partial(const __nv_bfloat16 *dQ, const __nv_bfloat16 *dK,
-                                                      const __nv_bfloat16 *dV, const __nv_bfloat16 *dXo,
-                                                      const uint8_t *M, int rows, int dx, int seg_rows, float *out) {
+__device__ __forceinline__ void bias_partial(const __nv_bfloat16 *dQ, const __nv_bfloat16 *dK,
+                                             const __nv_bfloat16 *dV, const __nv_bfloat16 *dXo, const uint8_t *M,
+                                             int rows, int dx, int seg_rows, float *out, int bx, int by) {
     __shared__ float red[8][256];
     const int w = threadIdx.x >> 5, t = threadIdx.x & 31;
-    const int strip = blockIdx.x, ncol = 3 * HD + dx;
+    const int strip = bx, ncol = 3 * HD + dx;
     const bool masked = strip >= 3;
     const __nv_bfloat16 *src = strip == 0 ? dQ : strip == 1 ? dK : strip == 2 ? dV : dXo;
     const int ld = masked ? dx : HD, c0 = (masked ? (strip - 3) * 256 : 0) + 8 * t;
     const bool active = c0 < ld;
-    const int r0 = blockIdx.y * seg_rows, r1 = min(rows, r0 + seg_rows);
+    const int r0 = by * seg_rows, r1 = min(rows, r0 + seg_rows);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (active) {
 #pragma unroll 4
@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(256) k_bias_partial(const __nv_bfloat16 *dQ, c
         float x = 0.f;
 #pragma unroll
         for (int k = 0; k < 8; ++k) x += red[k][col];
-        out[(size_t)blockIdx.y * ncol + gcol] = x;
+        out[(size_t)by * ncol + gcol] = x;
     }
 }
 
@@ -77,11 +77,11 @@ __device__ __forceinline__ float strided_sum(const float *src, int count, size_t
 // Row-kernel partials: out[z][e] = sum over CTAs of segment z of rparts[cta][e], e < dWfe+dWe
 // (blockIdx.y = z < gridDim.y - 1); the last row of blocks sums each graph's
 // dg_b = sum over its row blocks of their dg partials.
-__global__ void k_rparts_partial(const float *rparts, int ctas, int seg, float *out, float *dg, int B,
-                                 int ctas_per_graph) {
-    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+__device__ __forceinline__ void rparts_partial(const float *rparts, int ctas, int seg, float *out, float *dg, int B,
+                                               int ctas_per_graph, int bx, int by, int gy) {
+    const int e = bx * blockDim.x + threadIdx.x;
     constexpr int NE = DE * NF + NH * DE;
-    if (blockIdx.y + 1 == gridDim.y) {
+    if (by + 1 == gy) {
         if (e < B * NF) {
             const int b = e / NF, k = e % NF;
             dg[e] = strided_sum(rparts + (size_t)b * ctas_per_graph * RPART + NE + k, ctas_per_graph, RPART);
@@ -89,8 +89,26 @@ __global__ void k_rparts_partial(const float *rparts, int ctas, int seg, float *
         return;
     }
     if (e >= NE) return;
-    const int c0 = blockIdx.y * seg, c1 = min(ctas, c0 + seg);
-    out[(size_t)blockIdx.y * NE + e] = c1 > c0 ? strided_sum(rparts + (size_t)c0 * RPART + e, c1 - c0, RPART) : 0.f;
+    const int c0 = by * seg, c1 = min(ctas, c0 + seg);
+    out[(size_t)by * NE + e] = c1 > c0 ? strided_sum(rparts + (size_t)c0 * RPART + e, c1 - c0, RPART) : 0.f;
+}
+
+// The bias partials (CTA rows y < bsplits: column sums of dQ, dK, dV and the
+// masked dX' over row segments) and the row-block partials (the other rows:
+// sums of the pair kernel's per-row-block partials over CTA segments, and dg)
+// in one launch; the two jobs are independent.
+__global__ void __launch_bounds__(256) k_bwd_partials(const __nv_bfloat16 *dQ, const __nv_bfloat16 *dK,
+                                                      const __nv_bfloat16 *dV, const __nv_bfloat16 *dXo,
+                                                      const uint8_t *M, int rows, int dx, int seg_rows, float *bout,
+                                                      int bias_x, int bsplits, const float *rparts, int ctas, int seg,
+                                                      float *rout, float *dg, int B, int ctas_per_graph, int rp_x,
+                                                      int rp_y) {
+    if ((int)blockIdx.y < bsplits) {
+        if ((int)blockIdx.x < bias_x) bias_partial(dQ, dK, dV, dXo, M, rows, dx, seg_rows, bout, blockIdx.x, blockIdx.y);
+        return;
+    }
+    if ((int)blockIdx.x < rp_x)
+        rparts_partial(rparts, ctas, seg, rout, dg, B, ctas_per_graph, blockIdx.x, blockIdx.y - bsplits, rp_y);
 }
 
 struct DWPtrs {
@@ -127,7 +145,7 @@ __global__ void k_bwd_finish(const float *wparts, int wsplits, const float *bpar
     }
 }
 
-// dbf, dWfy, dy from dg (after k_rparts_partial).
+// dbf, dWfy, dy from dg (after k_bwd_partials).
 __global__ void k_film_grads(const float *dg, int B, int dy, const __nv_bfloat16 *y, const __nv_bfloat16 *Wfy,
                              float *dbf, float *dWfy, __nv_bfloat16 *dyo) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -267,16 +285,16 @@ cudaError_t launch_bwd_partials(const eaga_dims &d, const BwdArgs &a, const Fast
     const int rows = d.B * d.n;
     float *bparts = reinterpret_cast<float *>(ws + W.bparts);
     const int seg_rows = (rows + W.bsplits - 1) / W.bsplits;
-    k_bias_partial<<<dim3(3 + (d.dx + 255) / 256, W.bsplits), 256, 0, st>>>(
-        dQ, dK, dV, static_cast<const __nv_bfloat16 *>(a.dXout), a.M, rows, d.dx, seg_rows, bparts);
+    const int bias_x = 3 + (d.dx + 255) / 256;
     float *r2 = reinterpret_cast<float *>(ws + W.r2);
     float *dg = reinterpret_cast<float *>(ws + W.dg);
     const int ctas = W.n_rparts, seg = (ctas + W.rsplits - 1) / W.rsplits;
     constexpr int NE = DE * NF + NH * DE;
     const float *rparts = reinterpret_cast<const float *>(ws + W.rparts);
     const int xblocks = (std::max(NE, d.B * NF) + 255) / 256;
-    k_rparts_partial<<<dim3(xblocks, W.rsplits + 1), 256, 0, st>>>(rparts, ctas, seg, r2, dg, d.B,
-                                                                   (d.n + TB - 1) / TB);
+    k_bwd_partials<<<dim3(std::max(bias_x, xblocks), W.bsplits + W.rsplits + 1), 256, 0, st>>>(
+        dQ, dK, dV, static_cast<const __nv_bfloat16 *>(a.dXout), a.M, rows, d.dx, seg_rows, bparts, bias_x, W.bsplits,
+        rparts, ctas, seg, r2, dg, d.B, (d.n + TB - 1) / TB, xblocks, W.rsplits + 1);
     return cudaGetLastError();
 }
 

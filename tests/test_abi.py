@@ -176,7 +176,7 @@ def test_dispatch_rule(L, dims, fast):
     # H = 8, dh = 32, n even, dx a multiple of 64; every other supported shape
     # runs the CUDA-core kernels (4 and 10)
     d = eaga.dims(*dims)
-    assert (eaga.kernel_launches(d, False), eaga.kernel_launches(d, True)) == ((5, 13) if fast else (4, 10))
+    assert (eaga.kernel_launches(d, False), eaga.kernel_launches(d, True)) == ((5, 12) if fast else (4, 10))
 
 
 def test_dispatch_rejects_unsupported(L):

@@ -40,6 +40,6 @@ def test_header_is_c99_and_host_calls_work(tmp_path):
     assert r.returncode == 0, r.stderr
     wf, wb, sv, lf, lb, s, msg = r.stdout.split(maxsplit=6)
     assert int(wf) > 0 and int(wb) > int(wf) and int(sv) > 0
-    assert (int(lf), int(lb)) == (5, 13)              # the tcgen05 path for these dims
+    assert (int(lf), int(lb)) == (5, 12)              # the tcgen05 path for these dims
     assert int(s) == 2                                # n beyond the limits: EAGA_ERR_UNSUPPORTED, nothing launched
     assert msg.strip()
