@@ -348,3 +348,22 @@ def test_unknown_variant_is_refused(L):
         rc = L.eaga_backward_variant(ctypes.byref(d), v, fake, fake, fake, fake, ctypes.byref(w), fake, fake, fake,
                                      fake, fake, fake, ctypes.byref(w), fake, 1 << 40, None)
         assert rc == 1
+
+
+@no_cuda
+@pytest.mark.parametrize("dims_of", [lambda B: eaga.dims(B, 16, 64, 64, 16, 8, 32, "bf16"),
+                                     lambda B: eaga.dims(B, 8, 24, 24, 16, 2, 16, "fp32")],
+                         ids=["bf16-fast-892", "fp32-generic-H2-4080"])
+def test_noalloc_graph_limit_boundaries(L, dims_of):
+    """The no-allocation forward keeps its scratch in a fixed 64 KiB array:
+    256 + roundup256(8*H*B) bytes, plus 8 KiB of operand images on the
+    specialised path, must fit, so the largest batch is B = 892 there and
+    B = 4080 at H = 2 on the CUDA-core path.  One graph more is refused as
+    unsupported before any device work; the largest batch passes the size
+    check (and goes on to the device, which this CPU-only test does not have)."""
+    limit = 892 if dims_of(1).dtype == eaga.EAGA_BF16 else 4080
+    for B, refused in ((limit, False), (limit + 1, True)):
+        d = dims_of(B)
+        fw = forward_layout(d, far=True)
+        rc = L.eaga_forward_noalloc(ctypes.byref(d), *(fw.args()[:8]), None)
+        assert (rc == 2) == refused, (B, rc)   # 2: EAGA_ERR_UNSUPPORTED
